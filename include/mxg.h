@@ -1,0 +1,157 @@
+/*
+ * mxg — weight-quantized linear layer for speculative-decoding verify chunks,
+ * B200 (sm_100a).  C ABI of libmxg.so.
+ *
+ *     Y[M][N] = X[M][K] * dequant(W)^T      bf16 in, fp32 accumulate, bf16 out
+ *
+ * Two weight formats:
+ *
+ *  INT4 W4A16 (GPTQ, symmetric, group G along K).  Defined by the
+ *  "Qwen3.8-27B GPTQ-Int4-sym-G128" model card, section "Quantization
+ *  contract" (GPTQ INT4, symmetric, group size 128, desc_act=false, packed
+ *  int32) and the Eole Qwen3.8 recipe, section "Compressed-tensors INT4
+ *  layout" (symmetric grouped W4A16; group size 32, 64 or 128; asymmetric,
+ *  act-order and sparse exports rejected) and "INT4 tensor parallelism"
+ *  (packed weights are partitioned, then re-packed once for the kernel).
+ *  Codes q in 0..15, eight per int32 word along K: the code of row k = 8i + j
+ *  is bits [4j, 4j+3] of word (i, n) of qweight[K/8][N].  Weight
+ *  w[n][k] = (q - 8) * scale[k / G][n], scales fp16.
+ *
+ *  MXFP8 (OCP Microscaling).  Defined by the "Qwen3.8-27B-MXFP8 AutoRound"
+ *  model card: header (8-bit block FP with E8M0 group scales), section 2
+ *  (kernel constraints N >= 128 and K % 32 == 0) and section 8 (OCP MX
+ *  specification, one E8M0 shared scale per 32-element block).  Codes are
+ *  OCP E4M3 ("fn": bias 7, no infinities, S.1111.111 is NaN) in Wq[N][K]
+ *  (K contiguous), exponents E8M0 in Ws[N][K/32]; w = e4m3 * 2^(E - 127).
+ *
+ * Conventions for every entry point:
+ *  - All buffers are owned and allocated by the caller, in device memory of
+ *    the current CUDA device unless stated.  The library never allocates,
+ *    frees or synchronizes; every call is asynchronous and stream-ordered
+ *    on `stream` (0 = legacy default stream).
+ *  - Pointers must be non-NULL and 16-byte aligned.  Y must not alias any
+ *    input or the workspace.
+ *  - Errors are reported before any launch as a negative mxg_status; a
+ *    launch failure maps to MXG_ERR_CUDA.  A pipeline wait inside a kernel
+ *    that exceeds its time limit records MXG_ERR_TIMEOUT in the workspace
+ *    status word (read it with mxg_workspace_status) and the kernel returns.
+ *  - The GPU path does not scan inputs: NaN E4M3 codes (0x7F / 0xFF), E8M0
+ *    0xFF and non-finite scales give unspecified output.
+ */
+#ifndef MXG_H
+#define MXG_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define MXG_API __attribute__((visibility("default")))
+#else
+#define MXG_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MXG_OK = 0,
+    MXG_ERR_INVALID_ARG = -1,        /* NULL or misaligned pointer, M < 1, ... */
+    MXG_ERR_UNSUPPORTED_SHAPE = -2,  /* a size the format or the kernels reject */
+    MXG_ERR_WORKSPACE = -3,          /* workspace smaller than the size query */
+    MXG_ERR_CUDA = -4,               /* a CUDA runtime or launch error */
+    MXG_ERR_TIMEOUT = -5             /* a bounded in-kernel wait ran out */
+} mxg_status;
+
+/* Short English text for a status code (static storage, never NULL). */
+MXG_API const char *mxg_status_string(int status);
+
+/* ------------------------------------------------------------------ INT4 */
+
+/* Bytes of the re-packed weight buffer for a K x N layer with group size G:
+ * N*K/2 code bytes followed by 2*N*K/G scale bytes (no padding).  Returns 0
+ * for a shape w4a16_repack rejects. */
+MXG_API size_t w4a16_packed_bytes(int K, int N, int group_size);
+
+/* Offline re-pack (once per weight, after any fusion or sharding).
+ *   qweight  device, int32 [K/8][N], GPTQ words as described above.
+ *   scales   device, fp16 bits [K/G][N].
+ *   packed   device, caller-allocated, w4a16_packed_bytes(K, N, G) bytes.
+ * Layout written (private to this library, stable for a given K, N, G):
+ * codes as [N/16][K/64][32 lanes][16 B] so that one 16-byte load is one
+ * lane's mma fragment for four k16 steps, then scales as [N/16][K/G][16].
+ * Requirements: G in {32, 64, 128}; K % 64 == 0; K % G == 0; N % 64 == 0.
+ * Otherwise MXG_ERR_UNSUPPORTED_SHAPE. */
+MXG_API int w4a16_repack(const int32_t *qweight, const uint16_t *scales,
+                 int K, int N, int group_size, void *packed, cudaStream_t stream);
+
+/* Workspace bytes w4a16_gemm needs for this shape on the current device
+ * (split-K partial sums, arrival counters and the status word). */
+MXG_API size_t w4a16_workspace_bytes(int M, int N, int K, int group_size);
+
+/* Y = X * dequant(W)^T.
+ *   X         device, bf16 [M][K] row-major.
+ *   packed    device, output of w4a16_repack for (K, N, G).
+ *   Y         device, bf16 [M][N] row-major.
+ *   workspace device, >= w4a16_workspace_bytes(M, N, K, G) bytes, zero-filled
+ *             once before its first use; every call leaves it zero-filled
+ *             again (except the status word after an error).  Calls that
+ *             share a workspace must be ordered on one stream.
+ * M >= 1.  M <= 32 runs the weight-streaming path (the layer is bound by HBM
+ * bytes of W); larger M runs the tensor-core path.  Shape rules as for
+ * w4a16_repack. */
+MXG_API int w4a16_gemm(const void *X, const void *packed, int M, int N, int K, int group_size,
+               void *Y, void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* ----------------------------------------------------------------- MXFP8 */
+
+/* Workspace bytes mxfp8_gemm needs for this shape on the current device. */
+MXG_API size_t mxfp8_workspace_bytes(int M, int N, int K);
+
+/* Y = X * dequant(W)^T with MXFP8 weights.
+ *   X   device, bf16 [M][K];  Wq device, E4M3 [N][K];  Ws device, E8M0 [N][K/32];
+ *   Y   device, bf16 [M][N];  workspace as for w4a16_gemm.
+ * Requirements (the format's kernel constraints): N >= 128 and K % 32 == 0,
+ * else MXG_ERR_UNSUPPORTED_SHAPE.  N need not be a multiple of 16 and K need
+ * not be a multiple of 128: ragged tiles are predicated.  Activations stay
+ * bf16 (weight-only quantization). */
+MXG_API int mxfp8_gemm(const void *X, const uint8_t *Wq, const uint8_t *Ws, int M, int N, int K,
+               void *Y, void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* --------------------------------------------------- test and diagnostics */
+
+/* Decode a re-packed INT4 buffer with the device routines of the GEMM paths.
+ *   codes  device, uint8 [N][K]: the 4-bit codes;
+ *   w_fp32 device, float [N][K] or NULL: (q - 8) * scale, exact in fp32;
+ *   w_bf16 device, bf16 bits [N][K] or NULL: the bf16 nearest (q - 8) * scale
+ *          (ties to even), the operand of the tensor-core path. */
+MXG_API int w4a16_unpack(const void *packed, int K, int N, int group_size,
+                 uint8_t *codes, float *w_fp32, uint16_t *w_bf16, cudaStream_t stream);
+
+/* Decode MXFP8 weights with the device routine of the GEMM paths:
+ * w_bf16[N][K] = bf16 nearest e4m3(Wq) * 2^(Ws - 127) (exact whenever that
+ * value is a normal bf16). */
+MXG_API int mxfp8_dequant(const uint8_t *Wq, const uint8_t *Ws, int N, int K,
+                  uint16_t *w_bf16, cudaStream_t stream);
+
+/* Copy the workspace status word to the host (synchronizes `stream`).
+ * *status receives MXG_OK or the first error a kernel recorded. */
+MXG_API int mxg_workspace_status(const void *workspace, int *status, cudaStream_t stream);
+
+/* Runs one CTA whose pipeline wait can never complete (nothing arrives on
+ * its barrier) with a time limit of `limit_us` microseconds, to exercise the
+ * timeout path.  The kernel records MXG_ERR_TIMEOUT in the workspace status
+ * word and returns; the context stays usable.  workspace: >= 256 bytes. */
+MXG_API int mxg_selftest_wait_timeout(void *workspace, int limit_us, cudaStream_t stream);
+
+/* Path override for tests and benchmarks (process-wide):
+ * 0 = automatic (default), 1 = weight-streaming path, 2 = tensor-core path.
+ * The streaming path accepts M <= 32 only.  Returns the previous setting. */
+MXG_API int mxg_set_path(int path);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXG_H */

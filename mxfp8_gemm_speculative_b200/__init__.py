@@ -1,0 +1,236 @@
+"""Python binding of libmxg.so: weight-quantized linear layer on B200.
+
+    Y[M][N] = X[M][K] * dequant(W)^T     bf16 activations, fp32 accumulate, bf16 out
+
+with GPTQ-style symmetric INT4 weights (``w4a16_*``) or MXFP8 weights
+(``mxfp8_*``).  Every function here only marshals arguments into the C ABI
+declared in ``include/mxg.h`` (same names); all computation runs in the
+library's CUDA kernels.  PyTorch provides device memory and the current
+stream.  There is no CPU fallback: importing this module raises if the
+compiled library is missing.
+
+Workspace: the GEMMs need a caller-owned, zero-initialised workspace that
+they leave zeroed.  The functions below keep one per (device, stream) and
+grow it on demand; pass ``workspace=`` to manage it yourself.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmxg.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -c 'import __graft_entry__ as g; g.build()'`"
+        " (nvcc, sm_100a). There is no fallback implementation.")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_p = ctypes.c_void_p
+_i = ctypes.c_int
+_sz = ctypes.c_size_t
+
+_SIGS = {
+    "mxg_status_string": (ctypes.c_char_p, [_i]),
+    "w4a16_packed_bytes": (_sz, [_i, _i, _i]),
+    "w4a16_repack": (_i, [_p, _p, _i, _i, _i, _p, _p]),
+    "w4a16_workspace_bytes": (_sz, [_i, _i, _i, _i]),
+    "w4a16_gemm": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _sz, _p]),
+    "mxfp8_workspace_bytes": (_sz, [_i, _i, _i]),
+    "mxfp8_gemm": (_i, [_p, _p, _p, _i, _i, _i, _p, _p, _sz, _p]),
+    "w4a16_unpack": (_i, [_p, _i, _i, _i, _p, _p, _p, _p]),
+    "mxfp8_dequant": (_i, [_p, _p, _i, _i, _p, _p]),
+    "mxg_workspace_status": (_i, [_p, ctypes.POINTER(_i), _p]),
+    "mxg_selftest_wait_timeout": (_i, [_p, _i, _p]),
+    "mxg_set_path": (_i, [_i]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+EXPORTED = tuple(_SIGS)
+
+MXG_OK = 0
+MXG_ERR_INVALID_ARG = -1
+MXG_ERR_UNSUPPORTED_SHAPE = -2
+MXG_ERR_WORKSPACE = -3
+MXG_ERR_CUDA = -4
+MXG_ERR_TIMEOUT = -5
+
+
+class MxgError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {mxg_status_string(status)} (status {status})")
+        self.status = status
+
+
+def mxg_status_string(status: int) -> str:
+    return _lib.mxg_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != MXG_OK:
+        raise MxgError(status, what)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, dtype, name: str) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+# ------------------------------------------------------------- workspaces
+_ws_lock = threading.Lock()
+_ws_cache: dict[tuple[int, int], torch.Tensor] = {}
+
+
+def workspace(nbytes: int, device=None, stream=None) -> torch.Tensor:
+    """A zero-filled uint8 workspace of at least ``nbytes`` for (device, stream)."""
+    dev = torch.device("cuda", torch.cuda.current_device() if device is None else
+                       torch.device(device).index)
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    key = (dev.index, s.cuda_stream)
+    with _ws_lock:
+        ws = _ws_cache.get(key)
+        if ws is None or ws.numel() < nbytes:
+            ws = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=dev)
+            _ws_cache[key] = ws
+        return ws
+
+
+# -------------------------------------------------------------------- INT4
+def w4a16_packed_bytes(K: int, N: int, group_size: int = 128) -> int:
+    return int(_lib.w4a16_packed_bytes(K, N, group_size))
+
+
+def w4a16_repack(qweight: torch.Tensor, scales: torch.Tensor, group_size: int = 128,
+                 stream=None) -> torch.Tensor:
+    """Re-pack GPTQ words qweight[K/8][N] (int32) and scales[K/G][N] (fp16)."""
+    _need(qweight, torch.int32, "qweight")
+    if scales.dtype not in (torch.float16, torch.int16):
+        raise ValueError("scales must be float16 (or its int16 bit view)")
+    _need(scales, scales.dtype, "scales")
+    K = qweight.shape[0] * 8
+    N = qweight.shape[1]
+    nbytes = w4a16_packed_bytes(K, N, group_size)
+    if nbytes == 0:
+        raise MxgError(MXG_ERR_UNSUPPORTED_SHAPE, "w4a16_repack")
+    packed = torch.empty(nbytes, dtype=torch.uint8, device=qweight.device)
+    _check(_lib.w4a16_repack(_ptr(qweight), _ptr(scales), K, N, group_size, _ptr(packed),
+                             _stream(stream)), "w4a16_repack")
+    return packed
+
+
+def w4a16_workspace_bytes(M: int, N: int, K: int, group_size: int = 128) -> int:
+    return int(_lib.w4a16_workspace_bytes(M, N, K, group_size))
+
+
+def w4a16_gemm(x: torch.Tensor, packed: torch.Tensor, N: int, K: int, group_size: int = 128,
+               out: torch.Tensor | None = None, workspace_buf: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """Y = x * dequant(W)^T for x bf16 [M][K] and a re-packed INT4 weight."""
+    _need(x, torch.bfloat16, "x")
+    M = x.shape[0]
+    if x.dim() != 2 or x.shape[1] != K:
+        raise ValueError("x must be [M][K]")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(out, torch.bfloat16, "out")
+    need = w4a16_workspace_bytes(M, N, K, group_size)
+    ws = workspace_buf if workspace_buf is not None else workspace(need, x.device, stream)
+    _check(_lib.w4a16_gemm(_ptr(x), _ptr(packed), M, N, K, group_size, _ptr(out), _ptr(ws),
+                           ws.numel(), _stream(stream)), "w4a16_gemm")
+    return out
+
+
+def w4a16_unpack(packed: torch.Tensor, K: int, N: int, group_size: int = 128, stream=None):
+    """(codes uint8 [N][K], w_fp32 float32 [N][K], w_bf16 bfloat16 [N][K])."""
+    dev = packed.device
+    codes = torch.empty((N, K), dtype=torch.uint8, device=dev)
+    w32 = torch.empty((N, K), dtype=torch.float32, device=dev)
+    w16 = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    _check(_lib.w4a16_unpack(_ptr(packed), K, N, group_size, _ptr(codes), _ptr(w32), _ptr(w16),
+                             _stream(stream)), "w4a16_unpack")
+    return codes, w32, w16
+
+
+# ------------------------------------------------------------------- MXFP8
+def mxfp8_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(_lib.mxfp8_workspace_bytes(M, N, K))
+
+
+def mxfp8_gemm(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor,
+               out: torch.Tensor | None = None, workspace_buf: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """Y = x * dequant(W)^T for x bf16 [M][K], E4M3 codes wq[N][K], E8M0 ws[N][K/32]."""
+    _need(x, torch.bfloat16, "x")
+    if wq.dtype not in (torch.uint8, torch.float8_e4m3fn):
+        raise ValueError("wq must be uint8 or float8_e4m3fn")
+    if ws.dtype not in (torch.uint8, torch.float8_e8m0fnu):
+        raise ValueError("ws must be uint8 or float8_e8m0fnu")
+    _need(wq, wq.dtype, "wq")
+    _need(ws, ws.dtype, "ws")
+    M, K = x.shape
+    N = wq.shape[0]
+    if wq.shape[1] != K or ws.shape[0] != N or ws.shape[1] * 32 != K:
+        raise ValueError("shape mismatch between x, wq and ws")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(out, torch.bfloat16, "out")
+    need = mxfp8_workspace_bytes(M, N, K)
+    wsb = workspace_buf if workspace_buf is not None else workspace(need, x.device, stream)
+    _check(_lib.mxfp8_gemm(_ptr(x), _ptr(wq), _ptr(ws), M, N, K, _ptr(out), _ptr(wsb),
+                           wsb.numel(), _stream(stream)), "mxfp8_gemm")
+    return out
+
+
+def mxfp8_dequant(wq: torch.Tensor, ws: torch.Tensor, stream=None) -> torch.Tensor:
+    N, K = wq.shape
+    out = torch.empty((N, K), dtype=torch.bfloat16, device=wq.device)
+    _check(_lib.mxfp8_dequant(_ptr(wq), _ptr(ws), N, K, _ptr(out), _stream(stream)),
+           "mxfp8_dequant")
+    return out
+
+
+# ------------------------------------------------------------- diagnostics
+def mxg_workspace_status(workspace_buf: torch.Tensor, stream=None) -> int:
+    v = ctypes.c_int(0)
+    _check(_lib.mxg_workspace_status(_ptr(workspace_buf), ctypes.byref(v), _stream(stream)),
+           "mxg_workspace_status")
+    return v.value
+
+
+def mxg_selftest_wait_timeout(workspace_buf: torch.Tensor, limit_us: int, stream=None) -> None:
+    _check(_lib.mxg_selftest_wait_timeout(_ptr(workspace_buf), int(limit_us), _stream(stream)),
+           "mxg_selftest_wait_timeout")
+
+
+def mxg_set_path(path: int) -> int:
+    """0 = automatic, 1 = weight streaming, 2 = tensor cores; returns the previous value."""
+    r = int(_lib.mxg_set_path(int(path)))
+    if r < 0:
+        raise ValueError("path must be 0, 1 or 2")
+    return r
+
+
+def raw_lib() -> ctypes.CDLL:
+    """The loaded C library (for callers that pass raw pointers)."""
+    return _lib

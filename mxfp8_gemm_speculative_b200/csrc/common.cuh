@@ -1,0 +1,284 @@
+// Device helpers shared by the mxg kernels (sm_100a only).
+//
+// PTX wrappers for mbarriers, bulk and tensor copies, warp-level MMA and the
+// exact weight decoders of both formats.  Nothing here allocates or
+// synchronizes the device.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "mxg.h"
+
+namespace mxg {
+
+// ---------------------------------------------------------------- workspace
+// The first 256 bytes of every workspace are a header; `status` receives the
+// first error a kernel records and `where` a code for the place it happened.
+struct WsHeader {
+    int status;
+    int where;
+    int reserved[62];
+};
+static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
+
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per pipeline wait
+
+__device__ __forceinline__ void record_error(WsHeader *h, int status, int where)
+{
+    if (atomicCAS(&h->status, 0, status) == 0)
+        atomicExch(&h->where, where);
+}
+
+// ------------------------------------------------------------------- basics
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long global_ns()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ---------------------------------------------------------------- mbarriers
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+
+// Make barrier initialisation visible to the async proxy (TMA, tcgen05).
+__device__ __forceinline__ void fence_barrier_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete; false after
+// `limit_ns` nanoseconds without completion.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
+                                          unsigned long long limit_ns)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const unsigned long long t0 = global_ns();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try_wait(bar, parity))
+                return true;
+        if (global_ns() - t0 > limit_ns)
+            return false;
+    }
+}
+
+// ------------------------------------------------------------- bulk copies
+__device__ __forceinline__ uint64_t l2_policy_evict_first()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_last()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// Contiguous global -> shared copy completing on `bar` (bytes % 16 == 0,
+// both addresses 16-byte aligned).
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
+                                         uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
+// 2-D tiled tensor copy of box (c0, c1) into shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int c0, int c1,
+                                            uint64_t *bar, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map)
+{
+    asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+
+// ------------------------------------------------------------------ loads
+__device__ __forceinline__ uint4 lds128(const void *p)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(smem_u32(p)));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t lds32(const void *p)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)));
+    return v;
+}
+
+// Read-only 16-byte global load kept in L1 (activations are re-read by
+// many warps).
+__device__ __forceinline__ uint4 ldg128(const void *p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// 16-byte load from L2 (bypassing L1), for partial sums written by other CTAs.
+__device__ __forceinline__ float4 ldcg_f4(const float *p)
+{
+    return __ldcg(reinterpret_cast<const float4 *>(p));
+}
+
+// ----------------------------------------------------------- warp-level MMA
+// D(16x8, fp32) += A(16x16, bf16, row) * B(16x8, bf16, col).
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// --------------------------------------------------------- INT4 decoding
+// Two 4-bit codes q_lo = bits [s, s+3] and q_hi = bits [16+s, 16+s+3] of w,
+// returned as the bf16 pair (q_lo - 8, q_hi - 8).  Exact: 0x4300 | q is the
+// bf16 value 128 + q (one unit in the last place is 1 at exponent 7), and
+// subtracting 136 leaves the small integer q - 8.
+template <int S>
+__device__ __forceinline__ uint32_t int4_pair_minus8(uint32_t w)
+{
+    const uint32_t t = ((w >> S) & 0x000F000Fu) | 0x43004300u;
+    uint32_t r;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(t), "r"(0x3F803F80u), "r"(0xC308C308u));
+    return r;
+}
+
+// An fp16 scale s split as s = hi + lo with hi, lo both bf16: hi keeps the
+// top 8 significant bits of s, lo the remaining (at most 3) bits.  Both are
+// broadcast to the two halves of a bf16x2 register.
+struct ScaleSplit {
+    uint32_t hi2;
+    uint32_t lo2;
+};
+
+__device__ __forceinline__ ScaleSplit split_scale(uint16_t s_bits)
+{
+    const float f = __half2float(__ushort_as_half(s_bits));
+    const uint32_t fb = __float_as_uint(f);
+    const uint32_t hi = fb & 0xFFFF0000u;                 // truncated to bf16
+    const float lo = f - __uint_as_float(hi);              // exact remainder
+    const uint32_t lob = __float_as_uint(lo) >> 16;        // exact in bf16
+    ScaleSplit r;
+    r.hi2 = hi | (hi >> 16);
+    r.lo2 = lob | (lob << 16);
+    return r;
+}
+
+// bf16 nearest to (q - 8) * s for a pair of exact (q - 8) values, with one
+// rounding: (q-8)*lo is exact in bf16 (<= 4 x 3 significant bits), and the
+// fused multiply-add (q-8)*hi + (q-8)*lo rounds the exact product once.
+__device__ __forceinline__ uint32_t scale_pair_rn(uint32_t qm8, const ScaleSplit &s)
+{
+    uint32_t t, r;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(t) : "r"(qm8), "r"(s.lo2));
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(qm8), "r"(s.hi2), "r"(t));
+    return r;
+}
+
+// -------------------------------------------------------- MXFP8 decoding
+// fp32 value of an E8M0 exponent: 2^(E - 127) (E = 0 is the fp32 subnormal
+// 2^-127; E = 255, NaN in the format, is not checked).
+__device__ __forceinline__ float e8m0_to_f32(uint32_t e)
+{
+    return e ? __uint_as_float(e << 23) : __uint_as_float(0x00400000u);
+}
+
+// Four E4M3 codes (the bytes of w, byte 0 first) times `scale`, as two bf16
+// pairs: r01 = (w0, w1), r23 = (w2, w3).  E4M3 -> f16 is exact in hardware,
+// f16 -> f32 is exact, the product with a power of two is exact in fp32, and
+// the only rounding is the final fp32 -> bf16 (nearest, ties to even).
+__device__ __forceinline__ void e4m3x4_scaled(uint32_t w, float scale, uint32_t &r01, uint32_t &r23)
+{
+    uint32_t h01, h23;
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "mov.b32 {lo, hi}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, lo;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+        : "=r"(h01), "=r"(h23)
+        : "r"(w));
+    float2 f01 = __half22float2(*reinterpret_cast<__half2 *>(&h01));
+    float2 f23 = __half22float2(*reinterpret_cast<__half2 *>(&h23));
+    f01.x *= scale;
+    f01.y *= scale;
+    f23.x *= scale;
+    f23.y *= scale;
+    __nv_bfloat162 b01 = __float22bfloat162_rn(f01);
+    __nv_bfloat162 b23 = __float22bfloat162_rn(f23);
+    r01 = *reinterpret_cast<uint32_t *>(&b01);
+    r23 = *reinterpret_cast<uint32_t *>(&b23);
+}
+
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float v)
+{
+    return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+}  // namespace mxg

@@ -1,0 +1,88 @@
+// Internal launch interface of the mxg kernels (not part of the C ABI).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace mxg {
+
+// ------------------------------------------------------------ device facts
+struct DeviceInfo {
+    int sms;              // streaming multiprocessors
+    int smem_optin;       // max dynamic shared memory per block (bytes)
+};
+const DeviceInfo &device_info(int device);
+
+// ------------------------------------------------------------ workspace map
+// [0, 256)              header (status word)
+// [256, 256 + T)        arrival counters, T = round_up(4 * counters, 256)
+// [256 + T, ...)        fp32 partial sums
+struct WorkspaceMap {
+    size_t counters_off;
+    size_t counters;      // number of int counters
+    size_t partial_off;
+    size_t partial_bytes;
+    size_t total;
+};
+WorkspaceMap make_workspace_map(size_t counters, size_t partial_bytes);
+
+// ------------------------------------------------------ weight-streaming path
+// Stream-K plan: the layer's weight bytes are cut into equal "units" (one
+// n16 tile x one scale group, or one n16 tile x 128 k for MXFP8) and every
+// warp of a persistent grid takes one contiguous run of units.
+struct StreamPlan {
+    int tt;               // token tiles of 8 rows (ceil(M / 8)), 1..4
+    int variant;          // kernel variant (group mode for INT4)
+    int warps_per_cta;
+    int grid;             // CTAs
+    int Wt;               // active warps (<= grid * warps_per_cta, <= units)
+    long long units;      // total units
+    int upt;              // units per n16 tile
+    size_t smem;          // dynamic shared memory per CTA
+    size_t partial_bytes; // workspace for partial sums
+    int ntiles;           // n16 tiles (= arrival counters)
+};
+
+bool plan_w4a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan);
+cudaError_t launch_w4a16_stream(const StreamPlan &plan, const void *X, const void *packed, int M,
+                                int N, int K, int G, void *Y, void *workspace, cudaStream_t stream);
+
+bool plan_mxfp8_stream(int device, int M, int N, int K, StreamPlan *plan);
+cudaError_t launch_mxfp8_stream(const StreamPlan &plan, const void *X, const uint8_t *Wq,
+                                const uint8_t *Ws, int M, int N, int K, void *Y, void *workspace,
+                                cudaStream_t stream);
+
+// ----------------------------------------------------- tensor-core path
+struct TcPlan {
+    int bm, bn, bk;       // CTA tile
+    int mtiles, ntiles;   // output tiles
+    int splits;           // K splits (1 = none)
+    int grid;             // CTAs (persistent)
+    size_t smem;
+    size_t partial_bytes; // split-K partial sums
+    size_t counters;      // split-K arrival counters
+};
+bool plan_w4a16_tc(int device, int M, int N, int K, int G, TcPlan *plan);
+cudaError_t launch_w4a16_tc(const TcPlan &plan, const void *X, const void *packed, int M, int N,
+                            int K, int G, void *Y, void *workspace, cudaStream_t stream);
+bool plan_mxfp8_tc(int device, int M, int N, int K, TcPlan *plan);
+cudaError_t launch_mxfp8_tc(const TcPlan &plan, const void *X, const uint8_t *Wq,
+                            const uint8_t *Ws, int M, int N, int K, void *Y, void *workspace,
+                            cudaStream_t stream);
+
+// ------------------------------------------------------------ weight tools
+cudaError_t launch_w4a16_repack(const int32_t *qweight, const uint16_t *scales, int K, int N, int G,
+                                void *packed, cudaStream_t stream);
+cudaError_t launch_w4a16_unpack(const void *packed, int K, int N, int G, uint8_t *codes,
+                                float *w_fp32, uint16_t *w_bf16, cudaStream_t stream);
+cudaError_t launch_mxfp8_dequant(const uint8_t *Wq, const uint8_t *Ws, int N, int K,
+                                 uint16_t *w_bf16, cudaStream_t stream);
+cudaError_t launch_wait_timeout_selftest(void *workspace, int limit_us, cudaStream_t stream);
+
+// Encodes tensor maps through the driver entry point (no libcuda link).
+bool encode_tensor_map_2d(void *map, int dtype_cu, const void *base, uint64_t inner,
+                          uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
+                          uint32_t box_outer, int swizzle_cu);
+
+}  // namespace mxg

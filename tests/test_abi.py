@@ -1,0 +1,86 @@
+"""The C ABI library: loads, exports every declared symbol, validates
+arguments before touching the GPU (no kernel runs here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mxg.h")
+
+
+@pytest.fixture(scope="module")
+def mxg():
+    import __graft_entry__
+    __graft_entry__.build()
+    import mxfp8_gemm_speculative_b200 as m
+    return m
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*MXG_API\s+(?:const\s+)?[a-z_0-9]+\s*\**\s*([a-z_0-9]+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ["w4a16_packed_bytes", "w4a16_repack", "w4a16_workspace_bytes", "w4a16_gemm",
+                 "mxfp8_workspace_bytes", "mxfp8_gemm", "w4a16_unpack", "mxfp8_dequant",
+                 "mxg_status_string"]:
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(mxg):
+    lib = ctypes.CDLL(mxg.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(declared_functions()) == set(mxg.EXPORTED)
+
+
+def test_status_strings(mxg):
+    for s in range(-5, 1):
+        assert mxg.mxg_status_string(s) not in ("", "unknown status")
+    assert mxg.mxg_status_string(-99) == "unknown status"
+
+
+def test_packed_bytes(mxg):
+    assert mxg.w4a16_packed_bytes(5120, 17408, 128) == 44564480 + 1392640
+    assert mxg.w4a16_packed_bytes(5120, 5120, 128) == 13107200 + 409600
+    assert mxg.w4a16_packed_bytes(512, 512, 32) == 512 * 512 // 2 + 512 * 16 * 2
+    assert mxg.w4a16_packed_bytes(512, 512, 48) == 0       # group size
+    assert mxg.w4a16_packed_bytes(500, 512, 128) == 0      # K % G
+    assert mxg.w4a16_packed_bytes(512, 96, 128) == 0       # N % 64
+
+
+def test_arguments_rejected_before_launch(mxg):
+    lib = mxg.raw_lib()
+    a = ctypes.c_void_p(4096)          # aligned, never dereferenced on these paths
+    mis = ctypes.c_void_p(4096 + 8)
+    null = None
+    # NULL / misaligned pointers
+    assert lib.w4a16_gemm(null, a, 5, 512, 512, 128, a, a, 1 << 20, null) == mxg.MXG_ERR_INVALID_ARG
+    assert lib.w4a16_gemm(a, mis, 5, 512, 512, 128, a, a, 1 << 20, null) == mxg.MXG_ERR_INVALID_ARG
+    assert lib.mxfp8_gemm(a, a, mis, 4, 256, 512, a, a, 1 << 20, null) == mxg.MXG_ERR_INVALID_ARG
+    assert lib.w4a16_repack(a, null, 512, 512, 128, a, null) == mxg.MXG_ERR_INVALID_ARG
+    # M < 1
+    assert lib.w4a16_gemm(a, a, 0, 512, 512, 128, a, a, 1 << 20, null) == mxg.MXG_ERR_INVALID_ARG
+    # shapes the format or the kernels reject
+    assert lib.w4a16_gemm(a, a, 5, 512, 512, 96, a, a, 1 << 20, null) == mxg.MXG_ERR_UNSUPPORTED_SHAPE
+    assert lib.w4a16_gemm(a, a, 5, 96, 512, 128, a, a, 1 << 20, null) == mxg.MXG_ERR_UNSUPPORTED_SHAPE
+    assert lib.w4a16_repack(a, a, 480, 512, 32, a, null) == mxg.MXG_ERR_UNSUPPORTED_SHAPE
+    assert lib.mxfp8_gemm(a, a, a, 4, 96, 512, a, a, 1 << 20, null) == mxg.MXG_ERR_UNSUPPORTED_SHAPE
+    assert lib.mxfp8_gemm(a, a, a, 4, 256, 500, a, a, 1 << 20, null) == mxg.MXG_ERR_UNSUPPORTED_SHAPE
+    assert lib.mxfp8_dequant(a, a, 96, 512, a, null) == mxg.MXG_ERR_UNSUPPORTED_SHAPE
+    assert lib.w4a16_unpack(a, 512, 512, 128, mis, null, null, null) == mxg.MXG_ERR_INVALID_ARG
+    assert lib.mxg_selftest_wait_timeout(a, 0, null) == mxg.MXG_ERR_INVALID_ARG
+
+
+def test_path_override_roundtrip(mxg):
+    prev = mxg.mxg_set_path(1)
+    assert mxg.mxg_set_path(2) == 1
+    assert mxg.mxg_set_path(prev) == 2
+    with pytest.raises(ValueError):
+        mxg.mxg_set_path(3)

@@ -1,0 +1,231 @@
+"""GPU parity of the weight tools and the small-M (weight-streaming) path,
+through the C ABI, against the CPU oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from helpers import (assert_parity, assert_sampled_parity, bf16_tensor, bits_of_bf16, to_f64)
+
+pytestmark = pytest.mark.gpu
+
+DEV = torch.device("cuda", 0)
+
+
+@pytest.fixture(scope="module")
+def mxg():
+    import __graft_entry__
+    __graft_entry__.build()
+    import mxfp8_gemm_speculative_b200 as m
+    m.mxg_set_path(0)
+    return m
+
+
+def int4_device(lay):
+    qw = torch.from_numpy(lay.qweight).to(DEV)
+    sc = torch.from_numpy(lay.scales.view(np.int16)).to(DEV)
+    return qw, sc
+
+
+def run_int4(mxg, lay, path=0):
+    qw, sc = int4_device(lay)
+    packed = mxg.w4a16_repack(qw, sc, lay.group_size)
+    prev = mxg.mxg_set_path(path)
+    try:
+        y = mxg.w4a16_gemm(bf16_tensor(lay.X, DEV), packed, lay.N, lay.K, lay.group_size)
+    finally:
+        mxg.mxg_set_path(prev)
+    return y, packed
+
+
+# --------------------------------------------------------------- weight tools
+@pytest.mark.parametrize("K,N,G", [(512, 512, 128), (1024, 192, 64), (256, 320, 32), (384, 64, 128)])
+def test_repack_unpack_bit_exact(mxg, K, N, G):
+    lay = synth.int4_layer(1, K, N, G, seed=K + N + G)
+    qw, sc = int4_device(lay)
+    packed = mxg.w4a16_repack(qw, sc, G)
+    assert packed.numel() == mxg.w4a16_packed_bytes(K, N, G)
+    codes, w32, w16 = mxg.w4a16_unpack(packed, K, N, G)
+    ocodes, ow = oracle.w4a16_unpack(lay.qweight, lay.scales, K, N, G)
+    assert np.array_equal(codes.cpu().numpy(), ocodes)
+    assert np.array_equal(w32.cpu().numpy().astype(np.float64), ow)     # exact in fp32
+    want16 = oracle.round_bf16_array(ow)
+    assert np.array_equal(bits_of_bf16(w16), want16)
+
+
+def test_unpack_every_scale_pattern(mxg):
+    """All finite positive fp16 scales, every code: the bf16 dequant rounds once."""
+    K, N, G = 64, 64, 32
+    rng = np.random.default_rng(0)
+    all_pos = np.arange(1, 0x7C00, dtype=np.uint16)           # positive finite fp16
+    for start in range(0, all_pos.size, (K // G) * N):
+        chunk = all_pos[start:start + (K // G) * N]
+        sc = np.resize(chunk, (K // G) * N).reshape(K // G, N).astype(np.uint16)
+        codes = rng.integers(0, 16, size=(N, K), dtype=np.uint8)
+        lay = synth.Int4Layer(1, K, N, G, np.zeros((1, K), np.uint16), codes,
+                              synth.pack_codes_gptq(codes), sc)
+        qw, scd = int4_device(lay)
+        packed = mxg.w4a16_repack(qw, scd, G)
+        _, w32, w16 = mxg.w4a16_unpack(packed, K, N, G)
+        _, ow = oracle.w4a16_unpack(lay.qweight, sc, K, N, G)
+        assert np.array_equal(w32.cpu().numpy().astype(np.float64), ow)
+        assert np.array_equal(bits_of_bf16(w16), oracle.round_bf16_array(ow)), start
+
+
+@pytest.mark.parametrize("E", [100, 119, 121, 123, 127, 140])
+def test_mxfp8_dequant_bit_exact(mxg, E):
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    N, K = 128, 256
+    Wq = np.resize(codes, N * K).reshape(N, K).astype(np.uint8)
+    Ws = np.full((N, K // 32), E, dtype=np.uint8)
+    Ws[::3] = np.uint8(E - 2)
+    w16 = mxg.mxfp8_dequant(torch.from_numpy(Wq).to(DEV), torch.from_numpy(Ws).to(DEV))
+    ow = oracle.mxfp8_dequant(Wq, Ws, N, K)
+    assert np.array_equal(bits_of_bf16(w16), oracle.round_bf16_array(ow))
+
+
+# ------------------------------------------------------------ INT4 streaming
+M_STREAM = [1, 2, 3, 4, 5, 8, 16, 17, 31, 32]
+
+
+@pytest.mark.parametrize("M", M_STREAM)
+@pytest.mark.parametrize("K,N,G", [(512, 512, 128), (1024, 192, 64), (256, 320, 32), (1280, 640, 128)])
+def test_int4_stream_parity(mxg, M, K, N, G):
+    lay = synth.int4_layer(M, K, N, G, seed=7 * M + K + N + G)
+    y, _ = run_int4(mxg, lay, path=1)
+    ref = oracle.w4a16_gemm(lay.X, lay.qweight, lay.scales, M, N, K, G)
+    assert_parity(to_f64(y), ref, f"int4 stream M={M} K={K} N={N} G={G}")
+
+
+@pytest.mark.parametrize("M", [1, 5, 8, 13, 32])
+@pytest.mark.parametrize("G", [32, 64, 128])
+def test_int4_stream_exact_integer_regime(mxg, M, G):
+    rng = np.random.default_rng(M + G)
+    K, N = 1024, 256
+    xi = rng.integers(-3, 4, size=(M, K)).astype(np.float32)
+    X = torch.from_numpy(xi).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    codes = rng.integers(0, 16, size=(N, K), dtype=np.uint8)
+    e = rng.integers(-2, 3, size=(K // G, N))
+    sc = np.array([[np.float16(2.0 ** v) for v in row] for row in e]).view(np.uint16)
+    lay = synth.Int4Layer(M, K, N, G, X, codes, synth.pack_codes_gptq(codes), sc)
+    y, _ = run_int4(mxg, lay, path=1)
+    ref = oracle.w4a16_gemm(X, lay.qweight, sc, M, N, K, G)
+    want = oracle.round_bf16_array(ref).reshape(M, N)
+    assert np.array_equal(bits_of_bf16(y), want)
+
+
+def test_int4_identity_is_exact(mxg):
+    K = N = 512
+    codes = np.full((N, K), 8, dtype=np.uint8)
+    np.fill_diagonal(codes, 9)
+    sc = np.full((K // 128, N), 0x3000, dtype=np.uint16)   # 2^-3
+    X = synth.int4_layer(7, K, N, 128, seed=1).X
+    lay = synth.Int4Layer(7, K, N, 128, X, codes, synth.pack_codes_gptq(codes), sc)
+    y, _ = run_int4(mxg, lay, path=1)
+    xin = torch.from_numpy(X.view(np.int16)).view(torch.bfloat16).float() * 0.125
+    assert np.array_equal(bits_of_bf16(y), bits_of_bf16(xin.to(torch.bfloat16)))
+
+
+def test_int4_tiny_layer_config(mxg):
+    """M=1, K=N=512, group 128, seed 0: the tiny workload, in full."""
+    lay = synth.int4_layer(1, 512, 512, 128, seed=0)
+    y, _ = run_int4(mxg, lay)
+    ref = oracle.w4a16_gemm(lay.X, lay.qweight, lay.scales, 1, 512, 512, 128)
+    assert_parity(to_f64(y), ref, "tiny layer")
+
+
+def test_int4_deterministic_and_workspace_restored(mxg):
+    lay = synth.int4_layer(5, 2048, 1024, 128, seed=3)
+    qw, sc = int4_device(lay)
+    packed = mxg.w4a16_repack(qw, sc, 128)
+    ws = torch.zeros(mxg.w4a16_workspace_bytes(5, 1024, 2048, 128), dtype=torch.uint8, device=DEV)
+    x = bf16_tensor(lay.X, DEV)
+    y1 = mxg.w4a16_gemm(x, packed, 1024, 2048, 128, workspace_buf=ws)
+    y2 = mxg.w4a16_gemm(x, packed, 1024, 2048, 128, workspace_buf=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    assert int(ws.count_nonzero()) == 0
+    assert mxg.mxg_workspace_status(ws) == 0
+
+
+@pytest.mark.parametrize("li", [0, 1, 2])
+def test_int4_mtp4_verify_layers_sampled(mxg, li):
+    """The three MTP4 verify-chunk layers at full size (M=5): sampled outputs."""
+    K, N = synth.MTP4_VERIFY_LAYERS[li]
+    lay = synth.int4_layer(5, K, N, 128, seed=0, layer=li)
+    y, _ = run_int4(mxg, lay)
+    yf = to_f64(y)
+    rng = np.random.default_rng(li)
+    rows = rng.integers(0, 5, size=512)
+    cols = rng.integers(0, N, size=512)
+    ref = oracle.w4a16_gemm_at(lay.X, lay.qweight, lay.scales, 5, N, K, 128, rows, cols,
+                               nthreads=oracle.threads(64))
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    assert_sampled_parity(yf[rows, cols], ref, rms, f"MTP4 layer {li}")
+    # every column tile is written: no output left unset
+    assert np.isfinite(yf).all()
+
+
+# ------------------------------------------------------------ MXFP8 streaming
+@pytest.mark.parametrize("M", [1, 4, 5, 16, 17, 32])
+@pytest.mark.parametrize("N,K", [(128, 64), (130, 96), (256, 512), (1000, 2080)])
+def test_mxfp8_stream_parity(mxg, M, N, K):
+    lay = synth.mxfp8_layer(M, K, N, seed=M + N + K)
+    prev = mxg.mxg_set_path(1)
+    try:
+        y = mxg.mxfp8_gemm(bf16_tensor(lay.X, DEV), torch.from_numpy(lay.Wq).to(DEV),
+                           torch.from_numpy(lay.Ws).to(DEV))
+    finally:
+        mxg.mxg_set_path(prev)
+    ref = oracle.mxfp8_gemm(lay.X, lay.Wq, lay.Ws, M, N, K)
+    assert_parity(to_f64(y), ref, f"mxfp8 stream M={M} N={N} K={K}")
+
+
+def test_mxfp8_identity_is_exact(mxg):
+    K = N = 256
+    Wq = np.zeros((N, K), dtype=np.uint8)
+    np.fill_diagonal(Wq, 0x38)
+    Ws = np.full((N, K // 32), 124, dtype=np.uint8)
+    X = synth.mxfp8_layer(3, K, N, seed=2).X
+    y = mxg.mxfp8_gemm(bf16_tensor(X, DEV), torch.from_numpy(Wq).to(DEV), torch.from_numpy(Ws).to(DEV))
+    xin = torch.from_numpy(X.view(np.int16)).view(torch.bfloat16).float() * 0.125
+    assert np.array_equal(bits_of_bf16(y), bits_of_bf16(xin.to(torch.bfloat16)))
+
+
+def test_mxfp8_m4_full_size_sampled(mxg):
+    M, K, N = 4, 5120, 17408
+    lay = synth.mxfp8_layer(M, K, N, seed=0)
+    y = mxg.mxfp8_gemm(bf16_tensor(lay.X, DEV), torch.from_numpy(lay.Wq).to(DEV),
+                       torch.from_numpy(lay.Ws).to(DEV))
+    yf = to_f64(y)
+    rng = np.random.default_rng(5)
+    rows = rng.integers(0, M, size=512)
+    cols = rng.integers(0, N, size=512)
+    ref = oracle.mxfp8_gemm_at(lay.X, lay.Wq, lay.Ws, M, N, K, rows, cols,
+                               nthreads=oracle.threads(64))
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    assert_sampled_parity(yf[rows, cols], ref, rms, "mxfp8 M=4 full size")
+    assert np.isfinite(yf).all()
+
+
+# --------------------------------------------------------- failure handling
+def test_bounded_wait_reports_timeout(mxg):
+    ws = torch.zeros(4096, dtype=torch.uint8, device=DEV)
+    mxg.mxg_selftest_wait_timeout(ws, 2000)       # 2 ms limit on a wait nothing completes
+    assert mxg.mxg_workspace_status(ws) == mxg.MXG_ERR_TIMEOUT
+    # the context is still usable
+    lay = synth.int4_layer(2, 512, 512, 128, seed=9)
+    y, _ = run_int4(mxg, lay)
+    ref = oracle.w4a16_gemm(lay.X, lay.qweight, lay.scales, 2, 512, 512, 128)
+    assert_parity(to_f64(y), ref, "after timeout")
+
+
+def test_workspace_too_small_rejected(mxg):
+    lay = synth.int4_layer(5, 1024, 512, 128, seed=1)
+    qw, sc = int4_device(lay)
+    packed = mxg.w4a16_repack(qw, sc, 128)
+    ws = torch.zeros(256, dtype=torch.uint8, device=DEV)
+    with pytest.raises(mxg.MxgError) as e:
+        mxg.w4a16_gemm(bf16_tensor(lay.X, DEV), packed, 512, 1024, 128, workspace_buf=ws)
+    assert e.value.status == mxg.MXG_ERR_WORKSPACE
