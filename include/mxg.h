@@ -95,9 +95,12 @@ MXG_API size_t w4a16_workspace_bytes(int M, int N, int K, int group_size);
  *   packed    device, output of w4a16_repack for (K, N, G).
  *   Y         device, bf16 [M][N] row-major.
  *   workspace device, >= w4a16_workspace_bytes(M, N, K, G) bytes, zero-filled
- *             once before its first use; every call leaves it zero-filled
- *             again (except the status word after an error).  Calls that
- *             share a workspace must be ordered on one stream.
+ *             once before its first use.  Its first 256 bytes hold the status
+ *             word, then come arrival counters, then scratch for partial
+ *             sums; every call leaves the status word and the counters zero
+ *             again (except after an error, when the caller must zero it
+ *             before reuse), while the scratch keeps whatever it held.  Calls
+ *             that share a workspace must be ordered on one stream.
  * M >= 1.  M <= 32 runs the weight-streaming path (the layer is bound by HBM
  * bytes of W); larger M runs the tensor-core path.  Shape rules as for
  * w4a16_repack. */

@@ -82,7 +82,7 @@ WorkspaceMap make_workspace_map(size_t counters, size_t partial_bytes)
     WorkspaceMap m{};
     m.counters_off = sizeof(WsHeader);
     m.counters = counters;
-    m.partial_off = m.counters_off + round_up(counters * sizeof(int), 256);
+    m.partial_off = m.counters_off + kMaxCounters * sizeof(int);
     m.partial_bytes = partial_bytes;
     m.total = m.partial_off + round_up(partial_bytes, 256);
     return m;

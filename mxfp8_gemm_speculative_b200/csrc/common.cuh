@@ -169,13 +169,16 @@ __device__ __forceinline__ uint32_t lds32(const void *p)
 }
 
 // Read-only 16-byte global load kept in L1 (activations are re-read by
-// many warps).
+// many warps).  Visible to the compiler, which may schedule it early.
 __device__ __forceinline__ uint4 ldg128(const void *p)
 {
-    uint4 v;
-    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
+    return __ldg(reinterpret_cast<const uint4 *>(p));
+}
+
+__device__ __forceinline__ uint2 lds64(const void *p)
+{
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(smem_u32(p)));
     return v;
 }
 
@@ -190,11 +193,34 @@ __device__ __forceinline__ float4 ldcg_f4(const float *p)
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                                uint32_t a3, uint32_t b0, uint32_t b1)
 {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
         "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// D = A * B with a zero accumulator input (starts a new partial sum).
+__device__ __forceinline__ void mma_bf16_16816_zero(float (&d)[4], uint32_t a0, uint32_t a1,
+                                                    uint32_t a2, uint32_t a3, uint32_t b0,
+                                                    uint32_t b1)
+{
+    asm(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%10, %10, %10, %10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
+}
+
+// Arrival counter increment with acquire-release semantics at GPU scope:
+// publishes the caller's (and, after a warp barrier, its warp's) prior
+// stores and, for the last arriver, makes the other contributors' stores
+// visible.
+__device__ __forceinline__ int atomic_add_acq_rel(int *p, int v)
+{
+    int old;
+    asm volatile("atom.add.acq_rel.gpu.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
 }
 
 // --------------------------------------------------------- INT4 decoding
@@ -206,9 +232,11 @@ template <int S>
 __device__ __forceinline__ uint32_t int4_pair_minus8(uint32_t w)
 {
     const uint32_t t = ((w >> S) & 0x000F000Fu) | 0x43004300u;
-    uint32_t r;
-    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(t), "r"(0x3F803F80u), "r"(0xC308C308u));
-    return r;
+    // written with intrinsics so the compiler can fold the constant operand
+    const __nv_bfloat162 v = __hadd2(*reinterpret_cast<const __nv_bfloat162 *>(&t),
+                                     __halves2bfloat162(__ushort_as_bfloat16(0xC308),
+                                                        __ushort_as_bfloat16(0xC308)));
+    return *reinterpret_cast<const uint32_t *>(&v);
 }
 
 // An fp16 scale s split as s = hi + lo with hi, lo both bf16: hi keeps the
@@ -266,14 +294,19 @@ __device__ __forceinline__ void e4m3x4_scaled(uint32_t w, float scale, uint32_t 
         : "r"(w));
     float2 f01 = __half22float2(*reinterpret_cast<__half2 *>(&h01));
     float2 f23 = __half22float2(*reinterpret_cast<__half2 *>(&h23));
-    f01.x *= scale;
-    f01.y *= scale;
-    f23.x *= scale;
-    f23.y *= scale;
-    __nv_bfloat162 b01 = __float22bfloat162_rn(f01);
-    __nv_bfloat162 b23 = __float22bfloat162_rn(f23);
-    r01 = *reinterpret_cast<uint32_t *>(&b01);
-    r23 = *reinterpret_cast<uint32_t *>(&b23);
+    // packed fp32 multiplies (two lanes per instruction)
+    asm("{\n\t.reg .b64 a, b, s;\n\t"
+        "mov.b64 s, {%4, %4};\n\t"
+        "mov.b64 a, {%0, %1};\n\t"
+        "mov.b64 b, {%2, %3};\n\t"
+        "mul.rn.f32x2 a, a, s;\n\t"
+        "mul.rn.f32x2 b, b, s;\n\t"
+        "mov.b64 {%0, %1}, a;\n\t"
+        "mov.b64 {%2, %3}, b;\n\t}"
+        : "+f"(f01.x), "+f"(f01.y), "+f"(f23.x), "+f"(f23.y)
+        : "f"(scale));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r01) : "f"(f01.y), "f"(f01.x));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r23) : "f"(f23.y), "f"(f23.x));
 }
 
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float v)

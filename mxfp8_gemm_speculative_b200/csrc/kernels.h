@@ -15,9 +15,12 @@ struct DeviceInfo {
 const DeviceInfo &device_info(int device);
 
 // ------------------------------------------------------------ workspace map
-// [0, 256)              header (status word)
-// [256, 256 + T)        arrival counters, T = round_up(4 * counters, 256)
-// [256 + T, ...)        fp32 partial sums
+// [0, 256)                   header (status word)
+// [256, 256 + 4*kMaxCounters) arrival counters, at the same place for every
+//                            shape, so one zero-initialised workspace serves
+//                            calls of any shape (each call leaves them zero)
+// [then ...)                 fp32 partial sums (scratch)
+constexpr size_t kMaxCounters = 65536;
 struct WorkspaceMap {
     size_t counters_off;
     size_t counters;      // number of int counters

@@ -66,7 +66,7 @@ __device__ __forceinline__ void store_tile_y(const Params &p, int nt, const floa
 }
 
 template <int TT>
-__device__ __forceinline__ void flush_segment(const Params &p, int gw, int lane, long long nt,
+__device__ __noinline__ void flush_segment(const Params &p, int gw, int lane, long long nt,
                                               long long seg_begin, long long seg_end,
                                               long long run_begin, float (&acc)[TT][4])
 {
@@ -82,17 +82,15 @@ __device__ __forceinline__ void flush_segment(const Params &p, int gw, int lane,
     for (int tt = 0; tt < TT; ++tt)
         __stcg(reinterpret_cast<float4 *>(dst + 4 * tt),
                make_float4(acc[tt][0], acc[tt][1], acc[tt][2], acc[tt][3]));
-    __threadfence();
     __syncwarp();
     int old = 0;
     if (lane == 0)
-        old = atomicAdd(&p.counters[nt], 1);
+        old = atomic_add_acq_rel(&p.counters[nt], 1);
     old = __shfl_sync(0xffffffffu, old, 0);
     const int w_first = warp_of_unit(tile_begin, p.units, p.Wt);
     const int w_last = warp_of_unit(tile_end - 1, p.units, p.Wt);
     if (old != w_last - w_first)
         return;
-    __threadfence();
     float sum[TT][4];
 #pragma unroll
     for (int tt = 0; tt < TT; ++tt)
@@ -116,23 +114,23 @@ __device__ __forceinline__ void flush_segment(const Params &p, int gw, int lane,
         p.counters[nt] = 0;
 }
 
+// The E8M0 scales of one unit for lane (g, t): rows g and g + 8, block t.
 struct UnitScales {
-    float a, b;  // rows g and g + 8
+    float a, b;
 };
 
-__device__ __forceinline__ UnitScales load_unit_scales(const Params &p, long long u, int g, int t)
+__device__ __forceinline__ UnitScales load_unit_scales(const Params &p, long long tile, int kb,
+                                                       int g, int t)
 {
-    const long long nt = u / p.upt;
-    const int kb = (int)(u - nt * p.upt);
     const int blocks = p.K / 32;
     const int blk = kb * 4 + t;
-    const int ra = (int)nt * 16 + g, rb = ra + 8;
+    const long long ra = tile * 16 + g, rb = ra + 8;
     uint32_t ea = 127, eb = 127;  // any finite scale for zero-filled weights
     if (blk < blocks) {
         if (ra < p.N)
-            ea = __ldg(p.Ws + (size_t)ra * blocks + blk);
+            ea = __ldg(p.Ws + ra * blocks + blk);
         if (rb < p.N)
-            eb = __ldg(p.Ws + (size_t)rb * blocks + blk);
+            eb = __ldg(p.Ws + rb * blocks + blk);
     }
     return UnitScales{e8m0_to_f32(ea), e8m0_to_f32(eb)};
 }
@@ -156,7 +154,12 @@ __global__ void __launch_bounds__(kWarps * 32)
     const long long u0 = run_start(gw, p.units, p.Wt);
     const long long u1 = run_start(gw + 1, p.units, p.Wt);
     const int nstages = (int)(u1 - u0);
+    long long tile = u0 / p.upt;
+    int kb = (int)(u0 - tile * p.upt);
 
+    // lane 0 owns the ring; (itile, ikb) is the next unit to fetch
+    long long itile = tile;
+    int ikb = kb;
     uint64_t policy = 0;
     if (lane == 0) {
         prefetch_tensormap(&wq_map);
@@ -165,20 +168,16 @@ __global__ void __launch_bounds__(kWarps * 32)
             mbar_init(&bars[s], 1);
         fence_barrier_init();
         policy = l2_policy_evict_first();
+        for (int s = 0; s < min(kRing, nstages); ++s) {
+            mbar_arrive_expect_tx(&bars[s], kStage);
+            tma_load_2d(ring + s * kStage, &wq_map, ikb * 128, (int)itile * 16, &bars[s], policy);
+            if (++ikb == p.upt) {
+                ikb = 0;
+                ++itile;
+            }
+        }
     }
     __syncwarp();
-
-    auto issue = [&](int s) {
-        const int slot = s % kRing;
-        const long long u = u0 + s;
-        const long long nt = u / p.upt;
-        const int kb = (int)(u - nt * p.upt);
-        mbar_arrive_expect_tx(&bars[slot], kStage);
-        tma_load_2d(ring + slot * kStage, &wq_map, kb * 128, (int)nt * 16, &bars[slot], policy);
-    };
-    if (lane == 0)
-        for (int s = 0; s < min(kRing, nstages); ++s)
-            issue(s);
 
     float acc[TT][4];
 #pragma unroll
@@ -187,7 +186,6 @@ __global__ void __launch_bounds__(kWarps * 32)
         for (int e = 0; e < 4; ++e)
             acc[tt][e] = 0.f;
 
-    long long cur_nt = u0 / p.upt;
     long long seg_begin = u0;
     const uint16_t *xrow[TT];
     bool xvalid[TT];
@@ -197,25 +195,22 @@ __global__ void __launch_bounds__(kWarps * 32)
         xvalid[tt] = m < p.M;
         xrow[tt] = p.X + (size_t)(xvalid[tt] ? m : 0) * p.K;
     }
-    UnitScales sc_next = load_unit_scales(p, u0, g, t);
+    UnitScales sc_next = load_unit_scales(p, tile, kb, g, t);
     const int c_lo = ((2 * t) ^ g) * 16, c_hi = ((2 * t + 1) ^ g) * 16;
 
     for (int s = 0; s < nstages; ++s) {
         const long long u = u0 + s;
-        const long long nt = u / p.upt;
-        const int kb = (int)(u - nt * p.upt);
         const UnitScales sc = sc_next;
-        if (s + 1 < nstages)
-            sc_next = load_unit_scales(p, u + 1, g, t);
-        if (nt != cur_nt) {
-            flush_segment<TT>(p, gw, lane, cur_nt, seg_begin, u, u0, acc);
-#pragma unroll
-            for (int tt = 0; tt < TT; ++tt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    acc[tt][e] = 0.f;
-            cur_nt = nt;
-            seg_begin = u;
+        {
+            // scales of the next unit, one unit ahead
+            long long nt2 = tile;
+            int kb2 = kb + 1;
+            if (kb2 == p.upt) {
+                kb2 = 0;
+                ++nt2;
+            }
+            if (s + 1 < nstages)
+                sc_next = load_unit_scales(p, nt2, kb2, g, t);
         }
         const int kl = kb * 128 + t * 32;
         const bool kvalid = kl < p.K;
@@ -260,10 +255,28 @@ __global__ void __launch_bounds__(kWarps * 32)
         __syncwarp();
         if (lane == 0 && s + kRing < nstages) {
             fence_proxy_async_smem();  // our reads of this slot precede the next copy into it
-            issue(s + kRing);
+            mbar_arrive_expect_tx(&bars[slot], kStage);
+            tma_load_2d(ring + slot * kStage, &wq_map, ikb * 128, (int)itile * 16, &bars[slot],
+                        policy);
+            if (++ikb == p.upt) {
+                ikb = 0;
+                ++itile;
+            }
+        }
+        if (++kb == p.upt) {
+            flush_segment<TT>(p, gw, lane, tile, seg_begin, u + 1, u0, acc);
+#pragma unroll
+            for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    acc[tt][e] = 0.f;
+            ++tile;
+            kb = 0;
+            seg_begin = u + 1;
         }
     }
-    flush_segment<TT>(p, gw, lane, cur_nt, seg_begin, u1, u0, acc);
+    if (seg_begin < u1)
+        flush_segment<TT>(p, gw, lane, tile, seg_begin, u1, u0, acc);
 }
 
 const void *select_kernel(int tt)
@@ -293,6 +306,8 @@ bool plan_mxfp8_stream(int device, int M, int N, int K, StreamPlan *plan)
     pl.smem = kSmemBytes;
     pl.upt = (K + 127) / 128;
     pl.ntiles = (N + 15) / 16;
+    if ((size_t)pl.ntiles > kMaxCounters)
+        return false;
     pl.units = (long long)pl.ntiles * pl.upt;
     const void *fn = select_kernel(pl.tt);
     static int occ_cache[4] = {};

@@ -2,24 +2,27 @@
 //
 // At M <= 32 the layer reads each weight byte once and does 2*M flops per
 // weight: it is bound by HBM bytes of W.  The kernel therefore
-//  * cuts the re-packed weight stream into equal units (one n16 tile x one
-//    scale group) and gives every warp of a persistent grid one contiguous
-//    run of units (stream-K), so all SMs stream the same number of bytes;
-//  * moves each warp's run through its own ring of shared-memory stages with
-//    1-D bulk copies (cp.async.bulk, completion on an mbarrier), several
-//    stages in flight per warp, weights marked evict-first in L2;
-//  * decodes nibbles to exact bf16 (q - 8) in registers (mask/or + one
-//    bf16x2 fma per two weights) and multiplies on the tensor cores with
-//    m16n8k16 MMAs where the weights are the 16-row operand and the tokens
-//    the 8-column operand ("swap AB"), so M = 1..8 costs one MMA per 256
-//    weights;
-//  * applies the fp16 group scale once per group to the fp32 partial sum
-//    (G = 64, 128), or folds it into the bf16 weight with one rounding
-//    (G = 32, whose groups are narrower than one MMA's k span);
-//  * reduces the partial sums of n16 tiles shared by several warps through
-//    the workspace: each contributor stores its fragment, bumps the tile's
-//    arrival counter, and the last one adds all fragments in warp order
-//    (deterministic) and writes bf16 Y.  Nobody waits on anybody.
+//  * cuts the re-packed weight stream into equal units (one n32 tile x one
+//    scale-group span of max(G, 64) rows of K) and gives every warp of a
+//    persistent grid one contiguous run of units (stream-K), so all SMs
+//    stream the same number of bytes; a run is one contiguous byte range of
+//    the re-packed buffer, and never shorter than a few stages;
+//  * moves each warp's run through its own ring of shared-memory stages
+//    with 1-D bulk copies (cp.async.bulk, completion on an mbarrier), four
+//    2 KB stages in flight per warp, weights marked evict-first in L2;
+//  * decodes nibbles to exact bf16 (q - 8) in registers (shift + lop3 and
+//    one bf16x2 add per two weights) and multiplies on the tensor cores
+//    with m16n8k16 MMAs where the weights are the 16-row operand and the
+//    tokens the 8-column operand ("swap AB"); the two n16 halves of a unit
+//    share each activation fragment;
+//  * starts a zero-initialised partial sum per scale group (every MMA step
+//    lies inside one group for G = 32, 64, 128) and adds partial * scale
+//    in fp32 once per group, so weights are never rounded;
+//  * n32 tiles covered whole by one warp are written directly; a tile cut
+//    between warps is reduced through the workspace: at the end of its run
+//    each contributor stores its fragment and bumps the tile's arrival
+//    counter (acquire-release), and the last one adds all fragments in warp
+//    order (deterministic) and writes bf16 Y.  Nobody waits on anybody.
 #include <algorithm>
 
 #include "common.cuh"
@@ -28,33 +31,43 @@
 namespace mxg {
 namespace {
 
-constexpr int kWarps = 8;        // warps per CTA
-constexpr int kRing = 4;         // stages per warp
-constexpr int kStageCode = 2048; // code bytes per stage
-constexpr int kStageScale = 256; // scale bytes reserved per stage
+constexpr int kWarps = 8;         // warps per CTA
+#ifndef MXG_STREAM_RING
+#define MXG_STREAM_RING 4
+#endif
+#ifndef MXG_STREAM_MIN_STAGES
+#define MXG_STREAM_MIN_STAGES 6
+#endif
+constexpr int kRing = MXG_STREAM_RING;          // stages per warp
+constexpr int kMinStages = MXG_STREAM_MIN_STAGES;  // shortest run, in stages
+constexpr int kStageCode = 2048;  // code bytes per stage (two k64 chunks of an n32 tile)
+constexpr int kStageScale = 256;  // scale bytes reserved per stage
 constexpr int kStageBytes = kStageCode + kStageScale;
-constexpr int kWarpSmem = kRing * kStageBytes + kRing * 8;
+// per-warp ring: stages, then one mbarrier per stage; rounded so every
+// warp's ring (and every stage) starts 128-byte aligned
+constexpr int kWarpSmem = (kRing * kStageBytes + kRing * 8 + 127) / 128 * 128;
+static_assert(kStageBytes % 128 == 0, "stages must stay 128-byte aligned");
 
-// Group modes: 0 -> G = 128 (unit = 2 chunks, 1 scale row), 1 -> G = 64
-// (unit = 1 chunk, 1 scale row), 2 -> G = 32 (unit = 1 chunk, 2 scale rows).
+// Group modes: 0 -> G = 128, 1 -> G = 64, 2 -> G = 32.
 template <int GM>
 struct Mode {
-    static constexpr int kChunks = (GM == 0) ? 2 : 1;       // k64 chunks per unit
-    static constexpr int kScaleRows = (GM == 2) ? 2 : 1;    // 32-byte scale rows per unit
-    static constexpr int kUnitsPerStage = kStageCode / (kChunks * 512);
-    static constexpr bool kPostScale = (GM != 2);
+    static constexpr int kG = GM == 0 ? 128 : (GM == 1 ? 64 : 32);
+    static constexpr int kChunks = GM == 0 ? 2 : 1;          // k64 chunks per unit
+    static constexpr int kGroups = GM == 2 ? 2 : 1;          // scale groups per unit
+    static constexpr int kUnitsPerStage = 2 / kChunks;
+    static constexpr int kStepsPerGroup = kG / 16;            // MMA k16 steps per group
 };
 
 struct Params {
     const uint16_t *X;       // bf16 [M][K]
-    const uint8_t *codes;    // re-packed codes
-    const uint8_t *scales;   // re-packed scales
+    const uint8_t *codes;    // re-packed codes  [N/32][K/64][2][32][16 B]
+    const uint8_t *scales;   // re-packed scales [N/32][K/G][8][4 halves]
     uint16_t *Y;             // bf16 [M][N]
     WsHeader *hdr;
-    int *counters;           // [N/16]
-    float *partial;          // [Wt][2][32][4*TT]
+    int *counters;           // [N/32]
+    float *partial;          // [Wt][2][32][2*4*TT]
     int M, N, K;
-    int upt;                 // units per n16 tile
+    int upt;                 // units per n32 tile
     long long units;
     int Wt;
 };
@@ -71,75 +84,86 @@ __device__ __forceinline__ int warp_of_unit(long long u, long long units, int Wt
 }
 
 template <int TT>
-__device__ __forceinline__ void store_tile_y(const Params &p, int nt, const float (&v)[TT][4], int g,
-                                             int t)
+__device__ __forceinline__ void store_tile_y(const Params &p, long long tile,
+                                             const float (&v)[2][TT][4], int g, int t)
 {
 #pragma unroll
-    for (int tt = 0; tt < TT; ++tt)
+    for (int h = 0; h < 2; ++h)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int m = tt * 8 + 2 * t + (e & 1);
-            const int n = nt * 16 + g + ((e & 2) ? 8 : 0);
-            if (m < p.M)
-                p.Y[(size_t)m * p.N + n] = f32_to_bf16_bits(v[tt][e]);
-        }
+        for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int m = tt * 8 + 2 * t + (e & 1);
+                const long long n = tile * 32 + h * 16 + g + ((e & 2) ? 8 : 0);
+                if (m < p.M)
+                    p.Y[(size_t)m * p.N + n] = f32_to_bf16_bits(v[h][tt][e]);
+            }
 }
 
-// Finish the segment [seg_begin, seg_end) of n16 tile nt held in acc.
 template <int TT>
-__device__ __forceinline__ void flush_segment(const Params &p, int gw, int lane, long long nt,
-                                              long long seg_begin, long long seg_end,
-                                              long long run_begin, float (&acc)[TT][4])
+__device__ __forceinline__ void store_partial(const Params &p, int gw, int slot, int lane,
+                                              const float (&v)[2][TT][4])
+{
+    float *dst = p.partial + ((size_t)(gw * 2 + slot) * 32 + lane) * (8 * TT);
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int tt = 0; tt < TT; ++tt)
+            __stcg(reinterpret_cast<float4 *>(dst + (h * TT + tt) * 4),
+                   make_float4(v[h][tt][0], v[h][tt][1], v[h][tt][2], v[h][tt][3]));
+}
+
+// Run by the last contributor of a cut tile: add every fragment of the tile
+// in warp order and write bf16 Y.
+template <int TT>
+__device__ __noinline__ void reduce_tile(const Params &p, long long tile, int lane)
 {
     const int g = lane >> 2, t = lane & 3;
-    const long long tile_begin = nt * p.upt, tile_end = tile_begin + p.upt;
-    if (seg_begin == tile_begin && seg_end == tile_end) {
-        store_tile_y<TT>(p, (int)nt, acc, g, t);
-        return;
-    }
-    const int slot = (seg_begin == run_begin) ? 0 : 1;
-    float *dst = p.partial + ((size_t)(gw * 2 + slot) * 32 + lane) * (4 * TT);
-#pragma unroll
-    for (int tt = 0; tt < TT; ++tt)
-        __stcg(reinterpret_cast<float4 *>(dst + 4 * tt),
-               make_float4(acc[tt][0], acc[tt][1], acc[tt][2], acc[tt][3]));
-    __threadfence();
-    __syncwarp();
-    int old = 0;
-    if (lane == 0)
-        old = atomicAdd(&p.counters[nt], 1);
-    old = __shfl_sync(0xffffffffu, old, 0);
+    const long long tile_begin = tile * p.upt, tile_end = tile_begin + p.upt;
     const int w_first = warp_of_unit(tile_begin, p.units, p.Wt);
     const int w_last = warp_of_unit(tile_end - 1, p.units, p.Wt);
-    if (old != w_last - w_first)
-        return;
-    // last contributor: add every fragment of this tile in warp order
-    __threadfence();
-    float sum[TT][4];
+    float sum[2][TT][4];
 #pragma unroll
-    for (int tt = 0; tt < TT; ++tt)
+    for (int h = 0; h < 2; ++h)
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-            sum[tt][e] = 0.f;
+        for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                sum[h][tt][e] = 0.f;
+#pragma unroll 4
     for (int w = w_first; w <= w_last; ++w) {
         const int s = (run_start(w, p.units, p.Wt) >= tile_begin) ? 0 : 1;
-        const float *src = p.partial + ((size_t)(w * 2 + s) * 32 + lane) * (4 * TT);
+        const float *src = p.partial + ((size_t)(w * 2 + s) * 32 + lane) * (8 * TT);
 #pragma unroll
-        for (int tt = 0; tt < TT; ++tt) {
-            const float4 f = ldcg_f4(src + 4 * tt);
-            sum[tt][0] += f.x;
-            sum[tt][1] += f.y;
-            sum[tt][2] += f.z;
-            sum[tt][3] += f.w;
-        }
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int tt = 0; tt < TT; ++tt) {
+                const float4 f = ldcg_f4(src + (h * TT + tt) * 4);
+                sum[h][tt][0] += f.x;
+                sum[h][tt][1] += f.y;
+                sum[h][tt][2] += f.z;
+                sum[h][tt][3] += f.w;
+            }
     }
-    store_tile_y<TT>(p, (int)nt, sum, g, t);
+    store_tile_y<TT>(p, tile, sum, g, t);
     if (lane == 0)
-        p.counters[nt] = 0;  // leave the workspace zeroed for the next call
+        p.counters[tile] = 0;  // leave the counter zero for the next call
+}
+
+template <int TT>
+__device__ __forceinline__ void zero_acc(float (&a)[2][TT][4])
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                a[h][tt][e] = 0.f;
 }
 
 template <int TT, int GM>
-__global__ void __launch_bounds__(kWarps * 32) w4a16_stream_kernel(const Params p)
+__global__ void __launch_bounds__(kWarps * 32, TT == 1 ? 3 : 2) w4a16_stream_kernel(const Params p)
 {
     using MD = Mode<GM>;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -156,6 +180,10 @@ __global__ void __launch_bounds__(kWarps * 32) w4a16_stream_kernel(const Params 
     const long long u1 = run_start(gw + 1, p.units, p.Wt);
     const int nstages = (int)((u1 - u0 + MD::kUnitsPerStage - 1) / MD::kUnitsPerStage);
 
+    // lane 0 owns the ring: source pointers advance by one stage per issue
+    const uint8_t *csrc = p.codes + u0 * (MD::kChunks * 1024);
+    const uint8_t *ssrc = p.scales + u0 * (MD::kGroups * 64);
+    long long left = u1 - u0;  // units not yet requested
     uint64_t policy = 0;
     if (lane == 0) {
 #pragma unroll
@@ -163,141 +191,189 @@ __global__ void __launch_bounds__(kWarps * 32) w4a16_stream_kernel(const Params 
             mbar_init(&bars[s], 1);
         fence_barrier_init();
         policy = l2_policy_evict_first();
+        for (int s = 0; s < min(kRing, nstages); ++s) {
+            const int nu = (int)min((long long)MD::kUnitsPerStage, left);
+            const uint32_t cb = nu * MD::kChunks * 1024, sb = nu * MD::kGroups * 64;
+            uint8_t *dst = ring + s * kStageBytes;
+            mbar_arrive_expect_tx(&bars[s], cb + sb);
+            bulk_g2s(dst, csrc, cb, &bars[s], policy);
+            bulk_g2s(dst + kStageCode, ssrc, sb, &bars[s], policy);
+            csrc += cb;
+            ssrc += sb;
+            left -= nu;
+        }
     }
     __syncwarp();
 
-    auto issue = [&](int s) {
-        const int slot = s % kRing;
-        const long long ub = u0 + (long long)s * MD::kUnitsPerStage;
-        const int nu = (int)min((long long)MD::kUnitsPerStage, u1 - ub);
-        const uint32_t cbytes = nu * MD::kChunks * 512;
-        const uint32_t sbytes = nu * MD::kScaleRows * 32;
-        uint8_t *dst = ring + slot * kStageBytes;
-        mbar_arrive_expect_tx(&bars[slot], cbytes + sbytes);
-        bulk_g2s(dst, p.codes + ub * (MD::kChunks * 512), cbytes, &bars[slot], policy);
-        bulk_g2s(dst + kStageCode, p.scales + ub * (MD::kScaleRows * 32), sbytes, &bars[slot],
-                 policy);
-    };
-
-    if (lane == 0)
-        for (int s = 0; s < min(kRing, nstages); ++s)
-            issue(s);
-
-    float acc[TT][4];
-    float part[TT][4];
-#pragma unroll
-    for (int tt = 0; tt < TT; ++tt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-            acc[tt][e] = part[tt][e] = 0.f;
-
-    long long cur_nt = u0 / p.upt;
-    long long seg_begin = u0;
+    // activation rows of this lane: m = g + 8 tt; the lane reads k = 4t .. 4t+3
+    // of every k16 step
     const uint16_t *xrow[TT];
     bool xvalid[TT];
 #pragma unroll
     for (int tt = 0; tt < TT; ++tt) {
         const int m = tt * 8 + g;
         xvalid[tt] = m < p.M;
-        xrow[tt] = p.X + (size_t)(xvalid[tt] ? m : 0) * p.K;
+        xrow[tt] = p.X + (size_t)(xvalid[tt] ? m : 0) * p.K + 4 * t;
     }
+
+    float acc[2][TT][4], part[2][TT][4];
+    zero_acc<TT>(acc);
+    bool first_cut = false;  // the run's first segment ended inside the run, cut
+    long long first_tile = 0;
+
+    long long tile = u0 / p.upt;
+    int lu = (int)(u0 - tile * p.upt);     // unit inside the tile
+    const int kchunks = p.K / 64;
+    int kc = lu * MD::kChunks;             // chunk inside the tile
+    long long seg_begin = u0;
 
     for (int s = 0; s < nstages; ++s) {
         const int slot = s % kRing;
+        const uint8_t *stage = ring + slot * kStageBytes;
+        // activations of the stage's two chunks, requested before the wait
+        // (they do not depend on the copy); wide token tiles load per chunk
+        constexpr int kXStage = TT <= 2 ? 2 : 1;
+        uint2 xs[kXStage][TT][4];
+        const int kc1 = (kc + 1 == kchunks) ? 0 : kc + 1;
+        auto load_x = [&](int slot_x, int chunk) {
+#pragma unroll
+            for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint2 v = make_uint2(0, 0);
+                    if (xvalid[tt])
+                        v = __ldg(reinterpret_cast<const uint2 *>(xrow[tt] + chunk * 64 + 16 * j));
+                    xs[slot_x][tt][j] = v;
+                }
+        };
+        load_x(0, kc);
+        if (kXStage == 2)
+            load_x(kXStage - 1, kc1);
         if (!mbar_wait(&bars[slot], (s / kRing) & 1, kWaitLimitNs)) {
             if (lane == 0)
                 record_error(p.hdr, MXG_ERR_TIMEOUT, 100 + GM);
-            // give the copies still in flight a bounded chance to land
             for (int r = s + 1; r < min(s + kRing, nstages); ++r)
                 mbar_wait(&bars[r % kRing], (r / kRing) & 1, kWaitLimitNs / 16);
             return;
         }
-        const uint8_t *stage = ring + slot * kStageBytes;
-        const long long ub = u0 + (long long)s * MD::kUnitsPerStage;
 #pragma unroll
         for (int iu = 0; iu < MD::kUnitsPerStage; ++iu) {
-            const long long u = ub + iu;
-            if (u >= u1)
+            const long long u = u0 + (long long)s * MD::kUnitsPerStage + iu;
+            if (iu > 0 && u >= u1)
                 break;
-            const long long nt = u / p.upt;
-            if (nt != cur_nt) {
-                flush_segment<TT>(p, gw, lane, cur_nt, seg_begin, u, u0, acc);
-#pragma unroll
-                for (int tt = 0; tt < TT; ++tt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        acc[tt][e] = 0.f;
-                cur_nt = nt;
-                seg_begin = u;
-            }
-            const int lu = (int)(u - nt * p.upt);
-            const uint8_t *sc = stage + kStageCode + iu * (MD::kScaleRows * 32);
 #pragma unroll
             for (int ch = 0; ch < MD::kChunks; ++ch) {
-                const int kc = lu * MD::kChunks + ch;          // chunk inside the tile
-                const int kl = kc * 64 + t * 16;               // lane's first k
-                uint32_t xb[TT][8];
+                const int c2 = iu * MD::kChunks + ch;  // chunk inside the stage
+                const int xi = kXStage == 2 ? c2 : 0;
+                if (kXStage == 1 && c2 == 1)
+                    load_x(0, kc1);
+                const uint8_t *cp = stage + c2 * 1024 + lane * 16;
+                const uint4 wl = lds128(cp);
+                const uint4 wh = lds128(cp + 512);
+                const uint32_t w[2][4] = {{wl.x, wl.y, wl.z, wl.w}, {wh.x, wh.y, wh.z, wh.w}};
 #pragma unroll
-                for (int tt = 0; tt < TT; ++tt) {
-                    uint4 x0 = make_uint4(0, 0, 0, 0), x1 = x0;
-                    if (xvalid[tt]) {
-                        x0 = ldg128(xrow[tt] + kl);
-                        x1 = ldg128(xrow[tt] + kl + 8);
+                for (int j = 0; j < 4; ++j) {
+                    const int step = ch * 4 + j;  // k16 step inside the unit
+                    const bool first = (step % MD::kStepsPerGroup) == 0;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t a0 = int4_pair_minus8<0>(w[h][j]);
+                        const uint32_t a1 = int4_pair_minus8<4>(w[h][j]);
+                        const uint32_t a2 = int4_pair_minus8<8>(w[h][j]);
+                        const uint32_t a3 = int4_pair_minus8<12>(w[h][j]);
+#pragma unroll
+                        for (int tt = 0; tt < TT; ++tt) {
+                            if (first)
+                                mma_bf16_16816_zero(part[h][tt], a0, a1, a2, a3,
+                                                    xs[xi][tt][j].x, xs[xi][tt][j].y);
+                            else
+                                mma_bf16_16816(part[h][tt], a0, a1, a2, a3, xs[xi][tt][j].x,
+                                               xs[xi][tt][j].y);
+                        }
                     }
-                    xb[tt][0] = x0.x; xb[tt][1] = x0.y; xb[tt][2] = x0.z; xb[tt][3] = x0.w;
-                    xb[tt][4] = x1.x; xb[tt][5] = x1.y; xb[tt][6] = x1.z; xb[tt][7] = x1.w;
+                    if ((step + 1) % MD::kStepsPerGroup == 0) {
+                        // end of a scale group: acc += part * scale (fp32)
+                        const int gi = step / MD::kStepsPerGroup;  // group inside the unit
+                        const uint2 sv =
+                            lds64(stage + kStageCode + (iu * MD::kGroups + gi) * 64 + g * 8);
+                        const float2 s01 = __half22float2(*reinterpret_cast<const __half2 *>(&sv.x));
+                        const float2 s23 = __half22float2(*reinterpret_cast<const __half2 *>(&sv.y));
+#pragma unroll
+                        for (int tt = 0; tt < TT; ++tt) {
+                            acc[0][tt][0] = fmaf(part[0][tt][0], s01.x, acc[0][tt][0]);
+                            acc[0][tt][1] = fmaf(part[0][tt][1], s01.x, acc[0][tt][1]);
+                            acc[0][tt][2] = fmaf(part[0][tt][2], s01.y, acc[0][tt][2]);
+                            acc[0][tt][3] = fmaf(part[0][tt][3], s01.y, acc[0][tt][3]);
+                            acc[1][tt][0] = fmaf(part[1][tt][0], s23.x, acc[1][tt][0]);
+                            acc[1][tt][1] = fmaf(part[1][tt][1], s23.x, acc[1][tt][1]);
+                            acc[1][tt][2] = fmaf(part[1][tt][2], s23.y, acc[1][tt][2]);
+                            acc[1][tt][3] = fmaf(part[1][tt][3], s23.y, acc[1][tt][3]);
+                        }
+                    }
                 }
-                const uint4 wv = lds128(stage + (iu * MD::kChunks + ch) * 512 + lane * 16);
-                const uint32_t wj[4] = {wv.x, wv.y, wv.z, wv.w};
-                if constexpr (MD::kPostScale) {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const uint32_t a0 = int4_pair_minus8<0>(wj[j]);
-                        const uint32_t a1 = int4_pair_minus8<4>(wj[j]);
-                        const uint32_t a2 = int4_pair_minus8<8>(wj[j]);
-                        const uint32_t a3 = int4_pair_minus8<12>(wj[j]);
-#pragma unroll
-                        for (int tt = 0; tt < TT; ++tt)
-                            mma_bf16_16816(part[tt], a0, a1, a2, a3, xb[tt][2 * j], xb[tt][2 * j + 1]);
-                    }
-                } else {
-                    // G = 32: this lane's 16 rows are in scale row t / 2 of the unit
-                    const uint32_t sw = lds32(sc + (t >> 1) * 32 + g * 4);
-                    const ScaleSplit sa = split_scale((uint16_t)(sw & 0xFFFF));
-                    const ScaleSplit sb = split_scale((uint16_t)(sw >> 16));
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const uint32_t a0 = scale_pair_rn(int4_pair_minus8<0>(wj[j]), sa);
-                        const uint32_t a1 = scale_pair_rn(int4_pair_minus8<4>(wj[j]), sb);
-                        const uint32_t a2 = scale_pair_rn(int4_pair_minus8<8>(wj[j]), sa);
-                        const uint32_t a3 = scale_pair_rn(int4_pair_minus8<12>(wj[j]), sb);
-#pragma unroll
-                        for (int tt = 0; tt < TT; ++tt)
-                            mma_bf16_16816(acc[tt], a0, a1, a2, a3, xb[tt][2 * j], xb[tt][2 * j + 1]);
-                    }
-                }
+                kc = (kc + 1 == kchunks) ? 0 : kc + 1;
             }
-            if constexpr (MD::kPostScale) {
-                const uint32_t sw = lds32(sc + g * 4);
-                const float sa = __half2float(__ushort_as_half((uint16_t)(sw & 0xFFFF)));
-                const float sb = __half2float(__ushort_as_half((uint16_t)(sw >> 16)));
-#pragma unroll
-                for (int tt = 0; tt < TT; ++tt) {
-                    acc[tt][0] = fmaf(part[tt][0], sa, acc[tt][0]);
-                    acc[tt][1] = fmaf(part[tt][1], sa, acc[tt][1]);
-                    acc[tt][2] = fmaf(part[tt][2], sb, acc[tt][2]);
-                    acc[tt][3] = fmaf(part[tt][3], sb, acc[tt][3]);
-                    part[tt][0] = part[tt][1] = part[tt][2] = part[tt][3] = 0.f;
+            if (++lu == p.upt) {
+                // a tile ends inside the run
+                if (seg_begin == tile * p.upt) {
+                    store_tile_y<TT>(p, tile, acc, g, t);   // whole tile: write it now
+                } else {
+                    // the run's first segment, cut: park it in slot 0 now, announce it
+                    // at the end of the run
+                    store_partial<TT>(p, gw, 0, lane, acc);
+                    first_cut = true;
+                    first_tile = tile;
                 }
+                zero_acc<TT>(acc);
+                ++tile;
+                lu = 0;
+                seg_begin = u + 1;
             }
         }
         __syncwarp();
-        if (lane == 0 && s + kRing < nstages) {
+        if (lane == 0 && left > 0) {
             fence_proxy_async_smem();  // our reads of this slot precede the next copy into it
-            issue(s + kRing);
+            const int nu = (int)min((long long)MD::kUnitsPerStage, left);
+            const uint32_t cb = nu * MD::kChunks * 1024, sb = nu * MD::kGroups * 64;
+            uint8_t *dst = ring + slot * kStageBytes;
+            mbar_arrive_expect_tx(&bars[slot], cb + sb);
+            bulk_g2s(dst, csrc, cb, &bars[slot], policy);
+            bulk_g2s(dst + kStageCode, ssrc, sb, &bars[slot], policy);
+            csrc += cb;
+            ssrc += sb;
+            left -= nu;
         }
     }
-    flush_segment<TT>(p, gw, lane, cur_nt, seg_begin, u1, u0, acc);
+
+    // publish the cut segments: the first one (slot 0) and the last one
+    // (slot 0 if it is also the first segment of the run, else slot 1)
+    const bool last_cut = seg_begin < u1;
+    if (last_cut)
+        store_partial<TT>(p, gw, seg_begin == u0 ? 0 : 1, lane, acc);
+    if (!first_cut && !last_cut)
+        return;
+    __syncwarp();
+    int arrivals[2] = {0, 0};
+    if (lane == 0) {
+        if (first_cut)
+            arrivals[0] = atomic_add_acq_rel(&p.counters[first_tile], 1);
+        if (last_cut)
+            arrivals[1] = atomic_add_acq_rel(&p.counters[tile], 1);
+    }
+    arrivals[0] = __shfl_sync(0xffffffffu, arrivals[0], 0);
+    arrivals[1] = __shfl_sync(0xffffffffu, arrivals[1], 0);
+    if (first_cut) {
+        const int wf = warp_of_unit(first_tile * p.upt, p.units, p.Wt);
+        const int wl = warp_of_unit(first_tile * p.upt + p.upt - 1, p.units, p.Wt);
+        if (arrivals[0] == wl - wf)
+            reduce_tile<TT>(p, first_tile, lane);
+    }
+    if (last_cut) {
+        const int wf = warp_of_unit(tile * p.upt, p.units, p.Wt);
+        const int wl = warp_of_unit(tile * p.upt + p.upt - 1, p.units, p.Wt);
+        if (arrivals[1] == wl - wf)
+            reduce_tile<TT>(p, tile, lane);
+    }
 }
 
 template <int TT, int GM>
@@ -327,7 +403,7 @@ int group_mode(int G)
 
 bool plan_w4a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan)
 {
-    if (M < 1 || M > 32)
+    if (M < 1 || M > 32 || N % 32 != 0)
         return false;
     const DeviceInfo &di = device_info(device);
     StreamPlan pl{};
@@ -337,7 +413,9 @@ bool plan_w4a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan)
     pl.smem = (size_t)kWarps * kWarpSmem;
     const int unit_k = std::max(G, 64);
     pl.upt = K / unit_k;
-    pl.ntiles = N / 16;
+    pl.ntiles = N / 32;
+    if ((size_t)pl.ntiles > kMaxCounters)
+        return false;
     pl.units = (long long)pl.ntiles * pl.upt;
     const void *fn = select_kernel(pl.tt, pl.variant);
     if (!fn)
@@ -355,10 +433,13 @@ bool plan_w4a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan)
             return false;
         occ = o;
     }
+    // enough warps to fill the GPU, but no run shorter than kMinStages stages
+    const int units_per_stage = 2 / (unit_k / 64);
+    const long long min_units = (long long)kMinStages * units_per_stage;
     const long long max_warps = (long long)di.sms * occ * kWarps;
-    pl.Wt = (int)std::min<long long>(max_warps, pl.units);
+    pl.Wt = (int)std::max<long long>(1, std::min<long long>(max_warps, pl.units / min_units));
     pl.grid = (pl.Wt + kWarps - 1) / kWarps;
-    pl.partial_bytes = (size_t)pl.Wt * 2 * 32 * 4 * pl.tt * sizeof(float);
+    pl.partial_bytes = (size_t)pl.Wt * 2 * 32 * 2 * 4 * pl.tt * sizeof(float);
     *plan = pl;
     return true;
 }
@@ -366,6 +447,7 @@ bool plan_w4a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan)
 cudaError_t launch_w4a16_stream(const StreamPlan &pl, const void *X, const void *packed, int M,
                                 int N, int K, int G, void *Y, void *workspace, cudaStream_t stream)
 {
+    (void)G;
     const void *fn = select_kernel(pl.tt, pl.variant);
     if (!fn)
         return cudaErrorInvalidValue;

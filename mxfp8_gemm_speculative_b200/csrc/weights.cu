@@ -1,47 +1,56 @@
 // Offline weight re-pack for INT4 W4A16 and the decode kernels the tests use.
 //
 // Re-packed INT4 layout (one buffer, codes then scales):
-//   codes  [N/16][K/64][32 lanes][4 words]
-//   scales [N/16][K/G][16 halves]
-// For n16 tile `nt`, k64 chunk `c` and lane = 4*g + t (g = 0..7, t = 0..3),
-// the lane's 16 bytes hold columns n = 16nt + g and n + 8 for the sixteen
-// rows k = 64c + 16t .. 64c + 16t + 15.  Word j covers k0 = 64c + 16t + 4j:
-//   bits [ 0, 4) q(n,   k0)    [16,20) q(n,   k0+1)
-//   bits [ 4, 8) q(n+8, k0)    [20,24) q(n+8, k0+1)
-//   bits [ 8,12) q(n,   k0+2)  [24,28) q(n,   k0+3)
-//   bits [12,16) q(n+8, k0+2)  [28,32) q(n+8, k0+3)
-// so that masking (w >> 4r) & 0x000F000F yields a pair of codes that lands in
-// the two halves of one bf16x2 register: r = 0..3 give exactly the four A
-// registers of an m16n8k16 MMA step whose 16 k positions are the
-// k0 .. k0+3 of the four lanes t (the k order inside a step is permuted
-// consistently with the activations, which the sum does not see), and they
-// also give four consecutive k of one column for the tensor-core path.
-// Scales: the 16 halves of (nt, group) are ordered s[n0], s[n0+8], s[n0+1],
-// s[n0+9], ... so that lane g reads its two columns as one 32-bit word.
+//   codes  [N/32][K/64][2 halves][32 lanes][4 words]
+//   scales [N/32][K/G][8][4 halves]
+// For n32 tile T, k64 chunk c, half h and lane = 4*g + t (g = 0..7,
+// t = 0..3), the lane's 16 bytes hold columns na = 32T + 16h + g and
+// nb = na + 8.  Word j covers the four rows k0 = 64c + 16j + 4t .. k0 + 3:
+//   bits [ 0, 4) q(na, k0)    [16,20) q(na, k0+1)
+//   bits [ 4, 8) q(nb, k0)    [20,24) q(nb, k0+1)
+//   bits [ 8,12) q(na, k0+2)  [24,28) q(na, k0+3)
+//   bits [12,16) q(nb, k0+2)  [28,32) q(nb, k0+3)
+// so that (w >> 4r) & 0x000F000F puts a pair of codes in the two halves of
+// one bf16x2 register.  For the weight-streaming path, word j of the 32
+// lanes is exactly the A operand of one m16n8k16 MMA step over
+// k = 64c + 16j .. 64c + 16j + 15 (rows na, nb; lane t holds k positions
+// 4t .. 4t+3 of the step, and the activations are loaded in the same
+// order), so every step lies inside one group of 32.  For the tensor-core
+// path the same 16 bytes, decoded in register order (pair 0, pair 2) for
+// column na and (pair 1, pair 3) for nb, are exactly one thread's share of
+// a 16-lane x 256-bit tensor-memory store per word (lanes na, nb; columns
+// 2t, 2t+1 of the k16 block j).  Scales: entry (T, group, g) is the four
+// halves s[32T+g], s[32T+g+8], s[32T+16+g], s[32T+16+g+8].
 #include "common.cuh"
 #include "kernels.h"
 
 namespace mxg {
 namespace {
 
+__device__ __forceinline__ int chunk_k0(int c, int t, int j)
+{
+    return c * 64 + 16 * j + 4 * t;
+}
+
 __global__ void repack_codes_kernel(const int32_t *__restrict__ qweight, int K, int N,
                                     uint4 *__restrict__ out)
 {
-    const long long total = (long long)(N / 16) * (K / 64) * 32;
+    const long long total = (long long)(N / 32) * (K / 64) * 64;
     const long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x;
     if (idx >= total)
         return;
     const int lane = (int)(idx & 31);
-    const long long rest = idx >> 5;
+    const int h = (int)((idx >> 5) & 1);
+    const long long rest = idx >> 6;
     const int kc_count = K / 64;
     const int c = (int)(rest % kc_count);
-    const int nt = (int)(rest / kc_count);
+    const int T = (int)(rest / kc_count);
     const int g = lane >> 2, t = lane & 3;
-    const int na = nt * 16 + g, nb = na + 8;
+    const int na = T * 32 + h * 16 + g, nb = na + 8;
     uint32_t words[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        const int k0 = c * 64 + t * 16 + j * 4;
+        const int k0 = chunk_k0(c, t, j);
         const int shift = 4 * (k0 & 7);
         const uint32_t qa = ((uint32_t)qweight[(size_t)(k0 >> 3) * N + na]) >> shift;
         const uint32_t qb = ((uint32_t)qweight[(size_t)(k0 >> 3) * N + nb]) >> shift;
@@ -63,99 +72,78 @@ __global__ void repack_scales_kernel(const uint16_t *__restrict__ scales, int K,
                                      uint16_t *__restrict__ out)
 {
     const int groups = K / G;
-    const long long total = (long long)(N / 16) * groups * 16;
+    const long long total = (long long)(N / 32) * groups * 32;
     const long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x;
     if (idx >= total)
         return;
-    const int i = (int)(idx & 15);
-    const long long rest = idx >> 4;
+    const int i4 = (int)(idx & 3);
+    const int g = (int)((idx >> 2) & 7);
+    const long long rest = idx >> 5;
     const int grp = (int)(rest % groups);
-    const int nt = (int)(rest / groups);
-    const int n = nt * 16 + (i >> 1) + ((i & 1) ? 8 : 0);
+    const int T = (int)(rest / groups);
+    const int n = T * 32 + g + 8 * (i4 & 1) + 16 * (i4 >> 1);
     out[idx] = scales[(size_t)grp * N + n];
 }
 
 // One thread per 16-byte code chunk: writes 16 codes of two columns, and
 // optionally their fp32 and bf16 dequantized values, using the decoders of
 // the GEMM paths.
-__global__ void unpack_kernel(const uint4 *__restrict__ codes, const uint32_t *__restrict__ sc,
+__global__ void unpack_kernel(const uint4 *__restrict__ codes, const uint16_t *__restrict__ sc,
                               int K, int N, int G, uint8_t *__restrict__ out_codes,
                               float *__restrict__ w_fp32, uint16_t *__restrict__ w_bf16)
 {
-    const long long total = (long long)(N / 16) * (K / 64) * 32;
+    const long long total = (long long)(N / 32) * (K / 64) * 64;
     const long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x;
     if (idx >= total)
         return;
     const int lane = (int)(idx & 31);
-    const long long rest = idx >> 5;
+    const int h = (int)((idx >> 5) & 1);
+    const long long rest = idx >> 6;
     const int kc_count = K / 64;
     const int c = (int)(rest % kc_count);
-    const int nt = (int)(rest / kc_count);
+    const int T = (int)(rest / kc_count);
     const int g = lane >> 2, t = lane & 3;
     const int groups = K / G;
-    const int kbase = c * 64 + t * 16;
-    // the lane's 16 rows lie in one group for G >= 32
-    const uint32_t sword = sc[((size_t)nt * groups + kbase / G) * 8 + g];
-    const uint16_t s_a = (uint16_t)(sword & 0xFFFF), s_b = (uint16_t)(sword >> 16);
-    const ScaleSplit sp_a = split_scale(s_a), sp_b = split_scale(s_b);
-    const float fa = __half2float(__ushort_as_half(s_a)), fb = __half2float(__ushort_as_half(s_b));
     const uint4 v = codes[idx];
     const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+    const int na = T * 32 + h * 16 + g, nb = na + 8;
 
-    uint8_t qa[16], qb[16];
-    uint32_t ba[8], bb[8];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
+        const int k0 = chunk_k0(c, t, j);
+        const uint16_t *e = sc + ((size_t)T * groups + k0 / G) * 32 + g * 4 + 2 * h;
+        const uint16_t s_a = e[0], s_b = e[1];
+        const ScaleSplit sp_a = split_scale(s_a), sp_b = split_scale(s_b);
+        const float fa = __half2float(__ushort_as_half(s_a));
+        const float fb = __half2float(__ushort_as_half(s_b));
         const uint32_t w = wv[j];
-        // decoded exactly as the MMA operands: pairs (k0, k0+1) and (k0+2, k0+3)
-        const uint32_t a01 = int4_pair_minus8<0>(w), b01 = int4_pair_minus8<4>(w);
-        const uint32_t a23 = int4_pair_minus8<8>(w), b23 = int4_pair_minus8<12>(w);
-        ba[2 * j] = scale_pair_rn(a01, sp_a);
-        ba[2 * j + 1] = scale_pair_rn(a23, sp_a);
-        bb[2 * j] = scale_pair_rn(b01, sp_b);
-        bb[2 * j + 1] = scale_pair_rn(b23, sp_b);
-        qa[4 * j + 0] = (w >> 0) & 0xF;
-        qa[4 * j + 1] = (w >> 16) & 0xF;
-        qa[4 * j + 2] = (w >> 8) & 0xF;
-        qa[4 * j + 3] = (w >> 24) & 0xF;
-        qb[4 * j + 0] = (w >> 4) & 0xF;
-        qb[4 * j + 1] = (w >> 20) & 0xF;
-        qb[4 * j + 2] = (w >> 12) & 0xF;
-        qb[4 * j + 3] = (w >> 28) & 0xF;
-    }
-    const int na = nt * 16 + g, nb = na + 8;
-    const size_t oa = (size_t)na * K + kbase, ob = (size_t)nb * K + kbase;
-    if (out_codes) {
-        uint32_t pa[4], pb[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            pa[i] = qa[4 * i] | (qa[4 * i + 1] << 8) | (qa[4 * i + 2] << 16) | ((uint32_t)qa[4 * i + 3] << 24);
-            pb[i] = qb[4 * i] | (qb[4 * i + 1] << 8) | (qb[4 * i + 2] << 16) | ((uint32_t)qb[4 * i + 3] << 24);
+        const uint32_t ba0 = scale_pair_rn(int4_pair_minus8<0>(w), sp_a);
+        const uint32_t ba1 = scale_pair_rn(int4_pair_minus8<8>(w), sp_a);
+        const uint32_t bb0 = scale_pair_rn(int4_pair_minus8<4>(w), sp_b);
+        const uint32_t bb1 = scale_pair_rn(int4_pair_minus8<12>(w), sp_b);
+        const int qa[4] = {(int)(w & 0xF), (int)((w >> 16) & 0xF), (int)((w >> 8) & 0xF),
+                           (int)((w >> 24) & 0xF)};
+        const int qb[4] = {(int)((w >> 4) & 0xF), (int)((w >> 20) & 0xF), (int)((w >> 12) & 0xF),
+                           (int)((w >> 28) & 0xF)};
+        const size_t oa = (size_t)na * K + k0, ob = (size_t)nb * K + k0;
+        if (out_codes) {
+            *reinterpret_cast<uint32_t *>(out_codes + oa) =
+                qa[0] | (qa[1] << 8) | (qa[2] << 16) | ((uint32_t)qa[3] << 24);
+            *reinterpret_cast<uint32_t *>(out_codes + ob) =
+                qb[0] | (qb[1] << 8) | (qb[2] << 16) | ((uint32_t)qb[3] << 24);
         }
-        *reinterpret_cast<uint4 *>(out_codes + oa) = make_uint4(pa[0], pa[1], pa[2], pa[3]);
-        *reinterpret_cast<uint4 *>(out_codes + ob) = make_uint4(pb[0], pb[1], pb[2], pb[3]);
-    }
-    if (w_fp32) {
-#pragma unroll
-        for (int i = 0; i < 16; i += 4) {
-            float4 a, b;
-            a.x = (float)((int)qa[i] - 8) * fa;
-            a.y = (float)((int)qa[i + 1] - 8) * fa;
-            a.z = (float)((int)qa[i + 2] - 8) * fa;
-            a.w = (float)((int)qa[i + 3] - 8) * fa;
-            b.x = (float)((int)qb[i] - 8) * fb;
-            b.y = (float)((int)qb[i + 1] - 8) * fb;
-            b.z = (float)((int)qb[i + 2] - 8) * fb;
-            b.w = (float)((int)qb[i + 3] - 8) * fb;
-            *reinterpret_cast<float4 *>(w_fp32 + oa + i) = a;
-            *reinterpret_cast<float4 *>(w_fp32 + ob + i) = b;
+        if (w_fp32) {
+            *reinterpret_cast<float4 *>(w_fp32 + oa) =
+                make_float4((float)(qa[0] - 8) * fa, (float)(qa[1] - 8) * fa,
+                            (float)(qa[2] - 8) * fa, (float)(qa[3] - 8) * fa);
+            *reinterpret_cast<float4 *>(w_fp32 + ob) =
+                make_float4((float)(qb[0] - 8) * fb, (float)(qb[1] - 8) * fb,
+                            (float)(qb[2] - 8) * fb, (float)(qb[3] - 8) * fb);
         }
-    }
-    if (w_bf16) {
-        *reinterpret_cast<uint4 *>(w_bf16 + oa) = make_uint4(ba[0], ba[1], ba[2], ba[3]);
-        *reinterpret_cast<uint4 *>(w_bf16 + oa + 8) = make_uint4(ba[4], ba[5], ba[6], ba[7]);
-        *reinterpret_cast<uint4 *>(w_bf16 + ob) = make_uint4(bb[0], bb[1], bb[2], bb[3]);
-        *reinterpret_cast<uint4 *>(w_bf16 + ob + 8) = make_uint4(bb[4], bb[5], bb[6], bb[7]);
+        if (w_bf16) {
+            *reinterpret_cast<uint2 *>(w_bf16 + oa) = make_uint2(ba0, ba1);
+            *reinterpret_cast<uint2 *>(w_bf16 + ob) = make_uint2(bb0, bb1);
+        }
     }
 }
 
@@ -200,10 +188,10 @@ inline unsigned blocks_for(long long total, int threads)
 cudaError_t launch_w4a16_repack(const int32_t *qweight, const uint16_t *scales, int K, int N, int G,
                                 void *packed, cudaStream_t stream)
 {
-    const long long nchunks = (long long)(N / 16) * (K / 64) * 32;
+    const long long nchunks = (long long)(N / 32) * (K / 64) * 64;
     repack_codes_kernel<<<blocks_for(nchunks, 256), 256, 0, stream>>>(
         qweight, K, N, reinterpret_cast<uint4 *>(packed));
-    const long long nsc = (long long)(N / 16) * (K / G) * 16;
+    const long long nsc = (long long)(N / 32) * (K / G) * 32;
     uint16_t *sc_out = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(packed) + (size_t)N * K / 2);
     repack_scales_kernel<<<blocks_for(nsc, 256), 256, 0, stream>>>(scales, K, N, G, sc_out);
     return cudaGetLastError();
@@ -212,8 +200,8 @@ cudaError_t launch_w4a16_repack(const int32_t *qweight, const uint16_t *scales, 
 cudaError_t launch_w4a16_unpack(const void *packed, int K, int N, int G, uint8_t *codes,
                                 float *w_fp32, uint16_t *w_bf16, cudaStream_t stream)
 {
-    const long long nchunks = (long long)(N / 16) * (K / 64) * 32;
-    const uint32_t *sc = reinterpret_cast<const uint32_t *>(static_cast<const uint8_t *>(packed) +
+    const long long nchunks = (long long)(N / 32) * (K / 64) * 64;
+    const uint16_t *sc = reinterpret_cast<const uint16_t *>(static_cast<const uint8_t *>(packed) +
                                                             (size_t)N * K / 2);
     unpack_kernel<<<blocks_for(nchunks, 256), 256, 0, stream>>>(
         reinterpret_cast<const uint4 *>(packed), sc, K, N, G, codes, w_fp32, w_bf16);
