@@ -1,25 +1,33 @@
 // Tensor-core GEMM for larger M (MTP verify batches, prefill chunks).
 //
-// Y[M][N] = X[M][K] * dequant(W)^T on the 5th-generation tensor cores.
-// Persistent, warp-specialised CTA (one per SM), output tile 128 x 256,
-// k-block 64:
-//   warp 0        producer: tensor-map copies of the X tile (128-byte
-//                 swizzle, the MMA's A operand as is) and of the packed
-//                 weight tile (codes + scales) into two shared-memory rings;
-//   warp 1        allocates 512 TMEM columns (two 128 x 256 fp32
-//                 accumulators) and issues tcgen05.mma (kind::f16, bf16 x
-//                 bf16 -> fp32) from one thread; tcgen05.commit releases
-//                 the operand slots and publishes finished accumulators;
-//   warps 2..5    epilogue: tcgen05.ld of their 32 TMEM lanes, fp32 -> bf16,
-//                 stores to Y; overlaps the next tile's main loop;
-//   warps 6..13   dequantisers: packed weight slot -> bf16 B operand in the
-//                 128-byte-swizzled K-major layout the MMA reads, one
-//                 rounding per weight (INT4: (q - 8) * scale; MXFP8:
-//                 e4m3 * 2^(E - 127)), then a proxy fence so the tensor
-//                 core sees the generic-proxy stores.
-// Every wait is an mbarrier phase wait with a time limit; a timeout sets
-// a CTA-wide abort flag, records MXG_ERR_TIMEOUT and every role drains to
-// the final barrier, where TMEM is released.
+// Y[M][N] = X[M][K] * dequant(W)^T on the 5th-generation tensor cores, with
+// the roles of the operands swapped so that the dequantized weights never
+// touch shared memory:
+//   * a CTA pair (cluster of 2, tcgen05 cta_group::2) owns 256 weight
+//     columns (128 per CTA) x BT tokens; the MMA is D[n][m] += W[n][k] X[m][k]
+//     with M_mma = 256 weight columns, N_mma = BT tokens, K = 16 per step;
+//   * A = the weights, decoded by eight dequantiser warps per CTA straight
+//     from the packed bytes into tensor memory (tcgen05.st, 16 lanes x 256
+//     bits per store): the packed INT4 layout places one lane's 16 bytes
+//     exactly on one thread's share of such a store;
+//   * B = the activations, fetched by the tensor-map engine with the 128-byte
+//     swizzle (each CTA its BT/2 tokens; the pair's MMA reads both halves);
+//   * D = fp32 accumulators in tensor memory; four epilogue warps per CTA
+//     read them back (tcgen05.ld) and store bf16 Y.
+// Shared memory then only holds packed weights (0.5 or 1 byte per weight)
+// and activations, which keeps the pair inside the SM's shared-memory
+// bandwidth at full tensor rate.
+//
+// Warp roles per CTA (448 threads):
+//   warp 0        producer: activation and packed-weight copies;
+//   warp 1        tensor-memory allocation; in the even CTA also the single
+//                 thread that issues tcgen05.mma and tcgen05.commit;
+//   warps 2..5    epilogue;
+//   warps 6..13   dequantisers (warp w writes lanes 32*(w%4) + 16*h .. +15,
+//                 h = (w - 6) / 4).
+// Every wait is an mbarrier phase wait with a time limit; a timeout sets a
+// CTA-wide abort flag, records MXG_ERR_TIMEOUT and every role drains to the
+// end, where tensor memory is released.
 #include <algorithm>
 
 #include "common.cuh"
@@ -28,14 +36,11 @@
 namespace mxg {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64;
-constexpr int kSX = 4;   // X ring depth
-constexpr int kSW = 4;   // packed-weight ring depth
-constexpr int kSB = 3;   // bf16-weight ring depth
-constexpr int kXBytes = BM * BK * 2;                 // 16 KB
-constexpr int kWbBytes = BN * BK * 2;                // 32 KB
-constexpr int kWpBytes = 9 * 1024;                   // codes (8 KB or 16 KB MXFP8: see below)
-constexpr int kWpBytesMx = BN * BK;                  // 16 KB of E4M3 codes
+constexpr int BW = 128;  // weight columns per CTA
+constexpr int BK = 64;   // k per block
+constexpr int kSX = 4;   // activation ring
+constexpr int kSW = 4;   // packed-weight ring
+constexpr int kSA = 4;   // tensor-memory A ring (32 columns each)
 constexpr int kProducerWarp = 0, kMmaWarp = 1, kEpiWarp0 = 2, kNumEpiWarps = 4;
 constexpr int kDqWarp0 = 6, kNumDqWarps = 8;
 constexpr int kThreads = (kDqWarp0 + kNumDqWarps) * 32;
@@ -43,18 +48,20 @@ constexpr uint32_t kTmemCols = 512;
 
 enum Fmt { kInt4 = 0, kMxfp8 = 1 };
 
-template <int F>
+template <int F, int BT>
 struct Layout {
-    static constexpr int wp_bytes = (F == kInt4) ? kWpBytes : kWpBytesMx;
+    static constexpr int x_slot = (BT / 2) * BK * 2;                // bf16 activations
+    static constexpr int wp_slot = (F == kInt4) ? 5120 : BW * BK;   // packed weights
     static constexpr int x_off = 0;
-    static constexpr int wb_off = x_off + kSX * kXBytes;
-    static constexpr int wp_off = wb_off + kSB * kWbBytes;
-    static constexpr int bar_off = wp_off + kSW * wp_bytes;
-    // barriers: x_full, x_empty, wp_full, wp_empty, wb_full, wb_empty, acc_full, acc_empty
-    static constexpr int n_bars = 2 * kSX + 2 * kSW + 2 * kSB + 4;
+    static constexpr int wp_off = x_off + kSX * x_slot;
+    static constexpr int bar_off = wp_off + kSW * wp_slot;
+    static constexpr int n_bars = 2 * kSX + 2 * kSW + 2 * kSA + 2;
     static constexpr int misc_off = bar_off + n_bars * 8;
     static constexpr int total = misc_off + 16;
     static constexpr size_t smem_bytes = (size_t)total + 1024;  // + alignment slack
+    static constexpr uint32_t acc_col = 0;                     // D: columns [0, BT)
+    static constexpr uint32_t a_col = BT;                      // A ring after D
+    static_assert(BT + 32 * kSA <= (int)kTmemCols, "tensor memory budget");
 };
 
 struct TcParams {
@@ -66,19 +73,59 @@ struct TcParams {
     int num_tiles;
 };
 
-// ----------------------------------------------------------- tcgen05 PTX
-__device__ __forceinline__ void tmem_alloc(uint32_t *slot, uint32_t cols)
+// ----------------------------------------------------------- cluster PTX
+__device__ __forceinline__ uint32_t cluster_ctarank()
 {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Tensor copy into this CTA's shared memory that completes on an mbarrier of
+// the even CTA of the pair (no multicast).
+__device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *map, int c0, int c1,
+                                                 uint32_t leader_bar, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(c0), "r"(c1), "r"(leader_bar), "l"(policy)
+        : "memory");
+}
+
+// ----------------------------------------------------------- tcgen05 PTX
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t *slot, uint32_t cols)
+{
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(slot)),
                  "r"(cols)
                  : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols)
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t cols)
 {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols)
                  : "memory");
 }
 
@@ -92,23 +139,47 @@ __device__ __forceinline__ void tc_fence_after()
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-__device__ __forceinline__ void tc_commit(uint64_t *bar)
+// Arrive on the barrier at this offset in both CTAs of the pair once every
+// tcgen05 operation issued so far by this thread has completed.
+__device__ __forceinline__ void tc_commit_pair(uint64_t *bar)
 {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     smem_u32(bar))
-                 : "memory");
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(smem_u32(bar)),
+        "h"((uint16_t)0x3)
+        : "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, both K-major, kind::f16.
-__device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                           uint32_t idesc, uint32_t accumulate)
+// D[tmem] (+)= A[tmem] * B[smem]^T over the CTA pair, kind::f16.
+__device__ __forceinline__ void tc_mma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate)
 {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// 16 lanes x 256 bits, four times along the columns: thread (g, t) writes
+// lanes g and g + 8 of the 16-lane slab, columns 8r + 2t and 8r + 2t + 1 of
+// repetition r, from registers v[4r .. 4r + 3] (lane g: two columns, then
+// lane g + 8: two columns).
+__device__ __forceinline__ void tmem_st_16x256b_x4(uint32_t taddr, const uint32_t (&v)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+        "r"(v[15])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait()
+{
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // 32 consecutive fp32 columns of this thread's TMEM lane.
@@ -140,9 +211,13 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
     return d;
 }
 
-// Instruction descriptor: D fp32, A and B bf16, both K-major, M = 128, N = 256.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                            ((uint32_t)(BM >> 4) << 24);
+// Instruction descriptor: D fp32, A and B bf16, both K-major, M = 256 (pair), N = BT.
+template <int BT>
+__host__ __device__ constexpr uint32_t idesc_pair()
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BT >> 3) << 17) |
+           ((uint32_t)(256 >> 4) << 24);
+}
 
 // Bounded wait that also gives up as soon as another role has aborted.
 __device__ __forceinline__ bool role_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
@@ -166,112 +241,90 @@ __device__ __forceinline__ bool role_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
-// Byte offset of 16-byte chunk c of row r in a 128-byte-swizzled tile.
-__device__ __forceinline__ uint32_t sw128_off(int r, int c)
-{
-    return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
-}
-
-__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
-{
-    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
-                 "r"(d)
-                 : "memory");
-}
-
-__device__ __forceinline__ void sts64(uint32_t addr, uint32_t a, uint32_t b)
-{
-    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
-}
-
-// INT4: one packed 16-byte chunk (n32 tile tl, half h, lane) = two columns x
-// 16 k -> eight 8-byte bf16 stores into the 128-byte-swizzled B tile.
-// Word j holds k = 16j + 4t .. 16j + 4t + 3 of the k-block.
-__device__ __forceinline__ void dequant_int4_chunk(const uint8_t *wp_slot, uint32_t wb_slot, int tl,
-                                                   int h, int lane, int G, int gpk)
+// INT4: the dequantiser thread's 16 packed bytes (n32 tile q of the CTA,
+// half h, lane) -> 16 registers of bf16 pairs for a 16x256b x4 store.
+__device__ __forceinline__ void dequant_int4(const uint8_t *wp_slot, int q, int h, int lane, int G,
+                                             int gpk, uint32_t (&v)[16])
 {
     const int g = lane >> 2, t = lane & 3;
-    const uint4 v = lds128(wp_slot + tl * 1024 + h * 512 + lane * 16);
-    const uint32_t wj[4] = {v.x, v.y, v.z, v.w};
-    const int ra = tl * 32 + h * 16 + g, rb = ra + 8;
+    const uint4 c = lds128(wp_slot + q * 1024 + h * 512 + lane * 16);
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int gi = (16 * j + 4 * t) / G;  // group inside the k-block
-        const uint32_t sw = lds32(wp_slot + 8192 + tl * (64 * gpk) + gi * 64 + g * 8 + h * 4);
+        const uint32_t sw = lds32(wp_slot + 4096 + q * (64 * gpk) + gi * 64 + g * 8 + h * 4);
         const ScaleSplit sa = split_scale((uint16_t)(sw & 0xFFFF));
         const ScaleSplit sb = split_scale((uint16_t)(sw >> 16));
-        const uint32_t w = wj[j];
-        const int chunk = 2 * j + (t >> 1), half = (t & 1) * 8;
-        sts64(wb_slot + sw128_off(ra, chunk) + half, scale_pair_rn(int4_pair_minus8<0>(w), sa),
-              scale_pair_rn(int4_pair_minus8<8>(w), sa));
-        sts64(wb_slot + sw128_off(rb, chunk) + half, scale_pair_rn(int4_pair_minus8<4>(w), sb),
-              scale_pair_rn(int4_pair_minus8<12>(w), sb));
+        v[4 * j + 0] = scale_pair_rn(int4_pair_minus8<0>(w[j]), sa);
+        v[4 * j + 1] = scale_pair_rn(int4_pair_minus8<8>(w[j]), sa);
+        v[4 * j + 2] = scale_pair_rn(int4_pair_minus8<4>(w[j]), sb);
+        v[4 * j + 3] = scale_pair_rn(int4_pair_minus8<12>(w[j]), sb);
     }
 }
 
-// MXFP8: row r of the tile (64 codes, 64-byte swizzled rows) -> 128 bytes of bf16.
-__device__ __forceinline__ void dequant_mx_row(const uint8_t *wp_slot, uint32_t wb_slot, int r,
-                                               float s0, float s1)
+// MXFP8: rows ra = 32q + 16h + g and ra + 8 of the CTA's [128][64 B] code
+// tile (64-byte swizzle); for repetition j the thread needs k = 16j + 4t ..
+// 16j + 4t + 3 of both rows (one 32-bit word each).
+__device__ __forceinline__ void dequant_mx(const uint8_t *wp_slot, int q, int h, int lane,
+                                           const float (&sa)[2], const float (&sb)[2],
+                                           uint32_t (&v)[16])
 {
-    uint32_t out[32];
+    const int g = lane >> 2, t = lane & 3;
+    const int ra = q * 32 + h * 16 + g, rb = ra + 8;
+    const int swa = (ra >> 1) & 3, swb = (rb >> 1) & 3;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        const uint4 v = lds128(wp_slot + r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
-        const float s = (c < 2) ? s0 : s1;
-        e4m3x4_scaled(v.x, s, out[8 * c + 0], out[8 * c + 1]);
-        e4m3x4_scaled(v.y, s, out[8 * c + 2], out[8 * c + 3]);
-        e4m3x4_scaled(v.z, s, out[8 * c + 4], out[8 * c + 5]);
-        e4m3x4_scaled(v.w, s, out[8 * c + 6], out[8 * c + 7]);
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t wa = lds32(wp_slot + ra * 64 + ((j ^ swa) << 4) + 4 * t);
+        const uint32_t wb = lds32(wp_slot + rb * 64 + ((j ^ swb) << 4) + 4 * t);
+        e4m3x4_scaled(wa, sa[j >> 1], v[4 * j + 0], v[4 * j + 1]);
+        e4m3x4_scaled(wb, sb[j >> 1], v[4 * j + 2], v[4 * j + 3]);
     }
-#pragma unroll
-    for (int c = 0; c < 8; ++c)
-        sts128(wb_slot + sw128_off(r, c), out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
 }
 
-template <int F>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int F, int BT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap x_map,
                    const __grid_constant__ CUtensorMap w_map,
                    const __grid_constant__ CUtensorMap s_map, const TcParams p)
 {
-    using L = Layout<F>;
+    using L = Layout<F, BT>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::bar_off);
     uint64_t *x_full = bars, *x_empty = bars + kSX;
     uint64_t *wp_full = bars + 2 * kSX, *wp_empty = wp_full + kSW;
-    uint64_t *wb_full = wp_empty + kSW, *wb_empty = wb_full + kSB;
-    uint64_t *acc_full = wb_empty + kSB, *acc_empty = acc_full + 2;
+    uint64_t *a_full = wp_empty + kSW, *a_empty = a_full + kSA;
+    uint64_t *acc_full = a_empty + kSA, *acc_empty = acc_full + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::misc_off);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::misc_off + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();   // 0: issues the MMAs; 1: its pair
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kSX; ++i) {
-            mbar_init(&x_full[i], 1);
-            mbar_init(&x_empty[i], 1);
+            mbar_init(&x_full[i], 1);            // leader: producer arrive + both copies
+            mbar_init(&x_empty[i], 1);           // commit from the MMA
         }
         for (int i = 0; i < kSW; ++i) {
             mbar_init(&wp_full[i], 1);
             mbar_init(&wp_empty[i], kNumDqWarps);
         }
-        for (int i = 0; i < kSB; ++i) {
-            mbar_init(&wb_full[i], kNumDqWarps);
-            mbar_init(&wb_empty[i], 1);
+        for (int i = 0; i < kSA; ++i) {
+            mbar_init(&a_full[i], 2 * kNumDqWarps);   // leader: dequantisers of both CTAs
+            mbar_init(&a_empty[i], 1);                 // commit from the MMA
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&acc_full[i], 1);
-            mbar_init(&acc_empty[i], kNumEpiWarps);
-        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 2 * kNumEpiWarps);        // leader: epilogues of both CTAs
         *abort_flag = 0;
         fence_barrier_init();
     }
     if (warp == kMmaWarp)
-        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_alloc_pair(tmem_slot, kTmemCols);
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();   // barriers of both CTAs initialised, tensor memory allocated
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
@@ -287,203 +340,210 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t pol_x = l2_policy_evict_last();
             uint32_t it = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+            for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
                 const int nb = tile / p.mtiles, mt = tile % p.mtiles;
                 for (int kb = 0; kb < p.kblocks && ok; ++kb, ++it) {
-                    const int sw = it % kSW, sx = it % kSX;
-                    ok = role_wait(&wp_empty[sw], ((it / kSW) & 1) ^ 1, abort_flag, p.hdr, 301);
+                    const int sx = it % kSX, sw = it % kSW;
+                    // activations: this CTA's BT/2 tokens, completing on the leader's barrier
+                    ok = role_wait(&x_empty[sx], ((it / kSX) & 1) ^ 1, abort_flag, p.hdr, 401);
                     if (!ok)
                         break;
-                    uint8_t *wdst = smem + L::wp_off + sw * L::wp_bytes;
+                    if (rank == 0)
+                        mbar_arrive_expect_tx(&x_full[sx], 2u * L::x_slot);
+                    tma_load_2d_pair(smem + L::x_off + sx * L::x_slot, &x_map, kb * BK,
+                                     mt * BT + (int)rank * (BT / 2),
+                                     mapa_shared(smem_u32(&x_full[sx]), 0), pol_x);
+                    // packed weights of this CTA's 128 columns
+                    ok = role_wait(&wp_empty[sw], ((it / kSW) & 1) ^ 1, abort_flag, p.hdr, 402);
+                    if (!ok)
+                        break;
+                    uint8_t *wdst = smem + L::wp_off + sw * L::wp_slot;
+                    const int n32 = (nb * 2 * BW + (int)rank * BW) / 32;
                     if (F == kInt4) {
-                        const uint32_t sbytes = 512u * gpk;
-                        mbar_arrive_expect_tx(&wp_full[sw], 8192u + sbytes);
-                        tma_load_2d(wdst, &w_map, kb * 128, nb * 8, &wp_full[sw], pol_w);
-                        tma_load_2d(wdst + 8192, &s_map, (kb * 64 / p.G) * 8, nb * 8, &wp_full[sw],
+                        mbar_arrive_expect_tx(&wp_full[sw], 4096u + 256u * gpk);
+                        tma_load_2d(wdst, &w_map, kb * 128, n32, &wp_full[sw], pol_w);
+                        tma_load_2d(wdst + 4096, &s_map, (kb * BK / p.G) * 8, n32, &wp_full[sw],
                                     pol_w);
                     } else {
-                        mbar_arrive_expect_tx(&wp_full[sw], (uint32_t)kWpBytesMx);
-                        tma_load_2d(wdst, &w_map, kb * 64, nb * BN, &wp_full[sw], pol_w);
+                        mbar_arrive_expect_tx(&wp_full[sw], (uint32_t)(BW * BK));
+                        tma_load_2d(wdst, &w_map, kb * BK, n32 * 32, &wp_full[sw], pol_w);
                     }
-                    ok = role_wait(&x_empty[sx], ((it / kSX) & 1) ^ 1, abort_flag, p.hdr, 302);
-                    if (!ok)
-                        break;
-                    mbar_arrive_expect_tx(&x_full[sx], (uint32_t)kXBytes);
-                    tma_load_2d(smem + L::x_off + sx * kXBytes, &x_map, kb * 64, mt * BM, &x_full[sx],
-                                pol_x);
                 }
             }
         }
     } else if (warp == kMmaWarp) {
-        if (lane == 0) {
+        if (rank == 0 && lane == 0) {
+            constexpr uint32_t idesc = idesc_pair<BT>();
             uint32_t it = 0, tcount = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++tcount) {
-                const int acc = tcount & 1;
-                ok = role_wait(&acc_empty[acc], ((tcount >> 1) & 1) ^ 1, abort_flag, p.hdr, 311);
+            for (int tile = pair; tile < p.num_tiles && ok; tile += npairs, ++tcount) {
+                ok = role_wait(acc_empty, (tcount & 1) ^ 1, abort_flag, p.hdr, 411);
                 if (!ok)
                     break;
                 tc_fence_after();
-                const uint32_t d = tmem_base + acc * BN;
+                const uint32_t d = tmem_base + L::acc_col;
                 for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
-                    const int sx = it % kSX, sb = it % kSB;
-                    ok = role_wait(&x_full[sx], (it / kSX) & 1, abort_flag, p.hdr, 312) &&
-                         role_wait(&wb_full[sb], (it / kSB) & 1, abort_flag, p.hdr, 313);
+                    const int sx = it % kSX, sa = it % kSA;
+                    ok = role_wait(&x_full[sx], (it / kSX) & 1, abort_flag, p.hdr, 412) &&
+                         role_wait(&a_full[sa], (it / kSA) & 1, abort_flag, p.hdr, 413);
                     if (!ok)
                         break;
                     tc_fence_after();
-                    const uint32_t xa = smem_u32(smem + L::x_off + sx * kXBytes);
-                    const uint32_t wa = smem_u32(smem + L::wb_off + sb * kWbBytes);
+                    const uint32_t xa = smem_u32(smem + L::x_off + sx * L::x_slot);
+                    const uint32_t a = tmem_base + L::a_col + 32 * sa;
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)
-                        tc_mma_f16(d, sw128_desc(xa + 32 * k), sw128_desc(wa + 32 * k), kIdesc,
-                                   (kb > 0 || k > 0) ? 1u : 0u);
-                    tc_commit(&x_empty[sx]);
-                    tc_commit(&wb_empty[sb]);
+                        tc_mma_ts_pair(d, a + 8 * k, sw128_desc(xa + 32 * k), idesc,
+                                       (kb > 0 || k > 0) ? 1u : 0u);
+                    tc_commit_pair(&x_empty[sx]);
+                    tc_commit_pair(&a_empty[sa]);
                 }
                 if (ok)
-                    tc_commit(&acc_full[acc]);
+                    tc_commit_pair(acc_full);
             }
         }
     } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + kNumEpiWarps) {
         const int q = warp & 3;  // TMEM lane quadrant this warp may access
+        const uint32_t leader_acc_empty = mapa_shared(smem_u32(acc_empty), 0);
         uint32_t tcount = 0;
-        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
-            const int acc = tcount & 1;
-            if (!role_wait(&acc_full[acc], (tcount >> 1) & 1, abort_flag, p.hdr, 321))
+        for (int tile = pair; tile < p.num_tiles; tile += npairs, ++tcount) {
+            if (!role_wait(acc_full, tcount & 1, abort_flag, p.hdr, 421))
                 break;
             tc_fence_after();
             const int nb = tile / p.mtiles, mt = tile % p.mtiles;
-            const int row = mt * BM + q * 32 + lane;
-            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+            const int n = nb * 2 * BW + (int)rank * BW + q * 32 + lane;   // this thread's column
+            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + L::acc_col;
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
+            for (int c = 0; c < BT / 32; ++c) {
                 uint32_t r[32];
                 tmem_ld32(tbase + c * 32, r);
-                const int n0 = nb * BN + c * 32;
-                if (row < p.M && n0 < p.N) {
-                    uint32_t o[16];
+                const int m0 = mt * BT + c * 32;
+                if (n < p.N) {
+                    uint16_t *yc = p.Y + (size_t)m0 * p.N + n;
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        __nv_bfloat162 b = __floats2bfloat162_rn(__uint_as_float(r[2 * i]),
-                                                                 __uint_as_float(r[2 * i + 1]));
-                        o[i] = *reinterpret_cast<uint32_t *>(&b);
-                    }
-                    uint16_t *yrow = p.Y + (size_t)row * p.N;
-                    if (n0 + 32 <= p.N && (p.N & 7) == 0) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(yrow + n0);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
-                    } else {
-                        for (int i = 0; i < 32 && n0 + i < p.N; ++i)
-                            yrow[n0 + i] = (uint16_t)(o[i >> 1] >> ((i & 1) * 16));
-                    }
+                    for (int i = 0; i < 32; ++i)
+                        if (m0 + i < p.M)
+                            yc[(size_t)i * p.N] = f32_to_bf16_bits(__uint_as_float(r[i]));
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&acc_empty[acc]);
+                mbar_arrive_cluster(leader_acc_empty);
         }
     } else {
-        // dequantisers
+        // dequantisers: warp -> (quadrant q, half h) of the CTA's 128 weight rows
         const int dw = warp - kDqWarp0;
-        const int dt = dw * 32 + lane;
+        const int q = warp & 3, h = dw >> 2;
+        const int g = lane >> 2;
         uint32_t it = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+        for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
             const int nb = tile / p.mtiles;
             for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
-                const int sw = it % kSW, sb = it % kSB;
-                float s0 = 0.f, s1 = 0.f;
+                const int sw = it % kSW, sa = it % kSA;
+                float sca[2] = {1.f, 1.f}, scb[2] = {1.f, 1.f};
                 if (F == kMxfp8) {
-                    // the row's two E8M0 scales of this k-block (from L2)
-                    const int n = nb * BN + dt;
+                    // E8M0 scales of rows ra, ra + 8 for the two 32-blocks of this k-block
                     const int blocks = p.K / 32;
-                    const int b0 = kb * 2;
-                    uint32_t e0 = 127, e1 = 127;
-                    if (n < p.N) {
-                        e0 = __ldg(p.Ws + (size_t)n * blocks + b0);
-                        if (b0 + 1 < blocks)
-                            e1 = __ldg(p.Ws + (size_t)n * blocks + b0 + 1);
+                    const long long ra =
+                        (long long)nb * 2 * BW + (int)rank * BW + q * 32 + h * 16 + g;
+#pragma unroll
+                    for (int b = 0; b < 2; ++b) {
+                        const int blk = kb * 2 + b;
+                        uint32_t ea = 127, eb = 127;
+                        if (blk < blocks) {
+                            if (ra < p.N)
+                                ea = __ldg(p.Ws + ra * blocks + blk);
+                            if (ra + 8 < p.N)
+                                eb = __ldg(p.Ws + (ra + 8) * blocks + blk);
+                        }
+                        sca[b] = e8m0_to_f32(ea);
+                        scb[b] = e8m0_to_f32(eb);
                     }
-                    s0 = e8m0_to_f32(e0);
-                    s1 = e8m0_to_f32(e1);
                 }
-                ok = role_wait(&wp_full[sw], (it / kSW) & 1, abort_flag, p.hdr, 331) &&
-                     role_wait(&wb_empty[sb], ((it / kSB) & 1) ^ 1, abort_flag, p.hdr, 332);
+                ok = role_wait(&wp_full[sw], (it / kSW) & 1, abort_flag, p.hdr, 431) &&
+                     role_wait(&a_empty[sa], ((it / kSA) & 1) ^ 1, abort_flag, p.hdr, 432);
                 if (!ok)
                     break;
-                const uint8_t *wp_slot = smem + L::wp_off + sw * L::wp_bytes;
-                const uint32_t wb_slot = smem_u32(smem + L::wb_off + sb * kWbBytes);
-                if (F == kInt4) {
-                    dequant_int4_chunk(wp_slot, wb_slot, dw, 0, lane, p.G, gpk);
-                    dequant_int4_chunk(wp_slot, wb_slot, dw, 1, lane, p.G, gpk);
-                } else {
-                    dequant_mx_row(wp_slot, wb_slot, dt, s0, s1);
-                }
-                fence_proxy_async_smem();
+                tc_fence_after();
+                const uint8_t *wp_slot = smem + L::wp_off + sw * L::wp_slot;
+                uint32_t v[16];
+                if (F == kInt4)
+                    dequant_int4(wp_slot, q, h, lane, p.G, gpk, v);
+                else
+                    dequant_mx(wp_slot, q, h, lane, sca, scb, v);
+                tmem_st_16x256b_x4(
+                    tmem_base + ((uint32_t)(q * 32 + h * 16) << 16) + L::a_col + 32 * sa, v);
+                tmem_st_wait();
+                tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
-                    mbar_arrive(&wb_full[sb]);
                     mbar_arrive(&wp_empty[sw]);
+                    mbar_arrive_cluster(mapa_shared(smem_u32(&a_full[sa]), 0));
                 }
             }
         }
     }
 
+    // teardown: every role of both CTAs is done with tensor memory
     tc_fence_before();
     __syncthreads();
+    cluster_sync();
     tc_fence_after();
     if (warp == kMmaWarp)
-        tmem_dealloc(tmem_base, kTmemCols);
+        tmem_dealloc_pair(tmem_base, kTmemCols);
 }
 
-template <int F>
-bool tc_plan(int device, int M, int N, int K, TcPlan *plan)
-{
-    const DeviceInfo &di = device_info(device);
-    if ((size_t)di.smem_optin < Layout<F>::smem_bytes)
-        return false;
-    TcPlan pl{};
-    pl.bm = BM;
-    pl.bn = BN;
-    pl.bk = BK;
-    pl.mtiles = (M + BM - 1) / BM;
-    pl.ntiles = (N + BN - 1) / BN;
-    pl.splits = 1;
-    const int tiles = pl.mtiles * pl.ntiles;
-    pl.grid = std::min(tiles, di.sms);
-    pl.smem = Layout<F>::smem_bytes;
-    pl.partial_bytes = 0;
-    pl.counters = 0;
-    *plan = pl;
-    return true;
-}
-
-template <int F>
+template <int F, int BT>
 cudaError_t tc_launch(const TcPlan &pl, const CUtensorMap &xm, const CUtensorMap &wm,
                       const CUtensorMap &sm, TcParams p, cudaStream_t stream)
 {
-    const void *fn = reinterpret_cast<const void *>(&tc_gemm_kernel<F>);
+    const void *fn = reinterpret_cast<const void *>(&tc_gemm_kernel<F, BT>);
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e =
-            cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
+        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)Layout<F, BT>::smem_bytes);
         if (e != cudaSuccess)
             return e;
         attr_set = true;
     }
     void *args[] = {const_cast<CUtensorMap *>(&xm), const_cast<CUtensorMap *>(&wm),
                     const_cast<CUtensorMap *>(&sm), &p};
-    return cudaLaunchKernel(fn, dim3(pl.grid), dim3(kThreads), args, pl.smem, stream);
+    // the cluster shape (2, 1, 1) is part of the kernel
+    return cudaLaunchKernel(fn, dim3(pl.grid), dim3(kThreads), args, Layout<F, BT>::smem_bytes,
+                            stream);
 }
 
-bool x_map(CUtensorMap *m, const void *X, int M, int K)
+bool x_map(CUtensorMap *m, const void *X, int M, int K, int BT)
 {
     return encode_tensor_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)K, (uint64_t)M,
-                                (uint64_t)K * 2, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+                                (uint64_t)K * 2, BK, BT / 2, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+template <int F>
+bool tc_plan(int device, int M, int N, int K, TcPlan *plan)
+{
+    (void)K;
+    const DeviceInfo &di = device_info(device);
+    const int BT = M <= 128 ? 128 : 256;
+    const size_t smem = BT == 128 ? Layout<F, 128>::smem_bytes : Layout<F, 256>::smem_bytes;
+    if ((size_t)di.smem_optin < smem || di.sms < 2)
+        return false;
+    TcPlan pl{};
+    pl.bm = BT;
+    pl.bn = 2 * BW;
+    pl.bk = BK;
+    pl.mtiles = (M + BT - 1) / BT;
+    pl.ntiles = (N + 2 * BW - 1) / (2 * BW);
+    pl.splits = 1;
+    const int tiles = pl.mtiles * pl.ntiles;
+    pl.grid = 2 * std::min(tiles, di.sms / 2);
+    pl.smem = smem;
+    pl.partial_bytes = 0;
+    pl.counters = 0;
+    *plan = pl;
+    return true;
 }
 
 }  // namespace
@@ -501,14 +561,14 @@ cudaError_t launch_w4a16_tc(const TcPlan &pl, const void *X, const void *packed,
     const uint8_t *codes = static_cast<const uint8_t *>(packed);
     const uint8_t *scales = codes + (size_t)N * K / 2;
     const int gpk = std::max(1, BK / G);
-    if (!x_map(&xm, X, M, K) ||
-        // codes: rows = n32 tiles of 2K u64 words (K/64 chunks of 1 KB); box = one chunk x 8 tiles
+    if (!x_map(&xm, X, M, K, pl.bm) ||
+        // codes: rows = n32 tiles of 2K u64 words (K/64 chunks of 1 KB); box = one chunk x 4 tiles
         !encode_tensor_map_2d(&wm, CU_TENSOR_MAP_DATA_TYPE_UINT64, codes, (uint64_t)K * 2,
-                              (uint64_t)(N / 32), (uint64_t)K * 16, 128, 8,
+                              (uint64_t)(N / 32), (uint64_t)K * 16, 128, BW / 32,
                               CU_TENSOR_MAP_SWIZZLE_NONE) ||
         // scales: rows = n32 tiles, K/G groups of 8 u64 words (64 bytes) per row
         !encode_tensor_map_2d(&sm, CU_TENSOR_MAP_DATA_TYPE_UINT64, scales, (uint64_t)(K / G) * 8,
-                              (uint64_t)(N / 32), (uint64_t)(K / G) * 64, 8 * gpk, 8,
+                              (uint64_t)(N / 32), (uint64_t)(K / G) * 64, 8 * gpk, BW / 32,
                               CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     TcParams p{};
@@ -523,7 +583,9 @@ cudaError_t launch_w4a16_tc(const TcPlan &pl, const void *X, const void *packed,
     p.ntiles = pl.ntiles;
     p.kblocks = K / BK;
     p.num_tiles = pl.mtiles * pl.ntiles;
-    return tc_launch<kInt4>(pl, xm, wm, sm, p, stream);
+    if (pl.bm == 128)
+        return tc_launch<kInt4, 128>(pl, xm, wm, sm, p, stream);
+    return tc_launch<kInt4, 256>(pl, xm, wm, sm, p, stream);
 }
 
 bool plan_mxfp8_tc(int device, int M, int N, int K, TcPlan *plan)
@@ -536,9 +598,9 @@ cudaError_t launch_mxfp8_tc(const TcPlan &pl, const void *X, const uint8_t *Wq,
                             cudaStream_t stream)
 {
     alignas(64) CUtensorMap xm, wm;
-    if (!x_map(&xm, X, M, K) ||
+    if (!x_map(&xm, X, M, K, pl.bm) ||
         !encode_tensor_map_2d(&wm, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, (uint64_t)K, (uint64_t)N,
-                              (uint64_t)K, BK, BN, CU_TENSOR_MAP_SWIZZLE_64B))
+                              (uint64_t)K, BK, BW, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
     TcParams p{};
     p.Y = static_cast<uint16_t *>(Y);
@@ -552,7 +614,9 @@ cudaError_t launch_mxfp8_tc(const TcPlan &pl, const void *X, const uint8_t *Wq,
     p.ntiles = pl.ntiles;
     p.kblocks = (K + BK - 1) / BK;
     p.num_tiles = pl.mtiles * pl.ntiles;
-    return tc_launch<kMxfp8>(pl, xm, wm, wm, p, stream);
+    if (pl.bm == 128)
+        return tc_launch<kMxfp8, 128>(pl, xm, wm, wm, p, stream);
+    return tc_launch<kMxfp8, 256>(pl, xm, wm, wm, p, stream);
 }
 
 }  // namespace mxg

@@ -330,9 +330,10 @@ __global__ void __launch_bounds__(kWarps * 32, TT == 1 ? 3 : 2) w4a16_stream_ker
                 seg_begin = u + 1;
             }
         }
+        // every lane's reads of this slot have returned (their values are
+        // consumed above), so the slot can be refilled
         __syncwarp();
         if (lane == 0 && left > 0) {
-            fence_proxy_async_smem();  // our reads of this slot precede the next copy into it
             const int nu = (int)min((long long)MD::kUnitsPerStage, left);
             const uint32_t cb = nu * MD::kChunks * 1024, sb = nu * MD::kGroups * 64;
             uint8_t *dst = ring + slot * kStageBytes;
