@@ -114,6 +114,22 @@ bool encode_tensor_map_2d(void *map, int dtype_cu, const void *base, uint64_t in
     return r == CUDA_SUCCESS;
 }
 
+cudaError_t launch_pdl(const void *fn, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       void **args)
+{
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
 // Workspace needs of the two paths for one shape (0 when the path cannot run it).
 static size_t w4a16_stream_ws(int dev, int M, int N, int K, int G)
 {

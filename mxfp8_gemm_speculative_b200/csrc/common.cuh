@@ -77,15 +77,20 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// One bounded probe of the phase: the thread may be suspended (not issuing)
+// for up to kSuspendNs while the phase is incomplete, so waiting warps leave
+// the issue slots to working ones.
+constexpr uint32_t kSuspendNs = 1000000;  // 1 ms
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
         : "memory");
     return ok != 0;
 }
@@ -99,10 +104,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
         return true;
     const unsigned long long t0 = global_ns();
     while (true) {
-#pragma unroll 1
-        for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait(bar, parity))
-                return true;
+        if (mbar_try_wait(bar, parity))
+            return true;
         if (global_ns() - t0 > limit_ns)
             return false;
     }
@@ -146,9 +149,39 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
+// Warm L2 with one 2-D tensor-map box (a hint, like prefetch_l2).
+__device__ __forceinline__ void prefetch_tensor_l2(const CUtensorMap *map, int c0, int c1)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map),
+                 "r"(c0), "r"(c1)
+                 : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+
+// ------------------------------------------- programmatic dependent launch
+// Let the next kernel in the stream start its prologue on SMs this grid
+// frees (it still waits for this grid's results before touching them).
+__device__ __forceinline__ void pdl_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Wait until the grids this one depends on have completed and their memory
+// operations are visible (returns at once without such a dependency).
+__device__ __forceinline__ void pdl_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Warm L2 with a global byte range (16-byte aligned, size % 16 == 0).  Only a
+// hint: L2 is the point of coherence, so data written later is not hidden.
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 // ------------------------------------------------------------------ loads

@@ -83,6 +83,12 @@ cudaError_t launch_mxfp8_dequant(const uint8_t *Wq, const uint8_t *Ws, int N, in
                                  uint16_t *w_bf16, cudaStream_t stream);
 cudaError_t launch_wait_timeout_selftest(void *workspace, int limit_us, cudaStream_t stream);
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel of the stream drains (it calls griddepcontrol.wait
+// before touching anything that kernel could have written).
+cudaError_t launch_pdl(const void *fn, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       void **args);
+
 // Encodes tensor maps through the driver entry point (no libcuda link).
 bool encode_tensor_map_2d(void *map, int dtype_cu, const void *base, uint64_t inner,
                           uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,

@@ -26,6 +26,7 @@ constexpr int kWarps = 8;
 constexpr int kRing = 6;                  // stages per warp
 constexpr int kStage = 2048;              // one 16 x 128-byte box
 constexpr int kWarpSmem = kRing * kStage;
+constexpr int kMinUnits = 6;              // shortest run per warp
 
 struct Params {
     const uint16_t *X;       // bf16 [M][K]
@@ -36,18 +37,22 @@ struct Params {
     float *partial;          // [Wt][2][32][4*TT]
     int M, N, K;
     int upt;                 // units per n16 tile = ceil(K / 128)
-    long long units;
+    int units;
     int Wt;
+    int q, r;                // units = q * Wt + r: warps below r run q + 1 units, the rest q
 };
 
-__device__ __forceinline__ long long run_start(long long w, long long units, int Wt)
+// First unit of warp w's run.
+__device__ __forceinline__ int run_start(const Params &p, int w)
 {
-    return w * units / Wt;
+    return w * p.q + min(w, p.r);
 }
 
-__device__ __forceinline__ int warp_of_unit(long long u, long long units, int Wt)
+// The warp whose run contains unit u.
+__device__ __forceinline__ int warp_of_unit(const Params &p, int u)
 {
-    return (int)(((u + 1) * (long long)Wt - 1) / units);
+    const int big = p.r * (p.q + 1);
+    return u < big ? u / (p.q + 1) : p.r + (u - big) / p.q;
 }
 
 template <int TT>
@@ -66,39 +71,34 @@ __device__ __forceinline__ void store_tile_y(const Params &p, int nt, const floa
 }
 
 template <int TT>
-__device__ __noinline__ void flush_segment(const Params &p, int gw, int lane, long long nt,
-                                              long long seg_begin, long long seg_end,
-                                              long long run_begin, float (&acc)[TT][4])
+__device__ __forceinline__ void store_partial(const Params &p, int gw, int slot, int lane,
+                                              const float (&v)[TT][4])
 {
-    const int g = lane >> 2, t = lane & 3;
-    const long long tile_begin = nt * p.upt, tile_end = tile_begin + p.upt;
-    if (seg_begin == tile_begin && seg_end == tile_end) {
-        store_tile_y<TT>(p, (int)nt, acc, g, t);
-        return;
-    }
-    const int slot = (seg_begin == run_begin) ? 0 : 1;
     float *dst = p.partial + ((size_t)(gw * 2 + slot) * 32 + lane) * (4 * TT);
 #pragma unroll
     for (int tt = 0; tt < TT; ++tt)
         __stcg(reinterpret_cast<float4 *>(dst + 4 * tt),
-               make_float4(acc[tt][0], acc[tt][1], acc[tt][2], acc[tt][3]));
-    __syncwarp();
-    int old = 0;
-    if (lane == 0)
-        old = atomic_add_acq_rel(&p.counters[nt], 1);
-    old = __shfl_sync(0xffffffffu, old, 0);
-    const int w_first = warp_of_unit(tile_begin, p.units, p.Wt);
-    const int w_last = warp_of_unit(tile_end - 1, p.units, p.Wt);
-    if (old != w_last - w_first)
-        return;
+               make_float4(v[tt][0], v[tt][1], v[tt][2], v[tt][3]));
+}
+
+// Run by the last contributor of a cut tile: add every fragment of the tile
+// in warp order and write bf16 Y.
+template <int TT>
+__device__ __noinline__ void reduce_tile(const Params &p, int nt, int lane)
+{
+    const int g = lane >> 2, t = lane & 3;
+    const int tile_begin = nt * p.upt, tile_end = tile_begin + p.upt;
+    const int w_first = warp_of_unit(p, tile_begin);
+    const int w_last = warp_of_unit(p, tile_end - 1);
     float sum[TT][4];
 #pragma unroll
     for (int tt = 0; tt < TT; ++tt)
 #pragma unroll
         for (int e = 0; e < 4; ++e)
             sum[tt][e] = 0.f;
+#pragma unroll 4
     for (int w = w_first; w <= w_last; ++w) {
-        const int s = (run_start(w, p.units, p.Wt) >= tile_begin) ? 0 : 1;
+        const int s = (run_start(p, w) >= tile_begin) ? 0 : 1;
         const float *src = p.partial + ((size_t)(w * 2 + s) * 32 + lane) * (4 * TT);
 #pragma unroll
         for (int tt = 0; tt < TT; ++tt) {
@@ -109,7 +109,7 @@ __device__ __noinline__ void flush_segment(const Params &p, int gw, int lane, lo
             sum[tt][3] += f.w;
         }
     }
-    store_tile_y<TT>(p, (int)nt, sum, g, t);
+    store_tile_y<TT>(p, nt, sum, g, t);
     if (lane == 0)
         p.counters[nt] = 0;
 }
@@ -119,18 +119,18 @@ struct UnitScales {
     float a, b;
 };
 
-__device__ __forceinline__ UnitScales load_unit_scales(const Params &p, long long tile, int kb,
-                                                       int g, int t)
+__device__ __forceinline__ UnitScales load_unit_scales(const Params &p, int tile, int kb, int g,
+                                                       int t)
 {
     const int blocks = p.K / 32;
     const int blk = kb * 4 + t;
-    const long long ra = tile * 16 + g, rb = ra + 8;
+    const int ra = tile * 16 + g, rb = ra + 8;
     uint32_t ea = 127, eb = 127;  // any finite scale for zero-filled weights
     if (blk < blocks) {
         if (ra < p.N)
-            ea = __ldg(p.Ws + ra * blocks + blk);
+            ea = __ldg(p.Ws + (size_t)ra * blocks + blk);
         if (rb < p.N)
-            eb = __ldg(p.Ws + rb * blocks + blk);
+            eb = __ldg(p.Ws + (size_t)rb * blocks + blk);
     }
     return UnitScales{e8m0_to_f32(ea), e8m0_to_f32(eb)};
 }
@@ -145,21 +145,21 @@ __global__ void __launch_bounds__(kWarps * 32)
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gw = blockIdx.x * kWarps + warp;
+    pdl_launch_dependents();
     if (gw >= p.Wt)
         return;
     const int g = lane >> 2, t = lane & 3;
     uint8_t *ring = smem + (size_t)warp * kWarpSmem;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kWarps * kWarpSmem) + warp * kRing;
 
-    const long long u0 = run_start(gw, p.units, p.Wt);
-    const long long u1 = run_start(gw + 1, p.units, p.Wt);
-    const int nstages = (int)(u1 - u0);
-    long long tile = u0 / p.upt;
-    int kb = (int)(u0 - tile * p.upt);
+    const int u0 = run_start(p, gw);
+    const int u1 = run_start(p, gw + 1);
+    const int nstages = u1 - u0;
+    int tile = u0 / p.upt;
+    int kb = u0 - tile * p.upt;
 
     // lane 0 owns the ring; (itile, ikb) is the next unit to fetch
-    long long itile = tile;
-    int ikb = kb;
+    int itile = tile, ikb = kb;
     uint64_t policy = 0;
     if (lane == 0) {
         prefetch_tensormap(&wq_map);
@@ -168,9 +168,23 @@ __global__ void __launch_bounds__(kWarps * 32)
             mbar_init(&bars[s], 1);
         fence_barrier_init();
         policy = l2_policy_evict_first();
+        // while the previous kernel drains: pull the first units into L2
+        {
+            int pt = tile, pk = kb;
+            for (int s = 0; s < min(kRing, nstages); ++s) {
+                prefetch_tensor_l2(&wq_map, pk * 128, pt * 16);
+                if (++pk == p.upt) {
+                    pk = 0;
+                    ++pt;
+                }
+            }
+        }
+    }
+    pdl_wait();
+    if (lane == 0) {
         for (int s = 0; s < min(kRing, nstages); ++s) {
             mbar_arrive_expect_tx(&bars[s], kStage);
-            tma_load_2d(ring + s * kStage, &wq_map, ikb * 128, (int)itile * 16, &bars[s], policy);
+            tma_load_2d(ring + s * kStage, &wq_map, ikb * 128, itile * 16, &bars[s], policy);
             if (++ikb == p.upt) {
                 ikb = 0;
                 ++itile;
@@ -185,8 +199,10 @@ __global__ void __launch_bounds__(kWarps * 32)
 #pragma unroll
         for (int e = 0; e < 4; ++e)
             acc[tt][e] = 0.f;
+    bool first_cut = false;
+    int first_tile = 0;
+    int seg_begin = u0;
 
-    long long seg_begin = u0;
     const uint16_t *xrow[TT];
     bool xvalid[TT];
 #pragma unroll
@@ -196,25 +212,11 @@ __global__ void __launch_bounds__(kWarps * 32)
         xrow[tt] = p.X + (size_t)(xvalid[tt] ? m : 0) * p.K;
     }
     UnitScales sc_next = load_unit_scales(p, tile, kb, g, t);
-    const int c_lo = ((2 * t) ^ g) * 16, c_hi = ((2 * t + 1) ^ g) * 16;
-
-    for (int s = 0; s < nstages; ++s) {
-        const long long u = u0 + s;
-        const UnitScales sc = sc_next;
-        {
-            // scales of the next unit, one unit ahead
-            long long nt2 = tile;
-            int kb2 = kb + 1;
-            if (kb2 == p.upt) {
-                kb2 = 0;
-                ++nt2;
-            }
-            if (s + 1 < nstages)
-                sc_next = load_unit_scales(p, nt2, kb2, g, t);
-        }
-        const int kl = kb * 128 + t * 32;
+    // activation fragment of unit column kb: lane (g, t) takes k = 128 kb + 32t .. +31
+    constexpr bool kPipeX = TT <= 2;
+    auto load_x = [&](uint32_t (&dst)[TT][16], int kbx) {
+        const int kl = kbx * 128 + t * 32;
         const bool kvalid = kl < p.K;
-        uint32_t xb[TT][16];
 #pragma unroll
         for (int tt = 0; tt < TT; ++tt) {
 #pragma unroll
@@ -222,11 +224,38 @@ __global__ void __launch_bounds__(kWarps * 32)
                 uint4 v = make_uint4(0, 0, 0, 0);
                 if (xvalid[tt] && kvalid)
                     v = ldg128(xrow[tt] + kl + 8 * q);
-                xb[tt][4 * q + 0] = v.x;
-                xb[tt][4 * q + 1] = v.y;
-                xb[tt][4 * q + 2] = v.z;
-                xb[tt][4 * q + 3] = v.w;
+                dst[tt][4 * q + 0] = v.x;
+                dst[tt][4 * q + 1] = v.y;
+                dst[tt][4 * q + 2] = v.z;
+                dst[tt][4 * q + 3] = v.w;
             }
+        }
+    };
+    uint32_t xn[TT][16];
+    if (kPipeX)
+        load_x(xn, kb);
+    const int c_lo = ((2 * t) ^ g) * 16, c_hi = ((2 * t + 1) ^ g) * 16;
+
+    for (int s = 0; s < nstages; ++s) {
+        const int u = u0 + s;
+        const UnitScales sc = sc_next;
+        if (s + 1 < nstages) {
+            // scales of the next unit, one unit ahead
+            const bool wrap = kb + 1 == p.upt;
+            sc_next = load_unit_scales(p, wrap ? tile + 1 : tile, wrap ? 0 : kb + 1, g, t);
+        }
+        // activations of this unit (requested one unit ahead for narrow token tiles)
+        uint32_t xb[TT][16];
+        if (kPipeX) {
+#pragma unroll
+            for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    xb[tt][i] = xn[tt][i];
+            if (s + 1 < nstages)
+                load_x(xn, kb + 1 == p.upt ? 0 : kb + 1);
+        } else {
+            load_x(xb, kb);
         }
         const int slot = s % kRing;
         if (!mbar_wait(&bars[slot], (s / kRing) & 1, kWaitLimitNs)) {
@@ -252,19 +281,25 @@ __global__ void __launch_bounds__(kWarps * 32)
             for (int tt = 0; tt < TT; ++tt)
                 mma_bf16_16816(acc[tt], a0, a1, a2, a3, xb[tt][2 * j], xb[tt][2 * j + 1]);
         }
+        // every lane's reads of this slot have returned, so it can be refilled
         __syncwarp();
         if (lane == 0 && s + kRing < nstages) {
-            fence_proxy_async_smem();  // our reads of this slot precede the next copy into it
             mbar_arrive_expect_tx(&bars[slot], kStage);
-            tma_load_2d(ring + slot * kStage, &wq_map, ikb * 128, (int)itile * 16, &bars[slot],
-                        policy);
+            tma_load_2d(ring + slot * kStage, &wq_map, ikb * 128, itile * 16, &bars[slot], policy);
             if (++ikb == p.upt) {
                 ikb = 0;
                 ++itile;
             }
         }
         if (++kb == p.upt) {
-            flush_segment<TT>(p, gw, lane, tile, seg_begin, u + 1, u0, acc);
+            // a tile ends inside the run
+            if (seg_begin == tile * p.upt) {
+                store_tile_y<TT>(p, tile, acc, g, t);
+            } else {
+                store_partial<TT>(p, gw, 0, lane, acc);
+                first_cut = true;
+                first_tile = tile;
+            }
 #pragma unroll
             for (int tt = 0; tt < TT; ++tt)
 #pragma unroll
@@ -275,8 +310,35 @@ __global__ void __launch_bounds__(kWarps * 32)
             seg_begin = u + 1;
         }
     }
-    if (seg_begin < u1)
-        flush_segment<TT>(p, gw, lane, tile, seg_begin, u1, u0, acc);
+
+    // publish the cut segments (see the INT4 streaming kernel)
+    const bool last_cut = seg_begin < u1;
+    if (last_cut)
+        store_partial<TT>(p, gw, seg_begin == u0 ? 0 : 1, lane, acc);
+    if (!first_cut && !last_cut)
+        return;
+    __syncwarp();
+    int arrivals[2] = {0, 0};
+    if (lane == 0) {
+        if (first_cut)
+            arrivals[0] = atomic_add_acq_rel(&p.counters[first_tile], 1);
+        if (last_cut)
+            arrivals[1] = atomic_add_acq_rel(&p.counters[tile], 1);
+    }
+    arrivals[0] = __shfl_sync(0xffffffffu, arrivals[0], 0);
+    arrivals[1] = __shfl_sync(0xffffffffu, arrivals[1], 0);
+    if (first_cut) {
+        const int wf = warp_of_unit(p, first_tile * p.upt);
+        const int wl = warp_of_unit(p, first_tile * p.upt + p.upt - 1);
+        if (arrivals[0] == wl - wf)
+            reduce_tile<TT>(p, first_tile, lane);
+    }
+    if (last_cut) {
+        const int wf = warp_of_unit(p, tile * p.upt);
+        const int wl = warp_of_unit(p, tile * p.upt + p.upt - 1);
+        if (arrivals[1] == wl - wf)
+            reduce_tile<TT>(p, tile, lane);
+    }
 }
 
 const void *select_kernel(int tt)
@@ -309,6 +371,8 @@ bool plan_mxfp8_stream(int device, int M, int N, int K, StreamPlan *plan)
     if ((size_t)pl.ntiles > kMaxCounters)
         return false;
     pl.units = (long long)pl.ntiles * pl.upt;
+    if (pl.units > (1LL << 30))
+        return false;
     const void *fn = select_kernel(pl.tt);
     static int occ_cache[4] = {};
     int &occ = occ_cache[pl.tt - 1];
@@ -324,7 +388,8 @@ bool plan_mxfp8_stream(int device, int M, int N, int K, StreamPlan *plan)
         occ = o;
     }
     const long long max_warps = (long long)di.sms * occ * kWarps;
-    pl.Wt = (int)std::min<long long>(max_warps, pl.units);
+    // no run shorter than kMinUnits units (2 KB each)
+    pl.Wt = (int)std::max<long long>(1, std::min<long long>(max_warps, pl.units / kMinUnits));
     pl.grid = (pl.Wt + kWarps - 1) / kWarps;
     pl.partial_bytes = (size_t)pl.Wt * 2 * 32 * 4 * pl.tt * sizeof(float);
     *plan = pl;
@@ -354,10 +419,12 @@ cudaError_t launch_mxfp8_stream(const StreamPlan &pl, const void *X, const uint8
     p.N = N;
     p.K = K;
     p.upt = pl.upt;
-    p.units = pl.units;
+    p.units = (int)pl.units;
     p.Wt = pl.Wt;
+    p.q = (int)(pl.units / pl.Wt);
+    p.r = (int)(pl.units % pl.Wt);
     void *args[] = {&map, &p};
-    return cudaLaunchKernel(fn, dim3(pl.grid), dim3(kWarps * 32), args, pl.smem, stream);
+    return launch_pdl(fn, dim3(pl.grid), dim3(kWarps * 32), pl.smem, stream, args);
 }
 
 }  // namespace mxg

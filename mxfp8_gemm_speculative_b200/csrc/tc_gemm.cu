@@ -89,10 +89,12 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank)
     return r;
 }
 
+// Arrive on a barrier of either CTA of the pair.  What the waiter needs to
+// see is ordered by the tcgen05 fences around the hand-off, so the arrive
+// itself carries no cluster-scope release.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
 {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-                 : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 __device__ __forceinline__ void cluster_sync()
@@ -227,10 +229,8 @@ __device__ __forceinline__ bool role_wait(uint64_t *bar, uint32_t parity, volati
         return true;
     const unsigned long long t0 = global_ns();
     while (true) {
-#pragma unroll 1
-        for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait(bar, parity))
-                return true;
+        if (mbar_try_wait(bar, parity))
+            return true;
         if (*abort_flag)
             return false;
         if (global_ns() - t0 > kWaitLimitNs) {
@@ -246,15 +246,24 @@ __device__ __forceinline__ bool role_wait(uint64_t *bar, uint32_t parity, volati
 __device__ __forceinline__ void dequant_int4(const uint8_t *wp_slot, int q, int h, int lane, int G,
                                              int gpk, uint32_t (&v)[16])
 {
-    const int g = lane >> 2, t = lane & 3;
+    const int g = lane >> 2;
     const uint4 c = lds128(wp_slot + q * 1024 + h * 512 + lane * 16);
     const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+    // words 0-1 and 2-3 lie in one scale group each (the same one for G >= 64)
+    const uint8_t *sbase = wp_slot + 4096 + q * (64 * gpk) + g * 8 + h * 4;
+    const uint32_t sw0 = lds32(sbase);
+    const uint32_t sw1 = G == 32 ? lds32(sbase + 64) : sw0;
+    const ScaleSplit sa0 = split_scale((uint16_t)(sw0 & 0xFFFF));
+    const ScaleSplit sb0 = split_scale((uint16_t)(sw0 >> 16));
+    ScaleSplit sa1 = sa0, sb1 = sb0;
+    if (G == 32) {
+        sa1 = split_scale((uint16_t)(sw1 & 0xFFFF));
+        sb1 = split_scale((uint16_t)(sw1 >> 16));
+    }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        const int gi = (16 * j + 4 * t) / G;  // group inside the k-block
-        const uint32_t sw = lds32(wp_slot + 4096 + q * (64 * gpk) + gi * 64 + g * 8 + h * 4);
-        const ScaleSplit sa = split_scale((uint16_t)(sw & 0xFFFF));
-        const ScaleSplit sb = split_scale((uint16_t)(sw >> 16));
+        const ScaleSplit &sa = j < 2 ? sa0 : sa1;
+        const ScaleSplit &sb = j < 2 ? sb0 : sb1;
         v[4 * j + 0] = scale_pair_rn(int4_pair_minus8<0>(w[j]), sa);
         v[4 * j + 1] = scale_pair_rn(int4_pair_minus8<8>(w[j]), sa);
         v[4 * j + 2] = scale_pair_rn(int4_pair_minus8<4>(w[j]), sb);
@@ -302,6 +311,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();   // 0: issues the MMAs; 1: its pair
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    pdl_launch_dependents();
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kSX; ++i) {
@@ -323,9 +333,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     if (warp == kMmaWarp)
         tmem_alloc_pair(tmem_slot, kTmemCols);
+    if (threadIdx.x == 32 * kProducerWarp && pair < p.num_tiles) {
+        // while the previous kernel drains: pull the first k-blocks into L2
+        const int nb = pair / p.mtiles, mt = pair % p.mtiles;
+        const int n32 = (nb * 2 * BW + (int)rank * BW) / 32;
+        for (int kb = 0; kb < min(kSW, p.kblocks); ++kb) {
+            prefetch_tensor_l2(&x_map, kb * BK, mt * BT + (int)rank * (BT / 2));
+            if (F == kInt4)
+                prefetch_tensor_l2(&w_map, kb * 128, n32);
+            else
+                prefetch_tensor_l2(&w_map, kb * BK, n32 * 32);
+        }
+    }
     tc_fence_before();
     cluster_sync();   // barriers of both CTAs initialised, tensor memory allocated
     tc_fence_after();
+    pdl_wait();
     const uint32_t tmem_base = *tmem_slot;
 
     const int gpk = (F == kInt4) ? max(1, BK / p.G) : 1;  // scale groups per k-block
@@ -511,8 +534,7 @@ cudaError_t tc_launch(const TcPlan &pl, const CUtensorMap &xm, const CUtensorMap
     void *args[] = {const_cast<CUtensorMap *>(&xm), const_cast<CUtensorMap *>(&wm),
                     const_cast<CUtensorMap *>(&sm), &p};
     // the cluster shape (2, 1, 1) is part of the kernel
-    return cudaLaunchKernel(fn, dim3(pl.grid), dim3(kThreads), args, Layout<F, BT>::smem_bytes,
-                            stream);
+    return launch_pdl(fn, dim3(pl.grid), dim3(kThreads), Layout<F, BT>::smem_bytes, stream, args);
 }
 
 bool x_map(CUtensorMap *m, const void *X, int M, int K, int BT)

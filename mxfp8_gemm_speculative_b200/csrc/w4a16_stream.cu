@@ -68,23 +68,26 @@ struct Params {
     float *partial;          // [Wt][2][32][2*4*TT]
     int M, N, K;
     int upt;                 // units per n32 tile
-    long long units;
+    int units;
     int Wt;
+    int q, r;                // units = q * Wt + r: warps below r run q + 1 units, the rest q
 };
 
-__device__ __forceinline__ long long run_start(long long w, long long units, int Wt)
+// First unit of warp w's run.
+__device__ __forceinline__ int run_start(const Params &p, int w)
 {
-    return w * units / Wt;
+    return w * p.q + min(w, p.r);
 }
 
 // The warp whose run contains unit u.
-__device__ __forceinline__ int warp_of_unit(long long u, long long units, int Wt)
+__device__ __forceinline__ int warp_of_unit(const Params &p, int u)
 {
-    return (int)(((u + 1) * (long long)Wt - 1) / units);
+    const int big = p.r * (p.q + 1);   // units covered by the longer runs
+    return u < big ? u / (p.q + 1) : p.r + (u - big) / p.q;
 }
 
 template <int TT>
-__device__ __forceinline__ void store_tile_y(const Params &p, long long tile,
+__device__ __forceinline__ void store_tile_y(const Params &p, int tile,
                                              const float (&v)[2][TT][4], int g, int t)
 {
 #pragma unroll
@@ -94,7 +97,7 @@ __device__ __forceinline__ void store_tile_y(const Params &p, long long tile,
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int m = tt * 8 + 2 * t + (e & 1);
-                const long long n = tile * 32 + h * 16 + g + ((e & 2) ? 8 : 0);
+                const int n = tile * 32 + h * 16 + g + ((e & 2) ? 8 : 0);
                 if (m < p.M)
                     p.Y[(size_t)m * p.N + n] = f32_to_bf16_bits(v[h][tt][e]);
             }
@@ -116,12 +119,12 @@ __device__ __forceinline__ void store_partial(const Params &p, int gw, int slot,
 // Run by the last contributor of a cut tile: add every fragment of the tile
 // in warp order and write bf16 Y.
 template <int TT>
-__device__ __noinline__ void reduce_tile(const Params &p, long long tile, int lane)
+__device__ __noinline__ void reduce_tile(const Params &p, int tile, int lane)
 {
     const int g = lane >> 2, t = lane & 3;
-    const long long tile_begin = tile * p.upt, tile_end = tile_begin + p.upt;
-    const int w_first = warp_of_unit(tile_begin, p.units, p.Wt);
-    const int w_last = warp_of_unit(tile_end - 1, p.units, p.Wt);
+    const int tile_begin = tile * p.upt, tile_end = tile_begin + p.upt;
+    const int w_first = warp_of_unit(p, tile_begin);
+    const int w_last = warp_of_unit(p, tile_end - 1);
     float sum[2][TT][4];
 #pragma unroll
     for (int h = 0; h < 2; ++h)
@@ -132,7 +135,7 @@ __device__ __noinline__ void reduce_tile(const Params &p, long long tile, int la
                 sum[h][tt][e] = 0.f;
 #pragma unroll 4
     for (int w = w_first; w <= w_last; ++w) {
-        const int s = (run_start(w, p.units, p.Wt) >= tile_begin) ? 0 : 1;
+        const int s = (run_start(p, w) >= tile_begin) ? 0 : 1;
         const float *src = p.partial + ((size_t)(w * 2 + s) * 32 + lane) * (8 * TT);
 #pragma unroll
         for (int h = 0; h < 2; ++h)
@@ -163,12 +166,13 @@ __device__ __forceinline__ void zero_acc(float (&a)[2][TT][4])
 }
 
 template <int TT, int GM>
-__global__ void __launch_bounds__(kWarps * 32, TT == 1 ? 3 : 2) w4a16_stream_kernel(const Params p)
+__global__ void __launch_bounds__(kWarps * 32, 2) w4a16_stream_kernel(const Params p)
 {
     using MD = Mode<GM>;
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gw = blockIdx.x * kWarps + warp;
+    pdl_launch_dependents();
     if (gw >= p.Wt)
         return;  // the kernel has no CTA-wide barrier
     const int g = lane >> 2, t = lane & 3;
@@ -176,14 +180,14 @@ __global__ void __launch_bounds__(kWarps * 32, TT == 1 ? 3 : 2) w4a16_stream_ker
     uint8_t *ring = smem + (size_t)warp * kWarpSmem;
     uint64_t *bars = reinterpret_cast<uint64_t *>(ring + kRing * kStageBytes);
 
-    const long long u0 = run_start(gw, p.units, p.Wt);
-    const long long u1 = run_start(gw + 1, p.units, p.Wt);
-    const int nstages = (int)((u1 - u0 + MD::kUnitsPerStage - 1) / MD::kUnitsPerStage);
+    const int u0 = run_start(p, gw);
+    const int u1 = run_start(p, gw + 1);
+    const int nstages = (u1 - u0 + MD::kUnitsPerStage - 1) / MD::kUnitsPerStage;
 
     // lane 0 owns the ring: source pointers advance by one stage per issue
-    const uint8_t *csrc = p.codes + u0 * (MD::kChunks * 1024);
-    const uint8_t *ssrc = p.scales + u0 * (MD::kGroups * 64);
-    long long left = u1 - u0;  // units not yet requested
+    const uint8_t *csrc = p.codes + (size_t)u0 * (MD::kChunks * 1024);
+    const uint8_t *ssrc = p.scales + (size_t)u0 * (MD::kGroups * 64);
+    int left = u1 - u0;  // units not yet requested
     uint64_t policy = 0;
     if (lane == 0) {
 #pragma unroll
@@ -191,8 +195,17 @@ __global__ void __launch_bounds__(kWarps * 32, TT == 1 ? 3 : 2) w4a16_stream_ker
             mbar_init(&bars[s], 1);
         fence_barrier_init();
         policy = l2_policy_evict_first();
+        // while the previous kernel drains: pull the first stages into L2
+        {
+            const int nu = min(kRing * MD::kUnitsPerStage, left);
+            prefetch_l2(csrc, nu * MD::kChunks * 1024);
+            prefetch_l2(ssrc, nu * MD::kGroups * 64);
+        }
+    }
+    pdl_wait();
+    if (lane == 0) {
         for (int s = 0; s < min(kRing, nstages); ++s) {
-            const int nu = (int)min((long long)MD::kUnitsPerStage, left);
+            const int nu = min(MD::kUnitsPerStage, left);
             const uint32_t cb = nu * MD::kChunks * 1024, sb = nu * MD::kGroups * 64;
             uint8_t *dst = ring + s * kStageBytes;
             mbar_arrive_expect_tx(&bars[s], cb + sb);
@@ -219,36 +232,49 @@ __global__ void __launch_bounds__(kWarps * 32, TT == 1 ? 3 : 2) w4a16_stream_ker
     float acc[2][TT][4], part[2][TT][4];
     zero_acc<TT>(acc);
     bool first_cut = false;  // the run's first segment ended inside the run, cut
-    long long first_tile = 0;
+    int first_tile = 0;
 
-    long long tile = u0 / p.upt;
-    int lu = (int)(u0 - tile * p.upt);     // unit inside the tile
+    int tile = u0 / p.upt;
+    int lu = u0 - tile * p.upt;            // unit inside the tile
     const int kchunks = p.K / 64;
     int kc = lu * MD::kChunks;             // chunk inside the tile
-    long long seg_begin = u0;
+    int seg_begin = u0;
+
+    // Activation fragments of the stage's two chunks.  For narrow token tiles
+    // they are requested one stage ahead (a whole stage of work hides their
+    // L2 latency); wide token tiles load them per chunk.
+    constexpr bool kPipeX = TT <= 2;
+    auto inc = [&](int k) { return (k + 1 == kchunks) ? 0 : k + 1; };
+    uint2 xs[2][TT][4], xn[2][TT][4];
+    auto load_x = [&](uint2 (&dst)[2][TT][4], int slot_x, int chunk) {
+#pragma unroll
+        for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint2 v = make_uint2(0, 0);
+                if (xvalid[tt])
+                    v = __ldg(reinterpret_cast<const uint2 *>(xrow[tt] + chunk * 64 + 16 * j));
+                dst[slot_x][tt][j] = v;
+            }
+    };
+    if (kPipeX) {
+        load_x(xs, 0, kc);
+        load_x(xs, 1, inc(kc));
+    }
 
     for (int s = 0; s < nstages; ++s) {
         const int slot = s % kRing;
         const uint8_t *stage = ring + slot * kStageBytes;
-        // activations of the stage's two chunks, requested before the wait
-        // (they do not depend on the copy); wide token tiles load per chunk
-        constexpr int kXStage = TT <= 2 ? 2 : 1;
-        uint2 xs[kXStage][TT][4];
-        const int kc1 = (kc + 1 == kchunks) ? 0 : kc + 1;
-        auto load_x = [&](int slot_x, int chunk) {
-#pragma unroll
-            for (int tt = 0; tt < TT; ++tt)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    uint2 v = make_uint2(0, 0);
-                    if (xvalid[tt])
-                        v = __ldg(reinterpret_cast<const uint2 *>(xrow[tt] + chunk * 64 + 16 * j));
-                    xs[slot_x][tt][j] = v;
-                }
-        };
-        load_x(0, kc);
-        if (kXStage == 2)
-            load_x(kXStage - 1, kc1);
+        const int kc1 = inc(kc);
+        if (kPipeX) {
+            if (s + 1 < nstages) {
+                const int kn0 = inc(kc1);
+                load_x(xn, 0, kn0);
+                load_x(xn, 1, inc(kn0));
+            }
+        } else {
+            load_x(xs, 0, kc);
+        }
         if (!mbar_wait(&bars[slot], (s / kRing) & 1, kWaitLimitNs)) {
             if (lane == 0)
                 record_error(p.hdr, MXG_ERR_TIMEOUT, 100 + GM);
@@ -258,15 +284,15 @@ __global__ void __launch_bounds__(kWarps * 32, TT == 1 ? 3 : 2) w4a16_stream_ker
         }
 #pragma unroll
         for (int iu = 0; iu < MD::kUnitsPerStage; ++iu) {
-            const long long u = u0 + (long long)s * MD::kUnitsPerStage + iu;
+            const int u = u0 + s * MD::kUnitsPerStage + iu;
             if (iu > 0 && u >= u1)
                 break;
 #pragma unroll
             for (int ch = 0; ch < MD::kChunks; ++ch) {
                 const int c2 = iu * MD::kChunks + ch;  // chunk inside the stage
-                const int xi = kXStage == 2 ? c2 : 0;
-                if (kXStage == 1 && c2 == 1)
-                    load_x(0, kc1);
+                const int xi = kPipeX ? c2 : 0;
+                if (!kPipeX && c2 == 1)
+                    load_x(xs, 0, kc1);
                 const uint8_t *cp = stage + c2 * 1024 + lane * 16;
                 const uint4 wl = lds128(cp);
                 const uint4 wh = lds128(cp + 512);
@@ -330,11 +356,20 @@ __global__ void __launch_bounds__(kWarps * 32, TT == 1 ? 3 : 2) w4a16_stream_ker
                 seg_begin = u + 1;
             }
         }
+        if (kPipeX) {
+#pragma unroll
+            for (int c2 = 0; c2 < 2; ++c2)
+#pragma unroll
+                for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        xs[c2][tt][j] = xn[c2][tt][j];
+        }
         // every lane's reads of this slot have returned (their values are
         // consumed above), so the slot can be refilled
         __syncwarp();
         if (lane == 0 && left > 0) {
-            const int nu = (int)min((long long)MD::kUnitsPerStage, left);
+            const int nu = min(MD::kUnitsPerStage, left);
             const uint32_t cb = nu * MD::kChunks * 1024, sb = nu * MD::kGroups * 64;
             uint8_t *dst = ring + slot * kStageBytes;
             mbar_arrive_expect_tx(&bars[slot], cb + sb);
@@ -364,14 +399,14 @@ __global__ void __launch_bounds__(kWarps * 32, TT == 1 ? 3 : 2) w4a16_stream_ker
     arrivals[0] = __shfl_sync(0xffffffffu, arrivals[0], 0);
     arrivals[1] = __shfl_sync(0xffffffffu, arrivals[1], 0);
     if (first_cut) {
-        const int wf = warp_of_unit(first_tile * p.upt, p.units, p.Wt);
-        const int wl = warp_of_unit(first_tile * p.upt + p.upt - 1, p.units, p.Wt);
+        const int wf = warp_of_unit(p, first_tile * p.upt);
+        const int wl = warp_of_unit(p, first_tile * p.upt + p.upt - 1);
         if (arrivals[0] == wl - wf)
             reduce_tile<TT>(p, first_tile, lane);
     }
     if (last_cut) {
-        const int wf = warp_of_unit(tile * p.upt, p.units, p.Wt);
-        const int wl = warp_of_unit(tile * p.upt + p.upt - 1, p.units, p.Wt);
+        const int wf = warp_of_unit(p, tile * p.upt);
+        const int wl = warp_of_unit(p, tile * p.upt + p.upt - 1);
         if (arrivals[1] == wl - wf)
             reduce_tile<TT>(p, tile, lane);
     }
@@ -418,6 +453,8 @@ bool plan_w4a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan)
     if ((size_t)pl.ntiles > kMaxCounters)
         return false;
     pl.units = (long long)pl.ntiles * pl.upt;
+    if (pl.units > (1LL << 30))
+        return false;
     const void *fn = select_kernel(pl.tt, pl.variant);
     if (!fn)
         return false;
@@ -465,10 +502,12 @@ cudaError_t launch_w4a16_stream(const StreamPlan &pl, const void *X, const void 
     p.N = N;
     p.K = K;
     p.upt = pl.upt;
-    p.units = pl.units;
+    p.units = (int)pl.units;
     p.Wt = pl.Wt;
+    p.q = (int)(pl.units / pl.Wt);
+    p.r = (int)(pl.units % pl.Wt);
     void *args[] = {&p};
-    return cudaLaunchKernel(fn, dim3(pl.grid), dim3(kWarps * 32), args, pl.smem, stream);
+    return launch_pdl(fn, dim3(pl.grid), dim3(kWarps * 32), pl.smem, stream, args);
 }
 
 }  // namespace mxg
