@@ -107,6 +107,27 @@ MXG_API size_t w4a16_workspace_bytes(int M, int N, int K, int group_size);
 MXG_API int w4a16_gemm(const void *X, const void *packed, int M, int N, int K, int group_size,
                void *Y, void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* w4a16_gemm on the weight-streaming path without a caller workspace.  The
+ * source pages have no counterpart to this call: it exists for callers that
+ * cannot allocate a workspace (a plain C host with no device allocator of its
+ * own; a serving process whose device memory is reserved up front).  It
+ * allocates nothing: its scratch is one fixed 20 MiB array in device global
+ * memory, one per device and process, shared by every call of this entry
+ * point.
+ *   X, packed, Y, shape rules: as for w4a16_gemm, with 1 <= M <= 32 (else
+ *   MXG_ERR_UNSUPPORTED_SHAPE).  A shape whose partial sums and counters do
+ *   not fit the array returns MXG_ERR_WORKSPACE before any launch (on a
+ *   148-SM B200 every M <= 32 shape fits).
+ * The first call on a device does a one-time set-up with that device
+ * current: it looks the array up and zeroes its status word and counters on
+ * `stream`; make that first call before any stream capture.  Every completed
+ * call leaves the counters zero; the partial-sum scratch keeps the last
+ * call's contents.  Calls that are not ordered with respect to each other
+ * race on the array.  The status word of a timed-out wait stays inside the
+ * array (use w4a16_gemm with a workspace to read diagnostics). */
+MXG_API int w4a16_gemm_static_scratch(const void *X, const void *packed, int M, int N, int K,
+               int group_size, void *Y, cudaStream_t stream);
+
 /* ----------------------------------------------------------------- MXFP8 */
 
 /* Workspace bytes mxfp8_gemm needs for this shape on the current device. */

@@ -41,6 +41,7 @@ _SIGS = {
     "w4a16_repack": (_i, [_p, _p, _i, _i, _i, _p, _p]),
     "w4a16_workspace_bytes": (_sz, [_i, _i, _i, _i]),
     "w4a16_gemm": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _sz, _p]),
+    "w4a16_gemm_static_scratch": (_i, [_p, _p, _i, _i, _i, _i, _p, _p]),
     "mxfp8_workspace_bytes": (_sz, [_i, _i, _i]),
     "mxfp8_gemm": (_i, [_p, _p, _p, _i, _i, _i, _p, _p, _sz, _p]),
     "w4a16_unpack": (_i, [_p, _i, _i, _i, _p, _p, _p, _p]),
@@ -158,6 +159,22 @@ def w4a16_gemm(x: torch.Tensor, packed: torch.Tensor, N: int, K: int, group_size
     ws = workspace_buf if workspace_buf is not None else workspace(need, x.device, stream)
     _check(_lib.w4a16_gemm(_ptr(x), _ptr(packed), M, N, K, group_size, _ptr(out), _ptr(ws),
                            ws.numel(), _stream(stream)), "w4a16_gemm")
+    return out
+
+
+def w4a16_gemm_static_scratch(x: torch.Tensor, packed: torch.Tensor, N: int, K: int,
+                              group_size: int = 128, out: torch.Tensor | None = None,
+                              stream=None) -> torch.Tensor:
+    """w4a16_gemm (M <= 32) with the library's fixed device scratch instead of a workspace."""
+    _need(x, torch.bfloat16, "x")
+    M = x.shape[0]
+    if x.dim() != 2 or x.shape[1] != K:
+        raise ValueError("x must be [M][K]")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(out, torch.bfloat16, "out")
+    _check(_lib.w4a16_gemm_static_scratch(_ptr(x), _ptr(packed), M, N, K, group_size, _ptr(out),
+                                          _stream(stream)), "w4a16_gemm_static_scratch")
     return out
 
 
