@@ -147,7 +147,7 @@ def run_ours(args, rank, world, local_rank):
     # inputs: one seeded synthetic layer per shape (rank-dependent seed)
     step_bytes = sum(layer_weight_bytes(fmt, K, N, G) for K, N in layers)
     step_flops = sum(2 * M * N * K for K, N in layers)
-    pool = max(2, -(-3 * l2 // step_bytes))
+    pool = max(2, -(-int(args.pool_factor * l2) // step_bytes))
     xs, ys, weights, wss = [], [], [], []
     for li, (K, N) in enumerate(layers):
         if fmt == "int4":
@@ -197,8 +197,9 @@ def run_ours(args, rank, world, local_rank):
                     layer_call(li, p, stream)
             graphs.append(g)
     warmup, steps = args.warmup, args.steps
-    for i in range(warmup):
-        graphs[i % pool].replay()
+    with torch.cuda.stream(stream):          # replay() launches on the current stream
+        for i in range(warmup):
+            graphs[i % pool].replay()
     torch.cuda.synchronize(dev)
     status = max(abs(mxg.mxg_workspace_status(w)) for w in wss)
     if status:
@@ -212,10 +213,11 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-    t_start.record(stream)
-    for i in range(steps):
-        graphs[i % pool].replay()
-    t_end.record(stream)
+    with torch.cuda.stream(stream):
+        t_start.record(stream)
+        for i in range(steps):
+            graphs[i % pool].replay()
+        t_end.record(stream)
     torch.cuda.synchronize(dev)
     elapsed_ms = t_start.elapsed_time(t_end)
 
@@ -341,7 +343,8 @@ def run_ours(args, rank, world, local_rank):
             "format": fmt, "M": M, "layers_KxN": [f"{K}x{N}" for K, N in layers],
             "group_size": G if fmt == "int4" else 32,
             "weight_bytes_per_step": step_bytes, "flops_per_step": step_flops,
-            "l2": f"rotating weight pool of {pool} copies ({pool * step_bytes / 1e6:.0f} MB > 3 x L2)",
+            "l2": f"rotating weight pool of {pool} copies ({pool * step_bytes / 1e6:.0f} MB >= "
+                  f"{args.pool_factor:g} x L2)",
             "timing": "CUDA graphs of one step per pool slot, CUDA events on the launch stream; "
                       "kernel durations from a second live pass with an event pair around "
                       "each launch, queued behind a sleep kernel",
@@ -505,6 +508,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-budget", type=float, default=120.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pool-factor", type=float, default=3.0,
+                    help="rotating weight pool size in multiples of the L2 size")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

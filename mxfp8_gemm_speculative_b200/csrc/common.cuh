@@ -95,6 +95,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
+// Non-blocking probe: has the phase with the given parity completed?
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete; false after
 // `limit_ns` nanoseconds without completion.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
@@ -249,6 +263,19 @@ __device__ __forceinline__ void mma_bf16_16816_zero(float (&d)[4], uint32_t a0, 
 // publishes the caller's (and, after a warp barrier, its warp's) prior
 // stores and, for the last arriver, makes the other contributors' stores
 // visible.
+// Named barrier over `nthreads` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int *p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ int atomic_add_acq_rel(int *p, int v)
 {
     int old;
@@ -261,6 +288,15 @@ __device__ __forceinline__ int atomic_add_acq_rel(int *p, int v)
 // returned as the bf16 pair (q_lo - 8, q_hi - 8).  Exact: 0x4300 | q is the
 // bf16 value 128 + q (one unit in the last place is 1 at exponent 7), and
 // subtracting 136 leaves the small integer q - 8.
+// The same pair, returned as the bf16 pair (128 + q_lo, 128 + q_hi): one
+// mask-and-or, no arithmetic.  A product sum over such weights exceeds the
+// sum over (q - 8) by 136 times the sum of the activations.
+template <int S>
+__device__ __forceinline__ uint32_t int4_pair_plus128(uint32_t w)
+{
+    return ((w >> S) & 0x000F000Fu) | 0x43004300u;
+}
+
 template <int S>
 __device__ __forceinline__ uint32_t int4_pair_minus8(uint32_t w)
 {

@@ -3,26 +3,33 @@
 // At M <= 32 the layer reads each weight byte once and does 2*M flops per
 // weight: it is bound by HBM bytes of W.  The kernel therefore
 //  * cuts the re-packed weight stream into equal units (one n32 tile x one
-//    scale-group span of max(G, 64) rows of K) and gives every warp of a
-//    persistent grid one contiguous run of units (stream-K), so all SMs
-//    stream the same number of bytes; a run is one contiguous byte range of
-//    the re-packed buffer, and never shorter than a few stages;
-//  * moves each warp's run through its own ring of shared-memory stages
-//    with 1-D bulk copies (cp.async.bulk, completion on an mbarrier), four
-//    2 KB stages in flight per warp, weights marked evict-first in L2;
-//  * decodes nibbles to exact bf16 (q - 8) in registers (shift + lop3 and
-//    one bf16x2 add per two weights) and multiplies on the tensor cores
-//    with m16n8k16 MMAs where the weights are the 16-row operand and the
-//    tokens the 8-column operand ("swap AB"); the two n16 halves of a unit
-//    share each activation fragment;
+//    scale-group span of max(G, 64) rows of K) and gives every CTA of a
+//    persistent grid (one per SM) one contiguous run of units (stream-K at
+//    CTA granularity), so all SMs stream the same number of bytes;
+//  * the CTA's warps take the run's units in turn (unit i goes to warp
+//    i mod C), so every warp works on the same n32 tile at once and a warp
+//    the scheduler serves less only delays its own units;
+//  * each warp moves its units through its own ring of shared-memory slots
+//    with 1-D bulk copies (cp.async.bulk, completion on an mbarrier; codes
+//    and scales of a unit), several units ahead, weights marked evict-first
+//    in L2;
+//  * each warp decodes a pair of nibbles to the bf16 pair (128 + q) with one
+//    mask-and-or (plus a shift) and multiplies on the tensor cores with
+//    m16n8k16 MMAs where the weights are the 16-row operand and the tokens
+//    the 8-column operand ("swap AB"); the two n16 halves of a unit share
+//    each activation fragment, and one more MMA with an all-ones weight tile
+//    gives the per-token activation sum that turns (128 + q) into (q - 8);
 //  * starts a zero-initialised partial sum per scale group (every MMA step
-//    lies inside one group for G = 32, 64, 128) and adds partial * scale
-//    in fp32 once per group, so weights are never rounded;
-//  * n32 tiles covered whole by one warp are written directly; a tile cut
-//    between warps is reduced through the workspace: at the end of its run
-//    each contributor stores its fragment and bumps the tile's arrival
-//    counter (acquire-release), and the last one adds all fragments in warp
-//    order (deterministic) and writes bf16 Y.  Nobody waits on anybody.
+//    lies inside one group for G = 32, 64, 128) and adds
+//    (partial - 136 * activation sum) * scale in fp32 once per group, so
+//    weights are never rounded (every product is exact in fp32);
+//  * at the end of each tile every warp leaves its fragment in shared memory
+//    and goes on; the last warp to arrive adds the fragments.  A tile inside
+//    the CTA's run is written to Y at once.  A tile cut between CTAs is
+//    finished by the CTA holding its first unit, at the end of that CTA's
+//    run: the other contributors (for whom it is the first tile of the run)
+//    published their fragments early, so it adds them in CTA order
+//    (deterministic) and writes bf16 Y.
 #include <algorithm>
 
 #include "common.cuh"
@@ -31,22 +38,16 @@
 namespace mxg {
 namespace {
 
-constexpr int kWarps = 8;         // warps per CTA
-#ifndef MXG_STREAM_RING
-#define MXG_STREAM_RING 4
+#ifndef MXG_STREAM_CONSUMERS
+#define MXG_STREAM_CONSUMERS 12
 #endif
-#ifndef MXG_STREAM_MIN_STAGES
-#define MXG_STREAM_MIN_STAGES 6
+#ifndef MXG_STREAM_STAGES
+#define MXG_STREAM_STAGES 5
 #endif
-constexpr int kRing = MXG_STREAM_RING;          // stages per warp
-constexpr int kMinStages = MXG_STREAM_MIN_STAGES;  // shortest run, in stages
-constexpr int kStageCode = 2048;  // code bytes per stage (two k64 chunks of an n32 tile)
-constexpr int kStageScale = 256;  // scale bytes reserved per stage
-constexpr int kStageBytes = kStageCode + kStageScale;
-// per-warp ring: stages, then one mbarrier per stage; rounded so every
-// warp's ring (and every stage) starts 128-byte aligned
-constexpr int kWarpSmem = (kRing * kStageBytes + kRing * 8 + 127) / 128 * 128;
-static_assert(kStageBytes % 128 == 0, "stages must stay 128-byte aligned");
+constexpr int kConsumers = MXG_STREAM_CONSUMERS;  // warps per CTA
+constexpr int kThreads = kConsumers * 32;
+constexpr int kStages = MXG_STREAM_STAGES;       // ring slots per warp (one unit each)
+constexpr int kMinUnitsPerCta = 2 * kConsumers;  // shortest run
 
 // Group modes: 0 -> G = 128, 1 -> G = 64, 2 -> G = 32.
 template <int GM>
@@ -54,8 +55,27 @@ struct Mode {
     static constexpr int kG = GM == 0 ? 128 : (GM == 1 ? 64 : 32);
     static constexpr int kChunks = GM == 0 ? 2 : 1;          // k64 chunks per unit
     static constexpr int kGroups = GM == 2 ? 2 : 1;          // scale groups per unit
-    static constexpr int kUnitsPerStage = 2 / kChunks;
     static constexpr int kStepsPerGroup = kG / 16;            // MMA k16 steps per group
+    static constexpr int kCode = kChunks * 1024;              // code bytes per unit
+    static constexpr int kScale = kGroups * 64;               // scale bytes per unit
+};
+
+// Shared memory: every warp's ring of kStages slots (a slot holds one
+// unit's codes, then its scales), kRed reduction buffers of kConsumers
+// fragments (segment s of the run uses buffer s mod kRed), one mbarrier per
+// slot, then per reduction buffer an arrival count and a use count.
+template <int TT, int GM>
+struct Smem {
+    static constexpr int kFrag4 = 2 * TT * 32;                // float4 per warp fragment
+    static constexpr int kSlot = (Mode<GM>::kCode + Mode<GM>::kScale + 127) / 128 * 128;
+    static constexpr int kRed = TT <= 2 ? 4 : 2;
+    static constexpr size_t kRingBytes = (size_t)kConsumers * kStages * kSlot;
+    static constexpr size_t kRedBytes = (size_t)kRed * kConsumers * kFrag4 * 16;
+    static constexpr size_t kBarBytes = (size_t)kConsumers * kStages * 8;
+    static constexpr size_t kRedOff = kRingBytes;
+    static constexpr size_t kBarOff = kRedOff + kRedBytes;
+    static constexpr size_t kSyncOff = kBarOff + kBarBytes;
+    static constexpr size_t kTotal = kSyncOff + 2 * kRed * sizeof(int);
 };
 
 struct Params {
@@ -65,90 +85,110 @@ struct Params {
     uint16_t *Y;             // bf16 [M][N]
     WsHeader *hdr;
     int *counters;           // [N/32]
-    float *partial;          // [Wt][2][32][2*4*TT]
+    float4 *partial;         // [ctas][2*TT][32]: a CTA's fragment of its first, cut tile
     int M, N, K;
     int upt;                 // units per n32 tile
     int units;
-    int Wt;
-    int q, r;                // units = q * Wt + r: warps below r run q + 1 units, the rest q
+    int ctas;
+    int q, r;                // units = q * ctas + r: CTAs below r run q + 1 units, the rest q
 };
 
-// First unit of warp w's run.
-__device__ __forceinline__ int run_start(const Params &p, int w)
+// First unit of CTA c's run.
+__device__ __forceinline__ int run_start(const Params &p, int c)
 {
-    return w * p.q + min(w, p.r);
+    return c * p.q + min(c, p.r);
 }
 
-// The warp whose run contains unit u.
-__device__ __forceinline__ int warp_of_unit(const Params &p, int u)
+// The CTA whose run contains unit u.
+__device__ __forceinline__ int cta_of_unit(const Params &p, int u)
 {
     const int big = p.r * (p.q + 1);   // units covered by the longer runs
     return u < big ? u / (p.q + 1) : p.r + (u - big) / p.q;
 }
 
+// Writes the four outputs of fragment float4 j (= h * TT + tt) of `lane`.
 template <int TT>
-__device__ __forceinline__ void store_tile_y(const Params &p, int tile,
-                                             const float (&v)[2][TT][4], int g, int t)
+__device__ __forceinline__ void store_y4(const Params &p, int tile, int j, int lane, float4 v)
 {
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int tt = 0; tt < TT; ++tt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int m = tt * 8 + 2 * t + (e & 1);
-                const int n = tile * 32 + h * 16 + g + ((e & 2) ? 8 : 0);
-                if (m < p.M)
-                    p.Y[(size_t)m * p.N + n] = f32_to_bf16_bits(v[h][tt][e]);
-            }
-}
-
-template <int TT>
-__device__ __forceinline__ void store_partial(const Params &p, int gw, int slot, int lane,
-                                              const float (&v)[2][TT][4])
-{
-    float *dst = p.partial + ((size_t)(gw * 2 + slot) * 32 + lane) * (8 * TT);
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int tt = 0; tt < TT; ++tt)
-            __stcg(reinterpret_cast<float4 *>(dst + (h * TT + tt) * 4),
-                   make_float4(v[h][tt][0], v[h][tt][1], v[h][tt][2], v[h][tt][3]));
-}
-
-// Run by the last contributor of a cut tile: add every fragment of the tile
-// in warp order and write bf16 Y.
-template <int TT>
-__device__ __noinline__ void reduce_tile(const Params &p, int tile, int lane)
-{
+    const int h = j / TT, tt = j % TT;
     const int g = lane >> 2, t = lane & 3;
-    const int tile_begin = tile * p.upt, tile_end = tile_begin + p.upt;
-    const int w_first = warp_of_unit(p, tile_begin);
-    const int w_last = warp_of_unit(p, tile_end - 1);
-    float sum[2][TT][4];
+    const int m0 = tt * 8 + 2 * t;
+    const int n0 = tile * 32 + h * 16 + g;
+    const float e[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int tt = 0; tt < TT; ++tt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                sum[h][tt][e] = 0.f;
-#pragma unroll 4
-    for (int w = w_first; w <= w_last; ++w) {
-        const int s = (run_start(p, w) >= tile_begin) ? 0 : 1;
-        const float *src = p.partial + ((size_t)(w * 2 + s) * 32 + lane) * (8 * TT);
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int tt = 0; tt < TT; ++tt) {
-                const float4 f = ldcg_f4(src + (h * TT + tt) * 4);
-                sum[h][tt][0] += f.x;
-                sum[h][tt][1] += f.y;
-                sum[h][tt][2] += f.z;
-                sum[h][tt][3] += f.w;
-            }
+    for (int i = 0; i < 4; ++i) {
+        const int m = m0 + (i & 1);
+        const int n = n0 + ((i & 2) ? 8 : 0);
+        if (m < p.M)
+            p.Y[(size_t)m * p.N + n] = f32_to_bf16_bits(e[i]);
     }
-    store_tile_y<TT>(p, tile, sum, g, t);
+}
+
+// Run by warp 0 of a CTA whose segment of `tile` is cut (the tile goes on
+// in other CTAs' runs), with the CTA's warp fragments in `frags`.  The CTA
+// whose run holds the tile's first unit finishes that segment last in its
+// run: it adds the other contributors' fragments (in CTA order) to its own
+// and writes bf16 Y.  Every other contributor (its segment is the first one
+// of its run) publishes its fragment and bumps the tile's counter without
+// waiting for anybody.
+template <int TT>
+__device__ __noinline__ void finish_cut_tile(const Params &p, const float4 *frags, int c, int tile,
+                                             int lane)
+{
+    constexpr int F = 2 * TT;
+    constexpr int kFrag4 = F * 32;
+    float4 sum[F];
+#pragma unroll
+    for (int j = 0; j < F; ++j) {
+        sum[j] = frags[j * 32 + lane];
+        for (int w = 1; w < kConsumers; ++w) {
+            const float4 v = frags[w * kFrag4 + j * 32 + lane];
+            sum[j].x += v.x;
+            sum[j].y += v.y;
+            sum[j].z += v.z;
+            sum[j].w += v.w;
+        }
+    }
+    const int tile_begin = tile * p.upt;
+    const int c_first = cta_of_unit(p, tile_begin);
+    if (c != c_first) {
+#pragma unroll
+        for (int j = 0; j < F; ++j)
+            __stcg(p.partial + ((size_t)c * F + j) * 32 + lane, sum[j]);
+        __syncwarp();
+        if (lane == 0) {
+            __threadfence();
+            atomicAdd(&p.counters[tile], 1);
+        }
+        return;
+    }
+    const int c_last = cta_of_unit(p, tile_begin + p.upt - 1);
+    if (lane == 0) {
+        // the other contributors published early in their runs (or at their
+        // ends, for runs inside the tile); the wait is bounded
+        const unsigned long long t0 = global_ns();
+        while (ld_acquire_gpu(&p.counters[tile]) < c_last - c_first) {
+            if (global_ns() - t0 > kWaitLimitNs) {
+                record_error(p.hdr, MXG_ERR_TIMEOUT, 120);
+                break;
+            }
+            __nanosleep(64);
+        }
+    }
+    __syncwarp();
+    for (int cc = c_first + 1; cc <= c_last; ++cc) {
+#pragma unroll
+        for (int j = 0; j < F; ++j) {
+            const float4 f = __ldcg(p.partial + ((size_t)cc * F + j) * 32 + lane);
+            sum[j].x += f.x;
+            sum[j].y += f.y;
+            sum[j].z += f.z;
+            sum[j].w += f.w;
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < F; ++j)
+        store_y4<TT>(p, tile, j, lane, sum[j]);
     if (lane == 0)
         p.counters[tile] = 0;  // leave the counter zero for the next call
 }
@@ -165,59 +205,60 @@ __device__ __forceinline__ void zero_acc(float (&a)[2][TT][4])
                 a[h][tt][e] = 0.f;
 }
 
-template <int TT, int GM>
-__global__ void __launch_bounds__(kWarps * 32, 2) w4a16_stream_kernel(const Params p)
+// Copies unit u (codes, then scales) into a ring slot; completion on `bar`.
+template <int GM>
+__device__ __forceinline__ void fetch_unit(const Params &p, uint8_t *slot, uint64_t *bar, int u,
+                                           uint64_t policy)
 {
     using MD = Mode<GM>;
+    mbar_arrive_expect_tx(bar, MD::kCode + MD::kScale);
+    bulk_g2s(slot, p.codes + (size_t)u * MD::kCode, MD::kCode, bar, policy);
+    bulk_g2s(slot + MD::kCode, p.scales + (size_t)u * MD::kScale, MD::kScale, bar, policy);
+}
+
+template <int TT, int GM>
+__global__ void __launch_bounds__(kThreads, 1) w4a16_stream_kernel(const Params p)
+{
+    using MD = Mode<GM>;
+    using SL = Smem<TT, GM>;
+    constexpr int F = 2 * TT;  // float4 per lane fragment
     extern __shared__ __align__(128) uint8_t smem[];
+    float4 *red = reinterpret_cast<float4 *>(smem + SL::kRedOff);
+
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int gw = blockIdx.x * kWarps + warp;
     pdl_launch_dependents();
-    if (gw >= p.Wt)
-        return;  // the kernel has no CTA-wide barrier
-    const int g = lane >> 2, t = lane & 3;
-
-    uint8_t *ring = smem + (size_t)warp * kWarpSmem;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(ring + kRing * kStageBytes);
-
-    const int u0 = run_start(p, gw);
-    const int u1 = run_start(p, gw + 1);
-    const int nstages = (u1 - u0 + MD::kUnitsPerStage - 1) / MD::kUnitsPerStage;
-
-    // lane 0 owns the ring: source pointers advance by one stage per issue
-    const uint8_t *csrc = p.codes + (size_t)u0 * (MD::kChunks * 1024);
-    const uint8_t *ssrc = p.scales + (size_t)u0 * (MD::kGroups * 64);
-    int left = u1 - u0;  // units not yet requested
+    const int c = blockIdx.x;
+    const int U0 = run_start(p, c), U1 = run_start(p, c + 1);
+    const int n = U1 - U0;
+    uint8_t *ring = smem + (size_t)warp * kStages * SL::kSlot;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + SL::kBarOff) + warp * kStages;
     uint64_t policy = 0;
     if (lane == 0) {
-#pragma unroll
-        for (int s = 0; s < kRing; ++s)
-            mbar_init(&bars[s], 1);
+        for (int s = 0; s < kStages; ++s)
+            mbar_init(&full[s], 1);
         fence_barrier_init();
         policy = l2_policy_evict_first();
-        // while the previous kernel drains: pull the first stages into L2
-        {
-            const int nu = min(kRing * MD::kUnitsPerStage, left);
-            prefetch_l2(csrc, nu * MD::kChunks * 1024);
-            prefetch_l2(ssrc, nu * MD::kGroups * 64);
-        }
     }
+    int *red_count = reinterpret_cast<int *>(smem + SL::kSyncOff);  // arrivals per buffer
+    int *red_done = red_count + SL::kRed;                           // reductions per buffer
+    if (threadIdx.x == 0) {
+        for (int b = 0; b < 2 * SL::kRed; ++b)
+            red_count[b] = 0;
+        // while the previous kernel drains: pull the first units into L2
+        const int nu = min(kConsumers * kStages, n);
+        prefetch_l2(p.codes + (size_t)U0 * MD::kCode, nu * MD::kCode);
+        prefetch_l2(p.scales + (size_t)U0 * MD::kScale, nu * MD::kScale);
+    }
+    __syncthreads();
     pdl_wait();
-    if (lane == 0) {
-        for (int s = 0; s < min(kRing, nstages); ++s) {
-            const int nu = min(MD::kUnitsPerStage, left);
-            const uint32_t cb = nu * MD::kChunks * 1024, sb = nu * MD::kGroups * 64;
-            uint8_t *dst = ring + s * kStageBytes;
-            mbar_arrive_expect_tx(&bars[s], cb + sb);
-            bulk_g2s(dst, csrc, cb, &bars[s], policy);
-            bulk_g2s(dst + kStageCode, ssrc, sb, &bars[s], policy);
-            csrc += cb;
-            ssrc += sb;
-            left -= nu;
-        }
-    }
-    __syncwarp();
+    // this warp takes units warp, warp + C, ... of the run; its k-th unit
+    // goes to slot k mod kStages
+    if (lane == 0)
+        for (int k = 0; k < kStages && warp + k * kConsumers < n; ++k)
+            fetch_unit<GM>(p, ring + k * SL::kSlot, &full[k], U0 + warp + k * kConsumers, policy);
 
+    // ------------------------------------------------------------ consumers
+    const int g = lane >> 2, t = lane & 3;
     // activation rows of this lane: m = g + 8 tt; the lane reads k = 4t .. 4t+3
     // of every k16 step
     const uint16_t *xrow[TT];
@@ -228,72 +269,60 @@ __global__ void __launch_bounds__(kWarps * 32, 2) w4a16_stream_kernel(const Para
         xvalid[tt] = m < p.M;
         xrow[tt] = p.X + (size_t)(xvalid[tt] ? m : 0) * p.K + 4 * t;
     }
+    const int upt = p.upt;
 
-    float acc[2][TT][4], part[2][TT][4];
-    zero_acc<TT>(acc);
-    bool first_cut = false;  // the run's first segment ended inside the run, cut
-    int first_tile = 0;
-
-    int tile = u0 / p.upt;
-    int lu = u0 - tile * p.upt;            // unit inside the tile
-    const int kchunks = p.K / 64;
-    int kc = lu * MD::kChunks;             // chunk inside the tile
-    int seg_begin = u0;
-
-    // Activation fragments of the stage's two chunks.  For narrow token tiles
-    // they are requested one stage ahead (a whole stage of work hides their
-    // L2 latency); wide token tiles load them per chunk.
+    // Activation fragments of one unit, requested one unit ahead for narrow
+    // token tiles (a whole unit of work hides their L2 latency).
     constexpr bool kPipeX = TT <= 2;
-    auto inc = [&](int k) { return (k + 1 == kchunks) ? 0 : k + 1; };
-    uint2 xs[2][TT][4], xn[2][TT][4];
-    auto load_x = [&](uint2 (&dst)[2][TT][4], int slot_x, int chunk) {
+    uint2 xs[MD::kChunks][TT][4], xn[MD::kChunks][TT][4];
+    auto load_x = [&](uint2 (&dst)[MD::kChunks][TT][4], int u) {
+        const int kc = (u % upt) * MD::kChunks;  // first k64 chunk of unit u
 #pragma unroll
-        for (int tt = 0; tt < TT; ++tt)
+        for (int ch = 0; ch < MD::kChunks; ++ch)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                uint2 v = make_uint2(0, 0);
-                if (xvalid[tt])
-                    v = __ldg(reinterpret_cast<const uint2 *>(xrow[tt] + chunk * 64 + 16 * j));
-                dst[slot_x][tt][j] = v;
-            }
+            for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint2 v = make_uint2(0, 0);
+                    if (xvalid[tt])
+                        v = __ldg(reinterpret_cast<const uint2 *>(xrow[tt] + (kc + ch) * 64 +
+                                                                  16 * j));
+                    dst[ch][tt][j] = v;
+                }
     };
-    if (kPipeX) {
-        load_x(xs, 0, kc);
-        load_x(xs, 1, inc(kc));
-    }
 
-    for (int s = 0; s < nstages; ++s) {
-        const int slot = s % kRing;
-        const uint8_t *stage = ring + slot * kStageBytes;
-        const int kc1 = inc(kc);
-        if (kPipeX) {
-            if (s + 1 < nstages) {
-                const int kn0 = inc(kc1);
-                load_x(xn, 0, kn0);
-                load_x(xn, 1, inc(kn0));
+    constexpr uint32_t kOnes = 0x3F803F80u;  // bf16 pair (1, 1)
+    float acc[2][TT][4], part[2][TT][4], xsum[TT][4];
+    bool ok = true;
+    int i = warp;          // run index of this warp's next unit
+    int slot = 0;          // ring slot of unit i
+    uint32_t phase = 0;    // parity of the phase of unit i
+    if (kPipeX && i < n)
+        load_x(xs, U0 + i);
+    int sidx = 0;          // segment of the run
+    int tile = U0 / upt;
+    for (int seg = U0; seg < U1; ++tile) {
+        const int tile_begin = tile * upt;
+        const int seg_end = min(U1, tile_begin + upt);
+        zero_acc<TT>(acc);
+        for (; U0 + i < seg_end; i += kConsumers) {
+            const int u = U0 + i;
+            if (kPipeX) {
+                if (i + kConsumers < n)
+                    load_x(xn, u + kConsumers);
+            } else {
+                load_x(xs, u);
             }
-        } else {
-            load_x(xs, 0, kc);
-        }
-        if (!mbar_wait(&bars[slot], (s / kRing) & 1, kWaitLimitNs)) {
-            if (lane == 0)
-                record_error(p.hdr, MXG_ERR_TIMEOUT, 100 + GM);
-            for (int r = s + 1; r < min(s + kRing, nstages); ++r)
-                mbar_wait(&bars[r % kRing], (r / kRing) & 1, kWaitLimitNs / 16);
-            return;
-        }
-#pragma unroll
-        for (int iu = 0; iu < MD::kUnitsPerStage; ++iu) {
-            const int u = u0 + s * MD::kUnitsPerStage + iu;
-            if (iu > 0 && u >= u1)
-                break;
+            if (!mbar_wait(&full[slot], phase, ok ? kWaitLimitNs : 0)) {
+                if (ok && lane == 0)
+                    record_error(p.hdr, MXG_ERR_TIMEOUT, 100 + GM);
+                ok = false;
+            }
+            const uint8_t *st = ring + slot * SL::kSlot;
+            const uint8_t *ss = st + MD::kCode;
 #pragma unroll
             for (int ch = 0; ch < MD::kChunks; ++ch) {
-                const int c2 = iu * MD::kChunks + ch;  // chunk inside the stage
-                const int xi = kPipeX ? c2 : 0;
-                if (!kPipeX && c2 == 1)
-                    load_x(xs, 0, kc1);
-                const uint8_t *cp = stage + c2 * 1024 + lane * 16;
+                const uint8_t *cp = st + ch * 1024 + lane * 16;
                 const uint4 wl = lds128(cp);
                 const uint4 wh = lds128(cp + 512);
                 const uint32_t w[2][4] = {{wl.x, wl.y, wl.z, wl.w}, {wh.x, wh.y, wh.z, wh.w}};
@@ -302,113 +331,137 @@ __global__ void __launch_bounds__(kWarps * 32, 2) w4a16_stream_kernel(const Para
                     const int step = ch * 4 + j;  // k16 step inside the unit
                     const bool first = (step % MD::kStepsPerGroup) == 0;
 #pragma unroll
+                    for (int tt = 0; tt < TT; ++tt) {
+                        // per token: the sum of the step's activations (an MMA
+                        // with an all-ones weight tile)
+                        if (first)
+                            mma_bf16_16816_zero(xsum[tt], kOnes, kOnes, kOnes, kOnes,
+                                                xs[ch][tt][j].x, xs[ch][tt][j].y);
+                        else
+                            mma_bf16_16816(xsum[tt], kOnes, kOnes, kOnes, kOnes,
+                                           xs[ch][tt][j].x, xs[ch][tt][j].y);
+                    }
+#pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        const uint32_t a0 = int4_pair_minus8<0>(w[h][j]);
-                        const uint32_t a1 = int4_pair_minus8<4>(w[h][j]);
-                        const uint32_t a2 = int4_pair_minus8<8>(w[h][j]);
-                        const uint32_t a3 = int4_pair_minus8<12>(w[h][j]);
+                        const uint32_t a0 = int4_pair_plus128<0>(w[h][j]);
+                        const uint32_t a1 = int4_pair_plus128<4>(w[h][j]);
+                        const uint32_t a2 = int4_pair_plus128<8>(w[h][j]);
+                        const uint32_t a3 = int4_pair_plus128<12>(w[h][j]);
 #pragma unroll
                         for (int tt = 0; tt < TT; ++tt) {
                             if (first)
                                 mma_bf16_16816_zero(part[h][tt], a0, a1, a2, a3,
-                                                    xs[xi][tt][j].x, xs[xi][tt][j].y);
+                                                    xs[ch][tt][j].x, xs[ch][tt][j].y);
                             else
-                                mma_bf16_16816(part[h][tt], a0, a1, a2, a3, xs[xi][tt][j].x,
-                                               xs[xi][tt][j].y);
+                                mma_bf16_16816(part[h][tt], a0, a1, a2, a3, xs[ch][tt][j].x,
+                                               xs[ch][tt][j].y);
                         }
                     }
                     if ((step + 1) % MD::kStepsPerGroup == 0) {
-                        // end of a scale group: acc += part * scale (fp32)
+                        // end of a scale group: the MMAs summed (128 + q) * x, so
+                        // acc += (part - 136 * sum(x)) * scale, in fp32
                         const int gi = step / MD::kStepsPerGroup;  // group inside the unit
-                        const uint2 sv =
-                            lds64(stage + kStageCode + (iu * MD::kGroups + gi) * 64 + g * 8);
+                        const uint2 sv = lds64(ss + gi * 64 + g * 8);
                         const float2 s01 = __half22float2(*reinterpret_cast<const __half2 *>(&sv.x));
                         const float2 s23 = __half22float2(*reinterpret_cast<const __half2 *>(&sv.y));
+                        const float sc[2][2] = {{s01.x, s01.y}, {s23.x, s23.y}};
 #pragma unroll
-                        for (int tt = 0; tt < TT; ++tt) {
-                            acc[0][tt][0] = fmaf(part[0][tt][0], s01.x, acc[0][tt][0]);
-                            acc[0][tt][1] = fmaf(part[0][tt][1], s01.x, acc[0][tt][1]);
-                            acc[0][tt][2] = fmaf(part[0][tt][2], s01.y, acc[0][tt][2]);
-                            acc[0][tt][3] = fmaf(part[0][tt][3], s01.y, acc[0][tt][3]);
-                            acc[1][tt][0] = fmaf(part[1][tt][0], s23.x, acc[1][tt][0]);
-                            acc[1][tt][1] = fmaf(part[1][tt][1], s23.x, acc[1][tt][1]);
-                            acc[1][tt][2] = fmaf(part[1][tt][2], s23.y, acc[1][tt][2]);
-                            acc[1][tt][3] = fmaf(part[1][tt][3], s23.y, acc[1][tt][3]);
-                        }
+                        for (int h = 0; h < 2; ++h)
+#pragma unroll
+                            for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    // outputs e and e ^ 2 are rows g, g + 8 of token 2t + (e & 1)
+                                    const float v = fmaf(-136.f, xsum[tt][e & 1], part[h][tt][e]);
+                                    acc[h][tt][e] = fmaf(v, sc[h][e >> 1], acc[h][tt][e]);
+                                }
                     }
                 }
-                kc = (kc + 1 == kchunks) ? 0 : kc + 1;
             }
-            if (++lu == p.upt) {
-                // a tile ends inside the run
-                if (seg_begin == tile * p.upt) {
-                    store_tile_y<TT>(p, tile, acc, g, t);   // whole tile: write it now
-                } else {
-                    // the run's first segment, cut: park it in slot 0 now, announce it
-                    // at the end of the run
-                    store_partial<TT>(p, gw, 0, lane, acc);
-                    first_cut = true;
-                    first_tile = tile;
-                }
-                zero_acc<TT>(acc);
-                ++tile;
-                lu = 0;
-                seg_begin = u + 1;
+            // every lane's reads of the slot have returned (their values are
+            // consumed above): refill it with this warp's unit kStages ahead
+            __syncwarp();
+            if (lane == 0 && i + kStages * kConsumers < n)
+                fetch_unit<GM>(p, ring + slot * SL::kSlot, &full[slot],
+                               u + kStages * kConsumers, policy);
+            if (kPipeX) {
+#pragma unroll
+                for (int ch = 0; ch < MD::kChunks; ++ch)
+#pragma unroll
+                    for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            xs[ch][tt][j] = xn[ch][tt][j];
+            }
+            if (++slot == kStages) {
+                slot = 0;
+                phase ^= 1;
             }
         }
-        if (kPipeX) {
-#pragma unroll
-            for (int c2 = 0; c2 < 2; ++c2)
-#pragma unroll
-                for (int tt = 0; tt < TT; ++tt)
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        xs[c2][tt][j] = xn[c2][tt][j];
-        }
-        // every lane's reads of this slot have returned (their values are
-        // consumed above), so the slot can be refilled
-        __syncwarp();
-        if (lane == 0 && left > 0) {
-            const int nu = min(MD::kUnitsPerStage, left);
-            const uint32_t cb = nu * MD::kChunks * 1024, sb = nu * MD::kGroups * 64;
-            uint8_t *dst = ring + slot * kStageBytes;
-            mbar_arrive_expect_tx(&bars[slot], cb + sb);
-            bulk_g2s(dst, csrc, cb, &bars[slot], policy);
-            bulk_g2s(dst + kStageCode, ssrc, sb, &bars[slot], policy);
-            csrc += cb;
-            ssrc += sb;
-            left -= nu;
-        }
-    }
 
-    // publish the cut segments: the first one (slot 0) and the last one
-    // (slot 0 if it is also the first segment of the run, else slot 1)
-    const bool last_cut = seg_begin < u1;
-    if (last_cut)
-        store_partial<TT>(p, gw, seg_begin == u0 ? 0 : 1, lane, acc);
-    if (!first_cut && !last_cut)
-        return;
-    __syncwarp();
-    int arrivals[2] = {0, 0};
-    if (lane == 0) {
-        if (first_cut)
-            arrivals[0] = atomic_add_acq_rel(&p.counters[first_tile], 1);
-        if (last_cut)
-            arrivals[1] = atomic_add_acq_rel(&p.counters[tile], 1);
-    }
-    arrivals[0] = __shfl_sync(0xffffffffu, arrivals[0], 0);
-    arrivals[1] = __shfl_sync(0xffffffffu, arrivals[1], 0);
-    if (first_cut) {
-        const int wf = warp_of_unit(p, first_tile * p.upt);
-        const int wl = warp_of_unit(p, first_tile * p.upt + p.upt - 1);
-        if (arrivals[0] == wl - wf)
-            reduce_tile<TT>(p, first_tile, lane);
-    }
-    if (last_cut) {
-        const int wf = warp_of_unit(p, tile * p.upt);
-        const int wl = warp_of_unit(p, tile * p.upt + p.upt - 1);
-        if (arrivals[1] == wl - wf)
-            reduce_tile<TT>(p, tile, lane);
+        // ---- end of the tile segment.  Every warp leaves its fragment in the
+        // segment's reduction buffer and goes on; the last warp to arrive adds
+        // the fragments.  A buffer is reused kRed segments later, once the
+        // reduction of its previous segment is done.
+        const int rb = sidx % SL::kRed;
+        const int uses = sidx / SL::kRed;  // earlier segments that used buffer rb
+        if (uses > 0) {
+            if (lane == 0) {
+                const unsigned long long t0 = global_ns();
+                while (*reinterpret_cast<volatile int *>(&red_done[rb]) < uses) {
+                    if (global_ns() - t0 > kWaitLimitNs) {
+                        record_error(p.hdr, MXG_ERR_TIMEOUT, 130);
+                        break;
+                    }
+                    __nanosleep(32);
+                }
+                __threadfence_block();
+            }
+            __syncwarp();
+        }
+        float4 *frags = red + (size_t)rb * kConsumers * SL::kFrag4;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int tt = 0; tt < TT; ++tt)
+                frags[(size_t)warp * SL::kFrag4 + (h * TT + tt) * 32 + lane] =
+                    make_float4(acc[h][tt][0], acc[h][tt][1], acc[h][tt][2], acc[h][tt][3]);
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+            __threadfence_block();
+            last = atomicAdd(&red_count[rb], 1) == kConsumers - 1;
+            __threadfence_block();
+        }
+        if (__shfl_sync(0xffffffffu, last, 0)) {
+            if (lane == 0)
+                red_count[rb] = 0;
+            const bool whole = seg == tile_begin && seg_end == tile_begin + upt;
+            if (whole) {
+#pragma unroll
+                for (int j = 0; j < F; ++j) {
+                    float4 s = frags[j * 32 + lane];
+#pragma unroll
+                    for (int w = 1; w < kConsumers; ++w) {
+                        const float4 v = frags[(size_t)w * SL::kFrag4 + j * 32 + lane];
+                        s.x += v.x;
+                        s.y += v.y;
+                        s.z += v.z;
+                        s.w += v.w;
+                    }
+                    store_y4<TT>(p, tile, j, lane, s);
+                }
+            } else {
+                finish_cut_tile<TT>(p, frags, c, tile, lane);
+            }
+            __syncwarp();
+            if (lane == 0) {
+                __threadfence_block();
+                atomicAdd(&red_done[rb], 1);
+            }
+        }
+        ++sidx;
+        seg = seg_end;
     }
 }
 
@@ -430,6 +483,22 @@ const void *select_kernel(int tt, int gm)
     return nullptr;
 }
 
+template <int GM>
+size_t smem_bytes_gm(int tt)
+{
+    switch (tt) {
+    case 1: return Smem<1, GM>::kTotal;
+    case 2: return Smem<2, GM>::kTotal;
+    case 3: return Smem<3, GM>::kTotal;
+    default: return Smem<4, GM>::kTotal;
+    }
+}
+
+size_t smem_bytes(int tt, int gm)
+{
+    return gm == 0 ? smem_bytes_gm<0>(tt) : gm == 1 ? smem_bytes_gm<1>(tt) : smem_bytes_gm<2>(tt);
+}
+
 int group_mode(int G)
 {
     return G == 128 ? 0 : (G == 64 ? 1 : 2);
@@ -445,8 +514,10 @@ bool plan_w4a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan)
     StreamPlan pl{};
     pl.tt = (M + 7) / 8;
     pl.variant = group_mode(G);
-    pl.warps_per_cta = kWarps;
-    pl.smem = (size_t)kWarps * kWarpSmem;
+    pl.warps_per_cta = kConsumers;
+    pl.smem = smem_bytes(pl.tt, pl.variant);
+    if ((int)pl.smem > di.smem_optin)
+        return false;
     const int unit_k = std::max(G, 64);
     pl.upt = K / unit_k;
     pl.ntiles = N / 32;
@@ -458,26 +529,17 @@ bool plan_w4a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan)
     const void *fn = select_kernel(pl.tt, pl.variant);
     if (!fn)
         return false;
-    static int occ_cache[4][3] = {};
-    int &occ = occ_cache[pl.tt - 1][pl.variant];
-    if (occ == 0) {
+    static bool attr_set[4][3] = {};
+    if (!attr_set[pl.tt - 1][pl.variant]) {
         if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem) !=
             cudaSuccess)
             return false;
-        int o = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, fn, kWarps * 32, pl.smem) !=
-                cudaSuccess ||
-            o < 1)
-            return false;
-        occ = o;
+        attr_set[pl.tt - 1][pl.variant] = true;
     }
-    // enough warps to fill the GPU, but no run shorter than kMinStages stages
-    const int units_per_stage = 2 / (unit_k / 64);
-    const long long min_units = (long long)kMinStages * units_per_stage;
-    const long long max_warps = (long long)di.sms * occ * kWarps;
-    pl.Wt = (int)std::max<long long>(1, std::min<long long>(max_warps, pl.units / min_units));
-    pl.grid = (pl.Wt + kWarps - 1) / kWarps;
-    pl.partial_bytes = (size_t)pl.Wt * 2 * 32 * 2 * 4 * pl.tt * sizeof(float);
+    // one CTA per SM, but no run shorter than kMinUnitsPerCta units
+    pl.Wt = (int)std::max<long long>(1, std::min<long long>(di.sms, pl.units / kMinUnitsPerCta));
+    pl.grid = pl.Wt;
+    pl.partial_bytes = (size_t)pl.Wt * (2 * pl.tt * 32) * sizeof(float4);
     *plan = pl;
     return true;
 }
@@ -497,17 +559,17 @@ cudaError_t launch_w4a16_stream(const StreamPlan &pl, const void *X, const void 
     p.Y = static_cast<uint16_t *>(Y);
     p.hdr = static_cast<WsHeader *>(workspace);
     p.counters = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + wm.counters_off);
-    p.partial = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + wm.partial_off);
+    p.partial = reinterpret_cast<float4 *>(static_cast<uint8_t *>(workspace) + wm.partial_off);
     p.M = M;
     p.N = N;
     p.K = K;
     p.upt = pl.upt;
     p.units = (int)pl.units;
-    p.Wt = pl.Wt;
+    p.ctas = pl.Wt;
     p.q = (int)(pl.units / pl.Wt);
     p.r = (int)(pl.units % pl.Wt);
     void *args[] = {&p};
-    return launch_pdl(fn, dim3(pl.grid), dim3(kWarps * 32), pl.smem, stream, args);
+    return launch_pdl(fn, dim3(pl.grid), dim3(kThreads), pl.smem, stream, args);
 }
 
 }  // namespace mxg

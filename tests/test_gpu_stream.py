@@ -116,11 +116,16 @@ def test_int4_stream_exact_integer_regime(mxg, M, G):
 
 
 def test_int4_identity_is_exact(mxg):
+    """W = identity / 8 with small-integer activations: every product and
+    every partial sum of the weight-streaming path is exact in fp32, so Y is
+    X / 8 bit for bit (no weight is rounded anywhere on the path)."""
     K = N = 512
     codes = np.full((N, K), 8, dtype=np.uint8)
     np.fill_diagonal(codes, 9)
     sc = np.full((K // 128, N), 0x3000, dtype=np.uint16)   # 2^-3
-    X = synth.int4_layer(7, K, N, 128, seed=1).X
+    rng = np.random.default_rng(np.random.SeedSequence([1, 7]))
+    xi = rng.integers(-8, 9, size=(7, K)).astype(np.float32)
+    X = (torch.from_numpy(xi).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
     lay = synth.Int4Layer(7, K, N, 128, X, codes, synth.pack_codes_gptq(codes), sc)
     y, _ = run_int4(mxg, lay, path=1)
     xin = torch.from_numpy(X.view(np.int16)).view(torch.bfloat16).float() * 0.125
