@@ -79,8 +79,9 @@ MXG_API size_t w4a16_packed_bytes(int K, int N, int group_size);
  *   scales   device, fp16 bits [K/G][N].
  *   packed   device, caller-allocated, w4a16_packed_bytes(K, N, G) bytes.
  * Layout written (private to this library, stable for a given K, N, G):
- * codes as [N/16][K/64][32 lanes][16 B] so that one 16-byte load is one
- * lane's mma fragment for four k16 steps, then scales as [N/16][K/G][16].
+ * codes as [N/32][K/64][2 halves][32 lanes][16 B] (one 16-byte load is one
+ * lane's MMA fragment for four k16 steps of two weight columns), then scales
+ * as [N/32][K/G][8][4].
  * Requirements: G in {32, 64, 128}; K % 64 == 0; K % G == 0; N % 64 == 0.
  * Otherwise MXG_ERR_UNSUPPORTED_SHAPE. */
 MXG_API int w4a16_repack(const int32_t *qweight, const uint16_t *scales,
@@ -111,7 +112,7 @@ MXG_API int w4a16_gemm(const void *X, const void *packed, int M, int N, int K, i
  * source pages have no counterpart to this call: it exists for callers that
  * cannot allocate a workspace (a plain C host with no device allocator of its
  * own; a serving process whose device memory is reserved up front).  It
- * allocates nothing: its scratch is one fixed 20 MiB array in device global
+ * allocates nothing: its scratch is one fixed 2 MiB array in device global
  * memory, one per device and process, shared by every call of this entry
  * point.
  *   X, packed, Y, shape rules: as for w4a16_gemm, with 1 <= M <= 32 (else

@@ -32,19 +32,20 @@ WorkspaceMap make_workspace_map(size_t counters, size_t partial_bytes);
 
 // ------------------------------------------------------ weight-streaming path
 // Stream-K plan: the layer's weight bytes are cut into equal "units" (one
-// n16 tile x one scale group, or one n16 tile x 128 k for MXFP8) and every
-// warp of a persistent grid takes one contiguous run of units.
+// n32 tile x one scale-group span for INT4, one n16 tile x 128 k for MXFP8)
+// and every CTA (INT4) or warp (MXFP8) of a persistent grid takes one
+// contiguous run of units.
 struct StreamPlan {
     int tt;               // token tiles of 8 rows (ceil(M / 8)), 1..4
     int variant;          // kernel variant (group mode for INT4)
     int warps_per_cta;
     int grid;             // CTAs
-    int Wt;               // active warps (<= grid * warps_per_cta, <= units)
+    int Wt;               // runs: CTAs (INT4) or warps (MXFP8), <= units
     long long units;      // total units
-    int upt;              // units per n16 tile
+    int upt;              // units per output tile
     size_t smem;          // dynamic shared memory per CTA
     size_t partial_bytes; // workspace for partial sums
-    int ntiles;           // n16 tiles (= arrival counters)
+    int ntiles;           // output tiles (= arrival counters)
 };
 
 bool plan_w4a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan);

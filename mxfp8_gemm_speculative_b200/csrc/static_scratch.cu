@@ -25,11 +25,11 @@
 namespace mxg {
 namespace {
 
-// Header + counters (256 KiB) + partial sums.  The stream-K plan needs
-// 2 KiB of partials per active warp and 8-row token tile; with 2 CTAs of 8
-// warps per SM on 148 SMs and M <= 32 (4 token tiles) that is 18.5 MiB, so
-// 20 MiB holds every M <= 32 shape on a B200.
-constexpr size_t kStaticScratchBytes = size_t(20) << 20;
+// Header + counters (256 KiB) + partial sums.  The streaming plan keeps one
+// fragment of 1 KiB per CTA and 8-row token tile; with one CTA per SM on
+// 148 SMs and M <= 32 (4 token tiles) that is 592 KiB, so 2 MiB holds every
+// M <= 32 shape on a B200.
+constexpr size_t kStaticScratchBytes = size_t(2) << 20;
 __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
 constexpr int kMaxDev = 64;
