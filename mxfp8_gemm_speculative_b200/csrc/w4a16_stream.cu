@@ -3,7 +3,7 @@
 // At M <= 32 the layer reads each weight byte once and does 2*M flops per
 // weight: it is bound by HBM bytes of W.  The kernel therefore
 //  * cuts the re-packed weight stream into equal units (one n32 tile x one
-//    scale-group span of max(G, 64) rows of K) and gives every CTA of a
+//    or two spans of max(G, 64) rows of K) and gives every CTA of a
 //    persistent grid (one per SM) one contiguous run of units (stream-K at
 //    CTA granularity), so all SMs stream the same number of bytes;
 //  * the CTA's warps take the run's units in turn (unit i goes to warp
@@ -41,37 +41,43 @@ namespace {
 #ifndef MXG_STREAM_CONSUMERS
 #define MXG_STREAM_CONSUMERS 12
 #endif
-#ifndef MXG_STREAM_STAGES
-#define MXG_STREAM_STAGES 5
+#ifndef MXG_STREAM_CTAS_PER_SM
+#define MXG_STREAM_CTAS_PER_SM 1
+#endif
+#ifndef MXG_STREAM_STAGES_BIG
+#define MXG_STREAM_STAGES_BIG 3
 #endif
 constexpr int kConsumers = MXG_STREAM_CONSUMERS;  // warps per CTA
 constexpr int kThreads = kConsumers * 32;
-constexpr int kStages = MXG_STREAM_STAGES;       // ring slots per warp (one unit each)
+constexpr int kCtasPerSm = MXG_STREAM_CTAS_PER_SM;   // resident CTAs per SM (grid size / SMs)
 constexpr int kMinUnitsPerCta = 2 * kConsumers;  // shortest run
 
-// Group modes: 0 -> G = 128, 1 -> G = 64, 2 -> G = 32.
-template <int GM>
+// Group modes: 0 -> G = 128, 1 -> G = 64, 2 -> G = 32.  A unit (what one
+// ring slot holds) spans SU times max(G, 64) rows of K of one n32 tile.
+template <int GM, int SU>
 struct Mode {
     static constexpr int kG = GM == 0 ? 128 : (GM == 1 ? 64 : 32);
-    static constexpr int kChunks = GM == 0 ? 2 : 1;          // k64 chunks per unit
-    static constexpr int kGroups = GM == 2 ? 2 : 1;          // scale groups per unit
+    static constexpr int kChunks = (GM == 0 ? 2 : 1) * SU;    // k64 chunks per unit
+    static constexpr int kGroups = (GM == 2 ? 2 : 1) * SU;    // scale groups per unit
     static constexpr int kStepsPerGroup = kG / 16;            // MMA k16 steps per group
     static constexpr int kCode = kChunks * 1024;              // code bytes per unit
     static constexpr int kScale = kGroups * 64;               // scale bytes per unit
+    static constexpr int kStages = kCode >= 4096 ? MXG_STREAM_STAGES_BIG : 5;  // slots per warp
 };
 
 // Shared memory: every warp's ring of kStages slots (a slot holds one
 // unit's codes, then its scales), kRed reduction buffers of kConsumers
 // fragments (segment s of the run uses buffer s mod kRed), one mbarrier per
 // slot, then per reduction buffer an arrival count and a use count.
-template <int TT, int GM>
+template <int TT, int GM, int SU>
 struct Smem {
+    using MD = Mode<GM, SU>;
     static constexpr int kFrag4 = 2 * TT * 32;                // float4 per warp fragment
-    static constexpr int kSlot = (Mode<GM>::kCode + Mode<GM>::kScale + 127) / 128 * 128;
-    static constexpr int kRed = TT <= 2 ? 4 : 2;
-    static constexpr size_t kRingBytes = (size_t)kConsumers * kStages * kSlot;
+    static constexpr int kSlot = (MD::kCode + MD::kScale + 127) / 128 * 128;
+    static constexpr int kRed = TT == 1 ? 4 : 2;
+    static constexpr size_t kRingBytes = (size_t)kConsumers * MD::kStages * kSlot;
     static constexpr size_t kRedBytes = (size_t)kRed * kConsumers * kFrag4 * 16;
-    static constexpr size_t kBarBytes = (size_t)kConsumers * kStages * 8;
+    static constexpr size_t kBarBytes = (size_t)kConsumers * MD::kStages * 8;
     static constexpr size_t kRedOff = kRingBytes;
     static constexpr size_t kBarOff = kRedOff + kRedBytes;
     static constexpr size_t kSyncOff = kBarOff + kBarBytes;
@@ -206,21 +212,22 @@ __device__ __forceinline__ void zero_acc(float (&a)[2][TT][4])
 }
 
 // Copies unit u (codes, then scales) into a ring slot; completion on `bar`.
-template <int GM>
+template <int GM, int SU>
 __device__ __forceinline__ void fetch_unit(const Params &p, uint8_t *slot, uint64_t *bar, int u,
                                            uint64_t policy)
 {
-    using MD = Mode<GM>;
+    using MD = Mode<GM, SU>;
     mbar_arrive_expect_tx(bar, MD::kCode + MD::kScale);
     bulk_g2s(slot, p.codes + (size_t)u * MD::kCode, MD::kCode, bar, policy);
     bulk_g2s(slot + MD::kCode, p.scales + (size_t)u * MD::kScale, MD::kScale, bar, policy);
 }
 
-template <int TT, int GM>
-__global__ void __launch_bounds__(kThreads, 1) w4a16_stream_kernel(const Params p)
+template <int TT, int GM, int SU>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) w4a16_stream_kernel(const Params p)
 {
-    using MD = Mode<GM>;
-    using SL = Smem<TT, GM>;
+    using MD = Mode<GM, SU>;
+    using SL = Smem<TT, GM, SU>;
+    constexpr int kStages = MD::kStages;
     constexpr int F = 2 * TT;  // float4 per lane fragment
     extern __shared__ __align__(128) uint8_t smem[];
     float4 *red = reinterpret_cast<float4 *>(smem + SL::kRedOff);
@@ -255,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_stream_kernel(const Params 
     // goes to slot k mod kStages
     if (lane == 0)
         for (int k = 0; k < kStages && warp + k * kConsumers < n; ++k)
-            fetch_unit<GM>(p, ring + k * SL::kSlot, &full[k], U0 + warp + k * kConsumers, policy);
+            fetch_unit<GM, SU>(p, ring + k * SL::kSlot, &full[k], U0 + warp + k * kConsumers, policy);
 
     // ------------------------------------------------------------ consumers
     const int g = lane >> 2, t = lane & 3;
@@ -273,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_stream_kernel(const Params 
 
     // Activation fragments of one unit, requested one unit ahead for narrow
     // token tiles (a whole unit of work hides their L2 latency).
-    constexpr bool kPipeX = TT <= 2;
+    constexpr bool kPipeX = MD::kChunks * TT <= 4;
     uint2 xs[MD::kChunks][TT][4], xn[MD::kChunks][TT][4];
     auto load_x = [&](uint2 (&dst)[MD::kChunks][TT][4], int u) {
         const int kc = (u % upt) * MD::kChunks;  // first k64 chunk of unit u
@@ -382,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_stream_kernel(const Params 
             // consumed above): refill it with this warp's unit kStages ahead
             __syncwarp();
             if (lane == 0 && i + kStages * kConsumers < n)
-                fetch_unit<GM>(p, ring + slot * SL::kSlot, &full[slot],
+                fetch_unit<GM, SU>(p, ring + slot * SL::kSlot, &full[slot],
                                u + kStages * kConsumers, policy);
             if (kPipeX) {
 #pragma unroll
@@ -465,38 +472,49 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_stream_kernel(const Params 
     }
 }
 
-template <int TT, int GM>
+template <int TT, int GM, int SU>
 const void *kernel_ptr()
 {
-    return reinterpret_cast<const void *>(&w4a16_stream_kernel<TT, GM>);
+    return reinterpret_cast<const void *>(&w4a16_stream_kernel<TT, GM, SU>);
 }
 
-const void *select_kernel(int tt, int gm)
+// SU = 2 (two scale-group spans per unit) for up to two token tiles,
+// SU = 1 otherwise; variant = gm + 3 * (SU - 1).
+const void *select_kernel(int tt, int variant)
 {
-#define MXG_CASE(T, G_) \
-    if (tt == T && gm == G_) return kernel_ptr<T, G_>();
-    MXG_CASE(1, 0) MXG_CASE(1, 1) MXG_CASE(1, 2)
-    MXG_CASE(2, 0) MXG_CASE(2, 1) MXG_CASE(2, 2)
-    MXG_CASE(3, 0) MXG_CASE(3, 1) MXG_CASE(3, 2)
-    MXG_CASE(4, 0) MXG_CASE(4, 1) MXG_CASE(4, 2)
+#define MXG_CASE(T, G_, S_) \
+    if (tt == T && variant == G_ + 3 * (S_ - 1)) return kernel_ptr<T, G_, S_>();
+    MXG_CASE(1, 0, 1) MXG_CASE(1, 1, 1) MXG_CASE(1, 2, 1)
+    MXG_CASE(2, 0, 1) MXG_CASE(2, 1, 1) MXG_CASE(2, 2, 1)
+    MXG_CASE(3, 0, 1) MXG_CASE(3, 1, 1) MXG_CASE(3, 2, 1)
+    MXG_CASE(4, 0, 1) MXG_CASE(4, 1, 1) MXG_CASE(4, 2, 1)
+    MXG_CASE(1, 0, 2) MXG_CASE(1, 1, 2) MXG_CASE(1, 2, 2)
+    MXG_CASE(2, 0, 2) MXG_CASE(2, 1, 2) MXG_CASE(2, 2, 2)
 #undef MXG_CASE
     return nullptr;
 }
 
-template <int GM>
-size_t smem_bytes_gm(int tt)
+template <int GM, int SU>
+size_t smem_bytes_gs(int tt)
 {
     switch (tt) {
-    case 1: return Smem<1, GM>::kTotal;
-    case 2: return Smem<2, GM>::kTotal;
-    case 3: return Smem<3, GM>::kTotal;
-    default: return Smem<4, GM>::kTotal;
+    case 1: return Smem<1, GM, SU>::kTotal;
+    case 2: return Smem<2, GM, SU>::kTotal;
+    case 3: return Smem<3, GM, 1>::kTotal;
+    default: return Smem<4, GM, 1>::kTotal;
     }
 }
 
-size_t smem_bytes(int tt, int gm)
+size_t smem_bytes(int tt, int variant)
 {
-    return gm == 0 ? smem_bytes_gm<0>(tt) : gm == 1 ? smem_bytes_gm<1>(tt) : smem_bytes_gm<2>(tt);
+    switch (variant) {
+    case 0: return smem_bytes_gs<0, 1>(tt);
+    case 1: return smem_bytes_gs<1, 1>(tt);
+    case 2: return smem_bytes_gs<2, 1>(tt);
+    case 3: return smem_bytes_gs<0, 2>(tt);
+    case 4: return smem_bytes_gs<1, 2>(tt);
+    default: return smem_bytes_gs<2, 2>(tt);
+    }
 }
 
 int group_mode(int G)
@@ -513,13 +531,14 @@ bool plan_w4a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan)
     const DeviceInfo &di = device_info(device);
     StreamPlan pl{};
     pl.tt = (M + 7) / 8;
-    pl.variant = group_mode(G);
+    const int unit_k = std::max(G, 64);
+    const int su = (pl.tt <= 2 && (K / unit_k) % 2 == 0) ? 2 : 1;
+    pl.variant = group_mode(G) + 3 * (su - 1);
     pl.warps_per_cta = kConsumers;
     pl.smem = smem_bytes(pl.tt, pl.variant);
     if ((int)pl.smem > di.smem_optin)
         return false;
-    const int unit_k = std::max(G, 64);
-    pl.upt = K / unit_k;
+    pl.upt = K / (unit_k * su);
     pl.ntiles = N / 32;
     if ((size_t)pl.ntiles > kMaxCounters)
         return false;
@@ -529,15 +548,24 @@ bool plan_w4a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan)
     const void *fn = select_kernel(pl.tt, pl.variant);
     if (!fn)
         return false;
-    static bool attr_set[4][3] = {};
-    if (!attr_set[pl.tt - 1][pl.variant]) {
+    // resident CTAs per SM for this variant: every CTA of the grid must be
+    // resident at once (a cut tile's finishing CTA waits for the others)
+    static int occ_cache[4][6] = {};
+    int &occ = occ_cache[pl.tt - 1][pl.variant];
+    if (occ == 0) {
         if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem) !=
             cudaSuccess)
             return false;
-        attr_set[pl.tt - 1][pl.variant] = true;
+        int o = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, fn, kThreads, pl.smem) !=
+                cudaSuccess ||
+            o < 1)
+            return false;
+        occ = std::min(o, kCtasPerSm);
     }
-    // one CTA per SM, but no run shorter than kMinUnitsPerCta units
-    pl.Wt = (int)std::max<long long>(1, std::min<long long>(di.sms, pl.units / kMinUnitsPerCta));
+    // kCtasPerSm CTAs per SM, but no run shorter than kMinUnitsPerCta units
+    pl.Wt = (int)std::max<long long>(
+        1, std::min<long long>((long long)di.sms * occ, pl.units / kMinUnitsPerCta));
     pl.grid = pl.Wt;
     pl.partial_bytes = (size_t)pl.Wt * (2 * pl.tt * 32) * sizeof(float4);
     *plan = pl;
