@@ -16,6 +16,7 @@ grow it on demand; pass ``workspace=`` to manage it yourself.
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 import threading
 
@@ -117,6 +118,16 @@ def workspace(nbytes: int, device=None, stream=None) -> torch.Tensor:
         return ws
 
 
+@functools.lru_cache(maxsize=4096)
+def _need_bytes(kind: str, device: int, M: int, N: int, K: int, G: int = 0) -> int:
+    """Workspace size query, cached per (device, shape); the size depends on
+    the device's SM count, so the query runs with that device current."""
+    with torch.cuda.device(device):
+        if kind == "w4a16":
+            return int(_lib.w4a16_workspace_bytes(M, N, K, G))
+        return int(_lib.mxfp8_workspace_bytes(M, N, K))
+
+
 # -------------------------------------------------------------------- INT4
 def w4a16_packed_bytes(K: int, N: int, group_size: int = 128) -> int:
     return int(_lib.w4a16_packed_bytes(K, N, group_size))
@@ -155,8 +166,8 @@ def w4a16_gemm(x: torch.Tensor, packed: torch.Tensor, N: int, K: int, group_size
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     _need(out, torch.bfloat16, "out")
-    need = w4a16_workspace_bytes(M, N, K, group_size)
-    ws = workspace_buf if workspace_buf is not None else workspace(need, x.device, stream)
+    ws = (workspace_buf if workspace_buf is not None else
+          workspace(_need_bytes("w4a16", x.device.index, M, N, K, group_size), x.device, stream))
     _check(_lib.w4a16_gemm(_ptr(x), _ptr(packed), M, N, K, group_size, _ptr(out), _ptr(ws),
                            ws.numel(), _stream(stream)), "w4a16_gemm")
     return out
@@ -212,8 +223,8 @@ def mxfp8_gemm(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor,
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     _need(out, torch.bfloat16, "out")
-    need = mxfp8_workspace_bytes(M, N, K)
-    wsb = workspace_buf if workspace_buf is not None else workspace(need, x.device, stream)
+    wsb = (workspace_buf if workspace_buf is not None else
+           workspace(_need_bytes("mxfp8", x.device.index, M, N, K), x.device, stream))
     _check(_lib.mxfp8_gemm(_ptr(x), _ptr(wq), _ptr(ws), M, N, K, _ptr(out), _ptr(wsb),
                            wsb.numel(), _stream(stream)), "mxfp8_gemm")
     return out

@@ -240,7 +240,10 @@ int w4a16_gemm(const void *X, const void *packed, int M, int N, int K, int group
     StreamPlan sp;
     TcPlan tp;
     const bool s_ok = plan_w4a16_stream(dev, M, N, K, group_size, &sp);
-    const bool t_ok = plan_w4a16_tc(dev, M, N, K, group_size, &tp);
+    // the tensor-core plan only matters when the streaming path is not taken
+    const bool t_ok = (M <= 32 && s_ok && g_path.load() != 2)
+                          ? false
+                          : plan_w4a16_tc(dev, M, N, K, group_size, &tp);
     const int path = choose_path(M, s_ok, t_ok);
     if (path == 1) {
         if (workspace_bytes < make_workspace_map(sp.ntiles, sp.partial_bytes).total)
@@ -283,7 +286,9 @@ int mxfp8_gemm(const void *X, const uint8_t *Wq, const uint8_t *Ws, int M, int N
     StreamPlan sp;
     TcPlan tp;
     const bool s_ok = plan_mxfp8_stream(dev, M, N, K, &sp);
-    const bool t_ok = plan_mxfp8_tc(dev, M, N, K, &tp);
+    const bool t_ok = (M <= 32 && s_ok && g_path.load() != 2)
+                          ? false
+                          : plan_mxfp8_tc(dev, M, N, K, &tp);
     const int path = choose_path(M, s_ok, t_ok);
     if (path == 1) {
         if (workspace_bytes < make_workspace_map(sp.ntiles, sp.partial_bytes).total)

@@ -38,9 +38,6 @@ namespace {
 
 constexpr int BW = 128;  // weight columns per CTA
 constexpr int BK = 64;   // k per block
-constexpr int kSX = 4;   // activation ring
-constexpr int kSW = 4;   // packed-weight ring
-constexpr int kSA = 4;   // tensor-memory A ring (32 columns each)
 constexpr int kProducerWarp = 0, kMmaWarp = 1, kEpiWarp0 = 2, kNumEpiWarps = 4;
 constexpr int kDqWarp0 = 6, kNumDqWarps = 8;
 constexpr int kThreads = (kDqWarp0 + kNumDqWarps) * 32;
@@ -48,8 +45,14 @@ constexpr uint32_t kTmemCols = 512;
 
 enum Fmt { kInt4 = 0, kMxfp8 = 1 };
 
+// Ring depths: with 128 tokens per tile the activation and weight slots are
+// small and a k-block's MMA is short, so the rings are deeper to cover the
+// load latency.
 template <int F, int BT>
 struct Layout {
+    static constexpr int kSX = BT == 128 ? 8 : 4;    // activation ring
+    static constexpr int kSW = BT == 128 ? 12 : 8;   // packed-weight ring
+    static constexpr int kSA = BT == 128 ? 8 : 6;    // tensor-memory A ring (32 columns each)
     static constexpr int x_slot = (BT / 2) * BK * 2;                // bf16 activations
     static constexpr int wp_slot = (F == kInt4) ? 5120 : BW * BK;   // packed weights
     static constexpr int x_off = 0;
@@ -68,10 +71,24 @@ struct TcParams {
     uint16_t *Y;
     const uint8_t *Ws;     // MXFP8 scales [N][K/32]
     WsHeader *hdr;
+    float *partial;        // split-K partial sums [num_items][BT][2 * BW] (splits > 1)
+    int *counters;         // split-K arrivals per (tile, CTA of the pair, quadrant)
     int M, N, K, G;
     int mtiles, ntiles, kblocks;
     int num_tiles;
+    int splits;            // K splits per output tile
+    int num_items;         // num_tiles * splits work items
 };
+
+// Work item -> output tile and its k-block range [kb0, kb1).
+__device__ __forceinline__ void item_range(const TcParams &p, int item, int &tile, int &kb0,
+                                           int &kb1)
+{
+    tile = item / p.splits;
+    const int s = item - tile * p.splits;
+    kb0 = (int)((long long)s * p.kblocks / p.splits);
+    kb1 = (int)((long long)(s + 1) * p.kblocks / p.splits);
+}
 
 // ----------------------------------------------------------- cluster PTX
 __device__ __forceinline__ uint32_t cluster_ctarank()
@@ -301,10 +318,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::bar_off);
-    uint64_t *x_full = bars, *x_empty = bars + kSX;
-    uint64_t *wp_full = bars + 2 * kSX, *wp_empty = wp_full + kSW;
-    uint64_t *a_full = wp_empty + kSW, *a_empty = a_full + kSA;
-    uint64_t *acc_full = a_empty + kSA, *acc_empty = acc_full + 1;
+    uint64_t *x_full = bars, *x_empty = bars + L::kSX;
+    uint64_t *wp_full = bars + 2 * L::kSX, *wp_empty = wp_full + L::kSW;
+    uint64_t *a_full = wp_empty + L::kSW, *a_empty = a_full + L::kSA;
+    uint64_t *acc_full = a_empty + L::kSA, *acc_empty = acc_full + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::misc_off);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::misc_off + 4);
 
@@ -314,15 +331,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     pdl_launch_dependents();
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kSX; ++i) {
+        for (int i = 0; i < L::kSX; ++i) {
             mbar_init(&x_full[i], 1);            // leader: producer arrive + both copies
             mbar_init(&x_empty[i], 1);           // commit from the MMA
         }
-        for (int i = 0; i < kSW; ++i) {
+        for (int i = 0; i < L::kSW; ++i) {
             mbar_init(&wp_full[i], 1);
             mbar_init(&wp_empty[i], kNumDqWarps);
         }
-        for (int i = 0; i < kSA; ++i) {
+        for (int i = 0; i < L::kSA; ++i) {
             mbar_init(&a_full[i], 2 * kNumDqWarps);   // leader: dequantisers of both CTAs
             mbar_init(&a_empty[i], 1);                 // commit from the MMA
         }
@@ -333,11 +350,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     if (warp == kMmaWarp)
         tmem_alloc_pair(tmem_slot, kTmemCols);
-    if (threadIdx.x == 32 * kProducerWarp && pair < p.num_tiles) {
+    if (threadIdx.x == 32 * kProducerWarp && pair < p.num_items) {
         // while the previous kernel drains: pull the first k-blocks into L2
-        const int nb = pair / p.mtiles, mt = pair % p.mtiles;
+        int tile0, kb0, kb1;
+        item_range(p, pair, tile0, kb0, kb1);
+        const int nb = tile0 / p.mtiles, mt = tile0 % p.mtiles;
         const int n32 = (nb * 2 * BW + (int)rank * BW) / 32;
-        for (int kb = 0; kb < min(kSW, p.kblocks); ++kb) {
+        for (int kb = kb0; kb < min(kb0 + L::kSW, kb1); ++kb) {
             prefetch_tensor_l2(&x_map, kb * BK, mt * BT + (int)rank * (BT / 2));
             if (F == kInt4)
                 prefetch_tensor_l2(&w_map, kb * 128, n32);
@@ -363,12 +382,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const uint64_t pol_x = l2_policy_evict_last();
             uint32_t it = 0;
             bool ok = true;
-            for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
+            for (int item = pair; item < p.num_items && ok; item += npairs) {
+                int tile, kb0, kb1;
+                item_range(p, item, tile, kb0, kb1);
                 const int nb = tile / p.mtiles, mt = tile % p.mtiles;
-                for (int kb = 0; kb < p.kblocks && ok; ++kb, ++it) {
-                    const int sx = it % kSX, sw = it % kSW;
+                for (int kb = kb0; kb < kb1 && ok; ++kb, ++it) {
+                    const int sx = it % L::kSX, sw = it % L::kSW;
                     // activations: this CTA's BT/2 tokens, completing on the leader's barrier
-                    ok = role_wait(&x_empty[sx], ((it / kSX) & 1) ^ 1, abort_flag, p.hdr, 401);
+                    ok = role_wait(&x_empty[sx], ((it / L::kSX) & 1) ^ 1, abort_flag, p.hdr, 401);
                     if (!ok)
                         break;
                     if (rank == 0)
@@ -377,7 +398,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                      mt * BT + (int)rank * (BT / 2),
                                      mapa_shared(smem_u32(&x_full[sx]), 0), pol_x);
                     // packed weights of this CTA's 128 columns
-                    ok = role_wait(&wp_empty[sw], ((it / kSW) & 1) ^ 1, abort_flag, p.hdr, 402);
+                    ok = role_wait(&wp_empty[sw], ((it / L::kSW) & 1) ^ 1, abort_flag, p.hdr, 402);
                     if (!ok)
                         break;
                     uint8_t *wdst = smem + L::wp_off + sw * L::wp_slot;
@@ -399,16 +420,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             constexpr uint32_t idesc = idesc_pair<BT>();
             uint32_t it = 0, tcount = 0;
             bool ok = true;
-            for (int tile = pair; tile < p.num_tiles && ok; tile += npairs, ++tcount) {
+            for (int item = pair; item < p.num_items && ok; item += npairs, ++tcount) {
+                int tile, kb0, kb1;
+                item_range(p, item, tile, kb0, kb1);
                 ok = role_wait(acc_empty, (tcount & 1) ^ 1, abort_flag, p.hdr, 411);
                 if (!ok)
                     break;
                 tc_fence_after();
                 const uint32_t d = tmem_base + L::acc_col;
-                for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
-                    const int sx = it % kSX, sa = it % kSA;
-                    ok = role_wait(&x_full[sx], (it / kSX) & 1, abort_flag, p.hdr, 412) &&
-                         role_wait(&a_full[sa], (it / kSA) & 1, abort_flag, p.hdr, 413);
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                    const int sx = it % L::kSX, sa = it % L::kSA;
+                    ok = role_wait(&x_full[sx], (it / L::kSX) & 1, abort_flag, p.hdr, 412) &&
+                         role_wait(&a_full[sa], (it / L::kSA) & 1, abort_flag, p.hdr, 413);
                     if (!ok)
                         break;
                     tc_fence_after();
@@ -417,7 +440,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)
                         tc_mma_ts_pair(d, a + 8 * k, sw128_desc(xa + 32 * k), idesc,
-                                       (kb > 0 || k > 0) ? 1u : 0u);
+                                       (kb > kb0 || k > 0) ? 1u : 0u);
                     tc_commit_pair(&x_empty[sx]);
                     tc_commit_pair(&a_empty[sa]);
                 }
@@ -429,30 +452,104 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int q = warp & 3;  // TMEM lane quadrant this warp may access
         const uint32_t leader_acc_empty = mapa_shared(smem_u32(acc_empty), 0);
         uint32_t tcount = 0;
-        for (int tile = pair; tile < p.num_tiles; tile += npairs, ++tcount) {
+        for (int item = pair; item < p.num_items; item += npairs, ++tcount) {
+            int tile, kb0, kb1;
+            item_range(p, item, tile, kb0, kb1);
             if (!role_wait(acc_full, tcount & 1, abort_flag, p.hdr, 421))
                 break;
             tc_fence_after();
             const int nb = tile / p.mtiles, mt = tile % p.mtiles;
-            const int n = nb * 2 * BW + (int)rank * BW + q * 32 + lane;   // this thread's column
+            const int nloc = (int)rank * BW + q * 32;                    // warp's first column in the pair
+            const int n = nb * 2 * BW + nloc + lane;                      // this thread's column
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + L::acc_col;
+            if (p.splits == 1) {
 #pragma unroll 1
-            for (int c = 0; c < BT / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tbase + c * 32, r);
-                const int m0 = mt * BT + c * 32;
-                if (n < p.N) {
-                    uint16_t *yc = p.Y + (size_t)m0 * p.N + n;
+                for (int c = 0; c < BT / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tbase + c * 32, r);
+                    const int m0 = mt * BT + c * 32;
+                    if (n < p.N) {
+                        uint16_t *yc = p.Y + (size_t)m0 * p.N + n;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (m0 + i < p.M)
+                                yc[(size_t)i * p.N] = f32_to_bf16_bits(__uint_as_float(r[i]));
+                    }
+                }
+            } else {
+                // split K: this item's fp32 sums of the warp's 32 columns
+                float *pp = p.partial + (size_t)item * BT * (2 * BW) + nloc + lane;
+#pragma unroll 1
+                for (int c = 0; c < BT / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tbase + c * 32, r);
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
-                        if (m0 + i < p.M)
-                            yc[(size_t)i * p.N] = f32_to_bf16_bits(__uint_as_float(r[i]));
+                        __stcg(pp + (size_t)(c * 32 + i) * (2 * BW), __uint_as_float(r[i]));
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
                 mbar_arrive_cluster(leader_acc_empty);
+            if (p.splits > 1) {
+                // the last split of this (tile, CTA, quadrant) slab adds the splits
+                // in order and writes bf16 Y
+                int *cnt = p.counters + tile * 8 + (int)rank * 4 + q;
+                int last = 0;
+                if (lane == 0) {
+                    __threadfence();
+                    last = atomicAdd(cnt, 1) == p.splits - 1;
+                    if (last)
+                        __threadfence();
+                }
+                if (__shfl_sync(0xffffffffu, last, 0)) {
+                    const int c4 = (lane & 7) * 4;        // 4 columns per lane
+                    const int nc = nb * 2 * BW + nloc + c4;
+                    const float *src0 =
+                        p.partial + (size_t)tile * p.splits * BT * (2 * BW) + nloc + c4;
+                    // rows r = 4 * u + lane / 8, eight rows per pass; the
+                    // splits are added in order, each pass keeping its 8 loads
+                    // of a split in flight together
+#pragma unroll 1
+                    for (int rb = 0; rb < BT / 4; rb += 8) {
+                        float4 acc4[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            acc4[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+                        for (int sp = 0; sp < p.splits; ++sp) {
+                            float4 v[8];
+#pragma unroll
+                            for (int u = 0; u < 8; ++u)
+                                v[u] = __ldcg(reinterpret_cast<const float4 *>(
+                                    src0 + ((size_t)sp * BT + 4 * (rb + u) + (lane >> 3)) *
+                                               (2 * BW)));
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                acc4[u].x += v[u].x;
+                                acc4[u].y += v[u].y;
+                                acc4[u].z += v[u].z;
+                                acc4[u].w += v[u].w;
+                            }
+                        }
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int m = mt * BT + 4 * (rb + u) + (lane >> 3);
+                            if (m < p.M) {
+                                const float e[4] = {acc4[u].x, acc4[u].y, acc4[u].z, acc4[u].w};
+#pragma unroll
+                                for (int i = 0; i < 4; ++i)
+                                    if (nc + i < p.N)
+                                        p.Y[(size_t)m * p.N + nc + i] = f32_to_bf16_bits(e[i]);
+                            }
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0)
+                        *cnt = 0;  // leave the counter zero for the next call
+                }
+            }
         }
     } else {
         // dequantisers: warp -> (quadrant q, half h) of the CTA's 128 weight rows
@@ -461,10 +558,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int g = lane >> 2;
         uint32_t it = 0;
         bool ok = true;
-        for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
+        for (int item = pair; item < p.num_items && ok; item += npairs) {
+            int tile, kb0, kb1;
+            item_range(p, item, tile, kb0, kb1);
             const int nb = tile / p.mtiles;
-            for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
-                const int sw = it % kSW, sa = it % kSA;
+            for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                const int sw = it % L::kSW, sa = it % L::kSA;
                 float sca[2] = {1.f, 1.f}, scb[2] = {1.f, 1.f};
                 if (F == kMxfp8) {
                     // E8M0 scales of rows ra, ra + 8 for the two 32-blocks of this k-block
@@ -485,8 +584,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         scb[b] = e8m0_to_f32(eb);
                     }
                 }
-                ok = role_wait(&wp_full[sw], (it / kSW) & 1, abort_flag, p.hdr, 431) &&
-                     role_wait(&a_empty[sa], ((it / kSA) & 1) ^ 1, abort_flag, p.hdr, 432);
+                ok = role_wait(&wp_full[sw], (it / L::kSW) & 1, abort_flag, p.hdr, 431) &&
+                     role_wait(&a_empty[sa], ((it / L::kSA) & 1) ^ 1, abort_flag, p.hdr, 432);
                 if (!ok)
                     break;
                 tc_fence_after();
@@ -546,7 +645,6 @@ bool x_map(CUtensorMap *m, const void *X, int M, int K, int BT)
 template <int F>
 bool tc_plan(int device, int M, int N, int K, TcPlan *plan)
 {
-    (void)K;
     const DeviceInfo &di = device_info(device);
     const int BT = M <= 128 ? 128 : 256;
     const size_t smem = BT == 128 ? Layout<F, 128>::smem_bytes : Layout<F, 256>::smem_bytes;
@@ -558,12 +656,33 @@ bool tc_plan(int device, int M, int N, int K, TcPlan *plan)
     pl.bk = BK;
     pl.mtiles = (M + BT - 1) / BT;
     pl.ntiles = (N + 2 * BW - 1) / (2 * BW);
-    pl.splits = 1;
     const int tiles = pl.mtiles * pl.ntiles;
-    pl.grid = 2 * std::min(tiles, di.sms / 2);
+    const int pairs = di.sms / 2;
+    const int kblocks = (K + BK - 1) / BK;
+    // Split K when the tiles alone leave pairs idle: pick the split count
+    // that minimises the k-blocks of the busiest pair plus a charge of two
+    // k-blocks per split for writing and adding the fp32 partial sums.
+    int best = 1;
+    long long best_cost = (long long)((tiles + pairs - 1) / pairs) * kblocks;
+    if (tiles < pairs) {
+        for (int sp = 2; sp <= 16 && sp <= kblocks / 4; ++sp) {
+            const long long items = (long long)tiles * sp;
+            const long long cost =
+                ((items + pairs - 1) / pairs) * ((kblocks + sp - 1) / sp) + 2 * sp;
+            if (cost < best_cost) {
+                best_cost = cost;
+                best = sp;
+            }
+        }
+    }
+    pl.splits = best;
+    const int items = tiles * best;
+    if (best > 1 && (size_t)tiles * 8 > kMaxCounters)
+        return false;
+    pl.grid = 2 * std::min(items, pairs);
     pl.smem = smem;
-    pl.partial_bytes = 0;
-    pl.counters = 0;
+    pl.partial_bytes = best > 1 ? (size_t)items * BT * 2 * BW * sizeof(float) : 0;
+    pl.counters = best > 1 ? (size_t)tiles * 8 : 0;
     *plan = pl;
     return true;
 }
@@ -605,6 +724,13 @@ cudaError_t launch_w4a16_tc(const TcPlan &pl, const void *X, const void *packed,
     p.ntiles = pl.ntiles;
     p.kblocks = K / BK;
     p.num_tiles = pl.mtiles * pl.ntiles;
+    p.splits = pl.splits;
+    p.num_items = p.num_tiles * pl.splits;
+    {
+        const WorkspaceMap wsm = make_workspace_map(pl.counters, pl.partial_bytes);
+        p.counters = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + wsm.counters_off);
+        p.partial = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + wsm.partial_off);
+    }
     if (pl.bm == 128)
         return tc_launch<kInt4, 128>(pl, xm, wm, sm, p, stream);
     return tc_launch<kInt4, 256>(pl, xm, wm, sm, p, stream);
@@ -636,6 +762,13 @@ cudaError_t launch_mxfp8_tc(const TcPlan &pl, const void *X, const uint8_t *Wq,
     p.ntiles = pl.ntiles;
     p.kblocks = (K + BK - 1) / BK;
     p.num_tiles = pl.mtiles * pl.ntiles;
+    p.splits = pl.splits;
+    p.num_items = p.num_tiles * pl.splits;
+    {
+        const WorkspaceMap wsm = make_workspace_map(pl.counters, pl.partial_bytes);
+        p.counters = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + wsm.counters_off);
+        p.partial = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + wsm.partial_off);
+    }
     if (pl.bm == 128)
         return tc_launch<kMxfp8, 128>(pl, xm, wm, wm, p, stream);
     return tc_launch<kMxfp8, 256>(pl, xm, wm, wm, p, stream);
