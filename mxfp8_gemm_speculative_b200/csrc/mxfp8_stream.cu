@@ -1,16 +1,18 @@
 // MXFP8 weight-streaming GEMM for small M.
 //
-// Same structure as the INT4 streaming kernel: stream-K over units, one
-// shared-memory ring per warp, swap-AB m16n8k16 MMAs, last-arriver reduction
-// of shared tiles.  Differences:
+// Same structure as the INT4 streaming kernel (one contiguous stream-K run
+// of units per CTA, units dealt to the CTA's warps in turn, one ring of
+// bulk-copied slots per warp, swap-AB m16n8k16 MMAs, non-blocking tile
+// reductions through shared memory, cut tiles finished by the CTA holding
+// their first unit).  Differences:
 //  * the weights are consumed in their stored layout, Wq[N][K] (no re-pack):
-//    a unit is one n16 tile x 128 k, fetched as a 2-D tensor-map box of
-//    16 rows x 128 bytes with the 128-byte swizzle (conflict-free 16-byte
+//    a unit is one n16 tile x SU * 128 k, fetched as SU 2-D tensor-map boxes
+//    of 16 rows x 128 bytes with the 128-byte swizzle (conflict-free 16-byte
 //    shared loads by lane g of row g and row g + 8); rows past N and columns
 //    past K are zero-filled by the copy engine;
-//  * lane t of a unit owns k = 32t .. 32t + 31 of rows g and g + 8, which is
-//    exactly one E8M0 block, so each lane needs two scales per unit, loaded
-//    one stage ahead into registers;
+//  * lane t of a box owns k = 32t .. 32t + 31 of rows g and g + 8, which is
+//    exactly one E8M0 block, so each lane needs two scales per box, loaded
+//    one unit ahead into registers;
 //  * E4M3 -> bf16 with the block scale folded in (exact for normal bf16
 //    results): hardware e4m3x2 -> f16x2, f16 -> f32, times 2^(E-127), one
 //    rounding to bf16.
@@ -22,11 +24,34 @@
 namespace mxg {
 namespace {
 
-constexpr int kWarps = 8;
-constexpr int kRing = 6;                  // stages per warp
-constexpr int kStage = 2048;              // one 16 x 128-byte box
-constexpr int kWarpSmem = kRing * kStage;
-constexpr int kMinUnits = 6;              // shortest run per warp
+#ifndef MXG_MX_SU2_TT
+#define MXG_MX_SU2_TT 2
+#endif
+constexpr int kConsumers = 12;                  // warps per CTA
+constexpr int kThreads = kConsumers * 32;
+constexpr int kBox = 2048;                      // one 16 x 128-byte box
+constexpr int kMinUnitsPerCta = 2 * kConsumers; // shortest run
+
+// A unit (what one ring slot holds) is SU boxes along K of one n16 tile.
+template <int SU>
+struct Unit {
+    static constexpr int kBytes = SU * kBox;
+    static constexpr int kStages = SU == 2 ? 3 : 5;  // ring slots per warp
+};
+
+// Shared memory (1024-byte aligned for the swizzle): every warp's ring,
+// kRed reduction buffers of kConsumers fragments, one mbarrier per slot,
+// then per reduction buffer an arrival count and a use count.
+template <int TT, int SU>
+struct Smem {
+    static constexpr int kFrag4 = TT * 32;       // float4 per warp fragment
+    static constexpr int kRed = TT == 1 ? 4 : 2;
+    static constexpr size_t kRingBytes = (size_t)kConsumers * Unit<SU>::kStages * Unit<SU>::kBytes;
+    static constexpr size_t kRedOff = kRingBytes;
+    static constexpr size_t kBarOff = kRedOff + (size_t)kRed * kConsumers * kFrag4 * 16;
+    static constexpr size_t kSyncOff = kBarOff + (size_t)kConsumers * Unit<SU>::kStages * 8;
+    static constexpr size_t kTotal = kSyncOff + 2 * kRed * sizeof(int) + 1024;  // + alignment
+};
 
 struct Params {
     const uint16_t *X;       // bf16 [M][K]
@@ -34,97 +59,117 @@ struct Params {
     uint16_t *Y;             // bf16 [M][N]
     WsHeader *hdr;
     int *counters;           // [ceil(N/16)]
-    float *partial;          // [Wt][2][32][4*TT]
+    float4 *partial;         // [ctas][TT][32]: a CTA's fragment of its first, cut tile
     int M, N, K;
-    int upt;                 // units per n16 tile = ceil(K / 128)
+    int upt;                 // units per n16 tile
     int units;
-    int Wt;
-    int q, r;                // units = q * Wt + r: warps below r run q + 1 units, the rest q
+    int ctas;
+    int q, r;                // units = q * ctas + r: CTAs below r run q + 1 units, the rest q
 };
 
-// First unit of warp w's run.
-__device__ __forceinline__ int run_start(const Params &p, int w)
+// First unit of CTA c's run.
+__device__ __forceinline__ int run_start(const Params &p, int c)
 {
-    return w * p.q + min(w, p.r);
+    return c * p.q + min(c, p.r);
 }
 
-// The warp whose run contains unit u.
-__device__ __forceinline__ int warp_of_unit(const Params &p, int u)
+// The CTA whose run contains unit u.
+__device__ __forceinline__ int cta_of_unit(const Params &p, int u)
 {
     const int big = p.r * (p.q + 1);
     return u < big ? u / (p.q + 1) : p.r + (u - big) / p.q;
 }
 
-template <int TT>
-__device__ __forceinline__ void store_tile_y(const Params &p, int nt, const float (&v)[TT][4], int g,
-                                             int t)
-{
-#pragma unroll
-    for (int tt = 0; tt < TT; ++tt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int m = tt * 8 + 2 * t + (e & 1);
-            const int n = nt * 16 + g + ((e & 2) ? 8 : 0);
-            if (m < p.M && n < p.N)
-                p.Y[(size_t)m * p.N + n] = f32_to_bf16_bits(v[tt][e]);
-        }
-}
-
-template <int TT>
-__device__ __forceinline__ void store_partial(const Params &p, int gw, int slot, int lane,
-                                              const float (&v)[TT][4])
-{
-    float *dst = p.partial + ((size_t)(gw * 2 + slot) * 32 + lane) * (4 * TT);
-#pragma unroll
-    for (int tt = 0; tt < TT; ++tt)
-        __stcg(reinterpret_cast<float4 *>(dst + 4 * tt),
-               make_float4(v[tt][0], v[tt][1], v[tt][2], v[tt][3]));
-}
-
-// Run by the last contributor of a cut tile: add every fragment of the tile
-// in warp order and write bf16 Y.
-template <int TT>
-__device__ __noinline__ void reduce_tile(const Params &p, int nt, int lane)
+// Writes the four outputs of fragment float4 tt of `lane` for n16 tile nt.
+__device__ __forceinline__ void store_y4(const Params &p, int nt, int tt, int lane, float4 v)
 {
     const int g = lane >> 2, t = lane & 3;
-    const int tile_begin = nt * p.upt, tile_end = tile_begin + p.upt;
-    const int w_first = warp_of_unit(p, tile_begin);
-    const int w_last = warp_of_unit(p, tile_end - 1);
-    float sum[TT][4];
+    const float e[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int tt = 0; tt < TT; ++tt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-            sum[tt][e] = 0.f;
-#pragma unroll 4
-    for (int w = w_first; w <= w_last; ++w) {
-        const int s = (run_start(p, w) >= tile_begin) ? 0 : 1;
-        const float *src = p.partial + ((size_t)(w * 2 + s) * 32 + lane) * (4 * TT);
-#pragma unroll
-        for (int tt = 0; tt < TT; ++tt) {
-            const float4 f = ldcg_f4(src + 4 * tt);
-            sum[tt][0] += f.x;
-            sum[tt][1] += f.y;
-            sum[tt][2] += f.z;
-            sum[tt][3] += f.w;
-        }
+    for (int i = 0; i < 4; ++i) {
+        const int m = tt * 8 + 2 * t + (i & 1);
+        const int n = nt * 16 + g + ((i & 2) ? 8 : 0);
+        if (m < p.M && n < p.N)
+            p.Y[(size_t)m * p.N + n] = f32_to_bf16_bits(e[i]);
     }
-    store_tile_y<TT>(p, nt, sum, g, t);
-    if (lane == 0)
-        p.counters[nt] = 0;
 }
 
-// The E8M0 scales of one unit for lane (g, t): rows g and g + 8, block t.
-struct UnitScales {
-    float a, b;
-};
+// Sum of the kConsumers warp fragments (warp order) for this lane.
+template <int TT>
+__device__ __forceinline__ void sum_fragments(const float4 *frags, int lane, float4 (&sum)[TT])
+{
+#pragma unroll
+    for (int tt = 0; tt < TT; ++tt) {
+        sum[tt] = frags[tt * 32 + lane];
+        for (int w = 1; w < kConsumers; ++w) {
+            const float4 v = frags[w * TT * 32 + tt * 32 + lane];
+            sum[tt].x += v.x;
+            sum[tt].y += v.y;
+            sum[tt].z += v.z;
+            sum[tt].w += v.w;
+        }
+    }
+}
 
-__device__ __forceinline__ UnitScales load_unit_scales(const Params &p, int tile, int kb, int g,
-                                                       int t)
+// Run by one warp of a CTA whose segment of tile `nt` is cut (see the INT4
+// streaming kernel): the CTA holding the tile's first unit finishes it last
+// in its run and adds the other contributors' fragments in CTA order; every
+// other contributor publishes its fragment early without waiting.
+template <int TT>
+__device__ __noinline__ void finish_cut_tile(const Params &p, const float4 *frags, int c, int nt,
+                                             int lane)
+{
+    float4 sum[TT];
+    sum_fragments<TT>(frags, lane, sum);
+    const int tile_begin = nt * p.upt;
+    const int c_first = cta_of_unit(p, tile_begin);
+    if (c != c_first) {
+#pragma unroll
+        for (int tt = 0; tt < TT; ++tt)
+            __stcg(p.partial + ((size_t)c * TT + tt) * 32 + lane, sum[tt]);
+        __syncwarp();
+        if (lane == 0) {
+            __threadfence();
+            atomicAdd(&p.counters[nt], 1);
+        }
+        return;
+    }
+    const int c_last = cta_of_unit(p, tile_begin + p.upt - 1);
+    if (lane == 0) {
+        const unsigned long long t0 = global_ns();
+        while (ld_acquire_gpu(&p.counters[nt]) < c_last - c_first) {
+            if (global_ns() - t0 > kWaitLimitNs) {
+                record_error(p.hdr, MXG_ERR_TIMEOUT, 220);
+                break;
+            }
+            __nanosleep(64);
+        }
+    }
+    __syncwarp();
+    for (int cc = c_first + 1; cc <= c_last; ++cc) {
+#pragma unroll
+        for (int tt = 0; tt < TT; ++tt) {
+            const float4 f = __ldcg(p.partial + ((size_t)cc * TT + tt) * 32 + lane);
+            sum[tt].x += f.x;
+            sum[tt].y += f.y;
+            sum[tt].z += f.z;
+            sum[tt].w += f.w;
+        }
+    }
+#pragma unroll
+    for (int tt = 0; tt < TT; ++tt)
+        store_y4(p, nt, tt, lane, sum[tt]);
+    if (lane == 0)
+        p.counters[nt] = 0;  // leave the counter zero for the next call
+}
+
+// The E8M0 scales of box column kbox (128 k) for lane (g, t): rows g, g + 8,
+// block t of the box.
+__device__ __forceinline__ float2 box_scales(const Params &p, int nt, int kbox, int g, int t)
 {
     const int blocks = p.K / 32;
-    const int blk = kb * 4 + t;
-    const int ra = tile * 16 + g, rb = ra + 8;
+    const int blk = kbox * 4 + t;
+    const int ra = nt * 16 + g, rb = ra + 8;
     uint32_t ea = 127, eb = 127;  // any finite scale for zero-filled weights
     if (blk < blocks) {
         if (ra < p.N)
@@ -132,77 +177,71 @@ __device__ __forceinline__ UnitScales load_unit_scales(const Params &p, int tile
         if (rb < p.N)
             eb = __ldg(p.Ws + (size_t)rb * blocks + blk);
     }
-    return UnitScales{e8m0_to_f32(ea), e8m0_to_f32(eb)};
+    return make_float2(e8m0_to_f32(ea), e8m0_to_f32(eb));
 }
 
-template <int TT>
-__global__ void __launch_bounds__(kWarps * 32)
+// Copies unit u (SU boxes of one n16 tile) into a ring slot.
+template <int SU>
+__device__ __forceinline__ void fetch_unit(const Params &p, const CUtensorMap *map, uint8_t *slot,
+                                           uint64_t *bar, int u, uint64_t policy)
+{
+    const int nt = u / p.upt, ku = u - nt * p.upt;
+    mbar_arrive_expect_tx(bar, Unit<SU>::kBytes);
+#pragma unroll
+    for (int b = 0; b < SU; ++b)
+        tma_load_2d(slot + b * kBox, map, (ku * SU + b) * 128, nt * 16, bar, policy);
+}
+
+template <int TT, int SU>
+__global__ void __launch_bounds__(kThreads, 1)
     mxfp8_stream_kernel(const __grid_constant__ CUtensorMap wq_map, const Params p)
 {
+    using SL = Smem<TT, SU>;
+    constexpr int kStages = Unit<SU>::kStages;
     extern __shared__ uint8_t smem_raw[];
     // the 128-byte swizzle pattern needs 1024-byte aligned boxes
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float4 *red = reinterpret_cast<float4 *>(smem + SL::kRedOff);
+    int *red_count = reinterpret_cast<int *>(smem + SL::kSyncOff);  // arrivals per buffer
+    int *red_done = red_count + SL::kRed;                           // reductions per buffer
+
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int gw = blockIdx.x * kWarps + warp;
     pdl_launch_dependents();
-    if (gw >= p.Wt)
-        return;
-    const int g = lane >> 2, t = lane & 3;
-    uint8_t *ring = smem + (size_t)warp * kWarpSmem;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kWarps * kWarpSmem) + warp * kRing;
-
-    const int u0 = run_start(p, gw);
-    const int u1 = run_start(p, gw + 1);
-    const int nstages = u1 - u0;
-    int tile = u0 / p.upt;
-    int kb = u0 - tile * p.upt;
-
-    // lane 0 owns the ring; (itile, ikb) is the next unit to fetch
-    int itile = tile, ikb = kb;
+    const int c = blockIdx.x;
+    const int U0 = run_start(p, c), U1 = run_start(p, c + 1);
+    const int n = U1 - U0;
+    uint8_t *ring = smem + (size_t)warp * kStages * Unit<SU>::kBytes;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + SL::kBarOff) + warp * kStages;
     uint64_t policy = 0;
     if (lane == 0) {
         prefetch_tensormap(&wq_map);
-#pragma unroll
-        for (int s = 0; s < kRing; ++s)
-            mbar_init(&bars[s], 1);
+        for (int s = 0; s < kStages; ++s)
+            mbar_init(&full[s], 1);
         fence_barrier_init();
         policy = l2_policy_evict_first();
+    }
+    if (threadIdx.x == 0) {
+        for (int b = 0; b < 2 * SL::kRed; ++b)
+            red_count[b] = 0;
         // while the previous kernel drains: pull the first units into L2
-        {
-            int pt = tile, pk = kb;
-            for (int s = 0; s < min(kRing, nstages); ++s) {
-                prefetch_tensor_l2(&wq_map, pk * 128, pt * 16);
-                if (++pk == p.upt) {
-                    pk = 0;
-                    ++pt;
-                }
-            }
+        for (int k = 0; k < min(kConsumers * kStages, n); ++k) {
+            const int u = U0 + k, nt = u / p.upt, ku = u - nt * p.upt;
+#pragma unroll
+            for (int b = 0; b < SU; ++b)
+                prefetch_tensor_l2(&wq_map, (ku * SU + b) * 128, nt * 16);
         }
     }
+    __syncthreads();
     pdl_wait();
-    if (lane == 0) {
-        for (int s = 0; s < min(kRing, nstages); ++s) {
-            mbar_arrive_expect_tx(&bars[s], kStage);
-            tma_load_2d(ring + s * kStage, &wq_map, ikb * 128, itile * 16, &bars[s], policy);
-            if (++ikb == p.upt) {
-                ikb = 0;
-                ++itile;
-            }
-        }
-    }
-    __syncwarp();
+    // this warp takes units warp, warp + C, ... of the run; its k-th unit
+    // goes to slot k mod kStages
+    if (lane == 0)
+        for (int k = 0; k < kStages && warp + k * kConsumers < n; ++k)
+            fetch_unit<SU>(p, &wq_map, ring + k * Unit<SU>::kBytes, &full[k],
+                           U0 + warp + k * kConsumers, policy);
 
-    float acc[TT][4];
-#pragma unroll
-    for (int tt = 0; tt < TT; ++tt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-            acc[tt][e] = 0.f;
-    bool first_cut = false;
-    int first_tile = 0;
-    int seg_begin = u0;
-
+    const int g = lane >> 2, t = lane & 3;
     const uint16_t *xrow[TT];
     bool xvalid[TT];
 #pragma unroll
@@ -211,148 +250,204 @@ __global__ void __launch_bounds__(kWarps * 32)
         xvalid[tt] = m < p.M;
         xrow[tt] = p.X + (size_t)(xvalid[tt] ? m : 0) * p.K;
     }
-    UnitScales sc_next = load_unit_scales(p, tile, kb, g, t);
-    // activation fragment of unit column kb: lane (g, t) takes k = 128 kb + 32t .. +31
-    constexpr bool kPipeX = TT <= 2;
-    auto load_x = [&](uint32_t (&dst)[TT][16], int kbx) {
-        const int kl = kbx * 128 + t * 32;
-        const bool kvalid = kl < p.K;
+    const int upt = p.upt;
+    // activation fragments of one unit: for box b, lane (g, t) takes
+    // k = 128 (SU ku + b) + 32t .. +31; requested one unit ahead for narrow
+    // token tiles
+    constexpr bool kPipeX = SU * TT <= 2;
+    uint32_t xs[SU][TT][16], xn[SU][TT][16];
+    auto load_x = [&](uint32_t (&dst)[SU][TT][16], int u) {
+        const int ku = u % upt;
 #pragma unroll
-        for (int tt = 0; tt < TT; ++tt) {
+        for (int b = 0; b < SU; ++b) {
+            const int kl = (ku * SU + b) * 128 + t * 32;
+            const bool kvalid = kl < p.K;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint4 v = make_uint4(0, 0, 0, 0);
-                if (xvalid[tt] && kvalid)
-                    v = ldg128(xrow[tt] + kl + 8 * q);
-                dst[tt][4 * q + 0] = v.x;
-                dst[tt][4 * q + 1] = v.y;
-                dst[tt][4 * q + 2] = v.z;
-                dst[tt][4 * q + 3] = v.w;
-            }
+            for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint4 v = make_uint4(0, 0, 0, 0);
+                    if (xvalid[tt] && kvalid)
+                        v = ldg128(xrow[tt] + kl + 8 * q);
+                    dst[b][tt][4 * q + 0] = v.x;
+                    dst[b][tt][4 * q + 1] = v.y;
+                    dst[b][tt][4 * q + 2] = v.z;
+                    dst[b][tt][4 * q + 3] = v.w;
+                }
         }
     };
-    uint32_t xn[TT][16];
-    if (kPipeX)
-        load_x(xn, kb);
+    auto load_scales = [&](float2 (&dst)[SU], int u) {
+        const int nt = u / upt, ku = u - nt * upt;
+#pragma unroll
+        for (int b = 0; b < SU; ++b)
+            dst[b] = box_scales(p, nt, ku * SU + b, g, t);
+    };
     const int c_lo = ((2 * t) ^ g) * 16, c_hi = ((2 * t + 1) ^ g) * 16;
 
-    for (int s = 0; s < nstages; ++s) {
-        const int u = u0 + s;
-        const UnitScales sc = sc_next;
-        if (s + 1 < nstages) {
-            // scales of the next unit, one unit ahead
-            const bool wrap = kb + 1 == p.upt;
-            sc_next = load_unit_scales(p, wrap ? tile + 1 : tile, wrap ? 0 : kb + 1, g, t);
-        }
-        // activations of this unit (requested one unit ahead for narrow token tiles)
-        uint32_t xb[TT][16];
-        if (kPipeX) {
+    float acc[TT][4];
+    bool ok = true;
+    int i = warp;          // run index of this warp's next unit
+    int slot = 0;          // ring slot of unit i
+    uint32_t phase = 0;    // parity of the phase of unit i
+    float2 sc[SU], scn[SU];
+    if (i < n) {
+        load_scales(scn, U0 + i);
+        if (kPipeX)
+            load_x(xn, U0 + i);
+    }
+    int sidx = 0;          // segment of the run
+    int tile = U0 / upt;
+    for (int seg = U0; seg < U1; ++tile) {
+        const int tile_begin = tile * upt;
+        const int seg_end = min(U1, tile_begin + upt);
 #pragma unroll
-            for (int tt = 0; tt < TT; ++tt)
+        for (int tt = 0; tt < TT; ++tt)
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    xb[tt][i] = xn[tt][i];
-            if (s + 1 < nstages)
-                load_x(xn, kb + 1 == p.upt ? 0 : kb + 1);
-        } else {
-            load_x(xb, kb);
-        }
-        const int slot = s % kRing;
-        if (!mbar_wait(&bars[slot], (s / kRing) & 1, kWaitLimitNs)) {
-            if (lane == 0)
-                record_error(p.hdr, MXG_ERR_TIMEOUT, 200);
-            for (int r = s + 1; r < min(s + kRing, nstages); ++r)
-                mbar_wait(&bars[r % kRing], (r / kRing) & 1, kWaitLimitNs / 16);
-            return;
-        }
-        const uint8_t *stage = ring + slot * kStage;
-        const uint4 ra0 = lds128(stage + g * 128 + c_lo);
-        const uint4 ra1 = lds128(stage + g * 128 + c_hi);
-        const uint4 rb0 = lds128(stage + (g + 8) * 128 + c_lo);
-        const uint4 rb1 = lds128(stage + (g + 8) * 128 + c_hi);
-        const uint32_t wa[8] = {ra0.x, ra0.y, ra0.z, ra0.w, ra1.x, ra1.y, ra1.z, ra1.w};
-        const uint32_t wb[8] = {rb0.x, rb0.y, rb0.z, rb0.w, rb1.x, rb1.y, rb1.z, rb1.w};
+            for (int e = 0; e < 4; ++e)
+                acc[tt][e] = 0.f;
+        for (; U0 + i < seg_end; i += kConsumers) {
+            const int u = U0 + i;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            uint32_t a0, a1, a2, a3;
-            e4m3x4_scaled(wa[j], sc.a, a0, a2);
-            e4m3x4_scaled(wb[j], sc.b, a1, a3);
+            for (int b = 0; b < SU; ++b)
+                sc[b] = scn[b];
+            if (kPipeX) {
 #pragma unroll
-            for (int tt = 0; tt < TT; ++tt)
-                mma_bf16_16816(acc[tt], a0, a1, a2, a3, xb[tt][2 * j], xb[tt][2 * j + 1]);
-        }
-        // every lane's reads of this slot have returned, so it can be refilled
-        __syncwarp();
-        if (lane == 0 && s + kRing < nstages) {
-            mbar_arrive_expect_tx(&bars[slot], kStage);
-            tma_load_2d(ring + slot * kStage, &wq_map, ikb * 128, itile * 16, &bars[slot], policy);
-            if (++ikb == p.upt) {
-                ikb = 0;
-                ++itile;
-            }
-        }
-        if (++kb == p.upt) {
-            // a tile ends inside the run
-            if (seg_begin == tile * p.upt) {
-                store_tile_y<TT>(p, tile, acc, g, t);
+                for (int b = 0; b < SU; ++b)
+#pragma unroll
+                    for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+                        for (int k = 0; k < 16; ++k)
+                            xs[b][tt][k] = xn[b][tt][k];
+                if (i + kConsumers < n)
+                    load_x(xn, u + kConsumers);
             } else {
-                store_partial<TT>(p, gw, 0, lane, acc);
-                first_cut = true;
-                first_tile = tile;
+                load_x(xs, u);
             }
+            if (i + kConsumers < n)
+                load_scales(scn, u + kConsumers);
+            if (!mbar_wait(&full[slot], phase, ok ? kWaitLimitNs : 0)) {
+                if (ok && lane == 0)
+                    record_error(p.hdr, MXG_ERR_TIMEOUT, 200);
+                ok = false;
+            }
+            const uint8_t *st = ring + slot * Unit<SU>::kBytes;
 #pragma unroll
-            for (int tt = 0; tt < TT; ++tt)
+            for (int b = 0; b < SU; ++b) {
+                const uint8_t *box = st + b * kBox;
+                const uint4 ra0 = lds128(box + g * 128 + c_lo);
+                const uint4 ra1 = lds128(box + g * 128 + c_hi);
+                const uint4 rb0 = lds128(box + (g + 8) * 128 + c_lo);
+                const uint4 rb1 = lds128(box + (g + 8) * 128 + c_hi);
+                const uint32_t wa[8] = {ra0.x, ra0.y, ra0.z, ra0.w, ra1.x, ra1.y, ra1.z, ra1.w};
+                const uint32_t wb[8] = {rb0.x, rb0.y, rb0.z, rb0.w, rb1.x, rb1.y, rb1.z, rb1.w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    acc[tt][e] = 0.f;
-            ++tile;
-            kb = 0;
-            seg_begin = u + 1;
+                for (int j = 0; j < 8; ++j) {
+                    uint32_t a0, a1, a2, a3;
+                    e4m3x4_scaled(wa[j], sc[b].x, a0, a2);
+                    e4m3x4_scaled(wb[j], sc[b].y, a1, a3);
+#pragma unroll
+                    for (int tt = 0; tt < TT; ++tt)
+                        mma_bf16_16816(acc[tt], a0, a1, a2, a3, xs[b][tt][2 * j],
+                                       xs[b][tt][2 * j + 1]);
+                }
+            }
+            // every lane's reads of the slot have returned: refill it with
+            // this warp's unit kStages ahead
+            __syncwarp();
+            if (lane == 0 && i + kStages * kConsumers < n)
+                fetch_unit<SU>(p, &wq_map, ring + slot * Unit<SU>::kBytes, &full[slot],
+                               u + kStages * kConsumers, policy);
+            if (++slot == kStages) {
+                slot = 0;
+                phase ^= 1;
+            }
         }
-    }
 
-    // publish the cut segments (see the INT4 streaming kernel)
-    const bool last_cut = seg_begin < u1;
-    if (last_cut)
-        store_partial<TT>(p, gw, seg_begin == u0 ? 0 : 1, lane, acc);
-    if (!first_cut && !last_cut)
-        return;
-    __syncwarp();
-    int arrivals[2] = {0, 0};
-    if (lane == 0) {
-        if (first_cut)
-            arrivals[0] = atomic_add_acq_rel(&p.counters[first_tile], 1);
-        if (last_cut)
-            arrivals[1] = atomic_add_acq_rel(&p.counters[tile], 1);
-    }
-    arrivals[0] = __shfl_sync(0xffffffffu, arrivals[0], 0);
-    arrivals[1] = __shfl_sync(0xffffffffu, arrivals[1], 0);
-    if (first_cut) {
-        const int wf = warp_of_unit(p, first_tile * p.upt);
-        const int wl = warp_of_unit(p, first_tile * p.upt + p.upt - 1);
-        if (arrivals[0] == wl - wf)
-            reduce_tile<TT>(p, first_tile, lane);
-    }
-    if (last_cut) {
-        const int wf = warp_of_unit(p, tile * p.upt);
-        const int wl = warp_of_unit(p, tile * p.upt + p.upt - 1);
-        if (arrivals[1] == wl - wf)
-            reduce_tile<TT>(p, tile, lane);
+        // ---- end of the tile segment: every warp leaves its fragment in the
+        // segment's reduction buffer and goes on; the last to arrive adds them
+        const int rb = sidx % SL::kRed;
+        const int uses = sidx / SL::kRed;  // earlier segments that used buffer rb
+        if (uses > 0) {
+            if (lane == 0) {
+                const unsigned long long t0 = global_ns();
+                while (*reinterpret_cast<volatile int *>(&red_done[rb]) < uses) {
+                    if (global_ns() - t0 > kWaitLimitNs) {
+                        record_error(p.hdr, MXG_ERR_TIMEOUT, 230);
+                        break;
+                    }
+                    __nanosleep(32);
+                }
+                __threadfence_block();
+            }
+            __syncwarp();
+        }
+        float4 *frags = red + (size_t)rb * kConsumers * SL::kFrag4;
+#pragma unroll
+        for (int tt = 0; tt < TT; ++tt)
+            frags[(size_t)warp * SL::kFrag4 + tt * 32 + lane] =
+                make_float4(acc[tt][0], acc[tt][1], acc[tt][2], acc[tt][3]);
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+            __threadfence_block();
+            last = atomicAdd(&red_count[rb], 1) == kConsumers - 1;
+            __threadfence_block();
+        }
+        if (__shfl_sync(0xffffffffu, last, 0)) {
+            if (lane == 0)
+                red_count[rb] = 0;
+            const bool whole = seg == tile_begin && seg_end == tile_begin + upt;
+            if (whole) {
+                float4 sum[TT];
+                sum_fragments<TT>(frags, lane, sum);
+#pragma unroll
+                for (int tt = 0; tt < TT; ++tt)
+                    store_y4(p, tile, tt, lane, sum[tt]);
+            } else {
+                finish_cut_tile<TT>(p, frags, c, tile, lane);
+            }
+            __syncwarp();
+            if (lane == 0) {
+                __threadfence_block();
+                atomicAdd(&red_done[rb], 1);
+            }
+        }
+        ++sidx;
+        seg = seg_end;
     }
 }
 
-const void *select_kernel(int tt)
+template <int TT, int SU>
+const void *kernel_ptr()
 {
+    return reinterpret_cast<const void *>(&mxfp8_stream_kernel<TT, SU>);
+}
+
+// SU = 2 for narrow token tiles (MXG_MX_SU2_TT tiles of 8 at most), SU = 1 otherwise.
+const void *select_kernel(int tt, int su)
+{
+    if (su == 2)
+        return tt == 1 ? kernel_ptr<1, 2>() : tt == 2 ? kernel_ptr<2, 2>() : nullptr;
     switch (tt) {
-    case 1: return reinterpret_cast<const void *>(&mxfp8_stream_kernel<1>);
-    case 2: return reinterpret_cast<const void *>(&mxfp8_stream_kernel<2>);
-    case 3: return reinterpret_cast<const void *>(&mxfp8_stream_kernel<3>);
-    case 4: return reinterpret_cast<const void *>(&mxfp8_stream_kernel<4>);
+    case 1: return kernel_ptr<1, 1>();
+    case 2: return kernel_ptr<2, 1>();
+    case 3: return kernel_ptr<3, 1>();
+    case 4: return kernel_ptr<4, 1>();
     default: return nullptr;
     }
 }
 
-constexpr size_t kSmemBytes = 1024 + (size_t)kWarps * kWarpSmem + (size_t)kWarps * kRing * 8;
+size_t smem_bytes(int tt, int su)
+{
+    if (su == 2)
+        return tt == 1 ? Smem<1, 2>::kTotal : Smem<2, 2>::kTotal;
+    switch (tt) {
+    case 1: return Smem<1, 1>::kTotal;
+    case 2: return Smem<2, 1>::kTotal;
+    case 3: return Smem<3, 1>::kTotal;
+    default: return Smem<4, 1>::kTotal;
+    }
+}
 
 }  // namespace
 
@@ -363,35 +458,42 @@ bool plan_mxfp8_stream(int device, int M, int N, int K, StreamPlan *plan)
     const DeviceInfo &di = device_info(device);
     StreamPlan pl{};
     pl.tt = (M + 7) / 8;
-    pl.variant = 0;
-    pl.warps_per_cta = kWarps;
-    pl.smem = kSmemBytes;
-    pl.upt = (K + 127) / 128;
+    const int boxes = (K + 127) / 128;             // 128-k boxes per row
+    const int su = pl.tt <= MXG_MX_SU2_TT && boxes % 2 == 0 ? 2 : 1;
+    pl.variant = su;
+    pl.warps_per_cta = kConsumers;
+    pl.smem = smem_bytes(pl.tt, su);
+    if ((int)pl.smem > di.smem_optin)
+        return false;
+    pl.upt = boxes / su;
     pl.ntiles = (N + 15) / 16;
     if ((size_t)pl.ntiles > kMaxCounters)
         return false;
     pl.units = (long long)pl.ntiles * pl.upt;
     if (pl.units > (1LL << 30))
         return false;
-    const void *fn = select_kernel(pl.tt);
-    static int occ_cache[4] = {};
-    int &occ = occ_cache[pl.tt - 1];
+    const void *fn = select_kernel(pl.tt, su);
+    if (!fn)
+        return false;
+    // every CTA of the grid must be resident at once (a cut tile's finishing
+    // CTA waits for the others)
+    static int occ_cache[4][3] = {};
+    int &occ = occ_cache[pl.tt - 1][su];
     if (occ == 0) {
         if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem) !=
             cudaSuccess)
             return false;
         int o = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, fn, kWarps * 32, pl.smem) !=
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, fn, kThreads, pl.smem) !=
                 cudaSuccess ||
             o < 1)
             return false;
-        occ = o;
+        occ = std::min(o, 1);
     }
-    const long long max_warps = (long long)di.sms * occ * kWarps;
-    // no run shorter than kMinUnits units (2 KB each)
-    pl.Wt = (int)std::max<long long>(1, std::min<long long>(max_warps, pl.units / kMinUnits));
-    pl.grid = (pl.Wt + kWarps - 1) / kWarps;
-    pl.partial_bytes = (size_t)pl.Wt * 2 * 32 * 4 * pl.tt * sizeof(float);
+    pl.Wt = (int)std::max<long long>(
+        1, std::min<long long>((long long)di.sms * occ, pl.units / kMinUnitsPerCta));
+    pl.grid = pl.Wt;
+    pl.partial_bytes = (size_t)pl.Wt * pl.tt * 32 * sizeof(float4);
     *plan = pl;
     return true;
 }
@@ -400,7 +502,7 @@ cudaError_t launch_mxfp8_stream(const StreamPlan &pl, const void *X, const uint8
                                 const uint8_t *Ws, int M, int N, int K, void *Y, void *workspace,
                                 cudaStream_t stream)
 {
-    const void *fn = select_kernel(pl.tt);
+    const void *fn = select_kernel(pl.tt, pl.variant);
     if (!fn)
         return cudaErrorInvalidValue;
     alignas(64) CUtensorMap map;
@@ -414,17 +516,17 @@ cudaError_t launch_mxfp8_stream(const StreamPlan &pl, const void *X, const uint8
     p.Y = static_cast<uint16_t *>(Y);
     p.hdr = static_cast<WsHeader *>(workspace);
     p.counters = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + wm.counters_off);
-    p.partial = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + wm.partial_off);
+    p.partial = reinterpret_cast<float4 *>(static_cast<uint8_t *>(workspace) + wm.partial_off);
     p.M = M;
     p.N = N;
     p.K = K;
     p.upt = pl.upt;
     p.units = (int)pl.units;
-    p.Wt = pl.Wt;
+    p.ctas = pl.Wt;
     p.q = (int)(pl.units / pl.Wt);
     p.r = (int)(pl.units % pl.Wt);
     void *args[] = {&map, &p};
-    return launch_pdl(fn, dim3(pl.grid), dim3(kWarps * 32), pl.smem, stream, args);
+    return launch_pdl(fn, dim3(pl.grid), dim3(kThreads), pl.smem, stream, args);
 }
 
 }  // namespace mxg
