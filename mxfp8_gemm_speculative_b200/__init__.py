@@ -173,6 +173,58 @@ def w4a16_gemm(x: torch.Tensor, packed: torch.Tensor, N: int, K: int, group_size
     return out
 
 
+class PreparedCall:
+    """One library call with its arguments marshalled once, for a loop that
+    repeats it on the same buffers (a serving step).  The tensors are held
+    here so they stay alive; their contents may change between calls, their
+    storage must not move."""
+
+    def __init__(self, fn, args, what: str, keep):
+        self._fn, self._args, self._what, self._keep = fn, tuple(args), what, keep
+
+    def __call__(self) -> None:
+        status = self._fn(*self._args)
+        if status != MXG_OK:
+            raise MxgError(status, self._what)
+
+
+def prepare_w4a16_gemm(x: torch.Tensor, packed: torch.Tensor, N: int, K: int,
+                       group_size: int = 128, out: torch.Tensor | None = None,
+                       workspace_buf: torch.Tensor | None = None, stream=None):
+    """(call, out): ``call()`` runs w4a16_gemm(x, packed) into ``out``."""
+    _need(x, torch.bfloat16, "x")
+    M = x.shape[0]
+    if x.dim() != 2 or x.shape[1] != K:
+        raise ValueError("x must be [M][K]")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(out, torch.bfloat16, "out")
+    ws = (workspace_buf if workspace_buf is not None else
+          workspace(_need_bytes("w4a16", x.device.index, M, N, K, group_size), x.device, stream))
+    args = (_ptr(x), _ptr(packed), M, N, K, group_size, _ptr(out), _ptr(ws), ws.numel(),
+            _stream(stream))
+    return PreparedCall(_lib.w4a16_gemm, args, "w4a16_gemm", (x, packed, out, ws, stream)), out
+
+
+def prepare_mxfp8_gemm(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor,
+                       out: torch.Tensor | None = None, workspace_buf: torch.Tensor | None = None,
+                       stream=None):
+    """(call, out): ``call()`` runs mxfp8_gemm(x, wq, ws) into ``out``."""
+    _need(x, torch.bfloat16, "x")
+    M, K = x.shape
+    N = wq.shape[0]
+    if wq.shape[1] != K or ws.shape != (N, K // 32):
+        raise ValueError("shape mismatch between x, wq and ws")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(out, torch.bfloat16, "out")
+    wsb = (workspace_buf if workspace_buf is not None else
+           workspace(_need_bytes("mxfp8", x.device.index, M, N, K), x.device, stream))
+    args = (_ptr(x), _ptr(wq), _ptr(ws), M, N, K, _ptr(out), _ptr(wsb), wsb.numel(),
+            _stream(stream))
+    return PreparedCall(_lib.mxfp8_gemm, args, "mxfp8_gemm", (x, wq, ws, out, wsb, stream)), out
+
+
 def w4a16_gemm_static_scratch(x: torch.Tensor, packed: torch.Tensor, N: int, K: int,
                               group_size: int = 128, out: torch.Tensor | None = None,
                               stream=None) -> torch.Tensor:

@@ -241,3 +241,29 @@ def test_workspace_too_small_rejected(mxg):
     with pytest.raises(mxg.MxgError) as e:
         mxg.w4a16_gemm(bf16_tensor(lay.X, DEV), packed, 512, 1024, 128, workspace_buf=ws)
     assert e.value.status == mxg.MXG_ERR_WORKSPACE
+
+
+def test_prepared_calls_match_direct_calls(mxg):
+    """prepare_w4a16_gemm / prepare_mxfp8_gemm marshal once; each call reads the
+    buffers' current contents, so refilling x between calls behaves like a
+    fresh direct call."""
+    lay = synth.int4_layer(5, 1024, 512, 128, seed=21)
+    qw, sc = int4_device(lay)
+    packed = mxg.w4a16_repack(qw, sc, 128)
+    x = bf16_tensor(lay.X, DEV)
+    call, y = mxg.prepare_w4a16_gemm(x, packed, 512, 1024, 128)
+    for step in range(2):
+        if step:
+            x.copy_(torch.randn_like(x, dtype=torch.float32).to(torch.bfloat16))
+        call()
+        ref = mxg.w4a16_gemm(x, packed, 512, 1024, 128)
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int16), ref.view(torch.int16))
+    mlay = synth.mxfp8_layer(4, 512, 256, seed=22)
+    wq, ws = torch.from_numpy(mlay.Wq).to(DEV), torch.from_numpy(mlay.Ws).to(DEV)
+    xm = bf16_tensor(mlay.X, DEV)
+    mcall, ym = mxg.prepare_mxfp8_gemm(xm, wq, ws)
+    mcall()
+    mref = mxg.mxfp8_gemm(xm, wq, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(ym.view(torch.int16), mref.view(torch.int16))
