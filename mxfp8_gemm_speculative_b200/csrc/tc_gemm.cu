@@ -18,13 +18,15 @@
 // and activations, which keeps the pair inside the SM's shared-memory
 // bandwidth at full tensor rate.
 //
-// Warp roles per CTA (448 threads):
-//   warp 0        producer: activation and packed-weight copies;
+// Warp roles per CTA (480 threads):
+//   warp 0        producer of the activation copies;
 //   warp 1        tensor-memory allocation; in the even CTA also the single
 //                 thread that issues tcgen05.mma and tcgen05.commit;
 //   warps 2..5    epilogue;
 //   warps 6..13   dequantisers (warp w writes lanes 32*(w%4) + 16*h .. +15,
-//                 h = (w - 6) / 4).
+//                 h = (w - 6) / 4);
+//   warp 14       producer of the packed-weight copies, on a ring of its own
+//                 so the weights run ahead of the activations.
 // Every wait is an mbarrier phase wait with a time limit; a timeout sets a
 // CTA-wide abort flag, records MXG_ERR_TIMEOUT and every role drains to the
 // end, where tensor memory is released.
@@ -40,7 +42,8 @@ constexpr int BW = 128;  // weight columns per CTA
 constexpr int BK = 64;   // k per block
 constexpr int kProducerWarp = 0, kMmaWarp = 1, kEpiWarp0 = 2, kNumEpiWarps = 4;
 constexpr int kDqWarp0 = 6, kNumDqWarps = 8;
-constexpr int kThreads = (kDqWarp0 + kNumDqWarps) * 32;
+constexpr int kWProducerWarp = kDqWarp0 + kNumDqWarps;   // packed-weight loads
+constexpr int kThreads = (kWProducerWarp + 1) * 32;
 constexpr uint32_t kTmemCols = 512;
 
 enum Fmt { kInt4 = 0, kMxfp8 = 1 };
@@ -373,22 +376,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int gpk = (F == kInt4) ? max(1, BK / p.G) : 1;  // scale groups per k-block
 
     if (warp == kProducerWarp) {
+        // activations: this CTA's BT/2 tokens of every k-block, completing on
+        // the leader's barrier
         if (lane == 0) {
             prefetch_tensormap(&x_map);
-            prefetch_tensormap(&w_map);
-            if (F == kInt4)
-                prefetch_tensormap(&s_map);
-            const uint64_t pol_w = l2_policy_evict_first();
             const uint64_t pol_x = l2_policy_evict_last();
             uint32_t it = 0;
             bool ok = true;
             for (int item = pair; item < p.num_items && ok; item += npairs) {
                 int tile, kb0, kb1;
                 item_range(p, item, tile, kb0, kb1);
-                const int nb = tile / p.mtiles, mt = tile % p.mtiles;
+                const int mt = tile % p.mtiles;
                 for (int kb = kb0; kb < kb1 && ok; ++kb, ++it) {
-                    const int sx = it % L::kSX, sw = it % L::kSW;
-                    // activations: this CTA's BT/2 tokens, completing on the leader's barrier
+                    const int sx = it % L::kSX;
                     ok = role_wait(&x_empty[sx], ((it / L::kSX) & 1) ^ 1, abort_flag, p.hdr, 401);
                     if (!ok)
                         break;
@@ -397,12 +397,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     tma_load_2d_pair(smem + L::x_off + sx * L::x_slot, &x_map, kb * BK,
                                      mt * BT + (int)rank * (BT / 2),
                                      mapa_shared(smem_u32(&x_full[sx]), 0), pol_x);
-                    // packed weights of this CTA's 128 columns
+                }
+            }
+        }
+    } else if (warp == kWProducerWarp) {
+        // packed weights of this CTA's 128 columns, on their own deeper ring
+        // (not held back by the activation ring)
+        if (lane == 0) {
+            prefetch_tensormap(&w_map);
+            if (F == kInt4)
+                prefetch_tensormap(&s_map);
+            const uint64_t pol_w = l2_policy_evict_first();
+            uint32_t it = 0;
+            bool ok = true;
+            for (int item = pair; item < p.num_items && ok; item += npairs) {
+                int tile, kb0, kb1;
+                item_range(p, item, tile, kb0, kb1);
+                const int nb = tile / p.mtiles;
+                const int n32 = (nb * 2 * BW + (int)rank * BW) / 32;
+                for (int kb = kb0; kb < kb1 && ok; ++kb, ++it) {
+                    const int sw = it % L::kSW;
                     ok = role_wait(&wp_empty[sw], ((it / L::kSW) & 1) ^ 1, abort_flag, p.hdr, 402);
                     if (!ok)
                         break;
                     uint8_t *wdst = smem + L::wp_off + sw * L::wp_slot;
-                    const int n32 = (nb * 2 * BW + (int)rank * BW) / 32;
                     if (F == kInt4) {
                         mbar_arrive_expect_tx(&wp_full[sw], 4096u + 256u * gpk);
                         tma_load_2d(wdst, &w_map, kb * 128, n32, &wp_full[sw], pol_w);
@@ -551,7 +569,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
             }
         }
-    } else {
+    } else if (warp >= kDqWarp0 && warp < kDqWarp0 + kNumDqWarps) {
         // dequantisers: warp -> (quadrant q, half h) of the CTA's 128 weight rows
         const int dw = warp - kDqWarp0;
         const int q = warp & 3, h = dw >> 2;
