@@ -37,6 +37,16 @@
  *    status word (read it with mxg_workspace_status) and the kernel returns.
  *  - The GPU path does not scan inputs: NaN E4M3 codes (0x7F / 0xFF), E8M0
  *    0xFF and non-finite scales give unspecified output.
+ *  - GEMM kernels are launched with programmatic dependent launch: they may
+ *    start while the previous kernel on `stream` drains, and wait for it
+ *    before they read X or touch Y and the workspace.  The weight-streaming
+ *    kernels (M <= 32) also start loading WEIGHTS (packed, Wq, Ws) before
+ *    that wait, unless mxg_set_early_weight_loads(0) was called: the weight
+ *    buffers must then not be written by the kernel immediately before the
+ *    GEMM on `stream`.  w4a16_repack ends with a kernel that writes nothing,
+ *    so a GEMM may follow it directly; any other writer of weights needs
+ *    another launch, or a synchronization, between it and the GEMM (in
+ *    serving, weights are written once at load time).
  */
 #ifndef MXG_H
 #define MXG_H
@@ -174,6 +184,13 @@ MXG_API int mxg_selftest_wait_timeout(void *workspace, int limit_us, cudaStream_
  * 0 = automatic (default), 1 = weight-streaming path, 2 = tensor-core path.
  * The streaming path accepts M <= 32 only.  Returns the previous setting. */
 MXG_API int mxg_set_path(int path);
+
+/* Early weight loads of the weight-streaming kernels (process-wide):
+ * 1 = load the first weight tiles before waiting for the previous kernel on
+ * the stream (default), 0 = load everything after that wait, for callers
+ * that write weights in the kernel right before a GEMM.  Returns the
+ * previous setting, or -1 for a value other than 0 and 1. */
+MXG_API int mxg_set_early_weight_loads(int on);
 
 #ifdef __cplusplus
 }

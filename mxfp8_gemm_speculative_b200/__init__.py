@@ -50,6 +50,7 @@ _SIGS = {
     "mxg_workspace_status": (_i, [_p, ctypes.POINTER(_i), _p]),
     "mxg_selftest_wait_timeout": (_i, [_p, _i, _p]),
     "mxg_set_path": (_i, [_i]),
+    "mxg_set_early_weight_loads": (_i, [_i]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -134,8 +135,9 @@ def w4a16_packed_bytes(K: int, N: int, group_size: int = 128) -> int:
 
 
 def w4a16_repack(qweight: torch.Tensor, scales: torch.Tensor, group_size: int = 128,
-                 stream=None) -> torch.Tensor:
-    """Re-pack GPTQ words qweight[K/8][N] (int32) and scales[K/G][N] (fp16)."""
+                 stream=None, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Re-pack GPTQ words qweight[K/8][N] (int32) and scales[K/G][N] (fp16),
+    into `out` (uint8, w4a16_packed_bytes bytes) when given."""
     _need(qweight, torch.int32, "qweight")
     if scales.dtype not in (torch.float16, torch.int16):
         raise ValueError("scales must be float16 (or its int16 bit view)")
@@ -145,7 +147,13 @@ def w4a16_repack(qweight: torch.Tensor, scales: torch.Tensor, group_size: int = 
     nbytes = w4a16_packed_bytes(K, N, group_size)
     if nbytes == 0:
         raise MxgError(MXG_ERR_UNSUPPORTED_SHAPE, "w4a16_repack")
-    packed = torch.empty(nbytes, dtype=torch.uint8, device=qweight.device)
+    if out is None:
+        packed = torch.empty(nbytes, dtype=torch.uint8, device=qweight.device)
+    else:
+        _need(out, torch.uint8, "out")
+        if out.numel() != nbytes or out.device != qweight.device:
+            raise ValueError(f"out must hold {nbytes} bytes on {qweight.device}")
+        packed = out
     _check(_lib.w4a16_repack(_ptr(qweight), _ptr(scales), K, N, group_size, _ptr(packed),
                              _stream(stream)), "w4a16_repack")
     return packed
@@ -308,6 +316,17 @@ def mxg_set_path(path: int) -> int:
     r = int(_lib.mxg_set_path(int(path)))
     if r < 0:
         raise ValueError("path must be 0, 1 or 2")
+    return r
+
+
+def mxg_set_early_weight_loads(on: int) -> int:
+    """1 (default): the weight-streaming kernels load their first weight tiles
+    before waiting for the previous kernel on the stream; 0: after it, for
+    callers that write weights in the kernel right before a GEMM.  Returns
+    the previous value."""
+    r = int(_lib.mxg_set_early_weight_loads(int(on)))
+    if r < 0:
+        raise ValueError("on must be 0 or 1")
     return r
 
 

@@ -20,6 +20,7 @@ constexpr int kMaxDevices = 64;
 DeviceInfo g_info[kMaxDevices];
 std::once_flag g_info_once[kMaxDevices];
 std::atomic<int> g_path{0};
+std::atomic<int> g_early_weights{1};
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
@@ -61,6 +62,11 @@ bool mxfp8_shape_ok(int K, int N)
     return K > 0 && N >= 128 && K % 32 == 0;
 }
 }  // namespace
+
+bool early_weight_loads()
+{
+    return g_early_weights.load(std::memory_order_relaxed) != 0;
+}
 
 const DeviceInfo &device_info(int device)
 {
@@ -350,6 +356,13 @@ int mxg_set_path(int path)
     if (path < 0 || path > 2)
         return -1;
     return g_path.exchange(path);
+}
+
+int mxg_set_early_weight_loads(int on)
+{
+    if (on != 0 && on != 1)
+        return -1;
+    return g_early_weights.exchange(on);
 }
 
 }  // extern "C"

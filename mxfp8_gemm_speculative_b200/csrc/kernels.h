@@ -48,6 +48,11 @@ struct StreamPlan {
     int ntiles;           // output tiles (= arrival counters)
 };
 
+// Whether the streaming kernels load their first weights before waiting for
+// the previous kernel on the stream (process-wide, default on; see
+// mxg_set_early_weight_loads).
+bool early_weight_loads();
+
 bool plan_w4a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan);
 cudaError_t launch_w4a16_stream(const StreamPlan &plan, const void *X, const void *packed, int M,
                                 int N, int K, int G, void *Y, void *workspace, cudaStream_t stream);

@@ -65,6 +65,7 @@ struct Params {
     int units;
     int ctas;
     int q, r;                // units = q * ctas + r: CTAs below r run q + 1 units, the rest q
+    int early;               // load the first weights before waiting for the previous kernel
 };
 
 // First unit of CTA c's run.
@@ -233,13 +234,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     __syncthreads();
-    pdl_wait();
     // this warp takes units warp, warp + C, ... of the run; its k-th unit
-    // goes to slot k mod kStages
-    if (lane == 0)
-        for (int k = 0; k < kStages && warp + k * kConsumers < n; ++k)
-            fetch_unit<SU>(p, &wq_map, ring + k * Unit<SU>::kBytes, &full[k],
-                           U0 + warp + k * kConsumers, policy);
+    // goes to slot k mod kStages.  The weights are not written by the
+    // previous kernel on the stream (the caller's contract, unless it turned
+    // early weight loads off): the first slots fill while that kernel drains.
+    auto fill_ring = [&]() {
+        if (lane == 0)
+            for (int k = 0; k < kStages && warp + k * kConsumers < n; ++k)
+                fetch_unit<SU>(p, &wq_map, ring + k * Unit<SU>::kBytes, &full[k],
+                               U0 + warp + k * kConsumers, policy);
+    };
+    if (p.early)
+        fill_ring();
+    pdl_wait();
+    if (!p.early)
+        fill_ring();
 
     const int g = lane >> 2, t = lane & 3;
     const uint16_t *xrow[TT];
@@ -514,6 +523,7 @@ cudaError_t launch_mxfp8_stream(const StreamPlan &pl, const void *X, const uint8
     p.X = static_cast<const uint16_t *>(X);
     p.Ws = Ws;
     p.Y = static_cast<uint16_t *>(Y);
+    p.early = early_weight_loads() ? 1 : 0;
     p.hdr = static_cast<WsHeader *>(workspace);
     p.counters = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + wm.counters_off);
     p.partial = reinterpret_cast<float4 *>(static_cast<uint8_t *>(workspace) + wm.partial_off);

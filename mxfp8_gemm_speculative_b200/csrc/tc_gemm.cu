@@ -81,6 +81,7 @@ struct TcParams {
     int num_tiles;
     int splits;            // K splits per output tile
     int num_items;         // num_tiles * splits work items
+    int early;             // load the first weights before waiting for the previous kernel
 };
 
 // Work item -> output tile and its k-block range [kb0, kb1).
@@ -370,10 +371,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tc_fence_before();
     cluster_sync();   // barriers of both CTAs initialised, tensor memory allocated
     tc_fence_after();
-    pdl_wait();
     const uint32_t tmem_base = *tmem_slot;
 
     const int gpk = (F == kInt4) ? max(1, BK / p.G) : 1;  // scale groups per k-block
+
+    // Packed weights of this CTA's 128 columns (lane 0 of the weight
+    // producer), on their own deeper ring, not held back by the activation
+    // ring.  w_issue(n) issues the loads of the CTA's k-blocks in order until
+    // n of them have been issued.
+    int w_item = pair, w_tile = 0, w_kb = 0, w_kb1 = 0;
+    uint32_t w_it = 0;
+    if (w_item < p.num_items)
+        item_range(p, w_item, w_tile, w_kb, w_kb1);
+    auto w_issue = [&](uint32_t until) -> bool {
+        const uint64_t pol_w = l2_policy_evict_first();
+        while (w_item < p.num_items && w_it < until) {
+            if (w_kb >= w_kb1) {
+                w_item += npairs;
+                if (w_item < p.num_items)
+                    item_range(p, w_item, w_tile, w_kb, w_kb1);
+                continue;
+            }
+            const int sw = w_it % L::kSW;
+            if (!role_wait(&wp_empty[sw], ((w_it / L::kSW) & 1) ^ 1, abort_flag, p.hdr, 402))
+                return false;
+            const int nb = w_tile / p.mtiles;
+            const int n32 = (nb * 2 * BW + (int)rank * BW) / 32;
+            uint8_t *wdst = smem + L::wp_off + sw * L::wp_slot;
+            if (F == kInt4) {
+                mbar_arrive_expect_tx(&wp_full[sw], 4096u + 256u * gpk);
+                tma_load_2d(wdst, &w_map, w_kb * 128, n32, &wp_full[sw], pol_w);
+                tma_load_2d(wdst + 4096, &s_map, (w_kb * BK / p.G) * 8, n32, &wp_full[sw], pol_w);
+            } else {
+                mbar_arrive_expect_tx(&wp_full[sw], (uint32_t)(BW * BK));
+                tma_load_2d(wdst, &w_map, w_kb * BK, n32 * 32, &wp_full[sw], pol_w);
+            }
+            ++w_kb;
+            ++w_it;
+        }
+        return true;
+    };
+    if (warp == kWProducerWarp && lane == 0) {
+        prefetch_tensormap(&w_map);
+        if (F == kInt4)
+            prefetch_tensormap(&s_map);
+        // The weights are not written by the previous kernel on the stream
+        // (the caller's contract, unless it turned early weight loads off):
+        // the first ring of them fills while that kernel drains.  Everything
+        // else waits for it.
+        if (p.early)
+            w_issue(L::kSW);
+    }
+    pdl_wait();
 
     if (warp == kProducerWarp) {
         // activations: this CTA's BT/2 tokens of every k-block, completing on
@@ -401,38 +450,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp == kWProducerWarp) {
-        // packed weights of this CTA's 128 columns, on their own deeper ring
-        // (not held back by the activation ring)
-        if (lane == 0) {
-            prefetch_tensormap(&w_map);
-            if (F == kInt4)
-                prefetch_tensormap(&s_map);
-            const uint64_t pol_w = l2_policy_evict_first();
-            uint32_t it = 0;
-            bool ok = true;
-            for (int item = pair; item < p.num_items && ok; item += npairs) {
-                int tile, kb0, kb1;
-                item_range(p, item, tile, kb0, kb1);
-                const int nb = tile / p.mtiles;
-                const int n32 = (nb * 2 * BW + (int)rank * BW) / 32;
-                for (int kb = kb0; kb < kb1 && ok; ++kb, ++it) {
-                    const int sw = it % L::kSW;
-                    ok = role_wait(&wp_empty[sw], ((it / L::kSW) & 1) ^ 1, abort_flag, p.hdr, 402);
-                    if (!ok)
-                        break;
-                    uint8_t *wdst = smem + L::wp_off + sw * L::wp_slot;
-                    if (F == kInt4) {
-                        mbar_arrive_expect_tx(&wp_full[sw], 4096u + 256u * gpk);
-                        tma_load_2d(wdst, &w_map, kb * 128, n32, &wp_full[sw], pol_w);
-                        tma_load_2d(wdst + 4096, &s_map, (kb * BK / p.G) * 8, n32, &wp_full[sw],
-                                    pol_w);
-                    } else {
-                        mbar_arrive_expect_tx(&wp_full[sw], (uint32_t)(BW * BK));
-                        tma_load_2d(wdst, &w_map, kb * BK, n32 * 32, &wp_full[sw], pol_w);
-                    }
-                }
-            }
-        }
+        if (lane == 0)
+            w_issue(0xffffffffu);
     } else if (warp == kMmaWarp) {
         if (rank == 0 && lane == 0) {
             constexpr uint32_t idesc = idesc_pair<BT>();
@@ -744,6 +763,7 @@ cudaError_t launch_w4a16_tc(const TcPlan &pl, const void *X, const void *packed,
     p.num_tiles = pl.mtiles * pl.ntiles;
     p.splits = pl.splits;
     p.num_items = p.num_tiles * pl.splits;
+    p.early = early_weight_loads() ? 1 : 0;
     {
         const WorkspaceMap wsm = make_workspace_map(pl.counters, pl.partial_bytes);
         p.counters = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + wsm.counters_off);
@@ -782,6 +802,7 @@ cudaError_t launch_mxfp8_tc(const TcPlan &pl, const void *X, const uint8_t *Wq,
     p.num_tiles = pl.mtiles * pl.ntiles;
     p.splits = pl.splits;
     p.num_items = p.num_tiles * pl.splits;
+    p.early = early_weight_loads() ? 1 : 0;
     {
         const WorkspaceMap wsm = make_workspace_map(pl.counters, pl.partial_bytes);
         p.counters = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + wsm.counters_off);

@@ -97,6 +97,7 @@ struct Params {
     int units;
     int ctas;
     int q, r;                // units = q * ctas + r: CTAs below r run q + 1 units, the rest q
+    int early;               // load the first weights before waiting for the previous kernel
 };
 
 // First unit of CTA c's run.
@@ -257,12 +258,21 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) w4a16_stream_kernel(cons
         prefetch_l2(p.scales + (size_t)U0 * MD::kScale, nu * MD::kScale);
     }
     __syncthreads();
-    pdl_wait();
     // this warp takes units warp, warp + C, ... of the run; its k-th unit
-    // goes to slot k mod kStages
-    if (lane == 0)
-        for (int k = 0; k < kStages && warp + k * kConsumers < n; ++k)
-            fetch_unit<GM, SU>(p, ring + k * SL::kSlot, &full[k], U0 + warp + k * kConsumers, policy);
+    // goes to slot k mod kStages.  The weights are not written by the
+    // previous kernel on the stream (the caller's contract, unless it turned
+    // early weight loads off): the first slots fill while that kernel drains.
+    auto fill_ring = [&]() {
+        if (lane == 0)
+            for (int k = 0; k < kStages && warp + k * kConsumers < n; ++k)
+                fetch_unit<GM, SU>(p, ring + k * SL::kSlot, &full[k], U0 + warp + k * kConsumers,
+                                   policy);
+    };
+    if (p.early)
+        fill_ring();
+    pdl_wait();
+    if (!p.early)
+        fill_ring();
 
     // ------------------------------------------------------------ consumers
     const int g = lane >> 2, t = lane & 3;
@@ -585,6 +595,7 @@ cudaError_t launch_w4a16_stream(const StreamPlan &pl, const void *X, const void 
     p.codes = static_cast<const uint8_t *>(packed);
     p.scales = p.codes + (size_t)N * K / 2;
     p.Y = static_cast<uint16_t *>(Y);
+    p.early = early_weight_loads() ? 1 : 0;
     p.hdr = static_cast<WsHeader *>(workspace);
     p.counters = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + wm.counters_off);
     p.partial = reinterpret_cast<float4 *>(static_cast<uint8_t *>(workspace) + wm.partial_off);

@@ -178,6 +178,11 @@ __global__ void wait_timeout_kernel(WsHeader *hdr, unsigned long long limit_ns)
     }
 }
 
+// Launched after the re-pack kernels: a GEMM right after w4a16_repack on the
+// stream may load weights before it waits for the kernel before it, which is
+// then this one (it starts only once the re-pack kernels have completed).
+__global__ void repack_done_kernel() {}
+
 inline unsigned blocks_for(long long total, int threads)
 {
     return (unsigned)((total + threads - 1) / threads);
@@ -194,6 +199,7 @@ cudaError_t launch_w4a16_repack(const int32_t *qweight, const uint16_t *scales, 
     const long long nsc = (long long)(N / 32) * (K / G) * 32;
     uint16_t *sc_out = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(packed) + (size_t)N * K / 2);
     repack_scales_kernel<<<blocks_for(nsc, 256), 256, 0, stream>>>(scales, K, N, G, sc_out);
+    repack_done_kernel<<<1, 32, 0, stream>>>();
     return cudaGetLastError();
 }
 

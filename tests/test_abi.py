@@ -84,3 +84,11 @@ def test_path_override_roundtrip(mxg):
     assert mxg.mxg_set_path(prev) == 2
     with pytest.raises(ValueError):
         mxg.mxg_set_path(3)
+
+
+def test_early_weight_loads_roundtrip(mxg):
+    assert mxg.mxg_set_early_weight_loads(0) == 1  # on by default
+    assert mxg.mxg_set_early_weight_loads(1) == 0
+    with pytest.raises(ValueError):
+        mxg.mxg_set_early_weight_loads(2)
+    assert mxg.mxg_set_early_weight_loads(1) == 1

@@ -267,3 +267,46 @@ def test_prepared_calls_match_direct_calls(mxg):
     mref = mxg.mxfp8_gemm(xm, wq, ws)
     torch.cuda.synchronize()
     assert torch.equal(ym.view(torch.int16), mref.view(torch.int16))
+
+
+def test_early_weight_loads_match_late_loads(mxg):
+    """Weight tiles loaded before the wait for the previous kernel give the
+    same bits as loads after it; a GEMM issued right after w4a16_repack
+    re-packs new weights into a reused buffer and sees the new weights."""
+    lay = synth.int4_layer(5, 2048, 1024, 128, seed=31)
+    lay2 = synth.int4_layer(5, 2048, 1024, 128, seed=32)
+    qw, sc = int4_device(lay)
+    qw2, sc2 = int4_device(lay2)
+    x = bf16_tensor(lay.X, DEV)
+    packed = mxg.w4a16_repack(qw, sc, 128)
+    outs = {}
+    prev = mxg.mxg_set_early_weight_loads(1)
+    try:
+        for early in (1, 0):
+            mxg.mxg_set_early_weight_loads(early)
+            y1 = mxg.w4a16_gemm(x, packed, 1024, 2048, 128)
+            # re-pack other weights into the same buffer, GEMM right after
+            mxg.w4a16_repack(qw2, sc2, 128, out=packed)
+            y2 = mxg.w4a16_gemm(x, packed, 1024, 2048, 128)
+            mxg.w4a16_repack(qw, sc, 128, out=packed)
+            torch.cuda.synchronize()
+            outs[early] = (y1, y2)
+    finally:
+        mxg.mxg_set_early_weight_loads(prev)
+    for a, b in zip(outs[1], outs[0]):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    ref2 = oracle.w4a16_gemm(lay.X, lay2.qweight, lay2.scales, 5, 1024, 2048, 128)
+    assert_parity(to_f64(outs[1][1]), ref2, "GEMM right after re-pack")
+    mlay = synth.mxfp8_layer(4, 512, 256, seed=33)
+    wq, ws = torch.from_numpy(mlay.Wq).to(DEV), torch.from_numpy(mlay.Ws).to(DEV)
+    xm = bf16_tensor(mlay.X, DEV)
+    mouts = []
+    prev = mxg.mxg_set_early_weight_loads(1)
+    try:
+        for early in (1, 0):
+            mxg.mxg_set_early_weight_loads(early)
+            mouts.append(mxg.mxfp8_gemm(xm, wq, ws))
+    finally:
+        mxg.mxg_set_early_weight_loads(prev)
+    torch.cuda.synchronize()
+    assert torch.equal(mouts[0].view(torch.int16), mouts[1].view(torch.int16))
