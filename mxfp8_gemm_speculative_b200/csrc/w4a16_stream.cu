@@ -278,13 +278,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) w4a16_stream_kernel(cons
     const int g = lane >> 2, t = lane & 3;
     // activation rows of this lane: m = g + 8 tt; the lane reads k = 4t .. 4t+3
     // of every k16 step
+    // (rows m >= M read row 0 instead: their outputs are never stored)
     const uint16_t *xrow[TT];
-    bool xvalid[TT];
 #pragma unroll
     for (int tt = 0; tt < TT; ++tt) {
         const int m = tt * 8 + g;
-        xvalid[tt] = m < p.M;
-        xrow[tt] = p.X + (size_t)(xvalid[tt] ? m : 0) * p.K + 4 * t;
+        xrow[tt] = p.X + (size_t)(m < p.M ? m : 0) * p.K + 4 * t;
     }
     const int upt = p.upt;
 
@@ -292,20 +291,24 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) w4a16_stream_kernel(cons
     // token tiles (a whole unit of work hides their L2 latency).
     constexpr bool kPipeX = MD::kChunks * TT <= 4;
     uint2 xs[MD::kChunks][TT][4], xn[MD::kChunks][TT][4];
-    auto load_x = [&](uint2 (&dst)[MD::kChunks][TT][4], int u) {
-        const int kc = (u % upt) * MD::kChunks;  // first k64 chunk of unit u
+    // ku: the unit's place in its tile
+    auto load_x = [&](uint2 (&dst)[MD::kChunks][TT][4], int ku) {
+        const int kc = ku * MD::kChunks;  // first k64 chunk of the unit
 #pragma unroll
         for (int ch = 0; ch < MD::kChunks; ++ch)
 #pragma unroll
             for (int tt = 0; tt < TT; ++tt)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    uint2 v = make_uint2(0, 0);
-                    if (xvalid[tt])
-                        v = __ldg(reinterpret_cast<const uint2 *>(xrow[tt] + (kc + ch) * 64 +
-                                                                  16 * j));
-                    dst[ch][tt][j] = v;
-                }
+                for (int j = 0; j < 4; ++j)
+                    dst[ch][tt][j] = __ldg(
+                        reinterpret_cast<const uint2 *>(xrow[tt] + (kc + ch) * 64 + 16 * j));
+    };
+    // place in its tile of the unit kConsumers further on
+    auto next_ku = [&](int ku) {
+        ku += kConsumers;
+        while (ku >= upt)
+            ku -= upt;
+        return ku;
     };
 
     constexpr uint32_t kOnes = 0x3F803F80u;  // bf16 pair (1, 1)
@@ -314,8 +317,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) w4a16_stream_kernel(cons
     int i = warp;          // run index of this warp's next unit
     int slot = 0;          // ring slot of unit i
     uint32_t phase = 0;    // parity of the phase of unit i
+    int ku = (U0 + i) % upt;  // place of unit i in its tile
     if (kPipeX && i < n)
-        load_x(xs, U0 + i);
+        load_x(xs, ku);
     int sidx = 0;          // segment of the run
     int tile = U0 / upt;
     for (int seg = U0; seg < U1; ++tile) {
@@ -324,12 +328,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) w4a16_stream_kernel(cons
         zero_acc<TT>(acc);
         for (; U0 + i < seg_end; i += kConsumers) {
             const int u = U0 + i;
+            const int ku_next = next_ku(ku);
             if (kPipeX) {
                 if (i + kConsumers < n)
-                    load_x(xn, u + kConsumers);
+                    load_x(xn, ku_next);
             } else {
-                load_x(xs, u);
+                load_x(xs, ku);
             }
+            ku = ku_next;
             if (!mbar_wait(&full[slot], phase, ok ? kWaitLimitNs : 0)) {
                 if (ok && lane == 0)
                     record_error(p.hdr, MXG_ERR_TIMEOUT, 100 + GM);
