@@ -36,7 +36,9 @@ constexpr int kMinUnitsPerCta = 2 * kConsumers; // shortest run
 template <int SU>
 struct Unit {
     static constexpr int kBytes = SU * kBox;
-    static constexpr int kStages = SU == 2 ? 3 : 5;  // ring slots per warp
+    // ring slots per warp: shallow rings leave most of the SM's
+    // shared-memory/L1 split to L1, where the re-read activations hit
+    static constexpr int kStages = SU == 2 ? 2 : 3;
 };
 
 // Shared memory (1024-byte aligned for the swizzle): every warp's ring,
@@ -45,7 +47,9 @@ struct Unit {
 template <int TT, int SU>
 struct Smem {
     static constexpr int kFrag4 = TT * 32;       // float4 per warp fragment
-    static constexpr int kRed = TT == 1 ? 4 : 2;
+    // one reduction buffer: the smaller footprint leaves a larger L1 for the
+    // activation loads (every CTA re-reads X for each of its tiles)
+    static constexpr int kRed = 1;
     static constexpr size_t kRingBytes = (size_t)kConsumers * Unit<SU>::kStages * Unit<SU>::kBytes;
     static constexpr size_t kRedOff = kRingBytes;
     static constexpr size_t kBarOff = kRedOff + (size_t)kRed * kConsumers * kFrag4 * 16;

@@ -45,7 +45,7 @@ namespace {
 #define MXG_STREAM_CTAS_PER_SM 1
 #endif
 #ifndef MXG_STREAM_STAGES_BIG
-#define MXG_STREAM_STAGES_BIG 3
+#define MXG_STREAM_STAGES_BIG 2
 #endif
 constexpr int kConsumers = MXG_STREAM_CONSUMERS;  // warps per CTA
 constexpr int kThreads = kConsumers * 32;
@@ -62,7 +62,10 @@ struct Mode {
     static constexpr int kStepsPerGroup = kG / 16;            // MMA k16 steps per group
     static constexpr int kCode = kChunks * 1024;              // code bytes per unit
     static constexpr int kScale = kGroups * 64;               // scale bytes per unit
-    static constexpr int kStages = kCode >= 4096 ? MXG_STREAM_STAGES_BIG : 5;  // slots per warp
+    // slots per warp: shallow rings (12 warps x 2-3 slots keep enough bytes in
+    // flight) leave most of the SM's shared-memory/L1 split to L1, where the
+    // re-read activations hit
+    static constexpr int kStages = kCode >= 4096 ? MXG_STREAM_STAGES_BIG : 3;
 };
 
 // Shared memory: every warp's ring of kStages slots (a slot holds one
@@ -74,7 +77,11 @@ struct Smem {
     using MD = Mode<GM, SU>;
     static constexpr int kFrag4 = 2 * TT * 32;                // float4 per warp fragment
     static constexpr int kSlot = (MD::kCode + MD::kScale + 127) / 128 * 128;
-    static constexpr int kRed = TT == 1 ? 4 : 2;
+    // One reduction buffer: a warp that ends a segment before the previous
+    // segment's reduction is done waits for it (rarely), and the smaller
+    // shared-memory footprint leaves a larger L1 for the activation loads
+    // (every CTA re-reads X for each of its tiles).
+    static constexpr int kRed = 1;
     static constexpr size_t kRingBytes = (size_t)kConsumers * MD::kStages * kSlot;
     static constexpr size_t kRedBytes = (size_t)kRed * kConsumers * kFrag4 * 16;
     static constexpr size_t kBarBytes = (size_t)kConsumers * MD::kStages * 8;
