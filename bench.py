@@ -42,6 +42,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # workload -> (format, M, [(K, N)], group)
 WORKLOADS = {
     "mtp4_verify_int4": ("int4", 5, [(5120, 5120), (5120, 17408), (17408, 5120)], 128),
+    # the same step with the MLP gate and up projections fused into one
+    # 5120 -> 34816 layer (two 17408-column parts in one re-packed buffer)
+    "mtp4_verify_int4_fused": ("int4", 5, [(5120, 5120), (5120, 34816), (17408, 5120)], 128),
     "tiny_int4": ("int4", 1, [(512, 512)], 128),
     "c32_mtp3_int4": ("int4", 128, [(5120, 17408), (17408, 5120)], 128),
     "prefill_int4": ("int4", 8192, [(5120, 17408)], 128),
@@ -49,6 +52,8 @@ WORKLOADS = {
     "mxfp8_m128": ("mxfp8", 128, [(5120, 17408)], 32),
 }
 TENSOR_BOUND = {"c32_mtp3_int4", "prefill_int4", "mxfp8_m128"}
+# (workload, layer index) -> column counts of the projections fused into it
+FUSED_PARTS = {("mtp4_verify_int4_fused", 1): (17408, 17408)}
 
 
 def layer_weight_bytes(fmt, K, N, G):
@@ -172,7 +177,16 @@ def run_ours(args, rank, world, local_rank):
             lay = synth.int4_layer(M, K, N, G, seed=rank, layer=li)
             qw = torch.from_numpy(lay.qweight).to(dev)
             sc = torch.from_numpy(lay.scales.view(np.int16)).to(dev)
-            packed = mxg.w4a16_repack(qw, sc, G)
+            parts = FUSED_PARTS.get((args.workload, li))
+            if parts:
+                # fused projections: the parts' columns of the seeded layer,
+                # re-packed into one buffer
+                bounds = np.cumsum((0,) + parts)
+                packed = mxg.w4a16_repack_fused(
+                    [(qw[:, a:b].contiguous(), sc[:, a:b].contiguous())
+                     for a, b in zip(bounds[:-1], bounds[1:])], G)
+            else:
+                packed = mxg.w4a16_repack(qw, sc, G)
             del qw, sc
             weights.append([packed] + [packed.clone() for _ in range(pool - 1)])
             wss.append(torch.zeros(mxg.w4a16_workspace_bytes(M, N, K, G), dtype=torch.uint8,

@@ -97,6 +97,41 @@ MXG_API size_t w4a16_packed_bytes(int K, int N, int group_size);
 MXG_API int w4a16_repack(const int32_t *qweight, const uint16_t *scales,
                  int K, int N, int group_size, void *packed, cudaStream_t stream);
 
+/* The same re-pack from the compressed-tensors export of the same weights
+ * (the Eole recipe, section "Compressed-tensors INT4 layout": symmetric
+ * grouped W4A16 "pack-quantized" weights, which its converter only
+ * transposes into the GPTQ layout, without re-quantizing).
+ *   weight_packed  device, int32 [N][K/8]: word (n, i) holds the codes of
+ *                  rows k = 8i + j, j = 0..7, in bits [4j, 4j+3] (LSB first),
+ *                  the same code values as GPTQ (w = (q - 8) * scale).
+ *   weight_scale   device, fp16 bits [N][K/G].
+ *   packed         as for w4a16_repack; the bytes written are identical to
+ *                  w4a16_repack of the transposed words and scales.
+ * Requirements and errors as for w4a16_repack. */
+MXG_API int w4a16_repack_ct(const int32_t *weight_packed, const uint16_t *weight_scale,
+                 int K, int N, int group_size, void *packed, cudaStream_t stream);
+
+/* Fused projections (the Eole recipe, section "Pack inference projections":
+ * K/V/Q and gate/up projections that share their input are packed into one
+ * projection before the kernel re-pack, to cut launches per step).  Re-packs
+ * `count` GPTQ weights with the same K and group size, part i having Ns[i]
+ * columns, into ONE buffer for a layer of N = sum Ns[i] columns: part i is
+ * columns [Ns[0] + ... + Ns[i-1], ... + Ns[i]) of that layer (the bytes equal
+ * w4a16_repack of the parts' words and scales concatenated along N).  A
+ * w4a16_gemm with N = sum Ns[i] then computes every part in one launch, Y
+ * holding the parts' outputs side by side.
+ *   count            1..64;
+ *   qweights, scales host arrays of `count` device pointers (GPTQ layout,
+ *                    int32 [K/8][Ns[i]] and fp16 bits [K/G][Ns[i]]);
+ *   Ns               host array of `count` column counts;
+ *   packed           device, w4a16_packed_bytes(K, sum Ns[i], G) bytes.
+ * Requirements: every part as for w4a16_repack (so each Ns[i] % 64 == 0).
+ * Errors as for w4a16_repack; MXG_ERR_INVALID_ARG for a NULL array or a
+ * count outside 1..64. */
+MXG_API int w4a16_repack_fused(int count, const int32_t *const *qweights,
+                 const uint16_t *const *scales, const int *Ns, int K, int group_size,
+                 void *packed, cudaStream_t stream);
+
 /* Workspace bytes w4a16_gemm needs for this shape on the current device
  * (split-K partial sums, arrival counters and the status word). */
 MXG_API size_t w4a16_workspace_bytes(int M, int N, int K, int group_size);

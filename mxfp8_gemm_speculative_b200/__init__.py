@@ -40,6 +40,8 @@ _SIGS = {
     "mxg_status_string": (ctypes.c_char_p, [_i]),
     "w4a16_packed_bytes": (_sz, [_i, _i, _i]),
     "w4a16_repack": (_i, [_p, _p, _i, _i, _i, _p, _p]),
+    "w4a16_repack_ct": (_i, [_p, _p, _i, _i, _i, _p, _p]),
+    "w4a16_repack_fused": (_i, [_i, _p, _p, _p, _i, _i, _p, _p]),
     "w4a16_workspace_bytes": (_sz, [_i, _i, _i, _i]),
     "w4a16_gemm": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _sz, _p]),
     "w4a16_gemm_static_scratch": (_i, [_p, _p, _i, _i, _i, _i, _p, _p]),
@@ -134,28 +136,75 @@ def w4a16_packed_bytes(K: int, N: int, group_size: int = 128) -> int:
     return int(_lib.w4a16_packed_bytes(K, N, group_size))
 
 
+def _repack_out(words: torch.Tensor, K: int, N: int, group_size: int, out, what: str):
+    nbytes = w4a16_packed_bytes(K, N, group_size)
+    if nbytes == 0:
+        raise MxgError(MXG_ERR_UNSUPPORTED_SHAPE, what)
+    if out is None:
+        return torch.empty(nbytes, dtype=torch.uint8, device=words.device)
+    _need(out, torch.uint8, "out")
+    if out.numel() != nbytes or out.device != words.device:
+        raise ValueError(f"out must hold {nbytes} bytes on {words.device}")
+    return out
+
+
+def _need_scales(scales: torch.Tensor, name: str) -> None:
+    if scales.dtype not in (torch.float16, torch.int16):
+        raise ValueError(f"{name} must be float16 (or its int16 bit view)")
+    _need(scales, scales.dtype, name)
+
+
 def w4a16_repack(qweight: torch.Tensor, scales: torch.Tensor, group_size: int = 128,
                  stream=None, out: torch.Tensor | None = None) -> torch.Tensor:
     """Re-pack GPTQ words qweight[K/8][N] (int32) and scales[K/G][N] (fp16),
     into `out` (uint8, w4a16_packed_bytes bytes) when given."""
     _need(qweight, torch.int32, "qweight")
-    if scales.dtype not in (torch.float16, torch.int16):
-        raise ValueError("scales must be float16 (or its int16 bit view)")
-    _need(scales, scales.dtype, "scales")
+    _need_scales(scales, "scales")
     K = qweight.shape[0] * 8
     N = qweight.shape[1]
-    nbytes = w4a16_packed_bytes(K, N, group_size)
-    if nbytes == 0:
-        raise MxgError(MXG_ERR_UNSUPPORTED_SHAPE, "w4a16_repack")
-    if out is None:
-        packed = torch.empty(nbytes, dtype=torch.uint8, device=qweight.device)
-    else:
-        _need(out, torch.uint8, "out")
-        if out.numel() != nbytes or out.device != qweight.device:
-            raise ValueError(f"out must hold {nbytes} bytes on {qweight.device}")
-        packed = out
+    packed = _repack_out(qweight, K, N, group_size, out, "w4a16_repack")
     _check(_lib.w4a16_repack(_ptr(qweight), _ptr(scales), K, N, group_size, _ptr(packed),
                              _stream(stream)), "w4a16_repack")
+    return packed
+
+
+def w4a16_repack_ct(weight_packed: torch.Tensor, weight_scale: torch.Tensor,
+                    group_size: int = 128, stream=None,
+                    out: torch.Tensor | None = None) -> torch.Tensor:
+    """Re-pack compressed-tensors words weight_packed[N][K/8] (int32) and
+    weight_scale[N][K/G] (fp16) into the same buffer w4a16_repack makes."""
+    _need(weight_packed, torch.int32, "weight_packed")
+    _need_scales(weight_scale, "weight_scale")
+    N = weight_packed.shape[0]
+    K = weight_packed.shape[1] * 8
+    packed = _repack_out(weight_packed, K, N, group_size, out, "w4a16_repack_ct")
+    _check(_lib.w4a16_repack_ct(_ptr(weight_packed), _ptr(weight_scale), K, N, group_size,
+                                _ptr(packed), _stream(stream)), "w4a16_repack_ct")
+    return packed
+
+
+def w4a16_repack_fused(parts, group_size: int = 128, stream=None,
+                       out: torch.Tensor | None = None) -> torch.Tensor:
+    """One re-packed buffer for projections that share their input: `parts`
+    is a sequence of GPTQ (qweight[K/8][Ni], scales[K/G][Ni]) pairs with the
+    same K; the fused layer has N = sum Ni columns, part i's in order."""
+    parts = list(parts)
+    if not parts:
+        raise ValueError("parts must not be empty")
+    for qw, sc in parts:
+        _need(qw, torch.int32, "qweight")
+        _need_scales(sc, "scales")
+    K = parts[0][0].shape[0] * 8
+    if any(qw.shape[0] * 8 != K for qw, _ in parts):
+        raise ValueError("every part must have the same K")
+    Ns = [int(qw.shape[1]) for qw, _ in parts]
+    packed = _repack_out(parts[0][0], K, sum(Ns), group_size, out, "w4a16_repack_fused")
+    n = len(parts)
+    qptrs = (ctypes.c_void_p * n)(*[qw.data_ptr() for qw, _ in parts])
+    sptrs = (ctypes.c_void_p * n)(*[sc.data_ptr() for _, sc in parts])
+    narr = (ctypes.c_int * n)(*Ns)
+    _check(_lib.w4a16_repack_fused(n, qptrs, sptrs, narr, K, group_size, _ptr(packed),
+                                   _stream(stream)), "w4a16_repack_fused")
     return packed
 
 

@@ -217,7 +217,44 @@ int w4a16_repack(const int32_t *qweight, const uint16_t *scales, int K, int N, i
         return MXG_ERR_INVALID_ARG;
     if (!w4a16_shape_ok(K, N, group_size))
         return MXG_ERR_UNSUPPORTED_SHAPE;
-    return to_status(launch_w4a16_repack(qweight, scales, K, N, group_size, packed, stream));
+    return to_status(launch_w4a16_repack(qweight, scales, K, N, group_size, false, packed, stream));
+}
+
+int w4a16_repack_fused(int count, const int32_t *const *qweights, const uint16_t *const *scales,
+                       const int *Ns, int K, int group_size, void *packed, cudaStream_t stream)
+{
+    if (count < 1 || count > 64 || !qweights || !scales || !Ns || !aligned16(packed))
+        return MXG_ERR_INVALID_ARG;
+    long long N = 0;
+    for (int i = 0; i < count; ++i) {
+        if (!aligned16(qweights[i]) || !aligned16(scales[i]))
+            return MXG_ERR_INVALID_ARG;
+        if (!w4a16_shape_ok(K, Ns[i], group_size))
+            return MXG_ERR_UNSUPPORTED_SHAPE;
+        N += Ns[i];
+    }
+    if (N > (1LL << 30))
+        return MXG_ERR_UNSUPPORTED_SHAPE;
+    int n0 = 0;
+    for (int i = 0; i < count; ++i) {
+        const cudaError_t e = launch_w4a16_repack_part(qweights[i], scales[i], K, Ns[i], group_size,
+                                                       n0, (int)N, packed, stream);
+        if (e != cudaSuccess)
+            return to_status(e);
+        n0 += Ns[i];
+    }
+    return to_status(launch_repack_done(stream));
+}
+
+int w4a16_repack_ct(const int32_t *weight_packed, const uint16_t *weight_scale, int K, int N,
+                    int group_size, void *packed, cudaStream_t stream)
+{
+    if (!aligned16(weight_packed) || !aligned16(weight_scale) || !aligned16(packed))
+        return MXG_ERR_INVALID_ARG;
+    if (!w4a16_shape_ok(K, N, group_size))
+        return MXG_ERR_UNSUPPORTED_SHAPE;
+    return to_status(
+        launch_w4a16_repack(weight_packed, weight_scale, K, N, group_size, true, packed, stream));
 }
 
 size_t w4a16_workspace_bytes(int M, int N, int K, int group_size)

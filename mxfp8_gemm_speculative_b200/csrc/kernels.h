@@ -81,8 +81,15 @@ cudaError_t launch_mxfp8_tc(const TcPlan &plan, const void *X, const uint8_t *Wq
                             cudaStream_t stream);
 
 // ------------------------------------------------------------ weight tools
+// n_major: compressed-tensors inputs ([N][K/8] words, [N][K/G] scales)
+// instead of GPTQ's ([K/8][N], [K/G][N]).
 cudaError_t launch_w4a16_repack(const int32_t *qweight, const uint16_t *scales, int K, int N, int G,
-                                void *packed, cudaStream_t stream);
+                                bool n_major, void *packed, cudaStream_t stream);
+// Columns [n0, n0 + Np) of a fused buffer of N columns from GPTQ inputs of
+// Np columns (no completion kernel; launch_repack_done ends the re-pack).
+cudaError_t launch_w4a16_repack_part(const int32_t *qweight, const uint16_t *scales, int K, int Np,
+                                     int G, int n0, int N, void *packed, cudaStream_t stream);
+cudaError_t launch_repack_done(cudaStream_t stream);
 cudaError_t launch_w4a16_unpack(const void *packed, int K, int N, int G, uint8_t *codes,
                                 float *w_fp32, uint16_t *w_bf16, cudaStream_t stream);
 cudaError_t launch_mxfp8_dequant(const uint8_t *Wq, const uint8_t *Ws, int N, int K,

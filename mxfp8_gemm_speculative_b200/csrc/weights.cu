@@ -32,8 +32,12 @@ __device__ __forceinline__ int chunk_k0(int c, int t, int j)
     return c * 64 + 16 * j + 4 * t;
 }
 
+// Input words: word (i, n) (codes of rows 8i .. 8i+7 of column n, LSB
+// first) sits at qweight[i * wk + n * wn]: wk = N, wn = 1 for GPTQ
+// qweight[K/8][N]; wk = 1, wn = K/8 for compressed-tensors
+// weight_packed[N][K/8].
 __global__ void repack_codes_kernel(const int32_t *__restrict__ qweight, int K, int N,
-                                    uint4 *__restrict__ out)
+                                    size_t wk, size_t wn, uint4 *__restrict__ out)
 {
     const long long total = (long long)(N / 32) * (K / 64) * 64;
     const long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x;
@@ -52,8 +56,8 @@ __global__ void repack_codes_kernel(const int32_t *__restrict__ qweight, int K, 
     for (int j = 0; j < 4; ++j) {
         const int k0 = chunk_k0(c, t, j);
         const int shift = 4 * (k0 & 7);
-        const uint32_t qa = ((uint32_t)qweight[(size_t)(k0 >> 3) * N + na]) >> shift;
-        const uint32_t qb = ((uint32_t)qweight[(size_t)(k0 >> 3) * N + nb]) >> shift;
+        const uint32_t qa = ((uint32_t)qweight[(size_t)(k0 >> 3) * wk + na * wn]) >> shift;
+        const uint32_t qb = ((uint32_t)qweight[(size_t)(k0 >> 3) * wk + nb * wn]) >> shift;
         uint32_t w = 0;
         w |= (qa & 0xFu);
         w |= ((qa >> 4) & 0xFu) << 16;
@@ -68,8 +72,11 @@ __global__ void repack_codes_kernel(const int32_t *__restrict__ qweight, int K, 
     out[idx] = make_uint4(words[0], words[1], words[2], words[3]);
 }
 
+// Scale (group, n) sits at scales[group * sg + n * sn]: sg = N, sn = 1 for
+// GPTQ scales[K/G][N]; sg = 1, sn = K/G for compressed-tensors
+// weight_scale[N][K/G].
 __global__ void repack_scales_kernel(const uint16_t *__restrict__ scales, int K, int N, int G,
-                                     uint16_t *__restrict__ out)
+                                     size_t sg, size_t sn, uint16_t *__restrict__ out)
 {
     const int groups = K / G;
     const long long total = (long long)(N / 32) * groups * 32;
@@ -82,7 +89,7 @@ __global__ void repack_scales_kernel(const uint16_t *__restrict__ scales, int K,
     const int grp = (int)(rest % groups);
     const int T = (int)(rest / groups);
     const int n = T * 32 + g + 8 * (i4 & 1) + 16 * (i4 >> 1);
-    out[idx] = scales[(size_t)grp * N + n];
+    out[idx] = scales[(size_t)grp * sg + n * sn];
 }
 
 // One thread per 16-byte code chunk: writes 16 codes of two columns, and
@@ -190,15 +197,42 @@ inline unsigned blocks_for(long long total, int threads)
 
 }  // namespace
 
-cudaError_t launch_w4a16_repack(const int32_t *qweight, const uint16_t *scales, int K, int N, int G,
-                                void *packed, cudaStream_t stream)
+cudaError_t launch_w4a16_repack_part(const int32_t *qweight, const uint16_t *scales, int K, int Np,
+                                     int G, int n0, int N, void *packed, cudaStream_t stream)
 {
+    // part columns [n0, n0 + Np) of a fused layer with N columns: its n32
+    // tiles start at tile n0 / 32 in both the code and the scale region
+    const long long nchunks = (long long)(Np / 32) * (K / 64) * 64;
+    uint4 *codes = reinterpret_cast<uint4 *>(packed) + (size_t)(n0 / 32) * (K / 64) * 64;
+    repack_codes_kernel<<<blocks_for(nchunks, 256), 256, 0, stream>>>(qweight, K, Np, (size_t)Np,
+                                                                       1, codes);
+    const long long nsc = (long long)(Np / 32) * (K / G) * 32;
+    uint16_t *sc_out = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(packed) + (size_t)N * K / 2) +
+                       (size_t)(n0 / 32) * (K / G) * 32;
+    repack_scales_kernel<<<blocks_for(nsc, 256), 256, 0, stream>>>(scales, K, Np, G, (size_t)Np, 1,
+                                                                   sc_out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_repack_done(cudaStream_t stream)
+{
+    repack_done_kernel<<<1, 32, 0, stream>>>();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_w4a16_repack(const int32_t *qweight, const uint16_t *scales, int K, int N, int G,
+                                bool n_major, void *packed, cudaStream_t stream)
+{
+    // GPTQ inputs are K-major ([K/8][N] words, [K/G][N] scales), compressed-
+    // tensors inputs N-major ([N][K/8], [N][K/G]); the output is the same
+    const size_t wk = n_major ? 1 : (size_t)N, wn = n_major ? (size_t)K / 8 : 1;
+    const size_t sg = n_major ? 1 : (size_t)N, sn = n_major ? (size_t)(K / G) : 1;
     const long long nchunks = (long long)(N / 32) * (K / 64) * 64;
     repack_codes_kernel<<<blocks_for(nchunks, 256), 256, 0, stream>>>(
-        qweight, K, N, reinterpret_cast<uint4 *>(packed));
+        qweight, K, N, wk, wn, reinterpret_cast<uint4 *>(packed));
     const long long nsc = (long long)(N / 32) * (K / G) * 32;
     uint16_t *sc_out = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(packed) + (size_t)N * K / 2);
-    repack_scales_kernel<<<blocks_for(nsc, 256), 256, 0, stream>>>(scales, K, N, G, sc_out);
+    repack_scales_kernel<<<blocks_for(nsc, 256), 256, 0, stream>>>(scales, K, N, G, sg, sn, sc_out);
     repack_done_kernel<<<1, 32, 0, stream>>>();
     return cudaGetLastError();
 }

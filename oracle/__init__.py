@@ -63,6 +63,8 @@ def _bind(lib):
     lib.mxo_round_bf16.argtypes = [ctypes.c_double]
     lib.mxo_w4a16_unpack.restype = i
     lib.mxo_w4a16_unpack.argtypes = [p, p, i, i, i, p, p]
+    lib.mxo_w4a16_unpack_ct.restype = i
+    lib.mxo_w4a16_unpack_ct.argtypes = [p, p, i, i, i, p, p]
     lib.mxo_w4a16_pack.restype = i
     lib.mxo_w4a16_pack.argtypes = [p, i, i, p]
     lib.mxo_w4a16_gemm.restype = i
@@ -152,6 +154,24 @@ def w4a16_unpack(qweight: np.ndarray, scales: np.ndarray | None, K: int, N: int,
         _ptr(codes) if codes is not None else None,
         _ptr(w) if w is not None else None)
     _check(st, "w4a16_unpack")
+    return codes, w
+
+
+def w4a16_unpack_ct(weight_packed: np.ndarray, weight_scale: np.ndarray | None, K: int, N: int,
+                    group_size: int = 128, want_codes: bool = True,
+                    want_weights: bool = True):
+    """Codes[N][K] (uint8) and exact weights[N][K] (float64) of a
+    compressed-tensors export: words weight_packed[N][K/8], scales
+    weight_scale[N][K/G] (fp16 bits)."""
+    wp = _c(weight_packed, np.int32)
+    sc = _c(weight_scale, np.uint16) if weight_scale is not None else None
+    codes = np.empty((N, K), dtype=np.uint8) if want_codes else None
+    w = np.empty((N, K), dtype=np.float64) if want_weights else None
+    st = _load().mxo_w4a16_unpack_ct(
+        _ptr(wp), _ptr(sc) if sc is not None else None, K, N, group_size,
+        _ptr(codes) if codes is not None else None,
+        _ptr(w) if w is not None else None)
+    _check(st, "w4a16_unpack_ct")
     return codes, w
 
 

@@ -18,6 +18,13 @@
  *    the code of row k = 8i + j in bits [4j, 4j+3] (least significant nibble
  *    first); the zero point of a symmetric code is the implicit 8, so
  *    w[n][k] = (q - 8) * scale[k / G][n].
+ *  - The compressed-tensors export of the same weights (Eole Qwen3.8 recipe,
+ *    section "Compressed-tensors INT4 layout": symmetric grouped W4A16
+ *    pack-quantized weights that its converter transposes into the GPTQ
+ *    layout without re-quantizing).  Reading adopted: word (n, i) of
+ *    weight_packed[N][K/8] holds the code of row k = 8i + j of column n in
+ *    bits [4j, 4j+3], the same code values as GPTQ, and weight_scale[N][K/G]
+ *    holds scale (n, k / G); w[n][k] = (q - 8) * weight_scale[n][k / G].
  *  - fp16 scales (IEEE binary16) and bf16 activations (top half of an IEEE
  *    binary32); accumulation in fp32, output bf16 (Eole Qwen3.8 recipe,
  *    "INT4 weights / BF16 compute").
@@ -184,6 +191,28 @@ int mxo_w4a16_unpack(const int32_t *qweight, const uint16_t *scales,
                 codes[(size_t)n * K + k] = (uint8_t)w4a16_code(qweight, N, n, k);
             if (w)
                 w[(size_t)n * K + k] = w4a16_weight(qweight, scales, N, G, n, k);
+        }
+    return 0;
+}
+
+/* Unpack compressed-tensors words weight_packed[N][K/8] and scales
+ * weight_scale[N][K/G] into codes[N][K] (may be NULL) and weights w[N][K]
+ * (may be NULL), from the definition above (row n of the export is column n
+ * of the layer). */
+int mxo_w4a16_unpack_ct(const int32_t *weight_packed, const uint16_t *weight_scale,
+                        int K, int N, int G, uint8_t *codes, double *w)
+{
+    if (!weight_packed || !w4a16_args_ok(K, N, G) || (w && !weight_scale))
+        return -1;
+    for (int n = 0; n < N; ++n)
+        for (int k = 0; k < K; ++k) {
+            uint32_t word = (uint32_t)weight_packed[(size_t)n * (K / 8) + k / 8];
+            int q = (int)(word >> (4 * (k & 7))) & 0xF;
+            if (codes)
+                codes[(size_t)n * K + k] = (uint8_t)q;
+            if (w)
+                w[(size_t)n * K + k] =
+                    (double)(q - 8) * mxo_decode_fp16(weight_scale[(size_t)n * (K / G) + k / G]);
         }
     return 0;
 }

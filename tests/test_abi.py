@@ -65,12 +65,23 @@ def test_arguments_rejected_before_launch(mxg):
     assert lib.w4a16_gemm(a, mis, 5, 512, 512, 128, a, a, 1 << 20, null) == mxg.MXG_ERR_INVALID_ARG
     assert lib.mxfp8_gemm(a, a, mis, 4, 256, 512, a, a, 1 << 20, null) == mxg.MXG_ERR_INVALID_ARG
     assert lib.w4a16_repack(a, null, 512, 512, 128, a, null) == mxg.MXG_ERR_INVALID_ARG
+    assert lib.w4a16_repack_ct(null, a, 512, 512, 128, a, null) == mxg.MXG_ERR_INVALID_ARG
+    ptrs = (ctypes.c_void_p * 2)(4096, 8192)
+    ns = (ctypes.c_int * 2)(512, 256)
+    assert lib.w4a16_repack_fused(0, ptrs, ptrs, ns, 512, 128, a, null) == mxg.MXG_ERR_INVALID_ARG
+    assert lib.w4a16_repack_fused(2, null, ptrs, ns, 512, 128, a, null) == mxg.MXG_ERR_INVALID_ARG
+    assert lib.w4a16_repack_fused(2, ptrs, ptrs, ns, 512, 128, mis, null) == mxg.MXG_ERR_INVALID_ARG
+    bad = (ctypes.c_int * 2)(512, 96)
+    assert lib.w4a16_repack_fused(2, ptrs, ptrs, bad, 512, 128, a, null) == mxg.MXG_ERR_UNSUPPORTED_SHAPE
+    assert lib.w4a16_repack_ct(a, mis, 512, 512, 128, a, null) == mxg.MXG_ERR_INVALID_ARG
     # M < 1
     assert lib.w4a16_gemm(a, a, 0, 512, 512, 128, a, a, 1 << 20, null) == mxg.MXG_ERR_INVALID_ARG
     # shapes the format or the kernels reject
     assert lib.w4a16_gemm(a, a, 5, 512, 512, 96, a, a, 1 << 20, null) == mxg.MXG_ERR_UNSUPPORTED_SHAPE
     assert lib.w4a16_gemm(a, a, 5, 96, 512, 128, a, a, 1 << 20, null) == mxg.MXG_ERR_UNSUPPORTED_SHAPE
     assert lib.w4a16_repack(a, a, 480, 512, 32, a, null) == mxg.MXG_ERR_UNSUPPORTED_SHAPE
+    assert lib.w4a16_repack_ct(a, a, 480, 512, 32, a, null) == mxg.MXG_ERR_UNSUPPORTED_SHAPE
+    assert lib.w4a16_repack_ct(a, a, 512, 96, 128, a, null) == mxg.MXG_ERR_UNSUPPORTED_SHAPE
     assert lib.mxfp8_gemm(a, a, a, 4, 96, 512, a, a, 1 << 20, null) == mxg.MXG_ERR_UNSUPPORTED_SHAPE
     assert lib.mxfp8_gemm(a, a, a, 4, 256, 500, a, a, 1 << 20, null) == mxg.MXG_ERR_UNSUPPORTED_SHAPE
     assert lib.mxfp8_dequant(a, a, 96, 512, a, null) == mxg.MXG_ERR_UNSUPPORTED_SHAPE

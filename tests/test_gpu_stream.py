@@ -310,3 +310,47 @@ def test_early_weight_loads_match_late_loads(mxg):
         mxg.mxg_set_early_weight_loads(prev)
     torch.cuda.synchronize()
     assert torch.equal(mouts[0].view(torch.int16), mouts[1].view(torch.int16))
+
+
+@pytest.mark.parametrize("K,N,G", [(512, 512, 128), (1024, 192, 64), (256, 320, 32)])
+def test_repack_ct_matches_gptq_repack(mxg, K, N, G):
+    """The compressed-tensors export (words [N][K/8], scales [N][K/G]: the
+    GPTQ ones transposed) re-packs to the same bytes, and a GEMM on it
+    matches the oracle's unpack of the export."""
+    lay = synth.int4_layer(4, K, N, G, seed=K + 3 * N + G)
+    qw, sc = int4_device(lay)
+    ref = mxg.w4a16_repack(qw, sc, G)
+    wp = torch.from_numpy(np.ascontiguousarray(lay.qweight.T)).to(DEV)
+    ws = torch.from_numpy(np.ascontiguousarray(lay.scales.T).view(np.int16)).to(DEV)
+    packed = mxg.w4a16_repack_ct(wp, ws, G)
+    torch.cuda.synchronize()
+    assert torch.equal(packed, ref)
+    _, w = oracle.w4a16_unpack_ct(np.ascontiguousarray(lay.qweight.T),
+                                  np.ascontiguousarray(lay.scales.T), K, N, G)
+    y = mxg.w4a16_gemm(bf16_tensor(lay.X, DEV), packed, N, K, G)
+    x64 = (lay.X.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    assert_parity(to_f64(y), x64 @ w.T, "compressed-tensors GEMM")
+
+
+@pytest.mark.parametrize("K,Ns,G,M", [(512, (256, 128, 128), 128, 5), (1024, (192, 192), 64, 16),
+                                      (256, (64, 320), 32, 40)])
+def test_repack_fused_matches_concatenated_repack(mxg, K, Ns, G, M):
+    """A fused buffer of several projections (same K) is byte for byte the
+    re-pack of their words and scales concatenated along N, and one GEMM on it
+    (weight streaming, or tensor cores for M = 40) matches the oracle for
+    every part."""
+    lays = [synth.int4_layer(M, K, n, G, seed=100 * i + n + K) for i, n in enumerate(Ns)]
+    parts = [int4_device(lay) for lay in lays]
+    fused = mxg.w4a16_repack_fused(parts, G)
+    qcat = torch.cat([qw for qw, _ in parts], dim=1).contiguous()
+    scat = torch.cat([sc for _, sc in parts], dim=1).contiguous()
+    ref = mxg.w4a16_repack(qcat, scat, G)
+    torch.cuda.synchronize()
+    assert torch.equal(fused, ref)
+    N = sum(Ns)
+    y = to_f64(mxg.w4a16_gemm(bf16_tensor(lays[0].X, DEV), fused, N, K, G))
+    n0 = 0
+    for lay, n in zip(lays, Ns):
+        want = oracle.w4a16_gemm(lays[0].X, lay.qweight, lay.scales, M, n, K, G)
+        assert_parity(y[:, n0:n0 + n], want, f"fused part at column {n0}")
+        n0 += n

@@ -179,3 +179,48 @@ def test_invalid_arguments(orc):
         orc.w4a16_gemm(lay.X, lay.qweight, lay.scales, 1, 64, 128, 48)   # K % G != 0
     with pytest.raises(ValueError):
         orc.w4a16_gemm_at(lay.X, lay.qweight, lay.scales, 1, 64, 128, 64, [1], [0])  # row out of range
+
+
+# ------------------------------------------- compressed-tensors export
+def test_ct_nibble_order_and_row_index(orc):
+    """Word (n, i) of weight_packed[N][K/8] feeds rows 8i..8i+7 of column n,
+    least significant nibble first, and nothing else."""
+    K, N, G = 32, 6, 32
+    for n in range(N):
+        for i in range(K // 8):
+            wp = np.full((N, K // 8), np.uint32(0x88888888).view(np.int32), dtype=np.int32)
+            wp[n, i] = np.uint32(0xFEDCBA98).view(np.int32)
+            sc = np.full((N, K // G), 0x3C00, dtype=np.uint16)
+            codes, w = orc.w4a16_unpack_ct(wp, sc, K, N, G)
+            expect = np.full((N, K), 8, dtype=np.uint8)
+            expect[n, 8 * i:8 * i + 8] = [8, 9, 10, 11, 12, 13, 14, 15]
+            assert np.array_equal(codes, expect)
+            assert np.array_equal(w, expect.astype(np.float64) - 8.0)
+
+
+def test_ct_scale_index(orc):
+    """weight_scale[n][g] multiplies exactly rows g*G .. g*G+G-1 of column n."""
+    K, N = 256, 4
+    for G in (32, 64, 128):
+        for n in range(N):
+            for g in range(K // G):
+                wp = np.full((N, K // 8), np.uint32(0x99999999).view(np.int32), dtype=np.int32)
+                sc = np.full((N, K // G), 0x3C00, dtype=np.uint16)   # 1.0
+                sc[n, g] = 0x4400                                   # 4.0
+                _, w = orc.w4a16_unpack_ct(wp, sc, K, N, G)
+                expect = np.ones((N, K))
+                expect[n, g * G:(g + 1) * G] = 4.0
+                assert np.array_equal(w, expect)
+
+
+def test_ct_equals_gptq_of_transposed_words(orc):
+    """The export is the GPTQ words and scales transposed: both unpackers
+    (written separately) agree on random words."""
+    rng = np.random.default_rng(5)
+    for K, N, G in [(64, 64, 32), (256, 96, 64), (512, 40, 128)]:
+        qw = rng.integers(0, 2**32, size=(K // 8, N), dtype=np.uint64).astype(np.uint32).view(np.int32)
+        sc = (np.abs(rng.standard_normal((K // G, N))) * 0.01 + 1e-3).astype(np.float16).view(np.uint16)
+        c1, w1 = orc.w4a16_unpack(qw, sc, K, N, G)
+        c2, w2 = orc.w4a16_unpack_ct(np.ascontiguousarray(qw.T), np.ascontiguousarray(sc.T), K, N, G)
+        assert np.array_equal(c1, c2) and np.array_equal(w1, w2)
+        assert np.array_equal(w2, _numpy_dense_weights(qw, sc, K, N, G).T)

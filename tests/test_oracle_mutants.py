@@ -19,6 +19,9 @@ MUTANTS = {
     "zero_point_7": ("return (double)(q - 8) * s;", "return (double)(q - 7) * s;"),
     "nibble_order_reversed": ("(word >> (4 * (k % 8)))", "(word >> (4 * (7 - k % 8)))"),
     "word_column_shifted": ("qweight[(size_t)(k / 8) * N + n]", "qweight[(size_t)(k / 8) * N + (n + 1) % N]"),
+    "ct_words_read_as_gptq": ("weight_packed[(size_t)n * (K / 8) + k / 8]", "weight_packed[(size_t)(k / 8) * N + n]"),
+    "ct_nibble_order_reversed": ("(word >> (4 * (k & 7)))", "(word >> (4 * (7 - (k & 7))))"),
+    "ct_scales_read_as_gptq": ("weight_scale[(size_t)n * (K / G) + k / G]", "weight_scale[(size_t)(k / G) * N + n]"),
     "group_index_fixed_128": ("scales[(size_t)(k / G) * N + n]", "scales[(size_t)(k / 128) * N + n]"),
     "fp16_bias_off_by_one": ("ldexp((double)(1024 + f), e - 25)", "ldexp((double)(1024 + f), e - 24)"),
     "bf16_drops_implicit_bit": ("ldexp((double)(128 + f), e - 134)", "ldexp((double)(f), e - 134)"),
