@@ -50,6 +50,9 @@ WORKLOADS = {
     "prefill_int4": ("int4", 8192, [(5120, 17408)], 128),
     "mxfp8_m4": ("mxfp8", 4, [(5120, 17408)], 32),
     "mxfp8_m128": ("mxfp8", 128, [(5120, 17408)], 32),
+    # the paired dense bf16 GDN A/B projection (2 x 48 rows of 5120)
+    "gdn_ab_bf16_m4": ("bf16", 4, [(5120, 96)], 0),
+    "gdn_ab_bf16_m1": ("bf16", 1, [(5120, 96)], 0),
 }
 TENSOR_BOUND = {"c32_mtp3_int4", "prefill_int4", "mxfp8_m128"}
 # (workload, layer index) -> column counts of the projections fused into it
@@ -59,6 +62,8 @@ FUSED_PARTS = {("mtp4_verify_int4_fused", 1): (17408, 17408)}
 def layer_weight_bytes(fmt, K, N, G):
     if fmt == "int4":
         return N * K // 2 + N * (K // G) * 2
+    if fmt == "bf16":
+        return N * K * 2
     return N * K + N * (K // 32)
 
 
@@ -191,6 +196,12 @@ def run_ours(args, rank, world, local_rank):
             weights.append([packed] + [packed.clone() for _ in range(pool - 1)])
             wss.append(torch.zeros(mxg.w4a16_workspace_bytes(M, N, K, G), dtype=torch.uint8,
                                    device=dev))
+        elif fmt == "bf16":
+            lay = synth.bf16_layer(M, K, N, seed=rank, layer=li)
+            w = torch.from_numpy(lay.W.view(np.int16)).view(torch.bfloat16).to(dev)
+            weights.append([w] + [w.clone() for _ in range(pool - 1)])
+            wss.append(torch.zeros(mxg.raw_lib().bf16_gemm_small_workspace_bytes(M, N, K),
+                                   dtype=torch.uint8, device=dev))
         else:
             lay = synth.mxfp8_layer(M, K, N, seed=rank, layer=li)
             wq = torch.from_numpy(lay.Wq).to(dev)
@@ -208,6 +219,9 @@ def run_ours(args, rank, world, local_rank):
         if fmt == "int4":
             mxg.w4a16_gemm(xs[li], weights[li][p], N, K, G, out=ys[li], workspace_buf=wss[li],
                            stream=s)
+        elif fmt == "bf16":
+            mxg.bf16_gemm_small(xs[li], weights[li][p], out=ys[li], workspace_buf=wss[li],
+                                stream=s)
         else:
             wq, ws = weights[li][p]
             mxg.mxfp8_gemm(xs[li], wq, ws, out=ys[li], workspace_buf=wss[li], stream=s)
@@ -306,6 +320,9 @@ def run_ours(args, rank, world, local_rank):
             if fmt == "int4":
                 c, _ = mxg.prepare_w4a16_gemm(dev_x[li], weights[li][p], N, K, G, out=dev_y[li],
                                               workspace_buf=wss[li], stream=stream)
+            elif fmt == "bf16":
+                c, _ = mxg.prepare_bf16_gemm_small(dev_x[li], weights[li][p], out=dev_y[li],
+                                                   workspace_buf=wss[li], stream=stream)
             else:
                 wq, ws = weights[li][p]
                 c, _ = mxg.prepare_mxfp8_gemm(dev_x[li], wq, ws, out=dev_y[li],
@@ -359,7 +376,8 @@ def run_ours(args, rank, world, local_rank):
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": None,
                 "peak_source": f"{peak_kind} copy bandwidth"}
-    kernel_name = ("w4a16_stream_kernel" if (fmt == "int4" and M <= 32) else
+    kernel_name = ("bf16_small_kernel" if fmt == "bf16" else
+                   "w4a16_stream_kernel" if (fmt == "int4" and M <= 32) else
                    "mxfp8_stream_kernel" if M <= 32 else "tc_gemm_kernel")
     roof["kernel"] = kernel_name
     roof["per_layer_us"] = [round(k / kernel_launches * 1e3, 3) for k in kernel_ms]
@@ -384,7 +402,7 @@ def run_ours(args, rank, world, local_rank):
         "config": {
             "workload": args.workload,
             "format": fmt, "M": M, "layers_KxN": [f"{K}x{N}" for K, N in layers],
-            "group_size": G if fmt == "int4" else 32,
+            "group_size": G if fmt == "int4" else (32 if fmt == "mxfp8" else None),
             "weight_bytes_per_step": step_bytes, "flops_per_step": step_flops,
             "l2": f"rotating weight pool of {pool} copies ({pool * step_bytes / 1e6:.0f} MB >= "
                   f"{args.pool_factor:g} x L2)",
@@ -437,6 +455,8 @@ def oracle_step_runner(workload: str, cols_per_layer: int | None, seed: int = 0)
     for li, (K, N) in enumerate(layers):
         if fmt == "int4":
             lay = synth.int4_layer(M, K, N, G, seed=seed, layer=li)
+        elif fmt == "bf16":
+            lay = synth.bf16_layer(M, K, N, seed=seed, layer=li)
         else:
             lay = synth.mxfp8_layer(M, K, N, seed=seed, layer=li)
         prepared.append((K, N, lay))
@@ -446,6 +466,8 @@ def oracle_step_runner(workload: str, cols_per_layer: int | None, seed: int = 0)
         if fmt == "int4":
             return (np.ascontiguousarray(lay.qweight[:, c0:c1]),
                     np.ascontiguousarray(lay.scales[:, c0:c1]))
+        if fmt == "bf16":
+            return np.ascontiguousarray(lay.W[c0:c1]), None
         return (np.ascontiguousarray(lay.Wq[c0:c1]), np.ascontiguousarray(lay.Ws[c0:c1]))
 
     def run(nthreads: int):
@@ -459,6 +481,8 @@ def oracle_step_runner(workload: str, cols_per_layer: int | None, seed: int = 0)
             n = c1 - c0
             if fmt == "int4":
                 oracle.w4a16_gemm(lay.X, a, b, M, n, K, G, nthreads=nthreads)
+            elif fmt == "bf16":
+                oracle.bf16_gemm(lay.X, a, M, n, K)
             else:
                 oracle.mxfp8_gemm(lay.X, a, b, M, n, K, nthreads=nthreads)
             total_bytes += layer_weight_bytes(fmt, K, n, G)

@@ -189,6 +189,24 @@ MXG_API size_t mxfp8_workspace_bytes(int M, int N, int K);
 MXG_API int mxfp8_gemm(const void *X, const uint8_t *Wq, const uint8_t *Ws, int M, int N, int K,
                void *Y, void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* ------------------------------------- dense bf16, few output columns */
+
+/* Y = X * W^T with dense bf16 weights, for the paired GDN A/B projection of
+ * the Eole recipe (section "Pack inference projections": two dense bf16
+ * projections of 48 x 5120 computed together, N = 96, for single-token
+ * decoding and four-token verification; below the N >= 128 of the MXFP8
+ * path).  Latency-bound: one CTA per 8 rows of W, whose warps split K and
+ * add their fp32 partials in a fixed order (bitwise reproducible).
+ *   X  device, bf16 [M][K];  W device, bf16 [N][K] (K contiguous);
+ *   Y  device, bf16 [M][N];  workspace as for w4a16_gemm, sized by
+ *   bf16_gemm_small_workspace_bytes.
+ * Requirements: 1 <= M <= 8; 16 <= N <= 2048 with N % 16 == 0; K >= 64 and
+ * K % 64 == 0; else MXG_ERR_UNSUPPORTED_SHAPE.  Weights are read before the
+ * wait for the previous kernel (see the conventions above). */
+MXG_API size_t bf16_gemm_small_workspace_bytes(int M, int N, int K);
+MXG_API int bf16_gemm_small(const void *X, const void *W, int M, int N, int K, void *Y,
+               void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* --------------------------------------------------- test and diagnostics */
 
 /* Decode a re-packed INT4 buffer with the device routines of the GEMM paths.

@@ -51,6 +51,8 @@ _SIGS = {
     "mxfp8_dequant": (_i, [_p, _p, _i, _i, _p, _p]),
     "mxg_workspace_status": (_i, [_p, ctypes.POINTER(_i), _p]),
     "mxg_selftest_wait_timeout": (_i, [_p, _i, _p]),
+    "bf16_gemm_small_workspace_bytes": (_sz, [_i, _i, _i]),
+    "bf16_gemm_small": (_i, [_p, _p, _i, _i, _i, _p, _p, _sz, _p]),
     "mxg_set_path": (_i, [_i]),
     "mxg_set_early_weight_loads": (_i, [_i]),
 }
@@ -282,6 +284,26 @@ def prepare_mxfp8_gemm(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor,
     return PreparedCall(_lib.mxfp8_gemm, args, "mxfp8_gemm", (x, wq, ws, out, wsb, stream)), out
 
 
+def prepare_bf16_gemm_small(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = None,
+                            workspace_buf: torch.Tensor | None = None, stream=None):
+    """(call, out): ``call()`` runs bf16_gemm_small(x, w) into ``out``."""
+    _need(x, torch.bfloat16, "x")
+    _need(w, torch.bfloat16, "w")
+    M, K = x.shape
+    N = w.shape[0]
+    if w.shape[1] != K:
+        raise ValueError("x must be [M][K] and w [N][K]")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(out, torch.bfloat16, "out")
+    need = int(_lib.bf16_gemm_small_workspace_bytes(M, N, K))
+    if need == 0:
+        raise MxgError(MXG_ERR_UNSUPPORTED_SHAPE, "bf16_gemm_small")
+    wsb = workspace_buf if workspace_buf is not None else workspace(need, x.device, stream)
+    args = (_ptr(x), _ptr(w), M, N, K, _ptr(out), _ptr(wsb), wsb.numel(), _stream(stream))
+    return PreparedCall(_lib.bf16_gemm_small, args, "bf16_gemm_small", (x, w, out, wsb, stream)), out
+
+
 def w4a16_gemm_static_scratch(x: torch.Tensor, packed: torch.Tensor, N: int, K: int,
                               group_size: int = 128, out: torch.Tensor | None = None,
                               stream=None) -> torch.Tensor:
@@ -353,6 +375,28 @@ def mxg_workspace_status(workspace_buf: torch.Tensor, stream=None) -> int:
     _check(_lib.mxg_workspace_status(_ptr(workspace_buf), ctypes.byref(v), _stream(stream)),
            "mxg_workspace_status")
     return v.value
+
+
+def bf16_gemm_small(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = None,
+                    workspace_buf: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Y = x * w^T with dense bf16 w [N][K] (few columns, e.g. the paired
+    48 + 48 GDN A/B projection) and x bf16 [M][K], M <= 8."""
+    _need(x, torch.bfloat16, "x")
+    _need(w, torch.bfloat16, "w")
+    if x.dim() != 2 or w.dim() != 2 or x.shape[1] != w.shape[1]:
+        raise ValueError("x must be [M][K] and w [N][K]")
+    M, K = x.shape
+    N = w.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(out, torch.bfloat16, "out")
+    need = int(_lib.bf16_gemm_small_workspace_bytes(M, N, K))
+    if need == 0:
+        raise MxgError(MXG_ERR_UNSUPPORTED_SHAPE, "bf16_gemm_small")
+    ws = workspace_buf if workspace_buf is not None else workspace(need, x.device, stream)
+    _check(_lib.bf16_gemm_small(_ptr(x), _ptr(w), M, N, K, _ptr(out), _ptr(ws), ws.numel(),
+                                _stream(stream)), "bf16_gemm_small")
+    return out
 
 
 def mxg_selftest_wait_timeout(workspace_buf: torch.Tensor, limit_us: int, stream=None) -> None:

@@ -388,6 +388,27 @@ int mxg_selftest_wait_timeout(void *workspace, int limit_us, cudaStream_t stream
     return to_status(launch_wait_timeout_selftest(workspace, limit_us, stream));
 }
 
+size_t bf16_gemm_small_workspace_bytes(int M, int N, int K)
+{
+    SmallPlan sp;
+    if (!plan_bf16_small(M, N, K, &sp))
+        return 0;
+    return make_workspace_map(1, sp.partial_bytes).total;
+}
+
+int bf16_gemm_small(const void *X, const void *W, int M, int N, int K, void *Y, void *workspace,
+                    size_t workspace_bytes, cudaStream_t stream)
+{
+    if (!aligned16(X) || !aligned16(W) || !aligned16(Y) || !aligned16(workspace) || M < 1)
+        return MXG_ERR_INVALID_ARG;
+    SmallPlan sp;
+    if (!plan_bf16_small(M, N, K, &sp))
+        return MXG_ERR_UNSUPPORTED_SHAPE;
+    if (workspace_bytes < make_workspace_map(1, sp.partial_bytes).total)
+        return MXG_ERR_WORKSPACE;
+    return to_status(launch_bf16_small(sp, X, W, M, N, K, Y, workspace, stream));
+}
+
 int mxg_set_path(int path)
 {
     if (path < 0 || path > 2)

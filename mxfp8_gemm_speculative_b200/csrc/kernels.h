@@ -80,6 +80,18 @@ cudaError_t launch_mxfp8_tc(const TcPlan &plan, const void *X, const uint8_t *Wq
                             const uint8_t *Ws, int M, int N, int K, void *Y, void *workspace,
                             cudaStream_t stream);
 
+// ------------------------------------------ dense bf16, few output columns
+// Split-K plan: K in 64-wide chunks over `ctas` CTAs of N/16 warps each.
+struct SmallPlan {
+    int chunks;
+    int ctas;
+    int threads;
+    size_t partial_bytes;
+};
+bool plan_bf16_small(int M, int N, int K, SmallPlan *plan);
+cudaError_t launch_bf16_small(const SmallPlan &plan, const void *X, const void *W, int M, int N,
+                              int K, void *Y, void *workspace, cudaStream_t stream);
+
 // ------------------------------------------------------------ weight tools
 // n_major: compressed-tensors inputs ([N][K/8] words, [N][K/G] scales)
 // instead of GPTQ's ([K/8][N], [K/G][N]).

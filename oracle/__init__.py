@@ -17,6 +17,8 @@ Every function cites the passage it follows in ``oracle.c``'s header:
   "Compressed-tensors INT4 layout".
 * MXFP8: "Qwen3.8-27B-MXFP8 AutoRound" model card, header, section 2 (kernel
   constraints) and section 8 (OCP MX format, E8M0 scale per 32 elements).
+* Dense bf16 projections: Eole Qwen3.8 recipe, section "Pack inference
+  projections" (the paired GDN A/B projection).
 """
 from __future__ import annotations
 
@@ -63,6 +65,8 @@ def _bind(lib):
     lib.mxo_round_bf16.argtypes = [ctypes.c_double]
     lib.mxo_w4a16_unpack.restype = i
     lib.mxo_w4a16_unpack.argtypes = [p, p, i, i, i, p, p]
+    lib.mxo_bf16_gemm.restype = i
+    lib.mxo_bf16_gemm.argtypes = [p, p, i, i, i, p]
     lib.mxo_w4a16_unpack_ct.restype = i
     lib.mxo_w4a16_unpack_ct.argtypes = [p, p, i, i, i, p, p]
     lib.mxo_w4a16_pack.restype = i
@@ -249,3 +253,12 @@ def mxfp8_gemm_at(X_bits, Wq, Ws, M, N, K, rows, cols, nthreads: int = 1) -> np.
 def threads(requested: int) -> int:
     """Threads an oracle call with ``nthreads=requested`` actually uses."""
     return int(_load().mxo_threads(int(requested)))
+
+
+def bf16_gemm(X_bits: np.ndarray, W_bits: np.ndarray, M: int, N: int, K: int) -> np.ndarray:
+    """Y[M][N] in float64 (not rounded) of dense bf16 weights W[N][K]."""
+    x = _c(X_bits, np.uint16)
+    w = _c(W_bits, np.uint16)
+    Y = np.empty((M, N), dtype=np.float64)
+    _check(_load().mxo_bf16_gemm(_ptr(x), _ptr(w), M, N, K, _ptr(Y)), "bf16_gemm")
+    return Y

@@ -25,6 +25,10 @@
  *    weight_packed[N][K/8] holds the code of row k = 8i + j of column n in
  *    bits [4j, 4j+3], the same code values as GPTQ, and weight_scale[N][K/G]
  *    holds scale (n, k / G); w[n][k] = (q - 8) * weight_scale[n][k / G].
+ *  - Dense bf16 projections with few output columns (Eole Qwen3.8 recipe,
+ *    section "Pack inference projections": the paired 48 x 5120 GDN A/B
+ *    projections in bf16).  Reading adopted: W[N][K] row-major (the Linear
+ *    out x in layout), Y[m][n] = sum_k X[m][k] * W[n][k].
  *  - fp16 scales (IEEE binary16) and bf16 activations (top half of an IEEE
  *    binary32); accumulation in fp32, output bf16 (Eole Qwen3.8 recipe,
  *    "INT4 weights / BF16 compute").
@@ -413,4 +417,20 @@ int mxo_threads(int requested)
     (void)requested;
     return 1;
 #endif
+}
+
+/* Dense bf16 weights W[N][K]: Y[m][n] = sum over k ascending of
+ * X[m][k] * W[n][k], in double precision (not rounded). */
+int mxo_bf16_gemm(const uint16_t *X, const uint16_t *W, int M, int N, int K, double *Y)
+{
+    if (!X || !W || !Y || M <= 0 || N <= 0 || K <= 0)
+        return -1;
+    for (int m = 0; m < M; ++m)
+        for (int n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int k = 0; k < K; ++k)
+                acc += mxo_decode_bf16(X[(size_t)m * K + k]) * mxo_decode_bf16(W[(size_t)n * K + k]);
+            Y[(size_t)m * N + n] = acc;
+        }
+    return 0;
 }

@@ -17,6 +17,9 @@ Recipes (value distributions of the workloads the layer is measured on):
   E8M0 exponent per (row, 32-block) uniform in 119..123 (2^-8 .. 2^-4); X as
   above.
 
+* Dense bf16 (the paired GDN A/B projection): W bf16(0.02*z) [N][K], X as
+  above.
+
 RNG: numpy ``Generator(PCG64)`` seeded from ``SeedSequence([seed, layer])``,
 spawned into three independent streams (codes, scales, X).
 """
@@ -92,6 +95,23 @@ def mxfp8_layer(M: int, K: int, N: int, seed: int = 0, layer: int = 0,
     Ws = r_scales.integers(exp_lo, exp_hi + 1, size=(N, K // 32), dtype=np.uint8)
     X = bf16_bits_of_normals(r_x, (M, K))
     return Mxfp8Layer(M, K, N, X, Wq, Ws)
+
+
+@dataclass
+class Bf16Layer:
+    M: int
+    K: int
+    N: int
+    X: np.ndarray        # uint16 bf16 bits [M][K]
+    W: np.ndarray        # uint16 bf16 bits [N][K]
+
+
+def bf16_layer(M: int, K: int, N: int, seed: int = 0, layer: int = 0) -> Bf16Layer:
+    r_w, _, r_x = _streams(seed, layer)
+    z = r_w.standard_normal(size=(N, K), dtype=np.float32) * np.float32(0.02)
+    W = torch.from_numpy(z).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16).copy()
+    X = bf16_bits_of_normals(r_x, (M, K))
+    return Bf16Layer(M, K, N, X, W)
 
 
 # Layer shapes of the measured workloads (hidden 5120, MLP width 17408).

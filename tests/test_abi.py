@@ -87,6 +87,13 @@ def test_arguments_rejected_before_launch(mxg):
     assert lib.mxfp8_dequant(a, a, 96, 512, a, null) == mxg.MXG_ERR_UNSUPPORTED_SHAPE
     assert lib.w4a16_unpack(a, 512, 512, 128, mis, null, null, null) == mxg.MXG_ERR_INVALID_ARG
     assert lib.mxg_selftest_wait_timeout(a, 0, null) == mxg.MXG_ERR_INVALID_ARG
+    # dense bf16 few-column projection: M <= 8, 16 <= N <= 2048, N % 16, K % 64
+    for M, N, K in [(9, 96, 5120), (4, 100, 5120), (4, 2064, 5120), (4, 96, 5000), (4, 96, 0)]:
+        assert lib.bf16_gemm_small(a, a, M, N, K, a, a, 1 << 20, null) == mxg.MXG_ERR_UNSUPPORTED_SHAPE
+        assert lib.bf16_gemm_small_workspace_bytes(M, N, K) == 0
+    assert lib.bf16_gemm_small(a, mis, 4, 96, 5120, a, a, 1 << 20, null) == mxg.MXG_ERR_INVALID_ARG
+    assert lib.bf16_gemm_small(a, a, 4, 96, 5120, a, a, 256, null) == mxg.MXG_ERR_WORKSPACE
+    assert lib.bf16_gemm_small_workspace_bytes(4, 96, 5120) > 256
 
 
 def test_path_override_roundtrip(mxg):

@@ -13,7 +13,7 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "oracle.c")
 PIN_SUITES = ["tests/test_oracle_formats.py", "tests/test_oracle_int4.py",
-              "tests/test_oracle_mxfp8.py"]
+              "tests/test_oracle_mxfp8.py", "tests/test_oracle_bf16.py"]
 
 MUTANTS = {
     "zero_point_7": ("return (double)(q - 8) * s;", "return (double)(q - 7) * s;"),
@@ -30,6 +30,8 @@ MUTANTS = {
     "round_ties_away": ("r = (fmod(lo, 2.0) == 0.0) ? lo : lo + 1.0;", "r = lo + 1.0;"),
     "gemm_reversed_k": ("acc += x[k] * w[k];", "acc += x[k] * w[K - 1 - k];"),
     "mxfp8_block_index": ("Ws[(size_t)n * (K / 32) + k / 32]", "Ws[(size_t)n * (K / 32) + (k % 32) / 32]"),
+    "bf16_gemm_reversed_w": ("mxo_decode_bf16(W[(size_t)n * K + k])", "mxo_decode_bf16(W[(size_t)n * K + (K - 1 - k)])"),
+    "bf16_gemm_drops_last_k": ("            for (int k = 0; k < K; ++k)\n                acc += mxo_decode_bf16(X[(size_t)m * K + k]) * mxo_decode_bf16(W", "            for (int k = 0; k < K - 1; ++k)\n                acc += mxo_decode_bf16(X[(size_t)m * K + k]) * mxo_decode_bf16(W"),
     "mxfp8_gemm_drops_scale": ("w[k] = mxfp8_weight(Wq, Ws, K, n, k);", "w[k] = mxo_decode_e4m3(Wq[(size_t)n * K + k]);"),
 }
 
