@@ -19,6 +19,8 @@ Every function cites the passage it follows in ``oracle.c``'s header:
   constraints) and section 8 (OCP MX format, E8M0 scale per 32 elements).
 * Dense bf16 projections: Eole Qwen3.8 recipe, section "Pack inference
   projections" (the paired GDN A/B projection).
+* INT8 W8A16 head: Eole Qwen3.8 recipe, section "Optional vocabulary-head
+  quantization"; W4A16 LowLatency model card (INT8 lm_head, RTN g128).
 """
 from __future__ import annotations
 
@@ -65,6 +67,10 @@ def _bind(lib):
     lib.mxo_round_bf16.argtypes = [ctypes.c_double]
     lib.mxo_w4a16_unpack.restype = i
     lib.mxo_w4a16_unpack.argtypes = [p, p, i, i, i, p, p]
+    lib.mxo_w8a16_unpack.restype = i
+    lib.mxo_w8a16_unpack.argtypes = [p, p, i, i, i, p, p]
+    lib.mxo_w8a16_gemm.restype = i
+    lib.mxo_w8a16_gemm.argtypes = [p, p, p, i, i, i, i, p, i]
     lib.mxo_bf16_gemm.restype = i
     lib.mxo_bf16_gemm.argtypes = [p, p, i, i, i, p]
     lib.mxo_w4a16_unpack_ct.restype = i
@@ -261,4 +267,30 @@ def bf16_gemm(X_bits: np.ndarray, W_bits: np.ndarray, M: int, N: int, K: int) ->
     w = _c(W_bits, np.uint16)
     Y = np.empty((M, N), dtype=np.float64)
     _check(_load().mxo_bf16_gemm(_ptr(x), _ptr(w), M, N, K, _ptr(Y)), "bf16_gemm")
+    return Y
+
+
+def w8a16_unpack(qweight: np.ndarray, scales: np.ndarray | None, K: int, N: int,
+                 group_size: int = 128):
+    """Codes[N][K] (uint8) and exact weights[N][K] (float64) of INT8 words
+    qweight[K/4][N] with fp16 scales[K/G][N]."""
+    qw = _c(qweight, np.int32)
+    sc = _c(scales, np.uint16) if scales is not None else None
+    codes = np.empty((N, K), dtype=np.uint8)
+    w = np.empty((N, K), dtype=np.float64) if sc is not None else None
+    st = _load().mxo_w8a16_unpack(_ptr(qw), _ptr(sc) if sc is not None else None, K, N,
+                                  group_size, _ptr(codes), _ptr(w) if w is not None else None)
+    _check(st, "w8a16_unpack")
+    return codes, w
+
+
+def w8a16_gemm(X_bits: np.ndarray, qweight: np.ndarray, scales: np.ndarray,
+               M: int, N: int, K: int, group_size: int = 128, nthreads: int = 1) -> np.ndarray:
+    """Y[M][N] in float64 (not rounded) of INT8 W8A16 weights."""
+    x = _c(X_bits, np.uint16)
+    qw = _c(qweight, np.int32)
+    sc = _c(scales, np.uint16)
+    Y = np.empty((M, N), dtype=np.float64)
+    _check(_load().mxo_w8a16_gemm(_ptr(x), _ptr(qw), _ptr(sc), M, N, K, group_size, _ptr(Y),
+                                  int(nthreads)), "w8a16_gemm")
     return Y

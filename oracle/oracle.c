@@ -25,6 +25,14 @@
  *    weight_packed[N][K/8] holds the code of row k = 8i + j of column n in
  *    bits [4j, 4j+3], the same code values as GPTQ, and weight_scale[N][K/G]
  *    holds scale (n, k / G); w[n][k] = (q - 8) * weight_scale[n][k / G].
+ *  - INT8 W8A16 vocabulary head (Eole Qwen3.8 recipe, section "Optional
+ *    vocabulary-head quantization": symmetric group-wise round-to-nearest
+ *    int8, group size 32, 64 or 128; the W4A16 LowLatency model card: the
+ *    INT8 lm_head is RTN g128 in compressed-tensors form).  Reading adopted:
+ *    the GPTQ packing with 8-bit codes, word (i, n) of qweight[K/4][N] holding
+ *    the code of row k = 4i + j in bits [8j, 8j+7] (least significant byte
+ *    first), the implicit zero point 128 of a symmetric 8-bit code, so
+ *    w[n][k] = (q - 128) * scale[k / G][n] with fp16 scales.
  *  - Dense bf16 projections with few output columns (Eole Qwen3.8 recipe,
  *    section "Pack inference projections": the paired 48 x 5120 GDN A/B
  *    projections in bf16).  Reading adopted: W[N][K] row-major (the Linear
@@ -433,4 +441,67 @@ int mxo_bf16_gemm(const uint16_t *X, const uint16_t *W, int M, int N, int K, dou
             Y[(size_t)m * N + n] = acc;
         }
     return 0;
+}
+
+/* INT8 code of (n, k): byte k % 4 of word (k / 4, n) of qweight[K/4][N]. */
+static int w8a16_code(const int32_t *qweight, int N, int n, int k)
+{
+    uint32_t word = (uint32_t)qweight[(size_t)(k / 4) * N + n];
+    return (int)((word >> (8 * (k % 4))) & 0xFFu);
+}
+
+static int w8a16_args_ok(int K, int N, int G)
+{
+    return K > 0 && N > 0 && G > 0 && K % 4 == 0 && K % G == 0;
+}
+
+/* Codes[N][K] (may be NULL) and exact weights (q - 128) * scale (may be NULL). */
+int mxo_w8a16_unpack(const int32_t *qweight, const uint16_t *scales, int K, int N, int G,
+                     uint8_t *codes, double *w)
+{
+    if (!qweight || !w8a16_args_ok(K, N, G) || (w && !scales))
+        return -1;
+    for (int n = 0; n < N; ++n)
+        for (int k = 0; k < K; ++k) {
+            int q = w8a16_code(qweight, N, n, k);
+            if (codes)
+                codes[(size_t)n * K + k] = (uint8_t)q;
+            if (w)
+                w[(size_t)n * K + k] =
+                    (double)(q - 128) * mxo_decode_fp16(scales[(size_t)(k / G) * N + n]);
+        }
+    return 0;
+}
+
+/* Y[M][N] = X * dequant(W)^T for INT8 W8A16 weights, fp64, k ascending. */
+int mxo_w8a16_gemm(const uint16_t *X, const int32_t *qweight, const uint16_t *scales,
+                   int M, int N, int K, int G, double *Y, int nthreads)
+{
+    if (!X || !qweight || !scales || !Y || M <= 0 || !w8a16_args_ok(K, N, G))
+        return -1;
+    if (nthreads < 1)
+        nthreads = 1;
+    int bad = 0;
+#pragma omp parallel num_threads(nthreads) reduction(| : bad)
+    {
+        double *w = (double *)malloc(sizeof(double) * (size_t)K);
+        if (!w)
+            bad = 1;
+#pragma omp for schedule(static)
+        for (int n = 0; n < N; ++n) {
+            if (!w)
+                continue;
+            for (int k = 0; k < K; ++k)
+                w[k] = (double)(w8a16_code(qweight, N, n, k) - 128) *
+                       mxo_decode_fp16(scales[(size_t)(k / G) * N + n]);
+            for (int m = 0; m < M; ++m) {
+                double acc = 0.0;
+                for (int k = 0; k < K; ++k)
+                    acc += mxo_decode_bf16(X[(size_t)m * K + k]) * w[k];
+                Y[(size_t)m * N + n] = acc;
+            }
+        }
+        free(w);
+    }
+    return bad ? -1 : 0;
 }

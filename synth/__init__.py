@@ -19,6 +19,9 @@ Recipes (value distributions of the workloads the layer is measured on):
 
 * Dense bf16 (the paired GDN A/B projection): W bf16(0.02*z) [N][K], X as
   above.
+* INT8 W8A16 (the vocabulary head): codes uniform in 0..255, packed 4 per
+  int32 word along K (code of row k = 4i + j in bits [8j, 8j+7] of word
+  (i, n)); scales fp16(1e-4 + 0.001*|z|) per (group, column); X as above.
 
 RNG: numpy ``Generator(PCG64)`` seeded from ``SeedSequence([seed, layer])``,
 spawned into three independent streams (codes, scales, X).
@@ -95,6 +98,32 @@ def mxfp8_layer(M: int, K: int, N: int, seed: int = 0, layer: int = 0,
     Ws = r_scales.integers(exp_lo, exp_hi + 1, size=(N, K // 32), dtype=np.uint8)
     X = bf16_bits_of_normals(r_x, (M, K))
     return Mxfp8Layer(M, K, N, X, Wq, Ws)
+
+
+@dataclass
+class Int8Layer:
+    M: int
+    K: int
+    N: int
+    group_size: int
+    X: np.ndarray        # uint16 bf16 bits [M][K]
+    codes: np.ndarray    # uint8 [N][K], 0..255
+    qweight: np.ndarray  # int32 [K/4][N]
+    scales: np.ndarray   # uint16 fp16 bits [K/G][N]
+
+
+def int8_layer(M: int, K: int, N: int, group_size: int = 128, seed: int = 0,
+               layer: int = 0) -> Int8Layer:
+    r_codes, r_scales, r_x = _streams(seed, layer)
+    codes = r_codes.integers(0, 256, size=(N, K), dtype=np.uint8)
+    z = r_scales.standard_normal(size=(K // group_size, N), dtype=np.float32)
+    scales = (1e-4 + 0.001 * np.abs(z.astype(np.float64))).astype(np.float16)
+    X = bf16_bits_of_normals(r_x, (M, K))
+    # codes[N][K] -> words[K/4][N]: byte j of word (i, n) is code (n, 4i + j)
+    qweight = np.ascontiguousarray(codes.T).reshape(K // 4, 4, N).transpose(0, 2, 1)
+    qweight = np.ascontiguousarray(qweight).view(np.uint32).reshape(K // 4, N).view(np.int32)
+    return Int8Layer(M, K, N, group_size, X, codes, np.ascontiguousarray(qweight),
+                     scales.view(np.uint16).copy())
 
 
 @dataclass

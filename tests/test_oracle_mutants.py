@@ -13,7 +13,8 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "oracle.c")
 PIN_SUITES = ["tests/test_oracle_formats.py", "tests/test_oracle_int4.py",
-              "tests/test_oracle_mxfp8.py", "tests/test_oracle_bf16.py"]
+              "tests/test_oracle_mxfp8.py", "tests/test_oracle_bf16.py",
+              "tests/test_oracle_int8.py"]
 
 MUTANTS = {
     "zero_point_7": ("return (double)(q - 8) * s;", "return (double)(q - 7) * s;"),
@@ -32,6 +33,8 @@ MUTANTS = {
     "mxfp8_block_index": ("Ws[(size_t)n * (K / 32) + k / 32]", "Ws[(size_t)n * (K / 32) + (k % 32) / 32]"),
     "bf16_gemm_reversed_w": ("mxo_decode_bf16(W[(size_t)n * K + k])", "mxo_decode_bf16(W[(size_t)n * K + (K - 1 - k)])"),
     "bf16_gemm_drops_last_k": ("            for (int k = 0; k < K; ++k)\n                acc += mxo_decode_bf16(X[(size_t)m * K + k]) * mxo_decode_bf16(W", "            for (int k = 0; k < K - 1; ++k)\n                acc += mxo_decode_bf16(X[(size_t)m * K + k]) * mxo_decode_bf16(W"),
+    "int8_byte_order_reversed": ("(word >> (8 * (k % 4)))", "(word >> (8 * (3 - k % 4)))"),
+    "int8_zero_point_127": ("(double)(w8a16_code(qweight, N, n, k) - 128)", "(double)(w8a16_code(qweight, N, n, k) - 127)"),
     "mxfp8_gemm_drops_scale": ("w[k] = mxfp8_weight(Wq, Ws, K, n, k);", "w[k] = mxo_decode_e4m3(Wq[(size_t)n * K + k]);"),
 }
 
