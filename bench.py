@@ -50,6 +50,8 @@ WORKLOADS = {
     "prefill_int4": ("int4", 8192, [(5120, 17408)], 128),
     "mxfp8_m4": ("mxfp8", 4, [(5120, 17408)], 32),
     "mxfp8_m128": ("mxfp8", 128, [(5120, 17408)], 32),
+    # the INT8 vocabulary head (248 k columns) at the verify chunk of one stream
+    "head_int8_m5": ("int8", 5, [(5120, 248320)], 128),
     # the paired dense bf16 GDN A/B projection (2 x 48 rows of 5120)
     "gdn_ab_bf16_m4": ("bf16", 4, [(5120, 96)], 0),
     "gdn_ab_bf16_m1": ("bf16", 1, [(5120, 96)], 0),
@@ -64,6 +66,8 @@ def layer_weight_bytes(fmt, K, N, G):
         return N * K // 2 + N * (K // G) * 2
     if fmt == "bf16":
         return N * K * 2
+    if fmt == "int8":
+        return N * K + N * (K // G) * 2
     return N * K + N * (K // 32)
 
 
@@ -196,6 +200,15 @@ def run_ours(args, rank, world, local_rank):
             weights.append([packed] + [packed.clone() for _ in range(pool - 1)])
             wss.append(torch.zeros(mxg.w4a16_workspace_bytes(M, N, K, G), dtype=torch.uint8,
                                    device=dev))
+        elif fmt == "int8":
+            lay = synth.int8_layer(M, K, N, G, seed=rank, layer=li)
+            qw = torch.from_numpy(lay.qweight).to(dev)
+            sc = torch.from_numpy(lay.scales.view(np.int16)).to(dev)
+            packed = mxg.w8a16_repack(qw, sc, G)
+            del qw, sc
+            weights.append([packed] + [packed.clone() for _ in range(pool - 1)])
+            wss.append(torch.zeros(mxg.raw_lib().w8a16_workspace_bytes(M, N, K, G),
+                                   dtype=torch.uint8, device=dev))
         elif fmt == "bf16":
             lay = synth.bf16_layer(M, K, N, seed=rank, layer=li)
             w = torch.from_numpy(lay.W.view(np.int16)).view(torch.bfloat16).to(dev)
@@ -218,6 +231,9 @@ def run_ours(args, rank, world, local_rank):
         K, N = layers[li]
         if fmt == "int4":
             mxg.w4a16_gemm(xs[li], weights[li][p], N, K, G, out=ys[li], workspace_buf=wss[li],
+                           stream=s)
+        elif fmt == "int8":
+            mxg.w8a16_gemm(xs[li], weights[li][p], N, K, G, out=ys[li], workspace_buf=wss[li],
                            stream=s)
         elif fmt == "bf16":
             mxg.bf16_gemm_small(xs[li], weights[li][p], out=ys[li], workspace_buf=wss[li],
@@ -320,6 +336,9 @@ def run_ours(args, rank, world, local_rank):
             if fmt == "int4":
                 c, _ = mxg.prepare_w4a16_gemm(dev_x[li], weights[li][p], N, K, G, out=dev_y[li],
                                               workspace_buf=wss[li], stream=stream)
+            elif fmt == "int8":
+                c, _ = mxg.prepare_w8a16_gemm(dev_x[li], weights[li][p], N, K, G, out=dev_y[li],
+                                              workspace_buf=wss[li], stream=stream)
             elif fmt == "bf16":
                 c, _ = mxg.prepare_bf16_gemm_small(dev_x[li], weights[li][p], out=dev_y[li],
                                                    workspace_buf=wss[li], stream=stream)
@@ -377,7 +396,7 @@ def run_ours(args, rank, world, local_rank):
                 "frac": round(achieved / peak, 4), "traffic": None,
                 "peak_source": f"{peak_kind} copy bandwidth"}
     kernel_name = ("bf16_small_kernel" if fmt == "bf16" else
-                   "w4a16_stream_kernel" if (fmt == "int4" and M <= 32) else
+                   "w4a16_stream_kernel" if (fmt in ("int4", "int8") and M <= 32) else
                    "mxfp8_stream_kernel" if M <= 32 else "tc_gemm_kernel")
     roof["kernel"] = kernel_name
     roof["per_layer_us"] = [round(k / kernel_launches * 1e3, 3) for k in kernel_ms]
@@ -402,7 +421,7 @@ def run_ours(args, rank, world, local_rank):
         "config": {
             "workload": args.workload,
             "format": fmt, "M": M, "layers_KxN": [f"{K}x{N}" for K, N in layers],
-            "group_size": G if fmt == "int4" else (32 if fmt == "mxfp8" else None),
+            "group_size": G if fmt in ("int4", "int8") else (32 if fmt == "mxfp8" else None),
             "weight_bytes_per_step": step_bytes, "flops_per_step": step_flops,
             "l2": f"rotating weight pool of {pool} copies ({pool * step_bytes / 1e6:.0f} MB >= "
                   f"{args.pool_factor:g} x L2)",
@@ -457,13 +476,15 @@ def oracle_step_runner(workload: str, cols_per_layer: int | None, seed: int = 0)
             lay = synth.int4_layer(M, K, N, G, seed=seed, layer=li)
         elif fmt == "bf16":
             lay = synth.bf16_layer(M, K, N, seed=seed, layer=li)
+        elif fmt == "int8":
+            lay = synth.int8_layer(M, K, N, G, seed=seed, layer=li)
         else:
             lay = synth.mxfp8_layer(M, K, N, seed=seed, layer=li)
         prepared.append((K, N, lay))
     state = {"off": 0}
 
     def slice_inputs(K, N, lay, c0, c1):
-        if fmt == "int4":
+        if fmt in ("int4", "int8"):
             return (np.ascontiguousarray(lay.qweight[:, c0:c1]),
                     np.ascontiguousarray(lay.scales[:, c0:c1]))
         if fmt == "bf16":
@@ -481,6 +502,8 @@ def oracle_step_runner(workload: str, cols_per_layer: int | None, seed: int = 0)
             n = c1 - c0
             if fmt == "int4":
                 oracle.w4a16_gemm(lay.X, a, b, M, n, K, G, nthreads=nthreads)
+            elif fmt == "int8":
+                oracle.w8a16_gemm(lay.X, a, b, M, n, K, G, nthreads=nthreads)
             elif fmt == "bf16":
                 oracle.bf16_gemm(lay.X, a, M, n, K)
             else:

@@ -174,6 +174,38 @@ MXG_API int w4a16_gemm(const void *X, const void *packed, int M, int N, int K, i
 MXG_API int w4a16_gemm_static_scratch(const void *X, const void *packed, int M, int N, int K,
                int group_size, void *Y, cudaStream_t stream);
 
+/* ------------------------------------------------------------------ INT8 */
+
+/* INT8 W8A16 for the vocabulary head (the Eole recipe, section "Optional
+ * vocabulary-head quantization": symmetric group-wise round-to-nearest int8,
+ * group size 32, 64 or 128; the W4A16 LowLatency model card: INT8 lm_head,
+ * RTN g128).  Codes q in 0..255, four per int32 word along K: the code of
+ * row k = 4i + j is bits [8j, 8j+7] of word (i, n) of qweight[K/4][N];
+ * w[n][k] = (q - 128) * scale[k / G][n], scales fp16 [K/G][N].  Only the
+ * weight-streaming path exists for INT8 (M <= 32: decode and verify chunks
+ * against a vocabulary-sized N).
+ *
+ * Re-packed bytes: N*K code bytes (the codes split into a low-nibble and a
+ * high-nibble plane, each in the INT4 layout) then 2*N*K/G scale bytes;
+ * 0 for a shape w8a16_repack rejects. */
+MXG_API size_t w8a16_packed_bytes(int K, int N, int group_size);
+
+/* Offline re-pack: qweight device int32 [K/4][N]; scales device fp16 bits
+ * [K/G][N]; packed device, w8a16_packed_bytes(K, N, G) bytes.
+ * Requirements as for w4a16_repack (G in {32, 64, 128}; K % 64 == 0;
+ * K % G == 0; N % 64 == 0), else MXG_ERR_UNSUPPORTED_SHAPE. */
+MXG_API int w8a16_repack(const int32_t *qweight, const uint16_t *scales, int K, int N,
+                 int group_size, void *packed, cudaStream_t stream);
+
+/* Workspace bytes w8a16_gemm needs (0 for a rejected shape or M > 32). */
+MXG_API size_t w8a16_workspace_bytes(int M, int N, int K, int group_size);
+
+/* Y = X * dequant(W)^T for INT8 weights re-packed by w8a16_repack.
+ * Arguments, workspace and errors as for w4a16_gemm; 1 <= M <= 32, else
+ * MXG_ERR_UNSUPPORTED_SHAPE. */
+MXG_API int w8a16_gemm(const void *X, const void *packed, int M, int N, int K, int group_size,
+               void *Y, void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* ----------------------------------------------------------------- MXFP8 */
 
 /* Workspace bytes mxfp8_gemm needs for this shape on the current device. */

@@ -51,6 +51,10 @@ _SIGS = {
     "mxfp8_dequant": (_i, [_p, _p, _i, _i, _p, _p]),
     "mxg_workspace_status": (_i, [_p, ctypes.POINTER(_i), _p]),
     "mxg_selftest_wait_timeout": (_i, [_p, _i, _p]),
+    "w8a16_packed_bytes": (_sz, [_i, _i, _i]),
+    "w8a16_repack": (_i, [_p, _p, _i, _i, _i, _p, _p]),
+    "w8a16_workspace_bytes": (_sz, [_i, _i, _i, _i]),
+    "w8a16_gemm": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _sz, _p]),
     "bf16_gemm_small_workspace_bytes": (_sz, [_i, _i, _i]),
     "bf16_gemm_small": (_i, [_p, _p, _i, _i, _i, _p, _p, _sz, _p]),
     "mxg_set_path": (_i, [_i]),
@@ -375,6 +379,61 @@ def mxg_workspace_status(workspace_buf: torch.Tensor, stream=None) -> int:
     _check(_lib.mxg_workspace_status(_ptr(workspace_buf), ctypes.byref(v), _stream(stream)),
            "mxg_workspace_status")
     return v.value
+
+
+def w8a16_repack(qweight: torch.Tensor, scales: torch.Tensor, group_size: int = 128,
+                 stream=None) -> torch.Tensor:
+    """Re-pack INT8 words qweight[K/4][N] (int32, 4 codes per word along K,
+    zero point 128) and scales[K/G][N] (fp16)."""
+    _need(qweight, torch.int32, "qweight")
+    _need_scales(scales, "scales")
+    K = qweight.shape[0] * 4
+    N = qweight.shape[1]
+    nbytes = int(_lib.w8a16_packed_bytes(K, N, group_size))
+    if nbytes == 0:
+        raise MxgError(MXG_ERR_UNSUPPORTED_SHAPE, "w8a16_repack")
+    packed = torch.empty(nbytes, dtype=torch.uint8, device=qweight.device)
+    _check(_lib.w8a16_repack(_ptr(qweight), _ptr(scales), K, N, group_size, _ptr(packed),
+                             _stream(stream)), "w8a16_repack")
+    return packed
+
+
+def w8a16_gemm(x: torch.Tensor, packed: torch.Tensor, N: int, K: int, group_size: int = 128,
+               out: torch.Tensor | None = None, workspace_buf: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """Y = x * dequant(W)^T for x bf16 [M][K] (M <= 32) and a re-packed INT8 weight."""
+    _need(x, torch.bfloat16, "x")
+    M = x.shape[0]
+    if x.dim() != 2 or x.shape[1] != K:
+        raise ValueError("x must be [M][K]")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(out, torch.bfloat16, "out")
+    need = int(_lib.w8a16_workspace_bytes(M, N, K, group_size))
+    if need == 0:
+        raise MxgError(MXG_ERR_UNSUPPORTED_SHAPE, "w8a16_gemm")
+    ws = workspace_buf if workspace_buf is not None else workspace(need, x.device, stream)
+    _check(_lib.w8a16_gemm(_ptr(x), _ptr(packed), M, N, K, group_size, _ptr(out), _ptr(ws),
+                           ws.numel(), _stream(stream)), "w8a16_gemm")
+    return out
+
+
+def prepare_w8a16_gemm(x: torch.Tensor, packed: torch.Tensor, N: int, K: int,
+                       group_size: int = 128, out: torch.Tensor | None = None,
+                       workspace_buf: torch.Tensor | None = None, stream=None):
+    """(call, out): ``call()`` runs w8a16_gemm(x, packed) into ``out``."""
+    _need(x, torch.bfloat16, "x")
+    M = x.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(out, torch.bfloat16, "out")
+    need = int(_lib.w8a16_workspace_bytes(M, N, K, group_size))
+    if need == 0:
+        raise MxgError(MXG_ERR_UNSUPPORTED_SHAPE, "w8a16_gemm")
+    ws = workspace_buf if workspace_buf is not None else workspace(need, x.device, stream)
+    args = (_ptr(x), _ptr(packed), M, N, K, group_size, _ptr(out), _ptr(ws), ws.numel(),
+            _stream(stream))
+    return PreparedCall(_lib.w8a16_gemm, args, "w8a16_gemm", (x, packed, out, ws, stream)), out
 
 
 def bf16_gemm_small(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = None,

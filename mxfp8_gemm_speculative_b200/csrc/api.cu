@@ -302,6 +302,54 @@ int w4a16_gemm(const void *X, const void *packed, int M, int N, int K, int group
     return MXG_ERR_UNSUPPORTED_SHAPE;
 }
 
+size_t w8a16_packed_bytes(int K, int N, int group_size)
+{
+    if (!w4a16_shape_ok(K, N, group_size))
+        return 0;
+    return (size_t)N * K + (size_t)N * (K / group_size) * 2;
+}
+
+int w8a16_repack(const int32_t *qweight, const uint16_t *scales, int K, int N, int group_size,
+                 void *packed, cudaStream_t stream)
+{
+    if (!aligned16(qweight) || !aligned16(scales) || !aligned16(packed))
+        return MXG_ERR_INVALID_ARG;
+    if (!w4a16_shape_ok(K, N, group_size))
+        return MXG_ERR_UNSUPPORTED_SHAPE;
+    return to_status(launch_w8a16_repack(qweight, scales, K, N, group_size, packed, stream));
+}
+
+size_t w8a16_workspace_bytes(int M, int N, int K, int group_size)
+{
+    if (M < 1 || M > 32 || !w4a16_shape_ok(K, N, group_size))
+        return 0;
+    const int dev = current_device();
+    if (dev < 0)
+        return 0;
+    StreamPlan sp;
+    if (!plan_w8a16_stream(dev, M, N, K, group_size, &sp))
+        return 0;
+    return make_workspace_map(sp.ntiles, sp.partial_bytes).total;
+}
+
+int w8a16_gemm(const void *X, const void *packed, int M, int N, int K, int group_size, void *Y,
+               void *workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    if (!aligned16(X) || !aligned16(packed) || !aligned16(Y) || !aligned16(workspace) || M < 1)
+        return MXG_ERR_INVALID_ARG;
+    if (M > 32 || !w4a16_shape_ok(K, N, group_size))
+        return MXG_ERR_UNSUPPORTED_SHAPE;
+    const int dev = current_device();
+    if (dev < 0)
+        return MXG_ERR_CUDA;
+    StreamPlan sp;
+    if (!plan_w8a16_stream(dev, M, N, K, group_size, &sp))
+        return MXG_ERR_UNSUPPORTED_SHAPE;
+    if (workspace_bytes < make_workspace_map(sp.ntiles, sp.partial_bytes).total)
+        return MXG_ERR_WORKSPACE;
+    return to_status(launch_w4a16_stream(sp, X, packed, M, N, K, group_size, Y, workspace, stream));
+}
+
 size_t mxfp8_workspace_bytes(int M, int N, int K)
 {
     if (M < 1 || !mxfp8_shape_ok(K, N))

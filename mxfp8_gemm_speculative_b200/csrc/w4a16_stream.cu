@@ -54,13 +54,15 @@ constexpr int kMinUnitsPerCta = 2 * kConsumers;  // shortest run
 
 // Group modes: 0 -> G = 128, 1 -> G = 64, 2 -> G = 32.  A unit (what one
 // ring slot holds) spans SU times max(G, 64) rows of K of one n32 tile.
-template <int GM, int SU>
+// P code planes: 1 for INT4; 2 for INT8, whose codes are stored as a plane
+// of low nibbles and a plane of high nibbles, each in the INT4 layout.
+template <int GM, int SU, int P = 1>
 struct Mode {
     static constexpr int kG = GM == 0 ? 128 : (GM == 1 ? 64 : 32);
     static constexpr int kChunks = (GM == 0 ? 2 : 1) * SU;    // k64 chunks per unit
     static constexpr int kGroups = (GM == 2 ? 2 : 1) * SU;    // scale groups per unit
     static constexpr int kStepsPerGroup = kG / 16;            // MMA k16 steps per group
-    static constexpr int kCode = kChunks * 1024;              // code bytes per unit
+    static constexpr int kCode = kChunks * 1024 * P;          // code bytes per unit
     static constexpr int kScale = kGroups * 64;               // scale bytes per unit
     // slots per warp: shallow rings (12 warps x 2-3 slots keep enough bytes in
     // flight) leave most of the SM's shared-memory/L1 split to L1, where the
@@ -72,9 +74,9 @@ struct Mode {
 // unit's codes, then its scales), kRed reduction buffers of kConsumers
 // fragments (segment s of the run uses buffer s mod kRed), one mbarrier per
 // slot, then per reduction buffer an arrival count and a use count.
-template <int TT, int GM, int SU>
+template <int TT, int GM, int SU, int P = 1>
 struct Smem {
-    using MD = Mode<GM, SU>;
+    using MD = Mode<GM, SU, P>;
     static constexpr int kFrag4 = 2 * TT * 32;                // float4 per warp fragment
     static constexpr int kSlot = (MD::kCode + MD::kScale + 127) / 128 * 128;
     // One reduction buffer: a warp that ends a segment before the previous
@@ -220,21 +222,21 @@ __device__ __forceinline__ void zero_acc(float (&a)[2][TT][4])
 }
 
 // Copies unit u (codes, then scales) into a ring slot; completion on `bar`.
-template <int GM, int SU>
+template <int GM, int SU, int P>
 __device__ __forceinline__ void fetch_unit(const Params &p, uint8_t *slot, uint64_t *bar, int u,
                                            uint64_t policy)
 {
-    using MD = Mode<GM, SU>;
+    using MD = Mode<GM, SU, P>;
     mbar_arrive_expect_tx(bar, MD::kCode + MD::kScale);
     bulk_g2s(slot, p.codes + (size_t)u * MD::kCode, MD::kCode, bar, policy);
     bulk_g2s(slot + MD::kCode, p.scales + (size_t)u * MD::kScale, MD::kScale, bar, policy);
 }
 
-template <int TT, int GM, int SU>
+template <int TT, int GM, int SU, int P>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) w4a16_stream_kernel(const Params p)
 {
-    using MD = Mode<GM, SU>;
-    using SL = Smem<TT, GM, SU>;
+    using MD = Mode<GM, SU, P>;
+    using SL = Smem<TT, GM, SU, P>;
     constexpr int kStages = MD::kStages;
     constexpr int F = 2 * TT;  // float4 per lane fragment
     extern __shared__ __align__(128) uint8_t smem[];
@@ -272,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) w4a16_stream_kernel(cons
     auto fill_ring = [&]() {
         if (lane == 0)
             for (int k = 0; k < kStages && warp + k * kConsumers < n; ++k)
-                fetch_unit<GM, SU>(p, ring + k * SL::kSlot, &full[k], U0 + warp + k * kConsumers,
+                fetch_unit<GM, SU, P>(p, ring + k * SL::kSlot, &full[k], U0 + warp + k * kConsumers,
                                    policy);
     };
     if (p.early)
@@ -320,6 +322,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) w4a16_stream_kernel(cons
 
     constexpr uint32_t kOnes = 0x3F803F80u;  // bf16 pair (1, 1)
     float acc[2][TT][4], part[2][TT][4], xsum[TT][4];
+    float parthi[P == 2 ? 2 : 1][TT][4];  // INT8: sums over the high-nibble plane
     bool ok = true;
     int i = warp;          // run index of this warp's next unit
     int slot = 0;          // ring slot of unit i
@@ -352,10 +355,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) w4a16_stream_kernel(cons
             const uint8_t *ss = st + MD::kCode;
 #pragma unroll
             for (int ch = 0; ch < MD::kChunks; ++ch) {
-                const uint8_t *cp = st + ch * 1024 + lane * 16;
+                // INT4: [half][lane][16 B]; INT8: [half][plane][lane][16 B]
+                const uint8_t *cp = st + ch * 1024 * P + lane * 16;
                 const uint4 wl = lds128(cp);
-                const uint4 wh = lds128(cp + 512);
+                const uint4 wh = lds128(cp + 512 * P);
                 const uint32_t w[2][4] = {{wl.x, wl.y, wl.z, wl.w}, {wh.x, wh.y, wh.z, wh.w}};
+                uint32_t whi[2][4] = {};
+                if constexpr (P == 2) {
+                    const uint4 ul = lds128(cp + 512);
+                    const uint4 uh = lds128(cp + 1536);
+                    whi[0][0] = ul.x; whi[0][1] = ul.y; whi[0][2] = ul.z; whi[0][3] = ul.w;
+                    whi[1][0] = uh.x; whi[1][1] = uh.y; whi[1][2] = uh.z; whi[1][3] = uh.w;
+                }
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int step = ch * 4 + j;  // k16 step inside the unit
@@ -386,6 +397,21 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) w4a16_stream_kernel(cons
                                 mma_bf16_16816(part[h][tt], a0, a1, a2, a3, xs[ch][tt][j].x,
                                                xs[ch][tt][j].y);
                         }
+                        if constexpr (P == 2) {
+                            const uint32_t b0 = int4_pair_plus128<0>(whi[h][j]);
+                            const uint32_t b1 = int4_pair_plus128<4>(whi[h][j]);
+                            const uint32_t b2 = int4_pair_plus128<8>(whi[h][j]);
+                            const uint32_t b3 = int4_pair_plus128<12>(whi[h][j]);
+#pragma unroll
+                            for (int tt = 0; tt < TT; ++tt) {
+                                if (first)
+                                    mma_bf16_16816_zero(parthi[h][tt], b0, b1, b2, b3,
+                                                        xs[ch][tt][j].x, xs[ch][tt][j].y);
+                                else
+                                    mma_bf16_16816(parthi[h][tt], b0, b1, b2, b3,
+                                                   xs[ch][tt][j].x, xs[ch][tt][j].y);
+                            }
+                        }
                     }
                     if ((step + 1) % MD::kStepsPerGroup == 0) {
                         // end of a scale group: the MMAs summed (128 + q) * x, so
@@ -402,7 +428,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) w4a16_stream_kernel(cons
 #pragma unroll
                                 for (int e = 0; e < 4; ++e) {
                                     // outputs e and e ^ 2 are rows g, g + 8 of token 2t + (e & 1)
-                                    const float v = fmaf(-136.f, xsum[tt][e & 1], part[h][tt][e]);
+                                    float v;
+                                    if constexpr (P == 2) {
+                                        // INT8 q = 16 hi + lo: the planes summed
+                                        // (128 + hi) x and (128 + lo) x, so
+                                        // sum (q - 128) x = 16 Phi + Plo - 2304 sum(x)
+                                        v = fmaf(16.f, parthi[h][tt][e], part[h][tt][e]);
+                                        v = fmaf(-2304.f, xsum[tt][e & 1], v);
+                                    } else {
+                                        v = fmaf(-136.f, xsum[tt][e & 1], part[h][tt][e]);
+                                    }
                                     acc[h][tt][e] = fmaf(v, sc[h][e >> 1], acc[h][tt][e]);
                                 }
                     }
@@ -412,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) w4a16_stream_kernel(cons
             // consumed above): refill it with this warp's unit kStages ahead
             __syncwarp();
             if (lane == 0 && i + kStages * kConsumers < n)
-                fetch_unit<GM, SU>(p, ring + slot * SL::kSlot, &full[slot],
+                fetch_unit<GM, SU, P>(p, ring + slot * SL::kSlot, &full[slot],
                                u + kStages * kConsumers, policy);
             if (kPipeX) {
 #pragma unroll
@@ -495,10 +530,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) w4a16_stream_kernel(cons
     }
 }
 
-template <int TT, int GM, int SU>
+template <int TT, int GM, int SU, int P = 1>
 const void *kernel_ptr()
 {
-    return reinterpret_cast<const void *>(&w4a16_stream_kernel<TT, GM, SU>);
+    return reinterpret_cast<const void *>(&w4a16_stream_kernel<TT, GM, SU, P>);
 }
 
 // SU = 2 (two scale-group spans per unit) for up to two token tiles,
@@ -514,17 +549,25 @@ const void *select_kernel(int tt, int variant)
     MXG_CASE(1, 0, 2) MXG_CASE(1, 1, 2) MXG_CASE(1, 2, 2)
     MXG_CASE(2, 0, 2) MXG_CASE(2, 1, 2) MXG_CASE(2, 2, 2)
 #undef MXG_CASE
+    // INT8 (two code planes), SU = 1: variant = 6 + gm
+#define MXG_CASE8(T, G_) \
+    if (tt == T && variant == 6 + G_) return kernel_ptr<T, G_, 1, 2>();
+    MXG_CASE8(1, 0) MXG_CASE8(1, 1) MXG_CASE8(1, 2)
+    MXG_CASE8(2, 0) MXG_CASE8(2, 1) MXG_CASE8(2, 2)
+    MXG_CASE8(3, 0) MXG_CASE8(3, 1) MXG_CASE8(3, 2)
+    MXG_CASE8(4, 0) MXG_CASE8(4, 1) MXG_CASE8(4, 2)
+#undef MXG_CASE8
     return nullptr;
 }
 
-template <int GM, int SU>
+template <int GM, int SU, int P = 1>
 size_t smem_bytes_gs(int tt)
 {
     switch (tt) {
-    case 1: return Smem<1, GM, SU>::kTotal;
-    case 2: return Smem<2, GM, SU>::kTotal;
-    case 3: return Smem<3, GM, 1>::kTotal;
-    default: return Smem<4, GM, 1>::kTotal;
+    case 1: return Smem<1, GM, SU, P>::kTotal;
+    case 2: return Smem<2, GM, SU, P>::kTotal;
+    case 3: return Smem<3, GM, 1, P>::kTotal;
+    default: return Smem<4, GM, 1, P>::kTotal;
     }
 }
 
@@ -536,7 +579,10 @@ size_t smem_bytes(int tt, int variant)
     case 2: return smem_bytes_gs<2, 1>(tt);
     case 3: return smem_bytes_gs<0, 2>(tt);
     case 4: return smem_bytes_gs<1, 2>(tt);
-    default: return smem_bytes_gs<2, 2>(tt);
+    case 5: return smem_bytes_gs<2, 2>(tt);
+    case 6: return smem_bytes_gs<0, 1, 2>(tt);
+    case 7: return smem_bytes_gs<1, 1, 2>(tt);
+    default: return smem_bytes_gs<2, 1, 2>(tt);
     }
 }
 
@@ -547,7 +593,10 @@ int group_mode(int G)
 
 }  // namespace
 
-bool plan_w4a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan)
+namespace {
+
+// bits: 4 (INT4) or 8 (INT8, two code planes, one scale-group span per unit)
+bool plan_stream(int device, int M, int N, int K, int G, int bits, StreamPlan *plan)
 {
     if (M < 1 || M > 32 || N % 32 != 0)
         return false;
@@ -555,8 +604,8 @@ bool plan_w4a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan)
     StreamPlan pl{};
     pl.tt = (M + 7) / 8;
     const int unit_k = std::max(G, 64);
-    const int su = (pl.tt <= 2 && (K / unit_k) % 2 == 0) ? 2 : 1;
-    pl.variant = group_mode(G) + 3 * (su - 1);
+    const int su = (bits == 4 && pl.tt <= 2 && (K / unit_k) % 2 == 0) ? 2 : 1;
+    pl.variant = bits == 8 ? 6 + group_mode(G) : group_mode(G) + 3 * (su - 1);
     pl.warps_per_cta = kConsumers;
     pl.smem = smem_bytes(pl.tt, pl.variant);
     if ((int)pl.smem > di.smem_optin)
@@ -573,7 +622,7 @@ bool plan_w4a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan)
         return false;
     // resident CTAs per SM for this variant: every CTA of the grid must be
     // resident at once (a cut tile's finishing CTA waits for the others)
-    static int occ_cache[4][6] = {};
+    static int occ_cache[4][9] = {};
     int &occ = occ_cache[pl.tt - 1][pl.variant];
     if (occ == 0) {
         if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem) !=
@@ -595,6 +644,18 @@ bool plan_w4a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan)
     return true;
 }
 
+}  // namespace
+
+bool plan_w4a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan)
+{
+    return plan_stream(device, M, N, K, G, 4, plan);
+}
+
+bool plan_w8a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan)
+{
+    return plan_stream(device, M, N, K, G, 8, plan);
+}
+
 cudaError_t launch_w4a16_stream(const StreamPlan &pl, const void *X, const void *packed, int M,
                                 int N, int K, int G, void *Y, void *workspace, cudaStream_t stream)
 {
@@ -606,7 +667,8 @@ cudaError_t launch_w4a16_stream(const StreamPlan &pl, const void *X, const void 
     Params p{};
     p.X = static_cast<const uint16_t *>(X);
     p.codes = static_cast<const uint8_t *>(packed);
-    p.scales = p.codes + (size_t)N * K / 2;
+    // codes take half a byte per weight (INT4) or one byte in two planes (INT8)
+    p.scales = p.codes + (pl.variant >= 6 ? (size_t)N * K : (size_t)N * K / 2);
     p.Y = static_cast<uint16_t *>(Y);
     p.early = early_weight_loads() ? 1 : 0;
     p.hdr = static_cast<WsHeader *>(workspace);

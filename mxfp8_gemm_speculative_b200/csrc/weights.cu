@@ -72,6 +72,53 @@ __global__ void repack_codes_kernel(const int32_t *__restrict__ qweight, int K, 
     out[idx] = make_uint4(words[0], words[1], words[2], words[3]);
 }
 
+// INT8 codes (4 per int32 word along K, byte j = row 4i + j, zero point
+// 128) into two planes in the INT4 layout: one output pair per (tile, k64
+// chunk, half, lane), the low-nibble plane's 16 bytes then, 512 bytes on,
+// the high-nibble plane's.  Word (i, n) sits at qweight[i * N + n].
+__global__ void repack8_codes_kernel(const int32_t *__restrict__ qweight, int K, int N,
+                                     uint8_t *__restrict__ out)
+{
+    const long long total = (long long)(N / 32) * (K / 64) * 64;
+    const long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+    if (idx >= total)
+        return;
+    const int lane = (int)(idx & 31);
+    const int h = (int)((idx >> 5) & 1);
+    const long long rest = idx >> 6;
+    const int kc_count = K / 64;
+    const int c = (int)(rest % kc_count);
+    const int T = (int)(rest / kc_count);
+    const int g = lane >> 2, t = lane & 3;
+    const int na = T * 32 + h * 16 + g, nb = na + 8;
+    uint32_t lo[4], hi[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int k0 = chunk_k0(c, t, j);  // a multiple of 4: one word holds k0 .. k0 + 3
+        const uint32_t qa = (uint32_t)qweight[(size_t)(k0 >> 2) * N + na];
+        const uint32_t qb = (uint32_t)qweight[(size_t)(k0 >> 2) * N + nb];
+        // nibble plane p of code r (r = 0..3) of column a / b
+        auto nib = [](uint32_t q, int r, int p) { return (q >> (8 * r + 4 * p)) & 0xFu; };
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            uint32_t w = 0;
+            w |= nib(qa, 0, p);
+            w |= nib(qa, 1, p) << 16;
+            w |= nib(qb, 0, p) << 4;
+            w |= nib(qb, 1, p) << 20;
+            w |= nib(qa, 2, p) << 8;
+            w |= nib(qa, 3, p) << 24;
+            w |= nib(qb, 2, p) << 12;
+            w |= nib(qb, 3, p) << 28;
+            (p ? hi : lo)[j] = w;
+        }
+    }
+    // [T][c][h][plane][lane][16 B]
+    uint4 *base = reinterpret_cast<uint4 *>(out) + ((((size_t)T * kc_count + c) * 2 + h) * 2) * 32;
+    base[lane] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    base[32 + lane] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+}
+
 // Scale (group, n) sits at scales[group * sg + n * sn]: sg = N, sn = 1 for
 // GPTQ scales[K/G][N]; sg = 1, sn = K/G for compressed-tensors
 // weight_scale[N][K/G].
@@ -233,6 +280,20 @@ cudaError_t launch_w4a16_repack(const int32_t *qweight, const uint16_t *scales, 
     const long long nsc = (long long)(N / 32) * (K / G) * 32;
     uint16_t *sc_out = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(packed) + (size_t)N * K / 2);
     repack_scales_kernel<<<blocks_for(nsc, 256), 256, 0, stream>>>(scales, K, N, G, sg, sn, sc_out);
+    repack_done_kernel<<<1, 32, 0, stream>>>();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_w8a16_repack(const int32_t *qweight, const uint16_t *scales, int K, int N, int G,
+                                void *packed, cudaStream_t stream)
+{
+    const long long npairs = (long long)(N / 32) * (K / 64) * 64;
+    repack8_codes_kernel<<<blocks_for(npairs, 256), 256, 0, stream>>>(
+        qweight, K, N, static_cast<uint8_t *>(packed));
+    const long long nsc = (long long)(N / 32) * (K / G) * 32;
+    uint16_t *sc_out = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(packed) + (size_t)N * K);
+    repack_scales_kernel<<<blocks_for(nsc, 256), 256, 0, stream>>>(scales, K, N, G, (size_t)N, 1,
+                                                                   sc_out);
     repack_done_kernel<<<1, 32, 0, stream>>>();
     return cudaGetLastError();
 }

@@ -94,6 +94,13 @@ def test_arguments_rejected_before_launch(mxg):
     assert lib.bf16_gemm_small(a, mis, 4, 96, 5120, a, a, 1 << 20, null) == mxg.MXG_ERR_INVALID_ARG
     assert lib.bf16_gemm_small(a, a, 4, 96, 5120, a, a, 256, null) == mxg.MXG_ERR_WORKSPACE
     assert lib.bf16_gemm_small_workspace_bytes(4, 96, 5120) > 256
+    # INT8: the streaming path only (M <= 32), shape rules of the INT4 re-pack
+    assert lib.w8a16_gemm(a, a, 33, 512, 512, 128, a, a, 1 << 20, null) == mxg.MXG_ERR_UNSUPPORTED_SHAPE
+    assert lib.w8a16_gemm(a, a, 5, 512, 512, 96, a, a, 1 << 20, null) == mxg.MXG_ERR_UNSUPPORTED_SHAPE
+    assert lib.w8a16_gemm(a, mis, 5, 512, 512, 128, a, a, 1 << 20, null) == mxg.MXG_ERR_INVALID_ARG
+    assert lib.w8a16_repack(a, a, 480, 512, 32, a, null) == mxg.MXG_ERR_UNSUPPORTED_SHAPE
+    assert lib.w8a16_packed_bytes(5120, 248320, 128) == 5120 * 248320 + 248320 * 40 * 2
+    assert lib.w8a16_workspace_bytes(33, 512, 512, 128) == 0
 
 
 def test_path_override_roundtrip(mxg):
