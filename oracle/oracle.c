@@ -468,7 +468,7 @@ int mxo_w8a16_unpack(const int32_t *qweight, const uint16_t *scales, int K, int 
                 codes[(size_t)n * K + k] = (uint8_t)q;
             if (w)
                 w[(size_t)n * K + k] =
-                    (double)(q - 128) * mxo_decode_fp16(scales[(size_t)(k / G) * N + n]);
+                    (double)(q - 128) * mxo_decode_fp16(scales[(size_t)N * (k / G) + n]);
         }
     return 0;
 }
@@ -493,7 +493,7 @@ int mxo_w8a16_gemm(const uint16_t *X, const int32_t *qweight, const uint16_t *sc
                 continue;
             for (int k = 0; k < K; ++k)
                 w[k] = (double)(w8a16_code(qweight, N, n, k) - 128) *
-                       mxo_decode_fp16(scales[(size_t)(k / G) * N + n]);
+                       mxo_decode_fp16(scales[(size_t)N * (k / G) + n]);
             for (int m = 0; m < M; ++m) {
                 double acc = 0.0;
                 for (int k = 0; k < K; ++k)

@@ -34,6 +34,7 @@ MUTANTS = {
     "bf16_gemm_reversed_w": ("mxo_decode_bf16(W[(size_t)n * K + k])", "mxo_decode_bf16(W[(size_t)n * K + (K - 1 - k)])"),
     "bf16_gemm_drops_last_k": ("            for (int k = 0; k < K; ++k)\n                acc += mxo_decode_bf16(X[(size_t)m * K + k]) * mxo_decode_bf16(W", "            for (int k = 0; k < K - 1; ++k)\n                acc += mxo_decode_bf16(X[(size_t)m * K + k]) * mxo_decode_bf16(W"),
     "int8_byte_order_reversed": ("(word >> (8 * (k % 4)))", "(word >> (8 * (3 - k % 4)))"),
+    "int8_gemm_group_fixed_128": ("mxo_decode_fp16(scales[(size_t)N * (k / G) + n]);\n            for (int m", "mxo_decode_fp16(scales[(size_t)N * (k / 128) + n]);\n            for (int m"),
     "int8_zero_point_127": ("(double)(w8a16_code(qweight, N, n, k) - 128)", "(double)(w8a16_code(qweight, N, n, k) - 127)"),
     "mxfp8_gemm_drops_scale": ("w[k] = mxfp8_weight(Wq, Ws, K, n, k);", "w[k] = mxo_decode_e4m3(Wq[(size_t)n * K + k]);"),
 }
