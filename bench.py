@@ -28,6 +28,7 @@ import json
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -95,7 +96,10 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+        # the raw samples (the JSON line carries their summary); MXG_CLOCKS_DIR
+        # keeps them somewhere else than the system temporary directory
+        base = os.environ.get("MXG_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(base, f"mxg_clocks_gpu{gpu_index}.csv")
 
     def start(self):
         try:
@@ -417,7 +421,7 @@ def run_ours(args, rank, world, local_rank):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16" if fmt == "int4" else "bf16",
-        "data": "synthetic (seeded; BASELINE value distributions)",
+        "data": "synthetic (seeded; the value distributions of the layer formats)",
         "config": {
             "workload": args.workload,
             "format": fmt, "M": M, "layers_KxN": [f"{K}x{N}" for K, N in layers],
@@ -586,7 +590,7 @@ def run_reference(args, rank, world):
         "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded; BASELINE value distributions)",
+        "data": "synthetic (seeded; the value distributions of the layer formats)",
         "config": {"workload": args.workload, "format": fmt, "M": M,
                    "layers_KxN": [f"{K}x{N}" for K, N in layers]},
         "cpu_baseline": {"value": value, "unit": unit, "cores": used, "kind": "oracle",
