@@ -30,6 +30,12 @@
 //    run: the other contributors (for whom it is the first tile of the run)
 //    published their fragments early, so it adds them in CTA order
 //    (deterministic) and writes bf16 Y.
+//
+// The same kernel runs INT8 W8A16 weights (the vocabulary head): their
+// re-pack splits each 8-bit code q = 16 hi + lo into a plane of low and a
+// plane of high nibbles in the INT4 layout, the kernel decodes both planes
+// with the same mask-and-or, runs one MMA per plane and forms
+// 16 * P_hi + P_lo - 2304 * (activation sum) per group.
 #include <algorithm>
 
 #include "common.cuh"
