@@ -21,6 +21,10 @@ const DeviceInfo &device_info(int device);
 //                            calls of any shape (each call leaves them zero)
 // [then ...)                 fp32 partial sums (scratch)
 constexpr size_t kMaxCounters = 65536;
+// Devices for which per-device launch state (function attributes, occupancy)
+// is cached.
+constexpr int kMaxDeviceCache = 64;
+
 struct WorkspaceMap {
     size_t counters_off;
     size_t counters;      // number of int counters

@@ -17,6 +17,7 @@
 //    results): hardware e4m3x2 -> f16x2, f16 -> f32, times 2^(E-127), one
 //    rounding to bf16.
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -490,8 +491,12 @@ bool plan_mxfp8_stream(int device, int M, int N, int K, StreamPlan *plan)
         return false;
     // every CTA of the grid must be resident at once (a cut tile's finishing
     // CTA waits for the others)
-    static int occ_cache[4][3] = {};
-    int &occ = occ_cache[pl.tt - 1][su];
+    // (function attributes and occupancy are per device: cached per device)
+    if (device < 0 || device >= kMaxDeviceCache)
+        return false;
+    static std::atomic<int> occ_cache[kMaxDeviceCache][4][3];
+    std::atomic<int> &occ_slot = occ_cache[device][pl.tt - 1][su];
+    int occ = occ_slot.load(std::memory_order_acquire);
     if (occ == 0) {
         if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem) !=
             cudaSuccess)
@@ -502,6 +507,7 @@ bool plan_mxfp8_stream(int device, int M, int N, int K, StreamPlan *plan)
             o < 1)
             return false;
         occ = std::min(o, 1);
+        occ_slot.store(occ, std::memory_order_release);
     }
     pl.Wt = (int)std::max<long long>(
         1, std::min<long long>((long long)di.sms * occ, pl.units / kMinUnitsPerCta));

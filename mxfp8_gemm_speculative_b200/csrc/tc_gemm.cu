@@ -31,6 +31,7 @@
 // CTA-wide abort flag, records MXG_ERR_TIMEOUT and every role drains to the
 // end, where tensor memory is released.
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -659,13 +660,20 @@ cudaError_t tc_launch(const TcPlan &pl, const CUtensorMap &xm, const CUtensorMap
                       const CUtensorMap &sm, TcParams p, cudaStream_t stream)
 {
     const void *fn = reinterpret_cast<const void *>(&tc_gemm_kernel<F, BT>);
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)Layout<F, BT>::smem_bytes);
+    // the attribute is per device: set once on each
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev < 0 || dev >= kMaxDeviceCache)
+        return cudaErrorInvalidDevice;
+    static std::atomic<bool> attr_set[kMaxDeviceCache];
+    if (!attr_set[dev].load(std::memory_order_acquire)) {
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)Layout<F, BT>::smem_bytes);
         if (e != cudaSuccess)
             return e;
-        attr_set = true;
+        attr_set[dev].store(true, std::memory_order_release);
     }
     void *args[] = {const_cast<CUtensorMap *>(&xm), const_cast<CUtensorMap *>(&wm),
                     const_cast<CUtensorMap *>(&sm), &p};

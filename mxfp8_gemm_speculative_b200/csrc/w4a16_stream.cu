@@ -37,6 +37,7 @@
 // with the same mask-and-or, runs one MMA per plane and forms
 // 16 * P_hi + P_lo - 2304 * (activation sum) per group.
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -628,8 +629,12 @@ bool plan_stream(int device, int M, int N, int K, int G, int bits, StreamPlan *p
         return false;
     // resident CTAs per SM for this variant: every CTA of the grid must be
     // resident at once (a cut tile's finishing CTA waits for the others)
-    static int occ_cache[4][9] = {};
-    int &occ = occ_cache[pl.tt - 1][pl.variant];
+    // (function attributes and occupancy are per device: cached per device)
+    if (device < 0 || device >= kMaxDeviceCache)
+        return false;
+    static std::atomic<int> occ_cache[kMaxDeviceCache][4][9];
+    std::atomic<int> &occ_slot = occ_cache[device][pl.tt - 1][pl.variant];
+    int occ = occ_slot.load(std::memory_order_acquire);
     if (occ == 0) {
         if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem) !=
             cudaSuccess)
@@ -640,6 +645,7 @@ bool plan_stream(int device, int M, int N, int K, int G, int bits, StreamPlan *p
             o < 1)
             return false;
         occ = std::min(o, kCtasPerSm);
+        occ_slot.store(occ, std::memory_order_release);
     }
     // kCtasPerSm CTAs per SM, but no run shorter than kMinUnitsPerCta units
     pl.Wt = (int)std::max<long long>(
