@@ -197,6 +197,15 @@ MXG_API size_t w8a16_packed_bytes(int K, int N, int group_size);
 MXG_API int w8a16_repack(const int32_t *qweight, const uint16_t *scales, int K, int N,
                  int group_size, void *packed, cudaStream_t stream);
 
+/* The same re-pack from the compressed-tensors export of the head (the W4A16
+ * LowLatency model card: the INT8 lm_head is written in compressed-tensors
+ * form): weight_packed device int32 [N][K/4] (word (n, i) holds rows
+ * 4i .. 4i+3 of column n, least significant byte first, same code values),
+ * weight_scale device fp16 bits [N][K/G].  The bytes written equal
+ * w8a16_repack of the transposed words and scales. */
+MXG_API int w8a16_repack_ct(const int32_t *weight_packed, const uint16_t *weight_scale, int K,
+                 int N, int group_size, void *packed, cudaStream_t stream);
+
 /* Workspace bytes w8a16_gemm needs (0 for a rejected shape or M > 32). */
 MXG_API size_t w8a16_workspace_bytes(int M, int N, int K, int group_size);
 

@@ -53,6 +53,7 @@ _SIGS = {
     "mxg_selftest_wait_timeout": (_i, [_p, _i, _p]),
     "w8a16_packed_bytes": (_sz, [_i, _i, _i]),
     "w8a16_repack": (_i, [_p, _p, _i, _i, _i, _p, _p]),
+    "w8a16_repack_ct": (_i, [_p, _p, _i, _i, _i, _p, _p]),
     "w8a16_workspace_bytes": (_sz, [_i, _i, _i, _i]),
     "w8a16_gemm": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _sz, _p]),
     "bf16_gemm_small_workspace_bytes": (_sz, [_i, _i, _i]),
@@ -395,6 +396,23 @@ def w8a16_repack(qweight: torch.Tensor, scales: torch.Tensor, group_size: int = 
     packed = torch.empty(nbytes, dtype=torch.uint8, device=qweight.device)
     _check(_lib.w8a16_repack(_ptr(qweight), _ptr(scales), K, N, group_size, _ptr(packed),
                              _stream(stream)), "w8a16_repack")
+    return packed
+
+
+def w8a16_repack_ct(weight_packed: torch.Tensor, weight_scale: torch.Tensor,
+                    group_size: int = 128, stream=None) -> torch.Tensor:
+    """Re-pack the compressed-tensors INT8 export weight_packed[N][K/4]
+    (int32) and weight_scale[N][K/G] (fp16) into the w8a16_repack buffer."""
+    _need(weight_packed, torch.int32, "weight_packed")
+    _need_scales(weight_scale, "weight_scale")
+    N = weight_packed.shape[0]
+    K = weight_packed.shape[1] * 4
+    nbytes = int(_lib.w8a16_packed_bytes(K, N, group_size))
+    if nbytes == 0:
+        raise MxgError(MXG_ERR_UNSUPPORTED_SHAPE, "w8a16_repack_ct")
+    packed = torch.empty(nbytes, dtype=torch.uint8, device=weight_packed.device)
+    _check(_lib.w8a16_repack_ct(_ptr(weight_packed), _ptr(weight_scale), K, N, group_size,
+                                _ptr(packed), _stream(stream)), "w8a16_repack_ct")
     return packed
 
 

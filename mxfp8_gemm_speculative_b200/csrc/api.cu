@@ -316,7 +316,18 @@ int w8a16_repack(const int32_t *qweight, const uint16_t *scales, int K, int N, i
         return MXG_ERR_INVALID_ARG;
     if (!w4a16_shape_ok(K, N, group_size))
         return MXG_ERR_UNSUPPORTED_SHAPE;
-    return to_status(launch_w8a16_repack(qweight, scales, K, N, group_size, packed, stream));
+    return to_status(launch_w8a16_repack(qweight, scales, K, N, group_size, false, packed, stream));
+}
+
+int w8a16_repack_ct(const int32_t *weight_packed, const uint16_t *weight_scale, int K, int N,
+                    int group_size, void *packed, cudaStream_t stream)
+{
+    if (!aligned16(weight_packed) || !aligned16(weight_scale) || !aligned16(packed))
+        return MXG_ERR_INVALID_ARG;
+    if (!w4a16_shape_ok(K, N, group_size))
+        return MXG_ERR_UNSUPPORTED_SHAPE;
+    return to_status(
+        launch_w8a16_repack(weight_packed, weight_scale, K, N, group_size, true, packed, stream));
 }
 
 size_t w8a16_workspace_bytes(int M, int N, int K, int group_size)

@@ -111,8 +111,9 @@ cudaError_t launch_w4a16_repack_part(const int32_t *qweight, const uint16_t *sca
 cudaError_t launch_repack_done(cudaStream_t stream);
 // INT8 W8A16: GPTQ-style words [K/4][N] with 8-bit codes into two INT4-layout
 // code planes ([N/32][K/64][2][2 planes][32][16 B], N*K bytes), then scales.
+// n_major: compressed-tensors inputs ([N][K/4] words, [N][K/G] scales).
 cudaError_t launch_w8a16_repack(const int32_t *qweight, const uint16_t *scales, int K, int N, int G,
-                                void *packed, cudaStream_t stream);
+                                bool n_major, void *packed, cudaStream_t stream);
 cudaError_t launch_w4a16_unpack(const void *packed, int K, int N, int G, uint8_t *codes,
                                 float *w_fp32, uint16_t *w_bf16, cudaStream_t stream);
 cudaError_t launch_mxfp8_dequant(const uint8_t *Wq, const uint8_t *Ws, int N, int K,

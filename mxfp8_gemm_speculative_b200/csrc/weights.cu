@@ -75,9 +75,11 @@ __global__ void repack_codes_kernel(const int32_t *__restrict__ qweight, int K, 
 // INT8 codes (4 per int32 word along K, byte j = row 4i + j, zero point
 // 128) into two planes in the INT4 layout: one output pair per (tile, k64
 // chunk, half, lane), the low-nibble plane's 16 bytes then, 512 bytes on,
-// the high-nibble plane's.  Word (i, n) sits at qweight[i * N + n].
-__global__ void repack8_codes_kernel(const int32_t *__restrict__ qweight, int K, int N,
-                                     uint8_t *__restrict__ out)
+// the high-nibble plane's.  Word (i, n) sits at qweight[i * wk + n * wn]:
+// wk = N, wn = 1 for GPTQ-style [K/4][N]; wk = 1, wn = K/4 for the
+// compressed-tensors [N][K/4] export.
+__global__ void repack8_codes_kernel(const int32_t *__restrict__ qweight, int K, int N, size_t wk,
+                                     size_t wn, uint8_t *__restrict__ out)
 {
     const long long total = (long long)(N / 32) * (K / 64) * 64;
     const long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x;
@@ -95,8 +97,8 @@ __global__ void repack8_codes_kernel(const int32_t *__restrict__ qweight, int K,
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int k0 = chunk_k0(c, t, j);  // a multiple of 4: one word holds k0 .. k0 + 3
-        const uint32_t qa = (uint32_t)qweight[(size_t)(k0 >> 2) * N + na];
-        const uint32_t qb = (uint32_t)qweight[(size_t)(k0 >> 2) * N + nb];
+        const uint32_t qa = (uint32_t)qweight[(size_t)(k0 >> 2) * wk + na * wn];
+        const uint32_t qb = (uint32_t)qweight[(size_t)(k0 >> 2) * wk + nb * wn];
         // nibble plane p of code r (r = 0..3) of column a / b
         auto nib = [](uint32_t q, int r, int p) { return (q >> (8 * r + 4 * p)) & 0xFu; };
 #pragma unroll
@@ -285,15 +287,16 @@ cudaError_t launch_w4a16_repack(const int32_t *qweight, const uint16_t *scales, 
 }
 
 cudaError_t launch_w8a16_repack(const int32_t *qweight, const uint16_t *scales, int K, int N, int G,
-                                void *packed, cudaStream_t stream)
+                                bool n_major, void *packed, cudaStream_t stream)
 {
+    const size_t wk = n_major ? 1 : (size_t)N, wn = n_major ? (size_t)K / 4 : 1;
+    const size_t sg = n_major ? 1 : (size_t)N, sn = n_major ? (size_t)(K / G) : 1;
     const long long npairs = (long long)(N / 32) * (K / 64) * 64;
     repack8_codes_kernel<<<blocks_for(npairs, 256), 256, 0, stream>>>(
-        qweight, K, N, static_cast<uint8_t *>(packed));
+        qweight, K, N, wk, wn, static_cast<uint8_t *>(packed));
     const long long nsc = (long long)(N / 32) * (K / G) * 32;
     uint16_t *sc_out = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(packed) + (size_t)N * K);
-    repack_scales_kernel<<<blocks_for(nsc, 256), 256, 0, stream>>>(scales, K, N, G, (size_t)N, 1,
-                                                                   sc_out);
+    repack_scales_kernel<<<blocks_for(nsc, 256), 256, 0, stream>>>(scales, K, N, G, sg, sn, sc_out);
     repack_done_kernel<<<1, 32, 0, stream>>>();
     return cudaGetLastError();
 }

@@ -99,6 +99,8 @@ def test_arguments_rejected_before_launch(mxg):
     assert lib.w8a16_gemm(a, a, 5, 512, 512, 96, a, a, 1 << 20, null) == mxg.MXG_ERR_UNSUPPORTED_SHAPE
     assert lib.w8a16_gemm(a, mis, 5, 512, 512, 128, a, a, 1 << 20, null) == mxg.MXG_ERR_INVALID_ARG
     assert lib.w8a16_repack(a, a, 480, 512, 32, a, null) == mxg.MXG_ERR_UNSUPPORTED_SHAPE
+    assert lib.w8a16_repack_ct(a, a, 480, 512, 32, a, null) == mxg.MXG_ERR_UNSUPPORTED_SHAPE
+    assert lib.w8a16_repack_ct(a, mis, 512, 512, 32, a, null) == mxg.MXG_ERR_INVALID_ARG
     assert lib.w8a16_packed_bytes(5120, 248320, 128) == 5120 * 248320 + 248320 * 40 * 2
     assert lib.w8a16_workspace_bytes(33, 512, 512, 128) == 0
 

@@ -71,3 +71,18 @@ def test_int8_vocab_head_sampled(mxg):
     rms = float(np.sqrt(np.mean(ref ** 2)))
     assert_sampled_parity(y[:, cols].ravel(), ref.ravel(), rms, "INT8 head")
     assert np.isfinite(y).all()
+
+
+@pytest.mark.parametrize("K,N,G", [(512, 512, 128), (1024, 192, 64), (256, 320, 32)])
+def test_int8_repack_ct_matches(mxg, K, N, G):
+    """The compressed-tensors export ([N][K/4] words, [N][K/G] scales: the
+    GPTQ-style ones transposed) re-packs to the same bytes."""
+    lay = synth.int8_layer(3, K, N, G, seed=K + N)
+    qw = torch.from_numpy(lay.qweight).to(DEV)
+    sc = torch.from_numpy(lay.scales.view(np.int16)).to(DEV)
+    ref = mxg.w8a16_repack(qw, sc, G)
+    wp = torch.from_numpy(np.ascontiguousarray(lay.qweight.T)).to(DEV)
+    ws = torch.from_numpy(np.ascontiguousarray(lay.scales.T).view(np.int16)).to(DEV)
+    packed = mxg.w8a16_repack_ct(wp, ws, G)
+    torch.cuda.synchronize()
+    assert torch.equal(packed, ref)
