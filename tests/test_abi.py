@@ -119,3 +119,20 @@ def test_early_weight_loads_roundtrip(mxg):
     with pytest.raises(ValueError):
         mxg.mxg_set_early_weight_loads(2)
     assert mxg.mxg_set_early_weight_loads(1) == 1
+
+
+def test_binding_refuses_to_load_without_the_library(tmp_path):
+    """No CPU fallback: a copy of the binding without libmxg.so next to it
+    raises at import."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = tmp_path / "mxfp8_gemm_speculative_b200"
+    pkg.mkdir()
+    src = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                       "mxfp8_gemm_speculative_b200", "__init__.py")
+    shutil.copy(src, pkg / "__init__.py")
+    r = subprocess.run([sys.executable, "-c", "import mxfp8_gemm_speculative_b200"],
+                       cwd=tmp_path, capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0
+    assert "is missing" in r.stderr and "no fallback" in r.stderr
