@@ -10,7 +10,12 @@ value      weight-stream TB/s: (code + scale bytes of every layer in the step)
            / device time per step, whole job (all ranks).  For tensor-bound
            workloads the line's unit is TFLOP/s (2*M*N*K per layer).
 e2e        the same metric through the Python binding with host buffers:
-           every step copies X from pinned host memory and reads Y back.
+           every step copies X from pinned host memory and reads Y back (the
+           step, copies included, replayed as a CUDA graph per pool slot).
+Workloads  --workload picks the step: the MTP4 verify layers (default; also
+           with gate/up fused), the C32 MTP3 chunk (M = 128), a prefill chunk
+           (M = 8192), MXFP8 at M = 4 and 128, the INT8 vocabulary head and
+           the paired bf16 GDN A/B projection.
 roofline   the dominant kernel's algorithmic bytes (or flops) per launch over
            its average launch time, timed with CUDA events on its stream,
            against MEASURED_PEAKS.json.
