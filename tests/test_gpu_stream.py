@@ -354,3 +354,29 @@ def test_repack_fused_matches_concatenated_repack(mxg, K, Ns, G, M):
         want = oracle.w4a16_gemm(lays[0].X, lay.qweight, lay.scales, M, n, K, G)
         assert_parity(y[:, n0:n0 + n], want, f"fused part at column {n0}")
         n0 += n
+
+
+def test_tensor_parallel_shards_on_one_gpu(mxg):
+    """Column and row shards of one layer (as two ranks would hold them),
+    re-packed and run one after the other on this GPU: the column blocks are
+    the layer's columns, the row partials add up to the layer (the sum that
+    the row-parallel all-reduce does across GPUs is done here on the host)."""
+    from mxfp8_gemm_speculative_b200 import tp
+    M, K, N, G, P = 5, 2048, 1024, 128, 2
+    lay = synth.int4_layer(M, K, N, G, seed=12)
+    qw, sc = int4_device(lay)
+    x = bf16_tensor(lay.X, DEV)
+    ref = oracle.w4a16_gemm(lay.X, lay.qweight, lay.scales, M, N, K, G)
+    cols = []
+    for r in range(P):
+        q, s, n0, n1 = tp.column_shard(qw, sc, r, P)
+        packed = mxg.w4a16_repack(q.contiguous(), s.contiguous(), G)
+        cols.append(to_f64(mxg.w4a16_gemm(x, packed, n1 - n0, K, G)))
+    assert_parity(np.concatenate(cols, axis=1), ref, "column-parallel shards")
+    total = np.zeros((M, N))
+    for r in range(P):
+        q, s, k0, k1 = tp.row_shard(qw, sc, G, r, P)
+        packed = mxg.w4a16_repack(q.contiguous(), s.contiguous(), G)
+        y = tp.row_parallel_w4a16_gemm(x[:, k0:k1].contiguous(), packed, N, k1 - k0, G)
+        total += to_f64(y)
+    assert_parity(total, ref, "row-parallel shards")
