@@ -97,3 +97,16 @@ def test_invalid_arguments(orc):
     with pytest.raises(Exception):
         orc.w8a16_gemm(np.zeros((1, 64), np.uint16), np.zeros((16, 8), np.int32),
                        np.zeros((2, 8), np.uint16), 1, 8, 64, 48)
+
+
+def test_int8_with_int4_codes_equals_int4(orc):
+    """INT8 codes q + 120 for INT4 codes q (so q8 - 128 = q - 8) with the same
+    scales give the INT4 layer's Y exactly: the two formats' oracles agree."""
+    M, K, N, G = 3, 256, 32, 64
+    lay4 = synth.int4_layer(M, K, N, G, seed=21)
+    codes8 = (lay4.codes.astype(np.int32) + 120).astype(np.uint8)
+    qw8 = np.ascontiguousarray(codes8.T).reshape(K // 4, 4, N).transpose(0, 2, 1)
+    qw8 = np.ascontiguousarray(qw8).view(np.uint32).reshape(K // 4, N).view(np.int32)
+    y8 = orc.w8a16_gemm(lay4.X, qw8, lay4.scales, M, N, K, G)
+    y4 = orc.w4a16_gemm(lay4.X, lay4.qweight, lay4.scales, M, N, K, G)
+    assert np.array_equal(y8, y4)
