@@ -647,9 +647,14 @@ bool plan_stream(int device, int M, int N, int K, int G, int bits, StreamPlan *p
         occ = std::min(o, kCtasPerSm);
         occ_slot.store(occ, std::memory_order_release);
     }
-    // kCtasPerSm CTAs per SM, but no run shorter than kMinUnitsPerCta units
-    pl.Wt = (int)std::max<long long>(
-        1, std::min<long long>((long long)di.sms * occ, pl.units / kMinUnitsPerCta));
+    // kCtasPerSm CTAs per SM, but no run shorter than kMinUnitsPerCta units;
+    // a layer too small for 32 such runs gets at least one CTA per n32 tile
+    // instead (one CTA streaming many short tiles would serialise their
+    // reductions)
+    long long wt = std::min<long long>((long long)di.sms * occ, pl.units / kMinUnitsPerCta);
+    if (wt < 32)
+        wt = std::min<long long>((long long)di.sms * occ, std::max<long long>(wt, pl.ntiles));
+    pl.Wt = (int)std::max<long long>(1, wt);
     pl.grid = pl.Wt;
     pl.partial_bytes = (size_t)pl.Wt * (2 * pl.tt * 32) * sizeof(float4);
     *plan = pl;
