@@ -509,8 +509,13 @@ bool plan_mxfp8_stream(int device, int M, int N, int K, StreamPlan *plan)
         occ = std::min(o, 1);
         occ_slot.store(occ, std::memory_order_release);
     }
-    pl.Wt = (int)std::max<long long>(
-        1, std::min<long long>((long long)di.sms * occ, pl.units / kMinUnitsPerCta));
+    // no run shorter than kMinUnitsPerCta units; a layer too small for 32
+    // such runs gets at least one CTA per n16 tile instead (one CTA streaming
+    // many short tiles would serialise their reductions)
+    long long wt = std::min<long long>((long long)di.sms * occ, pl.units / kMinUnitsPerCta);
+    if (wt < 32)
+        wt = std::min<long long>((long long)di.sms * occ, std::max<long long>(wt, pl.ntiles));
+    pl.Wt = (int)std::max<long long>(1, wt);
     pl.grid = pl.Wt;
     pl.partial_bytes = (size_t)pl.Wt * pl.tt * 32 * sizeof(float4);
     *plan = pl;
