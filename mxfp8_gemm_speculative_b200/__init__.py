@@ -109,6 +109,62 @@ def _need(t: torch.Tensor, dtype, name: str) -> None:
         raise ValueError(f"{name} must be contiguous")
 
 
+# The C ABI takes plain pointers and cannot see buffer sizes: the binding
+# checks every buffer a kernel reads or writes against the call's shape
+# (type, then size, then layout and device), so a mismatch raises here
+# instead of reaching memory past the end of a tensor.
+def _same_device(t: torch.Tensor, device, name: str) -> None:
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+
+
+def _need_out(out: torch.Tensor, M: int, N: int, device) -> None:
+    if out.dtype != torch.bfloat16:
+        raise ValueError(f"out must be torch.bfloat16, got {out.dtype}")
+    if tuple(out.shape) != (M, N):
+        raise ValueError(f"out must be [{M}][{N}], got {list(out.shape)}")
+    _need(out, torch.bfloat16, "out")
+    _same_device(out, device, "out")
+
+
+def _need_weights(t: torch.Tensor, dtype, nbytes: int, device, name: str) -> None:
+    """t holds at least nbytes bytes of weights (nbytes = 0: a shape the
+    library rejects itself, with its own status)."""
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if nbytes and t.numel() * t.element_size() < nbytes:
+        raise ValueError(f"{name} holds {t.numel() * t.element_size()} bytes, the shape needs "
+                         f"{nbytes}")
+    _need(t, dtype, name)
+    _same_device(t, device, name)
+
+
+def _need_ws(ws: torch.Tensor, device) -> None:
+    if ws.dtype != torch.uint8:
+        raise ValueError(f"workspace_buf must be torch.uint8, got {ws.dtype}")
+    _need(ws, torch.uint8, "workspace_buf")
+    _same_device(ws, device, "workspace_buf")
+
+
+def _gemm_buffers(x: torch.Tensor, K: int, N: int, out, workspace_buf, need_ws, stream):
+    """(M, out, ws) for a GEMM on x [M][K]: `out` and `workspace_buf` checked,
+    or made (a [M][N] bf16 output; the cached workspace of `need_ws()`
+    bytes)."""
+    _need(x, torch.bfloat16, "x")
+    if x.dim() != 2 or x.shape[1] != K:
+        raise ValueError(f"x must be [M][{K}], got {list(x.shape)}")
+    M = x.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need_out(out, M, N, x.device)
+    if workspace_buf is None:
+        ws = workspace(need_ws(), x.device, stream)
+    else:
+        ws = workspace_buf
+        _need_ws(ws, x.device)
+    return M, out, ws
+
+
 # ------------------------------------------------------------- workspaces
 _ws_lock = threading.Lock()
 _ws_cache: dict[tuple[int, int], torch.Tensor] = {}
@@ -223,15 +279,10 @@ def w4a16_gemm(x: torch.Tensor, packed: torch.Tensor, N: int, K: int, group_size
                out: torch.Tensor | None = None, workspace_buf: torch.Tensor | None = None,
                stream=None) -> torch.Tensor:
     """Y = x * dequant(W)^T for x bf16 [M][K] and a re-packed INT4 weight."""
-    _need(x, torch.bfloat16, "x")
-    M = x.shape[0]
-    if x.dim() != 2 or x.shape[1] != K:
-        raise ValueError("x must be [M][K]")
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    _need(out, torch.bfloat16, "out")
-    ws = (workspace_buf if workspace_buf is not None else
-          workspace(_need_bytes("w4a16", x.device.index, M, N, K, group_size), x.device, stream))
+    M, out, ws = _gemm_buffers(
+        x, K, N, out, workspace_buf,
+        lambda: _need_bytes("w4a16", x.device.index, x.shape[0], N, K, group_size), stream)
+    _need_weights(packed, torch.uint8, w4a16_packed_bytes(K, N, group_size), x.device, "packed")
     _check(_lib.w4a16_gemm(_ptr(x), _ptr(packed), M, N, K, group_size, _ptr(out), _ptr(ws),
                            ws.numel(), _stream(stream)), "w4a16_gemm")
     return out
@@ -256,15 +307,10 @@ def prepare_w4a16_gemm(x: torch.Tensor, packed: torch.Tensor, N: int, K: int,
                        group_size: int = 128, out: torch.Tensor | None = None,
                        workspace_buf: torch.Tensor | None = None, stream=None):
     """(call, out): ``call()`` runs w4a16_gemm(x, packed) into ``out``."""
-    _need(x, torch.bfloat16, "x")
-    M = x.shape[0]
-    if x.dim() != 2 or x.shape[1] != K:
-        raise ValueError("x must be [M][K]")
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    _need(out, torch.bfloat16, "out")
-    ws = (workspace_buf if workspace_buf is not None else
-          workspace(_need_bytes("w4a16", x.device.index, M, N, K, group_size), x.device, stream))
+    M, out, ws = _gemm_buffers(
+        x, K, N, out, workspace_buf,
+        lambda: _need_bytes("w4a16", x.device.index, x.shape[0], N, K, group_size), stream)
+    _need_weights(packed, torch.uint8, w4a16_packed_bytes(K, N, group_size), x.device, "packed")
     args = (_ptr(x), _ptr(packed), M, N, K, group_size, _ptr(out), _ptr(ws), ws.numel(),
             _stream(stream))
     return PreparedCall(_lib.w4a16_gemm, args, "w4a16_gemm", (x, packed, out, ws, stream)), out
@@ -274,16 +320,9 @@ def prepare_mxfp8_gemm(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor,
                        out: torch.Tensor | None = None, workspace_buf: torch.Tensor | None = None,
                        stream=None):
     """(call, out): ``call()`` runs mxfp8_gemm(x, wq, ws) into ``out``."""
-    _need(x, torch.bfloat16, "x")
-    M, K = x.shape
-    N = wq.shape[0]
-    if wq.shape[1] != K or ws.shape != (N, K // 32):
-        raise ValueError("shape mismatch between x, wq and ws")
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    _need(out, torch.bfloat16, "out")
-    wsb = (workspace_buf if workspace_buf is not None else
-           workspace(_need_bytes("mxfp8", x.device.index, M, N, K), x.device, stream))
+    M, K, N = _mx_shapes(x, wq, ws)
+    M, out, wsb = _gemm_buffers(x, K, N, out, workspace_buf,
+                                lambda: _need_bytes("mxfp8", x.device.index, M, N, K), stream)
     args = (_ptr(x), _ptr(wq), _ptr(ws), M, N, K, _ptr(out), _ptr(wsb), wsb.numel(),
             _stream(stream))
     return PreparedCall(_lib.mxfp8_gemm, args, "mxfp8_gemm", (x, wq, ws, out, wsb, stream)), out
@@ -292,19 +331,8 @@ def prepare_mxfp8_gemm(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor,
 def prepare_bf16_gemm_small(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = None,
                             workspace_buf: torch.Tensor | None = None, stream=None):
     """(call, out): ``call()`` runs bf16_gemm_small(x, w) into ``out``."""
-    _need(x, torch.bfloat16, "x")
-    _need(w, torch.bfloat16, "w")
-    M, K = x.shape
-    N = w.shape[0]
-    if w.shape[1] != K:
-        raise ValueError("x must be [M][K] and w [N][K]")
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    _need(out, torch.bfloat16, "out")
-    need = int(_lib.bf16_gemm_small_workspace_bytes(M, N, K))
-    if need == 0:
-        raise MxgError(MXG_ERR_UNSUPPORTED_SHAPE, "bf16_gemm_small")
-    wsb = workspace_buf if workspace_buf is not None else workspace(need, x.device, stream)
+    M, K, N, need = _small_shapes(x, w)
+    M, out, wsb = _gemm_buffers(x, K, N, out, workspace_buf, lambda: need, stream)
     args = (_ptr(x), _ptr(w), M, N, K, _ptr(out), _ptr(wsb), wsb.numel(), _stream(stream))
     return PreparedCall(_lib.bf16_gemm_small, args, "bf16_gemm_small", (x, w, out, wsb, stream)), out
 
@@ -314,12 +342,13 @@ def w4a16_gemm_static_scratch(x: torch.Tensor, packed: torch.Tensor, N: int, K: 
                               stream=None) -> torch.Tensor:
     """w4a16_gemm (M <= 32) with the library's fixed device scratch instead of a workspace."""
     _need(x, torch.bfloat16, "x")
-    M = x.shape[0]
     if x.dim() != 2 or x.shape[1] != K:
-        raise ValueError("x must be [M][K]")
+        raise ValueError(f"x must be [M][{K}], got {list(x.shape)}")
+    M = x.shape[0]
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    _need(out, torch.bfloat16, "out")
+    _need_out(out, M, N, x.device)
+    _need_weights(packed, torch.uint8, w4a16_packed_bytes(K, N, group_size), x.device, "packed")
     _check(_lib.w4a16_gemm_static_scratch(_ptr(x), _ptr(packed), M, N, K, group_size, _ptr(out),
                                           _stream(stream)), "w4a16_gemm_static_scratch")
     return out
@@ -328,6 +357,7 @@ def w4a16_gemm_static_scratch(x: torch.Tensor, packed: torch.Tensor, N: int, K: 
 def w4a16_unpack(packed: torch.Tensor, K: int, N: int, group_size: int = 128, stream=None):
     """(codes uint8 [N][K], w_fp32 float32 [N][K], w_bf16 bfloat16 [N][K])."""
     dev = packed.device
+    _need_weights(packed, torch.uint8, w4a16_packed_bytes(K, N, group_size), dev, "packed")
     codes = torch.empty((N, K), dtype=torch.uint8, device=dev)
     w32 = torch.empty((N, K), dtype=torch.float32, device=dev)
     w16 = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
@@ -337,6 +367,26 @@ def w4a16_unpack(packed: torch.Tensor, K: int, N: int, group_size: int = 128, st
 
 
 # ------------------------------------------------------------------- MXFP8
+def _mx_shapes(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor):
+    """(M, K, N) of x [M][K] against E4M3 wq [N][K] and E8M0 ws [N][K/32]."""
+    _need(x, torch.bfloat16, "x")
+    if wq.dtype not in (torch.uint8, torch.float8_e4m3fn):
+        raise ValueError("wq must be uint8 or float8_e4m3fn")
+    if ws.dtype not in (torch.uint8, torch.float8_e8m0fnu):
+        raise ValueError("ws must be uint8 or float8_e8m0fnu")
+    if x.dim() != 2 or wq.dim() != 2 or ws.dim() != 2:
+        raise ValueError("x, wq and ws must be 2-D")
+    M, K = x.shape
+    N = wq.shape[0]
+    if wq.shape[1] != K or ws.shape[0] != N or ws.shape[1] * 32 != K:
+        raise ValueError("shape mismatch between x, wq and ws")
+    _need(wq, wq.dtype, "wq")
+    _need(ws, ws.dtype, "ws")
+    _same_device(wq, x.device, "wq")
+    _same_device(ws, x.device, "ws")
+    return M, K, N
+
+
 def mxfp8_workspace_bytes(M: int, N: int, K: int) -> int:
     return int(_lib.mxfp8_workspace_bytes(M, N, K))
 
@@ -345,22 +395,9 @@ def mxfp8_gemm(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor,
                out: torch.Tensor | None = None, workspace_buf: torch.Tensor | None = None,
                stream=None) -> torch.Tensor:
     """Y = x * dequant(W)^T for x bf16 [M][K], E4M3 codes wq[N][K], E8M0 ws[N][K/32]."""
-    _need(x, torch.bfloat16, "x")
-    if wq.dtype not in (torch.uint8, torch.float8_e4m3fn):
-        raise ValueError("wq must be uint8 or float8_e4m3fn")
-    if ws.dtype not in (torch.uint8, torch.float8_e8m0fnu):
-        raise ValueError("ws must be uint8 or float8_e8m0fnu")
-    _need(wq, wq.dtype, "wq")
-    _need(ws, ws.dtype, "ws")
-    M, K = x.shape
-    N = wq.shape[0]
-    if wq.shape[1] != K or ws.shape[0] != N or ws.shape[1] * 32 != K:
-        raise ValueError("shape mismatch between x, wq and ws")
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    _need(out, torch.bfloat16, "out")
-    wsb = (workspace_buf if workspace_buf is not None else
-           workspace(_need_bytes("mxfp8", x.device.index, M, N, K), x.device, stream))
+    M, K, N = _mx_shapes(x, wq, ws)
+    M, out, wsb = _gemm_buffers(x, K, N, out, workspace_buf,
+                                lambda: _need_bytes("mxfp8", x.device.index, M, N, K), stream)
     _check(_lib.mxfp8_gemm(_ptr(x), _ptr(wq), _ptr(ws), M, N, K, _ptr(out), _ptr(wsb),
                            wsb.numel(), _stream(stream)), "mxfp8_gemm")
     return out
@@ -416,21 +453,21 @@ def w8a16_repack_ct(weight_packed: torch.Tensor, weight_scale: torch.Tensor,
     return packed
 
 
+def _w8_ws_bytes(M: int, N: int, K: int, group_size: int) -> int:
+    need = int(_lib.w8a16_workspace_bytes(M, N, K, group_size))
+    if need == 0:
+        raise MxgError(MXG_ERR_UNSUPPORTED_SHAPE, "w8a16_gemm")
+    return need
+
+
 def w8a16_gemm(x: torch.Tensor, packed: torch.Tensor, N: int, K: int, group_size: int = 128,
                out: torch.Tensor | None = None, workspace_buf: torch.Tensor | None = None,
                stream=None) -> torch.Tensor:
     """Y = x * dequant(W)^T for x bf16 [M][K] (M <= 32) and a re-packed INT8 weight."""
-    _need(x, torch.bfloat16, "x")
-    M = x.shape[0]
-    if x.dim() != 2 or x.shape[1] != K:
-        raise ValueError("x must be [M][K]")
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    _need(out, torch.bfloat16, "out")
-    need = int(_lib.w8a16_workspace_bytes(M, N, K, group_size))
-    if need == 0:
-        raise MxgError(MXG_ERR_UNSUPPORTED_SHAPE, "w8a16_gemm")
-    ws = workspace_buf if workspace_buf is not None else workspace(need, x.device, stream)
+    M, out, ws = _gemm_buffers(x, K, N, out, workspace_buf,
+                               lambda: _w8_ws_bytes(x.shape[0], N, K, group_size), stream)
+    _need_weights(packed, torch.uint8, int(_lib.w8a16_packed_bytes(K, N, group_size)), x.device,
+                  "packed")
     _check(_lib.w8a16_gemm(_ptr(x), _ptr(packed), M, N, K, group_size, _ptr(out), _ptr(ws),
                            ws.numel(), _stream(stream)), "w8a16_gemm")
     return out
@@ -440,37 +477,36 @@ def prepare_w8a16_gemm(x: torch.Tensor, packed: torch.Tensor, N: int, K: int,
                        group_size: int = 128, out: torch.Tensor | None = None,
                        workspace_buf: torch.Tensor | None = None, stream=None):
     """(call, out): ``call()`` runs w8a16_gemm(x, packed) into ``out``."""
-    _need(x, torch.bfloat16, "x")
-    M = x.shape[0]
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    _need(out, torch.bfloat16, "out")
-    need = int(_lib.w8a16_workspace_bytes(M, N, K, group_size))
-    if need == 0:
-        raise MxgError(MXG_ERR_UNSUPPORTED_SHAPE, "w8a16_gemm")
-    ws = workspace_buf if workspace_buf is not None else workspace(need, x.device, stream)
+    M, out, ws = _gemm_buffers(x, K, N, out, workspace_buf,
+                               lambda: _w8_ws_bytes(x.shape[0], N, K, group_size), stream)
+    _need_weights(packed, torch.uint8, int(_lib.w8a16_packed_bytes(K, N, group_size)), x.device,
+                  "packed")
     args = (_ptr(x), _ptr(packed), M, N, K, group_size, _ptr(out), _ptr(ws), ws.numel(),
             _stream(stream))
     return PreparedCall(_lib.w8a16_gemm, args, "w8a16_gemm", (x, packed, out, ws, stream)), out
+
+
+def _small_shapes(x: torch.Tensor, w: torch.Tensor):
+    """(M, K, N, workspace bytes) of x [M][K] against dense bf16 w [N][K]."""
+    _need(x, torch.bfloat16, "x")
+    _need(w, torch.bfloat16, "w")
+    if x.dim() != 2 or w.dim() != 2 or x.shape[1] != w.shape[1]:
+        raise ValueError("x must be [M][K] and w [N][K]")
+    _same_device(w, x.device, "w")
+    M, K = x.shape
+    N = w.shape[0]
+    need = int(_lib.bf16_gemm_small_workspace_bytes(M, N, K))
+    if need == 0:
+        raise MxgError(MXG_ERR_UNSUPPORTED_SHAPE, "bf16_gemm_small")
+    return M, K, N, need
 
 
 def bf16_gemm_small(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = None,
                     workspace_buf: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """Y = x * w^T with dense bf16 w [N][K] (few columns, e.g. the paired
     48 + 48 GDN A/B projection) and x bf16 [M][K], M <= 8."""
-    _need(x, torch.bfloat16, "x")
-    _need(w, torch.bfloat16, "w")
-    if x.dim() != 2 or w.dim() != 2 or x.shape[1] != w.shape[1]:
-        raise ValueError("x must be [M][K] and w [N][K]")
-    M, K = x.shape
-    N = w.shape[0]
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    _need(out, torch.bfloat16, "out")
-    need = int(_lib.bf16_gemm_small_workspace_bytes(M, N, K))
-    if need == 0:
-        raise MxgError(MXG_ERR_UNSUPPORTED_SHAPE, "bf16_gemm_small")
-    ws = workspace_buf if workspace_buf is not None else workspace(need, x.device, stream)
+    M, K, N, need = _small_shapes(x, w)
+    M, out, ws = _gemm_buffers(x, K, N, out, workspace_buf, lambda: need, stream)
     _check(_lib.bf16_gemm_small(_ptr(x), _ptr(w), M, N, K, _ptr(out), _ptr(ws), ws.numel(),
                                 _stream(stream)), "bf16_gemm_small")
     return out

@@ -136,3 +136,39 @@ def test_binding_refuses_to_load_without_the_library(tmp_path):
                        cwd=tmp_path, capture_output=True, text=True, timeout=300)
     assert r.returncode != 0
     assert "is missing" in r.stderr and "no fallback" in r.stderr
+
+
+def test_binding_checks_buffers_before_the_call(mxg):
+    """The C ABI cannot see buffer sizes, so the binding checks every buffer
+    against the call's shape before any launch: type, then size, then
+    layout and device (CPU tensors here: the size checks fire first)."""
+    import torch
+    cuda0 = torch.device("cuda", 0)
+    # output: dtype, then exact [M][N]
+    with pytest.raises(ValueError, match="bfloat16"):
+        mxg._need_out(torch.empty((5, 512), dtype=torch.float32), 5, 512, cuda0)
+    with pytest.raises(ValueError, match=r"\[5\]\[512\]"):
+        mxg._need_out(torch.empty((5, 256), dtype=torch.bfloat16), 5, 512, cuda0)
+    with pytest.raises(ValueError, match=r"\[5\]\[512\]"):
+        mxg._need_out(torch.empty((512, 5), dtype=torch.bfloat16), 5, 512, cuda0)
+    with pytest.raises(ValueError, match="CUDA"):
+        mxg._need_out(torch.empty((5, 512), dtype=torch.bfloat16), 5, 512, cuda0)
+    # packed weights: dtype, then at least the bytes the shape needs
+    need = mxg.w4a16_packed_bytes(512, 512, 128)
+    with pytest.raises(ValueError, match="uint8"):
+        mxg._need_weights(torch.empty(need, dtype=torch.int8), torch.uint8, need, cuda0, "packed")
+    with pytest.raises(ValueError, match="needs"):
+        mxg._need_weights(torch.empty(need - 16, dtype=torch.uint8), torch.uint8, need, cuda0,
+                          "packed")
+    with pytest.raises(ValueError, match="CUDA"):
+        mxg._need_weights(torch.empty(need, dtype=torch.uint8), torch.uint8, need, cuda0, "packed")
+    # a shape the library rejects itself (0 bytes) is left to its status
+    with pytest.raises(ValueError, match="CUDA"):
+        mxg._need_weights(torch.empty(16, dtype=torch.uint8), torch.uint8, 0, cuda0, "packed")
+    # caller workspaces are bytes
+    with pytest.raises(ValueError, match="uint8"):
+        mxg._need_ws(torch.empty(1024, dtype=torch.int32), cuda0)
+    # x must be [M][K] for the K of the call
+    with pytest.raises(ValueError, match="CUDA"):
+        mxg._gemm_buffers(torch.empty((5, 512), dtype=torch.bfloat16), 512, 512, None, None,
+                          lambda: 0, None)

@@ -1,0 +1,167 @@
+"""The Python binding's argument marshalling, on CPU: every GEMM entry is
+called with CPU tensors against a recording stand-in for libmxg.so (the
+device checks and the stream lookup are stubbed), and the test checks the
+pointers, sizes and shape arguments each C function receives, in the order
+include/mxg.h declares them.  No kernel runs."""
+import ctypes
+
+import pytest
+import torch
+
+
+class FakeLib:
+    """Records every C call and returns MXG_OK; the size queries and the
+    status strings go to the real library (they need no GPU)."""
+
+    def __init__(self, real):
+        self.calls = []
+        self._real = real
+
+    def __getattr__(self, name):
+        if name == "w8a16_workspace_bytes":
+            # the real query looks at the current device (none here): the
+            # streaming path's rule, M <= 32, with a stand-in size
+            return lambda M, N, K, G: 4096 if 1 <= M <= 32 else 0
+        if name.endswith("_bytes") or name == "mxg_status_string":
+            return getattr(self._real, name)
+
+        def fn(*args):
+            self.calls.append((name, args))
+            return 0
+        return fn
+
+
+def _val(a):
+    return a.value if isinstance(a, ctypes.c_void_p) else a
+
+
+@pytest.fixture()
+def fake(monkeypatch):
+    import __graft_entry__
+    __graft_entry__.build()
+    import mxfp8_gemm_speculative_b200 as m
+    lib = FakeLib(m._lib)
+    monkeypatch.setattr(m, "_lib", lib)
+
+    def need_cpu(t, dtype, name):
+        if t.dtype != dtype:
+            raise ValueError(f"{name} must be {dtype}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    monkeypatch.setattr(m, "_need", need_cpu)
+    monkeypatch.setattr(m, "_stream", lambda stream=None: None)
+    monkeypatch.setattr(m, "workspace",
+                        lambda nbytes, device=None, stream=None: torch.zeros(max(nbytes, 256),
+                                                                             dtype=torch.uint8))
+    monkeypatch.setattr(m, "_need_bytes", lambda *a: 4096)
+    return m, lib
+
+
+def bf16(*shape):
+    return torch.zeros(shape, dtype=torch.bfloat16)
+
+
+def test_w4a16_calls(fake):
+    m, lib = fake
+    M, K, N, G = 5, 512, 256, 128
+    x = bf16(M, K)
+    packed = torch.zeros(m.w4a16_packed_bytes(K, N, G), dtype=torch.uint8)
+    y = m.w4a16_gemm(x, packed, N, K, G)
+    name, a = lib.calls[-1]
+    assert name == "w4a16_gemm"
+    assert [_val(v) for v in a[:6]] == [x.data_ptr(), packed.data_ptr(), M, N, K, G]
+    assert _val(a[6]) == y.data_ptr() and tuple(y.shape) == (M, N)
+    assert a[8] == 4096          # the workspace's bytes
+    call, y2 = m.prepare_w4a16_gemm(x, packed, N, K, G)
+    call()
+    name, a = lib.calls[-1]
+    assert name == "w4a16_gemm" and _val(a[6]) == y2.data_ptr() and a[2:6] == (M, N, K, G)
+    m.w4a16_gemm_static_scratch(x, packed, N, K, G)
+    name, a = lib.calls[-1]
+    assert name == "w4a16_gemm_static_scratch" and a[2:6] == (M, N, K, G)
+    codes, w32, w16 = m.w4a16_unpack(packed, K, N, G)
+    name, a = lib.calls[-1]
+    assert name == "w4a16_unpack" and a[1:4] == (K, N, G)
+    assert [_val(v) for v in a[4:7]] == [codes.data_ptr(), w32.data_ptr(), w16.data_ptr()]
+    # a caller output and workspace are used as given
+    out = bf16(M, N)
+    ws = torch.zeros(8192, dtype=torch.uint8)
+    m.w4a16_gemm(x, packed, N, K, G, out=out, workspace_buf=ws)
+    name, a = lib.calls[-1]
+    assert _val(a[6]) == out.data_ptr() and _val(a[7]) == ws.data_ptr() and a[8] == 8192
+
+
+def test_w4a16_rejects_mismatched_buffers(fake):
+    m, lib = fake
+    M, K, N, G = 5, 512, 256, 128
+    x = bf16(M, K)
+    packed = torch.zeros(m.w4a16_packed_bytes(K, N, G), dtype=torch.uint8)
+    n0 = len(lib.calls)
+    with pytest.raises(ValueError):
+        m.w4a16_gemm(x, packed[:-16], N, K, G)            # too few weight bytes
+    with pytest.raises(ValueError):
+        m.w4a16_gemm(x, packed, N, K, G, out=bf16(M, N - 64))
+    with pytest.raises(ValueError):
+        m.w4a16_gemm(bf16(M, K - 64), packed, N, K, G)    # x of another K
+    with pytest.raises(ValueError):
+        m.w4a16_gemm(x, packed, N, K, G, workspace_buf=torch.zeros(64, dtype=torch.int32))
+    with pytest.raises(ValueError):
+        m.prepare_w4a16_gemm(x, packed[:100], N, K, G)
+    with pytest.raises(ValueError):
+        m.w4a16_gemm_static_scratch(x, packed[:100], N, K, G)
+    assert len(lib.calls) == n0                            # nothing reached the library
+
+
+def test_w8a16_calls(fake):
+    m, lib = fake
+    M, K, N, G = 4, 512, 256, 128
+    x = bf16(M, K)
+    packed = torch.zeros(int(m.raw_lib().w8a16_packed_bytes(K, N, G)), dtype=torch.uint8)
+    y = m.w8a16_gemm(x, packed, N, K, G)
+    name, a = lib.calls[-1]
+    assert name == "w8a16_gemm" and a[2:6] == (M, N, K, G) and _val(a[6]) == y.data_ptr()
+    call, _ = m.prepare_w8a16_gemm(x, packed, N, K, G)
+    call()
+    assert lib.calls[-1][0] == "w8a16_gemm"
+    with pytest.raises(ValueError):
+        m.w8a16_gemm(x, packed[: packed.numel() // 2], N, K, G)
+    with pytest.raises(ValueError):
+        m.prepare_w8a16_gemm(bf16(M, K + 64), packed, N, K, G)
+    with pytest.raises(m.MxgError):
+        m.w8a16_gemm(bf16(33, K), packed, N, K, G)        # streaming path only
+
+
+def test_mxfp8_calls(fake):
+    m, lib = fake
+    M, K, N = 4, 512, 256
+    x = bf16(M, K)
+    wq = torch.zeros((N, K), dtype=torch.uint8)
+    ws = torch.zeros((N, K // 32), dtype=torch.uint8)
+    y = m.mxfp8_gemm(x, wq, ws)
+    name, a = lib.calls[-1]
+    assert name == "mxfp8_gemm"
+    assert [_val(v) for v in a[:3]] == [x.data_ptr(), wq.data_ptr(), ws.data_ptr()]
+    assert a[3:6] == (M, N, K) and _val(a[6]) == y.data_ptr()
+    call, _ = m.prepare_mxfp8_gemm(x, wq, ws)
+    call()
+    assert lib.calls[-1][0] == "mxfp8_gemm"
+    with pytest.raises(ValueError):
+        m.mxfp8_gemm(x, wq, ws[:, :-1])
+    with pytest.raises(ValueError):
+        m.mxfp8_gemm(x, wq, ws, out=bf16(M + 1, N))
+
+
+def test_bf16_small_calls(fake):
+    m, lib = fake
+    M, K, N = 4, 5120, 96
+    x, w = bf16(M, K), bf16(N, K)
+    y = m.bf16_gemm_small(x, w)
+    name, a = lib.calls[-1]
+    assert name == "bf16_gemm_small" and a[2:5] == (M, N, K) and _val(a[5]) == y.data_ptr()
+    call, _ = m.prepare_bf16_gemm_small(x, w)
+    call()
+    assert lib.calls[-1][0] == "bf16_gemm_small"
+    with pytest.raises(ValueError):
+        m.bf16_gemm_small(x, w, out=bf16(M, N + 16))
+    with pytest.raises(m.MxgError):
+        m.bf16_gemm_small(bf16(9, K), w)                  # M <= 8
