@@ -139,6 +139,11 @@ def _need_weights(t: torch.Tensor, dtype, nbytes: int, device, name: str) -> Non
     _same_device(t, device, name)
 
 
+def _need_shape(t: torch.Tensor, shape, name: str) -> None:
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must be {list(shape)}, got {list(t.shape)}")
+
+
 def _need_ws(ws: torch.Tensor, device) -> None:
     if ws.dtype != torch.uint8:
         raise ValueError(f"workspace_buf must be torch.uint8, got {ws.dtype}")
@@ -226,6 +231,8 @@ def w4a16_repack(qweight: torch.Tensor, scales: torch.Tensor, group_size: int = 
     K = qweight.shape[0] * 8
     N = qweight.shape[1]
     packed = _repack_out(qweight, K, N, group_size, out, "w4a16_repack")
+    _need_shape(scales, (K // group_size, N), "scales")
+    _same_device(scales, qweight.device, "scales")
     _check(_lib.w4a16_repack(_ptr(qweight), _ptr(scales), K, N, group_size, _ptr(packed),
                              _stream(stream)), "w4a16_repack")
     return packed
@@ -241,6 +248,8 @@ def w4a16_repack_ct(weight_packed: torch.Tensor, weight_scale: torch.Tensor,
     N = weight_packed.shape[0]
     K = weight_packed.shape[1] * 8
     packed = _repack_out(weight_packed, K, N, group_size, out, "w4a16_repack_ct")
+    _need_shape(weight_scale, (N, K // group_size), "weight_scale")
+    _same_device(weight_scale, weight_packed.device, "weight_scale")
     _check(_lib.w4a16_repack_ct(_ptr(weight_packed), _ptr(weight_scale), K, N, group_size,
                                 _ptr(packed), _stream(stream)), "w4a16_repack_ct")
     return packed
@@ -262,6 +271,10 @@ def w4a16_repack_fused(parts, group_size: int = 128, stream=None,
         raise ValueError("every part must have the same K")
     Ns = [int(qw.shape[1]) for qw, _ in parts]
     packed = _repack_out(parts[0][0], K, sum(Ns), group_size, out, "w4a16_repack_fused")
+    for i, (qw, sc) in enumerate(parts):
+        _need_shape(sc, (K // group_size, Ns[i]), f"scales of part {i}")
+        _same_device(qw, packed.device, f"qweight of part {i}")
+        _same_device(sc, packed.device, f"scales of part {i}")
     n = len(parts)
     qptrs = (ctypes.c_void_p * n)(*[qw.data_ptr() for qw, _ in parts])
     sptrs = (ctypes.c_void_p * n)(*[sc.data_ptr() for _, sc in parts])
@@ -404,7 +417,18 @@ def mxfp8_gemm(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor,
 
 
 def mxfp8_dequant(wq: torch.Tensor, ws: torch.Tensor, stream=None) -> torch.Tensor:
+    """bf16 [N][K] weights of E4M3 wq[N][K] and E8M0 ws[N][K/32]."""
+    if wq.dtype not in (torch.uint8, torch.float8_e4m3fn):
+        raise ValueError("wq must be uint8 or float8_e4m3fn")
+    if ws.dtype not in (torch.uint8, torch.float8_e8m0fnu):
+        raise ValueError("ws must be uint8 or float8_e8m0fnu")
+    if wq.dim() != 2:
+        raise ValueError("wq must be [N][K]")
     N, K = wq.shape
+    _need_shape(ws, (N, K // 32), "ws")
+    _need(wq, wq.dtype, "wq")
+    _need(ws, ws.dtype, "ws")
+    _same_device(ws, wq.device, "ws")
     out = torch.empty((N, K), dtype=torch.bfloat16, device=wq.device)
     _check(_lib.mxfp8_dequant(_ptr(wq), _ptr(ws), N, K, _ptr(out), _stream(stream)),
            "mxfp8_dequant")
@@ -412,7 +436,17 @@ def mxfp8_dequant(wq: torch.Tensor, ws: torch.Tensor, stream=None) -> torch.Tens
 
 
 # ------------------------------------------------------------- diagnostics
+def _need_header(workspace_buf: torch.Tensor) -> None:
+    """A workspace holding at least its 256-byte status header."""
+    if workspace_buf.dtype != torch.uint8:
+        raise ValueError(f"workspace_buf must be torch.uint8, got {workspace_buf.dtype}")
+    if workspace_buf.numel() < 256:
+        raise ValueError("workspace_buf must hold at least its 256-byte header")
+    _need(workspace_buf, torch.uint8, "workspace_buf")
+
+
 def mxg_workspace_status(workspace_buf: torch.Tensor, stream=None) -> int:
+    _need_header(workspace_buf)
     v = ctypes.c_int(0)
     _check(_lib.mxg_workspace_status(_ptr(workspace_buf), ctypes.byref(v), _stream(stream)),
            "mxg_workspace_status")
@@ -430,6 +464,8 @@ def w8a16_repack(qweight: torch.Tensor, scales: torch.Tensor, group_size: int = 
     nbytes = int(_lib.w8a16_packed_bytes(K, N, group_size))
     if nbytes == 0:
         raise MxgError(MXG_ERR_UNSUPPORTED_SHAPE, "w8a16_repack")
+    _need_shape(scales, (K // group_size, N), "scales")
+    _same_device(scales, qweight.device, "scales")
     packed = torch.empty(nbytes, dtype=torch.uint8, device=qweight.device)
     _check(_lib.w8a16_repack(_ptr(qweight), _ptr(scales), K, N, group_size, _ptr(packed),
                              _stream(stream)), "w8a16_repack")
@@ -447,6 +483,8 @@ def w8a16_repack_ct(weight_packed: torch.Tensor, weight_scale: torch.Tensor,
     nbytes = int(_lib.w8a16_packed_bytes(K, N, group_size))
     if nbytes == 0:
         raise MxgError(MXG_ERR_UNSUPPORTED_SHAPE, "w8a16_repack_ct")
+    _need_shape(weight_scale, (N, K // group_size), "weight_scale")
+    _same_device(weight_scale, weight_packed.device, "weight_scale")
     packed = torch.empty(nbytes, dtype=torch.uint8, device=weight_packed.device)
     _check(_lib.w8a16_repack_ct(_ptr(weight_packed), _ptr(weight_scale), K, N, group_size,
                                 _ptr(packed), _stream(stream)), "w8a16_repack_ct")
@@ -513,6 +551,7 @@ def bf16_gemm_small(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None =
 
 
 def mxg_selftest_wait_timeout(workspace_buf: torch.Tensor, limit_us: int, stream=None) -> None:
+    _need_header(workspace_buf)
     _check(_lib.mxg_selftest_wait_timeout(_ptr(workspace_buf), int(limit_us), _stream(stream)),
            "mxg_selftest_wait_timeout")
 

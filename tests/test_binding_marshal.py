@@ -165,3 +165,47 @@ def test_bf16_small_calls(fake):
         m.bf16_gemm_small(x, w, out=bf16(M, N + 16))
     with pytest.raises(m.MxgError):
         m.bf16_gemm_small(bf16(9, K), w)                  # M <= 8
+
+
+def test_repack_and_decoder_shapes(fake):
+    m, lib = fake
+    K, N, G = 512, 256, 128
+    qw = torch.zeros((K // 8, N), dtype=torch.int32)
+    sc = torch.zeros((K // G, N), dtype=torch.float16)
+    packed = m.w4a16_repack(qw, sc, G)
+    name, a = lib.calls[-1]
+    assert name == "w4a16_repack" and a[2:5] == (K, N, G) and _val(a[5]) == packed.data_ptr()
+    assert packed.numel() == m.w4a16_packed_bytes(K, N, G)
+    m.w4a16_repack_ct(qw.T.contiguous(), sc.T.contiguous(), G)
+    assert lib.calls[-1][0] == "w4a16_repack_ct" and lib.calls[-1][1][2:5] == (K, N, G)
+    m.w4a16_repack_fused([(qw, sc), (qw, sc)], G)
+    name, a = lib.calls[-1]
+    assert name == "w4a16_repack_fused" and a[0] == 2 and a[4:6] == (K, G)
+    q8 = torch.zeros((K // 4, N), dtype=torch.int32)
+    m.w8a16_repack(q8, sc, G)
+    assert lib.calls[-1][0] == "w8a16_repack" and lib.calls[-1][1][2:5] == (K, N, G)
+    n0 = len(lib.calls)
+    with pytest.raises(ValueError):
+        m.w4a16_repack(qw, sc[:, :-64], G)                 # scales of another N
+    with pytest.raises(ValueError):
+        m.w4a16_repack(qw, torch.zeros((K // 64, N), dtype=torch.float16), G)
+    with pytest.raises(ValueError):
+        m.w4a16_repack_ct(qw.T.contiguous(), sc, G)        # GPTQ-oriented scales
+    with pytest.raises(ValueError):
+        m.w4a16_repack_fused([(qw, sc), (qw, sc[:, :64])], G)
+    with pytest.raises(ValueError):
+        m.w8a16_repack(q8, sc[:1], G)
+    with pytest.raises(ValueError):
+        m.w8a16_repack_ct(q8.T.contiguous(), sc, G)
+    with pytest.raises(ValueError):
+        m.mxfp8_dequant(torch.zeros((N, K), dtype=torch.uint8),
+                        torch.zeros((N, K // 64), dtype=torch.uint8))
+    with pytest.raises(ValueError):
+        m.mxg_workspace_status(torch.zeros(128, dtype=torch.uint8))
+    with pytest.raises(ValueError):
+        m.mxg_selftest_wait_timeout(torch.zeros(64, dtype=torch.int32), 1000)
+    assert len(lib.calls) == n0
+    w16 = m.mxfp8_dequant(torch.zeros((N, K), dtype=torch.uint8),
+                          torch.zeros((N, K // 32), dtype=torch.uint8))
+    name, a = lib.calls[-1]
+    assert name == "mxfp8_dequant" and a[2:4] == (N, K) and _val(a[4]) == w16.data_ptr()
