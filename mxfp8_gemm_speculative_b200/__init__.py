@@ -176,7 +176,11 @@ _ws_cache: dict[tuple[int, int], torch.Tensor] = {}
 
 
 def workspace(nbytes: int, device=None, stream=None) -> torch.Tensor:
-    """A zero-filled uint8 workspace of at least ``nbytes`` for (device, stream)."""
+    """A zero-filled uint8 workspace of at least ``nbytes`` for (device, stream).
+    It is allocated and zeroed on that stream, so the zero fill is ordered
+    before the stream's next kernel, and the memory of a workspace it
+    replaces goes back to that stream's pool (reused only behind the calls
+    already queued there)."""
     dev = torch.device("cuda", torch.cuda.current_device() if device is None else
                        torch.device(device).index)
     s = stream if stream is not None else torch.cuda.current_stream(dev)
@@ -184,7 +188,8 @@ def workspace(nbytes: int, device=None, stream=None) -> torch.Tensor:
     with _ws_lock:
         ws = _ws_cache.get(key)
         if ws is None or ws.numel() < nbytes:
-            ws = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=dev)
+            with torch.cuda.stream(s):
+                ws = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=dev)
             _ws_cache[key] = ws
         return ws
 
