@@ -139,6 +139,16 @@ def _need_weights(t: torch.Tensor, dtype, nbytes: int, device, name: str) -> Non
     _same_device(t, device, name)
 
 
+def _empty(shape, dtype, device, stream) -> torch.Tensor:
+    """An uninitialised tensor for a result the library writes on `stream`:
+    allocated on that stream, so its memory, once freed, is reused only
+    behind the work already queued there."""
+    if stream is None:
+        return torch.empty(shape, dtype=dtype, device=device)
+    with torch.cuda.stream(stream):
+        return torch.empty(shape, dtype=dtype, device=device)
+
+
 def _need_shape(t: torch.Tensor, shape, name: str) -> None:
     if tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} must be {list(shape)}, got {list(t.shape)}")
@@ -160,7 +170,7 @@ def _gemm_buffers(x: torch.Tensor, K: int, N: int, out, workspace_buf, need_ws, 
         raise ValueError(f"x must be [M][{K}], got {list(x.shape)}")
     M = x.shape[0]
     if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+        out = _empty((M, N), torch.bfloat16, x.device, stream)
     _need_out(out, M, N, x.device)
     if workspace_buf is None:
         ws = workspace(need_ws(), x.device, stream)
@@ -209,12 +219,13 @@ def w4a16_packed_bytes(K: int, N: int, group_size: int = 128) -> int:
     return int(_lib.w4a16_packed_bytes(K, N, group_size))
 
 
-def _repack_out(words: torch.Tensor, K: int, N: int, group_size: int, out, what: str):
+def _repack_out(words: torch.Tensor, K: int, N: int, group_size: int, out, what: str,
+                stream=None):
     nbytes = w4a16_packed_bytes(K, N, group_size)
     if nbytes == 0:
         raise MxgError(MXG_ERR_UNSUPPORTED_SHAPE, what)
     if out is None:
-        return torch.empty(nbytes, dtype=torch.uint8, device=words.device)
+        return _empty(nbytes, torch.uint8, words.device, stream)
     _need(out, torch.uint8, "out")
     if out.numel() != nbytes or out.device != words.device:
         raise ValueError(f"out must hold {nbytes} bytes on {words.device}")
@@ -235,7 +246,7 @@ def w4a16_repack(qweight: torch.Tensor, scales: torch.Tensor, group_size: int = 
     _need_scales(scales, "scales")
     K = qweight.shape[0] * 8
     N = qweight.shape[1]
-    packed = _repack_out(qweight, K, N, group_size, out, "w4a16_repack")
+    packed = _repack_out(qweight, K, N, group_size, out, "w4a16_repack", stream)
     _need_shape(scales, (K // group_size, N), "scales")
     _same_device(scales, qweight.device, "scales")
     _check(_lib.w4a16_repack(_ptr(qweight), _ptr(scales), K, N, group_size, _ptr(packed),
@@ -252,7 +263,7 @@ def w4a16_repack_ct(weight_packed: torch.Tensor, weight_scale: torch.Tensor,
     _need_scales(weight_scale, "weight_scale")
     N = weight_packed.shape[0]
     K = weight_packed.shape[1] * 8
-    packed = _repack_out(weight_packed, K, N, group_size, out, "w4a16_repack_ct")
+    packed = _repack_out(weight_packed, K, N, group_size, out, "w4a16_repack_ct", stream)
     _need_shape(weight_scale, (N, K // group_size), "weight_scale")
     _same_device(weight_scale, weight_packed.device, "weight_scale")
     _check(_lib.w4a16_repack_ct(_ptr(weight_packed), _ptr(weight_scale), K, N, group_size,
@@ -275,7 +286,7 @@ def w4a16_repack_fused(parts, group_size: int = 128, stream=None,
     if any(qw.shape[0] * 8 != K for qw, _ in parts):
         raise ValueError("every part must have the same K")
     Ns = [int(qw.shape[1]) for qw, _ in parts]
-    packed = _repack_out(parts[0][0], K, sum(Ns), group_size, out, "w4a16_repack_fused")
+    packed = _repack_out(parts[0][0], K, sum(Ns), group_size, out, "w4a16_repack_fused", stream)
     for i, (qw, sc) in enumerate(parts):
         _need_shape(sc, (K // group_size, Ns[i]), f"scales of part {i}")
         _same_device(qw, packed.device, f"qweight of part {i}")
@@ -364,7 +375,7 @@ def w4a16_gemm_static_scratch(x: torch.Tensor, packed: torch.Tensor, N: int, K: 
         raise ValueError(f"x must be [M][{K}], got {list(x.shape)}")
     M = x.shape[0]
     if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+        out = _empty((M, N), torch.bfloat16, x.device, stream)
     _need_out(out, M, N, x.device)
     _need_weights(packed, torch.uint8, w4a16_packed_bytes(K, N, group_size), x.device, "packed")
     _check(_lib.w4a16_gemm_static_scratch(_ptr(x), _ptr(packed), M, N, K, group_size, _ptr(out),
@@ -376,9 +387,9 @@ def w4a16_unpack(packed: torch.Tensor, K: int, N: int, group_size: int = 128, st
     """(codes uint8 [N][K], w_fp32 float32 [N][K], w_bf16 bfloat16 [N][K])."""
     dev = packed.device
     _need_weights(packed, torch.uint8, w4a16_packed_bytes(K, N, group_size), dev, "packed")
-    codes = torch.empty((N, K), dtype=torch.uint8, device=dev)
-    w32 = torch.empty((N, K), dtype=torch.float32, device=dev)
-    w16 = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    codes = _empty((N, K), torch.uint8, dev, stream)
+    w32 = _empty((N, K), torch.float32, dev, stream)
+    w16 = _empty((N, K), torch.bfloat16, dev, stream)
     _check(_lib.w4a16_unpack(_ptr(packed), K, N, group_size, _ptr(codes), _ptr(w32), _ptr(w16),
                              _stream(stream)), "w4a16_unpack")
     return codes, w32, w16
@@ -434,7 +445,7 @@ def mxfp8_dequant(wq: torch.Tensor, ws: torch.Tensor, stream=None) -> torch.Tens
     _need(wq, wq.dtype, "wq")
     _need(ws, ws.dtype, "ws")
     _same_device(ws, wq.device, "ws")
-    out = torch.empty((N, K), dtype=torch.bfloat16, device=wq.device)
+    out = _empty((N, K), torch.bfloat16, wq.device, stream)
     _check(_lib.mxfp8_dequant(_ptr(wq), _ptr(ws), N, K, _ptr(out), _stream(stream)),
            "mxfp8_dequant")
     return out
@@ -471,7 +482,7 @@ def w8a16_repack(qweight: torch.Tensor, scales: torch.Tensor, group_size: int = 
         raise MxgError(MXG_ERR_UNSUPPORTED_SHAPE, "w8a16_repack")
     _need_shape(scales, (K // group_size, N), "scales")
     _same_device(scales, qweight.device, "scales")
-    packed = torch.empty(nbytes, dtype=torch.uint8, device=qweight.device)
+    packed = _empty(nbytes, torch.uint8, qweight.device, stream)
     _check(_lib.w8a16_repack(_ptr(qweight), _ptr(scales), K, N, group_size, _ptr(packed),
                              _stream(stream)), "w8a16_repack")
     return packed
@@ -490,7 +501,7 @@ def w8a16_repack_ct(weight_packed: torch.Tensor, weight_scale: torch.Tensor,
         raise MxgError(MXG_ERR_UNSUPPORTED_SHAPE, "w8a16_repack_ct")
     _need_shape(weight_scale, (N, K // group_size), "weight_scale")
     _same_device(weight_scale, weight_packed.device, "weight_scale")
-    packed = torch.empty(nbytes, dtype=torch.uint8, device=weight_packed.device)
+    packed = _empty(nbytes, torch.uint8, weight_packed.device, stream)
     _check(_lib.w8a16_repack_ct(_ptr(weight_packed), _ptr(weight_scale), K, N, group_size,
                                 _ptr(packed), _stream(stream)), "w8a16_repack_ct")
     return packed
