@@ -39,14 +39,18 @@
  *    0xFF and non-finite scales give unspecified output.
  *  - GEMM kernels are launched with programmatic dependent launch: they may
  *    start while the previous kernel on `stream` drains, and wait for it
- *    before they read X or touch Y and the workspace.  The weight-streaming
- *    kernels (M <= 32) also start loading WEIGHTS (packed, Wq, Ws) before
- *    that wait, unless mxg_set_early_weight_loads(0) was called: the weight
+ *    before they read X or touch Y and the workspace.  By default they also
+ *    start loading WEIGHTS (packed, Wq, Ws, W) before that wait: the weight
  *    buffers must then not be written by the kernel immediately before the
  *    GEMM on `stream`.  w4a16_repack ends with a kernel that writes nothing,
  *    so a GEMM may follow it directly; any other writer of weights needs
  *    another launch, or a synchronization, between it and the GEMM (in
- *    serving, weights are written once at load time).
+ *    serving, weights are written once at load time), or the call's
+ *    late_weights option (the *_ex entry points).
+ *  - No entry point keeps settings between calls: every choice a caller can
+ *    make is an argument of the call (mxg_gemm_options).  The only global
+ *    state is a per-device cache of device attributes and kernel launch
+ *    attributes, and the scratch array of w4a16_gemm_static_scratch.
  */
 #ifndef MXG_H
 #define MXG_H
@@ -71,8 +75,28 @@ typedef enum {
     MXG_ERR_UNSUPPORTED_SHAPE = -2,  /* a size the format or the kernels reject */
     MXG_ERR_WORKSPACE = -3,          /* workspace smaller than the size query */
     MXG_ERR_CUDA = -4,               /* a CUDA runtime or launch error */
-    MXG_ERR_TIMEOUT = -5             /* a bounded in-kernel wait ran out */
+    MXG_ERR_TIMEOUT = -5,            /* a bounded in-kernel wait ran out */
+    MXG_ERR_CAPTURE = -6             /* a one-time device set-up was asked for inside a
+                                        stream capture (make that first call outside it) */
 } mxg_status;
+
+/* Per-call options of the *_ex GEMM entry points.  NULL, or a struct whose
+ * fields are all zero, gives the behaviour of the plain entry points.
+ *   path          MXG_PATH_AUTO: M <= 32 streams the weights, larger M runs on
+ *                 the tensor cores; MXG_PATH_STREAM / MXG_PATH_TENSOR force
+ *                 one path (the streaming path takes M <= 32 only; a shape
+ *                 the forced path cannot run returns
+ *                 MXG_ERR_UNSUPPORTED_SHAPE).
+ *   late_weights  0: the kernels may load weights before waiting for the
+ *                 previous kernel on the stream (see the conventions above);
+ *                 1: only after that wait, for a caller whose previous kernel
+ *                 on the stream writes these weights.
+ * A value outside these returns MXG_ERR_INVALID_ARG before any launch. */
+enum { MXG_PATH_AUTO = 0, MXG_PATH_STREAM = 1, MXG_PATH_TENSOR = 2 };
+typedef struct mxg_gemm_options {
+    int path;
+    int late_weights;
+} mxg_gemm_options;
 
 /* Short English text for a status code (static storage, never NULL). */
 MXG_API const char *mxg_status_string(int status);
@@ -153,6 +177,11 @@ MXG_API size_t w4a16_workspace_bytes(int M, int N, int K, int group_size);
 MXG_API int w4a16_gemm(const void *X, const void *packed, int M, int N, int K, int group_size,
                void *Y, void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* w4a16_gemm with per-call options (NULL = the defaults of w4a16_gemm). */
+MXG_API int w4a16_gemm_ex(const void *X, const void *packed, int M, int N, int K,
+               int group_size, void *Y, void *workspace, size_t workspace_bytes,
+               const mxg_gemm_options *opts, cudaStream_t stream);
+
 /* w4a16_gemm on the weight-streaming path without a caller workspace.  The
  * source pages have no counterpart to this call: it exists for callers that
  * cannot allocate a workspace (a plain C host with no device allocator of its
@@ -166,13 +195,28 @@ MXG_API int w4a16_gemm(const void *X, const void *packed, int M, int N, int K, i
  *   148-SM B200 every M <= 32 shape fits).
  * The first call on a device does a one-time set-up with that device
  * current: it looks the array up and zeroes its status word and counters on
- * `stream`; make that first call before any stream capture.  Every completed
- * call leaves the counters zero; the partial-sum scratch keeps the last
- * call's contents.  Calls that are not ordered with respect to each other
- * race on the array.  The status word of a timed-out wait stays inside the
- * array (use w4a16_gemm with a workspace to read diagnostics). */
+ * `stream`; make that first call before any stream capture (inside one it
+ * returns MXG_ERR_CAPTURE, and a later call outside a capture sets up).
+ * Every call that completes without an error leaves the counters zero; the
+ * partial-sum scratch keeps the last call's contents.  Calls that are not
+ * ordered with respect to each other race on the array.  The array is 8 MiB
+ * per device (every M <= 32 shape fits on a 148-SM B200).
+ * A kernel that gives up a bounded wait records MXG_ERR_TIMEOUT in the
+ * array's status word and returns MXG_OK to nobody: callers check the status
+ * word with w4a16_static_scratch_status (for instance after each step of a
+ * serving loop, outside any capture) and clear it before further calls. */
 MXG_API int w4a16_gemm_static_scratch(const void *X, const void *packed, int M, int N, int K,
                int group_size, void *Y, cudaStream_t stream);
+
+/* Status word of this device's w4a16_gemm_static_scratch array (no
+ * counterpart on the source pages).  Copies it to *status (MXG_OK or the
+ * first error a kernel recorded, e.g. MXG_ERR_TIMEOUT); with reset = 1 also
+ * zeroes the status word and the arrival counters, which a timed-out call
+ * may have left non-zero, so later calls start clean.  Stream-ordered on
+ * `stream` (behind the calls queued there) and synchronizes it.  Does the
+ * array's one-time set-up if no call did yet (so not inside a capture).
+ * reset other than 0 or 1, or a NULL status: MXG_ERR_INVALID_ARG. */
+MXG_API int w4a16_static_scratch_status(int *status, int reset, cudaStream_t stream);
 
 /* ------------------------------------------------------------------ INT8 */
 
@@ -215,6 +259,12 @@ MXG_API size_t w8a16_workspace_bytes(int M, int N, int K, int group_size);
 MXG_API int w8a16_gemm(const void *X, const void *packed, int M, int N, int K, int group_size,
                void *Y, void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* w8a16_gemm with per-call options (NULL = defaults; path MXG_PATH_TENSOR is
+ * MXG_ERR_INVALID_ARG: INT8 has the weight-streaming path only). */
+MXG_API int w8a16_gemm_ex(const void *X, const void *packed, int M, int N, int K,
+               int group_size, void *Y, void *workspace, size_t workspace_bytes,
+               const mxg_gemm_options *opts, cudaStream_t stream);
+
 /* ----------------------------------------------------------------- MXFP8 */
 
 /* Workspace bytes mxfp8_gemm needs for this shape on the current device. */
@@ -229,6 +279,11 @@ MXG_API size_t mxfp8_workspace_bytes(int M, int N, int K);
  * bf16 (weight-only quantization). */
 MXG_API int mxfp8_gemm(const void *X, const uint8_t *Wq, const uint8_t *Ws, int M, int N, int K,
                void *Y, void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* mxfp8_gemm with per-call options (NULL = the defaults of mxfp8_gemm). */
+MXG_API int mxfp8_gemm_ex(const void *X, const uint8_t *Wq, const uint8_t *Ws, int M, int N,
+               int K, void *Y, void *workspace, size_t workspace_bytes,
+               const mxg_gemm_options *opts, cudaStream_t stream);
 
 /* ------------------------------------- dense bf16, few output columns */
 
@@ -247,6 +302,13 @@ MXG_API int mxfp8_gemm(const void *X, const uint8_t *Wq, const uint8_t *Ws, int 
 MXG_API size_t bf16_gemm_small_workspace_bytes(int M, int N, int K);
 MXG_API int bf16_gemm_small(const void *X, const void *W, int M, int N, int K, void *Y,
                void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* bf16_gemm_small with per-call options (NULL = defaults; only
+ * late_weights applies, a path other than MXG_PATH_AUTO is
+ * MXG_ERR_INVALID_ARG). */
+MXG_API int bf16_gemm_small_ex(const void *X, const void *W, int M, int N, int K, void *Y,
+               void *workspace, size_t workspace_bytes, const mxg_gemm_options *opts,
+               cudaStream_t stream);
 
 /* --------------------------------------------------- test and diagnostics */
 
@@ -271,20 +333,10 @@ MXG_API int mxg_workspace_status(const void *workspace, int *status, cudaStream_
 /* Runs one CTA whose pipeline wait can never complete (nothing arrives on
  * its barrier) with a time limit of `limit_us` microseconds, to exercise the
  * timeout path.  The kernel records MXG_ERR_TIMEOUT in the workspace status
- * word and returns; the context stays usable.  workspace: >= 256 bytes. */
+ * word and returns; the context stays usable.  workspace: >= 256 bytes, or
+ * NULL for the static scratch array of w4a16_gemm_static_scratch on the
+ * current device (read and clear it with w4a16_static_scratch_status). */
 MXG_API int mxg_selftest_wait_timeout(void *workspace, int limit_us, cudaStream_t stream);
-
-/* Path override for tests and benchmarks (process-wide):
- * 0 = automatic (default), 1 = weight-streaming path, 2 = tensor-core path.
- * The streaming path accepts M <= 32 only.  Returns the previous setting. */
-MXG_API int mxg_set_path(int path);
-
-/* Early weight loads of the weight-streaming kernels (process-wide):
- * 1 = load the first weight tiles before waiting for the previous kernel on
- * the stream (default), 0 = load everything after that wait, for callers
- * that write weights in the kernel right before a GEMM.  Returns the
- * previous setting, or -1 for a value other than 0 and 1. */
-MXG_API int mxg_set_early_weight_loads(int on);
 
 #ifdef __cplusplus
 }

@@ -44,9 +44,12 @@ _SIGS = {
     "w4a16_repack_fused": (_i, [_i, _p, _p, _p, _i, _i, _p, _p]),
     "w4a16_workspace_bytes": (_sz, [_i, _i, _i, _i]),
     "w4a16_gemm": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _sz, _p]),
+    "w4a16_gemm_ex": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _sz, _p, _p]),
+    "w4a16_static_scratch_status": (_i, [ctypes.POINTER(_i), _i, _p]),
     "w4a16_gemm_static_scratch": (_i, [_p, _p, _i, _i, _i, _i, _p, _p]),
     "mxfp8_workspace_bytes": (_sz, [_i, _i, _i]),
     "mxfp8_gemm": (_i, [_p, _p, _p, _i, _i, _i, _p, _p, _sz, _p]),
+    "mxfp8_gemm_ex": (_i, [_p, _p, _p, _i, _i, _i, _p, _p, _sz, _p, _p]),
     "w4a16_unpack": (_i, [_p, _i, _i, _i, _p, _p, _p, _p]),
     "mxfp8_dequant": (_i, [_p, _p, _i, _i, _p, _p]),
     "mxg_workspace_status": (_i, [_p, ctypes.POINTER(_i), _p]),
@@ -56,10 +59,10 @@ _SIGS = {
     "w8a16_repack_ct": (_i, [_p, _p, _i, _i, _i, _p, _p]),
     "w8a16_workspace_bytes": (_sz, [_i, _i, _i, _i]),
     "w8a16_gemm": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _sz, _p]),
+    "w8a16_gemm_ex": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _sz, _p, _p]),
     "bf16_gemm_small_workspace_bytes": (_sz, [_i, _i, _i]),
     "bf16_gemm_small": (_i, [_p, _p, _i, _i, _i, _p, _p, _sz, _p]),
-    "mxg_set_path": (_i, [_i]),
-    "mxg_set_early_weight_loads": (_i, [_i]),
+    "bf16_gemm_small_ex": (_i, [_p, _p, _i, _i, _i, _p, _p, _sz, _p, _p]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -74,6 +77,23 @@ MXG_ERR_UNSUPPORTED_SHAPE = -2
 MXG_ERR_WORKSPACE = -3
 MXG_ERR_CUDA = -4
 MXG_ERR_TIMEOUT = -5
+MXG_ERR_CAPTURE = -6
+
+PATH_AUTO, PATH_STREAM, PATH_TENSOR = 0, 1, 2
+
+
+class GemmOptions(ctypes.Structure):
+    """mxg_gemm_options of include/mxg.h: per-call path and weight-load
+    timing."""
+    _fields_ = [("path", ctypes.c_int), ("late_weights", ctypes.c_int)]
+
+
+def _options(path: int = PATH_AUTO, late_weights: bool = False):
+    """A pointer to the call's options, or None for the defaults.  The
+    structure is kept alive by the returned pointer object."""
+    if path == PATH_AUTO and not late_weights:
+        return None
+    return ctypes.pointer(GemmOptions(int(path), 1 if late_weights else 0))
 
 
 class MxgError(RuntimeError):
@@ -95,9 +115,30 @@ def _ptr(t: torch.Tensor | None):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream=None):
-    s = stream if stream is not None else torch.cuda.current_stream()
+def _stream(stream=None, device=None):
+    """The CUDA stream handle a call runs on: ``stream``, which must live on
+    ``device``, or that device's current stream."""
+    if stream is None:
+        s = torch.cuda.current_stream(device)
+    else:
+        s = stream
+        sdev = getattr(s, "device", None)
+        if device is not None and sdev is not None and torch.device(sdev) != torch.device(device):
+            raise ValueError(f"stream is on {sdev}, the call's tensors on {device}")
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def _on_device(device):
+    """Makes ``device`` current for a C call: the library plans and launches
+    on the current device (its SM count, its kernels, its static scratch)."""
+    return torch.cuda.device(device)
+
+
+def _dev_call(device, what: str, fn, *args, stream=None) -> None:
+    """fn(*args, stream handle) with ``device`` current; raises on a nonzero
+    status."""
+    with _on_device(device):
+        _check(fn(*args, _stream(stream, device)), what)
 
 
 def _need(t: torch.Tensor, dtype, name: str) -> None:
@@ -249,8 +290,8 @@ def w4a16_repack(qweight: torch.Tensor, scales: torch.Tensor, group_size: int = 
     packed = _repack_out(qweight, K, N, group_size, out, "w4a16_repack", stream)
     _need_shape(scales, (K // group_size, N), "scales")
     _same_device(scales, qweight.device, "scales")
-    _check(_lib.w4a16_repack(_ptr(qweight), _ptr(scales), K, N, group_size, _ptr(packed),
-                             _stream(stream)), "w4a16_repack")
+    _dev_call(qweight.device, "w4a16_repack", _lib.w4a16_repack, _ptr(qweight), _ptr(scales), K, N,
+              group_size, _ptr(packed), stream=stream)
     return packed
 
 
@@ -266,8 +307,8 @@ def w4a16_repack_ct(weight_packed: torch.Tensor, weight_scale: torch.Tensor,
     packed = _repack_out(weight_packed, K, N, group_size, out, "w4a16_repack_ct", stream)
     _need_shape(weight_scale, (N, K // group_size), "weight_scale")
     _same_device(weight_scale, weight_packed.device, "weight_scale")
-    _check(_lib.w4a16_repack_ct(_ptr(weight_packed), _ptr(weight_scale), K, N, group_size,
-                                _ptr(packed), _stream(stream)), "w4a16_repack_ct")
+    _dev_call(weight_packed.device, "w4a16_repack_ct", _lib.w4a16_repack_ct, _ptr(weight_packed),
+              _ptr(weight_scale), K, N, group_size, _ptr(packed), stream=stream)
     return packed
 
 
@@ -295,8 +336,8 @@ def w4a16_repack_fused(parts, group_size: int = 128, stream=None,
     qptrs = (ctypes.c_void_p * n)(*[qw.data_ptr() for qw, _ in parts])
     sptrs = (ctypes.c_void_p * n)(*[sc.data_ptr() for _, sc in parts])
     narr = (ctypes.c_int * n)(*Ns)
-    _check(_lib.w4a16_repack_fused(n, qptrs, sptrs, narr, K, group_size, _ptr(packed),
-                                   _stream(stream)), "w4a16_repack_fused")
+    _dev_call(packed.device, "w4a16_repack_fused", _lib.w4a16_repack_fused, n, qptrs, sptrs, narr,
+              K, group_size, _ptr(packed), stream=stream)
     return packed
 
 
@@ -306,14 +347,18 @@ def w4a16_workspace_bytes(M: int, N: int, K: int, group_size: int = 128) -> int:
 
 def w4a16_gemm(x: torch.Tensor, packed: torch.Tensor, N: int, K: int, group_size: int = 128,
                out: torch.Tensor | None = None, workspace_buf: torch.Tensor | None = None,
-               stream=None) -> torch.Tensor:
-    """Y = x * dequant(W)^T for x bf16 [M][K] and a re-packed INT4 weight."""
+               stream=None, path: int = PATH_AUTO, late_weights: bool = False) -> torch.Tensor:
+    """Y = x * dequant(W)^T for x bf16 [M][K] and a re-packed INT4 weight.
+    ``path`` forces the weight-streaming (1) or tensor-core (2) path;
+    ``late_weights`` makes the kernel load weights only after the previous
+    kernel on the stream (for weights that kernel writes)."""
     M, out, ws = _gemm_buffers(
         x, K, N, out, workspace_buf,
         lambda: _need_bytes("w4a16", x.device.index, x.shape[0], N, K, group_size), stream)
     _need_weights(packed, torch.uint8, w4a16_packed_bytes(K, N, group_size), x.device, "packed")
-    _check(_lib.w4a16_gemm(_ptr(x), _ptr(packed), M, N, K, group_size, _ptr(out), _ptr(ws),
-                           ws.numel(), _stream(stream)), "w4a16_gemm")
+    _dev_call(x.device, "w4a16_gemm", _lib.w4a16_gemm_ex, _ptr(x), _ptr(packed), M, N, K,
+              group_size, _ptr(out), _ptr(ws), ws.numel(), _options(path, late_weights),
+              stream=stream)
     return out
 
 
@@ -323,47 +368,55 @@ class PreparedCall:
     here so they stay alive; their contents may change between calls, their
     storage must not move."""
 
-    def __init__(self, fn, args, what: str, keep):
+    def __init__(self, fn, args, what: str, keep, device):
         self._fn, self._args, self._what, self._keep = fn, tuple(args), what, keep
+        self._device = device
 
     def __call__(self) -> None:
-        status = self._fn(*self._args)
+        with _on_device(self._device):
+            status = self._fn(*self._args)
         if status != MXG_OK:
             raise MxgError(status, self._what)
 
 
 def prepare_w4a16_gemm(x: torch.Tensor, packed: torch.Tensor, N: int, K: int,
                        group_size: int = 128, out: torch.Tensor | None = None,
-                       workspace_buf: torch.Tensor | None = None, stream=None):
+                       workspace_buf: torch.Tensor | None = None, stream=None,
+                       path: int = PATH_AUTO, late_weights: bool = False):
     """(call, out): ``call()`` runs w4a16_gemm(x, packed) into ``out``."""
     M, out, ws = _gemm_buffers(
         x, K, N, out, workspace_buf,
         lambda: _need_bytes("w4a16", x.device.index, x.shape[0], N, K, group_size), stream)
     _need_weights(packed, torch.uint8, w4a16_packed_bytes(K, N, group_size), x.device, "packed")
     args = (_ptr(x), _ptr(packed), M, N, K, group_size, _ptr(out), _ptr(ws), ws.numel(),
-            _stream(stream))
-    return PreparedCall(_lib.w4a16_gemm, args, "w4a16_gemm", (x, packed, out, ws, stream)), out
+            _options(path, late_weights), _stream(stream, x.device))
+    return PreparedCall(_lib.w4a16_gemm_ex, args, "w4a16_gemm", (x, packed, out, ws, stream),
+                        x.device), out
 
 
 def prepare_mxfp8_gemm(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor,
                        out: torch.Tensor | None = None, workspace_buf: torch.Tensor | None = None,
-                       stream=None):
+                       stream=None, path: int = PATH_AUTO, late_weights: bool = False):
     """(call, out): ``call()`` runs mxfp8_gemm(x, wq, ws) into ``out``."""
     M, K, N = _mx_shapes(x, wq, ws)
     M, out, wsb = _gemm_buffers(x, K, N, out, workspace_buf,
                                 lambda: _need_bytes("mxfp8", x.device.index, M, N, K), stream)
     args = (_ptr(x), _ptr(wq), _ptr(ws), M, N, K, _ptr(out), _ptr(wsb), wsb.numel(),
-            _stream(stream))
-    return PreparedCall(_lib.mxfp8_gemm, args, "mxfp8_gemm", (x, wq, ws, out, wsb, stream)), out
+            _options(path, late_weights), _stream(stream, x.device))
+    return PreparedCall(_lib.mxfp8_gemm_ex, args, "mxfp8_gemm", (x, wq, ws, out, wsb, stream),
+                        x.device), out
 
 
 def prepare_bf16_gemm_small(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = None,
-                            workspace_buf: torch.Tensor | None = None, stream=None):
+                            workspace_buf: torch.Tensor | None = None, stream=None,
+                            late_weights: bool = False):
     """(call, out): ``call()`` runs bf16_gemm_small(x, w) into ``out``."""
     M, K, N, need = _small_shapes(x, w)
     M, out, wsb = _gemm_buffers(x, K, N, out, workspace_buf, lambda: need, stream)
-    args = (_ptr(x), _ptr(w), M, N, K, _ptr(out), _ptr(wsb), wsb.numel(), _stream(stream))
-    return PreparedCall(_lib.bf16_gemm_small, args, "bf16_gemm_small", (x, w, out, wsb, stream)), out
+    args = (_ptr(x), _ptr(w), M, N, K, _ptr(out), _ptr(wsb), wsb.numel(),
+            _options(PATH_AUTO, late_weights), _stream(stream, x.device))
+    return PreparedCall(_lib.bf16_gemm_small_ex, args, "bf16_gemm_small",
+                        (x, w, out, wsb, stream), x.device), out
 
 
 def w4a16_gemm_static_scratch(x: torch.Tensor, packed: torch.Tensor, N: int, K: int,
@@ -378,8 +431,8 @@ def w4a16_gemm_static_scratch(x: torch.Tensor, packed: torch.Tensor, N: int, K: 
         out = _empty((M, N), torch.bfloat16, x.device, stream)
     _need_out(out, M, N, x.device)
     _need_weights(packed, torch.uint8, w4a16_packed_bytes(K, N, group_size), x.device, "packed")
-    _check(_lib.w4a16_gemm_static_scratch(_ptr(x), _ptr(packed), M, N, K, group_size, _ptr(out),
-                                          _stream(stream)), "w4a16_gemm_static_scratch")
+    _dev_call(x.device, "w4a16_gemm_static_scratch", _lib.w4a16_gemm_static_scratch, _ptr(x),
+              _ptr(packed), M, N, K, group_size, _ptr(out), stream=stream)
     return out
 
 
@@ -390,8 +443,8 @@ def w4a16_unpack(packed: torch.Tensor, K: int, N: int, group_size: int = 128, st
     codes = _empty((N, K), torch.uint8, dev, stream)
     w32 = _empty((N, K), torch.float32, dev, stream)
     w16 = _empty((N, K), torch.bfloat16, dev, stream)
-    _check(_lib.w4a16_unpack(_ptr(packed), K, N, group_size, _ptr(codes), _ptr(w32), _ptr(w16),
-                             _stream(stream)), "w4a16_unpack")
+    _dev_call(packed.device, "w4a16_unpack", _lib.w4a16_unpack, _ptr(packed), K, N, group_size,
+              _ptr(codes), _ptr(w32), _ptr(w16), stream=stream)
     return codes, w32, w16
 
 
@@ -422,13 +475,13 @@ def mxfp8_workspace_bytes(M: int, N: int, K: int) -> int:
 
 def mxfp8_gemm(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor,
                out: torch.Tensor | None = None, workspace_buf: torch.Tensor | None = None,
-               stream=None) -> torch.Tensor:
+               stream=None, path: int = PATH_AUTO, late_weights: bool = False) -> torch.Tensor:
     """Y = x * dequant(W)^T for x bf16 [M][K], E4M3 codes wq[N][K], E8M0 ws[N][K/32]."""
     M, K, N = _mx_shapes(x, wq, ws)
     M, out, wsb = _gemm_buffers(x, K, N, out, workspace_buf,
                                 lambda: _need_bytes("mxfp8", x.device.index, M, N, K), stream)
-    _check(_lib.mxfp8_gemm(_ptr(x), _ptr(wq), _ptr(ws), M, N, K, _ptr(out), _ptr(wsb),
-                           wsb.numel(), _stream(stream)), "mxfp8_gemm")
+    _dev_call(x.device, "mxfp8_gemm", _lib.mxfp8_gemm_ex, _ptr(x), _ptr(wq), _ptr(ws), M, N, K,
+              _ptr(out), _ptr(wsb), wsb.numel(), _options(path, late_weights), stream=stream)
     return out
 
 
@@ -446,8 +499,8 @@ def mxfp8_dequant(wq: torch.Tensor, ws: torch.Tensor, stream=None) -> torch.Tens
     _need(ws, ws.dtype, "ws")
     _same_device(ws, wq.device, "ws")
     out = _empty((N, K), torch.bfloat16, wq.device, stream)
-    _check(_lib.mxfp8_dequant(_ptr(wq), _ptr(ws), N, K, _ptr(out), _stream(stream)),
-           "mxfp8_dequant")
+    _dev_call(wq.device, "mxfp8_dequant", _lib.mxfp8_dequant, _ptr(wq), _ptr(ws), N, K, _ptr(out),
+              stream=stream)
     return out
 
 
@@ -464,8 +517,8 @@ def _need_header(workspace_buf: torch.Tensor) -> None:
 def mxg_workspace_status(workspace_buf: torch.Tensor, stream=None) -> int:
     _need_header(workspace_buf)
     v = ctypes.c_int(0)
-    _check(_lib.mxg_workspace_status(_ptr(workspace_buf), ctypes.byref(v), _stream(stream)),
-           "mxg_workspace_status")
+    _dev_call(workspace_buf.device, "mxg_workspace_status", _lib.mxg_workspace_status,
+              _ptr(workspace_buf), ctypes.byref(v), stream=stream)
     return v.value
 
 
@@ -483,8 +536,8 @@ def w8a16_repack(qweight: torch.Tensor, scales: torch.Tensor, group_size: int = 
     _need_shape(scales, (K // group_size, N), "scales")
     _same_device(scales, qweight.device, "scales")
     packed = _empty(nbytes, torch.uint8, qweight.device, stream)
-    _check(_lib.w8a16_repack(_ptr(qweight), _ptr(scales), K, N, group_size, _ptr(packed),
-                             _stream(stream)), "w8a16_repack")
+    _dev_call(qweight.device, "w8a16_repack", _lib.w8a16_repack, _ptr(qweight), _ptr(scales), K, N,
+              group_size, _ptr(packed), stream=stream)
     return packed
 
 
@@ -502,8 +555,8 @@ def w8a16_repack_ct(weight_packed: torch.Tensor, weight_scale: torch.Tensor,
     _need_shape(weight_scale, (N, K // group_size), "weight_scale")
     _same_device(weight_scale, weight_packed.device, "weight_scale")
     packed = _empty(nbytes, torch.uint8, weight_packed.device, stream)
-    _check(_lib.w8a16_repack_ct(_ptr(weight_packed), _ptr(weight_scale), K, N, group_size,
-                                _ptr(packed), _stream(stream)), "w8a16_repack_ct")
+    _dev_call(weight_packed.device, "w8a16_repack_ct", _lib.w8a16_repack_ct, _ptr(weight_packed),
+              _ptr(weight_scale), K, N, group_size, _ptr(packed), stream=stream)
     return packed
 
 
@@ -516,28 +569,31 @@ def _w8_ws_bytes(M: int, N: int, K: int, group_size: int) -> int:
 
 def w8a16_gemm(x: torch.Tensor, packed: torch.Tensor, N: int, K: int, group_size: int = 128,
                out: torch.Tensor | None = None, workspace_buf: torch.Tensor | None = None,
-               stream=None) -> torch.Tensor:
+               stream=None, late_weights: bool = False) -> torch.Tensor:
     """Y = x * dequant(W)^T for x bf16 [M][K] (M <= 32) and a re-packed INT8 weight."""
     M, out, ws = _gemm_buffers(x, K, N, out, workspace_buf,
                                lambda: _w8_ws_bytes(x.shape[0], N, K, group_size), stream)
     _need_weights(packed, torch.uint8, int(_lib.w8a16_packed_bytes(K, N, group_size)), x.device,
                   "packed")
-    _check(_lib.w8a16_gemm(_ptr(x), _ptr(packed), M, N, K, group_size, _ptr(out), _ptr(ws),
-                           ws.numel(), _stream(stream)), "w8a16_gemm")
+    _dev_call(x.device, "w8a16_gemm", _lib.w8a16_gemm_ex, _ptr(x), _ptr(packed), M, N, K,
+              group_size, _ptr(out), _ptr(ws), ws.numel(), _options(PATH_AUTO, late_weights),
+              stream=stream)
     return out
 
 
 def prepare_w8a16_gemm(x: torch.Tensor, packed: torch.Tensor, N: int, K: int,
                        group_size: int = 128, out: torch.Tensor | None = None,
-                       workspace_buf: torch.Tensor | None = None, stream=None):
+                       workspace_buf: torch.Tensor | None = None, stream=None,
+                       late_weights: bool = False):
     """(call, out): ``call()`` runs w8a16_gemm(x, packed) into ``out``."""
     M, out, ws = _gemm_buffers(x, K, N, out, workspace_buf,
                                lambda: _w8_ws_bytes(x.shape[0], N, K, group_size), stream)
     _need_weights(packed, torch.uint8, int(_lib.w8a16_packed_bytes(K, N, group_size)), x.device,
                   "packed")
     args = (_ptr(x), _ptr(packed), M, N, K, group_size, _ptr(out), _ptr(ws), ws.numel(),
-            _stream(stream))
-    return PreparedCall(_lib.w8a16_gemm, args, "w8a16_gemm", (x, packed, out, ws, stream)), out
+            _options(PATH_AUTO, late_weights), _stream(stream, x.device))
+    return PreparedCall(_lib.w8a16_gemm_ex, args, "w8a16_gemm", (x, packed, out, ws, stream),
+                        x.device), out
 
 
 def _small_shapes(x: torch.Tensor, w: torch.Tensor):
@@ -556,39 +612,45 @@ def _small_shapes(x: torch.Tensor, w: torch.Tensor):
 
 
 def bf16_gemm_small(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = None,
-                    workspace_buf: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+                    workspace_buf: torch.Tensor | None = None, stream=None,
+                    late_weights: bool = False) -> torch.Tensor:
     """Y = x * w^T with dense bf16 w [N][K] (few columns, e.g. the paired
     48 + 48 GDN A/B projection) and x bf16 [M][K], M <= 8."""
     M, K, N, need = _small_shapes(x, w)
     M, out, ws = _gemm_buffers(x, K, N, out, workspace_buf, lambda: need, stream)
-    _check(_lib.bf16_gemm_small(_ptr(x), _ptr(w), M, N, K, _ptr(out), _ptr(ws), ws.numel(),
-                                _stream(stream)), "bf16_gemm_small")
+    _dev_call(x.device, "bf16_gemm_small", _lib.bf16_gemm_small_ex, _ptr(x), _ptr(w), M, N, K,
+              _ptr(out), _ptr(ws), ws.numel(), _options(PATH_AUTO, late_weights),
+              stream=stream)
     return out
 
 
-def mxg_selftest_wait_timeout(workspace_buf: torch.Tensor, limit_us: int, stream=None) -> None:
+def mxg_selftest_wait_timeout(workspace_buf: torch.Tensor | None, limit_us: int,
+                              stream=None, device=None) -> None:
+    """Runs the library's bounded-wait self-test, which records
+    MXG_ERR_TIMEOUT in ``workspace_buf``'s status word, or (None) in the
+    static scratch array of ``device`` (default: the current device)."""
+    if workspace_buf is None:
+        dev = torch.device("cuda", torch.cuda.current_device() if device is None else
+                           torch.device(device).index)
+        _dev_call(dev, "mxg_selftest_wait_timeout", _lib.mxg_selftest_wait_timeout, None,
+                  int(limit_us), stream=stream)
+        return
     _need_header(workspace_buf)
-    _check(_lib.mxg_selftest_wait_timeout(_ptr(workspace_buf), int(limit_us), _stream(stream)),
-           "mxg_selftest_wait_timeout")
+    _dev_call(workspace_buf.device, "mxg_selftest_wait_timeout", _lib.mxg_selftest_wait_timeout,
+              _ptr(workspace_buf), int(limit_us), stream=stream)
 
 
-def mxg_set_path(path: int) -> int:
-    """0 = automatic, 1 = weight streaming, 2 = tensor cores; returns the previous value."""
-    r = int(_lib.mxg_set_path(int(path)))
-    if r < 0:
-        raise ValueError("path must be 0, 1 or 2")
-    return r
-
-
-def mxg_set_early_weight_loads(on: int) -> int:
-    """1 (default): the weight-streaming kernels load their first weight tiles
-    before waiting for the previous kernel on the stream; 0: after it, for
-    callers that write weights in the kernel right before a GEMM.  Returns
-    the previous value."""
-    r = int(_lib.mxg_set_early_weight_loads(int(on)))
-    if r < 0:
-        raise ValueError("on must be 0 or 1")
-    return r
+def w4a16_static_scratch_status(reset: bool = False, stream=None, device=None) -> int:
+    """The status word of the static scratch array of ``device`` (default:
+    the current device): 0, or the first error a kernel recorded there.
+    ``reset`` also zeroes the status word and the arrival counters.
+    Synchronizes the stream."""
+    dev = torch.device("cuda", torch.cuda.current_device() if device is None else
+                       torch.device(device).index)
+    v = ctypes.c_int(0)
+    _dev_call(dev, "w4a16_static_scratch_status", _lib.w4a16_static_scratch_status,
+              ctypes.byref(v), 1 if reset else 0, stream=stream)
+    return v.value
 
 
 def raw_lib() -> ctypes.CDLL:

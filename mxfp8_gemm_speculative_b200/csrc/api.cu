@@ -19,8 +19,6 @@ namespace {
 constexpr int kMaxDevices = 64;
 DeviceInfo g_info[kMaxDevices];
 std::once_flag g_info_once[kMaxDevices];
-std::atomic<int> g_path{0};
-std::atomic<int> g_early_weights{1};
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
@@ -62,11 +60,6 @@ bool mxfp8_shape_ok(int K, int N)
     return K > 0 && N >= 128 && K % 32 == 0;
 }
 }  // namespace
-
-bool early_weight_loads()
-{
-    return g_early_weights.load(std::memory_order_relaxed) != 0;
-}
 
 const DeviceInfo &device_info(int device)
 {
@@ -169,13 +162,29 @@ static size_t mxfp8_tc_ws(int dev, int M, int N, int K)
     return make_workspace_map(tp.counters, tp.partial_bytes).total;
 }
 
-// 1 = streaming, 2 = tensor cores, 0 = no path.
-static int choose_path(int M, bool stream_ok, bool tc_ok)
+// The call's options with the defaults filled in; false for values outside
+// their documented range.
+static bool resolve_options(const mxg_gemm_options *o, int *path, bool *early)
 {
-    const int forced = g_path.load();
-    if (forced == 1)
+    *path = MXG_PATH_AUTO;
+    *early = true;
+    if (!o)
+        return true;
+    if (o->path < MXG_PATH_AUTO || o->path > MXG_PATH_TENSOR)
+        return false;
+    if (o->late_weights != 0 && o->late_weights != 1)
+        return false;
+    *path = o->path;
+    *early = o->late_weights == 0;
+    return true;
+}
+
+// 1 = streaming, 2 = tensor cores, 0 = no path.
+static int choose_path(int forced, int M, bool stream_ok, bool tc_ok)
+{
+    if (forced == MXG_PATH_STREAM)
         return stream_ok ? 1 : 0;
-    if (forced == 2)
+    if (forced == MXG_PATH_TENSOR)
         return tc_ok ? 2 : 0;
     if (M <= 32 && stream_ok)
         return 1;
@@ -199,6 +208,8 @@ const char *mxg_status_string(int status)
     case MXG_ERR_WORKSPACE: return "workspace too small";
     case MXG_ERR_CUDA: return "CUDA runtime or launch error";
     case MXG_ERR_TIMEOUT: return "a bounded in-kernel wait timed out";
+    case MXG_ERR_CAPTURE:
+        return "a call that needs its one-time device set-up was made during stream capture";
     default: return "unknown status";
     }
 }
@@ -270,9 +281,14 @@ size_t w4a16_workspace_bytes(int M, int N, int K, int group_size)
     return r ? r : sizeof(WsHeader);
 }
 
-int w4a16_gemm(const void *X, const void *packed, int M, int N, int K, int group_size, void *Y,
-               void *workspace, size_t workspace_bytes, cudaStream_t stream)
+int w4a16_gemm_ex(const void *X, const void *packed, int M, int N, int K, int group_size, void *Y,
+                  void *workspace, size_t workspace_bytes, const mxg_gemm_options *opts,
+                  cudaStream_t stream)
 {
+    int forced = 0;
+    bool early = true;
+    if (!resolve_options(opts, &forced, &early))
+        return MXG_ERR_INVALID_ARG;
     if (!aligned16(X) || !aligned16(packed) || !aligned16(Y) || !aligned16(workspace) || M < 1)
         return MXG_ERR_INVALID_ARG;
     if (!w4a16_shape_ok(K, N, group_size))
@@ -284,22 +300,30 @@ int w4a16_gemm(const void *X, const void *packed, int M, int N, int K, int group
     TcPlan tp;
     const bool s_ok = plan_w4a16_stream(dev, M, N, K, group_size, &sp);
     // the tensor-core plan only matters when the streaming path is not taken
-    const bool t_ok = (M <= 32 && s_ok && g_path.load() != 2)
+    const bool t_ok = (M <= 32 && s_ok && forced != MXG_PATH_TENSOR)
                           ? false
                           : plan_w4a16_tc(dev, M, N, K, group_size, &tp);
-    const int path = choose_path(M, s_ok, t_ok);
+    const int path = choose_path(forced, M, s_ok, t_ok);
     if (path == 1) {
         if (workspace_bytes < make_workspace_map(sp.ntiles, sp.partial_bytes).total)
             return MXG_ERR_WORKSPACE;
         return to_status(
-            launch_w4a16_stream(sp, X, packed, M, N, K, group_size, Y, workspace, stream));
+            launch_w4a16_stream(sp, X, packed, M, N, K, group_size, Y, workspace, early, stream));
     }
     if (path == 2) {
         if (workspace_bytes < make_workspace_map(tp.counters, tp.partial_bytes).total)
             return MXG_ERR_WORKSPACE;
-        return to_status(launch_w4a16_tc(tp, X, packed, M, N, K, group_size, Y, workspace, stream));
+        return to_status(
+            launch_w4a16_tc(tp, X, packed, M, N, K, group_size, Y, workspace, early, stream));
     }
     return MXG_ERR_UNSUPPORTED_SHAPE;
+}
+
+int w4a16_gemm(const void *X, const void *packed, int M, int N, int K, int group_size, void *Y,
+               void *workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    return w4a16_gemm_ex(X, packed, M, N, K, group_size, Y, workspace, workspace_bytes, nullptr,
+                         stream);
 }
 
 size_t w8a16_packed_bytes(int K, int N, int group_size)
@@ -343,9 +367,14 @@ size_t w8a16_workspace_bytes(int M, int N, int K, int group_size)
     return make_workspace_map(sp.ntiles, sp.partial_bytes).total;
 }
 
-int w8a16_gemm(const void *X, const void *packed, int M, int N, int K, int group_size, void *Y,
-               void *workspace, size_t workspace_bytes, cudaStream_t stream)
+int w8a16_gemm_ex(const void *X, const void *packed, int M, int N, int K, int group_size, void *Y,
+                  void *workspace, size_t workspace_bytes, const mxg_gemm_options *opts,
+                  cudaStream_t stream)
 {
+    int forced = 0;
+    bool early = true;
+    if (!resolve_options(opts, &forced, &early) || forced == MXG_PATH_TENSOR)
+        return MXG_ERR_INVALID_ARG;   // INT8 has the weight-streaming path only
     if (!aligned16(X) || !aligned16(packed) || !aligned16(Y) || !aligned16(workspace) || M < 1)
         return MXG_ERR_INVALID_ARG;
     if (M > 32 || !w4a16_shape_ok(K, N, group_size))
@@ -358,7 +387,15 @@ int w8a16_gemm(const void *X, const void *packed, int M, int N, int K, int group
         return MXG_ERR_UNSUPPORTED_SHAPE;
     if (workspace_bytes < make_workspace_map(sp.ntiles, sp.partial_bytes).total)
         return MXG_ERR_WORKSPACE;
-    return to_status(launch_w4a16_stream(sp, X, packed, M, N, K, group_size, Y, workspace, stream));
+    return to_status(
+        launch_w4a16_stream(sp, X, packed, M, N, K, group_size, Y, workspace, early, stream));
+}
+
+int w8a16_gemm(const void *X, const void *packed, int M, int N, int K, int group_size, void *Y,
+               void *workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    return w8a16_gemm_ex(X, packed, M, N, K, group_size, Y, workspace, workspace_bytes, nullptr,
+                         stream);
 }
 
 size_t mxfp8_workspace_bytes(int M, int N, int K)
@@ -374,9 +411,14 @@ size_t mxfp8_workspace_bytes(int M, int N, int K)
     return r ? r : sizeof(WsHeader);
 }
 
-int mxfp8_gemm(const void *X, const uint8_t *Wq, const uint8_t *Ws, int M, int N, int K, void *Y,
-               void *workspace, size_t workspace_bytes, cudaStream_t stream)
+int mxfp8_gemm_ex(const void *X, const uint8_t *Wq, const uint8_t *Ws, int M, int N, int K,
+                  void *Y, void *workspace, size_t workspace_bytes, const mxg_gemm_options *opts,
+                  cudaStream_t stream)
 {
+    int forced = 0;
+    bool early = true;
+    if (!resolve_options(opts, &forced, &early))
+        return MXG_ERR_INVALID_ARG;
     if (!aligned16(X) || !aligned16(Wq) || !aligned16(Ws) || !aligned16(Y) ||
         !aligned16(workspace) || M < 1)
         return MXG_ERR_INVALID_ARG;
@@ -388,21 +430,28 @@ int mxfp8_gemm(const void *X, const uint8_t *Wq, const uint8_t *Ws, int M, int N
     StreamPlan sp;
     TcPlan tp;
     const bool s_ok = plan_mxfp8_stream(dev, M, N, K, &sp);
-    const bool t_ok = (M <= 32 && s_ok && g_path.load() != 2)
+    const bool t_ok = (M <= 32 && s_ok && forced != MXG_PATH_TENSOR)
                           ? false
                           : plan_mxfp8_tc(dev, M, N, K, &tp);
-    const int path = choose_path(M, s_ok, t_ok);
+    const int path = choose_path(forced, M, s_ok, t_ok);
     if (path == 1) {
         if (workspace_bytes < make_workspace_map(sp.ntiles, sp.partial_bytes).total)
             return MXG_ERR_WORKSPACE;
-        return to_status(launch_mxfp8_stream(sp, X, Wq, Ws, M, N, K, Y, workspace, stream));
+        return to_status(
+            launch_mxfp8_stream(sp, X, Wq, Ws, M, N, K, Y, workspace, early, stream));
     }
     if (path == 2) {
         if (workspace_bytes < make_workspace_map(tp.counters, tp.partial_bytes).total)
             return MXG_ERR_WORKSPACE;
-        return to_status(launch_mxfp8_tc(tp, X, Wq, Ws, M, N, K, Y, workspace, stream));
+        return to_status(launch_mxfp8_tc(tp, X, Wq, Ws, M, N, K, Y, workspace, early, stream));
     }
     return MXG_ERR_UNSUPPORTED_SHAPE;
+}
+
+int mxfp8_gemm(const void *X, const uint8_t *Wq, const uint8_t *Ws, int M, int N, int K, void *Y,
+               void *workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    return mxfp8_gemm_ex(X, Wq, Ws, M, N, K, Y, workspace, workspace_bytes, nullptr, stream);
 }
 
 int w4a16_unpack(const void *packed, int K, int N, int group_size, uint8_t *codes, float *w_fp32,
@@ -442,8 +491,18 @@ int mxg_workspace_status(const void *workspace, int *status, cudaStream_t stream
 
 int mxg_selftest_wait_timeout(void *workspace, int limit_us, cudaStream_t stream)
 {
-    if (!aligned16(workspace) || limit_us < 1 || limit_us > 10000000)
+    if ((workspace && !aligned16(workspace)) || limit_us < 1 || limit_us > 10000000)
         return MXG_ERR_INVALID_ARG;
+    if (!workspace) {
+        // the static scratch array of w4a16_gemm_static_scratch on this device
+        const int dev = current_device();
+        if (dev < 0)
+            return MXG_ERR_CUDA;
+        int st = MXG_OK;
+        workspace = static_scratch(dev, stream, &st);
+        if (!workspace)
+            return st;
+    }
     return to_status(launch_wait_timeout_selftest(workspace, limit_us, stream));
 }
 
@@ -455,9 +514,13 @@ size_t bf16_gemm_small_workspace_bytes(int M, int N, int K)
     return make_workspace_map(1, sp.partial_bytes).total;
 }
 
-int bf16_gemm_small(const void *X, const void *W, int M, int N, int K, void *Y, void *workspace,
-                    size_t workspace_bytes, cudaStream_t stream)
+int bf16_gemm_small_ex(const void *X, const void *W, int M, int N, int K, void *Y, void *workspace,
+                       size_t workspace_bytes, const mxg_gemm_options *opts, cudaStream_t stream)
 {
+    int forced = 0;
+    bool early = true;
+    if (!resolve_options(opts, &forced, &early) || forced != MXG_PATH_AUTO)
+        return MXG_ERR_INVALID_ARG;   // one kernel: no path to choose
     if (!aligned16(X) || !aligned16(W) || !aligned16(Y) || !aligned16(workspace) || M < 1)
         return MXG_ERR_INVALID_ARG;
     SmallPlan sp;
@@ -465,21 +528,13 @@ int bf16_gemm_small(const void *X, const void *W, int M, int N, int K, void *Y, 
         return MXG_ERR_UNSUPPORTED_SHAPE;
     if (workspace_bytes < make_workspace_map(1, sp.partial_bytes).total)
         return MXG_ERR_WORKSPACE;
-    return to_status(launch_bf16_small(sp, X, W, M, N, K, Y, workspace, stream));
+    return to_status(launch_bf16_small(sp, X, W, M, N, K, Y, workspace, early, stream));
 }
 
-int mxg_set_path(int path)
+int bf16_gemm_small(const void *X, const void *W, int M, int N, int K, void *Y, void *workspace,
+                    size_t workspace_bytes, cudaStream_t stream)
 {
-    if (path < 0 || path > 2)
-        return -1;
-    return g_path.exchange(path);
-}
-
-int mxg_set_early_weight_loads(int on)
-{
-    if (on != 0 && on != 1)
-        return -1;
-    return g_early_weights.exchange(on);
+    return bf16_gemm_small_ex(X, W, M, N, K, Y, workspace, workspace_bytes, nullptr, stream);
 }
 
 }  // extern "C"

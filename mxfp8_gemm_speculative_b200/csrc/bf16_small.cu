@@ -133,7 +133,7 @@ bool plan_bf16_small(int M, int N, int K, SmallPlan *plan)
 }
 
 cudaError_t launch_bf16_small(const SmallPlan &pl, const void *X, const void *W, int M, int N, int K,
-                              void *Y, void *workspace, cudaStream_t stream)
+                              void *Y, void *workspace, bool early, cudaStream_t stream)
 {
     (void)workspace;
     SmallParams p{};
@@ -144,7 +144,7 @@ cudaError_t launch_bf16_small(const SmallPlan &pl, const void *X, const void *W,
     p.N = N;
     p.K = K;
     p.chunks = pl.chunks;
-    p.early = early_weight_loads() ? 1 : 0;
+    p.early = early ? 1 : 0;
     void *args[] = {&p};
     return launch_pdl(reinterpret_cast<const void *>(&bf16_small_kernel), dim3(pl.ctas),
                       dim3(pl.threads), 0, stream, args);

@@ -52,22 +52,20 @@ struct StreamPlan {
     int ntiles;           // output tiles (= arrival counters)
 };
 
-// Whether the streaming kernels load their first weights before waiting for
-// the previous kernel on the stream (process-wide, default on; see
-// mxg_set_early_weight_loads).
-bool early_weight_loads();
-
 bool plan_w4a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan);
 // INT8 W8A16 (two code planes) on the same kernel; launch_w4a16_stream runs
 // either plan.
 bool plan_w8a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan);
+// early: load the first weights before waiting for the previous kernel on
+// the stream (every launch function below takes it per call).
 cudaError_t launch_w4a16_stream(const StreamPlan &plan, const void *X, const void *packed, int M,
-                                int N, int K, int G, void *Y, void *workspace, cudaStream_t stream);
+                                int N, int K, int G, void *Y, void *workspace, bool early,
+                                cudaStream_t stream);
 
 bool plan_mxfp8_stream(int device, int M, int N, int K, StreamPlan *plan);
 cudaError_t launch_mxfp8_stream(const StreamPlan &plan, const void *X, const uint8_t *Wq,
                                 const uint8_t *Ws, int M, int N, int K, void *Y, void *workspace,
-                                cudaStream_t stream);
+                                bool early, cudaStream_t stream);
 
 // ----------------------------------------------------- tensor-core path
 struct TcPlan {
@@ -81,11 +79,12 @@ struct TcPlan {
 };
 bool plan_w4a16_tc(int device, int M, int N, int K, int G, TcPlan *plan);
 cudaError_t launch_w4a16_tc(const TcPlan &plan, const void *X, const void *packed, int M, int N,
-                            int K, int G, void *Y, void *workspace, cudaStream_t stream);
+                            int K, int G, void *Y, void *workspace, bool early,
+                            cudaStream_t stream);
 bool plan_mxfp8_tc(int device, int M, int N, int K, TcPlan *plan);
 cudaError_t launch_mxfp8_tc(const TcPlan &plan, const void *X, const uint8_t *Wq,
                             const uint8_t *Ws, int M, int N, int K, void *Y, void *workspace,
-                            cudaStream_t stream);
+                            bool early, cudaStream_t stream);
 
 // ------------------------------------------ dense bf16, few output columns
 // Split-K plan: K in 64-wide chunks over `ctas` CTAs of N/16 warps each.
@@ -97,7 +96,7 @@ struct SmallPlan {
 };
 bool plan_bf16_small(int M, int N, int K, SmallPlan *plan);
 cudaError_t launch_bf16_small(const SmallPlan &plan, const void *X, const void *W, int M, int N,
-                              int K, void *Y, void *workspace, cudaStream_t stream);
+                              int K, void *Y, void *workspace, bool early, cudaStream_t stream);
 
 // ------------------------------------------------------------ weight tools
 // n_major: compressed-tensors inputs ([N][K/8] words, [N][K/G] scales)
@@ -119,6 +118,13 @@ cudaError_t launch_w4a16_unpack(const void *packed, int K, int N, int G, uint8_t
 cudaError_t launch_mxfp8_dequant(const uint8_t *Wq, const uint8_t *Ws, int N, int K,
                                  uint16_t *w_bf16, cudaStream_t stream);
 cudaError_t launch_wait_timeout_selftest(void *workspace, int limit_us, cudaStream_t stream);
+
+// The static scratch array of w4a16_gemm_static_scratch on device `dev`
+// (current), set up on `stream` by the first successful call; NULL with
+// *status set (MXG_ERR_CAPTURE while `stream` is captured before that
+// set-up, MXG_ERR_CUDA otherwise).
+void *static_scratch(int dev, cudaStream_t stream, int *status);
+size_t static_scratch_bytes();
 
 // Launch with programmatic stream serialization: the kernel may start while
 // the previous kernel of the stream drains (it calls griddepcontrol.wait

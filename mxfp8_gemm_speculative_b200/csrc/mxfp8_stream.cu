@@ -524,7 +524,7 @@ bool plan_mxfp8_stream(int device, int M, int N, int K, StreamPlan *plan)
 
 cudaError_t launch_mxfp8_stream(const StreamPlan &pl, const void *X, const uint8_t *Wq,
                                 const uint8_t *Ws, int M, int N, int K, void *Y, void *workspace,
-                                cudaStream_t stream)
+                                bool early, cudaStream_t stream)
 {
     const void *fn = select_kernel(pl.tt, pl.variant);
     if (!fn)
@@ -538,7 +538,7 @@ cudaError_t launch_mxfp8_stream(const StreamPlan &pl, const void *X, const uint8
     p.X = static_cast<const uint16_t *>(X);
     p.Ws = Ws;
     p.Y = static_cast<uint16_t *>(Y);
-    p.early = early_weight_loads() ? 1 : 0;
+    p.early = early ? 1 : 0;
     p.hdr = static_cast<WsHeader *>(workspace);
     p.counters = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + wm.counters_off);
     p.partial = reinterpret_cast<float4 *>(static_cast<uint8_t *>(workspace) + wm.partial_off);

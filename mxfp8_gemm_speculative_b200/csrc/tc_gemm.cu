@@ -741,7 +741,8 @@ bool plan_w4a16_tc(int device, int M, int N, int K, int G, TcPlan *plan)
 }
 
 cudaError_t launch_w4a16_tc(const TcPlan &pl, const void *X, const void *packed, int M, int N,
-                            int K, int G, void *Y, void *workspace, cudaStream_t stream)
+                            int K, int G, void *Y, void *workspace, bool early,
+                            cudaStream_t stream)
 {
     alignas(64) CUtensorMap xm, wm, sm;
     const uint8_t *codes = static_cast<const uint8_t *>(packed);
@@ -771,7 +772,7 @@ cudaError_t launch_w4a16_tc(const TcPlan &pl, const void *X, const void *packed,
     p.num_tiles = pl.mtiles * pl.ntiles;
     p.splits = pl.splits;
     p.num_items = p.num_tiles * pl.splits;
-    p.early = early_weight_loads() ? 1 : 0;
+    p.early = early ? 1 : 0;
     {
         const WorkspaceMap wsm = make_workspace_map(pl.counters, pl.partial_bytes);
         p.counters = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + wsm.counters_off);
@@ -789,7 +790,7 @@ bool plan_mxfp8_tc(int device, int M, int N, int K, TcPlan *plan)
 
 cudaError_t launch_mxfp8_tc(const TcPlan &pl, const void *X, const uint8_t *Wq,
                             const uint8_t *Ws, int M, int N, int K, void *Y, void *workspace,
-                            cudaStream_t stream)
+                            bool early, cudaStream_t stream)
 {
     alignas(64) CUtensorMap xm, wm;
     if (!x_map(&xm, X, M, K, pl.bm) ||
@@ -810,7 +811,7 @@ cudaError_t launch_mxfp8_tc(const TcPlan &pl, const void *X, const uint8_t *Wq,
     p.num_tiles = pl.mtiles * pl.ntiles;
     p.splits = pl.splits;
     p.num_items = p.num_tiles * pl.splits;
-    p.early = early_weight_loads() ? 1 : 0;
+    p.early = early ? 1 : 0;
     {
         const WorkspaceMap wsm = make_workspace_map(pl.counters, pl.partial_bytes);
         p.counters = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + wsm.counters_off);

@@ -1,35 +1,42 @@
 // INT4 W4A16 weight-streaming GEMM for small M (decode / MTP verify chunks).
 //
 // At M <= 32 the layer reads each weight byte once and does 2*M flops per
-// weight: it is bound by HBM bytes of W.  The kernel therefore
-//  * cuts the re-packed weight stream into equal units (one n32 tile x one
-//    or two spans of max(G, 64) rows of K) and gives every CTA of a
-//    persistent grid (one per SM) one contiguous run of units (stream-K at
-//    CTA granularity), so all SMs stream the same number of bytes;
-//  * the CTA's warps take the run's units in turn (unit i goes to warp
-//    i mod C), so every warp works on the same n32 tile at once and a warp
-//    the scheduler serves less only delays its own units;
-//  * each warp moves its units through its own ring of shared-memory slots
-//    with 1-D bulk copies (cp.async.bulk, completion on an mbarrier; codes
-//    and scales of a unit), several units ahead, weights marked evict-first
-//    in L2;
-//  * each warp decodes a pair of nibbles to the bf16 pair (128 + q) with one
+// weight: it is bound by HBM bytes of W, and the whole design is about
+// keeping enough weight bytes in flight on every SM while the decode and the
+// MMAs run behind them.
+//
+//  * Columns are taken eight n32 tiles (256 columns) at a time, a "column
+//    group".  The weight stream of a group row is cut into units of
+//    max(KS, G) rows of K (KS = rows per pipeline stage), and every CTA of a
+//    one-CTA-per-SM grid takes one contiguous run of units (stream-K), so all
+//    SMs stream the same number of bytes.
+//  * One producer warp fills a CTA-wide ring of stages with 2-D tensor-map
+//    copies (TMA): per stage the codes of the eight tiles for KS rows of K
+//    (one box), their scales (one box) and the activations X for the same
+//    rows (64-wide boxes with 128-byte swizzle; rows past M are zero-filled by
+//    the copy).  Completion is an mbarrier per stage; the consumers release a
+//    stage through a second mbarrier.  Weights are marked evict-first in L2,
+//    the activations evict-last (every CTA re-reads them).
+//  * Eight consumer warps, warp w owning tile w of the group for the whole
+//    K range of the CTA's segment: no reduction between warps.  Each warp
+//    decodes a pair of nibbles to the bf16 pair (128 + q) with one
 //    mask-and-or (plus a shift) and multiplies on the tensor cores with
 //    m16n8k16 MMAs where the weights are the 16-row operand and the tokens
-//    the 8-column operand ("swap AB"); the two n16 halves of a unit share
-//    each activation fragment, and one more MMA with an all-ones weight tile
-//    gives the per-token activation sum that turns (128 + q) into (q - 8);
-//  * starts a zero-initialised partial sum per scale group (every MMA step
-//    lies inside one group for G = 32, 64, 128) and adds
-//    (partial - 136 * activation sum) * scale in fp32 once per group, so
-//    weights are never rounded (every product is exact in fp32);
-//  * at the end of each tile every warp leaves its fragment in shared memory
-//    and goes on; the last warp to arrive adds the fragments.  A tile inside
-//    the CTA's run is written to Y at once.  A tile cut between CTAs is
-//    finished by the CTA holding its first unit, at the end of that CTA's
-//    run: the other contributors (for whom it is the first tile of the run)
-//    published their fragments early, so it adds them in CTA order
-//    (deterministic) and writes bf16 Y.
+//    the 8-column operand ("swap AB"); one more MMA with an all-ones weight
+//    tile gives the per-token activation sum that turns (128 + q) into
+//    (q - 8).  A zero-initialised partial sum per scale group is folded in
+//    as acc += (part - 136 * activation sum) * scale in fp32, so weights are
+//    never rounded (every product is exact in fp32).
+//  * A group row cut between CTAs is finished by the CTA holding its first
+//    unit, which reaches it last in its run; the other contributors (for
+//    whom it is the first segment of their run) publish their fragments
+//    early, so the finisher adds them in CTA order (deterministic) and
+//    writes bf16 Y.  A group row inside one run is written directly.
+//  * The footprint (9 warps, <= 112 registers for M <= 16, ~100 KB of shared
+//    memory) lets two CTAs share an SM: the next GEMM on the stream (launched
+//    with programmatic dependent launch) becomes resident while this one
+//    streams, issues its first weight copies and warms L2 with the next part
+//    of its run, and only then waits for this grid before reading X.
 //
 // The same kernel runs INT8 W8A16 weights (the vocabulary head): their
 // re-pack splits each 8-bit code q = 16 hi + lo into a plane of low and a
@@ -45,78 +52,84 @@
 namespace mxg {
 namespace {
 
-#ifndef MXG_STREAM_CONSUMERS
-#define MXG_STREAM_CONSUMERS 12
+#ifndef MXG_STREAM_KS
+#define MXG_STREAM_KS 64
 #endif
-#ifndef MXG_STREAM_CTAS_PER_SM
-#define MXG_STREAM_CTAS_PER_SM 1
+#ifndef MXG_STREAM_RING_KB
+#define MXG_STREAM_RING_KB 104
 #endif
-#ifndef MXG_STREAM_STAGES_BIG
-#define MXG_STREAM_STAGES_BIG 2
+#ifndef MXG_STREAM_RING2_KB
+#define MXG_STREAM_RING2_KB 192
 #endif
-constexpr int kConsumers = MXG_STREAM_CONSUMERS;  // warps per CTA
-constexpr int kThreads = kConsumers * 32;
-constexpr int kCtasPerSm = MXG_STREAM_CTAS_PER_SM;   // resident CTAs per SM (grid size / SMs)
-constexpr int kMinUnitsPerCta = 2 * kConsumers;  // shortest run
+#ifndef MXG_STREAM_WPT2_MAX_TT
+#define MXG_STREAM_WPT2_MAX_TT 0
+#endif
+#ifndef MXG_STREAM_PF_STAGES
+#define MXG_STREAM_PF_STAGES 12
+#endif
 
-// Group modes: 0 -> G = 128, 1 -> G = 64, 2 -> G = 32.  A unit (what one
-// ring slot holds) spans SU times max(G, 64) rows of K of one n32 tile.
-// P code planes: 1 for INT4; 2 for INT8, whose codes are stored as a plane
-// of low nibbles and a plane of high nibbles, each in the INT4 layout.
-template <int GM, int SU, int P = 1>
-struct Mode {
-    static constexpr int kG = GM == 0 ? 128 : (GM == 1 ? 64 : 32);
-    static constexpr int kChunks = (GM == 0 ? 2 : 1) * SU;    // k64 chunks per unit
-    static constexpr int kGroups = (GM == 2 ? 2 : 1) * SU;    // scale groups per unit
-    static constexpr int kStepsPerGroup = kG / 16;            // MMA k16 steps per group
-    static constexpr int kCode = kChunks * 1024 * P;          // code bytes per unit
-    static constexpr int kScale = kGroups * 64;               // scale bytes per unit
-    // slots per warp: shallow rings (12 warps x 2-3 slots keep enough bytes in
-    // flight) leave most of the SM's shared-memory/L1 split to L1, where the
-    // re-read activations hit
-    static constexpr int kStages = kCode >= 4096 ? MXG_STREAM_STAGES_BIG : 3;
+constexpr int kWarps = 8;                     // n32 tiles of a column group
+
+// Consumer warps per tile: two for narrow token tiles (each takes every
+// other stage of the run, so a warp has two stages' time for the latency
+// chain of one), one for wide ones (whose registers allow no more warps).
+template <int TT>
+struct Wpt {
+    static constexpr int value = TT <= MXG_STREAM_WPT2_MAX_TT ? 2 : 1;
 };
 
-// Shared memory: every warp's ring of kStages slots (a slot holds one
-// unit's codes, then its scales), kRed reduction buffers of kConsumers
-// fragments (segment s of the run uses buffer s mod kRed), one mbarrier per
-// slot, then per reduction buffer an arrival count and a use count.
-template <int TT, int GM, int SU, int P = 1>
-struct Smem {
-    using MD = Mode<GM, SU, P>;
-    static constexpr int kFrag4 = 2 * TT * 32;                // float4 per warp fragment
-    static constexpr int kSlot = (MD::kCode + MD::kScale + 127) / 128 * 128;
-    // One reduction buffer: a warp that ends a segment before the previous
-    // segment's reduction is done waits for it (rarely), and the smaller
-    // shared-memory footprint leaves a larger L1 for the activation loads
-    // (every CTA re-reads X for each of its tiles).
-    static constexpr int kRed = 1;
-    static constexpr size_t kRingBytes = (size_t)kConsumers * MD::kStages * kSlot;
-    static constexpr size_t kRedBytes = (size_t)kRed * kConsumers * kFrag4 * 16;
-    static constexpr size_t kBarBytes = (size_t)kConsumers * MD::kStages * 8;
-    static constexpr size_t kRedOff = kRingBytes;
-    static constexpr size_t kBarOff = kRedOff + kRedBytes;
-    static constexpr size_t kSyncOff = kBarOff + kBarBytes;
-    static constexpr size_t kTotal = kSyncOff + 2 * kRed * sizeof(int);
+// Group modes: 0 -> G = 128, 1 -> G = 64, 2 -> G = 32.  P code planes: 1 for
+// INT4; 2 for INT8 (low and high nibbles, each in the INT4 layout).
+template <int TT, int GM, int P>
+struct Cfg {
+    static constexpr int kWPT = Wpt<TT>::value;
+    static constexpr int kConsumers = kWarps * kWPT;
+    static constexpr int kThreads = (kConsumers + 1) * 32;         // + the producer warp
+    static constexpr int kProducer = kConsumers;                   // its warp index
+    // one CTA per SM with two consumer warps per tile; with one, the ring
+    // leaves room for a second CTA (the next GEMM on the stream)
+    static constexpr int kRingBytes = (kWPT == 2 ? MXG_STREAM_RING2_KB : MXG_STREAM_RING_KB) * 1024;
+    static constexpr int kG = GM == 0 ? 128 : (GM == 1 ? 64 : 32);
+    static constexpr int kKS = P == 2 ? 64 : MXG_STREAM_KS;       // rows of K per stage
+    static constexpr int kChunks = kKS / 64;                       // k64 chunks per stage
+    static constexpr int kSteps = kKS / 16;                        // k16 MMA steps per stage
+    static constexpr int kStepsPerGroup = kG / 16;
+    // steps between scale epilogues: a group, or a stage when a group spans
+    // stages that different warps take
+    static constexpr int kEpi = (kWPT == 2 && kStepsPerGroup > kSteps) ? kSteps : kStepsPerGroup;
+    static constexpr int kUS = kG > kKS ? kG / kKS : 1;            // stages per stream-K unit
+    static constexpr int kUnitK = kUS * kKS;                       // rows of K per unit
+    static constexpr int kScaleGroups = kKS >= kG ? kKS / kG : 1;  // groups in a stage's scale box
+    static constexpr int kCodeTile = kChunks * 1024 * P;           // code bytes of a tile per stage
+    static constexpr int kCode = kWarps * kCodeTile;
+    static constexpr int kXBox = 128 * 8 * TT;                     // 64 k x 8TT rows of bf16
+    static constexpr int kX = kChunks * kXBox;
+    static constexpr int kScaleTile = 64 * kScaleGroups;
+    static constexpr int kScale = kWarps * kScaleTile;
+    static constexpr int kTx = kX + kCode + kScale;                // bytes landing per stage
+    static constexpr int kStage = (kTx + 1023) / 1024 * 1024;      // X boxes stay 1024-aligned
+    static constexpr int kStages = kRingBytes / kStage > 3 ? kRingBytes / kStage : 3;
+    static constexpr int kF = 2 * TT;                              // float4 per lane fragment
+    // fragments the second warp of a tile hands to the first at a segment end
+    static constexpr int kXchgOff = kStages * kStage;
+    static constexpr int kXchg = kWPT == 2 ? kWarps * kF * 32 * 16 : 0;
+    static constexpr int kBarOff = kXchgOff + kXchg;
+    static constexpr size_t kSmem = (size_t)kBarOff + 2 * kStages * 8 + 1024;  // + alignment
 };
 
 struct Params {
-    const uint16_t *X;       // bf16 [M][K]
-    const uint8_t *codes;    // re-packed codes  [N/32][K/64][2][32][16 B]
-    const uint8_t *scales;   // re-packed scales [N/32][K/G][8][4 halves]
     uint16_t *Y;             // bf16 [M][N]
     WsHeader *hdr;
-    int *counters;           // [N/32]
-    float4 *partial;         // [ctas][2*TT][32]: a CTA's fragment of its first, cut tile
-    int M, N, K;
-    int upt;                 // units per n32 tile
-    int units;
-    int ctas;
+    int *counters;           // [column groups * 8]
+    float4 *partial;         // [ctas][8 warps][2*TT][32]: a CTA's fragments of its first, cut group row
+    int M, N;
+    int ntiles;              // N / 32
+    int upr;                 // units per group row
     int q, r;                // units = q * ctas + r: CTAs below r run q + 1 units, the rest q
     int early;               // load the first weights before waiting for the previous kernel
+    int pf_stages;           // stages after the ring warmed in L2 at entry
 };
 
-// First unit of CTA c's run.
 __device__ __forceinline__ int run_start(const Params &p, int c)
 {
     return c * p.q + min(c, p.r);
@@ -147,37 +160,106 @@ __device__ __forceinline__ void store_y4(const Params &p, int tile, int j, int l
     }
 }
 
-// Run by warp 0 of a CTA whose segment of `tile` is cut (the tile goes on
-// in other CTAs' runs), with the CTA's warp fragments in `frags`.  The CTA
-// whose run holds the tile's first unit finishes that segment last in its
+// ------------------------------------------------------------------ producer
+template <int TT, int GM, int P>
+__device__ __forceinline__ void produce(const Params &p, const CUtensorMap *cmap,
+                                        const CUtensorMap *smap, const CUtensorMap *xmap,
+                                        uint8_t *ring, uint64_t *full, uint64_t *empty, int S0,
+                                        int ns)
+{
+    using C = Cfg<TT, GM, P>;
+    constexpr int R = C::kStages;
+    const int spr = p.upr * C::kUS;   // stages per group row
+    const uint64_t pol_w = l2_policy_evict_first();
+    const uint64_t pol_x = l2_policy_evict_last();
+    prefetch_tensormap(cmap);
+    prefetch_tensormap(smap);
+    prefetch_tensormap(xmap);
+    // box coordinates of run stage s: codes x (u64), group row y (tiles), first k
+    auto coords = [&](int s, int &cx, int &sx, int &ty, int &k0) {
+        const int a = S0 + s;
+        const int gr = a / spr, ks = a - gr * spr;
+        k0 = ks * C::kKS;
+        cx = ks * (C::kCodeTile / 8);
+        sx = (k0 / C::kG) * 8;
+        ty = gr * kWarps;
+    };
+    auto issue_w = [&](int s) {
+        int cx, sx, ty, k0;
+        coords(s, cx, sx, ty, k0);
+        uint8_t *st = ring + (size_t)(s % R) * C::kStage;
+        uint64_t *bar = &full[s % R];
+        mbar_arrive_expect_tx(bar, C::kTx);
+        tma_load_2d(st + C::kX, cmap, cx, ty, bar, pol_w);
+        tma_load_2d(st + C::kX + C::kCode, smap, sx, ty, bar, pol_w);
+    };
+    auto issue_x = [&](int s) {
+        int cx, sx, ty, k0;
+        coords(s, cx, sx, ty, k0);
+        uint8_t *st = ring + (size_t)(s % R) * C::kStage;
+#pragma unroll
+        for (int ch = 0; ch < C::kChunks; ++ch)
+            tma_load_2d(st + ch * C::kXBox, xmap, k0 + 64 * ch, 0, &full[s % R], pol_x);
+    };
+    const int first = min(R, ns);
+    // Weights are not written by the previous kernel on the stream (the
+    // caller's contract, unless early loads are off): the first stages fill,
+    // and the stages after them are pulled into L2, while that kernel drains.
+    if (p.early)
+        for (int s = 0; s < first; ++s)
+            issue_w(s);
+    const int pf_end = min(ns, R + p.pf_stages);
+    for (int s = R; s < pf_end; ++s) {
+        int cx, sx, ty, k0;
+        coords(s, cx, sx, ty, k0);
+        prefetch_tensor_l2(cmap, cx, ty);
+        prefetch_tensor_l2(smap, sx, ty);
+    }
+    pdl_wait();
+    if (!p.early)
+        for (int s = 0; s < first; ++s)
+            issue_w(s);
+    for (int s = 0; s < first; ++s)
+        issue_x(s);
+    int issued = first;
+    for (int s = first; s < ns; ++s) {
+        // stage s reuses the slot of stage s - R: its release is phase
+        // (s / R - 1) of that slot's empty barrier
+        if (!mbar_wait(&empty[s % R], (uint32_t)((s / R - 1) & 1), kWaitLimitNs)) {
+            record_error(p.hdr, MXG_ERR_TIMEOUT, 140 + GM);
+            break;
+        }
+        issue_w(s);
+        issue_x(s);
+        issued = s + 1;
+    }
+    // every copy this CTA issued has landed before it exits (the consumers
+    // wait for them too; this only matters after a timeout)
+    for (int s = max(0, issued - R); s < issued; ++s)
+        if (!mbar_wait(&full[s % R], (uint32_t)((s / R) & 1), kWaitLimitNs))
+            record_error(p.hdr, MXG_ERR_TIMEOUT, 150 + GM);
+}
+
+// ----------------------------------------------------------------- finisher
+// Run by warp `warp` of a CTA whose segment of group row `gr` is cut (the
+// row goes on in other CTAs' runs), with the warp's fragment in `sum`.  The
+// CTA whose run holds the row's first unit finishes that segment last in its
 // run: it adds the other contributors' fragments (in CTA order) to its own
 // and writes bf16 Y.  Every other contributor (its segment is the first one
 // of its run) publishes its fragment and bumps the tile's counter without
 // waiting for anybody.
 template <int TT>
-__device__ __noinline__ void finish_cut_tile(const Params &p, const float4 *frags, int c, int tile,
-                                             int lane)
+__device__ __forceinline__ void finish_cut(const Params &p, float4 (&sum)[2 * TT], int c, int gr,
+                                        int warp, int lane)
 {
     constexpr int F = 2 * TT;
-    constexpr int kFrag4 = F * 32;
-    float4 sum[F];
-#pragma unroll
-    for (int j = 0; j < F; ++j) {
-        sum[j] = frags[j * 32 + lane];
-        for (int w = 1; w < kConsumers; ++w) {
-            const float4 v = frags[w * kFrag4 + j * 32 + lane];
-            sum[j].x += v.x;
-            sum[j].y += v.y;
-            sum[j].z += v.z;
-            sum[j].w += v.w;
-        }
-    }
-    const int tile_begin = tile * p.upt;
-    const int c_first = cta_of_unit(p, tile_begin);
+    const int tile = gr * kWarps + warp;
+    const int c_first = cta_of_unit(p, gr * p.upr);
+    float4 *mine = p.partial + ((size_t)c * kWarps + warp) * F * 32;
     if (c != c_first) {
 #pragma unroll
         for (int j = 0; j < F; ++j)
-            __stcg(p.partial + ((size_t)c * F + j) * 32 + lane, sum[j]);
+            __stcg(mine + j * 32 + lane, sum[j]);
         __syncwarp();
         if (lane == 0) {
             __threadfence();
@@ -185,10 +267,8 @@ __device__ __noinline__ void finish_cut_tile(const Params &p, const float4 *frag
         }
         return;
     }
-    const int c_last = cta_of_unit(p, tile_begin + p.upt - 1);
+    const int c_last = cta_of_unit(p, (gr + 1) * p.upr - 1);
     if (lane == 0) {
-        // the other contributors published early in their runs (or at their
-        // ends, for runs inside the tile); the wait is bounded
         const unsigned long long t0 = global_ns();
         while (ld_acquire_gpu(&p.counters[tile]) < c_last - c_first) {
             if (global_ns() - t0 > kWaitLimitNs) {
@@ -200,9 +280,10 @@ __device__ __noinline__ void finish_cut_tile(const Params &p, const float4 *frag
     }
     __syncwarp();
     for (int cc = c_first + 1; cc <= c_last; ++cc) {
+        const float4 *src = p.partial + ((size_t)cc * kWarps + warp) * F * 32;
 #pragma unroll
         for (int j = 0; j < F; ++j) {
-            const float4 f = __ldcg(p.partial + ((size_t)cc * F + j) * 32 + lane);
+            const float4 f = __ldcg(src + j * 32 + lane);
             sum[j].x += f.x;
             sum[j].y += f.y;
             sum[j].z += f.z;
@@ -212,385 +293,296 @@ __device__ __noinline__ void finish_cut_tile(const Params &p, const float4 *frag
 #pragma unroll
     for (int j = 0; j < F; ++j)
         store_y4<TT>(p, tile, j, lane, sum[j]);
+    __syncwarp();
     if (lane == 0)
         p.counters[tile] = 0;  // leave the counter zero for the next call
 }
 
-template <int TT>
-__device__ __forceinline__ void zero_acc(float (&a)[2][TT][4])
+// ------------------------------------------------------------------- kernel
+template <int TT, int GM, int P>
+__global__ void __launch_bounds__(Cfg<TT, GM, P>::kThreads,
+                                  Cfg<TT, GM, P>::kWPT == 1 && TT <= 2 ? 2 : 1)
+    w4a16_stream_kernel(const __grid_constant__ CUtensorMap cmap,
+                        const __grid_constant__ CUtensorMap smap,
+                        const __grid_constant__ CUtensorMap xmap, const Params p)
 {
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int tt = 0; tt < TT; ++tt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                a[h][tt][e] = 0.f;
-}
-
-// Copies unit u (codes, then scales) into a ring slot; completion on `bar`.
-template <int GM, int SU, int P>
-__device__ __forceinline__ void fetch_unit(const Params &p, uint8_t *slot, uint64_t *bar, int u,
-                                           uint64_t policy)
-{
-    using MD = Mode<GM, SU, P>;
-    mbar_arrive_expect_tx(bar, MD::kCode + MD::kScale);
-    bulk_g2s(slot, p.codes + (size_t)u * MD::kCode, MD::kCode, bar, policy);
-    bulk_g2s(slot + MD::kCode, p.scales + (size_t)u * MD::kScale, MD::kScale, bar, policy);
-}
-
-template <int TT, int GM, int SU, int P>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm) w4a16_stream_kernel(const Params p)
-{
-    using MD = Mode<GM, SU, P>;
-    using SL = Smem<TT, GM, SU, P>;
-    constexpr int kStages = MD::kStages;
-    constexpr int F = 2 * TT;  // float4 per lane fragment
-    extern __shared__ __align__(128) uint8_t smem[];
-    float4 *red = reinterpret_cast<float4 *>(smem + SL::kRedOff);
+    using C = Cfg<TT, GM, P>;
+    constexpr int R = C::kStages;
+    constexpr int F = C::kF;
+    extern __shared__ uint8_t smem_raw[];
+    // 1024-byte alignment for the swizzled activation boxes
+    uint8_t *ring = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    uint64_t *full = reinterpret_cast<uint64_t *>(ring + C::kBarOff);
+    uint64_t *empty = full + R;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_launch_dependents();
     const int c = blockIdx.x;
     const int U0 = run_start(p, c), U1 = run_start(p, c + 1);
-    const int n = U1 - U0;
-    uint8_t *ring = smem + (size_t)warp * kStages * SL::kSlot;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + SL::kBarOff) + warp * kStages;
-    uint64_t policy = 0;
-    if (lane == 0) {
-        for (int s = 0; s < kStages; ++s)
-            mbar_init(&full[s], 1);
-        fence_barrier_init();
-        policy = l2_policy_evict_first();
-    }
-    int *red_count = reinterpret_cast<int *>(smem + SL::kSyncOff);  // arrivals per buffer
-    int *red_done = red_count + SL::kRed;                           // reductions per buffer
+    const int S0 = U0 * C::kUS;
+    const int ns = (U1 - U0) * C::kUS;
     if (threadIdx.x == 0) {
-        for (int b = 0; b < 2 * SL::kRed; ++b)
-            red_count[b] = 0;
-        // while the previous kernel drains: pull the first units into L2
-        const int nu = min(kConsumers * kStages, n);
-        prefetch_l2(p.codes + (size_t)U0 * MD::kCode, nu * MD::kCode);
-        prefetch_l2(p.scales + (size_t)U0 * MD::kScale, nu * MD::kScale);
+        for (int s = 0; s < R; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kWarps);   // one warp of each tile takes a stage
+        }
+        fence_barrier_init();
     }
     __syncthreads();
-    // this warp takes units warp, warp + C, ... of the run; its k-th unit
-    // goes to slot k mod kStages.  The weights are not written by the
-    // previous kernel on the stream (the caller's contract, unless it turned
-    // early weight loads off): the first slots fill while that kernel drains.
-    auto fill_ring = [&]() {
+    if (warp == C::kProducer) {
         if (lane == 0)
-            for (int k = 0; k < kStages && warp + k * kConsumers < n; ++k)
-                fetch_unit<GM, SU, P>(p, ring + k * SL::kSlot, &full[k], U0 + warp + k * kConsumers,
-                                   policy);
-    };
-    if (p.early)
-        fill_ring();
-    pdl_wait();
-    if (!p.early)
-        fill_ring();
+            produce<TT, GM, P>(p, &cmap, &smap, &xmap, ring, full, empty, S0, ns);
+        return;
+    }
 
     // ------------------------------------------------------------ consumers
+    pdl_wait();   // Y, the counters and the partials may be in use before it
     const int g = lane >> 2, t = lane & 3;
-    // activation rows of this lane: m = g + 8 tt; the lane reads k = 4t .. 4t+3
-    // of every k16 step
-    // (rows m >= M read row 0 instead: their outputs are never stored)
-    const uint16_t *xrow[TT];
+    const int wt = warp % kWarps;        // this warp's tile in the column group
+    const int parity = warp / kWarps;    // which stages of the run it takes
+    // swizzled offsets of this lane's activations inside a 64-k box: row
+    // 8 tt + g, bytes 32 j + 8 t of the row; the 16-byte chunk index is
+    // XORed with the row modulo 8 by the 128-byte swizzle
+    uint32_t xoff[4];
 #pragma unroll
-    for (int tt = 0; tt < TT; ++tt) {
-        const int m = tt * 8 + g;
-        xrow[tt] = p.X + (size_t)(m < p.M ? m : 0) * p.K + 4 * t;
-    }
-    const int upt = p.upt;
-
-    // Activation fragments of one unit, requested one unit ahead for narrow
-    // token tiles (a whole unit of work hides their L2 latency).
-    constexpr bool kPipeX = MD::kChunks * TT <= 4;
-    uint2 xs[MD::kChunks][TT][4], xn[MD::kChunks][TT][4];
-    // ku: the unit's place in its tile
-    auto load_x = [&](uint2 (&dst)[MD::kChunks][TT][4], int ku) {
-        const int kc = ku * MD::kChunks;  // first k64 chunk of the unit
-#pragma unroll
-        for (int ch = 0; ch < MD::kChunks; ++ch)
-#pragma unroll
-            for (int tt = 0; tt < TT; ++tt)
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    dst[ch][tt][j] = __ldg(
-                        reinterpret_cast<const uint2 *>(xrow[tt] + (kc + ch) * 64 + 16 * j));
-    };
-    // place in its tile of the unit kConsumers further on
-    auto next_ku = [&](int ku) {
-        ku += kConsumers;
-        while (ku >= upt)
-            ku -= upt;
-        return ku;
-    };
+    for (int j = 0; j < 4; ++j)
+        xoff[j] = g * 128 + (((2 * j + (t >> 1)) ^ g) << 4) + 8 * (t & 1);
 
     constexpr uint32_t kOnes = 0x3F803F80u;  // bf16 pair (1, 1)
     float acc[2][TT][4], part[2][TT][4], xsum[TT][4];
     float parthi[P == 2 ? 2 : 1][TT][4];  // INT8: sums over the high-nibble plane
     bool ok = true;
-    int i = warp;          // run index of this warp's next unit
-    int slot = 0;          // ring slot of unit i
-    uint32_t phase = 0;    // parity of the phase of unit i
-    int ku = (U0 + i) % upt;  // place of unit i in its tile
-    if (kPipeX && i < n)
-        load_x(xs, ku);
-    int sidx = 0;          // segment of the run
-    int tile = U0 / upt;
-    for (int seg = U0; seg < U1; ++tile) {
-        const int tile_begin = tile * upt;
-        const int seg_end = min(U1, tile_begin + upt);
-        zero_acc<TT>(acc);
-        for (; U0 + i < seg_end; i += kConsumers) {
-            const int u = U0 + i;
-            const int ku_next = next_ku(ku);
-            if (kPipeX) {
-                if (i + kConsumers < n)
-                    load_x(xn, ku_next);
-            } else {
-                load_x(xs, ku);
-            }
-            ku = ku_next;
-            if (!mbar_wait(&full[slot], phase, ok ? kWaitLimitNs : 0)) {
-                if (ok && lane == 0)
-                    record_error(p.hdr, MXG_ERR_TIMEOUT, 100 + GM);
-                ok = false;
-            }
-            const uint8_t *st = ring + slot * SL::kSlot;
-            const uint8_t *ss = st + MD::kCode;
-#pragma unroll
-            for (int ch = 0; ch < MD::kChunks; ++ch) {
-                // INT4: [half][lane][16 B]; INT8: [half][plane][lane][16 B]
-                const uint8_t *cp = st + ch * 1024 * P + lane * 16;
-                const uint4 wl = lds128(cp);
-                const uint4 wh = lds128(cp + 512 * P);
-                const uint32_t w[2][4] = {{wl.x, wl.y, wl.z, wl.w}, {wh.x, wh.y, wh.z, wh.w}};
-                uint32_t whi[2][4] = {};
-                if constexpr (P == 2) {
-                    const uint4 ul = lds128(cp + 512);
-                    const uint4 uh = lds128(cp + 1536);
-                    whi[0][0] = ul.x; whi[0][1] = ul.y; whi[0][2] = ul.z; whi[0][3] = ul.w;
-                    whi[1][0] = uh.x; whi[1][1] = uh.y; whi[1][2] = uh.z; whi[1][3] = uh.w;
-                }
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int step = ch * 4 + j;  // k16 step inside the unit
-                    const bool first = (step % MD::kStepsPerGroup) == 0;
-#pragma unroll
-                    for (int tt = 0; tt < TT; ++tt) {
-                        // per token: the sum of the step's activations (an MMA
-                        // with an all-ones weight tile)
-                        if (first)
-                            mma_bf16_16816_zero(xsum[tt], kOnes, kOnes, kOnes, kOnes,
-                                                xs[ch][tt][j].x, xs[ch][tt][j].y);
-                        else
-                            mma_bf16_16816(xsum[tt], kOnes, kOnes, kOnes, kOnes,
-                                           xs[ch][tt][j].x, xs[ch][tt][j].y);
-                    }
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const uint32_t a0 = int4_pair_plus128<0>(w[h][j]);
-                        const uint32_t a1 = int4_pair_plus128<4>(w[h][j]);
-                        const uint32_t a2 = int4_pair_plus128<8>(w[h][j]);
-                        const uint32_t a3 = int4_pair_plus128<12>(w[h][j]);
-#pragma unroll
-                        for (int tt = 0; tt < TT; ++tt) {
-                            if (first)
-                                mma_bf16_16816_zero(part[h][tt], a0, a1, a2, a3,
-                                                    xs[ch][tt][j].x, xs[ch][tt][j].y);
-                            else
-                                mma_bf16_16816(part[h][tt], a0, a1, a2, a3, xs[ch][tt][j].x,
-                                               xs[ch][tt][j].y);
-                        }
-                        if constexpr (P == 2) {
-                            const uint32_t b0 = int4_pair_plus128<0>(whi[h][j]);
-                            const uint32_t b1 = int4_pair_plus128<4>(whi[h][j]);
-                            const uint32_t b2 = int4_pair_plus128<8>(whi[h][j]);
-                            const uint32_t b3 = int4_pair_plus128<12>(whi[h][j]);
-#pragma unroll
-                            for (int tt = 0; tt < TT; ++tt) {
-                                if (first)
-                                    mma_bf16_16816_zero(parthi[h][tt], b0, b1, b2, b3,
-                                                        xs[ch][tt][j].x, xs[ch][tt][j].y);
-                                else
-                                    mma_bf16_16816(parthi[h][tt], b0, b1, b2, b3,
-                                                   xs[ch][tt][j].x, xs[ch][tt][j].y);
-                            }
-                        }
-                    }
-                    if ((step + 1) % MD::kStepsPerGroup == 0) {
-                        // end of a scale group: the MMAs summed (128 + q) * x, so
-                        // acc += (part - 136 * sum(x)) * scale, in fp32
-                        const int gi = step / MD::kStepsPerGroup;  // group inside the unit
-                        const uint2 sv = lds64(ss + gi * 64 + g * 8);
-                        const float2 s01 = __half22float2(*reinterpret_cast<const __half2 *>(&sv.x));
-                        const float2 s23 = __half22float2(*reinterpret_cast<const __half2 *>(&sv.y));
-                        const float sc[2][2] = {{s01.x, s01.y}, {s23.x, s23.y}};
-#pragma unroll
-                        for (int h = 0; h < 2; ++h)
-#pragma unroll
-                            for (int tt = 0; tt < TT; ++tt)
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    // outputs e and e ^ 2 are rows g, g + 8 of token 2t + (e & 1)
-                                    float v;
-                                    if constexpr (P == 2) {
-                                        // INT8 q = 16 hi + lo: the planes summed
-                                        // (128 + hi) x and (128 + lo) x, so
-                                        // sum (q - 128) x = 16 Phi + Plo - 2304 sum(x)
-                                        v = fmaf(16.f, parthi[h][tt][e], part[h][tt][e]);
-                                        v = fmaf(-2304.f, xsum[tt][e & 1], v);
-                                    } else {
-                                        v = fmaf(-136.f, xsum[tt][e & 1], part[h][tt][e]);
-                                    }
-                                    acc[h][tt][e] = fmaf(v, sc[h][e >> 1], acc[h][tt][e]);
-                                }
-                    }
-                }
-            }
-            // every lane's reads of the slot have returned (their values are
-            // consumed above): refill it with this warp's unit kStages ahead
-            __syncwarp();
-            if (lane == 0 && i + kStages * kConsumers < n)
-                fetch_unit<GM, SU, P>(p, ring + slot * SL::kSlot, &full[slot],
-                               u + kStages * kConsumers, policy);
-            if (kPipeX) {
-#pragma unroll
-                for (int ch = 0; ch < MD::kChunks; ++ch)
-#pragma unroll
-                    for (int tt = 0; tt < TT; ++tt)
-#pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            xs[ch][tt][j] = xn[ch][tt][j];
-            }
-            if (++slot == kStages) {
-                slot = 0;
-                phase ^= 1;
-            }
-        }
-
-        // ---- end of the tile segment.  Every warp leaves its fragment in the
-        // segment's reduction buffer and goes on; the last warp to arrive adds
-        // the fragments.  A buffer is reused kRed segments later, once the
-        // reduction of its previous segment is done.
-        const int rb = sidx % SL::kRed;
-        const int uses = sidx / SL::kRed;  // earlier segments that used buffer rb
-        if (uses > 0) {
-            if (lane == 0) {
-                const unsigned long long t0 = global_ns();
-                while (*reinterpret_cast<volatile int *>(&red_done[rb]) < uses) {
-                    if (global_ns() - t0 > kWaitLimitNs) {
-                        record_error(p.hdr, MXG_ERR_TIMEOUT, 130);
-                        break;
-                    }
-                    __nanosleep(32);
-                }
-                __threadfence_block();
-            }
-            __syncwarp();
-        }
-        float4 *frags = red + (size_t)rb * kConsumers * SL::kFrag4;
+    int s = 0;   // run stage
+    for (int u = U0; u < U1;) {
+        const int gr = u / p.upr;
+        const int seg_begin = u;
+        const int seg_end = min(U1, (gr + 1) * p.upr);
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
             for (int tt = 0; tt < TT; ++tt)
-                frags[(size_t)warp * SL::kFrag4 + (h * TT + tt) * 32 + lane] =
-                    make_float4(acc[h][tt][0], acc[h][tt][1], acc[h][tt][2], acc[h][tt][3]);
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) {
-            __threadfence_block();
-            last = atomicAdd(&red_count[rb], 1) == kConsumers - 1;
-            __threadfence_block();
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    acc[h][tt][e] = 0.f;
+        for (; u < seg_end; ++u) {
+#pragma unroll
+            for (int su = 0; su < C::kUS; ++su, ++s) {
+                if (C::kWPT == 2 && (s & 1) != parity)
+                    continue;   // the other warp of the tile takes this stage
+                const int slot = s % R;
+                if (!mbar_wait(&full[slot], (uint32_t)((s / R) & 1), ok ? kWaitLimitNs : 0)) {
+                    if (ok && lane == 0)
+                        record_error(p.hdr, MXG_ERR_TIMEOUT, 100 + GM);
+                    ok = false;
+                }
+                const uint8_t *st = ring + (size_t)slot * C::kStage;
+                const uint8_t *cs = st + C::kX + wt * C::kCodeTile;
+                const uint8_t *ss = st + C::kX + C::kCode + wt * C::kScaleTile;
+#pragma unroll
+                for (int ch = 0; ch < C::kChunks; ++ch) {
+                    // INT4: [half][lane][16 B]; INT8: [half][plane][lane][16 B]
+                    const uint8_t *cp = cs + ch * 1024 * P + lane * 16;
+                    const uint4 wl = lds128(cp);
+                    const uint4 wh = lds128(cp + 512 * P);
+                    const uint32_t w[2][4] = {{wl.x, wl.y, wl.z, wl.w}, {wh.x, wh.y, wh.z, wh.w}};
+                    uint32_t whi[2][4] = {};
+                    if constexpr (P == 2) {
+                        const uint4 ul = lds128(cp + 512);
+                        const uint4 uh = lds128(cp + 1536);
+                        whi[0][0] = ul.x; whi[0][1] = ul.y; whi[0][2] = ul.z; whi[0][3] = ul.w;
+                        whi[1][0] = uh.x; whi[1][1] = uh.y; whi[1][2] = uh.z; whi[1][3] = uh.w;
+                    }
+                    const uint8_t *xb = st + ch * C::kXBox;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        // k16 step inside the unit (one warp) or the stage (two)
+                        const int gstep = (C::kWPT == 1 ? su * C::kSteps : 0) + ch * 4 + j;
+                        const bool first = (gstep % C::kEpi) == 0;
+                        const bool last = ((gstep + 1) % C::kEpi) == 0;
+                        uint2 xf[TT];
+#pragma unroll
+                        for (int tt = 0; tt < TT; ++tt)
+                            xf[tt] = lds64(xb + tt * 1024 + xoff[j]);
+#pragma unroll
+                        for (int tt = 0; tt < TT; ++tt) {
+                            // per token: the sum of the step's activations (an
+                            // MMA with an all-ones weight tile)
+                            if (first)
+                                mma_bf16_16816_zero(xsum[tt], kOnes, kOnes, kOnes, kOnes, xf[tt].x,
+                                                    xf[tt].y);
+                            else
+                                mma_bf16_16816(xsum[tt], kOnes, kOnes, kOnes, kOnes, xf[tt].x,
+                                               xf[tt].y);
+                        }
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint32_t a0 = int4_pair_plus128<0>(w[h][j]);
+                            const uint32_t a1 = int4_pair_plus128<4>(w[h][j]);
+                            const uint32_t a2 = int4_pair_plus128<8>(w[h][j]);
+                            const uint32_t a3 = int4_pair_plus128<12>(w[h][j]);
+#pragma unroll
+                            for (int tt = 0; tt < TT; ++tt) {
+                                if (first)
+                                    mma_bf16_16816_zero(part[h][tt], a0, a1, a2, a3, xf[tt].x,
+                                                        xf[tt].y);
+                                else
+                                    mma_bf16_16816(part[h][tt], a0, a1, a2, a3, xf[tt].x,
+                                                   xf[tt].y);
+                            }
+                            if constexpr (P == 2) {
+                                const uint32_t b0 = int4_pair_plus128<0>(whi[h][j]);
+                                const uint32_t b1 = int4_pair_plus128<4>(whi[h][j]);
+                                const uint32_t b2 = int4_pair_plus128<8>(whi[h][j]);
+                                const uint32_t b3 = int4_pair_plus128<12>(whi[h][j]);
+#pragma unroll
+                                for (int tt = 0; tt < TT; ++tt) {
+                                    if (first)
+                                        mma_bf16_16816_zero(parthi[h][tt], b0, b1, b2, b3,
+                                                            xf[tt].x, xf[tt].y);
+                                    else
+                                        mma_bf16_16816(parthi[h][tt], b0, b1, b2, b3, xf[tt].x,
+                                                       xf[tt].y);
+                                }
+                            }
+                        }
+                        if (last) {
+                            // end of a scale group: the MMAs summed (128 + q) * x,
+                            // so acc += (part - 136 * sum(x)) * scale, in fp32
+                            const int gi = C::kScaleGroups > 1 ? (ch * 4 + j) / C::kStepsPerGroup
+                                                               : 0;
+                            const uint2 sv = lds64(ss + gi * 64 + g * 8);
+                            const float2 s01 =
+                                __half22float2(*reinterpret_cast<const __half2 *>(&sv.x));
+                            const float2 s23 =
+                                __half22float2(*reinterpret_cast<const __half2 *>(&sv.y));
+                            const float sc[2][2] = {{s01.x, s01.y}, {s23.x, s23.y}};
+#pragma unroll
+                            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                                for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e) {
+                                        // outputs e and e ^ 2 are rows g, g + 8 of
+                                        // token 2t + (e & 1)
+                                        float v;
+                                        if constexpr (P == 2) {
+                                            // INT8 q = 16 hi + lo: the planes summed
+                                            // (128 + hi) x and (128 + lo) x, so
+                                            // sum (q - 128) x = 16 Phi + Plo - 2304 sum(x)
+                                            v = fmaf(16.f, parthi[h][tt][e], part[h][tt][e]);
+                                            v = fmaf(-2304.f, xsum[tt][e & 1], v);
+                                        } else {
+                                            v = fmaf(-136.f, xsum[tt][e & 1], part[h][tt][e]);
+                                        }
+                                        acc[h][tt][e] = fmaf(v, sc[h][e >> 1], acc[h][tt][e]);
+                                    }
+                        }
+                    }
+                }
+                // every lane's reads of the stage have returned (their values
+                // are consumed above): release it to the producer
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&empty[slot]);
+            }
         }
-        if (__shfl_sync(0xffffffffu, last, 0)) {
-            if (lane == 0)
-                red_count[rb] = 0;
-            const bool whole = seg == tile_begin && seg_end == tile_begin + upt;
-            if (whole) {
+
+        // ---- end of the segment: this warp's tile of group row gr
+        float4 sum[F];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int tt = 0; tt < TT; ++tt)
+                sum[h * TT + tt] =
+                    make_float4(acc[h][tt][0], acc[h][tt][1], acc[h][tt][2], acc[h][tt][3]);
+        if constexpr (C::kWPT == 2) {
+            // the tile's second warp hands its fragment to the first (a named
+            // barrier per tile: ids 1..8, the tile's two warps)
+            float4 *xch = reinterpret_cast<float4 *>(ring + C::kXchgOff) + wt * F * 32;
+            if (parity == 1)
+#pragma unroll
+                for (int j = 0; j < F; ++j)
+                    xch[j * 32 + lane] = sum[j];
+            named_bar_sync(1 + wt, 64);
+            if (parity == 0)
 #pragma unroll
                 for (int j = 0; j < F; ++j) {
-                    float4 s = frags[j * 32 + lane];
-#pragma unroll
-                    for (int w = 1; w < kConsumers; ++w) {
-                        const float4 v = frags[(size_t)w * SL::kFrag4 + j * 32 + lane];
-                        s.x += v.x;
-                        s.y += v.y;
-                        s.z += v.z;
-                        s.w += v.w;
-                    }
-                    store_y4<TT>(p, tile, j, lane, s);
+                    const float4 v = xch[j * 32 + lane];
+                    sum[j].x += v.x;
+                    sum[j].y += v.y;
+                    sum[j].z += v.z;
+                    sum[j].w += v.w;
                 }
+            named_bar_sync(1 + wt, 64);   // read before the next segment's write
+            if (parity == 1)
+                continue;
+        }
+        const int tile = gr * kWarps + wt;
+        if (tile < p.ntiles) {
+            const bool whole = seg_begin == gr * p.upr && seg_end == (gr + 1) * p.upr;
+            if (whole) {
+#pragma unroll
+                for (int j = 0; j < F; ++j)
+                    store_y4<TT>(p, tile, j, lane, sum[j]);
             } else {
-                finish_cut_tile<TT>(p, frags, c, tile, lane);
-            }
-            __syncwarp();
-            if (lane == 0) {
-                __threadfence_block();
-                atomicAdd(&red_done[rb], 1);
+                finish_cut<TT>(p, sum, c, gr, wt, lane);
             }
         }
-        ++sidx;
-        seg = seg_end;
     }
 }
 
-template <int TT, int GM, int SU, int P = 1>
+template <int TT, int GM, int P>
 const void *kernel_ptr()
 {
-    return reinterpret_cast<const void *>(&w4a16_stream_kernel<TT, GM, SU, P>);
+    return reinterpret_cast<const void *>(&w4a16_stream_kernel<TT, GM, P>);
 }
 
-// SU = 2 (two scale-group spans per unit) for up to two token tiles,
-// SU = 1 otherwise; variant = gm + 3 * (SU - 1).
+// variant = group mode (INT4) or 3 + group mode (INT8)
 const void *select_kernel(int tt, int variant)
 {
-#define MXG_CASE(T, G_, S_) \
-    if (tt == T && variant == G_ + 3 * (S_ - 1)) return kernel_ptr<T, G_, S_>();
-    MXG_CASE(1, 0, 1) MXG_CASE(1, 1, 1) MXG_CASE(1, 2, 1)
-    MXG_CASE(2, 0, 1) MXG_CASE(2, 1, 1) MXG_CASE(2, 2, 1)
-    MXG_CASE(3, 0, 1) MXG_CASE(3, 1, 1) MXG_CASE(3, 2, 1)
-    MXG_CASE(4, 0, 1) MXG_CASE(4, 1, 1) MXG_CASE(4, 2, 1)
-    MXG_CASE(1, 0, 2) MXG_CASE(1, 1, 2) MXG_CASE(1, 2, 2)
-    MXG_CASE(2, 0, 2) MXG_CASE(2, 1, 2) MXG_CASE(2, 2, 2)
+#define MXG_CASE(T, V) \
+    if (tt == T && variant == V) return kernel_ptr<T, V % 3, V / 3 + 1>();
+    MXG_CASE(1, 0) MXG_CASE(1, 1) MXG_CASE(1, 2) MXG_CASE(1, 3) MXG_CASE(1, 4) MXG_CASE(1, 5)
+    MXG_CASE(2, 0) MXG_CASE(2, 1) MXG_CASE(2, 2) MXG_CASE(2, 3) MXG_CASE(2, 4) MXG_CASE(2, 5)
+    MXG_CASE(3, 0) MXG_CASE(3, 1) MXG_CASE(3, 2) MXG_CASE(3, 3) MXG_CASE(3, 4) MXG_CASE(3, 5)
+    MXG_CASE(4, 0) MXG_CASE(4, 1) MXG_CASE(4, 2) MXG_CASE(4, 3) MXG_CASE(4, 4) MXG_CASE(4, 5)
 #undef MXG_CASE
-    // INT8 (two code planes), SU = 1: variant = 6 + gm
-#define MXG_CASE8(T, G_) \
-    if (tt == T && variant == 6 + G_) return kernel_ptr<T, G_, 1, 2>();
-    MXG_CASE8(1, 0) MXG_CASE8(1, 1) MXG_CASE8(1, 2)
-    MXG_CASE8(2, 0) MXG_CASE8(2, 1) MXG_CASE8(2, 2)
-    MXG_CASE8(3, 0) MXG_CASE8(3, 1) MXG_CASE8(3, 2)
-    MXG_CASE8(4, 0) MXG_CASE8(4, 1) MXG_CASE8(4, 2)
-#undef MXG_CASE8
     return nullptr;
 }
 
-template <int GM, int SU, int P = 1>
-size_t smem_bytes_gs(int tt)
+template <int TT>
+void cfg_of(int variant, size_t *smem, int *us, int *ks, int *code_tile, int *g, int *threads)
 {
-    switch (tt) {
-    case 1: return Smem<1, GM, SU, P>::kTotal;
-    case 2: return Smem<2, GM, SU, P>::kTotal;
-    case 3: return Smem<3, GM, 1, P>::kTotal;
-    default: return Smem<4, GM, 1, P>::kTotal;
+#define MXG_CFG(V)                                         \
+    if (variant == V) {                                    \
+        using C = Cfg<TT, V % 3, V / 3 + 1>;               \
+        *smem = C::kSmem;                                  \
+        *us = C::kUS;                                      \
+        *ks = C::kKS;                                      \
+        *code_tile = C::kCodeTile;                         \
+        *g = C::kG;                                        \
+        *threads = C::kThreads;                            \
+        return;                                            \
     }
+    MXG_CFG(0) MXG_CFG(1) MXG_CFG(2) MXG_CFG(3) MXG_CFG(4) MXG_CFG(5)
+#undef MXG_CFG
 }
 
-size_t smem_bytes(int tt, int variant)
+struct VariantCfg {
+    size_t smem;
+    int us, ks, code_tile, g, threads;
+};
+
+VariantCfg variant_cfg(int tt, int variant)
 {
-    switch (variant) {
-    case 0: return smem_bytes_gs<0, 1>(tt);
-    case 1: return smem_bytes_gs<1, 1>(tt);
-    case 2: return smem_bytes_gs<2, 1>(tt);
-    case 3: return smem_bytes_gs<0, 2>(tt);
-    case 4: return smem_bytes_gs<1, 2>(tt);
-    case 5: return smem_bytes_gs<2, 2>(tt);
-    case 6: return smem_bytes_gs<0, 1, 2>(tt);
-    case 7: return smem_bytes_gs<1, 1, 2>(tt);
-    default: return smem_bytes_gs<2, 1, 2>(tt);
+    VariantCfg v{};
+    switch (tt) {
+    case 1: cfg_of<1>(variant, &v.smem, &v.us, &v.ks, &v.code_tile, &v.g, &v.threads); break;
+    case 2: cfg_of<2>(variant, &v.smem, &v.us, &v.ks, &v.code_tile, &v.g, &v.threads); break;
+    case 3: cfg_of<3>(variant, &v.smem, &v.us, &v.ks, &v.code_tile, &v.g, &v.threads); break;
+    default: cfg_of<4>(variant, &v.smem, &v.us, &v.ks, &v.code_tile, &v.g, &v.threads); break;
     }
+    return v;
 }
 
 int group_mode(int G)
@@ -598,41 +590,40 @@ int group_mode(int G)
     return G == 128 ? 0 : (G == 64 ? 1 : 2);
 }
 
-}  // namespace
-
-namespace {
-
-// bits: 4 (INT4) or 8 (INT8, two code planes, one scale-group span per unit)
+// bits: 4 (INT4) or 8 (INT8, two code planes)
 bool plan_stream(int device, int M, int N, int K, int G, int bits, StreamPlan *plan)
 {
-    if (M < 1 || M > 32 || N % 32 != 0)
+    if (M < 1 || M > 32 || N % 64 != 0 || K % 64 != 0 || K % G != 0)
+        return false;
+    if (device < 0 || device >= kMaxDeviceCache)
         return false;
     const DeviceInfo &di = device_info(device);
     StreamPlan pl{};
     pl.tt = (M + 7) / 8;
-    const int unit_k = std::max(G, 64);
-    const int su = (bits == 4 && pl.tt <= 2 && (K / unit_k) % 2 == 0) ? 2 : 1;
-    pl.variant = bits == 8 ? 6 + group_mode(G) : group_mode(G) + 3 * (su - 1);
-    pl.warps_per_cta = kConsumers;
-    pl.smem = smem_bytes(pl.tt, pl.variant);
+    pl.variant = (bits == 8 ? 3 : 0) + group_mode(G);
+    const VariantCfg vc = variant_cfg(pl.tt, pl.variant);
+    pl.warps_per_cta = vc.threads / 32;
+    pl.smem = vc.smem;
     if ((int)pl.smem > di.smem_optin)
         return false;
-    pl.upt = K / (unit_k * su);
-    pl.ntiles = N / 32;
+    const int unit_k = vc.us * vc.ks;
+    if (K % unit_k != 0)
+        return false;
+    pl.upt = K / unit_k;                      // units per group row
+    const int ngroups = (N / 32 + kWarps - 1) / kWarps;
+    pl.ntiles = ngroups * kWarps;             // arrival counters (one per tile slot)
     if ((size_t)pl.ntiles > kMaxCounters)
         return false;
-    pl.units = (long long)pl.ntiles * pl.upt;
+    pl.units = (long long)ngroups * pl.upt;
     if (pl.units > (1LL << 30))
         return false;
     const void *fn = select_kernel(pl.tt, pl.variant);
     if (!fn)
         return false;
-    // resident CTAs per SM for this variant: every CTA of the grid must be
-    // resident at once (a cut tile's finishing CTA waits for the others)
-    // (function attributes and occupancy are per device: cached per device)
-    if (device < 0 || device >= kMaxDeviceCache)
-        return false;
-    static std::atomic<int> occ_cache[kMaxDeviceCache][4][9];
+    // every CTA of the grid must be resident at once (a cut row's finishing
+    // CTA waits for the others); function attributes and occupancy are per
+    // device: cached per device
+    static std::atomic<int> occ_cache[kMaxDeviceCache][4][6];
     std::atomic<int> &occ_slot = occ_cache[device][pl.tt - 1][pl.variant];
     int occ = occ_slot.load(std::memory_order_acquire);
     if (occ == 0) {
@@ -640,23 +631,18 @@ bool plan_stream(int device, int M, int N, int K, int G, int bits, StreamPlan *p
             cudaSuccess)
             return false;
         int o = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, fn, kThreads, pl.smem) !=
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, fn, vc.threads, pl.smem) !=
                 cudaSuccess ||
             o < 1)
             return false;
-        occ = std::min(o, kCtasPerSm);
+        occ = o;
         occ_slot.store(occ, std::memory_order_release);
     }
-    // kCtasPerSm CTAs per SM, but no run shorter than kMinUnitsPerCta units;
-    // a layer too small for 32 such runs gets at least one CTA per n32 tile
-    // instead (one CTA streaming many short tiles would serialise their
-    // reductions)
-    long long wt = std::min<long long>((long long)di.sms * occ, pl.units / kMinUnitsPerCta);
-    if (wt < 32)
-        wt = std::min<long long>((long long)di.sms * occ, std::max<long long>(wt, pl.ntiles));
-    pl.Wt = (int)std::max<long long>(1, wt);
+    // one CTA per SM (a second resident CTA, where it fits, is left to the
+    // next GEMM on the stream), no run shorter than one unit
+    pl.Wt = (int)std::max<long long>(1, std::min<long long>(di.sms, pl.units));
     pl.grid = pl.Wt;
-    pl.partial_bytes = (size_t)pl.Wt * (2 * pl.tt * 32) * sizeof(float4);
+    pl.partial_bytes = (size_t)pl.Wt * kWarps * (2 * pl.tt * 32) * sizeof(float4);
     *plan = pl;
     return true;
 }
@@ -674,33 +660,49 @@ bool plan_w8a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan)
 }
 
 cudaError_t launch_w4a16_stream(const StreamPlan &pl, const void *X, const void *packed, int M,
-                                int N, int K, int G, void *Y, void *workspace, cudaStream_t stream)
+                                int N, int K, int G, void *Y, void *workspace, bool early,
+                                cudaStream_t stream)
 {
-    (void)G;
     const void *fn = select_kernel(pl.tt, pl.variant);
     if (!fn)
         return cudaErrorInvalidValue;
+    const VariantCfg vc = variant_cfg(pl.tt, pl.variant);
+    const int planes = pl.variant >= 3 ? 2 : 1;
+    const uint8_t *codes = static_cast<const uint8_t *>(packed);
+    // codes take half a byte per weight (INT4) or one byte in two planes (INT8)
+    const uint8_t *scales = codes + (size_t)N * K / 2 * planes;
+    const uint64_t tiles = (uint64_t)N / 32;
+    alignas(64) CUtensorMap cmap, smap, xmap;
+    // codes: one row of 16 * K * planes bytes per n32 tile, in 8-byte elements
+    // scales: one row of 64 * K / G bytes per tile
+    // X: bf16 [M][K], boxes of 64 k x 8 TT rows with 128-byte swizzle
+    if (!encode_tensor_map_2d(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT64, codes,
+                              (uint64_t)K * 2 * planes, tiles, (uint64_t)K * 16 * planes,
+                              (uint32_t)(vc.code_tile / 8), kWarps, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !encode_tensor_map_2d(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT64, scales,
+                              (uint64_t)(K / G) * 8, tiles, (uint64_t)(K / G) * 64,
+                              (uint32_t)(vc.ks >= G ? vc.ks / G : 1) * 8, kWarps,
+                              CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !encode_tensor_map_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)K,
+                              (uint64_t)M, (uint64_t)K * 2, 64, (uint32_t)(8 * pl.tt),
+                              CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
     const WorkspaceMap wm = make_workspace_map(pl.ntiles, pl.partial_bytes);
     Params p{};
-    p.X = static_cast<const uint16_t *>(X);
-    p.codes = static_cast<const uint8_t *>(packed);
-    // codes take half a byte per weight (INT4) or one byte in two planes (INT8)
-    p.scales = p.codes + (pl.variant >= 6 ? (size_t)N * K : (size_t)N * K / 2);
     p.Y = static_cast<uint16_t *>(Y);
-    p.early = early_weight_loads() ? 1 : 0;
+    p.early = early ? 1 : 0;
+    p.pf_stages = MXG_STREAM_PF_STAGES;
     p.hdr = static_cast<WsHeader *>(workspace);
     p.counters = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + wm.counters_off);
     p.partial = reinterpret_cast<float4 *>(static_cast<uint8_t *>(workspace) + wm.partial_off);
     p.M = M;
     p.N = N;
-    p.K = K;
-    p.upt = pl.upt;
-    p.units = (int)pl.units;
-    p.ctas = pl.Wt;
+    p.ntiles = N / 32;
+    p.upr = pl.upt;
     p.q = (int)(pl.units / pl.Wt);
     p.r = (int)(pl.units % pl.Wt);
-    void *args[] = {&p};
-    return launch_pdl(fn, dim3(pl.grid), dim3(kThreads), pl.smem, stream, args);
+    void *args[] = {&cmap, &smap, &xmap, &p};
+    return launch_pdl(fn, dim3(pl.grid), dim3(vc.threads), pl.smem, stream, args);
 }
 
 }  // namespace mxg

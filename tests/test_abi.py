@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(mxg):
 
 
 def test_status_strings(mxg):
-    for s in range(-5, 1):
+    for s in range(-6, 1):
         assert mxg.mxg_status_string(s) not in ("", "unknown status")
     assert mxg.mxg_status_string(-99) == "unknown status"
 
@@ -105,20 +105,53 @@ def test_arguments_rejected_before_launch(mxg):
     assert lib.w8a16_workspace_bytes(33, 512, 512, 128) == 0
 
 
-def test_path_override_roundtrip(mxg):
-    prev = mxg.mxg_set_path(1)
-    assert mxg.mxg_set_path(2) == 1
-    assert mxg.mxg_set_path(prev) == 2
-    with pytest.raises(ValueError):
-        mxg.mxg_set_path(3)
+def test_per_call_options_rejected_before_launch(mxg):
+    """The *_ex entry points check their options before anything else: a
+    path or late_weights value outside its range, or a path the format does
+    not have, is MXG_ERR_INVALID_ARG (no kernel runs here)."""
+    lib = mxg.raw_lib()
+    a = ctypes.c_void_p(4096)
+    null = None
+
+    def opts(path, late):
+        return ctypes.byref(mxg.GemmOptions(path, late))
+    for bad in [opts(3, 0), opts(-1, 0), opts(0, 2)]:
+        assert lib.w4a16_gemm_ex(a, a, 5, 512, 512, 128, a, a, 1 << 20, bad, null) == \
+            mxg.MXG_ERR_INVALID_ARG
+        assert lib.mxfp8_gemm_ex(a, a, a, 4, 256, 512, a, a, 1 << 20, bad, null) == \
+            mxg.MXG_ERR_INVALID_ARG
+        assert lib.w8a16_gemm_ex(a, a, 5, 512, 512, 128, a, a, 1 << 20, bad, null) == \
+            mxg.MXG_ERR_INVALID_ARG
+        assert lib.bf16_gemm_small_ex(a, a, 4, 96, 5120, a, a, 1 << 20, bad, null) == \
+            mxg.MXG_ERR_INVALID_ARG
+    # INT8 has no tensor-core path; the bf16 projection has no path choice
+    assert lib.w8a16_gemm_ex(a, a, 5, 512, 512, 128, a, a, 1 << 20, opts(2, 0), null) == \
+        mxg.MXG_ERR_INVALID_ARG
+    assert lib.bf16_gemm_small_ex(a, a, 4, 96, 5120, a, a, 1 << 20, opts(1, 0), null) == \
+        mxg.MXG_ERR_INVALID_ARG
+    # valid options reach the usual argument checks
+    assert lib.w4a16_gemm_ex(a, a, 0, 512, 512, 128, a, a, 1 << 20, opts(1, 1), null) == \
+        mxg.MXG_ERR_INVALID_ARG          # M < 1
+    assert lib.w4a16_gemm_ex(a, a, 5, 512, 512, 96, a, a, 1 << 20, null, null) == \
+        mxg.MXG_ERR_UNSUPPORTED_SHAPE
+    assert lib.bf16_gemm_small_ex(a, a, 4, 96, 5120, a, a, 256, opts(0, 1), null) == \
+        mxg.MXG_ERR_WORKSPACE
 
 
-def test_early_weight_loads_roundtrip(mxg):
-    assert mxg.mxg_set_early_weight_loads(0) == 1  # on by default
-    assert mxg.mxg_set_early_weight_loads(1) == 0
-    with pytest.raises(ValueError):
-        mxg.mxg_set_early_weight_loads(2)
-    assert mxg.mxg_set_early_weight_loads(1) == 1
+def test_no_process_wide_settings(mxg):
+    """Every choice a caller makes is an argument of its call: the library
+    exports no setter that would change another caller's behaviour."""
+    names = declared_functions()
+    assert not [n for n in names if "set_" in n]
+    lib = ctypes.CDLL(mxg.LIB_PATH)
+    assert not hasattr(lib, "mxg_set_path") and not hasattr(lib, "mxg_set_early_weight_loads")
+
+
+def test_static_scratch_status_rejects_bad_arguments(mxg):
+    lib = mxg.raw_lib()
+    v = ctypes.c_int(0)
+    assert lib.w4a16_static_scratch_status(None, 0, None) == mxg.MXG_ERR_INVALID_ARG
+    assert lib.w4a16_static_scratch_status(ctypes.byref(v), 2, None) == mxg.MXG_ERR_INVALID_ARG
 
 
 def test_binding_refuses_to_load_without_the_library(tmp_path):

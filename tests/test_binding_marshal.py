@@ -15,6 +15,8 @@ class FakeLib:
 
     def __init__(self, real):
         self.calls = []
+        self.devices = []     # the device current during each recorded call
+        self.current = []
         self._real = real
 
     def __getattr__(self, name):
@@ -27,6 +29,7 @@ class FakeLib:
 
         def fn(*args):
             self.calls.append((name, args))
+            self.devices.append(self.current[-1] if self.current else None)
             return 0
         return fn
 
@@ -49,7 +52,21 @@ def fake(monkeypatch):
         if not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
     monkeypatch.setattr(m, "_need", need_cpu)
-    monkeypatch.setattr(m, "_stream", lambda stream=None: None)
+
+    class OnDevice:
+        """Records the device made current around each C call."""
+
+        def __init__(self, device):
+            self.device = device
+
+        def __enter__(self):
+            lib.current.append(self.device)
+
+        def __exit__(self, *exc):
+            lib.current.pop()
+    monkeypatch.setattr(m, "_on_device", OnDevice)
+    monkeypatch.setattr(m, "_stream",
+                        lambda stream=None, device=None: ("stream", stream, device))
     monkeypatch.setattr(m, "workspace",
                         lambda nbytes, device=None, stream=None: torch.zeros(max(nbytes, 256),
                                                                              dtype=torch.uint8))
@@ -68,14 +85,18 @@ def test_w4a16_calls(fake):
     packed = torch.zeros(m.w4a16_packed_bytes(K, N, G), dtype=torch.uint8)
     y = m.w4a16_gemm(x, packed, N, K, G)
     name, a = lib.calls[-1]
-    assert name == "w4a16_gemm"
+    assert name == "w4a16_gemm_ex"
     assert [_val(v) for v in a[:6]] == [x.data_ptr(), packed.data_ptr(), M, N, K, G]
     assert _val(a[6]) == y.data_ptr() and tuple(y.shape) == (M, N)
     assert a[8] == 4096          # the workspace's bytes
+    assert a[9] is None          # default options: NULL
+    m.w4a16_gemm(x, packed, N, K, G, path=m.PATH_STREAM, late_weights=True)
+    opts = lib.calls[-1][1][9].contents
+    assert (opts.path, opts.late_weights) == (1, 1)
     call, y2 = m.prepare_w4a16_gemm(x, packed, N, K, G)
     call()
     name, a = lib.calls[-1]
-    assert name == "w4a16_gemm" and _val(a[6]) == y2.data_ptr() and a[2:6] == (M, N, K, G)
+    assert name == "w4a16_gemm_ex" and _val(a[6]) == y2.data_ptr() and a[2:6] == (M, N, K, G)
     m.w4a16_gemm_static_scratch(x, packed, N, K, G)
     name, a = lib.calls[-1]
     assert name == "w4a16_gemm_static_scratch" and a[2:6] == (M, N, K, G)
@@ -119,10 +140,10 @@ def test_w8a16_calls(fake):
     packed = torch.zeros(int(m.raw_lib().w8a16_packed_bytes(K, N, G)), dtype=torch.uint8)
     y = m.w8a16_gemm(x, packed, N, K, G)
     name, a = lib.calls[-1]
-    assert name == "w8a16_gemm" and a[2:6] == (M, N, K, G) and _val(a[6]) == y.data_ptr()
+    assert name == "w8a16_gemm_ex" and a[2:6] == (M, N, K, G) and _val(a[6]) == y.data_ptr()
     call, _ = m.prepare_w8a16_gemm(x, packed, N, K, G)
     call()
-    assert lib.calls[-1][0] == "w8a16_gemm"
+    assert lib.calls[-1][0] == "w8a16_gemm_ex"
     with pytest.raises(ValueError):
         m.w8a16_gemm(x, packed[: packed.numel() // 2], N, K, G)
     with pytest.raises(ValueError):
@@ -139,12 +160,12 @@ def test_mxfp8_calls(fake):
     ws = torch.zeros((N, K // 32), dtype=torch.uint8)
     y = m.mxfp8_gemm(x, wq, ws)
     name, a = lib.calls[-1]
-    assert name == "mxfp8_gemm"
+    assert name == "mxfp8_gemm_ex"
     assert [_val(v) for v in a[:3]] == [x.data_ptr(), wq.data_ptr(), ws.data_ptr()]
     assert a[3:6] == (M, N, K) and _val(a[6]) == y.data_ptr()
     call, _ = m.prepare_mxfp8_gemm(x, wq, ws)
     call()
-    assert lib.calls[-1][0] == "mxfp8_gemm"
+    assert lib.calls[-1][0] == "mxfp8_gemm_ex"
     with pytest.raises(ValueError):
         m.mxfp8_gemm(x, wq, ws[:, :-1])
     with pytest.raises(ValueError):
@@ -157,10 +178,10 @@ def test_bf16_small_calls(fake):
     x, w = bf16(M, K), bf16(N, K)
     y = m.bf16_gemm_small(x, w)
     name, a = lib.calls[-1]
-    assert name == "bf16_gemm_small" and a[2:5] == (M, N, K) and _val(a[5]) == y.data_ptr()
+    assert name == "bf16_gemm_small_ex" and a[2:5] == (M, N, K) and _val(a[5]) == y.data_ptr()
     call, _ = m.prepare_bf16_gemm_small(x, w)
     call()
-    assert lib.calls[-1][0] == "bf16_gemm_small"
+    assert lib.calls[-1][0] == "bf16_gemm_small_ex"
     with pytest.raises(ValueError):
         m.bf16_gemm_small(x, w, out=bf16(M, N + 16))
     with pytest.raises(m.MxgError):
@@ -209,3 +230,45 @@ def test_repack_and_decoder_shapes(fake):
                           torch.zeros((N, K // 32), dtype=torch.uint8))
     name, a = lib.calls[-1]
     assert name == "mxfp8_dequant" and a[2:4] == (N, K) and _val(a[4]) == w16.data_ptr()
+
+
+def test_calls_run_on_the_tensors_device_and_stream(fake):
+    """Every C call runs with its tensors' device current (the library plans
+    for, and launches on, the current device) and gets a stream of that
+    device: the caller's, or the device's current one."""
+    m, lib = fake
+    M, K, N, G = 5, 512, 256, 128
+    x = bf16(M, K)
+    packed = torch.zeros(m.w4a16_packed_bytes(K, N, G), dtype=torch.uint8)
+    sentinel = object()
+    m.w4a16_gemm(x, packed, N, K, G, stream=sentinel)
+    assert lib.devices[-1] == x.device
+    assert lib.calls[-1][1][-1] == ("stream", sentinel, x.device)
+    m.w4a16_gemm(x, packed, N, K, G)
+    assert lib.calls[-1][1][-1] == ("stream", None, x.device)
+    call, _ = m.prepare_w4a16_gemm(x, packed, N, K, G, stream=sentinel)
+    call()
+    assert lib.devices[-1] == x.device and lib.calls[-1][1][-1] == ("stream", sentinel, x.device)
+    wq = torch.zeros((N, K), dtype=torch.uint8)
+    ws = torch.zeros((N, K // 32), dtype=torch.uint8)
+    m.mxfp8_gemm(x, wq, ws)
+    assert lib.devices[-1] == x.device
+    m.w4a16_repack(torch.zeros((K // 8, N), dtype=torch.int32),
+                   torch.zeros((K // G, N), dtype=torch.float16), G)
+    assert lib.devices[-1] == x.device
+    assert not lib.current                      # every device context was left
+
+
+def test_stream_of_another_device_is_refused():
+    """A stream that lives on another device than the call's tensors is
+    refused before any C call."""
+    import __graft_entry__
+    __graft_entry__.build()
+    import mxfp8_gemm_speculative_b200 as m
+
+    class FakeStream:
+        device = torch.device("cuda", 1)
+        cuda_stream = 0
+    with pytest.raises(ValueError):
+        m._stream(FakeStream(), torch.device("cuda", 0))
+    assert m._stream(FakeStream(), torch.device("cuda", 1)).value is None

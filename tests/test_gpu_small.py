@@ -45,14 +45,8 @@ def test_bf16_small_deterministic(mxg):
     x, w = bf16_tensor(lay.X, DEV), bf16_tensor(lay.W, DEV)
     ws = torch.zeros(mxg.raw_lib().bf16_gemm_small_workspace_bytes(M, N, K), dtype=torch.uint8,
                      device=DEV)
-    outs = []
-    prev = mxg.mxg_set_early_weight_loads(1)
-    try:
-        for early in (1, 1, 0):
-            mxg.mxg_set_early_weight_loads(early)
-            outs.append(mxg.bf16_gemm_small(x, w, workspace_buf=ws))
-    finally:
-        mxg.mxg_set_early_weight_loads(prev)
+    outs = [mxg.bf16_gemm_small(x, w, workspace_buf=ws, late_weights=late)
+            for late in (False, False, True)]
     torch.cuda.synchronize()
     assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
     assert torch.equal(outs[0].view(torch.int16), outs[2].view(torch.int16))

@@ -18,7 +18,6 @@ def mxg():
     import __graft_entry__
     __graft_entry__.build()
     import mxfp8_gemm_speculative_b200 as m
-    m.mxg_set_path(0)
     return m
 
 
@@ -31,11 +30,7 @@ def int4_device(lay):
 def run_int4(mxg, lay, path=0):
     qw, sc = int4_device(lay)
     packed = mxg.w4a16_repack(qw, sc, lay.group_size)
-    prev = mxg.mxg_set_path(path)
-    try:
-        y = mxg.w4a16_gemm(bf16_tensor(lay.X, DEV), packed, lay.N, lay.K, lay.group_size)
-    finally:
-        mxg.mxg_set_path(prev)
+    y = mxg.w4a16_gemm(bf16_tensor(lay.X, DEV), packed, lay.N, lay.K, lay.group_size, path=path)
     return y, packed
 
 
@@ -184,12 +179,8 @@ def test_int4_mtp4_verify_layers_sampled(mxg, li):
 @pytest.mark.parametrize("N,K", [(128, 64), (130, 96), (256, 512), (1000, 2080)])
 def test_mxfp8_stream_parity(mxg, M, N, K):
     lay = synth.mxfp8_layer(M, K, N, seed=M + N + K)
-    prev = mxg.mxg_set_path(1)
-    try:
-        y = mxg.mxfp8_gemm(bf16_tensor(lay.X, DEV), torch.from_numpy(lay.Wq).to(DEV),
-                           torch.from_numpy(lay.Ws).to(DEV))
-    finally:
-        mxg.mxg_set_path(prev)
+    y = mxg.mxfp8_gemm(bf16_tensor(lay.X, DEV), torch.from_numpy(lay.Wq).to(DEV),
+                       torch.from_numpy(lay.Ws).to(DEV), path=1)
     ref = oracle.mxfp8_gemm(lay.X, lay.Wq, lay.Ws, M, N, K)
     assert_parity(to_f64(y), ref, f"mxfp8 stream M={M} N={N} K={K}")
 
@@ -280,19 +271,15 @@ def test_early_weight_loads_match_late_loads(mxg):
     x = bf16_tensor(lay.X, DEV)
     packed = mxg.w4a16_repack(qw, sc, 128)
     outs = {}
-    prev = mxg.mxg_set_early_weight_loads(1)
-    try:
-        for early in (1, 0):
-            mxg.mxg_set_early_weight_loads(early)
-            y1 = mxg.w4a16_gemm(x, packed, 1024, 2048, 128)
-            # re-pack other weights into the same buffer, GEMM right after
-            mxg.w4a16_repack(qw2, sc2, 128, out=packed)
-            y2 = mxg.w4a16_gemm(x, packed, 1024, 2048, 128)
-            mxg.w4a16_repack(qw, sc, 128, out=packed)
-            torch.cuda.synchronize()
-            outs[early] = (y1, y2)
-    finally:
-        mxg.mxg_set_early_weight_loads(prev)
+    for early in (1, 0):
+        late = not early
+        y1 = mxg.w4a16_gemm(x, packed, 1024, 2048, 128, late_weights=late)
+        # re-pack other weights into the same buffer, GEMM right after
+        mxg.w4a16_repack(qw2, sc2, 128, out=packed)
+        y2 = mxg.w4a16_gemm(x, packed, 1024, 2048, 128, late_weights=late)
+        mxg.w4a16_repack(qw, sc, 128, out=packed)
+        torch.cuda.synchronize()
+        outs[early] = (y1, y2)
     for a, b in zip(outs[1], outs[0]):
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))
     ref2 = oracle.w4a16_gemm(lay.X, lay2.qweight, lay2.scales, 5, 1024, 2048, 128)
@@ -300,14 +287,7 @@ def test_early_weight_loads_match_late_loads(mxg):
     mlay = synth.mxfp8_layer(4, 512, 256, seed=33)
     wq, ws = torch.from_numpy(mlay.Wq).to(DEV), torch.from_numpy(mlay.Ws).to(DEV)
     xm = bf16_tensor(mlay.X, DEV)
-    mouts = []
-    prev = mxg.mxg_set_early_weight_loads(1)
-    try:
-        for early in (1, 0):
-            mxg.mxg_set_early_weight_loads(early)
-            mouts.append(mxg.mxfp8_gemm(xm, wq, ws))
-    finally:
-        mxg.mxg_set_early_weight_loads(prev)
+    mouts = [mxg.mxfp8_gemm(xm, wq, ws, late_weights=late) for late in (False, True)]
     torch.cuda.synchronize()
     assert torch.equal(mouts[0].view(torch.int16), mouts[1].view(torch.int16))
 

@@ -18,7 +18,6 @@ def mxg():
     import __graft_entry__
     __graft_entry__.build()
     import mxfp8_gemm_speculative_b200 as m
-    m.mxg_set_path(0)
     return m
 
 
@@ -26,24 +25,15 @@ def int4_gemm(mxg, lay, path):
     qw = torch.from_numpy(lay.qweight).to(DEV)
     sc = torch.from_numpy(lay.scales.view(np.int16)).to(DEV)
     packed = mxg.w4a16_repack(qw, sc, lay.group_size)
-    prev = mxg.mxg_set_path(path)
-    try:
-        y = mxg.w4a16_gemm(bf16_tensor(lay.X, DEV), packed, lay.N, lay.K, lay.group_size)
-        ws = mxg.workspace(0)
-        assert mxg.mxg_workspace_status(ws) == 0
-    finally:
-        mxg.mxg_set_path(prev)
+    y = mxg.w4a16_gemm(bf16_tensor(lay.X, DEV), packed, lay.N, lay.K, lay.group_size, path=path)
+    assert mxg.mxg_workspace_status(mxg.workspace(0)) == 0
     return y
 
 
 def mxfp8_gemm(mxg, lay, path):
-    prev = mxg.mxg_set_path(path)
-    try:
-        y = mxg.mxfp8_gemm(bf16_tensor(lay.X, DEV), torch.from_numpy(lay.Wq).to(DEV),
-                           torch.from_numpy(lay.Ws).to(DEV))
-        assert mxg.mxg_workspace_status(mxg.workspace(0)) == 0
-    finally:
-        mxg.mxg_set_path(prev)
+    y = mxg.mxfp8_gemm(bf16_tensor(lay.X, DEV), torch.from_numpy(lay.Wq).to(DEV),
+                       torch.from_numpy(lay.Ws).to(DEV), path=path)
+    assert mxg.mxg_workspace_status(mxg.workspace(0)) == 0
     return y
 
 
