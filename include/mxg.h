@@ -112,10 +112,13 @@ MXG_API size_t w4a16_packed_bytes(int K, int N, int group_size);
  *   qweight  device, int32 [K/8][N], GPTQ words as described above.
  *   scales   device, fp16 bits [K/G][N].
  *   packed   device, caller-allocated, w4a16_packed_bytes(K, N, G) bytes.
- * Layout written (private to this library, stable for a given K, N, G):
- * codes as [N/32][K/64][2 halves][32 lanes][16 B] (one 16-byte load is one
- * lane's MMA fragment for four k16 steps of two weight columns), then scales
- * as [N/32][K/G][8][4].
+ * Layout written (private to this library, stable for a given K, N, G), by
+ * column groups of 256 columns (eight n32 tiles; the last group holds the
+ * remaining tiles when N % 256 != 0): codes as [N/256 groups][K/64][tiles of
+ * the group][2 halves][32 lanes][16 B] (one 16-byte load is one lane's MMA
+ * fragment for four k16 steps of two weight columns; the codes of a group
+ * for any run of k64 chunks are contiguous), then scales as [N/256 groups]
+ * [K/G][tiles of the group][8][4].
  * Requirements: G in {32, 64, 128}; K % 64 == 0; K % G == 0; N % 64 == 0.
  * Otherwise MXG_ERR_UNSUPPORTED_SHAPE. */
 MXG_API int w4a16_repack(const int32_t *qweight, const uint16_t *scales,

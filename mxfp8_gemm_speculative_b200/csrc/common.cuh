@@ -33,6 +33,41 @@ __device__ __forceinline__ void record_error(WsHeader *h, int status, int where)
         atomicExch(&h->where, where);
 }
 
+// ------------------------------------------------ re-packed weight layout
+// The re-packed INT4 (P = 1 code plane) and INT8 (P = 2: a plane of low and
+// a plane of high nibbles) weights are stored by column groups of eight n32
+// tiles (256 columns; when N is not a multiple of 256 the last group holds
+// the remaining tiles).  Codes: group gr takes 8 * 16 * K * P bytes (less
+// for the last group), as K/64 chunks of [tiles of the group][1024 * P B]; the
+// 1024 * P bytes of one tile and chunk are [2 halves][P planes][32 lanes]
+// [16 B].  So the codes of a group for any run of k64 chunks form one
+// contiguous range, which both GEMM paths move with one bulk copy.  Scales
+// follow all the codes: group gr takes 8 * (K/G) * 64 bytes (less for the
+// last group), as K/G scale groups of [tiles of the group][64 B], the 64
+// bytes of a tile being [8][4 halves] (see the re-pack).
+__host__ __device__ __forceinline__ int group_tiles(int gr, int ntiles)
+{
+    return ntiles - 8 * gr < 8 ? ntiles - 8 * gr : 8;
+}
+
+// Byte offset of the codes of (n32 tile, k64 chunk) in a layer of ntiles tiles.
+__host__ __device__ __forceinline__ size_t code_offset(int tile, int chunk, int K, int ntiles,
+                                                       int P)
+{
+    const int gr = tile >> 3;
+    return (size_t)gr * 8 * 16 * K * P +
+           ((size_t)chunk * group_tiles(gr, ntiles) + (tile & 7)) * 1024 * P;
+}
+
+// Byte offset, inside the scale region, of the 64 scale bytes of (n32 tile,
+// scale group).
+__host__ __device__ __forceinline__ size_t scale_offset(int tile, int kgroup, int K, int G,
+                                                        int ntiles)
+{
+    const int gr = tile >> 3;
+    return (size_t)gr * 8 * (K / G) * 64 + ((size_t)kgroup * group_tiles(gr, ntiles) + (tile & 7)) * 64;
+}
+
 // ------------------------------------------------------------------- basics
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
@@ -226,6 +261,24 @@ __device__ __forceinline__ uint2 lds64(const void *p)
 {
     uint2 v;
     asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(smem_u32(p)));
+    return v;
+}
+
+// The same shared-memory loads from a 32-bit shared-window address (no
+// generic-to-shared conversion per access).
+__device__ __forceinline__ uint4 lds128a(uint32_t a)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(a));
+    return v;
+}
+
+__device__ __forceinline__ uint2 lds64a(uint32_t a)
+{
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
     return v;
 }
 

@@ -36,20 +36,25 @@ WorkspaceMap make_workspace_map(size_t counters, size_t partial_bytes);
 
 // ------------------------------------------------------ weight-streaming path
 // Stream-K plan: the layer's weight bytes are cut into equal "units" (one
-// n32 tile x one scale-group span for INT4, one n16 tile x 128 k for MXFP8)
-// and every CTA (INT4) or warp (MXFP8) of a persistent grid takes one
-// contiguous run of units.
+// 256-column group x 128 rows of K for INT4 and INT8, one n16 tile x 128 k
+// for MXFP8) and every CTA (INT4) or warp (MXFP8) of a persistent grid takes
+// one contiguous run of units.
 struct StreamPlan {
     int tt;               // token tiles of 8 rows (ceil(M / 8)), 1..4
-    int variant;          // kernel variant (group mode for INT4)
+    int variant;          // kernel variant
     int warps_per_cta;
     int grid;             // CTAs
     int Wt;               // runs: CTAs (INT4) or warps (MXFP8), <= units
     long long units;      // total units
-    int upt;              // units per output tile
+    int upt;              // units per output tile (INT4: per group row)
     size_t smem;          // dynamic shared memory per CTA
     size_t partial_bytes; // workspace for partial sums
-    int ntiles;           // output tiles (= arrival counters)
+    int ntiles;           // arrival counters
+    // INT4 / INT8: pieces per group row (0: stream-K runs across rows);
+    // shared-memory plan: ring stages and region offsets
+    int split;
+    int ring;
+    int x_off, xs_off, xchg_off, bar_off;
 };
 
 bool plan_w4a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan);

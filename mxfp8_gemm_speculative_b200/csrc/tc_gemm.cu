@@ -74,6 +74,8 @@ struct Layout {
 struct TcParams {
     uint16_t *Y;
     const uint8_t *Ws;     // MXFP8 scales [N][K/32]
+    const uint8_t *codes;  // INT4: re-packed codes (column-group layout, common.cuh)
+    const uint8_t *scales; // INT4: re-packed scales
     WsHeader *hdr;
     float *partial;        // split-K partial sums [num_items][BT][2 * BW] (splits > 1)
     int *counters;         // split-K arrivals per (tile, CTA of the pair, quadrant)
@@ -271,10 +273,12 @@ __device__ __forceinline__ void dequant_int4(const uint8_t *wp_slot, int q, int 
     const int g = lane >> 2;
     const uint4 c = lds128(wp_slot + q * 1024 + h * 512 + lane * 16);
     const uint32_t w[4] = {c.x, c.y, c.z, c.w};
-    // words 0-1 and 2-3 lie in one scale group each (the same one for G >= 64)
-    const uint8_t *sbase = wp_slot + 4096 + q * (64 * gpk) + g * 8 + h * 4;
+    // words 0-1 and 2-3 lie in one scale group each (the same one for G >= 64);
+    // the slot holds the scales as [gpk groups][4 tiles][64 B]
+    (void)gpk;
+    const uint8_t *sbase = wp_slot + 4096 + q * 64 + g * 8 + h * 4;
     const uint32_t sw0 = lds32(sbase);
-    const uint32_t sw1 = G == 32 ? lds32(sbase + 64) : sw0;
+    const uint32_t sw1 = G == 32 ? lds32(sbase + 256) : sw0;
     const ScaleSplit sa0 = split_scale((uint16_t)(sw0 & 0xFFFF));
     const ScaleSplit sb0 = split_scale((uint16_t)(sw0 >> 16));
     ScaleSplit sa1 = sa0, sb1 = sb0;
@@ -361,12 +365,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         item_range(p, pair, tile0, kb0, kb1);
         const int nb = tile0 / p.mtiles, mt = tile0 % p.mtiles;
         const int n32 = (nb * 2 * BW + (int)rank * BW) / 32;
+        const int ntl = F == kInt4 ? max(0, min(4, group_tiles(nb, p.N / 32) - 4 * (int)rank)) : 0;
         for (int kb = kb0; kb < min(kb0 + L::kSW, kb1); ++kb) {
             prefetch_tensor_l2(&x_map, kb * BK, mt * BT + (int)rank * (BT / 2));
-            if (F == kInt4)
-                prefetch_tensor_l2(&w_map, kb * 128, n32);
-            else
+            if (F == kInt4) {
+                if (ntl > 0)
+                    prefetch_l2(p.codes + code_offset(n32, kb, p.K, p.N / 32, 1), ntl * 1024);
+            } else {
                 prefetch_tensor_l2(&w_map, kb * BK, n32 * 32);
+            }
         }
     }
     tc_fence_before();
@@ -400,9 +407,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int n32 = (nb * 2 * BW + (int)rank * BW) / 32;
             uint8_t *wdst = smem + L::wp_off + sw * L::wp_slot;
             if (F == kInt4) {
-                mbar_arrive_expect_tx(&wp_full[sw], 4096u + 256u * gpk);
-                tma_load_2d(wdst, &w_map, w_kb * 128, n32, &wp_full[sw], pol_w);
-                tma_load_2d(wdst + 4096, &s_map, (w_kb * BK / p.G) * 8, n32, &wp_full[sw], pol_w);
+                // this CTA's tiles of the column group (all four, or fewer
+                // in a last group of fewer than eight): codes of the k-block
+                // and the scales of its gpk groups, each one contiguous range
+                // per scale group
+                const int ntl = max(0, min(4, group_tiles(n32 >> 3, p.N / 32) - (n32 & 7)));
+                mbar_arrive_expect_tx(&wp_full[sw], (uint32_t)ntl * (1024u + 64u * gpk));
+                if (ntl > 0) {
+                    bulk_g2s(wdst, p.codes + code_offset(n32, w_kb, p.K, p.N / 32, 1),
+                             ntl * 1024, &wp_full[sw], pol_w);
+                    for (int gi = 0; gi < gpk; ++gi)
+                        bulk_g2s(wdst + 4096 + gi * 256,
+                                 p.scales + scale_offset(n32, w_kb * BK / p.G + gi, p.K, p.G,
+                                                         p.N / 32),
+                                 ntl * 64, &wp_full[sw], pol_w);
+                }
             } else {
                 mbar_arrive_expect_tx(&wp_full[sw], (uint32_t)(BW * BK));
                 tma_load_2d(wdst, &w_map, w_kb * BK, n32 * 32, &wp_full[sw], pol_w);
@@ -413,9 +432,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         return true;
     };
     if (warp == kWProducerWarp && lane == 0) {
-        prefetch_tensormap(&w_map);
-        if (F == kInt4)
-            prefetch_tensormap(&s_map);
+        if (F != kInt4)
+            prefetch_tensormap(&w_map);
         // The weights are not written by the previous kernel on the stream
         // (the caller's contract, unless it turned early weight loads off):
         // the first ring of them fills while that kernel drains.  Everything
@@ -744,23 +762,16 @@ cudaError_t launch_w4a16_tc(const TcPlan &pl, const void *X, const void *packed,
                             int K, int G, void *Y, void *workspace, bool early,
                             cudaStream_t stream)
 {
-    alignas(64) CUtensorMap xm, wm, sm;
+    alignas(64) CUtensorMap xm;
     const uint8_t *codes = static_cast<const uint8_t *>(packed);
-    const uint8_t *scales = codes + (size_t)N * K / 2;
-    const int gpk = std::max(1, BK / G);
-    if (!x_map(&xm, X, M, K, pl.bm) ||
-        // codes: rows = n32 tiles of 2K u64 words (K/64 chunks of 1 KB); box = one chunk x 4 tiles
-        !encode_tensor_map_2d(&wm, CU_TENSOR_MAP_DATA_TYPE_UINT64, codes, (uint64_t)K * 2,
-                              (uint64_t)(N / 32), (uint64_t)K * 16, 128, BW / 32,
-                              CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        // scales: rows = n32 tiles, K/G groups of 8 u64 words (64 bytes) per row
-        !encode_tensor_map_2d(&sm, CU_TENSOR_MAP_DATA_TYPE_UINT64, scales, (uint64_t)(K / G) * 8,
-                              (uint64_t)(N / 32), (uint64_t)(K / G) * 64, 8 * gpk, BW / 32,
-                              CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (!x_map(&xm, X, M, K, pl.bm))
         return cudaErrorInvalidValue;
     TcParams p{};
     p.Y = static_cast<uint16_t *>(Y);
     p.Ws = nullptr;
+    // weights are moved with bulk copies of the column-group layout
+    p.codes = codes;
+    p.scales = codes + (size_t)N * K / 2;
     p.hdr = static_cast<WsHeader *>(workspace);
     p.M = M;
     p.N = N;
@@ -778,9 +789,10 @@ cudaError_t launch_w4a16_tc(const TcPlan &pl, const void *X, const void *packed,
         p.counters = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + wsm.counters_off);
         p.partial = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + wsm.partial_off);
     }
+    // the weight tensor-map parameters are unused on the INT4 path
     if (pl.bm == 128)
-        return tc_launch<kInt4, 128>(pl, xm, wm, sm, p, stream);
-    return tc_launch<kInt4, 256>(pl, xm, wm, sm, p, stream);
+        return tc_launch<kInt4, 128>(pl, xm, xm, xm, p, stream);
+    return tc_launch<kInt4, 256>(pl, xm, xm, xm, p, stream);
 }
 
 bool plan_mxfp8_tc(int device, int M, int N, int K, TcPlan *plan)

@@ -1,42 +1,47 @@
 // INT4 W4A16 weight-streaming GEMM for small M (decode / MTP verify chunks).
 //
 // At M <= 32 the layer reads each weight byte once and does 2*M flops per
-// weight: it is bound by HBM bytes of W, and the whole design is about
-// keeping enough weight bytes in flight on every SM while the decode and the
-// MMAs run behind them.
+// weight: it is bound by HBM bytes of W, and the design is about keeping
+// enough weight bytes in flight on every SM while the decode and the MMAs
+// run behind them, with few, large copies.
 //
 //  * Columns are taken eight n32 tiles (256 columns) at a time, a "column
-//    group".  The weight stream of a group row is cut into units of
-//    max(KS, G) rows of K (KS = rows per pipeline stage), and every CTA of a
-//    one-CTA-per-SM grid takes one contiguous run of units (stream-K), so all
-//    SMs stream the same number of bytes.
-//  * One producer warp fills a CTA-wide ring of stages with 2-D tensor-map
-//    copies (TMA): per stage the codes of the eight tiles for KS rows of K
-//    (one box), their scales (one box) and the activations X for the same
-//    rows (64-wide boxes with 128-byte swizzle; rows past M are zero-filled by
-//    the copy).  Completion is an mbarrier per stage; the consumers release a
-//    stage through a second mbarrier.  Weights are marked evict-first in L2,
-//    the activations evict-last (every CTA re-reads them).
-//  * Eight consumer warps, warp w owning tile w of the group for the whole
-//    K range of the CTA's segment: no reduction between warps.  Each warp
-//    decodes a pair of nibbles to the bf16 pair (128 + q) with one
-//    mask-and-or (plus a shift) and multiplies on the tensor cores with
-//    m16n8k16 MMAs where the weights are the 16-row operand and the tokens
-//    the 8-column operand ("swap AB"); one more MMA with an all-ones weight
-//    tile gives the per-token activation sum that turns (128 + q) into
-//    (q - 8).  A zero-initialised partial sum per scale group is folded in
-//    as acc += (part - 136 * activation sum) * scale in fp32, so weights are
+//    group" of the re-packed layout (common.cuh), in which the codes of a
+//    group for 128 rows of K are one contiguous 16 KB range and their scales
+//    one contiguous range.  The stream of a group row is cut into units of
+//    128 rows (one pipeline stage).  With fewer group rows than SMs (the
+//    decode layers), every row is split into S equal pieces, one CTA each,
+//    so every CTA has one segment and the pieces of a row end together;
+//    with more rows, every CTA of a one-CTA-per-SM grid takes one contiguous
+//    run of units across rows (stream-K).  Either way all SMs stream about
+//    the same number of bytes.
+//  * One producer thread fills a CTA-wide ring of stages with two 1-D bulk
+//    copies per stage (codes, scales), completion on an mbarrier per stage;
+//    the consumers release a stage through a second mbarrier.  Weights are
+//    marked evict-first in L2.
+//  * The activations X of the CTA's run (the k ranges of its at most two
+//    group-row segments, or all of K when the run spans more rows) are
+//    copied into shared memory once, one bulk copy per row and range, and
+//    the per-group activation sums are formed once from them (one all-ones
+//    MMA per 16 rows of K).  When they do not fit beside the ring (wide
+//    token tiles, long runs) every stage also carries its activations (2-D
+//    tensor-map boxes with 128-byte swizzle) and every warp forms the sums
+//    with its own all-ones MMAs.
+//  * Consumer warps own tiles: warp w (and, for M <= 16, warp w + 8, the two
+//    taking alternate stages) owns tile w of the group for the whole K range
+//    of the CTA's segment, so no warp reduces against another except the
+//    pair at a segment end.  Each warp decodes a pair of nibbles to the bf16
+//    pair (128 + q) with one mask-and-or (plus a shift) and multiplies on the
+//    tensor cores with m16n8k16 MMAs where the weights are the 16-row operand
+//    and the tokens the 8-column operand ("swap AB").  A zero-initialised
+//    partial sum per scale group is folded in as
+//    acc += (part - 136 * activation sum) * scale in fp32, so weights are
 //    never rounded (every product is exact in fp32).
 //  * A group row cut between CTAs is finished by the CTA holding its first
 //    unit, which reaches it last in its run; the other contributors (for
 //    whom it is the first segment of their run) publish their fragments
 //    early, so the finisher adds them in CTA order (deterministic) and
 //    writes bf16 Y.  A group row inside one run is written directly.
-//  * The footprint (9 warps, <= 112 registers for M <= 16, ~100 KB of shared
-//    memory) lets two CTAs share an SM: the next GEMM on the stream (launched
-//    with programmatic dependent launch) becomes resident while this one
-//    streams, issues its first weight copies and warms L2 with the next part
-//    of its run, and only then waits for this grid before reading X.
 //
 // The same kernel runs INT8 W8A16 weights (the vocabulary head): their
 // re-pack splits each 8-bit code q = 16 hi + lo into a plane of low and a
@@ -52,23 +57,21 @@
 namespace mxg {
 namespace {
 
-#ifndef MXG_STREAM_KS
-#define MXG_STREAM_KS 64
+#ifndef MXG_STREAM_PF_STAGES
+#define MXG_STREAM_PF_STAGES 8
 #endif
-#ifndef MXG_STREAM_RING_KB
-#define MXG_STREAM_RING_KB 104
-#endif
-#ifndef MXG_STREAM_RING2_KB
-#define MXG_STREAM_RING2_KB 192
+#ifndef MXG_STREAM_MAX_RING_KB
+#define MXG_STREAM_MAX_RING_KB 200
 #endif
 #ifndef MXG_STREAM_WPT2_MAX_TT
-#define MXG_STREAM_WPT2_MAX_TT 0
-#endif
-#ifndef MXG_STREAM_PF_STAGES
-#define MXG_STREAM_PF_STAGES 12
+#define MXG_STREAM_WPT2_MAX_TT 2
 #endif
 
-constexpr int kWarps = 8;                     // n32 tiles of a column group
+constexpr int kWarps = 8;          // n32 tiles of a column group
+constexpr int kKS = 128;           // rows of K per stage (= per stream-K unit)
+constexpr int kChunks = kKS / 64;  // k64 chunks per stage
+constexpr int kXPad = 16;          // bf16 columns of padding per resident activation row
+constexpr int kMaxSmem = 227 * 1024;
 
 // Consumer warps per tile: two for narrow token tiles (each takes every
 // other stage of the run, so a warp has two stages' time for the latency
@@ -79,67 +82,103 @@ struct Wpt {
 };
 
 // Group modes: 0 -> G = 128, 1 -> G = 64, 2 -> G = 32.  P code planes: 1 for
-// INT4; 2 for INT8 (low and high nibbles, each in the INT4 layout).
-template <int TT, int GM, int P>
+// INT4; 2 for INT8 (low and high nibbles, each in the INT4 layout).  XR: the
+// activations are resident for the whole run (1) or carried by every stage (0).
+template <int TT, int GM, int P, int XR>
 struct Cfg {
     static constexpr int kWPT = Wpt<TT>::value;
     static constexpr int kConsumers = kWarps * kWPT;
     static constexpr int kThreads = (kConsumers + 1) * 32;         // + the producer warp
     static constexpr int kProducer = kConsumers;                   // its warp index
-    // one CTA per SM with two consumer warps per tile; with one, the ring
-    // leaves room for a second CTA (the next GEMM on the stream)
-    static constexpr int kRingBytes = (kWPT == 2 ? MXG_STREAM_RING2_KB : MXG_STREAM_RING_KB) * 1024;
     static constexpr int kG = GM == 0 ? 128 : (GM == 1 ? 64 : 32);
-    static constexpr int kKS = P == 2 ? 64 : MXG_STREAM_KS;       // rows of K per stage
-    static constexpr int kChunks = kKS / 64;                       // k64 chunks per stage
-    static constexpr int kSteps = kKS / 16;                        // k16 MMA steps per stage
     static constexpr int kStepsPerGroup = kG / 16;
-    // steps between scale epilogues: a group, or a stage when a group spans
-    // stages that different warps take
-    static constexpr int kEpi = (kWPT == 2 && kStepsPerGroup > kSteps) ? kSteps : kStepsPerGroup;
-    static constexpr int kUS = kG > kKS ? kG / kKS : 1;            // stages per stream-K unit
-    static constexpr int kUnitK = kUS * kKS;                       // rows of K per unit
-    static constexpr int kScaleGroups = kKS >= kG ? kKS / kG : 1;  // groups in a stage's scale box
-    static constexpr int kCodeTile = kChunks * 1024 * P;           // code bytes of a tile per stage
-    static constexpr int kCode = kWarps * kCodeTile;
+    static constexpr int kGroupsPerStage = kKS / kG;
     static constexpr int kXBox = 128 * 8 * TT;                     // 64 k x 8TT rows of bf16
-    static constexpr int kX = kChunks * kXBox;
-    static constexpr int kScaleTile = 64 * kScaleGroups;
-    static constexpr int kScale = kWarps * kScaleTile;
-    static constexpr int kTx = kX + kCode + kScale;                // bytes landing per stage
-    static constexpr int kStage = (kTx + 1023) / 1024 * 1024;      // X boxes stay 1024-aligned
-    static constexpr int kStages = kRingBytes / kStage > 3 ? kRingBytes / kStage : 3;
+    static constexpr int kX = XR ? 0 : kChunks * kXBox;           // staged activations
+    static constexpr int kCodeMax = kChunks * kWarps * 1024 * P;   // codes of a full group
+    static constexpr int kScaleMax = kGroupsPerStage * kWarps * 64;
+    static constexpr int kStage = XR ? (kX + kCodeMax + kScaleMax + 127) / 128 * 128
+                                     : (kX + kCodeMax + kScaleMax + 1023) / 1024 * 1024;
     static constexpr int kF = 2 * TT;                              // float4 per lane fragment
-    // fragments the second warp of a tile hands to the first at a segment end
-    static constexpr int kXchgOff = kStages * kStage;
     static constexpr int kXchg = kWPT == 2 ? kWarps * kF * 32 * 16 : 0;
-    static constexpr int kBarOff = kXchgOff + kXchg;
-    static constexpr size_t kSmem = (size_t)kBarOff + 2 * kStages * 8 + 1024;  // + alignment
 };
 
 struct Params {
+    const uint16_t *X;       // bf16 [M][K]
+    const uint8_t *codes;    // re-packed codes (column-group layout)
+    const uint8_t *scales;   // re-packed scales
     uint16_t *Y;             // bf16 [M][N]
     WsHeader *hdr;
     int *counters;           // [column groups * 8]
-    float4 *partial;         // [ctas][8 warps][2*TT][32]: a CTA's fragments of its first, cut group row
-    int M, N;
+    float4 *partial;         // [ctas][8 tiles][2*TT][32]: a CTA's fragments of its first, cut group row
+    int M, N, K;
     int ntiles;              // N / 32
-    int upr;                 // units per group row
-    int q, r;                // units = q * ctas + r: CTAs below r run q + 1 units, the rest q
+    int upr;                 // units (stages) per group row: ceil(K / 128)
+    int q, r;                // stream-K: units = q * ctas + r: CTAs below r run q + 1 units
+    int S;                   // pieces per group row (row split), or 0 (stream-K)
+    int R;                   // ring stages
+    int x_off, xs_off, xchg_off, bar_off;   // shared-memory regions (bytes from the base)
     int early;               // load the first weights before waiting for the previous kernel
     int pf_stages;           // stages after the ring warmed in L2 at entry
 };
 
-__device__ __forceinline__ int run_start(const Params &p, int c)
+// First unit of CTA c's run: piece c % S of row c / S (row split), or
+// stream-K's c-th run (CTAs below r run q + 1 units, the rest q).  c may be
+// the CTA count (the end of the last run).
+__host__ __device__ __forceinline__ int run_start(int q, int r, int S, int upr, int c)
 {
-    return c * p.q + min(c, p.r);
+    if (S > 0)
+        return (c / S) * upr + (c % S) * upr / S;
+    return c * q + (c < r ? c : r);
 }
 
 // The CTA whose run contains unit u.
 __device__ __forceinline__ int cta_of_unit(const Params &p, int u)
 {
+    if (p.S > 0) {
+        const int row = u / p.upr, o = u - row * p.upr;
+        int i = (o * p.S) / p.upr;   // piece i covers [i * upr / S, (i + 1) * upr / S)
+        while (i + 1 < p.S && (i + 1) * p.upr / p.S <= o)
+            ++i;
+        while (i > 0 && i * p.upr / p.S > o)
+            --i;
+        return row * p.S + i;
+    }
     const int big = p.r * (p.q + 1);   // units covered by the longer runs
     return u < big ? u / (p.q + 1) : p.r + (u - big) / p.q;
+}
+
+// The resident activation windows of the run [U0, U1): one per segment
+// (group row) when the run touches at most two rows and the two ranges are
+// shorter than K together, else one window [0, K) for every segment.
+struct XWindows {
+    int n;                   // windows
+    int klo[2], cols[2];     // k range of each window
+    bool fullk;
+};
+
+__host__ __device__ inline XWindows x_windows(int U0, int U1, int upr, int K)
+{
+    XWindows w{};
+    const int row0 = U0 / upr, row1 = (U1 - 1) / upr;
+    int cols = 0;
+    if (row1 - row0 <= 1) {
+        for (int rr = row0, i = 0; rr <= row1; ++rr, ++i) {
+            const int a = (U0 > rr * upr ? U0 : rr * upr) - rr * upr;
+            const int b = (U1 < (rr + 1) * upr ? U1 : (rr + 1) * upr) - rr * upr;
+            w.klo[i] = a * kKS;
+            w.cols[i] = (b * kKS < K ? b * kKS : K) - a * kKS;
+            cols += w.cols[i];
+        }
+        w.n = row1 - row0 + 1;
+    }
+    if (row1 - row0 > 1 || cols >= K) {
+        w.n = 1;
+        w.klo[0] = 0;
+        w.cols[0] = K;
+        w.fullk = true;
+    }
+    return w;
 }
 
 // Writes the four outputs of fragment float4 j (= h * TT + tt) of `lane`.
@@ -161,45 +200,53 @@ __device__ __forceinline__ void store_y4(const Params &p, int tile, int j, int l
 }
 
 // ------------------------------------------------------------------ producer
-template <int TT, int GM, int P>
-__device__ __forceinline__ void produce(const Params &p, const CUtensorMap *cmap,
-                                        const CUtensorMap *smap, const CUtensorMap *xmap,
-                                        uint8_t *ring, uint64_t *full, uint64_t *empty, int S0,
+template <int TT, int GM, int P, int XR>
+__device__ __forceinline__ void produce(const Params &p, const CUtensorMap *xmap, uint8_t *smem,
+                                        uint64_t *full, uint64_t *empty, uint64_t *xbar, int U0,
                                         int ns)
 {
-    using C = Cfg<TT, GM, P>;
-    constexpr int R = C::kStages;
-    const int spr = p.upr * C::kUS;   // stages per group row
+    using C = Cfg<TT, GM, P, XR>;
+    const int R = p.R;
+    const int K = p.K;
     const uint64_t pol_w = l2_policy_evict_first();
     const uint64_t pol_x = l2_policy_evict_last();
-    prefetch_tensormap(cmap);
-    prefetch_tensormap(smap);
-    prefetch_tensormap(xmap);
-    // box coordinates of run stage s: codes x (u64), group row y (tiles), first k
-    auto coords = [&](int s, int &cx, int &sx, int &ty, int &k0) {
-        const int a = S0 + s;
-        const int gr = a / spr, ks = a - gr * spr;
-        k0 = ks * C::kKS;
-        cx = ks * (C::kCodeTile / 8);
-        sx = (k0 / C::kG) * 8;
-        ty = gr * kWarps;
+    if (!XR)
+        prefetch_tensormap(xmap);
+    // source ranges of run stage s
+    struct Src {
+        const uint8_t *codes, *scales;
+        uint32_t code_bytes, scale_bytes;
+        int k0;
+    };
+    auto source = [&](int s) {
+        const int a = U0 + s;
+        const int gr = a / p.upr, ks = a - gr * p.upr;
+        const int nt = group_tiles(gr, p.ntiles);
+        Src src;
+        src.k0 = ks * kKS;
+        const int nch = K - src.k0 >= kKS ? kChunks : (K - src.k0) / 64;
+        const int ngs = (nch * 64 + C::kG - 1) / C::kG;
+        src.codes = p.codes + (size_t)gr * kWarps * 16 * K * P + (size_t)ks * kChunks * nt * 1024 * P;
+        src.scales = p.scales + (size_t)gr * kWarps * (K / C::kG) * 64 +
+                     (size_t)(src.k0 / C::kG) * nt * 64;
+        src.code_bytes = (uint32_t)(nch * nt * 1024 * P);
+        src.scale_bytes = (uint32_t)(ngs * nt * 64);
+        return src;
     };
     auto issue_w = [&](int s) {
-        int cx, sx, ty, k0;
-        coords(s, cx, sx, ty, k0);
-        uint8_t *st = ring + (size_t)(s % R) * C::kStage;
+        const Src src = source(s);
+        uint8_t *st = smem + (size_t)(s % R) * C::kStage;
         uint64_t *bar = &full[s % R];
-        mbar_arrive_expect_tx(bar, C::kTx);
-        tma_load_2d(st + C::kX, cmap, cx, ty, bar, pol_w);
-        tma_load_2d(st + C::kX + C::kCode, smap, sx, ty, bar, pol_w);
+        mbar_arrive_expect_tx(bar, src.code_bytes + src.scale_bytes + (XR ? 0 : C::kX));
+        bulk_g2s(st + C::kX, src.codes, src.code_bytes, bar, pol_w);
+        bulk_g2s(st + C::kX + C::kCodeMax, src.scales, src.scale_bytes, bar, pol_w);
     };
-    auto issue_x = [&](int s) {
-        int cx, sx, ty, k0;
-        coords(s, cx, sx, ty, k0);
-        uint8_t *st = ring + (size_t)(s % R) * C::kStage;
+    auto issue_x = [&](int s) {   // staged activations of stage s
+        const Src src = source(s);
+        uint8_t *st = smem + (size_t)(s % R) * C::kStage;
 #pragma unroll
-        for (int ch = 0; ch < C::kChunks; ++ch)
-            tma_load_2d(st + ch * C::kXBox, xmap, k0 + 64 * ch, 0, &full[s % R], pol_x);
+        for (int ch = 0; ch < kChunks; ++ch)
+            tma_load_2d(st + ch * C::kXBox, xmap, src.k0 + 64 * ch, 0, &full[s % R], pol_x);
     };
     const int first = min(R, ns);
     // Weights are not written by the previous kernel on the stream (the
@@ -210,17 +257,33 @@ __device__ __forceinline__ void produce(const Params &p, const CUtensorMap *cmap
             issue_w(s);
     const int pf_end = min(ns, R + p.pf_stages);
     for (int s = R; s < pf_end; ++s) {
-        int cx, sx, ty, k0;
-        coords(s, cx, sx, ty, k0);
-        prefetch_tensor_l2(cmap, cx, ty);
-        prefetch_tensor_l2(smap, sx, ty);
+        const Src src = source(s);
+        prefetch_l2(src.codes, src.code_bytes);
     }
     pdl_wait();
     if (!p.early)
         for (int s = 0; s < first; ++s)
             issue_w(s);
-    for (int s = 0; s < first; ++s)
-        issue_x(s);
+    if (XR) {
+        // the run's activations, one bulk copy per row and window
+        const XWindows xw = x_windows(U0, U0 + ns, p.upr, K);
+        const int rows = min(p.M, 8 * TT);
+        uint32_t bytes = 0;
+        for (int w = 0; w < xw.n; ++w)
+            bytes += (uint32_t)rows * xw.cols[w] * 2;
+        mbar_arrive_expect_tx(xbar, bytes);
+        uint32_t base = p.x_off;
+        for (int w = 0; w < xw.n; ++w) {
+            const uint32_t stride = (xw.cols[w] + kXPad) * 2;
+            for (int m = 0; m < rows; ++m)
+                bulk_g2s(smem + base + m * stride, p.X + (size_t)m * K + xw.klo[w],
+                         (uint32_t)xw.cols[w] * 2, xbar, pol_x);
+            base += 8 * TT * stride;
+        }
+    } else {
+        for (int s = 0; s < first; ++s)
+            issue_x(s);
+    }
     int issued = first;
     for (int s = first; s < ns; ++s) {
         // stage s reuses the slot of stage s - R: its release is phase
@@ -230,7 +293,8 @@ __device__ __forceinline__ void produce(const Params &p, const CUtensorMap *cmap
             break;
         }
         issue_w(s);
-        issue_x(s);
+        if (!XR)
+            issue_x(s);
         issued = s + 1;
     }
     // every copy this CTA issued has landed before it exits (the consumers
@@ -238,24 +302,26 @@ __device__ __forceinline__ void produce(const Params &p, const CUtensorMap *cmap
     for (int s = max(0, issued - R); s < issued; ++s)
         if (!mbar_wait(&full[s % R], (uint32_t)((s / R) & 1), kWaitLimitNs))
             record_error(p.hdr, MXG_ERR_TIMEOUT, 150 + GM);
+    if (XR && !mbar_wait(xbar, 0, kWaitLimitNs))
+        record_error(p.hdr, MXG_ERR_TIMEOUT, 160 + GM);
 }
 
 // ----------------------------------------------------------------- finisher
-// Run by warp `warp` of a CTA whose segment of group row `gr` is cut (the
-// row goes on in other CTAs' runs), with the warp's fragment in `sum`.  The
-// CTA whose run holds the row's first unit finishes that segment last in its
-// run: it adds the other contributors' fragments (in CTA order) to its own
-// and writes bf16 Y.  Every other contributor (its segment is the first one
-// of its run) publishes its fragment and bumps the tile's counter without
-// waiting for anybody.
+// Run by the warp owning tile slot `wt` of a CTA whose segment of group row
+// `gr` is cut (the row goes on in other CTAs' runs), with the warp's fragment
+// in `sum`.  The CTA whose run holds the row's first unit finishes that
+// segment last in its run: it adds the other contributors' fragments (in CTA
+// order) to its own and writes bf16 Y.  Every other contributor (its segment
+// is the first one of its run) publishes its fragment and bumps the tile's
+// counter without waiting for anybody.
 template <int TT>
 __device__ __forceinline__ void finish_cut(const Params &p, float4 (&sum)[2 * TT], int c, int gr,
-                                        int warp, int lane)
+                                           int wt, int lane)
 {
     constexpr int F = 2 * TT;
-    const int tile = gr * kWarps + warp;
+    const int tile = gr * kWarps + wt;
     const int c_first = cta_of_unit(p, gr * p.upr);
-    float4 *mine = p.partial + ((size_t)c * kWarps + warp) * F * 32;
+    float4 *mine = p.partial + ((size_t)c * kWarps + wt) * F * 32;
     if (c != c_first) {
 #pragma unroll
         for (int j = 0; j < F; ++j)
@@ -280,7 +346,7 @@ __device__ __forceinline__ void finish_cut(const Params &p, float4 (&sum)[2 * TT
     }
     __syncwarp();
     for (int cc = c_first + 1; cc <= c_last; ++cc) {
-        const float4 *src = p.partial + ((size_t)cc * kWarps + warp) * F * 32;
+        const float4 *src = p.partial + ((size_t)cc * kWarps + wt) * F * 32;
 #pragma unroll
         for (int j = 0; j < F; ++j) {
             const float4 f = __ldcg(src + j * 32 + lane);
@@ -299,39 +365,38 @@ __device__ __forceinline__ void finish_cut(const Params &p, float4 (&sum)[2 * TT
 }
 
 // ------------------------------------------------------------------- kernel
-template <int TT, int GM, int P>
-__global__ void __launch_bounds__(Cfg<TT, GM, P>::kThreads,
-                                  Cfg<TT, GM, P>::kWPT == 1 && TT <= 2 ? 2 : 1)
-    w4a16_stream_kernel(const __grid_constant__ CUtensorMap cmap,
-                        const __grid_constant__ CUtensorMap smap,
-                        const __grid_constant__ CUtensorMap xmap, const Params p)
+template <int TT, int GM, int P, int XR>
+__global__ void __launch_bounds__(Cfg<TT, GM, P, XR>::kThreads, 1)
+    w4a16_stream_kernel(const __grid_constant__ CUtensorMap xmap, const Params p)
 {
-    using C = Cfg<TT, GM, P>;
-    constexpr int R = C::kStages;
+    using C = Cfg<TT, GM, P, XR>;
     constexpr int F = C::kF;
+    constexpr uint32_t kOnes = 0x3F803F80u;  // bf16 pair (1, 1)
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the swizzled activation boxes
-    uint8_t *ring = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-    uint64_t *full = reinterpret_cast<uint64_t *>(ring + C::kBarOff);
+    uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    const int R = p.R;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.bar_off);
     uint64_t *empty = full + R;
+    uint64_t *xbar = empty + R;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_launch_dependents();
     const int c = blockIdx.x;
-    const int U0 = run_start(p, c), U1 = run_start(p, c + 1);
-    const int S0 = U0 * C::kUS;
-    const int ns = (U1 - U0) * C::kUS;
+    const int U0 = run_start(p.q, p.r, p.S, p.upr, c), U1 = run_start(p.q, p.r, p.S, p.upr, c + 1);
+    const int ns = U1 - U0;
     if (threadIdx.x == 0) {
         for (int s = 0; s < R; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kWarps);   // one warp of each tile takes a stage
         }
+        mbar_init(xbar, 1);
         fence_barrier_init();
     }
     __syncthreads();
     if (warp == C::kProducer) {
         if (lane == 0)
-            produce<TT, GM, P>(p, &cmap, &smap, &xmap, ring, full, empty, S0, ns);
+            produce<TT, GM, P, XR>(p, &xmap, smem, full, empty, xbar, U0, ns);
         return;
     }
 
@@ -340,23 +405,81 @@ __global__ void __launch_bounds__(Cfg<TT, GM, P>::kThreads,
     const int g = lane >> 2, t = lane & 3;
     const int wt = warp % kWarps;        // this warp's tile in the column group
     const int parity = warp / kWarps;    // which stages of the run it takes
-    // swizzled offsets of this lane's activations inside a 64-k box: row
-    // 8 tt + g, bytes 32 j + 8 t of the row; the 16-byte chunk index is
+    const uint32_t sb = smem_u32(smem);  // shared-window address of the base
+    bool ok = true;
+
+    // resident activations: windows, and the per-group activation sums
+    // (table [group of the windows][8 TT tokens], fp32)
+    XWindows xw{};
+    if constexpr (XR != 0) {
+        xw = x_windows(U0, U1, p.upr, p.K);
+        if (!mbar_wait(xbar, 0, kWaitLimitNs)) {
+            if (lane == 0)
+                record_error(p.hdr, MXG_ERR_TIMEOUT, 110 + GM);
+            ok = false;
+        }
+        // entry e = (group of the windows, token tile): one all-ones MMA per
+        // 16 rows of K; lanes 0..3 hold the sums of tokens 2t, 2t+1
+        const int ngr0 = xw.cols[0] / C::kG;
+        const int ngr1 = xw.n > 1 ? xw.cols[1] / C::kG : 0;
+        const int entries = (ngr0 + ngr1) * TT;
+        const uint32_t stride0 = (xw.cols[0] + kXPad) * 2;
+        for (int e = warp; e < entries; e += C::kConsumers) {
+            const int gi = e / TT, tt = e % TT;
+            const int w = gi < ngr0 ? 0 : 1;
+            const int gl = gi - (w ? ngr0 : 0);
+            const uint32_t base = p.x_off + (w ? 8 * TT * stride0 : 0);
+            const uint32_t stride = ((w ? xw.cols[1] : xw.cols[0]) + kXPad) * 2;
+            const uint32_t row = sb + base + (8 * tt + g) * stride + (gl * C::kG + 4 * t) * 2;
+            float a[4];
+#pragma unroll
+            for (int j = 0; j < C::kStepsPerGroup; ++j) {
+                const uint2 b = lds64a(row + 32 * j);
+                if (j == 0)
+                    mma_bf16_16816_zero(a, kOnes, kOnes, kOnes, kOnes, b.x, b.y);
+                else
+                    mma_bf16_16816(a, kOnes, kOnes, kOnes, kOnes, b.x, b.y);
+            }
+            if (g == 0)
+                *reinterpret_cast<float2 *>(smem + p.xs_off + (gi * 8 * TT + 8 * tt + 2 * t) * 4) =
+                    make_float2(a[0], a[1]);
+        }
+        named_bar_sync(9, C::kConsumers * 32);   // the table is complete
+    }
+    // swizzled offsets of this lane's activations inside a staged 64-k box:
+    // row 8 tt + g, bytes 32 j + 8 t of the row; the 16-byte chunk index is
     // XORed with the row modulo 8 by the 128-byte swizzle
     uint32_t xoff[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j)
         xoff[j] = g * 128 + (((2 * j + (t >> 1)) ^ g) << 4) + 8 * (t & 1);
 
-    constexpr uint32_t kOnes = 0x3F803F80u;  // bf16 pair (1, 1)
     float acc[2][TT][4], part[2][TT][4], xsum[TT][4];
     float parthi[P == 2 ? 2 : 1][TT][4];  // INT8: sums over the high-nibble plane
-    bool ok = true;
-    int s = 0;   // run stage
-    for (int u = U0; u < U1;) {
-        const int gr = u / p.upr;
-        const int seg_begin = u;
+    // this warp's stages of the run: s = parity, parity + WPT, ...; the ring
+    // slot and phase of stage s follow it incrementally
+    int s = parity;
+    int slot = parity;
+    uint32_t phase = 0;
+    int seg = 0;
+    for (int seg_begin = U0; seg_begin < U1; ++seg) {
+        const int gr = seg_begin / p.upr;
         const int seg_end = min(U1, (gr + 1) * p.upr);
+        const int nt = group_tiles(gr, p.ntiles);
+        const bool live = wt < nt;           // a last group may hold fewer tiles
+        // resident window of this segment: the shared-memory address of this
+        // lane's token row at k = 0 of the row and the stride between token
+        // rows; the table row of the segment's k = 0
+        uint32_t xrow = 0, xstride = 0;
+        int xg0 = 0;
+        if constexpr (XR != 0) {
+            const int w = xw.fullk ? 0 : seg;
+            const int xklo = w ? xw.klo[1] : xw.klo[0];
+            const uint32_t stride0 = (xw.cols[0] + kXPad) * 2;
+            xstride = ((w ? xw.cols[1] : xw.cols[0]) + kXPad) * 2;
+            xrow = sb + p.x_off + (w ? 8 * TT * stride0 : 0) + g * xstride + 8 * t - xklo * 2;
+            xg0 = (w ? xw.cols[0] / C::kG : 0) - xklo / C::kG;
+        }
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -364,62 +487,66 @@ __global__ void __launch_bounds__(Cfg<TT, GM, P>::kThreads,
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
                     acc[h][tt][e] = 0.f;
-        for (; u < seg_end; ++u) {
+        for (; U0 + s < seg_end; s += C::kWPT) {
+            const int k0 = (U0 + s - gr * p.upr) * kKS;   // first row of K of the stage
+            if (!mbar_wait(&full[slot], phase, ok ? kWaitLimitNs : 0)) {
+                if (ok && lane == 0)
+                    record_error(p.hdr, MXG_ERR_TIMEOUT, 100 + GM);
+                ok = false;
+            }
+            const uint32_t st = sb + slot * C::kStage;
+            const uint32_t cs = st + C::kX + wt * 1024 * P + lane * 16;
+            const uint32_t ss = st + C::kX + C::kCodeMax + wt * 64 + g * 8;
+            if (live) {
 #pragma unroll
-            for (int su = 0; su < C::kUS; ++su, ++s) {
-                if (C::kWPT == 2 && (s & 1) != parity)
-                    continue;   // the other warp of the tile takes this stage
-                const int slot = s % R;
-                if (!mbar_wait(&full[slot], (uint32_t)((s / R) & 1), ok ? kWaitLimitNs : 0)) {
-                    if (ok && lane == 0)
-                        record_error(p.hdr, MXG_ERR_TIMEOUT, 100 + GM);
-                    ok = false;
-                }
-                const uint8_t *st = ring + (size_t)slot * C::kStage;
-                const uint8_t *cs = st + C::kX + wt * C::kCodeTile;
-                const uint8_t *ss = st + C::kX + C::kCode + wt * C::kScaleTile;
-#pragma unroll
-                for (int ch = 0; ch < C::kChunks; ++ch) {
+                for (int ch = 0; ch < kChunks; ++ch) {
+                    if (ch > 0 && k0 + 64 * ch >= p.K)
+                        break;   // the last stage of a row may hold one chunk
                     // INT4: [half][lane][16 B]; INT8: [half][plane][lane][16 B]
-                    const uint8_t *cp = cs + ch * 1024 * P + lane * 16;
-                    const uint4 wl = lds128(cp);
-                    const uint4 wh = lds128(cp + 512 * P);
-                    const uint32_t w[2][4] = {{wl.x, wl.y, wl.z, wl.w}, {wh.x, wh.y, wh.z, wh.w}};
+                    const uint32_t cp = cs + ch * nt * 1024 * P;
+                    const uint4 wl = lds128a(cp);
+                    const uint4 wh = lds128a(cp + 512 * P);
+                    const uint32_t wv[2][4] = {{wl.x, wl.y, wl.z, wl.w}, {wh.x, wh.y, wh.z, wh.w}};
                     uint32_t whi[2][4] = {};
                     if constexpr (P == 2) {
-                        const uint4 ul = lds128(cp + 512);
-                        const uint4 uh = lds128(cp + 1536);
+                        const uint4 ul = lds128a(cp + 512);
+                        const uint4 uh = lds128a(cp + 1536);
                         whi[0][0] = ul.x; whi[0][1] = ul.y; whi[0][2] = ul.z; whi[0][3] = ul.w;
                         whi[1][0] = uh.x; whi[1][1] = uh.y; whi[1][2] = uh.z; whi[1][3] = uh.w;
                     }
-                    const uint8_t *xb = st + ch * C::kXBox;
+                    const uint32_t xk = xrow + (k0 + 64 * ch) * 2;   // resident: k of the chunk
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        // k16 step inside the unit (one warp) or the stage (two)
-                        const int gstep = (C::kWPT == 1 ? su * C::kSteps : 0) + ch * 4 + j;
-                        const bool first = (gstep % C::kEpi) == 0;
-                        const bool last = ((gstep + 1) % C::kEpi) == 0;
+                        const int step = ch * 4 + j;   // k16 step inside the stage
+                        const bool first = (step % C::kStepsPerGroup) == 0;
+                        const bool last = ((step + 1) % C::kStepsPerGroup) == 0;
                         uint2 xf[TT];
 #pragma unroll
-                        for (int tt = 0; tt < TT; ++tt)
-                            xf[tt] = lds64(xb + tt * 1024 + xoff[j]);
-#pragma unroll
                         for (int tt = 0; tt < TT; ++tt) {
-                            // per token: the sum of the step's activations (an
-                            // MMA with an all-ones weight tile)
-                            if (first)
-                                mma_bf16_16816_zero(xsum[tt], kOnes, kOnes, kOnes, kOnes, xf[tt].x,
-                                                    xf[tt].y);
+                            if constexpr (XR != 0)
+                                xf[tt] = lds64a(xk + tt * 8 * xstride + 32 * j);
                             else
-                                mma_bf16_16816(xsum[tt], kOnes, kOnes, kOnes, kOnes, xf[tt].x,
-                                               xf[tt].y);
+                                xf[tt] = lds64a(st + ch * C::kXBox + tt * 1024 + xoff[j]);
+                        }
+                        if constexpr (XR == 0) {
+#pragma unroll
+                            for (int tt = 0; tt < TT; ++tt) {
+                                // per token: the sum of the step's activations
+                                // (an MMA with an all-ones weight tile)
+                                if (first)
+                                    mma_bf16_16816_zero(xsum[tt], kOnes, kOnes, kOnes, kOnes,
+                                                        xf[tt].x, xf[tt].y);
+                                else
+                                    mma_bf16_16816(xsum[tt], kOnes, kOnes, kOnes, kOnes,
+                                                   xf[tt].x, xf[tt].y);
+                            }
                         }
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
-                            const uint32_t a0 = int4_pair_plus128<0>(w[h][j]);
-                            const uint32_t a1 = int4_pair_plus128<4>(w[h][j]);
-                            const uint32_t a2 = int4_pair_plus128<8>(w[h][j]);
-                            const uint32_t a3 = int4_pair_plus128<12>(w[h][j]);
+                            const uint32_t a0 = int4_pair_plus128<0>(wv[h][j]);
+                            const uint32_t a1 = int4_pair_plus128<4>(wv[h][j]);
+                            const uint32_t a2 = int4_pair_plus128<8>(wv[h][j]);
+                            const uint32_t a3 = int4_pair_plus128<12>(wv[h][j]);
 #pragma unroll
                             for (int tt = 0; tt < TT; ++tt) {
                                 if (first)
@@ -448,14 +575,30 @@ __global__ void __launch_bounds__(Cfg<TT, GM, P>::kThreads,
                         if (last) {
                             // end of a scale group: the MMAs summed (128 + q) * x,
                             // so acc += (part - 136 * sum(x)) * scale, in fp32
-                            const int gi = C::kScaleGroups > 1 ? (ch * 4 + j) / C::kStepsPerGroup
-                                                               : 0;
-                            const uint2 sv = lds64(ss + gi * 64 + g * 8);
+                            const int gi = step / C::kStepsPerGroup;   // group in the stage
+                            const uint2 sv = lds64a(ss + gi * nt * 64);
                             const float2 s01 =
                                 __half22float2(*reinterpret_cast<const __half2 *>(&sv.x));
                             const float2 s23 =
                                 __half22float2(*reinterpret_cast<const __half2 *>(&sv.y));
                             const float sc[2][2] = {{s01.x, s01.y}, {s23.x, s23.y}};
+                            float2 xsv[TT];
+                            if constexpr (XR != 0) {
+                                // table row of the group: k0 / G + gi from the
+                                // segment's origin
+                                const uint32_t xa = sb + p.xs_off +
+                                                    ((xg0 + k0 / C::kG + gi) * 8 * TT + 2 * t) * 4;
+#pragma unroll
+                                for (int tt = 0; tt < TT; ++tt) {
+                                    const uint2 v = lds64a(xa + tt * 32);
+                                    xsv[tt] = make_float2(__uint_as_float(v.x),
+                                                          __uint_as_float(v.y));
+                                }
+                            } else {
+#pragma unroll
+                                for (int tt = 0; tt < TT; ++tt)
+                                    xsv[tt] = make_float2(xsum[tt][0], xsum[tt][1]);
+                            }
 #pragma unroll
                             for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -464,26 +607,32 @@ __global__ void __launch_bounds__(Cfg<TT, GM, P>::kThreads,
                                     for (int e = 0; e < 4; ++e) {
                                         // outputs e and e ^ 2 are rows g, g + 8 of
                                         // token 2t + (e & 1)
+                                        const float xe = (e & 1) ? xsv[tt].y : xsv[tt].x;
                                         float v;
                                         if constexpr (P == 2) {
                                             // INT8 q = 16 hi + lo: the planes summed
                                             // (128 + hi) x and (128 + lo) x, so
                                             // sum (q - 128) x = 16 Phi + Plo - 2304 sum(x)
                                             v = fmaf(16.f, parthi[h][tt][e], part[h][tt][e]);
-                                            v = fmaf(-2304.f, xsum[tt][e & 1], v);
+                                            v = fmaf(-2304.f, xe, v);
                                         } else {
-                                            v = fmaf(-136.f, xsum[tt][e & 1], part[h][tt][e]);
+                                            v = fmaf(-136.f, xe, part[h][tt][e]);
                                         }
                                         acc[h][tt][e] = fmaf(v, sc[h][e >> 1], acc[h][tt][e]);
                                     }
                         }
                     }
                 }
-                // every lane's reads of the stage have returned (their values
-                // are consumed above): release it to the producer
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&empty[slot]);
+            }
+            // every lane's reads of the stage have returned (their values
+            // are consumed above): release it to the producer
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&empty[slot]);
+            slot += C::kWPT;
+            if (slot >= R) {
+                slot -= R;
+                phase ^= 1;
             }
         }
 
@@ -495,10 +644,12 @@ __global__ void __launch_bounds__(Cfg<TT, GM, P>::kThreads,
             for (int tt = 0; tt < TT; ++tt)
                 sum[h * TT + tt] =
                     make_float4(acc[h][tt][0], acc[h][tt][1], acc[h][tt][2], acc[h][tt][3]);
+        const int seg_first = seg_begin;
+        seg_begin = seg_end;
         if constexpr (C::kWPT == 2) {
             // the tile's second warp hands its fragment to the first (a named
             // barrier per tile: ids 1..8, the tile's two warps)
-            float4 *xch = reinterpret_cast<float4 *>(ring + C::kXchgOff) + wt * F * 32;
+            float4 *xch = reinterpret_cast<float4 *>(smem + p.xchg_off) + wt * F * 32;
             if (parity == 1)
 #pragma unroll
                 for (int j = 0; j < F; ++j)
@@ -517,13 +668,12 @@ __global__ void __launch_bounds__(Cfg<TT, GM, P>::kThreads,
             if (parity == 1)
                 continue;
         }
-        const int tile = gr * kWarps + wt;
-        if (tile < p.ntiles) {
-            const bool whole = seg_begin == gr * p.upr && seg_end == (gr + 1) * p.upr;
+        if (live) {
+            const bool whole = seg_first == gr * p.upr && seg_end == (gr + 1) * p.upr;
             if (whole) {
 #pragma unroll
                 for (int j = 0; j < F; ++j)
-                    store_y4<TT>(p, tile, j, lane, sum[j]);
+                    store_y4<TT>(p, gr * kWarps + wt, j, lane, sum[j]);
             } else {
                 finish_cut<TT>(p, sum, c, gr, wt, lane);
             }
@@ -531,63 +681,74 @@ __global__ void __launch_bounds__(Cfg<TT, GM, P>::kThreads,
     }
 }
 
-template <int TT, int GM, int P>
+// variant = group mode + 3 * (INT8) + 6 * (resident activations)
+template <int TT, int V>
 const void *kernel_ptr()
 {
-    return reinterpret_cast<const void *>(&w4a16_stream_kernel<TT, GM, P>);
+    return reinterpret_cast<const void *>(&w4a16_stream_kernel<TT, V % 3, (V / 3) % 2 + 1, V / 6>);
 }
 
-// variant = group mode (INT4) or 3 + group mode (INT8)
 const void *select_kernel(int tt, int variant)
 {
 #define MXG_CASE(T, V) \
-    if (tt == T && variant == V) return kernel_ptr<T, V % 3, V / 3 + 1>();
+    if (tt == T && variant == V) return kernel_ptr<T, V>();
     MXG_CASE(1, 0) MXG_CASE(1, 1) MXG_CASE(1, 2) MXG_CASE(1, 3) MXG_CASE(1, 4) MXG_CASE(1, 5)
+    MXG_CASE(1, 6) MXG_CASE(1, 7) MXG_CASE(1, 8) MXG_CASE(1, 9) MXG_CASE(1, 10) MXG_CASE(1, 11)
     MXG_CASE(2, 0) MXG_CASE(2, 1) MXG_CASE(2, 2) MXG_CASE(2, 3) MXG_CASE(2, 4) MXG_CASE(2, 5)
+    MXG_CASE(2, 6) MXG_CASE(2, 7) MXG_CASE(2, 8) MXG_CASE(2, 9) MXG_CASE(2, 10) MXG_CASE(2, 11)
     MXG_CASE(3, 0) MXG_CASE(3, 1) MXG_CASE(3, 2) MXG_CASE(3, 3) MXG_CASE(3, 4) MXG_CASE(3, 5)
     MXG_CASE(4, 0) MXG_CASE(4, 1) MXG_CASE(4, 2) MXG_CASE(4, 3) MXG_CASE(4, 4) MXG_CASE(4, 5)
 #undef MXG_CASE
     return nullptr;
 }
 
-template <int TT>
-void cfg_of(int variant, size_t *smem, int *us, int *ks, int *code_tile, int *g, int *threads)
-{
-#define MXG_CFG(V)                                         \
-    if (variant == V) {                                    \
-        using C = Cfg<TT, V % 3, V / 3 + 1>;               \
-        *smem = C::kSmem;                                  \
-        *us = C::kUS;                                      \
-        *ks = C::kKS;                                      \
-        *code_tile = C::kCodeTile;                         \
-        *g = C::kG;                                        \
-        *threads = C::kThreads;                            \
-        return;                                            \
-    }
-    MXG_CFG(0) MXG_CFG(1) MXG_CFG(2) MXG_CFG(3) MXG_CFG(4) MXG_CFG(5)
-#undef MXG_CFG
-}
-
 struct VariantCfg {
-    size_t smem;
-    int us, ks, code_tile, g, threads;
+    int stage, xchg, threads, consumers, g, xbox;
 };
 
-VariantCfg variant_cfg(int tt, int variant)
+template <int TT, int V>
+VariantCfg cfg_one()
 {
-    VariantCfg v{};
-    switch (tt) {
-    case 1: cfg_of<1>(variant, &v.smem, &v.us, &v.ks, &v.code_tile, &v.g, &v.threads); break;
-    case 2: cfg_of<2>(variant, &v.smem, &v.us, &v.ks, &v.code_tile, &v.g, &v.threads); break;
-    case 3: cfg_of<3>(variant, &v.smem, &v.us, &v.ks, &v.code_tile, &v.g, &v.threads); break;
-    default: cfg_of<4>(variant, &v.smem, &v.us, &v.ks, &v.code_tile, &v.g, &v.threads); break;
-    }
-    return v;
+    using C = Cfg<TT, V % 3, (V / 3) % 2 + 1, V / 6>;
+    return {C::kStage, C::kXchg, C::kThreads, C::kConsumers, C::kG, C::kXBox};
+}
+
+VariantCfg variant_cfg(int tt, int v)
+{
+#define MXG_CFG(T, V) \
+    if (tt == T && v == V) return cfg_one<T, V>();
+    MXG_CFG(1, 0) MXG_CFG(1, 1) MXG_CFG(1, 2) MXG_CFG(1, 3) MXG_CFG(1, 4) MXG_CFG(1, 5)
+    MXG_CFG(1, 6) MXG_CFG(1, 7) MXG_CFG(1, 8) MXG_CFG(1, 9) MXG_CFG(1, 10) MXG_CFG(1, 11)
+    MXG_CFG(2, 0) MXG_CFG(2, 1) MXG_CFG(2, 2) MXG_CFG(2, 3) MXG_CFG(2, 4) MXG_CFG(2, 5)
+    MXG_CFG(2, 6) MXG_CFG(2, 7) MXG_CFG(2, 8) MXG_CFG(2, 9) MXG_CFG(2, 10) MXG_CFG(2, 11)
+    MXG_CFG(3, 0) MXG_CFG(3, 1) MXG_CFG(3, 2) MXG_CFG(3, 3) MXG_CFG(3, 4) MXG_CFG(3, 5)
+    MXG_CFG(4, 0) MXG_CFG(4, 1) MXG_CFG(4, 2) MXG_CFG(4, 3) MXG_CFG(4, 4) MXG_CFG(4, 5)
+#undef MXG_CFG
+    return {};
 }
 
 int group_mode(int G)
 {
     return G == 128 ? 0 : (G == 64 ? 1 : 2);
+}
+
+// Shared-memory regions of a launch: ring, then resident activations and
+// their sums, then the pair exchange, then the barriers.
+struct SmemPlan {
+    int R, x_off, xs_off, xchg_off, bar_off;
+    size_t total;
+};
+
+SmemPlan smem_plan(const VariantCfg &vc, int R, int xbytes, int xsbytes)
+{
+    SmemPlan s{};
+    s.R = R;
+    s.x_off = R * vc.stage;
+    s.xs_off = s.x_off + (xbytes + 127) / 128 * 128;
+    s.xchg_off = s.xs_off + (xsbytes + 127) / 128 * 128;
+    s.bar_off = s.xchg_off + vc.xchg;
+    s.total = (size_t)s.bar_off + (2 * R + 1) * 8 + 1024;   // + alignment
+    return s;
 }
 
 // bits: 4 (INT4) or 8 (INT8, two code planes)
@@ -600,48 +761,89 @@ bool plan_stream(int device, int M, int N, int K, int G, int bits, StreamPlan *p
     const DeviceInfo &di = device_info(device);
     StreamPlan pl{};
     pl.tt = (M + 7) / 8;
-    pl.variant = (bits == 8 ? 3 : 0) + group_mode(G);
-    const VariantCfg vc = variant_cfg(pl.tt, pl.variant);
-    pl.warps_per_cta = vc.threads / 32;
-    pl.smem = vc.smem;
-    if ((int)pl.smem > di.smem_optin)
-        return false;
-    const int unit_k = vc.us * vc.ks;
-    if (K % unit_k != 0)
-        return false;
-    pl.upt = K / unit_k;                      // units per group row
-    const int ngroups = (N / 32 + kWarps - 1) / kWarps;
-    pl.ntiles = ngroups * kWarps;             // arrival counters (one per tile slot)
+    const int ntiles = N / 32;
+    const int ngroups = (ntiles + kWarps - 1) / kWarps;
+    pl.upt = (K + kKS - 1) / kKS;                  // units (stages) per group row
+    pl.ntiles = ngroups * kWarps;                  // arrival counters (one per tile slot)
     if ((size_t)pl.ntiles > kMaxCounters)
         return false;
     pl.units = (long long)ngroups * pl.upt;
     if (pl.units > (1LL << 30))
         return false;
+    // fewer group rows than SMs: S pieces per row (at most one unit each);
+    // else stream-K with one CTA per SM, no run shorter than one unit
+    int S = 0;
+    if (ngroups < di.sms) {
+        S = std::min(di.sms / ngroups, pl.upt);
+        pl.Wt = ngroups * S;
+    } else {
+        pl.Wt = (int)std::max<long long>(1, std::min<long long>(di.sms, pl.units));
+    }
+    pl.grid = pl.Wt;
+    pl.split = S;
+    const int q = (int)(pl.units / pl.Wt), r = (int)(pl.units % pl.Wt);
+    const int base = (bits == 8 ? 3 : 0) + group_mode(G);
+    const int budget = std::min(di.smem_optin, kMaxSmem);
+    // resident activations for narrow token tiles, when they fit beside a
+    // ring of at least six stages: the largest windows over all runs
+    bool xr = false;
+    int xbytes = 0, xsbytes = 0;
+    if (pl.tt <= 2) {
+        int xcols = 0, xgroups = 0;
+        for (int cc = 0; cc < pl.Wt; ++cc) {
+            const int U0 = run_start(q, r, S, pl.upt, cc), U1 = run_start(q, r, S, pl.upt, cc + 1);
+            const XWindows w = x_windows(U0, U1, pl.upt, K);
+            int cols = 0, groups = 0;
+            for (int i = 0; i < w.n; ++i) {
+                cols += w.cols[i] + kXPad;
+                groups += w.cols[i] / G;
+            }
+            xcols = std::max(xcols, cols);
+            xgroups = std::max(xgroups, groups);
+        }
+        xbytes = xcols * 2 * 8 * pl.tt;
+        xsbytes = xgroups * 8 * pl.tt * 4;
+        const VariantCfg vr = variant_cfg(pl.tt, base + 6);
+        if ((int)smem_plan(vr, 6, xbytes, xsbytes).total <= budget)
+            xr = true;
+    }
+    pl.variant = base + (xr ? 6 : 0);
+    const VariantCfg vc = variant_cfg(pl.tt, pl.variant);
+    if (!xr)
+        xbytes = xsbytes = 0;
+    // the deepest ring that fits, up to MXG_STREAM_MAX_RING_KB of stages
+    int R = (MXG_STREAM_MAX_RING_KB * 1024) / vc.stage;
+    while (R > 2 && (int)smem_plan(vc, R, xbytes, xsbytes).total > budget)
+        --R;
+    if (R < 3)
+        return false;
+    const SmemPlan sp = smem_plan(vc, R, xbytes, xsbytes);
+    pl.smem = sp.total;
+    pl.ring = R;
+    pl.x_off = sp.x_off;
+    pl.xs_off = sp.xs_off;
+    pl.xchg_off = sp.xchg_off;
+    pl.bar_off = sp.bar_off;
+    pl.warps_per_cta = vc.threads / 32;
     const void *fn = select_kernel(pl.tt, pl.variant);
     if (!fn)
         return false;
     // every CTA of the grid must be resident at once (a cut row's finishing
-    // CTA waits for the others); function attributes and occupancy are per
-    // device: cached per device
-    static std::atomic<int> occ_cache[kMaxDeviceCache][4][6];
+    // CTA waits for the others); the attribute is set per device and variant
+    // to the largest shared memory a launch may ask for
+    static std::atomic<int> occ_cache[kMaxDeviceCache][4][12];
     std::atomic<int> &occ_slot = occ_cache[device][pl.tt - 1][pl.variant];
-    int occ = occ_slot.load(std::memory_order_acquire);
-    if (occ == 0) {
-        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem) !=
+    if (occ_slot.load(std::memory_order_acquire) == 0) {
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, budget) !=
             cudaSuccess)
             return false;
         int o = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, fn, vc.threads, pl.smem) !=
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, fn, vc.threads, budget) !=
                 cudaSuccess ||
             o < 1)
             return false;
-        occ = o;
-        occ_slot.store(occ, std::memory_order_release);
+        occ_slot.store(o, std::memory_order_release);
     }
-    // one CTA per SM (a second resident CTA, where it fits, is left to the
-    // next GEMM on the stream), no run shorter than one unit
-    pl.Wt = (int)std::max<long long>(1, std::min<long long>(di.sms, pl.units));
-    pl.grid = pl.Wt;
     pl.partial_bytes = (size_t)pl.Wt * kWarps * (2 * pl.tt * 32) * sizeof(float4);
     *plan = pl;
     return true;
@@ -663,32 +865,26 @@ cudaError_t launch_w4a16_stream(const StreamPlan &pl, const void *X, const void 
                                 int N, int K, int G, void *Y, void *workspace, bool early,
                                 cudaStream_t stream)
 {
+    (void)G;
     const void *fn = select_kernel(pl.tt, pl.variant);
     if (!fn)
         return cudaErrorInvalidValue;
     const VariantCfg vc = variant_cfg(pl.tt, pl.variant);
-    const int planes = pl.variant >= 3 ? 2 : 1;
+    const int planes = (pl.variant / 3) % 2 + 1;
     const uint8_t *codes = static_cast<const uint8_t *>(packed);
-    // codes take half a byte per weight (INT4) or one byte in two planes (INT8)
-    const uint8_t *scales = codes + (size_t)N * K / 2 * planes;
-    const uint64_t tiles = (uint64_t)N / 32;
-    alignas(64) CUtensorMap cmap, smap, xmap;
-    // codes: one row of 16 * K * planes bytes per n32 tile, in 8-byte elements
-    // scales: one row of 64 * K / G bytes per tile
-    // X: bf16 [M][K], boxes of 64 k x 8 TT rows with 128-byte swizzle
-    if (!encode_tensor_map_2d(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT64, codes,
-                              (uint64_t)K * 2 * planes, tiles, (uint64_t)K * 16 * planes,
-                              (uint32_t)(vc.code_tile / 8), kWarps, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !encode_tensor_map_2d(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT64, scales,
-                              (uint64_t)(K / G) * 8, tiles, (uint64_t)(K / G) * 64,
-                              (uint32_t)(vc.ks >= G ? vc.ks / G : 1) * 8, kWarps,
-                              CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !encode_tensor_map_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)K,
+    alignas(64) CUtensorMap xmap;
+    // X: bf16 [M][K], boxes of 64 k x 8 TT rows with 128-byte swizzle (used
+    // by the variants whose stages carry their activations)
+    if (!encode_tensor_map_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)K,
                               (uint64_t)M, (uint64_t)K * 2, 64, (uint32_t)(8 * pl.tt),
                               CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     const WorkspaceMap wm = make_workspace_map(pl.ntiles, pl.partial_bytes);
     Params p{};
+    p.X = static_cast<const uint16_t *>(X);
+    p.codes = codes;
+    // codes take half a byte per weight (INT4) or one byte in two planes (INT8)
+    p.scales = codes + (size_t)N * K / 2 * planes;
     p.Y = static_cast<uint16_t *>(Y);
     p.early = early ? 1 : 0;
     p.pf_stages = MXG_STREAM_PF_STAGES;
@@ -697,11 +893,18 @@ cudaError_t launch_w4a16_stream(const StreamPlan &pl, const void *X, const void 
     p.partial = reinterpret_cast<float4 *>(static_cast<uint8_t *>(workspace) + wm.partial_off);
     p.M = M;
     p.N = N;
+    p.K = K;
     p.ntiles = N / 32;
     p.upr = pl.upt;
     p.q = (int)(pl.units / pl.Wt);
     p.r = (int)(pl.units % pl.Wt);
-    void *args[] = {&cmap, &smap, &xmap, &p};
+    p.S = pl.split;
+    p.R = pl.ring;
+    p.x_off = pl.x_off;
+    p.xs_off = pl.xs_off;
+    p.xchg_off = pl.xchg_off;
+    p.bar_off = pl.bar_off;
+    void *args[] = {&xmap, &p};
     return launch_pdl(fn, dim3(pl.grid), dim3(vc.threads), pl.smem, stream, args);
 }
 

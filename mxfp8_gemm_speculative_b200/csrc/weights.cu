@@ -1,8 +1,9 @@
 // Offline weight re-pack for INT4 W4A16 and the decode kernels the tests use.
 //
-// Re-packed INT4 layout (one buffer, codes then scales):
-//   codes  [N/32][K/64][2 halves][32 lanes][4 words]
-//   scales [N/32][K/G][8][4 halves]
+// Re-packed INT4 layout (one buffer, codes then scales), by column groups of
+// eight n32 tiles (code_offset / scale_offset in common.cuh):
+//   codes  [N/256 groups][K/64 chunks][tiles of the group][2 halves][32 lanes][4 words]
+//   scales [N/256 groups][K/G][tiles of the group][8][4 halves]
 // For n32 tile T, k64 chunk c, half h and lane = 4*g + t (g = 0..7,
 // t = 0..3), the lane's 16 bytes hold columns na = 32T + 16h + g and
 // nb = na + 8.  Word j covers the four rows k0 = 64c + 16j + 4t .. k0 + 3:
@@ -36,8 +37,11 @@ __device__ __forceinline__ int chunk_k0(int c, int t, int j)
 // first) sits at qweight[i * wk + n * wn]: wk = N, wn = 1 for GPTQ
 // qweight[K/8][N]; wk = 1, wn = K/8 for compressed-tensors
 // weight_packed[N][K/8].
+// Tiles [tile0, tile0 + N/32) of a layer of ntiles tiles (a fused part
+// starts at a later tile).
 __global__ void repack_codes_kernel(const int32_t *__restrict__ qweight, int K, int N,
-                                    size_t wk, size_t wn, uint4 *__restrict__ out)
+                                    size_t wk, size_t wn, int tile0, int ntiles,
+                                    uint8_t *__restrict__ out)
 {
     const long long total = (long long)(N / 32) * (K / 64) * 64;
     const long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x;
@@ -69,7 +73,8 @@ __global__ void repack_codes_kernel(const int32_t *__restrict__ qweight, int K, 
         w |= ((qb >> 12) & 0xFu) << 28;
         words[j] = w;
     }
-    out[idx] = make_uint4(words[0], words[1], words[2], words[3]);
+    *reinterpret_cast<uint4 *>(out + code_offset(tile0 + T, c, K, ntiles, 1) + h * 512 +
+                               lane * 16) = make_uint4(words[0], words[1], words[2], words[3]);
 }
 
 // INT8 codes (4 per int32 word along K, byte j = row 4i + j, zero point
@@ -79,7 +84,7 @@ __global__ void repack_codes_kernel(const int32_t *__restrict__ qweight, int K, 
 // wk = N, wn = 1 for GPTQ-style [K/4][N]; wk = 1, wn = K/4 for the
 // compressed-tensors [N][K/4] export.
 __global__ void repack8_codes_kernel(const int32_t *__restrict__ qweight, int K, int N, size_t wk,
-                                     size_t wn, uint8_t *__restrict__ out)
+                                     size_t wn, int ntiles, uint8_t *__restrict__ out)
 {
     const long long total = (long long)(N / 32) * (K / 64) * 64;
     const long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x;
@@ -115,8 +120,8 @@ __global__ void repack8_codes_kernel(const int32_t *__restrict__ qweight, int K,
             (p ? hi : lo)[j] = w;
         }
     }
-    // [T][c][h][plane][lane][16 B]
-    uint4 *base = reinterpret_cast<uint4 *>(out) + ((((size_t)T * kc_count + c) * 2 + h) * 2) * 32;
+    // (T, c): [h][plane][lane][16 B]
+    uint4 *base = reinterpret_cast<uint4 *>(out + code_offset(T, c, K, ntiles, 2)) + h * 2 * 32;
     base[lane] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     base[32 + lane] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
 }
@@ -125,7 +130,8 @@ __global__ void repack8_codes_kernel(const int32_t *__restrict__ qweight, int K,
 // GPTQ scales[K/G][N]; sg = 1, sn = K/G for compressed-tensors
 // weight_scale[N][K/G].
 __global__ void repack_scales_kernel(const uint16_t *__restrict__ scales, int K, int N, int G,
-                                     size_t sg, size_t sn, uint16_t *__restrict__ out)
+                                     size_t sg, size_t sn, int tile0, int ntiles,
+                                     uint8_t *__restrict__ out)
 {
     const int groups = K / G;
     const long long total = (long long)(N / 32) * groups * 32;
@@ -138,13 +144,14 @@ __global__ void repack_scales_kernel(const uint16_t *__restrict__ scales, int K,
     const int grp = (int)(rest % groups);
     const int T = (int)(rest / groups);
     const int n = T * 32 + g + 8 * (i4 & 1) + 16 * (i4 >> 1);
-    out[idx] = scales[(size_t)grp * sg + n * sn];
+    reinterpret_cast<uint16_t *>(out + scale_offset(tile0 + T, grp, K, G, ntiles))[g * 4 + i4] =
+        scales[(size_t)grp * sg + n * sn];
 }
 
 // One thread per 16-byte code chunk: writes 16 codes of two columns, and
 // optionally their fp32 and bf16 dequantized values, using the decoders of
 // the GEMM paths.
-__global__ void unpack_kernel(const uint4 *__restrict__ codes, const uint16_t *__restrict__ sc,
+__global__ void unpack_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ sc,
                               int K, int N, int G, uint8_t *__restrict__ out_codes,
                               float *__restrict__ w_fp32, uint16_t *__restrict__ w_bf16)
 {
@@ -159,15 +166,18 @@ __global__ void unpack_kernel(const uint4 *__restrict__ codes, const uint16_t *_
     const int c = (int)(rest % kc_count);
     const int T = (int)(rest / kc_count);
     const int g = lane >> 2, t = lane & 3;
-    const int groups = K / G;
-    const uint4 v = codes[idx];
+    const int ntiles = N / 32;
+    const uint4 v =
+        *reinterpret_cast<const uint4 *>(codes + code_offset(T, c, K, ntiles, 1) + h * 512 + lane * 16);
     const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
     const int na = T * 32 + h * 16 + g, nb = na + 8;
 
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int k0 = chunk_k0(c, t, j);
-        const uint16_t *e = sc + ((size_t)T * groups + k0 / G) * 32 + g * 4 + 2 * h;
+        const uint16_t *e =
+            reinterpret_cast<const uint16_t *>(sc + scale_offset(T, k0 / G, K, G, ntiles)) + g * 4 +
+            2 * h;
         const uint16_t s_a = e[0], s_b = e[1];
         const ScaleSplit sp_a = split_scale(s_a), sp_b = split_scale(s_b);
         const float fa = __half2float(__ushort_as_half(s_a));
@@ -250,16 +260,14 @@ cudaError_t launch_w4a16_repack_part(const int32_t *qweight, const uint16_t *sca
                                      int G, int n0, int N, void *packed, cudaStream_t stream)
 {
     // part columns [n0, n0 + Np) of a fused layer with N columns: its n32
-    // tiles start at tile n0 / 32 in both the code and the scale region
+    // tiles are tiles n0 / 32 onwards of the fused layer
     const long long nchunks = (long long)(Np / 32) * (K / 64) * 64;
-    uint4 *codes = reinterpret_cast<uint4 *>(packed) + (size_t)(n0 / 32) * (K / 64) * 64;
-    repack_codes_kernel<<<blocks_for(nchunks, 256), 256, 0, stream>>>(qweight, K, Np, (size_t)Np,
-                                                                       1, codes);
+    uint8_t *out = static_cast<uint8_t *>(packed);
+    repack_codes_kernel<<<blocks_for(nchunks, 256), 256, 0, stream>>>(
+        qweight, K, Np, (size_t)Np, 1, n0 / 32, N / 32, out);
     const long long nsc = (long long)(Np / 32) * (K / G) * 32;
-    uint16_t *sc_out = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(packed) + (size_t)N * K / 2) +
-                       (size_t)(n0 / 32) * (K / G) * 32;
-    repack_scales_kernel<<<blocks_for(nsc, 256), 256, 0, stream>>>(scales, K, Np, G, (size_t)Np, 1,
-                                                                   sc_out);
+    repack_scales_kernel<<<blocks_for(nsc, 256), 256, 0, stream>>>(
+        scales, K, Np, G, (size_t)Np, 1, n0 / 32, N / 32, out + (size_t)N * K / 2);
     return cudaGetLastError();
 }
 
@@ -277,11 +285,12 @@ cudaError_t launch_w4a16_repack(const int32_t *qweight, const uint16_t *scales, 
     const size_t wk = n_major ? 1 : (size_t)N, wn = n_major ? (size_t)K / 8 : 1;
     const size_t sg = n_major ? 1 : (size_t)N, sn = n_major ? (size_t)(K / G) : 1;
     const long long nchunks = (long long)(N / 32) * (K / 64) * 64;
-    repack_codes_kernel<<<blocks_for(nchunks, 256), 256, 0, stream>>>(
-        qweight, K, N, wk, wn, reinterpret_cast<uint4 *>(packed));
+    uint8_t *out = static_cast<uint8_t *>(packed);
+    repack_codes_kernel<<<blocks_for(nchunks, 256), 256, 0, stream>>>(qweight, K, N, wk, wn, 0,
+                                                                       N / 32, out);
     const long long nsc = (long long)(N / 32) * (K / G) * 32;
-    uint16_t *sc_out = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(packed) + (size_t)N * K / 2);
-    repack_scales_kernel<<<blocks_for(nsc, 256), 256, 0, stream>>>(scales, K, N, G, sg, sn, sc_out);
+    repack_scales_kernel<<<blocks_for(nsc, 256), 256, 0, stream>>>(scales, K, N, G, sg, sn, 0,
+                                                                   N / 32, out + (size_t)N * K / 2);
     repack_done_kernel<<<1, 32, 0, stream>>>();
     return cudaGetLastError();
 }
@@ -293,10 +302,10 @@ cudaError_t launch_w8a16_repack(const int32_t *qweight, const uint16_t *scales, 
     const size_t sg = n_major ? 1 : (size_t)N, sn = n_major ? (size_t)(K / G) : 1;
     const long long npairs = (long long)(N / 32) * (K / 64) * 64;
     repack8_codes_kernel<<<blocks_for(npairs, 256), 256, 0, stream>>>(
-        qweight, K, N, wk, wn, static_cast<uint8_t *>(packed));
+        qweight, K, N, wk, wn, N / 32, static_cast<uint8_t *>(packed));
     const long long nsc = (long long)(N / 32) * (K / G) * 32;
-    uint16_t *sc_out = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(packed) + (size_t)N * K);
-    repack_scales_kernel<<<blocks_for(nsc, 256), 256, 0, stream>>>(scales, K, N, G, sg, sn, sc_out);
+    repack_scales_kernel<<<blocks_for(nsc, 256), 256, 0, stream>>>(
+        scales, K, N, G, sg, sn, 0, N / 32, static_cast<uint8_t *>(packed) + (size_t)N * K);
     repack_done_kernel<<<1, 32, 0, stream>>>();
     return cudaGetLastError();
 }
@@ -305,10 +314,9 @@ cudaError_t launch_w4a16_unpack(const void *packed, int K, int N, int G, uint8_t
                                 float *w_fp32, uint16_t *w_bf16, cudaStream_t stream)
 {
     const long long nchunks = (long long)(N / 32) * (K / 64) * 64;
-    const uint16_t *sc = reinterpret_cast<const uint16_t *>(static_cast<const uint8_t *>(packed) +
-                                                            (size_t)N * K / 2);
-    unpack_kernel<<<blocks_for(nchunks, 256), 256, 0, stream>>>(
-        reinterpret_cast<const uint4 *>(packed), sc, K, N, G, codes, w_fp32, w_bf16);
+    const uint8_t *pk = static_cast<const uint8_t *>(packed);
+    unpack_kernel<<<blocks_for(nchunks, 256), 256, 0, stream>>>(pk, pk + (size_t)N * K / 2, K, N, G,
+                                                                codes, w_fp32, w_bf16);
     return cudaGetLastError();
 }
 
