@@ -202,7 +202,7 @@ MXG_API int w4a16_gemm_ex(const void *X, const void *packed, int M, int N, int K
  * returns MXG_ERR_CAPTURE, and a later call outside a capture sets up).
  * Every call that completes without an error leaves the counters zero; the
  * partial-sum scratch keeps the last call's contents.  Calls that are not
- * ordered with respect to each other race on the array.  The array is 8 MiB
+ * ordered with respect to each other race on the array.  The array is 16 MiB
  * per device (every M <= 32 shape fits on a 148-SM B200).
  * A kernel that gives up a bounded wait records MXG_ERR_TIMEOUT in the
  * array's status word and returns MXG_OK to nobody: callers check the status

@@ -312,6 +312,28 @@ __device__ __forceinline__ void mma_bf16_16816_zero(float (&d)[4], uint32_t a0, 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
 }
 
+// The same MMAs on fp16 operands.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1)
+{
+    asm(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_f16_16816_zero(float (&d)[4], uint32_t a0, uint32_t a1,
+                                                   uint32_t a2, uint32_t a3, uint32_t b0,
+                                                   uint32_t b1)
+{
+    asm(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%10, %10, %10, %10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
+}
+
 // Arrival counter increment with acquire-release semantics at GPU scope:
 // publishes the caller's (and, after a warp barrier, its warp's) prior
 // stores and, for the last arriver, makes the other contributors' stores
@@ -354,6 +376,23 @@ __device__ __forceinline__ uint32_t int4_pair_plus128(uint32_t w)
     const uint32_t x = S ? (w >> S) : w;
     // (x & mask) | magic: truth table 0xEA for (a & b) | c
     asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(x), "r"(0x000F000Fu), "r"(0x43004300u));
+    return r;
+}
+
+// The fp16 form: with the magic 0x6400 (1024.0, whose unit in the last
+// place is 1) a nibble anywhere in the low byte of a half lands in the
+// mantissa, so one mask-and-or gives the pair (1024 + q_lo, 1024 + q_hi)
+// from bits 0..3 / 16..19 (HI = 0) or (1024 + 16 q_lo, 1024 + 16 q_hi) from
+// bits 4..7 / 20..23 (HI = 1); a shift by 8 reaches the other two nibble
+// positions.  Four registers of a 32-bit word then take four mask-and-ors
+// and one shift, not four and three.
+template <int HI>
+__device__ __forceinline__ uint32_t int4_pair_f16(uint32_t x)
+{
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;"
+        : "=r"(r)
+        : "r"(x), "r"(HI ? 0x00F000F0u : 0x000F000Fu), "r"(0x64006400u));
     return r;
 }
 

@@ -30,10 +30,10 @@ namespace mxg {
 namespace {
 
 // Header + counters (256 KiB) + partial sums.  The streaming plan keeps, per
-// CTA, one fragment of 512 bytes per consumer warp (8) and 8-row token tile;
-// with one CTA per SM on 148 SMs and M <= 32 (4 token tiles) that is
-// 4.6 MiB, so 8 MiB holds every M <= 32 shape on a B200.
-constexpr size_t kStaticScratchBytes = size_t(8) << 20;
+// CTA, two fragment slots of 512 bytes per consumer warp (8) and 8-row token
+// tile; with one CTA per SM on 148 SMs and M <= 32 (4 token tiles) that is
+// 9.3 MiB, so 16 MiB holds every M <= 32 shape on a B200.
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;
 __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
 constexpr int kMaxDev = 64;

@@ -21,27 +21,30 @@
 //    marked evict-first in L2.
 //  * The activations X of the CTA's run (the k ranges of its at most two
 //    group-row segments, or all of K when the run spans more rows) are
-//    copied into shared memory once, one bulk copy per row and range, and
-//    the per-group activation sums are formed once from them (one all-ones
-//    MMA per 16 rows of K).  When they do not fit beside the ring (wide
-//    token tiles, long runs) every stage also carries its activations (2-D
+//    copied into shared memory once by the consumer warps' own loads (after
+//    an L2 prefetch issued at entry), as fp16 values scaled per (scale
+//    group, token) by a power of two 2^-e, with a table of the sums of the
+//    stored values and 2^e.  When they do not fit beside the ring (wide
+//    token tiles, long runs) every stage carries its bf16 activations (2-D
 //    tensor-map boxes with 128-byte swizzle) and every warp forms the sums
-//    with its own all-ones MMAs.
+//    with all-ones MMAs.
 //  * Consumer warps own tiles: warp w (and, for M <= 16, warp w + 8, the two
 //    taking alternate stages) owns tile w of the group for the whole K range
 //    of the CTA's segment, so no warp reduces against another except the
-//    pair at a segment end.  Each warp decodes a pair of nibbles to the bf16
-//    pair (128 + q) with one mask-and-or (plus a shift) and multiplies on the
-//    tensor cores with m16n8k16 MMAs where the weights are the 16-row operand
-//    and the tokens the 8-column operand ("swap AB").  A zero-initialised
-//    partial sum per scale group is folded in as
-//    acc += (part - 136 * activation sum) * scale in fp32, so weights are
-//    never rounded (every product is exact in fp32).
-//  * A group row cut between CTAs is finished by the CTA holding its first
-//    unit, which reaches it last in its run; the other contributors (for
-//    whom it is the first segment of their run) publish their fragments
-//    early, so the finisher adds them in CTA order (deterministic) and
-//    writes bf16 Y.  A group row inside one run is written directly.
+//    pair at a segment end.  The tensor cores run m16n8k16 MMAs where the
+//    weights are the 16-row operand and the tokens the 8-column operand
+//    ("swap AB").  The decode is integer logic only, and that logic is the
+//    loop's busiest pipe: on fp16 windows four mask-and-ors and one shift
+//    turn a 32-bit word of codes into the pairs 1024 + q (rows g of the
+//    fragment) and 1024 + 16 q (rows g + 8); on bf16 stages four
+//    mask-and-ors and three shifts give 128 + q.  A zero-initialised partial
+//    sum per scale group is folded in fp32 as acc += (part - c * activation
+//    sum) * scale, with c and a factor 1/16 per fragment row, so weights
+//    are never rounded (every product is exact in fp32).
+//  * A group row cut between CTAs: every contributor publishes its fragment
+//    and counts itself in the tile's counter; the last one to arrive adds
+//    all fragments in CTA order (deterministic) and writes bf16 Y, so no CTA
+//    waits for another.  A group row inside one run is written directly.
 //
 // The same kernel runs INT8 W8A16 weights (the vocabulary head): their
 // re-pack splits each 8-bit code q = 16 hi + lo into a plane of low and a
@@ -62,6 +65,12 @@ namespace {
 #endif
 #ifndef MXG_STREAM_MAX_RING_KB
 #define MXG_STREAM_MAX_RING_KB 200
+#endif
+#ifndef MXG_STREAM_X_PREFETCH
+#define MXG_STREAM_X_PREFETCH 1
+#endif
+#ifndef MXG_STREAM_EARLY_MAX
+#define MXG_STREAM_EARLY_MAX 64
 #endif
 #ifndef MXG_STREAM_WPT2_MAX_TT
 #define MXG_STREAM_WPT2_MAX_TT 2
@@ -110,7 +119,8 @@ struct Params {
     uint16_t *Y;             // bf16 [M][N]
     WsHeader *hdr;
     int *counters;           // [column groups * 8]
-    float4 *partial;         // [ctas][8 tiles][2*TT][32]: a CTA's fragments of its first, cut group row
+    float4 *partial;         // [ctas][2 slots][8 tiles][2*TT][32]: a CTA's fragments of its cut rows
+    int frag;                // float4 per fragment: 2 * TT * 32
     int M, N, K;
     int ntiles;              // N / 32
     int upr;                 // units (stages) per group row: ceil(K / 128)
@@ -202,7 +212,7 @@ __device__ __forceinline__ void store_y4(const Params &p, int tile, int j, int l
 // ------------------------------------------------------------------ producer
 template <int TT, int GM, int P, int XR>
 __device__ __forceinline__ void produce(const Params &p, const CUtensorMap *xmap, uint8_t *smem,
-                                        uint64_t *full, uint64_t *empty, uint64_t *xbar, int U0,
+                                        uint64_t *full, uint64_t *empty, int U0,
                                         int ns)
 {
     using C = Cfg<TT, GM, P, XR>;
@@ -249,41 +259,33 @@ __device__ __forceinline__ void produce(const Params &p, const CUtensorMap *xmap
             tma_load_2d(st + ch * C::kXBox, xmap, src.k0 + 64 * ch, 0, &full[s % R], pol_x);
     };
     const int first = min(R, ns);
+    if (XR && MXG_STREAM_X_PREFETCH) {
+        // the run's activations are pulled into L2 ahead of the weights, so
+        // the consumers' loads of them after the wait do not queue behind
+        // the ring (a hint: L2 is coherent, data written later is not hidden)
+        const XWindows xw = x_windows(U0, U0 + ns, p.upr, K);
+        const int rows = min(p.M, 8 * TT);
+        for (int w = 0; w < xw.n; ++w)
+            for (int m = 0; m < rows; ++m)
+                prefetch_l2(p.X + (size_t)m * K + xw.klo[w], (uint32_t)xw.cols[w] * 2);
+    }
     // Weights are not written by the previous kernel on the stream (the
     // caller's contract, unless early loads are off): the first stages fill,
     // and the stages after them are pulled into L2, while that kernel drains.
-    if (p.early)
-        for (int s = 0; s < first; ++s)
-            issue_w(s);
+    const int early_n = p.early ? min(first, MXG_STREAM_EARLY_MAX) : 0;
+    for (int s = 0; s < early_n; ++s)
+        issue_w(s);
     const int pf_end = min(ns, R + p.pf_stages);
     for (int s = R; s < pf_end; ++s) {
         const Src src = source(s);
         prefetch_l2(src.codes, src.code_bytes);
     }
     pdl_wait();
-    if (!p.early)
-        for (int s = 0; s < first; ++s)
-            issue_w(s);
-    if (XR) {
-        // the run's activations, one bulk copy per row and window
-        const XWindows xw = x_windows(U0, U0 + ns, p.upr, K);
-        const int rows = min(p.M, 8 * TT);
-        uint32_t bytes = 0;
-        for (int w = 0; w < xw.n; ++w)
-            bytes += (uint32_t)rows * xw.cols[w] * 2;
-        mbar_arrive_expect_tx(xbar, bytes);
-        uint32_t base = p.x_off;
-        for (int w = 0; w < xw.n; ++w) {
-            const uint32_t stride = (xw.cols[w] + kXPad) * 2;
-            for (int m = 0; m < rows; ++m)
-                bulk_g2s(smem + base + m * stride, p.X + (size_t)m * K + xw.klo[w],
-                         (uint32_t)xw.cols[w] * 2, xbar, pol_x);
-            base += 8 * TT * stride;
-        }
-    } else {
+    for (int s = early_n; s < first; ++s)
+        issue_w(s);
+    if (!XR)
         for (int s = 0; s < first; ++s)
             issue_x(s);
-    }
     int issued = first;
     for (int s = first; s < ns; ++s) {
         // stage s reuses the slot of stage s - R: its release is phase
@@ -302,64 +304,78 @@ __device__ __forceinline__ void produce(const Params &p, const CUtensorMap *xmap
     for (int s = max(0, issued - R); s < issued; ++s)
         if (!mbar_wait(&full[s % R], (uint32_t)((s / R) & 1), kWaitLimitNs))
             record_error(p.hdr, MXG_ERR_TIMEOUT, 150 + GM);
-    if (XR && !mbar_wait(xbar, 0, kWaitLimitNs))
-        record_error(p.hdr, MXG_ERR_TIMEOUT, 160 + GM);
 }
 
 // ----------------------------------------------------------------- finisher
+// Fragment slot of CTA cc for group row gr: 0 when gr is the first row of its
+// run, else 1 (a cut row can only be the first or the last segment of a run).
+__device__ __forceinline__ float4 *partial_of(const Params &p, int cc, int gr, int wt)
+{
+    const int row0 = run_start(p.q, p.r, p.S, p.upr, cc) / p.upr;
+    return p.partial + ((size_t)(cc * 2 + (row0 == gr ? 0 : 1)) * kWarps + wt) * (size_t)p.frag;
+}
+
 // Run by the warp owning tile slot `wt` of a CTA whose segment of group row
 // `gr` is cut (the row goes on in other CTAs' runs), with the warp's fragment
-// in `sum`.  The CTA whose run holds the row's first unit finishes that
-// segment last in its run: it adds the other contributors' fragments (in CTA
-// order) to its own and writes bf16 Y.  Every other contributor (its segment
-// is the first one of its run) publishes its fragment and bumps the tile's
-// counter without waiting for anybody.
+// in `sum`.  Every contributor publishes its fragment in its own slot and
+// counts itself in the tile's counter; the one that arrives last adds all the
+// row's fragments in CTA order (so the sum does not depend on which CTA ends
+// last) and writes bf16 Y.  No CTA waits for another.
 template <int TT>
 __device__ __forceinline__ void finish_cut(const Params &p, float4 (&sum)[2 * TT], int c, int gr,
                                            int wt, int lane)
 {
     constexpr int F = 2 * TT;
+    constexpr int kB = F >= 8 ? 1 : 8 / F;   // contributors whose fragments load together
     const int tile = gr * kWarps + wt;
     const int c_first = cta_of_unit(p, gr * p.upr);
-    float4 *mine = p.partial + ((size_t)c * kWarps + wt) * F * 32;
-    if (c != c_first) {
-#pragma unroll
-        for (int j = 0; j < F; ++j)
-            __stcg(mine + j * 32 + lane, sum[j]);
-        __syncwarp();
-        if (lane == 0) {
-            __threadfence();
-            atomicAdd(&p.counters[tile], 1);
-        }
-        return;
-    }
     const int c_last = cta_of_unit(p, (gr + 1) * p.upr - 1);
-    if (lane == 0) {
-        const unsigned long long t0 = global_ns();
-        while (ld_acquire_gpu(&p.counters[tile]) < c_last - c_first) {
-            if (global_ns() - t0 > kWaitLimitNs) {
-                record_error(p.hdr, MXG_ERR_TIMEOUT, 120);
-                break;
-            }
-            __nanosleep(64);
-        }
-    }
-    __syncwarp();
-    for (int cc = c_first + 1; cc <= c_last; ++cc) {
-        const float4 *src = p.partial + ((size_t)cc * kWarps + wt) * F * 32;
+    float4 *mine = partial_of(p, c, gr, wt);
 #pragma unroll
-        for (int j = 0; j < F; ++j) {
-            const float4 f = __ldcg(src + j * 32 + lane);
-            sum[j].x += f.x;
-            sum[j].y += f.y;
-            sum[j].z += f.z;
-            sum[j].w += f.w;
+    for (int j = 0; j < F; ++j)
+        __stcg(mine + j * 32 + lane, sum[j]);
+    __syncwarp();
+    int old = 0;
+    if (lane == 0)
+        old = atomic_add_acq_rel(&p.counters[tile], 1);   // releases the fragment
+    old = __shfl_sync(0xFFFFFFFFu, old, 0);
+    if (old != c_last - c_first)
+        return;
+    // the last contributor (its acquire saw every other release)
+    float4 tot[F];
+#pragma unroll
+    for (int j = 0; j < F; ++j)
+        tot[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c0 = c_first; c0 <= c_last; c0 += kB) {
+        float4 f[kB][F];
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+            const int cc = c0 + u;
+            if (cc <= c_last && cc != c) {
+                const float4 *src = partial_of(p, cc, gr, wt);
+#pragma unroll
+                for (int j = 0; j < F; ++j)
+                    f[u][j] = __ldcg(src + j * 32 + lane);
+            } else {
+#pragma unroll
+                for (int j = 0; j < F; ++j)
+                    f[u][j] = sum[j];
+            }
         }
+#pragma unroll
+        for (int u = 0; u < kB; ++u)
+            if (c0 + u <= c_last)
+#pragma unroll
+                for (int j = 0; j < F; ++j) {
+                    tot[j].x += f[u][j].x;
+                    tot[j].y += f[u][j].y;
+                    tot[j].z += f[u][j].z;
+                    tot[j].w += f[u][j].w;
+                }
     }
 #pragma unroll
     for (int j = 0; j < F; ++j)
-        store_y4<TT>(p, tile, j, lane, sum[j]);
-    __syncwarp();
+        store_y4<TT>(p, tile, j, lane, tot[j]);
     if (lane == 0)
         p.counters[tile] = 0;  // leave the counter zero for the next call
 }
@@ -378,7 +394,6 @@ __global__ void __launch_bounds__(Cfg<TT, GM, P, XR>::kThreads, 1)
     const int R = p.R;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.bar_off);
     uint64_t *empty = full + R;
-    uint64_t *xbar = empty + R;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_launch_dependents();
@@ -390,13 +405,12 @@ __global__ void __launch_bounds__(Cfg<TT, GM, P, XR>::kThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kWarps);   // one warp of each tile takes a stage
         }
-        mbar_init(xbar, 1);
         fence_barrier_init();
     }
     __syncthreads();
     if (warp == C::kProducer) {
         if (lane == 0)
-            produce<TT, GM, P, XR>(p, &xmap, smem, full, empty, xbar, U0, ns);
+            produce<TT, GM, P, XR>(p, &xmap, smem, full, empty, U0, ns);
         return;
     }
 
@@ -408,43 +422,93 @@ __global__ void __launch_bounds__(Cfg<TT, GM, P, XR>::kThreads, 1)
     const uint32_t sb = smem_u32(smem);  // shared-window address of the base
     bool ok = true;
 
-    // resident activations: windows, and the per-group activation sums
-    // (table [group of the windows][8 TT tokens], fp32)
+    // resident activations: windows of fp16 values, and per (group of the
+    // windows, token) the sum of the stored values and their power-of-two
+    // factor (table [group][8 TT tokens] of float2)
     XWindows xw{};
     if constexpr (XR != 0) {
         xw = x_windows(U0, U1, p.upr, p.K);
-        if (!mbar_wait(xbar, 0, kWaitLimitNs)) {
-            if (lane == 0)
-                record_error(p.hdr, MXG_ERR_TIMEOUT, 110 + GM);
-            ok = false;
-        }
-        // entry e = (group of the windows, token tile): one all-ones MMA per
-        // 16 rows of K; lanes 0..3 hold the sums of tokens 2t, 2t+1
+        // One pass: every (group, token) segment of G activations is read by
+        // a team of G / 8 lanes, 16 bytes each (the consumers' own loads: a
+        // bulk copy would queue behind the ring's weight copies, which the
+        // producer issued before the wait and which may take microseconds to
+        // drain on a CTA that started late).  The team scales the segment by
+        // the power of two 2^-e that brings its largest magnitude into
+        // [2^14, 2^15), so every bf16 value becomes an fp16 value exactly
+        // (unless it is 2^28 times smaller than the largest one), stores it,
+        // and enters the sum of the stored values and 2^e in the table.
+        constexpr int L = C::kG / 8;   // lanes per segment
+        constexpr int kTeams = C::kConsumers * (32 / L);
+        const int rows = min(p.M, 8 * TT);
         const int ngr0 = xw.cols[0] / C::kG;
         const int ngr1 = xw.n > 1 ? xw.cols[1] / C::kG : 0;
-        const int entries = (ngr0 + ngr1) * TT;
+        const int nseg0 = ngr0 * rows, nseg = (ngr0 + ngr1) * rows;
         const uint32_t stride0 = (xw.cols[0] + kXPad) * 2;
-        for (int e = warp; e < entries; e += C::kConsumers) {
-            const int gi = e / TT, tt = e % TT;
-            const int w = gi < ngr0 ? 0 : 1;
-            const int gl = gi - (w ? ngr0 : 0);
-            const uint32_t base = p.x_off + (w ? 8 * TT * stride0 : 0);
-            const uint32_t stride = ((w ? xw.cols[1] : xw.cols[0]) + kXPad) * 2;
-            const uint32_t row = sb + base + (8 * tt + g) * stride + (gl * C::kG + 4 * t) * 2;
-            float a[4];
+        const uint32_t stride1 = (xw.n > 1 ? xw.cols[1] + kXPad : 0) * 2;
+        const int team = warp * (32 / L) + lane / L, piece = lane % L;
+        for (int i0 = 0; i0 < nseg; i0 += 4 * kTeams) {   // the same trip count in every lane
+            uint4 v[4];
+            uint32_t dst[4];
+            int ent[4];
 #pragma unroll
-            for (int j = 0; j < C::kStepsPerGroup; ++j) {
-                const uint2 b = lds64a(row + 32 * j);
-                if (j == 0)
-                    mma_bf16_16816_zero(a, kOnes, kOnes, kOnes, kOnes, b.x, b.y);
-                else
-                    mma_bf16_16816(a, kOnes, kOnes, kOnes, kOnes, b.x, b.y);
+            for (int u = 0; u < 4; ++u) {
+                const int sgi = i0 + u * kTeams + team;
+                v[u] = make_uint4(0u, 0u, 0u, 0u);
+                dst[u] = 0;
+                ent[u] = -1;
+                if (sgi < nseg) {
+                    const int w = sgi < nseg0 ? 0 : 1;
+                    const int loc = sgi - (w ? nseg0 : 0);
+                    const int gl = loc / rows, m = loc - gl * rows;
+                    const int k = (w ? xw.klo[1] : xw.klo[0]) + gl * C::kG + piece * 8;
+                    v[u] = __ldcg(reinterpret_cast<const uint4 *>(p.X + (size_t)m * p.K + k));
+                    dst[u] = p.x_off + (w ? 8 * TT * stride0 : 0) + m * (w ? stride1 : stride0) +
+                             (gl * C::kG + piece * 8) * 2;
+                    ent[u] = ((w ? ngr0 : 0) + gl) * 8 * TT + m;
+                }
             }
-            if (g == 0)
-                *reinterpret_cast<float2 *>(smem + p.xs_off + (gi * 8 * TT + 8 * tt + 2 * t) * 4) =
-                    make_float2(a[0], a[1]);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const uint32_t b[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                float f[8];
+                float mx = 0.f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    f[2 * i] = __uint_as_float(b[i] << 16);
+                    f[2 * i + 1] = __uint_as_float(b[i] & 0xFFFF0000u);
+                    mx = fmaxf(mx, fmaxf(fabsf(f[2 * i]), fabsf(f[2 * i + 1])));
+                }
+#pragma unroll
+                for (int o = L / 2; o >= 1; o >>= 1)
+                    mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+                // e = exponent(mx) - 14, within [-126, 126]; zeros and
+                // non-finite segments are stored unscaled
+                const int E = (int)((__float_as_uint(mx) >> 23) & 0xFF);
+                int e = 0;
+                if (mx > 0.f && E != 0xFF)
+                    e = max(-126, min(126, E - 127 - 14));
+                const float down = __uint_as_float((uint32_t)(127 - e) << 23);
+                uint32_t h[4];
+                float sum = 0.f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const __half2 hv = __floats2half2_rn(f[2 * i] * down, f[2 * i + 1] * down);
+                    h[i] = *reinterpret_cast<const uint32_t *>(&hv);
+                    const float2 back = __half22float2(hv);
+                    sum += back.x + back.y;
+                }
+#pragma unroll
+                for (int o = L / 2; o >= 1; o >>= 1)
+                    sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+                if (ent[u] >= 0) {
+                    *reinterpret_cast<uint4 *>(smem + dst[u]) = make_uint4(h[0], h[1], h[2], h[3]);
+                    if (piece == 0)
+                        *reinterpret_cast<float2 *>(smem + p.xs_off + ent[u] * 8) =
+                            make_float2(sum, __uint_as_float((uint32_t)(127 + e) << 23));
+                }
+            }
         }
-        named_bar_sync(9, C::kConsumers * 32);   // the table is complete
+        named_bar_sync(9, C::kConsumers * 32);   // the windows and the table are complete
     }
     // swizzled offsets of this lane's activations inside a staged 64-k box:
     // row 8 tt + g, bytes 32 j + 8 t of the row; the 16-byte chunk index is
@@ -543,38 +607,71 @@ __global__ void __launch_bounds__(Cfg<TT, GM, P, XR>::kThreads, 1)
                         }
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
-                            const uint32_t a0 = int4_pair_plus128<0>(wv[h][j]);
-                            const uint32_t a1 = int4_pair_plus128<4>(wv[h][j]);
-                            const uint32_t a2 = int4_pair_plus128<8>(wv[h][j]);
-                            const uint32_t a3 = int4_pair_plus128<12>(wv[h][j]);
-#pragma unroll
-                            for (int tt = 0; tt < TT; ++tt) {
-                                if (first)
-                                    mma_bf16_16816_zero(part[h][tt], a0, a1, a2, a3, xf[tt].x,
-                                                        xf[tt].y);
-                                else
-                                    mma_bf16_16816(part[h][tt], a0, a1, a2, a3, xf[tt].x,
-                                                   xf[tt].y);
-                            }
-                            if constexpr (P == 2) {
-                                const uint32_t b0 = int4_pair_plus128<0>(whi[h][j]);
-                                const uint32_t b1 = int4_pair_plus128<4>(whi[h][j]);
-                                const uint32_t b2 = int4_pair_plus128<8>(whi[h][j]);
-                                const uint32_t b3 = int4_pair_plus128<12>(whi[h][j]);
+                            if constexpr (XR != 0) {
+                                // fp16: registers a0, a2 (rows g) hold 1024 + q,
+                                // a1, a3 (rows g + 8) hold 1024 + 16 q
+                                const uint32_t w = wv[h][j], w8 = w >> 8;
+                                const uint32_t a0 = int4_pair_f16<0>(w);
+                                const uint32_t a1 = int4_pair_f16<1>(w);
+                                const uint32_t a2 = int4_pair_f16<0>(w8);
+                                const uint32_t a3 = int4_pair_f16<1>(w8);
 #pragma unroll
                                 for (int tt = 0; tt < TT; ++tt) {
                                     if (first)
-                                        mma_bf16_16816_zero(parthi[h][tt], b0, b1, b2, b3,
-                                                            xf[tt].x, xf[tt].y);
+                                        mma_f16_16816_zero(part[h][tt], a0, a1, a2, a3, xf[tt].x,
+                                                           xf[tt].y);
                                     else
-                                        mma_bf16_16816(parthi[h][tt], b0, b1, b2, b3, xf[tt].x,
+                                        mma_f16_16816(part[h][tt], a0, a1, a2, a3, xf[tt].x,
+                                                      xf[tt].y);
+                                }
+                                if constexpr (P == 2) {
+                                    const uint32_t u = whi[h][j], u8 = u >> 8;
+                                    const uint32_t b0 = int4_pair_f16<0>(u);
+                                    const uint32_t b1 = int4_pair_f16<1>(u);
+                                    const uint32_t b2 = int4_pair_f16<0>(u8);
+                                    const uint32_t b3 = int4_pair_f16<1>(u8);
+#pragma unroll
+                                    for (int tt = 0; tt < TT; ++tt) {
+                                        if (first)
+                                            mma_f16_16816_zero(parthi[h][tt], b0, b1, b2, b3,
+                                                               xf[tt].x, xf[tt].y);
+                                        else
+                                            mma_f16_16816(parthi[h][tt], b0, b1, b2, b3,
+                                                          xf[tt].x, xf[tt].y);
+                                    }
+                                }
+                            } else {
+                                const uint32_t a0 = int4_pair_plus128<0>(wv[h][j]);
+                                const uint32_t a1 = int4_pair_plus128<4>(wv[h][j]);
+                                const uint32_t a2 = int4_pair_plus128<8>(wv[h][j]);
+                                const uint32_t a3 = int4_pair_plus128<12>(wv[h][j]);
+#pragma unroll
+                                for (int tt = 0; tt < TT; ++tt) {
+                                    if (first)
+                                        mma_bf16_16816_zero(part[h][tt], a0, a1, a2, a3, xf[tt].x,
+                                                            xf[tt].y);
+                                    else
+                                        mma_bf16_16816(part[h][tt], a0, a1, a2, a3, xf[tt].x,
                                                        xf[tt].y);
+                                }
+                                if constexpr (P == 2) {
+                                    const uint32_t b0 = int4_pair_plus128<0>(whi[h][j]);
+                                    const uint32_t b1 = int4_pair_plus128<4>(whi[h][j]);
+                                    const uint32_t b2 = int4_pair_plus128<8>(whi[h][j]);
+                                    const uint32_t b3 = int4_pair_plus128<12>(whi[h][j]);
+#pragma unroll
+                                    for (int tt = 0; tt < TT; ++tt) {
+                                        if (first)
+                                            mma_bf16_16816_zero(parthi[h][tt], b0, b1, b2, b3,
+                                                                xf[tt].x, xf[tt].y);
+                                        else
+                                            mma_bf16_16816(parthi[h][tt], b0, b1, b2, b3,
+                                                           xf[tt].x, xf[tt].y);
+                                    }
                                 }
                             }
                         }
                         if (last) {
-                            // end of a scale group: the MMAs summed (128 + q) * x,
-                            // so acc += (part - 136 * sum(x)) * scale, in fp32
                             const int gi = step / C::kStepsPerGroup;   // group in the stage
                             const uint2 sv = lds64a(ss + gi * nt * 64);
                             const float2 s01 =
@@ -582,44 +679,69 @@ __global__ void __launch_bounds__(Cfg<TT, GM, P, XR>::kThreads, 1)
                             const float2 s23 =
                                 __half22float2(*reinterpret_cast<const __half2 *>(&sv.y));
                             const float sc[2][2] = {{s01.x, s01.y}, {s23.x, s23.y}};
-                            float2 xsv[TT];
                             if constexpr (XR != 0) {
-                                // table row of the group: k0 / G + gi from the
-                                // segment's origin
+                                // end of a scale group, fp16 windows: per token the
+                                // table holds the sum S of the stored values x' and
+                                // their factor f (x = f x').  Rows g summed
+                                // (1024 + q) x', rows g + 8 (1024 + 16 q) x', so
+                                // sum (q - 8) x = f (part - 1032 S) for rows g and
+                                // f / 16 (part - 1152 S) for rows g + 8; INT8 (q =
+                                // 16 hi + lo over two planes): f (16 Phi + Plo -
+                                // 17536 S) and f / 16 (16 Phi + Plo - 19456 S).
                                 const uint32_t xa = sb + p.xs_off +
-                                                    ((xg0 + k0 / C::kG + gi) * 8 * TT + 2 * t) * 4;
+                                                    ((xg0 + k0 / C::kG + gi) * 8 * TT + 2 * t) * 8;
 #pragma unroll
                                 for (int tt = 0; tt < TT; ++tt) {
-                                    const uint2 v = lds64a(xa + tt * 32);
-                                    xsv[tt] = make_float2(__uint_as_float(v.x),
-                                                          __uint_as_float(v.y));
+                                    const uint4 tv = lds128a(xa + tt * 64);
+                                    const float xs[2] = {__uint_as_float(tv.x), __uint_as_float(tv.z)};
+                                    const float fx[2] = {__uint_as_float(tv.y), __uint_as_float(tv.w)};
+#pragma unroll
+                                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                                        for (int e = 0; e < 4; ++e) {
+                                            // outputs e and e ^ 2 are rows g, g + 8
+                                            // of token 2t + (e & 1)
+                                            const int rh = e >> 1, tp = e & 1;
+                                            float v;
+                                            if constexpr (P == 2) {
+                                                v = fmaf(16.f, parthi[h][tt][e], part[h][tt][e]);
+                                                v = fmaf(rh ? -19456.f : -17536.f, xs[tp], v);
+                                            } else {
+                                                v = fmaf(rh ? -1152.f : -1032.f, xs[tp], part[h][tt][e]);
+                                            }
+                                            const float w = sc[h][rh] * (rh ? 0.0625f : 1.f) * fx[tp];
+                                            acc[h][tt][e] = fmaf(v, w, acc[h][tt][e]);
+                                        }
                                 }
                             } else {
+                                // end of a scale group: the MMAs summed (128 + q) * x,
+                                // so acc += (part - 136 * sum(x)) * scale, in fp32
+                                float2 xsv[TT];
 #pragma unroll
                                 for (int tt = 0; tt < TT; ++tt)
                                     xsv[tt] = make_float2(xsum[tt][0], xsum[tt][1]);
-                            }
 #pragma unroll
-                            for (int h = 0; h < 2; ++h)
+                                for (int h = 0; h < 2; ++h)
 #pragma unroll
-                                for (int tt = 0; tt < TT; ++tt)
+                                    for (int tt = 0; tt < TT; ++tt)
 #pragma unroll
-                                    for (int e = 0; e < 4; ++e) {
-                                        // outputs e and e ^ 2 are rows g, g + 8 of
-                                        // token 2t + (e & 1)
-                                        const float xe = (e & 1) ? xsv[tt].y : xsv[tt].x;
-                                        float v;
-                                        if constexpr (P == 2) {
-                                            // INT8 q = 16 hi + lo: the planes summed
-                                            // (128 + hi) x and (128 + lo) x, so
-                                            // sum (q - 128) x = 16 Phi + Plo - 2304 sum(x)
-                                            v = fmaf(16.f, parthi[h][tt][e], part[h][tt][e]);
-                                            v = fmaf(-2304.f, xe, v);
-                                        } else {
-                                            v = fmaf(-136.f, xe, part[h][tt][e]);
+                                        for (int e = 0; e < 4; ++e) {
+                                            // outputs e and e ^ 2 are rows g, g + 8 of
+                                            // token 2t + (e & 1)
+                                            const float xe = (e & 1) ? xsv[tt].y : xsv[tt].x;
+                                            float v;
+                                            if constexpr (P == 2) {
+                                                // INT8 q = 16 hi + lo: the planes summed
+                                                // (128 + hi) x and (128 + lo) x, so
+                                                // sum (q - 128) x = 16 Phi + Plo - 2304 sum(x)
+                                                v = fmaf(16.f, parthi[h][tt][e], part[h][tt][e]);
+                                                v = fmaf(-2304.f, xe, v);
+                                            } else {
+                                                v = fmaf(-136.f, xe, part[h][tt][e]);
+                                            }
+                                            acc[h][tt][e] = fmaf(v, sc[h][e >> 1], acc[h][tt][e]);
                                         }
-                                        acc[h][tt][e] = fmaf(v, sc[h][e >> 1], acc[h][tt][e]);
-                                    }
+                            }
                         }
                     }
                 }
@@ -747,7 +869,7 @@ SmemPlan smem_plan(const VariantCfg &vc, int R, int xbytes, int xsbytes)
     s.xs_off = s.x_off + (xbytes + 127) / 128 * 128;
     s.xchg_off = s.xs_off + (xsbytes + 127) / 128 * 128;
     s.bar_off = s.xchg_off + vc.xchg;
-    s.total = (size_t)s.bar_off + (2 * R + 1) * 8 + 1024;   // + alignment
+    s.total = (size_t)s.bar_off + 2 * R * 8 + 1024;   // + alignment
     return s;
 }
 
@@ -802,7 +924,7 @@ bool plan_stream(int device, int M, int N, int K, int G, int bits, StreamPlan *p
             xgroups = std::max(xgroups, groups);
         }
         xbytes = xcols * 2 * 8 * pl.tt;
-        xsbytes = xgroups * 8 * pl.tt * 4;
+        xsbytes = xgroups * 8 * pl.tt * 8;   // (sum, factor) per group and token
         const VariantCfg vr = variant_cfg(pl.tt, base + 6);
         if ((int)smem_plan(vr, 6, xbytes, xsbytes).total <= budget)
             xr = true;
@@ -828,9 +950,8 @@ bool plan_stream(int device, int M, int N, int K, int G, int bits, StreamPlan *p
     const void *fn = select_kernel(pl.tt, pl.variant);
     if (!fn)
         return false;
-    // every CTA of the grid must be resident at once (a cut row's finishing
-    // CTA waits for the others); the attribute is set per device and variant
-    // to the largest shared memory a launch may ask for
+    // the attribute is set per device and variant to the largest shared
+    // memory a launch may ask for
     static std::atomic<int> occ_cache[kMaxDeviceCache][4][12];
     std::atomic<int> &occ_slot = occ_cache[device][pl.tt - 1][pl.variant];
     if (occ_slot.load(std::memory_order_acquire) == 0) {
@@ -844,7 +965,7 @@ bool plan_stream(int device, int M, int N, int K, int G, int bits, StreamPlan *p
             return false;
         occ_slot.store(o, std::memory_order_release);
     }
-    pl.partial_bytes = (size_t)pl.Wt * kWarps * (2 * pl.tt * 32) * sizeof(float4);
+    pl.partial_bytes = (size_t)pl.Wt * 2 * kWarps * (2 * pl.tt * 32) * sizeof(float4);
     *plan = pl;
     return true;
 }
@@ -891,6 +1012,7 @@ cudaError_t launch_w4a16_stream(const StreamPlan &pl, const void *X, const void 
     p.hdr = static_cast<WsHeader *>(workspace);
     p.counters = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + wm.counters_off);
     p.partial = reinterpret_cast<float4 *>(static_cast<uint8_t *>(workspace) + wm.partial_off);
+    p.frag = 2 * pl.tt * 32;
     p.M = M;
     p.N = N;
     p.K = K;
