@@ -1,24 +1,38 @@
 """Benchmark of the weight-quantized linear layer on B200.
 
 One JSON line on rank 0.  A "step" is one pass of the hot path over one
-batch of synthetic inputs: for the default workload (single-stream MTP4
+batch of synthetic input: for the headline workload (single-stream MTP4
 verify chunk, M = 5 = 1 + 4 drafted tokens) that is the three INT4 layers
 5120->5120, 5120->17408 and 17408->5120 (group 128), each a w4a16_gemm
 through the C ABI.  Weights are re-packed once, outside the timed region.
 
-value      weight-stream TB/s: (code + scale bytes of every layer in the step)
-           / device time per step, whole job (all ranks).  For tensor-bound
-           workloads the line's unit is TFLOP/s (2*M*N*K per layer).
-e2e        the same metric through the Python binding with host buffers:
-           every step copies X from pinned host memory and reads Y back (the
-           step, copies included, replayed as a CUDA graph per pool slot).
-Workloads  --workload picks the step: the MTP4 verify layers (default; also
-           with gate/up fused), the C32 MTP3 chunk (M = 128), a prefill chunk
-           (M = 8192), MXFP8 at M = 4 and 128, the INT8 vocabulary head and
-           the paired bf16 GDN A/B projection.
-roofline   the dominant kernel's algorithmic bytes (or flops) per launch over
-           its average launch time, timed with CUDA events on its stream,
-           against MEASURED_PEAKS.json.
+value      weight-stream TB/s of the headline workload: (code + scale bytes
+           of every layer in the step) / device time per step, whole job
+           (all ranks).  Tensor-bound workloads are in TFLOP/s (2*M*N*K).
+configs    the other measured configurations, each timed the same way on
+           its own rotating weight pool: the tiny INT4 layer, the C32 MTP3
+           chunk (M = 128), the prefill chunk (M = 8192) and MXFP8 at M = 4
+           and M = 128 (default), with value, time per step, median / p10 /
+           p90 over the steps, the in-step time of every layer and the
+           roofline fractions.
+e2e        the same metric through the public API with host buffers: per
+           step the host-to-device copy of the step's X from pinned memory,
+           the layers, the device-to-host copy of every Y, then a stream
+           synchronize, timed on the host clock (e2e_graph: the same steps
+           captured as one CUDA graph over the pool slots and replayed, as a
+           serving loop does, timed with device events).
+timing     exactly --steps steps, replayed from CUDA graphs that hold one
+           step on every slot of the weight pool in turn (the launches
+           overlap their neighbours through programmatic dependent launch
+           inside a replay), CUDA events on the launch stream.
+roofline   every layer of a step runs the same kernel, so the dominant
+           kernel's time inside the step is the step time (its layers'
+           in-step times add up to it exactly: each layer's share is the
+           difference between the step cut after that layer and the step
+           cut before it, both timed as graphs with the same PDL overlap);
+           achieved = algorithmic bytes (or flops) per step / step time,
+           against MEASURED_PEAKS.json.  The same kernels timed one launch
+           at a time (no overlap with a neighbour) are reported beside it.
 L2         every step reads a different copy of the weights from a rotating
            pool of at least 3 x L2 bytes, so weights come from HBM.
 
@@ -31,6 +45,7 @@ from __future__ import annotations
 import argparse
 import json
 import os
+import platform
 import statistics
 import subprocess
 import tempfile
@@ -43,6 +58,7 @@ if ROOT not in sys.path:
 
 import numpy as np  # noqa: E402
 
+METRIC = "W4A16/MXFP8 GEMM weight-stream TB/s and TFLOP/s vs roofline, M=1..8192"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # workload -> (format, M, [(K, N)], group)
@@ -63,8 +79,20 @@ WORKLOADS = {
     "gdn_ab_bf16_m1": ("bf16", 1, [(5120, 96)], 0),
 }
 TENSOR_BOUND = {"c32_mtp3_int4", "prefill_int4", "mxfp8_m128"}
+# both fractions are reported for these (the ridge regime)
+BOTH_FRACTIONS = {"c32_mtp3_int4", "mxfp8_m128"}
 # (workload, layer index) -> column counts of the projections fused into it
 FUSED_PARTS = {("mtp4_verify_int4_fused", 1): (17408, 17408)}
+# the five measured configurations besides nothing else: the headline first
+DEFAULT_CONFIGS = ["mtp4_verify_int4", "tiny_int4", "c32_mtp3_int4", "prefill_int4",
+                   "mxfp8_m4", "mxfp8_m128"]
+# at least this many timed steps for a secondary configuration (its timed
+# region stays above a millisecond or so); the headline times exactly --steps
+MIN_STEPS = {"tiny_int4": 400, "mtp4_verify_int4": 200, "mtp4_verify_int4_fused": 200,
+             "c32_mtp3_int4": 100, "prefill_int4": 10, "mxfp8_m4": 200, "mxfp8_m128": 100,
+             "head_int8_m5": 20, "gdn_ab_bf16_m4": 400, "gdn_ab_bf16_m1": 400}
+KERNELS = {"bf16": "bf16_small_kernel", "int4": "w4a16_stream_kernel",
+           "int8": "w4a16_stream_kernel", "mxfp8": "mxfp8_stream_kernel"}
 
 
 def layer_weight_bytes(fmt, K, N, G):
@@ -75,6 +103,21 @@ def layer_weight_bytes(fmt, K, N, G):
     if fmt == "int8":
         return N * K + N * (K // G) * 2
     return N * K + N * (K // 32)
+
+
+def kernel_of(fmt, M):
+    if fmt in ("int4", "mxfp8") and M > 32:
+        return "tc_gemm_kernel"
+    return KERNELS[fmt]
+
+
+def arith_dtype(fmt, M):
+    """Operand type of the tensor-core products of a workload: the INT4 and
+    INT8 weight streams at M <= 16 multiply fp16 operands (codes decoded
+    exactly to 1024 + q or 1024 + 16 q, activations scaled per group by a
+    power of two into fp16 exactly); every other path multiplies bf16
+    operands.  Accumulation is fp32 throughout."""
+    return "f16" if fmt in ("int4", "int8") and M <= 16 else "bf16"
 
 
 def load_peaks():
@@ -90,6 +133,23 @@ def load_peaks():
 def dist_env():
     return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
             int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
+
+
+def quantiles(xs):
+    """(median, p10, p90) of a list of numbers."""
+    a = np.asarray(xs, dtype=np.float64)
+    return (float(np.median(a)), float(np.percentile(a, 10)), float(np.percentile(a, 90)))
 
 
 # --------------------------------------------------------------------- clocks
@@ -144,7 +204,6 @@ class ClockSampler:
                         reasons.add(name)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        # samples under load: the upper half of the observed clocks
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
                 "samples": len(sm), "reasons": sorted(reasons)}
 
@@ -168,305 +227,404 @@ def job_value(units_per_rank: float, world: int, elapsed_max_ms: float) -> float
 
 
 # ------------------------------------------------------------------ our arm
-def run_ours(args, rank, world, local_rank):
+class Workload:
+    """Seeded inputs of one workload on one device: per layer a rotating pool
+    of weight copies (>= pool_factor x L2 bytes per step), X, Y and a
+    workspace, and the library call of each layer."""
+
+    def __init__(self, name, rank, dev, pool_factor):
+        import torch
+
+        import mxfp8_gemm_speculative_b200 as mxg
+        import synth
+        self.mxg, self.name, self.dev = mxg, name, dev
+        self.fmt, self.M, self.layers, self.G = WORKLOADS[name]
+        fmt, M, G = self.fmt, self.M, self.G
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        self.step_bytes = sum(layer_weight_bytes(fmt, K, N, G) for K, N in self.layers)
+        self.step_flops = sum(2 * M * N * K for K, N in self.layers)
+        self.pool = max(2, -(-int(pool_factor * l2) // self.step_bytes))
+        self.xs, self.ys, self.weights, self.wss = [], [], [], []
+        for li, (K, N) in enumerate(self.layers):
+            if fmt == "int4":
+                lay = synth.int4_layer(M, K, N, G, seed=rank, layer=li)
+                qw = torch.from_numpy(lay.qweight).to(dev)
+                sc = torch.from_numpy(lay.scales.view(np.int16)).to(dev)
+                parts = FUSED_PARTS.get((name, li))
+                if parts:
+                    # fused projections: the parts' columns of the seeded layer,
+                    # re-packed into one buffer
+                    bounds = np.cumsum((0,) + parts)
+                    packed = mxg.w4a16_repack_fused(
+                        [(qw[:, a:b].contiguous(), sc[:, a:b].contiguous())
+                         for a, b in zip(bounds[:-1], bounds[1:])], G)
+                else:
+                    packed = mxg.w4a16_repack(qw, sc, G)
+                del qw, sc
+                self.weights.append([packed] + [packed.clone() for _ in range(self.pool - 1)])
+                need = mxg.w4a16_workspace_bytes(M, N, K, G)
+            elif fmt == "int8":
+                lay = synth.int8_layer(M, K, N, G, seed=rank, layer=li)
+                qw = torch.from_numpy(lay.qweight).to(dev)
+                sc = torch.from_numpy(lay.scales.view(np.int16)).to(dev)
+                packed = mxg.w8a16_repack(qw, sc, G)
+                del qw, sc
+                self.weights.append([packed] + [packed.clone() for _ in range(self.pool - 1)])
+                need = mxg.raw_lib().w8a16_workspace_bytes(M, N, K, G)
+            elif fmt == "bf16":
+                lay = synth.bf16_layer(M, K, N, seed=rank, layer=li)
+                w = torch.from_numpy(lay.W.view(np.int16)).view(torch.bfloat16).to(dev)
+                self.weights.append([w] + [w.clone() for _ in range(self.pool - 1)])
+                need = mxg.raw_lib().bf16_gemm_small_workspace_bytes(M, N, K)
+            else:
+                lay = synth.mxfp8_layer(M, K, N, seed=rank, layer=li)
+                wq = torch.from_numpy(lay.Wq).to(dev)
+                ws = torch.from_numpy(lay.Ws).to(dev)
+                self.weights.append([(wq, ws)] + [(wq.clone(), ws.clone())
+                                                  for _ in range(self.pool - 1)])
+                need = mxg.mxfp8_workspace_bytes(M, N, K)
+            self.wss.append(torch.zeros(need, dtype=torch.uint8, device=dev))
+            self.xs.append(torch.from_numpy(lay.X.view(np.int16)).view(torch.bfloat16).to(dev))
+            self.ys.append(torch.empty((M, N), dtype=torch.bfloat16, device=dev))
+        self.kernel = kernel_of(fmt, M)
+
+    def call(self, li, p, s, x=None, y=None):
+        """Layer li on pool slot p, on stream s (X and Y default to the
+        workload's device buffers)."""
+        mxg, fmt, G = self.mxg, self.fmt, self.G
+        K, N = self.layers[li]
+        x = self.xs[li] if x is None else x
+        y = self.ys[li] if y is None else y
+        w = self.weights[li][p]
+        if fmt == "int4":
+            mxg.w4a16_gemm(x, w, N, K, G, out=y, workspace_buf=self.wss[li], stream=s)
+        elif fmt == "int8":
+            mxg.w8a16_gemm(x, w, N, K, G, out=y, workspace_buf=self.wss[li], stream=s)
+        elif fmt == "bf16":
+            mxg.bf16_gemm_small(x, w, out=y, workspace_buf=self.wss[li], stream=s)
+        else:
+            mxg.mxfp8_gemm(x, w[0], w[1], out=y, workspace_buf=self.wss[li], stream=s)
+
+    def status(self):
+        return max(abs(self.mxg.mxg_workspace_status(w)) for w in self.wss)
+
+
+def capture(torch, stream, fn):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    return g
+
+
+def time_cycles(torch, stream, full, rem, steps, pool, per_cycle_events):
+    """Device time of exactly `steps` steps: `steps // pool` replays of the
+    graph `full` (one step on every pool slot) and, when `pool` does not
+    divide `steps`, one replay of `rem` (the first steps % pool slots).  With
+    per_cycle_events, an event between replays gives the ms per step of
+    every full cycle."""
+    n_full, r = divmod(steps, pool)
+    n_ev = (n_full + 2) if per_cycle_events else 2
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    with torch.cuda.stream(stream):
+        evs[0].record(stream)
+        for c in range(n_full):
+            full.replay()
+            if per_cycle_events:
+                evs[c + 1].record(stream)
+        if r:
+            rem.replay()
+        evs[-1].record(stream)
+    torch.cuda.synchronize()
+    total = evs[0].elapsed_time(evs[-1])
+    per = ([evs[c].elapsed_time(evs[c + 1]) / pool for c in range(n_full)]
+           if per_cycle_events else [])
+    return total, per
+
+
+def isolated_launch_us(torch, wl, stream, launches):
+    """Each layer timed one launch at a time: an event pair around every
+    launch, the launches queued behind a sleep kernel so every pair brackets
+    exactly one kernel (no overlap with a neighbour)."""
+    nl = len(wl.layers)
+    acc = [0.0] * nl
+    done = 0
+    with torch.cuda.stream(stream):
+        while done < launches:
+            nb = min(64, launches - done)
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * nl * nb)]
+            torch.cuda._sleep(20_000_000)
+            for i in range(nb):
+                p = (done + i) % wl.pool
+                for li in range(nl):
+                    evs[2 * (i * nl + li)].record(stream)
+                    wl.call(li, p, stream)
+                    evs[2 * (i * nl + li) + 1].record(stream)
+            torch.cuda.synchronize()
+            for i in range(nb):
+                for li in range(nl):
+                    acc[li] += evs[2 * (i * nl + li)].elapsed_time(evs[2 * (i * nl + li) + 1])
+            done += nb
+    return [a / launches * 1e3 for a in acc]
+
+
+def measure(wl, steps, warmup, world, dev, args, with_e2e):
+    """Times one workload: exactly `steps` steps after `warmup`, replayed
+    from CUDA graphs that hold one step on every pool slot in turn (a
+    serving loop's graph of consecutive layers: the launches overlap their
+    neighbours through programmatic dependent launch, within a replay and
+    not across the replay boundary); per-cycle quantiles; in-step per-layer
+    times; one-launch-at-a-time kernel times; the e2e figures."""
     import torch
     import torch.distributed as dist
 
-    import mxfp8_gemm_speculative_b200 as mxg
-    import synth
+    stream = torch.cuda.Stream(dev)
+    nl = len(wl.layers)
+    pool = wl.pool
+    r = steps % pool
+
+    def cycle(j, slots):
+        # slots' steps, each cut after layer j (j = nl: whole steps)
+        return capture(torch, stream, lambda: [wl.call(li, p, stream)
+                                               for p in slots for li in range(j)])
+
+    with torch.cuda.stream(stream):
+        for li in range(nl):
+            wl.call(li, 0, stream)          # plans and kernel attributes outside capture
+        torch.cuda.synchronize(dev)
+        full = {j: cycle(j, range(pool)) for j in range(1, nl + 1)}
+        rem = {j: cycle(j, range(r)) for j in range(1, nl + 1)} if r else {}
+    with torch.cuda.stream(stream):
+        for _ in range(-(-warmup // pool)):
+            full[nl].replay()
+    torch.cuda.synchronize(dev)
+    status = wl.status()
+    if status:
+        raise RuntimeError(f"{wl.name}: kernel reported status {-status}")
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    elapsed_ms, _ = time_cycles(torch, stream, full[nl], rem.get(nl), steps, pool, False)
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
+    # the distribution over full cycles (an event between replays), same steps
+    _, per_step = time_cycles(torch, stream, full[nl], rem.get(nl), steps, pool, True)
+    # in-step share of every layer: steps cut after layer j minus steps cut
+    # after layer j - 1
+    in_step = []
+    if nl > 1:
+        prev = 0.0
+        for j in range(1, nl + 1):
+            t, _ = time_cycles(torch, stream, full[j], rem.get(j), steps, pool, False)
+            in_step.append((t - prev) / steps * 1e3)
+            prev = t
+        # rescale so the shares add up to the whole-step time measured above
+        scale = (elapsed_ms / steps * 1e3) / max(sum(in_step), 1e-9)
+        in_step = [v * scale for v in in_step]
+    else:
+        in_step = [elapsed_ms / steps * 1e3]
+    iso = isolated_launch_us(torch, wl, stream, max(wl.pool, min(steps, args.kernel_steps)))
+    if wl.status():
+        raise RuntimeError(f"{wl.name}: kernel reported a status")
+    res = {"elapsed_ms": elapsed_ms, "per_step_ms": per_step, "in_step_us": in_step,
+           "isolated_us": iso, "cycle_steps": pool}
+    if with_e2e:
+        res.update(measure_e2e(wl, stream, steps, world, dev, args))
+    del full, rem
+    return res
+
+
+def measure_e2e(wl, stream, steps, world, dev, args):
+    """End to end through the public API with host buffers."""
+    import torch
+    import torch.distributed as dist
+
+    e2e_steps = max(1, min(args.e2e_steps, max(steps, 1)))
+    x_sizes = [x.numel() for x in wl.xs]
+    y_sizes = [y.numel() for y in wl.ys]
+    host_x = torch.cat([x.reshape(-1).cpu() for x in wl.xs]).pin_memory()
+    host_y = torch.empty(sum(y_sizes), dtype=torch.bfloat16).pin_memory()
+    dev_xbuf = torch.empty(sum(x_sizes), dtype=torch.bfloat16, device=dev)
+    dev_ybuf = torch.empty(sum(y_sizes), dtype=torch.bfloat16, device=dev)
+    dev_x = [v.view(x.shape) for v, x in zip(torch.split(dev_xbuf, x_sizes), wl.xs)]
+    dev_y = [v.view(y.shape) for v, y in zip(torch.split(dev_ybuf, y_sizes), wl.ys)]
+    h2d, d2h = host_x.numel() * 2, host_y.numel() * 2
+    nl = len(wl.layers)
+
+    def step(p):
+        dev_xbuf.copy_(host_x, non_blocking=True)
+        for li in range(nl):
+            wl.call(li, p, stream, x=dev_x[li], y=dev_y[li])
+        host_y.copy_(dev_ybuf, non_blocking=True)
+
+    # (1) eager: what a Python caller of the public API sees, host clock
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            step(i % wl.pool)
+        stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        t0 = time.perf_counter()
+        for i in range(e2e_steps):
+            step(i % wl.pool)
+            stream.synchronize()            # the result is on the host
+        eager_ms = (time.perf_counter() - t0) * 1e3
+    eager_ms = max_over_ranks(eager_ms, world, dev)
+    # (2) the steps captured as one graph over the pool slots and replayed,
+    # device events
+    pool = wl.pool
+    r = e2e_steps % pool
+    with torch.cuda.stream(stream):
+        full = capture(torch, stream, lambda: [step(p) for p in range(pool)])
+        rem = capture(torch, stream, lambda: [step(p) for p in range(r)]) if r else None
+        full.replay()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+    graph_ms, _ = time_cycles(torch, stream, full, rem, e2e_steps, pool, False)
+    graph_ms = max_over_ranks(graph_ms, world, dev)
+    del full, rem
+    return {"e2e_steps": e2e_steps, "e2e_eager_ms": eager_ms, "e2e_graph_ms": graph_ms,
+            "h2d": h2d, "d2h": d2h}
+
+
+def summarize(wl, res, steps, world, peaks, peak_kind):
+    """The measured numbers of one workload as a JSON-able dict."""
+    tensor_bound = wl.name in TENSOR_BOUND
+    elapsed_ms = res["elapsed_ms"]
+    ms_per_step = elapsed_ms / steps
+    if tensor_bound:
+        unit = "TFLOP/s"
+        value = job_value(wl.step_flops * steps, world, elapsed_ms) / 1e12
+    else:
+        unit = "TB/s"
+        value = job_value(wl.step_bytes * steps, world, elapsed_ms) / 1e12
+    med, p10, p90 = quantiles(res["per_step_ms"]) if res["per_step_ms"] else (None,) * 3
+    # in-step time of the dominant kernel = every layer of the step
+    k_us = sum(res["in_step_us"])
+    hbm_gbs = wl.step_bytes / (k_us * 1e-6) / 1e9
+    tflops = wl.step_flops / (k_us * 1e-6) / 1e12
+    if tensor_bound:
+        roof = {"bound": "tensor", "achieved": round(tflops, 2), "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(tflops / peaks["bf16_tflops"], 4),
+                "peak_source": f"{peak_kind} bf16 dense (burst)",
+                "frac_of_sustained": round(tflops / peaks["bf16_tflops_sustained"], 4)}
+    else:
+        roof = {"bound": "hbm", "achieved": round(hbm_gbs, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(hbm_gbs / peaks["hbm_gbs"], 4),
+                "peak_source": f"{peak_kind} copy bandwidth"}
+    if wl.name in BOTH_FRACTIONS:
+        roof["fractions"] = {"hbm": round(hbm_gbs / peaks["hbm_gbs"], 4),
+                             "tensor": round(tflops / peaks["bf16_tflops"], 4),
+                             "hbm_gbs": round(hbm_gbs, 1), "tflops": round(tflops, 2)}
+    roof["traffic"] = traffic_from_profiles(wl.kernel, wl.name)
+    roof["kernel"] = wl.kernel
+    roof["in_step_us_per_layer"] = [round(v, 3) for v in res["in_step_us"]]
+    roof["isolated_us_per_layer"] = [round(v, 3) for v in res["isolated_us"]]
+    iso_us = sum(res["isolated_us"])
+    roof["isolated_achieved"] = round(
+        (wl.step_flops / (iso_us * 1e-6) / 1e12) if tensor_bound
+        else (wl.step_bytes / (iso_us * 1e-6) / 1e9), 2)
+    out = {"value": round(value, 4), "unit": unit, "ms_per_step": round(ms_per_step, 6),
+           "steps": steps,
+           "step_ms_quantiles": {"median": med, "p10": p10, "p90": p90,
+                                 "over": f"{len(res['per_step_ms'])} replays of "
+                                         f"{res['cycle_steps']} steps (ms per step)"},
+           "tbps": round(job_value(wl.step_bytes * steps, world, elapsed_ms) / 1e12, 4),
+           "tflops": round(job_value(wl.step_flops * steps, world, elapsed_ms) / 1e12, 3),
+           "roofline": roof,
+           "config": {"workload": wl.name, "format": wl.fmt, "M": wl.M,
+                      "dtype": arith_dtype(wl.fmt, wl.M),
+                      "layers_KxN": [f"{K}x{N}" for K, N in wl.layers],
+                      "group_size": (wl.G if wl.fmt in ("int4", "int8")
+                                     else (32 if wl.fmt == "mxfp8" else None)),
+                      "weight_bytes_per_step": wl.step_bytes, "flops_per_step": wl.step_flops,
+                      "l2": f"rotating weight pool of {wl.pool} copies "
+                            f"({wl.pool * wl.step_bytes / 1e6:.0f} MB per layer set)"},
+           "gpu_launches": len(wl.layers) * steps}
+    if "e2e_eager_ms" in res:
+        n = res["e2e_steps"]
+        units = (wl.step_flops if tensor_bound else wl.step_bytes) * n
+        scale = 1e12
+        out["e2e"] = {"value": round(job_value(units, world, res["e2e_eager_ms"]) / scale, 4),
+                      "unit": unit, "h2d_bytes_per_step": res["h2d"],
+                      "d2h_bytes_per_step": res["d2h"], "steps": n,
+                      "path": "public Python API per step: pinned-host copy of every layer's X "
+                              "in, the layer calls (C ABI), copy of every Y out, stream "
+                              "synchronize; host clock"}
+        out["e2e_graph"] = {"value": round(job_value(units, world, res["e2e_graph_ms"]) / scale, 4),
+                            "unit": unit, "steps": n,
+                            "path": "the same steps captured as one CUDA graph over the pool "
+                                    "slots and replayed; device events"}
+    return out
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     if world > 1:
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
-
-    fmt, M, layers, G = WORKLOADS[args.workload]
-    tensor_bound = args.workload in TENSOR_BOUND
-    props = torch.cuda.get_device_properties(dev)
-    l2 = props.L2_cache_size
-
-    # inputs: one seeded synthetic layer per shape (rank-dependent seed)
-    step_bytes = sum(layer_weight_bytes(fmt, K, N, G) for K, N in layers)
-    step_flops = sum(2 * M * N * K for K, N in layers)
-    pool = max(2, -(-int(args.pool_factor * l2) // step_bytes))
-    xs, ys, weights, wss = [], [], [], []
-    for li, (K, N) in enumerate(layers):
-        if fmt == "int4":
-            lay = synth.int4_layer(M, K, N, G, seed=rank, layer=li)
-            qw = torch.from_numpy(lay.qweight).to(dev)
-            sc = torch.from_numpy(lay.scales.view(np.int16)).to(dev)
-            parts = FUSED_PARTS.get((args.workload, li))
-            if parts:
-                # fused projections: the parts' columns of the seeded layer,
-                # re-packed into one buffer
-                bounds = np.cumsum((0,) + parts)
-                packed = mxg.w4a16_repack_fused(
-                    [(qw[:, a:b].contiguous(), sc[:, a:b].contiguous())
-                     for a, b in zip(bounds[:-1], bounds[1:])], G)
-            else:
-                packed = mxg.w4a16_repack(qw, sc, G)
-            del qw, sc
-            weights.append([packed] + [packed.clone() for _ in range(pool - 1)])
-            wss.append(torch.zeros(mxg.w4a16_workspace_bytes(M, N, K, G), dtype=torch.uint8,
-                                   device=dev))
-        elif fmt == "int8":
-            lay = synth.int8_layer(M, K, N, G, seed=rank, layer=li)
-            qw = torch.from_numpy(lay.qweight).to(dev)
-            sc = torch.from_numpy(lay.scales.view(np.int16)).to(dev)
-            packed = mxg.w8a16_repack(qw, sc, G)
-            del qw, sc
-            weights.append([packed] + [packed.clone() for _ in range(pool - 1)])
-            wss.append(torch.zeros(mxg.raw_lib().w8a16_workspace_bytes(M, N, K, G),
-                                   dtype=torch.uint8, device=dev))
-        elif fmt == "bf16":
-            lay = synth.bf16_layer(M, K, N, seed=rank, layer=li)
-            w = torch.from_numpy(lay.W.view(np.int16)).view(torch.bfloat16).to(dev)
-            weights.append([w] + [w.clone() for _ in range(pool - 1)])
-            wss.append(torch.zeros(mxg.raw_lib().bf16_gemm_small_workspace_bytes(M, N, K),
-                                   dtype=torch.uint8, device=dev))
-        else:
-            lay = synth.mxfp8_layer(M, K, N, seed=rank, layer=li)
-            wq = torch.from_numpy(lay.Wq).to(dev)
-            ws = torch.from_numpy(lay.Ws).to(dev)
-            weights.append([(wq, ws)] + [(wq.clone(), ws.clone()) for _ in range(pool - 1)])
-            wss.append(torch.zeros(mxg.mxfp8_workspace_bytes(M, N, K), dtype=torch.uint8,
-                                   device=dev))
-        xs.append(torch.from_numpy(lay.X.view(np.int16)).view(torch.bfloat16).to(dev))
-        ys.append(torch.empty((M, N), dtype=torch.bfloat16, device=dev))
-
-    stream = torch.cuda.Stream(dev)
-
-    def layer_call(li, p, s):
-        K, N = layers[li]
-        if fmt == "int4":
-            mxg.w4a16_gemm(xs[li], weights[li][p], N, K, G, out=ys[li], workspace_buf=wss[li],
-                           stream=s)
-        elif fmt == "int8":
-            mxg.w8a16_gemm(xs[li], weights[li][p], N, K, G, out=ys[li], workspace_buf=wss[li],
-                           stream=s)
-        elif fmt == "bf16":
-            mxg.bf16_gemm_small(xs[li], weights[li][p], out=ys[li], workspace_buf=wss[li],
-                                stream=s)
-        else:
-            wq, ws = weights[li][p]
-            mxg.mxfp8_gemm(xs[li], wq, ws, out=ys[li], workspace_buf=wss[li], stream=s)
-
-    # Graphs: a step is every layer once on pool slot p.  Plain graphs (one
-    # per slot) time the steps; a second set with an event pair around every
-    # launch times the kernels themselves (two sets, so one can be read while
-    # the other runs).
-    nl = len(layers)
-    with torch.cuda.stream(stream):
-        for li in range(nl):
-            layer_call(li, 0, stream)           # plans and kernel attributes outside capture
-        torch.cuda.synchronize(dev)
-        graphs = []
-        for p in range(pool):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                for li in range(nl):
-                    layer_call(li, p, stream)
-            graphs.append(g)
-    warmup, steps = args.warmup, args.steps
-    with torch.cuda.stream(stream):          # replay() launches on the current stream
-        for i in range(warmup):
-            graphs[i % pool].replay()
-    torch.cuda.synchronize(dev)
-    status = max(abs(mxg.mxg_workspace_status(w)) for w in wss)
-    if status:
-        raise RuntimeError(f"kernel reported status {-status}")
+    peaks, peak_kind = load_peaks()
+    names = [args.workload]
+    if args.configs == "default":
+        names += [n for n in DEFAULT_CONFIGS if n != args.workload]
+    elif args.configs and args.configs != "none":
+        names += [n for n in args.configs.split(",") if n and n != args.workload]
+    for n in names:
+        if n not in WORKLOADS:
+            raise SystemExit(f"unknown workload {n}")
 
     clocks = ClockSampler(local_rank)
     clocks.start()
-    time.sleep(0.3)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        t_start.record(stream)
-        for i in range(steps):
-            graphs[i % pool].replay()
-        t_end.record(stream)
-    torch.cuda.synchronize(dev)
-    elapsed_ms = t_start.elapsed_time(t_end)
-
-    # kernel durations over a second live pass: the stream is held by a
-    # sleep kernel while a batch of launches, each between two events, is
-    # queued behind it, so every event pair brackets exactly one kernel
-    kernel_ms = [0.0] * nl
-    kernel_launches = 0
-    want = max(pool, min(steps, args.kernel_steps))
-    batch = 64
-    with torch.cuda.stream(stream):
-        while kernel_launches < want:
-            nb_steps = min(batch, want - kernel_launches)
-            evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * nl * nb_steps)]
-            torch.cuda._sleep(20_000_000)
-            for i in range(nb_steps):
-                p = (kernel_launches + i) % pool
-                for li in range(nl):
-                    evs[2 * (i * nl + li)].record(stream)
-                    layer_call(li, p, stream)
-                    evs[2 * (i * nl + li) + 1].record(stream)
-            torch.cuda.synchronize(dev)
-            for i in range(nb_steps):
-                for li in range(nl):
-                    kernel_ms[li] += evs[2 * (i * nl + li)].elapsed_time(evs[2 * (i * nl + li) + 1])
-            kernel_launches += nb_steps
+    results = {}
+    for i, name in enumerate(names):
+        head = i == 0
+        wl = Workload(name, rank, dev, args.pool_factor)
+        steps = args.steps if head else max(args.steps, MIN_STEPS.get(name, args.steps))
+        warmup = args.warmup if head else max(args.warmup, 3)
+        res = measure(wl, steps, warmup, world, dev, args, with_e2e=head or args.e2e_all)
+        results[name] = summarize(wl, res, steps, world, peaks, peak_kind)
+        del wl
+        torch.cuda.empty_cache()
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
 
-    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
-    ms_per_step = elapsed_ms / steps
-
-    # ------------------------------------------------------------- e2e arm
-    e2e_steps = max(1, min(args.e2e_steps, steps))
-    # one pinned host buffer holds every layer's X (and one every layer's Y):
-    # a step copies X in once, runs the layers, and reads Y back once
-    x_sizes = [x.numel() for x in xs]
-    y_sizes = [y.numel() for y in ys]
-    host_x = torch.cat([x.reshape(-1).cpu() for x in xs]).pin_memory()
-    host_y = torch.empty(sum(y_sizes), dtype=torch.bfloat16).pin_memory()
-    dev_xbuf = torch.empty(sum(x_sizes), dtype=torch.bfloat16, device=dev)
-    dev_ybuf = torch.empty(sum(y_sizes), dtype=torch.bfloat16, device=dev)
-    dev_x = [v.view(x.shape) for v, x in zip(torch.split(dev_xbuf, x_sizes), xs)]
-    dev_y = [v.view(y.shape) for v, y in zip(torch.split(dev_ybuf, y_sizes), ys)]
-    h2d = host_x.numel() * 2
-    d2h = host_y.numel() * 2
-
-    # the layer calls of every pool slot, marshalled once (binding.prepare_*)
-    prepared = []
-    for p in range(pool):
-        calls = []
-        for li, (K, N) in enumerate(layers):
-            if fmt == "int4":
-                c, _ = mxg.prepare_w4a16_gemm(dev_x[li], weights[li][p], N, K, G, out=dev_y[li],
-                                              workspace_buf=wss[li], stream=stream)
-            elif fmt == "int8":
-                c, _ = mxg.prepare_w8a16_gemm(dev_x[li], weights[li][p], N, K, G, out=dev_y[li],
-                                              workspace_buf=wss[li], stream=stream)
-            elif fmt == "bf16":
-                c, _ = mxg.prepare_bf16_gemm_small(dev_x[li], weights[li][p], out=dev_y[li],
-                                                   workspace_buf=wss[li], stream=stream)
-            else:
-                wq, ws = weights[li][p]
-                c, _ = mxg.prepare_mxfp8_gemm(dev_x[li], wq, ws, out=dev_y[li],
-                                              workspace_buf=wss[li], stream=stream)
-            calls.append(c)
-        prepared.append(calls)
-
-    def e2e_step(p):
-        dev_xbuf.copy_(host_x, non_blocking=True)
-        for call in prepared[p]:
-            call()
-        host_y.copy_(dev_ybuf, non_blocking=True)
-
-    # A serving loop replays the step as a CUDA graph: one graph per pool slot
-    # holding the step's host-to-device copy, its layer calls (the prepared
-    # binding calls) and its device-to-host copy.
-    with torch.cuda.stream(stream):
-        for i in range(3):
-            e2e_step(i % pool)
-        torch.cuda.synchronize(dev)
-        e2e_graphs = []
-        for p in range(pool):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                e2e_step(p)
-            e2e_graphs.append(g)
-        for i in range(3):
-            e2e_graphs[i % pool].replay()
-        torch.cuda.synchronize(dev)
-        if world > 1:
-            dist.barrier()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for i in range(e2e_steps):
-            e2e_graphs[i % pool].replay()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    e2e_ms = max_over_ranks(e2e_ms, world, dev)
-
-    peaks, peak_kind = load_peaks()
-    if tensor_bound:
-        unit = "TFLOP/s"
-        value = job_value(step_flops * steps, world, elapsed_ms) / 1e12
-        e2e_value = job_value(step_flops * e2e_steps, world, e2e_ms) / 1e12
-    else:
-        unit = "TB/s"
-        value = job_value(step_bytes * steps, world, elapsed_ms) / 1e12
-        e2e_value = job_value(step_bytes * e2e_steps, world, e2e_ms) / 1e12
-
-    # dominant kernel: every layer of the step runs the same kernel
-    k_total_ms = sum(kernel_ms)
-    if tensor_bound:
-        achieved = step_flops * kernel_launches / (k_total_ms * 1e-3) / 1e12
-        peak = peaks["bf16_tflops"]
-        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
-                "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
-                "peak_source": f"{peak_kind} bf16 dense (burst)"}
-    else:
-        achieved = step_bytes * kernel_launches / (k_total_ms * 1e-3) / 1e9
-        peak = peaks["hbm_gbs"]
-        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": None,
-                "peak_source": f"{peak_kind} copy bandwidth"}
-    kernel_name = ("bf16_small_kernel" if fmt == "bf16" else
-                   "w4a16_stream_kernel" if (fmt in ("int4", "int8") and M <= 32) else
-                   "mxfp8_stream_kernel" if M <= 32 else "tc_gemm_kernel")
-    roof["kernel"] = kernel_name
-    roof["per_layer_us"] = [round(k / kernel_launches * 1e3, 3) for k in kernel_ms]
-    roof["timed_launches"] = kernel_launches * nl
-    traffic = traffic_from_profiles(kernel_name, args.workload)
-    if traffic is not None:
-        roof["traffic"] = traffic
-
+    head = results[args.workload]
+    props = torch.cuda.get_device_properties(dev)
     line = {
-        "metric": "W4A16/MXFP8 GEMM weight-stream TB/s and TFLOP/s vs roofline, M=1..8192",
-        "value": round(value, 4),
-        "unit": unit,
+        "metric": METRIC,
+        "value": head["value"],
+        "unit": head["unit"],
         "n_gpus": world,
-        "steps": steps,
-        "warmup": warmup,
-        "ms_per_step": round(ms_per_step, 6),
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": head["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",  # every path multiplies bf16 operands with fp32 accumulation
+        "dtype": arith_dtype(WORKLOADS[args.workload][0], WORKLOADS[args.workload][1]),
         "data": "synthetic (seeded; the value distributions of the layer formats)",
-        "config": {
-            "workload": args.workload,
-            "format": fmt, "M": M, "layers_KxN": [f"{K}x{N}" for K, N in layers],
-            "group_size": G if fmt in ("int4", "int8") else (32 if fmt == "mxfp8" else None),
-            "weight_bytes_per_step": step_bytes, "flops_per_step": step_flops,
-            "l2": f"rotating weight pool of {pool} copies ({pool * step_bytes / 1e6:.0f} MB >= "
-                  f"{args.pool_factor:g} x L2)",
-            "timing": "CUDA graphs of one step per pool slot, CUDA events on the launch stream; "
-                      "kernel durations from a second live pass with an event pair around "
-                      "each launch, queued behind a sleep kernel",
-            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-        },
-        "tflops": round(step_flops * steps / (elapsed_ms * 1e-3) / 1e12 * world, 3),
-        "tbps": round(step_bytes * steps / (elapsed_ms * 1e-3) / 1e12 * world, 4),
-        "e2e": {"value": round(e2e_value, 4), "unit": unit, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                "path": "python binding (calls prepared once), the step captured once per "
-                        "pool slot as a CUDA graph and replayed: per step one pinned-host copy "
-                        "of every layer's X in, the layers, one copy of every layer's Y out"},
-        "roofline": roof,
-        "gpu_launches": len(layers) * steps,
+        "config": dict(head["config"], **{
+            "timing": "CUDA graphs of one step on every weight-pool slot, replayed for exactly "
+                      "--steps steps, CUDA events on the launch stream; weights from a rotating "
+                      "pool >= 3 x L2 (inputs larger than L2)",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}),
+        "step_ms_quantiles": head["step_ms_quantiles"],
+        "tflops": head["tflops"],
+        "tbps": head["tbps"],
+        "e2e": head.get("e2e"),
+        "e2e_graph": head.get("e2e_graph"),
+        "roofline": head["roofline"],
+        "gpu_launches": head["gpu_launches"],
         "clocks": clk,
         "gpu": props.name,
+        "configs": {n: r for n, r in results.items() if n != args.workload},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.workload, budget_s=args.cpu_budget)
     if world > 1:
-        graphs.clear()
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
@@ -537,37 +695,46 @@ def oracle_step_runner(workload: str, cols_per_layer: int | None, seed: int = 0)
     return run, fmt
 
 
+def _oracle_rate(workload: str, nthreads: int, budget_s: float):
+    """(value in the workload's unit, column slice, passes, seconds) of the
+    oracle on `nthreads` threads, about budget_s seconds of work."""
+    fmt, M, layers, G = WORKLOADS[workload]
+    probe, _ = oracle_step_runner(workload, 64)
+    t0 = time.perf_counter()
+    probe(nthreads)
+    dt = max(time.perf_counter() - t0, 1e-6)
+    full_cols = max(N for _, N in layers)
+    cols = int(min(full_cols, max(16, 64 * budget_s / dt / 2)))
+    run, _ = oracle_step_runner(workload, cols)
+    t0 = time.perf_counter()
+    b, f = run(nthreads)
+    passes = 1
+    while time.perf_counter() - t0 < 0.5 * budget_s:
+        run(nthreads)
+        passes += 1
+    dt = time.perf_counter() - t0
+    b, f = b * passes, f * passes
+    value = (f / dt / 1e12) if workload in TENSOR_BOUND else (b / dt / 1e12)
+    return value, cols, passes, dt
+
+
 def cpu_baseline(workload: str, budget_s: float = 20.0):
     import oracle
     oracle.build()
     cores = os.cpu_count() or 1
     used = oracle.threads(cores)
     fmt, M, layers, G = WORKLOADS[workload]
-    # size the column slice so one pass stays within the budget
-    probe, _ = oracle_step_runner(workload, 64)
-    t0 = time.perf_counter()
-    b, f = probe(used)
-    dt = max(time.perf_counter() - t0, 1e-6)
-    full_cols = max(N for _, N in layers)
-    cols = int(min(full_cols, max(64, 64 * budget_s / dt / 2)))
-    run, _ = oracle_step_runner(workload, cols)
-    t0 = time.perf_counter()
-    b, f = run(used)
-    dt = time.perf_counter() - t0
-    # whole passes until about half the budget is spent (the first one counts)
-    passes = 1
-    while time.perf_counter() - t0 < 0.5 * budget_s:
-        run(used)
-        passes += 1
-    dt = time.perf_counter() - t0
-    b, f = b * passes, f * passes
-    tensor_bound = workload in TENSOR_BOUND
-    value = (f / dt / 1e12) if tensor_bound else (b / dt / 1e12)
-    return {"value": value, "unit": "TFLOP/s" if tensor_bound else "TB/s", "cores": used,
-            "kind": "oracle",
+    value, cols, passes, dt = _oracle_rate(workload, used, budget_s * 0.75)
+    v1, cols1, passes1, dt1 = _oracle_rate(workload, 1, budget_s * 0.25)
+    unit = "TFLOP/s" if workload in TENSOR_BOUND else "TB/s"
+    return {"value": value, "unit": unit, "cores": used, "kind": "oracle",
+            "cpu_model": cpu_model(),
             "sample": f"{cols} of the output columns of every layer of {workload} "
                       f"(M={M}), {passes} pass(es), {dt:.1f} s, fp64 C oracle, "
-                      f"OpenMP over columns"}
+                      f"OpenMP over columns on {used} threads",
+            "single_thread": {"value": v1, "unit": unit, "cores": 1,
+                              "sample": f"{cols1} output columns of every layer, "
+                                        f"{passes1} pass(es), {dt1:.1f} s"}}
 
 
 def run_reference(args, rank, world):
@@ -603,7 +770,7 @@ def run_reference(args, rank, world):
               f"fp64 C oracle, {used} threads")
     line = {
         "impl": "reference",
-        "metric": "W4A16/MXFP8 GEMM weight-stream TB/s and TFLOP/s vs roofline, M=1..8192",
+        "metric": METRIC,
         "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -611,7 +778,7 @@ def run_reference(args, rank, world):
         "config": {"workload": args.workload, "format": fmt, "M": M,
                    "layers_KxN": [f"{K}x{N}" for K, N in layers]},
         "cpu_baseline": {"value": value, "unit": unit, "cores": used, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -620,12 +787,18 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="mtp4_verify_int4")
-    ap.add_argument("--e2e-steps", type=int, default=2000)
-    ap.add_argument("--kernel-steps", type=int, default=512)
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="mtp4_verify_int4",
+                    help="the headline workload (the line's value)")
+    ap.add_argument("--configs", default="default",
+                    help="further workloads measured into the line's 'configs': 'default' "
+                         "(the five configurations), 'none', or a comma list")
+    ap.add_argument("--e2e-all", action="store_true",
+                    help="measure the e2e figures for every configuration, not only the headline")
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--kernel-steps", type=int, default=64)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-budget", type=float, default=120.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
