@@ -51,12 +51,13 @@ enum Fmt { kInt4 = 0, kMxfp8 = 1 };
 
 // Ring depths: with 128 tokens per tile the activation and weight slots are
 // small and a k-block's MMA is short, so the rings are deeper to cover the
-// load latency.
+// load latency; the A ring takes the tensor memory the accumulator leaves.
 template <int F, int BT>
 struct Layout {
-    static constexpr int kSX = BT == 128 ? 8 : 4;    // activation ring
-    static constexpr int kSW = BT == 128 ? 12 : 8;   // packed-weight ring
-    static constexpr int kSA = BT == 128 ? 8 : 6;    // tensor-memory A ring (32 columns each)
+    static constexpr int kSX = BT == 128 ? 8 : 5;    // activation ring
+    static constexpr int kSW = BT == 128 ? (F == kInt4 ? 24 : 16)
+                                         : (F == kInt4 ? 16 : 12);   // packed-weight ring
+    static constexpr int kSA = BT == 128 ? 12 : 8;   // tensor-memory A ring (32 columns each)
     static constexpr int x_slot = (BT / 2) * BK * 2;                // bf16 activations
     static constexpr int wp_slot = (F == kInt4) ? 5120 : BW * BK;   // packed weights
     static constexpr int x_off = 0;
@@ -86,6 +87,20 @@ struct TcParams {
     int num_items;         // num_tiles * splits work items
     int early;             // load the first weights before waiting for the previous kernel
 };
+
+// Output tile -> weight block nb (256 columns) and token tile mt.  With
+// several token tiles the tiles run token-tile-major: the pairs working at
+// the same time share one activation tile and sweep all weight blocks, which
+// stay in L2 (marked evict-last) from one token tile to the next, so each
+// weight and activation byte is read from DRAM about once.
+__device__ __forceinline__ int tile_nb(const TcParams &p, int tile)
+{
+    return p.mtiles > 1 ? tile % p.ntiles : tile / p.mtiles;
+}
+__device__ __forceinline__ int tile_mt(const TcParams &p, int tile)
+{
+    return p.mtiles > 1 ? tile / p.ntiles : tile % p.mtiles;
+}
 
 // Work item -> output tile and its k-block range [kb0, kb1).
 __device__ __forceinline__ void item_range(const TcParams &p, int item, int &tile, int &kb0,
@@ -363,7 +378,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // while the previous kernel drains: pull the first k-blocks into L2
         int tile0, kb0, kb1;
         item_range(p, pair, tile0, kb0, kb1);
-        const int nb = tile0 / p.mtiles, mt = tile0 % p.mtiles;
+        const int nb = tile_nb(p, tile0), mt = tile_mt(p, tile0);
         const int n32 = (nb * 2 * BW + (int)rank * BW) / 32;
         const int ntl = F == kInt4 ? max(0, min(4, group_tiles(nb, p.N / 32) - 4 * (int)rank)) : 0;
         for (int kb = kb0; kb < min(kb0 + L::kSW, kb1); ++kb) {
@@ -392,7 +407,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (w_item < p.num_items)
         item_range(p, w_item, w_tile, w_kb, w_kb1);
     auto w_issue = [&](uint32_t until) -> bool {
-        const uint64_t pol_w = l2_policy_evict_first();
+        // weights stream once when there is one token tile, else they are
+        // read again by every token tile
+        const uint64_t pol_w = p.mtiles > 1 ? l2_policy_evict_last() : l2_policy_evict_first();
         while (w_item < p.num_items && w_it < until) {
             if (w_kb >= w_kb1) {
                 w_item += npairs;
@@ -403,7 +420,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int sw = w_it % L::kSW;
             if (!role_wait(&wp_empty[sw], ((w_it / L::kSW) & 1) ^ 1, abort_flag, p.hdr, 402))
                 return false;
-            const int nb = w_tile / p.mtiles;
+            const int nb = tile_nb(p, w_tile);
             const int n32 = (nb * 2 * BW + (int)rank * BW) / 32;
             uint8_t *wdst = smem + L::wp_off + sw * L::wp_slot;
             if (F == kInt4) {
@@ -448,13 +465,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // the leader's barrier
         if (lane == 0) {
             prefetch_tensormap(&x_map);
-            const uint64_t pol_x = l2_policy_evict_last();
+            // one token tile: read by every weight block; several: each is
+            // read by the pairs of one sweep and then not again
+            const uint64_t pol_x = p.mtiles > 1 ? l2_policy_evict_first() : l2_policy_evict_last();
             uint32_t it = 0;
             bool ok = true;
             for (int item = pair; item < p.num_items && ok; item += npairs) {
                 int tile, kb0, kb1;
                 item_range(p, item, tile, kb0, kb1);
-                const int mt = tile % p.mtiles;
+                const int mt = tile_mt(p, tile);
                 for (int kb = kb0; kb < kb1 && ok; ++kb, ++it) {
                     const int sx = it % L::kSX;
                     ok = role_wait(&x_empty[sx], ((it / L::kSX) & 1) ^ 1, abort_flag, p.hdr, 401);
@@ -473,8 +492,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             w_issue(0xffffffffu);
     } else if (warp == kMmaWarp) {
         if (rank == 0 && lane == 0) {
+            // One thread issues every MMA of the pair, so its own instruction
+            // latency bounds the rate at 128 tokens (a k-block's four MMAs
+            // take 256 tensor cycles): one barrier wait per k-block (the
+            // leader's dequantisers check the activations before they
+            // release a block), ring slots and phases kept incrementally,
+            // descriptors formed by addition.
             constexpr uint32_t idesc = idesc_pair<BT>();
-            uint32_t it = 0, tcount = 0;
+            const uint64_t xdesc0 = sw128_desc(smem_u32(smem + L::x_off));
+            uint32_t sx = 0, sa = 0, pa = 0, tcount = 0;
             bool ok = true;
             for (int item = pair; item < p.num_items && ok; item += npairs, ++tcount) {
                 int tile, kb0, kb1;
@@ -484,21 +510,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     break;
                 tc_fence_after();
                 const uint32_t d = tmem_base + L::acc_col;
-                for (int kb = kb0; kb < kb1; ++kb, ++it) {
-                    const int sx = it % L::kSX, sa = it % L::kSA;
-                    ok = role_wait(&x_full[sx], (it / L::kSX) & 1, abort_flag, p.hdr, 412) &&
-                         role_wait(&a_full[sa], (it / L::kSA) & 1, abort_flag, p.hdr, 413);
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    ok = role_wait(&a_full[sa], pa, abort_flag, p.hdr, 413);
                     if (!ok)
                         break;
                     tc_fence_after();
-                    const uint32_t xa = smem_u32(smem + L::x_off + sx * L::x_slot);
+                    const uint64_t bd = xdesc0 + (uint64_t)((sx * L::x_slot) >> 4);
                     const uint32_t a = tmem_base + L::a_col + 32 * sa;
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)
-                        tc_mma_ts_pair(d, a + 8 * k, sw128_desc(xa + 32 * k), idesc,
+                        tc_mma_ts_pair(d, a + 8 * k, bd + 2 * k, idesc,
                                        (kb > kb0 || k > 0) ? 1u : 0u);
                     tc_commit_pair(&x_empty[sx]);
                     tc_commit_pair(&a_empty[sa]);
+                    if (++sx == L::kSX)
+                        sx = 0;
+                    if (++sa == L::kSA) {
+                        sa = 0;
+                        pa ^= 1;
+                    }
                 }
                 if (ok)
                     tc_commit_pair(acc_full);
@@ -514,7 +544,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (!role_wait(acc_full, tcount & 1, abort_flag, p.hdr, 421))
                 break;
             tc_fence_after();
-            const int nb = tile / p.mtiles, mt = tile % p.mtiles;
+            const int nb = tile_nb(p, tile), mt = tile_mt(p, tile);
             const int nloc = (int)rank * BW + q * 32;                    // warp's first column in the pair
             const int n = nb * 2 * BW + nloc + lane;                      // this thread's column
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + L::acc_col;
@@ -617,12 +647,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int item = pair; item < p.num_items && ok; item += npairs) {
             int tile, kb0, kb1;
             item_range(p, item, tile, kb0, kb1);
-            const int nb = tile / p.mtiles;
-            for (int kb = kb0; kb < kb1; ++kb, ++it) {
-                const int sw = it % L::kSW, sa = it % L::kSA;
-                float sca[2] = {1.f, 1.f}, scb[2] = {1.f, 1.f};
+            const int nb = tile_nb(p, tile);
+            // k-block kb at ring position itk: its E8M0 scales (MXFP8)
+            auto mx_scales = [&](int kb, float (&sca)[2], float (&scb)[2]) {
+                sca[0] = sca[1] = scb[0] = scb[1] = 1.f;
                 if (F == kMxfp8) {
-                    // E8M0 scales of rows ra, ra + 8 for the two 32-blocks of this k-block
+                    // rows ra, ra + 8 for the two 32-blocks of this k-block
                     const int blocks = p.K / 32;
                     const long long ra =
                         (long long)nb * 2 * BW + (int)rank * BW + q * 32 + h * 16 + g;
@@ -640,27 +670,69 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         scb[b] = e8m0_to_f32(eb);
                     }
                 }
-                ok = role_wait(&wp_full[sw], (it / L::kSW) & 1, abort_flag, p.hdr, 431) &&
-                     role_wait(&a_empty[sa], ((it / L::kSA) & 1) ^ 1, abort_flag, p.hdr, 432);
+            };
+            auto ready = [&](uint32_t itk) -> bool {
+                return role_wait(&wp_full[itk % L::kSW], (itk / L::kSW) & 1, abort_flag, p.hdr,
+                                 431) &&
+                       role_wait(&a_empty[itk % L::kSA], ((itk / L::kSA) & 1) ^ 1, abort_flag,
+                                 p.hdr, 432);
+            };
+            auto decode = [&](uint32_t itk, const float (&sca)[2], const float (&scb)[2],
+                              uint32_t (&vv)[16]) {
+                const uint8_t *wp_slot = smem + L::wp_off + (itk % L::kSW) * L::wp_slot;
+                if (F == kInt4)
+                    dequant_int4(wp_slot, q, h, lane, p.G, gpk, vv);
+                else
+                    dequant_mx(wp_slot, q, h, lane, sca, scb, vv);
+            };
+            auto store = [&](uint32_t itk, const uint32_t (&vv)[16]) {
+                tmem_st_16x256b_x4(tmem_base + ((uint32_t)(q * 32 + h * 16) << 16) + L::a_col +
+                                       32 * (itk % L::kSA),
+                                   vv);
+            };
+            // the store of block itk has completed: hand the slot to the MMA
+            // and the packed weights back to their producer.  In the leader
+            // the block's activations must have landed too (the MMA thread
+            // waits on this barrier alone).
+            auto release = [&](uint32_t itk) {
+                if (rank == 0 && !role_wait(&x_full[itk % L::kSX], (itk / L::kSX) & 1, abort_flag,
+                                            p.hdr, 412))
+                    ok = false;
+                if (lane == 0) {
+                    mbar_arrive(&wp_empty[itk % L::kSW]);
+                    mbar_arrive_cluster(mapa_shared(smem_u32(&a_full[itk % L::kSA]), 0));
+                }
+            };
+            // Two k-blocks per pass: their decodes are independent chains the
+            // scheduler interleaves, so a warp keeps twice the work in flight
+            // (a lone block's decode is bound by its dependency latency, not
+            // by issue).  With one block left the second decode repeats it.
+            for (int kb = kb0; kb < kb1; kb += 2) {
+                const bool two = kb + 1 < kb1;
+                const uint32_t it1 = two ? it + 1 : it;
+                float sa0[2], sb0[2], sa1[2], sb1[2];
+                mx_scales(kb, sa0, sb0);
+                mx_scales(two ? kb + 1 : kb, sa1, sb1);
+                ok = ready(it) && (!two || ready(it + 1));
                 if (!ok)
                     break;
                 tc_fence_after();
-                const uint8_t *wp_slot = smem + L::wp_off + sw * L::wp_slot;
-                uint32_t v[16];
-                if (F == kInt4)
-                    dequant_int4(wp_slot, q, h, lane, p.G, gpk, v);
-                else
-                    dequant_mx(wp_slot, q, h, lane, sca, scb, v);
-                tmem_st_16x256b_x4(
-                    tmem_base + ((uint32_t)(q * 32 + h * 16) << 16) + L::a_col + 32 * sa, v);
+                uint32_t v0[16], v1[16];
+                decode(it, sa0, sb0, v0);
+                decode(it1, sa1, sb1, v1);
+                store(it, v0);
+                if (two)
+                    store(it1, v1);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&wp_empty[sw]);
-                    mbar_arrive_cluster(mapa_shared(smem_u32(&a_full[sa]), 0));
-                }
+                release(it);
+                if (two)
+                    release(it1);
+                it += two ? 2 : 1;
             }
+            if (!ok)
+                break;
         }
     }
 
