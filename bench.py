@@ -91,6 +91,9 @@ DEFAULT_CONFIGS = ["mtp4_verify_int4", "tiny_int4", "c32_mtp3_int4", "prefill_in
 MIN_STEPS = {"tiny_int4": 400, "mtp4_verify_int4": 200, "mtp4_verify_int4_fused": 200,
              "c32_mtp3_int4": 100, "prefill_int4": 10, "mxfp8_m4": 200, "mxfp8_m128": 100,
              "head_int8_m5": 20, "gdn_ab_bf16_m4": 400, "gdn_ab_bf16_m1": 400}
+# MXFP8 at M <= 16 runs on the re-packed layout (mxfp8_repack, once, outside
+# the timed region) through mxfp8_gemm_packed; larger M on the stored layout
+MXFP8_PACKED_MAX_M = 16
 KERNELS = {"bf16": "bf16_small_kernel", "int4": "w4a16_stream_kernel",
            "int8": "w4a16_stream_kernel", "mxfp8": "mxfp8_stream_kernel"}
 
@@ -108,6 +111,8 @@ def layer_weight_bytes(fmt, K, N, G):
 def kernel_of(fmt, M):
     if fmt in ("int4", "mxfp8") and M > 32:
         return "tc_gemm_kernel"
+    if fmt == "mxfp8" and M <= MXFP8_PACKED_MAX_M:
+        return "w4a16_stream_kernel"   # the re-packed MXFP8 variant of the weight stream
     return KERNELS[fmt]
 
 
@@ -117,7 +122,7 @@ def arith_dtype(fmt, M):
     exactly to 1024 + q or 1024 + 16 q, activations scaled per group by a
     power of two into fp16 exactly); every other path multiplies bf16
     operands.  Accumulation is fp32 throughout."""
-    return "f16" if fmt in ("int4", "int8") and M <= 16 else "bf16"
+    return "f16" if fmt in ("int4", "int8", "mxfp8") and M <= 16 else "bf16"
 
 
 def load_peaks():
@@ -280,9 +285,15 @@ class Workload:
                 lay = synth.mxfp8_layer(M, K, N, seed=rank, layer=li)
                 wq = torch.from_numpy(lay.Wq).to(dev)
                 ws = torch.from_numpy(lay.Ws).to(dev)
-                self.weights.append([(wq, ws)] + [(wq.clone(), ws.clone())
-                                                  for _ in range(self.pool - 1)])
-                need = mxg.mxfp8_workspace_bytes(M, N, K)
+                if M <= MXFP8_PACKED_MAX_M:
+                    packed = mxg.mxfp8_repack(wq, ws)
+                    del wq, ws
+                    self.weights.append([packed] + [packed.clone() for _ in range(self.pool - 1)])
+                    need = mxg.mxfp8_packed_workspace_bytes(M, N, K)
+                else:
+                    self.weights.append([(wq, ws)] + [(wq.clone(), ws.clone())
+                                                      for _ in range(self.pool - 1)])
+                    need = mxg.mxfp8_workspace_bytes(M, N, K)
             self.wss.append(torch.zeros(need, dtype=torch.uint8, device=dev))
             self.xs.append(torch.from_numpy(lay.X.view(np.int16)).view(torch.bfloat16).to(dev))
             self.ys.append(torch.empty((M, N), dtype=torch.bfloat16, device=dev))
@@ -302,6 +313,8 @@ class Workload:
             mxg.w8a16_gemm(x, w, N, K, G, out=y, workspace_buf=self.wss[li], stream=s)
         elif fmt == "bf16":
             mxg.bf16_gemm_small(x, w, out=y, workspace_buf=self.wss[li], stream=s)
+        elif self.M <= MXFP8_PACKED_MAX_M:
+            mxg.mxfp8_gemm_packed(x, w, N, K, out=y, workspace_buf=self.wss[li], stream=s)
         else:
             mxg.mxfp8_gemm(x, w[0], w[1], out=y, workspace_buf=self.wss[li], stream=s)
 

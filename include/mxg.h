@@ -288,6 +288,49 @@ MXG_API int mxfp8_gemm_ex(const void *X, const uint8_t *Wq, const uint8_t *Ws, i
                int K, void *Y, void *workspace, size_t workspace_bytes,
                const mxg_gemm_options *opts, cudaStream_t stream);
 
+/* Re-packed MXFP8 for the decode shapes: this library's arrangement of the
+ * format's codes and scales (the format fixes the values, not the layout).
+ * The codes and E8M0 scales are laid out by column groups of 256 so that a
+ * group's 128 rows of K are one contiguous range, like the INT4 layout;
+ * mxfp8_gemm_packed streams them with one bulk copy per stage, converts
+ * E4M3 pairs to f16 pairs in hardware (exact), multiplies on fp16 tensor
+ * cores against the activations converted to fp16 with a power-of-two
+ * factor per 64 rows of K and token (exact unless a value is 2^28 times
+ * smaller than the largest of its 64), and applies 2^(E - 127) per 32-k
+ * block in fp32.
+ * Packed bytes: N*K codes then N*K/32 scales; 0 for a rejected shape
+ * (N % 64 == 0 and K % 64 == 0 are required). */
+MXG_API size_t mxfp8_packed_bytes(int N, int K);
+
+/* Offline re-pack: Wq device E4M3 [N][K], Ws device E8M0 [N][K/32], packed
+ * device, mxfp8_packed_bytes(N, K) bytes (all 16-byte aligned, else
+ * MXG_ERR_INVALID_ARG).  MXG_ERR_UNSUPPORTED_SHAPE unless N % 64 == 0 and
+ * K % 64 == 0.  Asynchronous on `stream`; Wq and Ws may be freed once the
+ * stream has passed the call. */
+MXG_API int mxfp8_repack(const uint8_t *Wq, const uint8_t *Ws, int N, int K, void *packed,
+                 cudaStream_t stream);
+
+/* Workspace bytes mxfp8_gemm_packed needs (0 for a rejected shape, M > 16,
+ * or activations too wide to stay resident). */
+MXG_API size_t mxfp8_packed_workspace_bytes(int M, int N, int K);
+
+/* Y = X * dequant(W)^T from mxfp8_repack's buffer: the same result as
+ * mxfp8_gemm on the original Wq, Ws up to fp32 summation order.
+ *   X device bf16 [M][K]; packed as above; Y device bf16 [M][N];
+ *   workspace as for w4a16_gemm, sized by mxfp8_packed_workspace_bytes.
+ * 1 <= M <= 16 (the weight-streaming path only; larger M goes to mxfp8_gemm
+ * with the original layout), N % 64 == 0, K % 64 == 0, and the CTA's
+ * activations must fit in shared memory beside the ring; else
+ * MXG_ERR_UNSUPPORTED_SHAPE. */
+MXG_API int mxfp8_gemm_packed(const void *X, const void *packed, int M, int N, int K, void *Y,
+               void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* mxfp8_gemm_packed with per-call options (NULL = defaults; path
+ * MXG_PATH_TENSOR is MXG_ERR_INVALID_ARG). */
+MXG_API int mxfp8_gemm_packed_ex(const void *X, const void *packed, int M, int N, int K,
+               void *Y, void *workspace, size_t workspace_bytes,
+               const mxg_gemm_options *opts, cudaStream_t stream);
+
 /* ------------------------------------- dense bf16, few output columns */
 
 /* Y = X * W^T with dense bf16 weights, for the paired GDN A/B projection of

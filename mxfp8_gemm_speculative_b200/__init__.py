@@ -50,6 +50,11 @@ _SIGS = {
     "mxfp8_workspace_bytes": (_sz, [_i, _i, _i]),
     "mxfp8_gemm": (_i, [_p, _p, _p, _i, _i, _i, _p, _p, _sz, _p]),
     "mxfp8_gemm_ex": (_i, [_p, _p, _p, _i, _i, _i, _p, _p, _sz, _p, _p]),
+    "mxfp8_packed_bytes": (_sz, [_i, _i]),
+    "mxfp8_repack": (_i, [_p, _p, _i, _i, _p, _p]),
+    "mxfp8_packed_workspace_bytes": (_sz, [_i, _i, _i]),
+    "mxfp8_gemm_packed": (_i, [_p, _p, _i, _i, _i, _p, _p, _sz, _p]),
+    "mxfp8_gemm_packed_ex": (_i, [_p, _p, _i, _i, _i, _p, _p, _sz, _p, _p]),
     "w4a16_unpack": (_i, [_p, _i, _i, _i, _p, _p, _p, _p]),
     "mxfp8_dequant": (_i, [_p, _p, _i, _i, _p, _p]),
     "mxg_workspace_status": (_i, [_p, ctypes.POINTER(_i), _p]),
@@ -482,6 +487,52 @@ def mxfp8_gemm(x: torch.Tensor, wq: torch.Tensor, ws: torch.Tensor,
                                 lambda: _need_bytes("mxfp8", x.device.index, M, N, K), stream)
     _dev_call(x.device, "mxfp8_gemm", _lib.mxfp8_gemm_ex, _ptr(x), _ptr(wq), _ptr(ws), M, N, K,
               _ptr(out), _ptr(wsb), wsb.numel(), _options(path, late_weights), stream=stream)
+    return out
+
+
+def mxfp8_repack(wq: torch.Tensor, ws: torch.Tensor, stream=None) -> torch.Tensor:
+    """Re-pack E4M3 wq[N][K] and E8M0 ws[N][K/32] for mxfp8_gemm_packed."""
+    if wq.dtype not in (torch.uint8, torch.float8_e4m3fn):
+        raise ValueError("wq must be uint8 or float8_e4m3fn")
+    if ws.dtype not in (torch.uint8, torch.float8_e8m0fnu):
+        raise ValueError("ws must be uint8 or float8_e8m0fnu")
+    if wq.dim() != 2:
+        raise ValueError("wq must be [N][K]")
+    N, K = wq.shape
+    nbytes = int(_lib.mxfp8_packed_bytes(N, K))
+    if nbytes == 0:
+        raise MxgError(MXG_ERR_UNSUPPORTED_SHAPE, "mxfp8_repack")
+    _need_shape(ws, (N, K // 32), "ws")
+    _need(wq, wq.dtype, "wq")
+    _need(ws, ws.dtype, "ws")
+    _same_device(ws, wq.device, "ws")
+    packed = _empty(nbytes, torch.uint8, wq.device, stream)
+    _dev_call(wq.device, "mxfp8_repack", _lib.mxfp8_repack, _ptr(wq), _ptr(ws), N, K,
+              _ptr(packed), stream=stream)
+    return packed
+
+
+def _mxp_ws_bytes(M: int, N: int, K: int) -> int:
+    need = int(_lib.mxfp8_packed_workspace_bytes(M, N, K))
+    if need == 0:
+        raise MxgError(MXG_ERR_UNSUPPORTED_SHAPE, "mxfp8_gemm_packed")
+    return need
+
+
+def mxfp8_packed_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(_lib.mxfp8_packed_workspace_bytes(M, N, K))
+
+
+def mxfp8_gemm_packed(x: torch.Tensor, packed: torch.Tensor, N: int, K: int,
+                      out: torch.Tensor | None = None, workspace_buf: torch.Tensor | None = None,
+                      stream=None, late_weights: bool = False) -> torch.Tensor:
+    """Y = x * dequant(W)^T for x bf16 [M][K] (M <= 16) and mxfp8_repack's buffer."""
+    M, out, ws = _gemm_buffers(x, K, N, out, workspace_buf,
+                               lambda: _mxp_ws_bytes(x.shape[0], N, K), stream)
+    _need_weights(packed, torch.uint8, int(_lib.mxfp8_packed_bytes(N, K)), x.device, "packed")
+    _dev_call(x.device, "mxfp8_gemm_packed", _lib.mxfp8_gemm_packed_ex, _ptr(x), _ptr(packed), M,
+              N, K, _ptr(out), _ptr(ws), ws.numel(), _options(PATH_AUTO, late_weights),
+              stream=stream)
     return out
 
 

@@ -454,6 +454,72 @@ int mxfp8_gemm(const void *X, const uint8_t *Wq, const uint8_t *Ws, int M, int N
     return mxfp8_gemm_ex(X, Wq, Ws, M, N, K, Y, workspace, workspace_bytes, nullptr, stream);
 }
 
+namespace {
+bool mxfp8_packed_shape_ok(int K, int N)
+{
+    return K > 0 && N > 0 && K % 64 == 0 && N % 64 == 0;
+}
+}  // namespace
+
+size_t mxfp8_packed_bytes(int N, int K)
+{
+    if (!mxfp8_packed_shape_ok(K, N))
+        return 0;
+    return (size_t)N * K + (size_t)N * (K / 32);
+}
+
+int mxfp8_repack(const uint8_t *Wq, const uint8_t *Ws, int N, int K, void *packed,
+                 cudaStream_t stream)
+{
+    if (!aligned16(Wq) || !aligned16(Ws) || !aligned16(packed))
+        return MXG_ERR_INVALID_ARG;
+    if (!mxfp8_packed_shape_ok(K, N))
+        return MXG_ERR_UNSUPPORTED_SHAPE;
+    return to_status(launch_mxfp8_repack(Wq, Ws, N, K, packed, stream));
+}
+
+size_t mxfp8_packed_workspace_bytes(int M, int N, int K)
+{
+    if (M < 1 || M > 16 || !mxfp8_packed_shape_ok(K, N))
+        return 0;
+    const int dev = current_device();
+    if (dev < 0)
+        return 0;
+    StreamPlan sp;
+    if (!plan_mxfp8_packed_stream(dev, M, N, K, &sp))
+        return 0;
+    return make_workspace_map(sp.ntiles, sp.partial_bytes).total;
+}
+
+int mxfp8_gemm_packed_ex(const void *X, const void *packed, int M, int N, int K, void *Y,
+                         void *workspace, size_t workspace_bytes, const mxg_gemm_options *opts,
+                         cudaStream_t stream)
+{
+    int forced = 0;
+    bool early = true;
+    if (!resolve_options(opts, &forced, &early) || forced == MXG_PATH_TENSOR)
+        return MXG_ERR_INVALID_ARG;   // the re-packed layout has the weight-streaming path only
+    if (!aligned16(X) || !aligned16(packed) || !aligned16(Y) || !aligned16(workspace) || M < 1)
+        return MXG_ERR_INVALID_ARG;
+    if (M > 16 || !mxfp8_packed_shape_ok(K, N))
+        return MXG_ERR_UNSUPPORTED_SHAPE;
+    const int dev = current_device();
+    if (dev < 0)
+        return MXG_ERR_CUDA;
+    StreamPlan sp;
+    if (!plan_mxfp8_packed_stream(dev, M, N, K, &sp))
+        return MXG_ERR_UNSUPPORTED_SHAPE;
+    if (workspace_bytes < make_workspace_map(sp.ntiles, sp.partial_bytes).total)
+        return MXG_ERR_WORKSPACE;
+    return to_status(launch_w4a16_stream(sp, X, packed, M, N, K, 64, Y, workspace, early, stream));
+}
+
+int mxfp8_gemm_packed(const void *X, const void *packed, int M, int N, int K, void *Y,
+                      void *workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    return mxfp8_gemm_packed_ex(X, packed, M, N, K, Y, workspace, workspace_bytes, nullptr, stream);
+}
+
 int w4a16_unpack(const void *packed, int K, int N, int group_size, uint8_t *codes, float *w_fp32,
                  uint16_t *w_bf16, cudaStream_t stream)
 {

@@ -243,6 +243,13 @@ __device__ __forceinline__ uint4 lds128(const void *p)
     return v;
 }
 
+__device__ __forceinline__ uint32_t lds32a(uint32_t a)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+
 __device__ __forceinline__ uint32_t lds32(const void *p)
 {
     uint32_t v;
@@ -445,6 +452,18 @@ __device__ __forceinline__ uint32_t scale_pair_rn(uint32_t qm8, const ScaleSplit
 __device__ __forceinline__ float e8m0_to_f32(uint32_t e)
 {
     return e ? __uint_as_float(e << 23) : __uint_as_float(0x00400000u);
+}
+
+// Four E4M3 codes (the bytes of w, byte 0 first) as two f16 pairs: r01 =
+// (w0, w1), r23 = (w2, w3); exact (every E4M3 value is an f16 value).
+__device__ __forceinline__ void e4m3x2_f16x2(uint32_t w, uint32_t &r01, uint32_t &r23)
+{
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "mov.b32 {lo, hi}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, lo;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+        : "=r"(r01), "=r"(r23)
+        : "r"(w));
 }
 
 // Four E4M3 codes (the bytes of w, byte 0 first) times `scale`, as two bf16

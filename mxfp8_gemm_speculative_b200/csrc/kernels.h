@@ -61,6 +61,9 @@ bool plan_w4a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan)
 // INT8 W8A16 (two code planes) on the same kernel; launch_w4a16_stream runs
 // either plan.
 bool plan_w8a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan);
+// Re-packed MXFP8 (mxfp8_repack) on the same kernel, M <= 16; launch with
+// launch_w4a16_stream and G = 64.
+bool plan_mxfp8_packed_stream(int device, int M, int N, int K, StreamPlan *plan);
 // early: load the first weights before waiting for the previous kernel on
 // the stream (every launch function below takes it per call).
 cudaError_t launch_w4a16_stream(const StreamPlan &plan, const void *X, const void *packed, int M,
@@ -120,6 +123,8 @@ cudaError_t launch_w8a16_repack(const int32_t *qweight, const uint16_t *scales, 
                                 bool n_major, void *packed, cudaStream_t stream);
 cudaError_t launch_w4a16_unpack(const void *packed, int K, int N, int G, uint8_t *codes,
                                 float *w_fp32, uint16_t *w_bf16, cudaStream_t stream);
+cudaError_t launch_mxfp8_repack(const uint8_t *Wq, const uint8_t *Ws, int N, int K, void *packed,
+                               cudaStream_t stream);
 cudaError_t launch_mxfp8_dequant(const uint8_t *Wq, const uint8_t *Ws, int N, int K,
                                  uint16_t *w_bf16, cudaStream_t stream);
 cudaError_t launch_wait_timeout_selftest(void *workspace, int limit_us, cudaStream_t stream);

@@ -381,7 +381,7 @@ __device__ __forceinline__ void finish_cut(const Params &p, float4 (&sum)[2 * TT
 }
 
 // ------------------------------------------------------------------- kernel
-template <int TT, int GM, int P, int XR>
+template <int TT, int GM, int P, int XR, int MX>
 __global__ void __launch_bounds__(Cfg<TT, GM, P, XR>::kThreads, 1)
     w4a16_stream_kernel(const __grid_constant__ CUtensorMap xmap, const Params p)
 {
@@ -561,7 +561,82 @@ __global__ void __launch_bounds__(Cfg<TT, GM, P, XR>::kThreads, 1)
             const uint32_t st = sb + slot * C::kStage;
             const uint32_t cs = st + C::kX + wt * 1024 * P + lane * 16;
             const uint32_t ss = st + C::kX + C::kCodeMax + wt * 64 + g * 8;
-            if (live) {
+            if (MX && live) {
+                // MXFP8: per k64 chunk and tile, [half][pair of steps][lane][16 B];
+                // step j of the lane holds (row na, nb) x k0 .. k0 + 3 as
+                // E4M3 pairs (na k0 k0+1 | nb k0 k0+1), (na k0+2 k0+3 | nb ...),
+                // which the hardware converts to f16 pairs exactly; a partial
+                // per 32-k block is scaled by 2^(E - 127) and the window factor
+#pragma unroll
+                for (int ch = 0; ch < kChunks; ++ch) {
+                    if (ch > 0 && k0 + 64 * ch >= p.K)
+                        break;   // the last stage of a row may hold one chunk
+                    const uint32_t cp = cs + ch * nt * 2048;
+                    uint4 wq[2][2];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int q = 0; q < 2; ++q)
+                            wq[h][q] = lds128a(cp + h * 1024 + q * 512);
+                    const uint32_t xk = xrow + (k0 + 64 * ch) * 2;
+                    // window factors of the chunk (table group = chunk)
+                    float2 fx[TT];
+                    {
+                        const uint32_t xa =
+                            sb + p.xs_off + ((xg0 + k0 / C::kG + ch) * 8 * TT + 2 * t) * 8;
+#pragma unroll
+                        for (int tt = 0; tt < TT; ++tt) {
+                            const uint4 tv = lds128a(xa + tt * 64);
+                            fx[tt] = make_float2(__uint_as_float(tv.y), __uint_as_float(tv.w));
+                        }
+                    }
+#pragma unroll
+                    for (int b = 0; b < 2; ++b) {
+                        // E8M0 of rows na, nb (half 0) and na, nb (half 1)
+                        const uint32_t s4 = lds32a(st + C::kX + C::kCodeMax + (ch * nt + wt) * 64 +
+                                                   b * 32 + g * 4);
+                        const float sc[2][2] = {{e8m0_to_f32(s4 & 0xFF), e8m0_to_f32((s4 >> 8) & 0xFF)},
+                                                {e8m0_to_f32((s4 >> 16) & 0xFF), e8m0_to_f32(s4 >> 24)}};
+#pragma unroll
+                        for (int jj = 0; jj < 2; ++jj) {
+                            const int j = 2 * b + jj;
+                            uint2 xf[TT];
+#pragma unroll
+                            for (int tt = 0; tt < TT; ++tt)
+                                xf[tt] = lds64a(xk + tt * 8 * xstride + 32 * j);
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                const uint32_t w0 = jj ? wq[h][b].z : wq[h][b].x;
+                                const uint32_t w1 = jj ? wq[h][b].w : wq[h][b].y;
+                                uint32_t a0, a1, a2, a3;
+                                e4m3x2_f16x2(w0, a0, a1);
+                                e4m3x2_f16x2(w1, a2, a3);
+#pragma unroll
+                                for (int tt = 0; tt < TT; ++tt) {
+                                    if (jj == 0)
+                                        mma_f16_16816_zero(part[h][tt], a0, a1, a2, a3, xf[tt].x,
+                                                           xf[tt].y);
+                                    else
+                                        mma_f16_16816(part[h][tt], a0, a1, a2, a3, xf[tt].x,
+                                                      xf[tt].y);
+                                }
+                            }
+                        }
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+#pragma unroll
+                            for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    // outputs e and e ^ 2 are rows g, g + 8 of
+                                    // token 2t + (e & 1)
+                                    const float f = (e & 1) ? fx[tt].y : fx[tt].x;
+                                    acc[h][tt][e] =
+                                        fmaf(part[h][tt][e], sc[h][e >> 1] * f, acc[h][tt][e]);
+                                }
+                    }
+                }
+            } else if (live) {
 #pragma unroll
                 for (int ch = 0; ch < kChunks; ++ch) {
                     if (ch > 0 && k0 + 64 * ch >= p.K)
@@ -803,11 +878,23 @@ __global__ void __launch_bounds__(Cfg<TT, GM, P, XR>::kThreads, 1)
     }
 }
 
-// variant = group mode + 3 * (INT8) + 6 * (resident activations)
+// variant = group mode + 3 * (INT8) + 6 * (resident activations), or 12:
+// MXFP8 (64-k scale chunks, two bytes per tile lane and step, resident
+// activations)
+template <int V>
+struct VariantOf {
+    static constexpr int kGM = V == 12 ? 1 : V % 3;
+    static constexpr int kP = V == 12 ? 2 : (V / 3) % 2 + 1;
+    static constexpr int kXR = V == 12 ? 1 : V / 6;
+    static constexpr int kMX = V == 12 ? 1 : 0;
+};
+
 template <int TT, int V>
 const void *kernel_ptr()
 {
-    return reinterpret_cast<const void *>(&w4a16_stream_kernel<TT, V % 3, (V / 3) % 2 + 1, V / 6>);
+    using W = VariantOf<V>;
+    return reinterpret_cast<const void *>(
+        &w4a16_stream_kernel<TT, W::kGM, W::kP, W::kXR, W::kMX>);
 }
 
 const void *select_kernel(int tt, int variant)
@@ -818,6 +905,7 @@ const void *select_kernel(int tt, int variant)
     MXG_CASE(1, 6) MXG_CASE(1, 7) MXG_CASE(1, 8) MXG_CASE(1, 9) MXG_CASE(1, 10) MXG_CASE(1, 11)
     MXG_CASE(2, 0) MXG_CASE(2, 1) MXG_CASE(2, 2) MXG_CASE(2, 3) MXG_CASE(2, 4) MXG_CASE(2, 5)
     MXG_CASE(2, 6) MXG_CASE(2, 7) MXG_CASE(2, 8) MXG_CASE(2, 9) MXG_CASE(2, 10) MXG_CASE(2, 11)
+    MXG_CASE(1, 12) MXG_CASE(2, 12)
     MXG_CASE(3, 0) MXG_CASE(3, 1) MXG_CASE(3, 2) MXG_CASE(3, 3) MXG_CASE(3, 4) MXG_CASE(3, 5)
     MXG_CASE(4, 0) MXG_CASE(4, 1) MXG_CASE(4, 2) MXG_CASE(4, 3) MXG_CASE(4, 4) MXG_CASE(4, 5)
 #undef MXG_CASE
@@ -831,7 +919,8 @@ struct VariantCfg {
 template <int TT, int V>
 VariantCfg cfg_one()
 {
-    using C = Cfg<TT, V % 3, (V / 3) % 2 + 1, V / 6>;
+    using W = VariantOf<V>;
+    using C = Cfg<TT, W::kGM, W::kP, W::kXR>;
     return {C::kStage, C::kXchg, C::kThreads, C::kConsumers, C::kG, C::kXBox};
 }
 
@@ -843,6 +932,7 @@ VariantCfg variant_cfg(int tt, int v)
     MXG_CFG(1, 6) MXG_CFG(1, 7) MXG_CFG(1, 8) MXG_CFG(1, 9) MXG_CFG(1, 10) MXG_CFG(1, 11)
     MXG_CFG(2, 0) MXG_CFG(2, 1) MXG_CFG(2, 2) MXG_CFG(2, 3) MXG_CFG(2, 4) MXG_CFG(2, 5)
     MXG_CFG(2, 6) MXG_CFG(2, 7) MXG_CFG(2, 8) MXG_CFG(2, 9) MXG_CFG(2, 10) MXG_CFG(2, 11)
+    MXG_CFG(1, 12) MXG_CFG(2, 12)
     MXG_CFG(3, 0) MXG_CFG(3, 1) MXG_CFG(3, 2) MXG_CFG(3, 3) MXG_CFG(3, 4) MXG_CFG(3, 5)
     MXG_CFG(4, 0) MXG_CFG(4, 1) MXG_CFG(4, 2) MXG_CFG(4, 3) MXG_CFG(4, 4) MXG_CFG(4, 5)
 #undef MXG_CFG
@@ -873,10 +963,13 @@ SmemPlan smem_plan(const VariantCfg &vc, int R, int xbytes, int xsbytes)
     return s;
 }
 
-// bits: 4 (INT4) or 8 (INT8, two code planes)
+// bits: 4 (INT4), 8 (INT8, two code planes) or 0 (re-packed MXFP8: G = 64
+// chunks, resident activations only, so M <= 16)
 bool plan_stream(int device, int M, int N, int K, int G, int bits, StreamPlan *plan)
 {
     if (M < 1 || M > 32 || N % 64 != 0 || K % 64 != 0 || K % G != 0)
+        return false;
+    if (bits == 0 && (G != 64 || M > 16))
         return false;
     if (device < 0 || device >= kMaxDeviceCache)
         return false;
@@ -904,10 +997,10 @@ bool plan_stream(int device, int M, int N, int K, int G, int bits, StreamPlan *p
     pl.grid = pl.Wt;
     pl.split = S;
     const int q = (int)(pl.units / pl.Wt), r = (int)(pl.units % pl.Wt);
-    const int base = (bits == 8 ? 3 : 0) + group_mode(G);
+    const int base = bits == 0 ? 6 : (bits == 8 ? 3 : 0) + group_mode(G);
     const int budget = std::min(di.smem_optin, kMaxSmem);
     // resident activations for narrow token tiles, when they fit beside a
-    // ring of at least six stages: the largest windows over all runs
+    // deep enough ring: the largest windows over all runs
     bool xr = false;
     int xbytes = 0, xsbytes = 0;
     if (pl.tt <= 2) {
@@ -925,10 +1018,14 @@ bool plan_stream(int device, int M, int N, int K, int G, int bits, StreamPlan *p
         }
         xbytes = xcols * 2 * 8 * pl.tt;
         xsbytes = xgroups * 8 * pl.tt * 8;   // (sum, factor) per group and token
+        // at least six stages (96 KB of INT4 codes), four for MXFP8's
+        // twice larger stages
         const VariantCfg vr = variant_cfg(pl.tt, base + 6);
-        if ((int)smem_plan(vr, 6, xbytes, xsbytes).total <= budget)
+        if ((int)smem_plan(vr, bits == 0 ? 4 : 6, xbytes, xsbytes).total <= budget)
             xr = true;
     }
+    if (bits == 0 && !xr)
+        return false;
     pl.variant = base + (xr ? 6 : 0);
     const VariantCfg vc = variant_cfg(pl.tt, pl.variant);
     if (!xr)
@@ -952,7 +1049,7 @@ bool plan_stream(int device, int M, int N, int K, int G, int bits, StreamPlan *p
         return false;
     // the attribute is set per device and variant to the largest shared
     // memory a launch may ask for
-    static std::atomic<int> occ_cache[kMaxDeviceCache][4][12];
+    static std::atomic<int> occ_cache[kMaxDeviceCache][4][13];
     std::atomic<int> &occ_slot = occ_cache[device][pl.tt - 1][pl.variant];
     if (occ_slot.load(std::memory_order_acquire) == 0) {
         if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, budget) !=
@@ -982,6 +1079,11 @@ bool plan_w8a16_stream(int device, int M, int N, int K, int G, StreamPlan *plan)
     return plan_stream(device, M, N, K, G, 8, plan);
 }
 
+bool plan_mxfp8_packed_stream(int device, int M, int N, int K, StreamPlan *plan)
+{
+    return plan_stream(device, M, N, K, 64, 0, plan);
+}
+
 cudaError_t launch_w4a16_stream(const StreamPlan &pl, const void *X, const void *packed, int M,
                                 int N, int K, int G, void *Y, void *workspace, bool early,
                                 cudaStream_t stream)
@@ -991,7 +1093,7 @@ cudaError_t launch_w4a16_stream(const StreamPlan &pl, const void *X, const void 
     if (!fn)
         return cudaErrorInvalidValue;
     const VariantCfg vc = variant_cfg(pl.tt, pl.variant);
-    const int planes = (pl.variant / 3) % 2 + 1;
+    const int planes = pl.variant == 12 ? 2 : (pl.variant / 3) % 2 + 1;
     const uint8_t *codes = static_cast<const uint8_t *>(packed);
     alignas(64) CUtensorMap xmap;
     // X: bf16 [M][K], boxes of 64 k x 8 TT rows with 128-byte swizzle (used

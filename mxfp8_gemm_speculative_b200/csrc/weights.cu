@@ -229,6 +229,66 @@ __global__ void mxfp8_dequant_kernel(const uint32_t *__restrict__ Wq, const uint
     out[idx] = make_uint2(r01, r23);
 }
 
+// MXFP8 re-pack for the weight-streaming kernel, by column groups of eight
+// n32 tiles like the INT4 layout:
+//   codes  [N/256 groups][K/64 chunks][tiles of the group][2 halves][2 pairs of steps][32 lanes][16 B]
+//   scales [N/256 groups][K/64 chunks][tiles of the group][2 blocks][8][4 B]
+// Lane 4g + t of half h holds columns na = 32T + 16h + g and nb = na + 8;
+// for step j (k0 = 64c + 16j + 4t) its 8 bytes are the E4M3 codes
+// (na, k0) (na, k0+1) (nb, k0) (nb, k0+1) (na, k0+2) (na, k0+3) (nb, k0+2)
+// (nb, k0+3): the f16 pairs of one m16n8k16 A operand after the hardware
+// conversion, in the INT4 layout's k order.  Scale entry (T, c, b, g) holds
+// the E8M0 of block 2c + b for columns 32T + g, +8, +16, +24.
+__global__ void mxfp8_repack_codes_kernel(const uint32_t *__restrict__ Wq, int N, int K,
+                                          int ntiles, uint8_t *__restrict__ out)
+{
+    const long long total = (long long)(N / 32) * (K / 64) * 2 * 2 * 32;
+    const long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+    if (idx >= total)
+        return;
+    const int lane = (int)(idx & 31);
+    const int q = (int)((idx >> 5) & 1);      // pair of steps 2q, 2q + 1
+    const int h = (int)((idx >> 6) & 1);
+    const long long rest = idx >> 7;
+    const int kc_count = K / 64;
+    const int c = (int)(rest % kc_count);
+    const int T = (int)(rest / kc_count);
+    const int g = lane >> 2, t = lane & 3;
+    const size_t na = (size_t)T * 32 + h * 16 + g, nb = na + 8;
+    uint32_t w[4];
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+        const int k0 = chunk_k0(c, t, 2 * q + s);   // 4 codes of each column
+        const uint32_t qa = Wq[(na * K + k0) >> 2];
+        const uint32_t qb = Wq[(nb * K + k0) >> 2];
+        w[2 * s] = (qa & 0xFFFFu) | (qb << 16);
+        w[2 * s + 1] = (qa >> 16) | (qb & 0xFFFF0000u);
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(out + code_offset(T, c, K, ntiles, 2)) + (h * 2 + q) * 32;
+    dst[lane] = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__global__ void mxfp8_repack_scales_kernel(const uint8_t *__restrict__ Ws, int N, int K,
+                                           int ntiles, uint8_t *__restrict__ out)
+{
+    const long long total = (long long)(N / 32) * (K / 64) * 2 * 8;
+    const long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+    if (idx >= total)
+        return;
+    const int g = (int)(idx & 7);
+    const int b = (int)((idx >> 3) & 1);
+    const long long rest = idx >> 4;
+    const int kc_count = K / 64;
+    const int c = (int)(rest % kc_count);
+    const int T = (int)(rest / kc_count);
+    const size_t blocks = (size_t)K / 32, blk = (size_t)c * 2 + b, n0 = (size_t)T * 32 + g;
+    const uint32_t v = (uint32_t)Ws[n0 * blocks + blk] | ((uint32_t)Ws[(n0 + 8) * blocks + blk] << 8) |
+                       ((uint32_t)Ws[(n0 + 16) * blocks + blk] << 16) |
+                       ((uint32_t)Ws[(n0 + 24) * blocks + blk] << 24);
+    // scale_offset with G = 64: 64 bytes per tile and chunk
+    *reinterpret_cast<uint32_t *>(out + scale_offset(T, c, K, 64, ntiles) + b * 32 + g * 4) = v;
+}
+
 __global__ void wait_timeout_kernel(WsHeader *hdr, unsigned long long limit_ns)
 {
     __shared__ __align__(8) uint64_t bar;
@@ -317,6 +377,20 @@ cudaError_t launch_w4a16_unpack(const void *packed, int K, int N, int G, uint8_t
     const uint8_t *pk = static_cast<const uint8_t *>(packed);
     unpack_kernel<<<blocks_for(nchunks, 256), 256, 0, stream>>>(pk, pk + (size_t)N * K / 2, K, N, G,
                                                                 codes, w_fp32, w_bf16);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_mxfp8_repack(const uint8_t *Wq, const uint8_t *Ws, int N, int K, void *packed,
+                               cudaStream_t stream)
+{
+    uint8_t *out = static_cast<uint8_t *>(packed);
+    const long long nc = (long long)(N / 32) * (K / 64) * 128;
+    mxfp8_repack_codes_kernel<<<blocks_for(nc, 256), 256, 0, stream>>>(
+        reinterpret_cast<const uint32_t *>(Wq), N, K, N / 32, out);
+    const long long ns = (long long)(N / 32) * (K / 64) * 16;
+    mxfp8_repack_scales_kernel<<<blocks_for(ns, 256), 256, 0, stream>>>(Ws, N, K, N / 32,
+                                                                        out + (size_t)N * K);
+    repack_done_kernel<<<1, 32, 0, stream>>>();
     return cudaGetLastError();
 }
 
