@@ -424,21 +424,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int n32 = (nb * 2 * BW + (int)rank * BW) / 32;
             uint8_t *wdst = smem + L::wp_off + sw * L::wp_slot;
             if (F == kInt4) {
-                // this CTA's tiles of the column group (all four, or fewer
-                // in a last group of fewer than eight): codes of the k-block
-                // and the scales of its gpk groups, each one contiguous range
-                // per scale group
-                const int ntl = max(0, min(4, group_tiles(n32 >> 3, p.N / 32) - (n32 & 7)));
-                mbar_arrive_expect_tx(&wp_full[sw], (uint32_t)ntl * (1024u + 64u * gpk));
-                if (ntl > 0) {
-                    bulk_g2s(wdst, p.codes + code_offset(n32, w_kb, p.K, p.N / 32, 1),
-                             ntl * 1024, &wp_full[sw], pol_w);
-                    for (int gi = 0; gi < gpk; ++gi)
-                        bulk_g2s(wdst + 4096 + gi * 256,
-                                 p.scales + scale_offset(n32, w_kb * BK / p.G + gi, p.K, p.G,
-                                                         p.N / 32),
-                                 ntl * 64, &wp_full[sw], pol_w);
-                }
+                // this CTA's four tiles of the column group: the codes of the
+                // k-block (one 4 KB range) and the scales of its gpk groups
+                // (256 B each), as tensor-map boxes over rows of one tile's
+                // 1 KB of codes / 64 B of scales (the tensor engine moves
+                // these faster than plain bulk copies of the same bytes).
+                // In a last group of fewer than eight tiles the box's rows
+                // past the group belong to the next chunk or lie past the
+                // end (zero-filled): their columns are past N and unused.
+                mbar_arrive_expect_tx(&wp_full[sw], 4096u + 256u * gpk);
+                tma_load_2d(wdst, &w_map, 0,
+                            (int)(code_offset(n32, w_kb, p.K, p.N / 32, 1) >> 10), &wp_full[sw],
+                            pol_w);
+                for (int gi = 0; gi < gpk; ++gi)
+                    tma_load_2d(wdst + 4096 + gi * 256, &s_map, 0,
+                                (int)(scale_offset(n32, w_kb * BK / p.G + gi, p.K, p.G, p.N / 32) >> 6),
+                                &wp_full[sw], pol_w);
             } else {
                 mbar_arrive_expect_tx(&wp_full[sw], (uint32_t)(BW * BK));
                 tma_load_2d(wdst, &w_map, w_kb * BK, n32 * 32, &wp_full[sw], pol_w);
@@ -449,8 +450,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         return true;
     };
     if (warp == kWProducerWarp && lane == 0) {
-        if (F != kInt4)
-            prefetch_tensormap(&w_map);
+        prefetch_tensormap(&w_map);
+        if (F == kInt4)
+            prefetch_tensormap(&s_map);
         // The weights are not written by the previous kernel on the stream
         // (the caller's contract, unless it turned early weight loads off):
         // the first ring of them fills while that kernel drains.  Everything
@@ -834,14 +836,23 @@ cudaError_t launch_w4a16_tc(const TcPlan &pl, const void *X, const void *packed,
                             int K, int G, void *Y, void *workspace, bool early,
                             cudaStream_t stream)
 {
-    alignas(64) CUtensorMap xm;
+    alignas(64) CUtensorMap xm, wm, sm;
     const uint8_t *codes = static_cast<const uint8_t *>(packed);
-    if (!x_map(&xm, X, M, K, pl.bm))
+    if (!x_map(&xm, X, M, K, pl.bm) ||
+        // codes: rows of one tile's 1 KB for one k64 chunk (128 u64), in
+        // memory order; box = 4 rows (the CTA's four tiles of a chunk)
+        !encode_tensor_map_2d(&wm, CU_TENSOR_MAP_DATA_TYPE_UINT64, codes, 128,
+                              (uint64_t)(N / 32) * (K / 64), 1024, 128, BW / 32,
+                              CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        // scales: rows of one tile's 64 B for one group (8 u64); box = 4 rows
+        !encode_tensor_map_2d(&sm, CU_TENSOR_MAP_DATA_TYPE_UINT64, codes + (size_t)N * K / 2, 8,
+                              (uint64_t)(N / 32) * (K / G), 64, 8, BW / 32,
+                              CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     TcParams p{};
     p.Y = static_cast<uint16_t *>(Y);
     p.Ws = nullptr;
-    // weights are moved with bulk copies of the column-group layout
+    // weights are moved with tensor-map boxes over the column-group layout
     p.codes = codes;
     p.scales = codes + (size_t)N * K / 2;
     p.hdr = static_cast<WsHeader *>(workspace);
@@ -861,10 +872,9 @@ cudaError_t launch_w4a16_tc(const TcPlan &pl, const void *X, const void *packed,
         p.counters = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + wsm.counters_off);
         p.partial = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + wsm.partial_off);
     }
-    // the weight tensor-map parameters are unused on the INT4 path
     if (pl.bm == 128)
-        return tc_launch<kInt4, 128>(pl, xm, xm, xm, p, stream);
-    return tc_launch<kInt4, 256>(pl, xm, xm, xm, p, stream);
+        return tc_launch<kInt4, 128>(pl, xm, wm, sm, p, stream);
+    return tc_launch<kInt4, 256>(pl, xm, wm, sm, p, stream);
 }
 
 bool plan_mxfp8_tc(int device, int M, int N, int K, TcPlan *plan)
