@@ -19,12 +19,13 @@ e2e        the same metric through the public API with host buffers: per
            step the host-to-device copy of the step's X from pinned memory,
            the layers, the device-to-host copy of every Y, then a stream
            synchronize, timed on the host clock (e2e_graph: the same steps
-           captured as one CUDA graph over the pool slots and replayed, as a
-           serving loop does, timed with device events).
-timing     exactly --steps steps, replayed from CUDA graphs that hold one
-           step on every slot of the weight pool in turn (the launches
-           overlap their neighbours through programmatic dependent launch
-           inside a replay), CUDA events on the launch stream.
+           captured as CUDA graphs over consecutive pool slots and replayed,
+           as a serving loop does, timed with device events).
+timing     exactly --steps steps, replayed from CUDA graphs of up to 16
+           consecutive steps on consecutive slots of the weight pool (the
+           launches overlap their neighbours through programmatic dependent
+           launch inside a replay), CUDA events on the launch stream;
+           median / p10 / p90 over the replays (ms per step).
 roofline   every layer of a step runs the same kernel, so the dominant
            kernel's time inside the step is the step time (its layers'
            in-step times add up to it exactly: each layer's share is the
@@ -299,6 +300,15 @@ class Workload:
             self.ys.append(torch.empty((M, N), dtype=torch.bfloat16, device=dev))
         self.kernel = kernel_of(fmt, M)
 
+    def round_pool(self, seg):
+        """Grow the weight pool to a multiple of `seg` slots (more copies of
+        the same weights), so graphs of `seg` steps tile it exactly."""
+        while self.pool % seg:
+            for w in self.weights:
+                w.append(w[0].clone() if not isinstance(w[0], tuple)
+                         else tuple(t.clone() for t in w[0]))
+            self.pool += 1
+
     def call(self, li, p, s, x=None, y=None):
         """Layer li on pool slot p, on stream s (X and Y default to the
         workload's device buffers)."""
@@ -329,28 +339,32 @@ def capture(torch, stream, fn):
     return g
 
 
-def time_cycles(torch, stream, full, rem, steps, pool, per_cycle_events):
-    """Device time of exactly `steps` steps: `steps // pool` replays of the
-    graph `full` (one step on every pool slot) and, when `pool` does not
-    divide `steps`, one replay of `rem` (the first steps % pool slots).  With
-    per_cycle_events, an event between replays gives the ms per step of
-    every full cycle."""
-    n_full, r = divmod(steps, pool)
-    n_ev = (n_full + 2) if per_cycle_events else 2
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+def segment_len(steps: int, pool: int) -> int:
+    """Steps per captured graph: the largest divisor of `steps` that is at
+    most min(pool, 16), so the timed region is whole replays."""
+    cap = max(1, min(pool, 16))
+    return max(d for d in range(1, cap + 1) if steps % d == 0)
+
+
+def time_segments(torch, stream, graphs, steps, seg, per_replay_events):
+    """Device time of exactly `steps` steps replayed as `steps // seg` graph
+    replays, graph i % len(graphs) at replay i (the graphs hold consecutive
+    runs of `seg` pool slots, so the replays walk the pool in order).  With
+    per_replay_events, an event between replays gives the ms per step of
+    every replay."""
+    n = steps // seg
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1 if per_replay_events else 2)]
     with torch.cuda.stream(stream):
         evs[0].record(stream)
-        for c in range(n_full):
-            full.replay()
-            if per_cycle_events:
-                evs[c + 1].record(stream)
-        if r:
-            rem.replay()
-        evs[-1].record(stream)
+        for i in range(n):
+            graphs[i % len(graphs)].replay()
+            if per_replay_events:
+                evs[i + 1].record(stream)
+        if not per_replay_events:
+            evs[1].record(stream)
     torch.cuda.synchronize()
     total = evs[0].elapsed_time(evs[-1])
-    per = ([evs[c].elapsed_time(evs[c + 1]) / pool for c in range(n_full)]
-           if per_cycle_events else [])
+    per = ([evs[i].elapsed_time(evs[i + 1]) / seg for i in range(n)] if per_replay_events else [])
     return total, per
 
 
@@ -382,33 +396,35 @@ def isolated_launch_us(torch, wl, stream, launches):
 
 def measure(wl, steps, warmup, world, dev, args, with_e2e):
     """Times one workload: exactly `steps` steps after `warmup`, replayed
-    from CUDA graphs that hold one step on every pool slot in turn (a
-    serving loop's graph of consecutive layers: the launches overlap their
-    neighbours through programmatic dependent launch, within a replay and
-    not across the replay boundary); per-cycle quantiles; in-step per-layer
-    times; one-launch-at-a-time kernel times; the e2e figures."""
+    from CUDA graphs of `seg` consecutive steps on consecutive weight-pool
+    slots (a serving loop's graph of consecutive layers: the launches overlap
+    their neighbours through programmatic dependent launch, within a replay
+    and not across the replay boundary); per-replay quantiles; in-step
+    per-layer times; one-launch-at-a-time kernel times; the e2e figures."""
     import torch
     import torch.distributed as dist
 
     stream = torch.cuda.Stream(dev)
     nl = len(wl.layers)
-    pool = wl.pool
-    r = steps % pool
+    seg = segment_len(steps, wl.pool)
+    wl.round_pool(seg)
+    nseg = wl.pool // seg
 
-    def cycle(j, slots):
-        # slots' steps, each cut after layer j (j = nl: whole steps)
-        return capture(torch, stream, lambda: [wl.call(li, p, stream)
-                                               for p in slots for li in range(j)])
+    def graphs_for(j):
+        # the pool's segments, each step cut after layer j (j = nl: whole steps)
+        return [capture(torch, stream, lambda o=o: [wl.call(li, p, stream)
+                                                    for p in range(o, o + seg)
+                                                    for li in range(j)])
+                for o in range(0, wl.pool, seg)]
 
     with torch.cuda.stream(stream):
         for li in range(nl):
             wl.call(li, 0, stream)          # plans and kernel attributes outside capture
         torch.cuda.synchronize(dev)
-        full = {j: cycle(j, range(pool)) for j in range(1, nl + 1)}
-        rem = {j: cycle(j, range(r)) for j in range(1, nl + 1)} if r else {}
+        graphs = {j: graphs_for(j) for j in range(1, nl + 1)}
     with torch.cuda.stream(stream):
-        for _ in range(-(-warmup // pool)):
-            full[nl].replay()
+        for i in range(max(nseg, -(-warmup // seg))):
+            graphs[nl][i % nseg].replay()
     torch.cuda.synchronize(dev)
     status = wl.status()
     if status:
@@ -416,17 +432,17 @@ def measure(wl, steps, warmup, world, dev, args, with_e2e):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    elapsed_ms, _ = time_cycles(torch, stream, full[nl], rem.get(nl), steps, pool, False)
+    elapsed_ms, _ = time_segments(torch, stream, graphs[nl], steps, seg, False)
     elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
-    # the distribution over full cycles (an event between replays), same steps
-    _, per_step = time_cycles(torch, stream, full[nl], rem.get(nl), steps, pool, True)
+    # the distribution over replays (an event between replays), same steps
+    _, per_step = time_segments(torch, stream, graphs[nl], steps, seg, True)
     # in-step share of every layer: steps cut after layer j minus steps cut
     # after layer j - 1
     in_step = []
     if nl > 1:
         prev = 0.0
         for j in range(1, nl + 1):
-            t, _ = time_cycles(torch, stream, full[j], rem.get(j), steps, pool, False)
+            t, _ = time_segments(torch, stream, graphs[j], steps, seg, False)
             in_step.append((t - prev) / steps * 1e3)
             prev = t
         # rescale so the shares add up to the whole-step time measured above
@@ -438,14 +454,14 @@ def measure(wl, steps, warmup, world, dev, args, with_e2e):
     if wl.status():
         raise RuntimeError(f"{wl.name}: kernel reported a status")
     res = {"elapsed_ms": elapsed_ms, "per_step_ms": per_step, "in_step_us": in_step,
-           "isolated_us": iso, "cycle_steps": pool}
+           "isolated_us": iso, "cycle_steps": seg}
     if with_e2e:
-        res.update(measure_e2e(wl, stream, steps, world, dev, args))
-    del full, rem
+        res.update(measure_e2e(wl, stream, steps, world, dev, args, seg))
+    del graphs
     return res
 
 
-def measure_e2e(wl, stream, steps, world, dev, args):
+def measure_e2e(wl, stream, steps, world, dev, args, seg):
     """End to end through the public API with host buffers."""
     import torch
     import torch.distributed as dist
@@ -481,20 +497,19 @@ def measure_e2e(wl, stream, steps, world, dev, args):
             stream.synchronize()            # the result is on the host
         eager_ms = (time.perf_counter() - t0) * 1e3
     eager_ms = max_over_ranks(eager_ms, world, dev)
-    # (2) the steps captured as one graph over the pool slots and replayed,
-    # device events
-    pool = wl.pool
-    r = e2e_steps % pool
+    # (2) the steps captured as graphs of `seg` consecutive pool slots and
+    # replayed, device events
+    eseg = segment_len(e2e_steps, seg)
     with torch.cuda.stream(stream):
-        full = capture(torch, stream, lambda: [step(p) for p in range(pool)])
-        rem = capture(torch, stream, lambda: [step(p) for p in range(r)]) if r else None
-        full.replay()
+        graphs = [capture(torch, stream, lambda o=o: [step(p) for p in range(o, o + eseg)])
+                  for o in range(0, wl.pool - eseg + 1, eseg)]
+        graphs[0].replay()
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
-    graph_ms, _ = time_cycles(torch, stream, full, rem, e2e_steps, pool, False)
+    graph_ms, _ = time_segments(torch, stream, graphs, e2e_steps, eseg, False)
     graph_ms = max_over_ranks(graph_ms, world, dev)
-    del full, rem
+    del graphs
     return {"e2e_steps": e2e_steps, "e2e_eager_ms": eager_ms, "e2e_graph_ms": graph_ms,
             "h2d": h2d, "d2h": d2h}
 
@@ -565,8 +580,8 @@ def summarize(wl, res, steps, world, peaks, peak_kind):
                               "synchronize; host clock"}
         out["e2e_graph"] = {"value": round(job_value(units, world, res["e2e_graph_ms"]) / scale, 4),
                             "unit": unit, "steps": n,
-                            "path": "the same steps captured as one CUDA graph over the pool "
-                                    "slots and replayed; device events"}
+                            "path": "the same steps captured as CUDA graphs over consecutive "
+                                    "pool slots and replayed; device events"}
     return out
 
 
@@ -620,9 +635,9 @@ def run_ours(args, rank, world, local_rank):
         "dtype": arith_dtype(WORKLOADS[args.workload][0], WORKLOADS[args.workload][1]),
         "data": "synthetic (seeded; the value distributions of the layer formats)",
         "config": dict(head["config"], **{
-            "timing": "CUDA graphs of one step on every weight-pool slot, replayed for exactly "
-                      "--steps steps, CUDA events on the launch stream; weights from a rotating "
-                      "pool >= 3 x L2 (inputs larger than L2)",
+            "timing": "CUDA graphs of up to 16 consecutive steps on consecutive weight-pool "
+                      "slots, replayed for exactly --steps steps, CUDA events on the launch "
+                      "stream; weights from a rotating pool >= 3 x L2 (inputs larger than L2)",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}),
         "step_ms_quantiles": head["step_ms_quantiles"],
         "tflops": head["tflops"],
