@@ -531,9 +531,17 @@ def summarize(wl, res, steps, world, peaks, peak_kind):
     hbm_gbs = wl.step_bytes / (k_us * 1e-6) / 1e9
     tflops = wl.step_flops / (k_us * 1e-6) / 1e12
     if tensor_bound:
-        roof = {"bound": "tensor", "achieved": round(tflops, 2), "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": round(tflops / peaks["bf16_tflops"], 4),
-                "peak_source": f"{peak_kind} bf16 dense (burst)",
+        # the sustained peak (a seconds-long cuBLAS loop under the power cap)
+        # for a timed region of back-to-back GEMMs longer than 0.1 s, the
+        # burst peak otherwise; both fractions are reported
+        sustained = elapsed_ms > 100.0
+        pk = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": round(tflops, 2), "peak": pk,
+                "unit": "TFLOP/s", "frac": round(tflops / pk, 4),
+                "peak_source": (f"{peak_kind} bf16 dense, sustained (timed region "
+                                f"{elapsed_ms / 1e3:.2f} s of back-to-back GEMMs)" if sustained
+                                else f"{peak_kind} bf16 dense (burst)"),
+                "frac_of_burst": round(tflops / peaks["bf16_tflops"], 4),
                 "frac_of_sustained": round(tflops / peaks["bf16_tflops_sustained"], 4)}
     else:
         roof = {"bound": "hbm", "achieved": round(hbm_gbs, 1), "peak": peaks["hbm_gbs"],
@@ -603,21 +611,24 @@ def run_ours(args, rank, world, local_rank):
         if n not in WORKLOADS:
             raise SystemExit(f"unknown workload {n}")
 
-    clocks = ClockSampler(local_rank)
-    clocks.start()
     results = {}
     for i, name in enumerate(names):
         head = i == 0
         wl = Workload(name, rank, dev, args.pool_factor)
         steps = args.steps if head else max(args.steps, MIN_STEPS.get(name, args.steps))
         warmup = args.warmup if head else max(args.warmup, 3)
+        # clocks sampled while this workload is measured
+        clocks = ClockSampler(local_rank)
+        clocks.start()
         res = measure(wl, steps, warmup, world, dev, args, with_e2e=head or args.e2e_all)
+        clk_w = clocks.stop()
         results[name] = summarize(wl, res, steps, world, peaks, peak_kind)
+        results[name]["clocks"] = clk_w
         del wl
         torch.cuda.empty_cache()
     if world > 1:
         dist.barrier()
-    clk = clocks.stop()
+    clk = results[args.workload]["clocks"]
 
     head = results[args.workload]
     props = torch.cuda.get_device_properties(dev)

@@ -55,9 +55,8 @@ enum Fmt { kInt4 = 0, kMxfp8 = 1 };
 template <int F, int BT>
 struct Layout {
     static constexpr int kSX = BT == 128 ? 8 : 5;    // activation ring
-    static constexpr int kSW = BT == 128 ? (F == kInt4 ? 24 : 16)
-                                         : (F == kInt4 ? 16 : 12);   // packed-weight ring
-    static constexpr int kSA = BT == 128 ? 12 : 8;   // tensor-memory A ring (32 columns each)
+    static constexpr int kSW = BT == 128 ? (F == kInt4 ? 24 : 16) : (F == kInt4 ? 16 : 12);   // packed-weight ring
+    static constexpr int kSA = BT == 128 ? 12 : 8;    // tensor-memory A ring (32 columns each)
     static constexpr int x_slot = (BT / 2) * BK * 2;                // bf16 activations
     static constexpr int wp_slot = (F == kInt4) ? 5120 : BW * BK;   // packed weights
     static constexpr int x_off = 0;
@@ -75,8 +74,6 @@ struct Layout {
 struct TcParams {
     uint16_t *Y;
     const uint8_t *Ws;     // MXFP8 scales [N][K/32]
-    const uint8_t *codes;  // INT4: re-packed codes (column-group layout, common.cuh)
-    const uint8_t *scales; // INT4: re-packed scales
     WsHeader *hdr;
     float *partial;        // split-K partial sums [num_items][BT][2 * BW] (splits > 1)
     int *counters;         // split-K arrivals per (tile, CTA of the pair, quadrant)
@@ -92,7 +89,7 @@ struct TcParams {
 // several token tiles the tiles run token-tile-major: the pairs working at
 // the same time share one activation tile and sweep all weight blocks, which
 // stay in L2 (marked evict-last) from one token tile to the next, so each
-// weight and activation byte is read from DRAM about once.
+// weight and activation byte is read from DRAM a few times at most.
 __device__ __forceinline__ int tile_nb(const TcParams &p, int tile)
 {
     return p.mtiles > 1 ? tile % p.ntiles : tile / p.mtiles;
@@ -288,8 +285,7 @@ __device__ __forceinline__ void dequant_int4(const uint8_t *wp_slot, int q, int 
     const int g = lane >> 2;
     const uint4 c = lds128(wp_slot + q * 1024 + h * 512 + lane * 16);
     const uint32_t w[4] = {c.x, c.y, c.z, c.w};
-    // words 0-1 and 2-3 lie in one scale group each (the same one for G >= 64);
-    // the slot holds the scales as [gpk groups][4 tiles][64 B]
+    // words 0-1 and 2-3 lie in one scale group each (the same one for G >= 64)
     (void)gpk;
     const uint8_t *sbase = wp_slot + 4096 + q * 64 + g * 8 + h * 4;
     const uint32_t sw0 = lds32(sbase);
@@ -380,15 +376,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         item_range(p, pair, tile0, kb0, kb1);
         const int nb = tile_nb(p, tile0), mt = tile_mt(p, tile0);
         const int n32 = (nb * 2 * BW + (int)rank * BW) / 32;
-        const int ntl = F == kInt4 ? max(0, min(4, group_tiles(nb, p.N / 32) - 4 * (int)rank)) : 0;
         for (int kb = kb0; kb < min(kb0 + L::kSW, kb1); ++kb) {
             prefetch_tensor_l2(&x_map, kb * BK, mt * BT + (int)rank * (BT / 2));
-            if (F == kInt4) {
-                if (ntl > 0)
-                    prefetch_l2(p.codes + code_offset(n32, kb, p.K, p.N / 32, 1), ntl * 1024);
-            } else {
+            if (F == kInt4)
+                prefetch_tensor_l2(&w_map, 0, (int)(code_offset(n32, kb, p.K, p.N / 32, 1) >> 10));
+            else
                 prefetch_tensor_l2(&w_map, kb * BK, n32 * 32);
-            }
         }
     }
     tc_fence_before();
@@ -407,8 +400,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (w_item < p.num_items)
         item_range(p, w_item, w_tile, w_kb, w_kb1);
     auto w_issue = [&](uint32_t until) -> bool {
-        // weights stream once when there is one token tile, else they are
-        // read again by every token tile
+        // weights stream once when there is one token tile, else every token
+        // tile reads them again
         const uint64_t pol_w = p.mtiles > 1 ? l2_policy_evict_last() : l2_policy_evict_first();
         while (w_item < p.num_items && w_it < until) {
             if (w_kb >= w_kb1) {
@@ -424,18 +417,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int n32 = (nb * 2 * BW + (int)rank * BW) / 32;
             uint8_t *wdst = smem + L::wp_off + sw * L::wp_slot;
             if (F == kInt4) {
-                // this CTA's four tiles of the column group: the codes of the
-                // k-block (one 4 KB range) and the scales of its gpk groups
-                // (256 B each), as tensor-map boxes over rows of one tile's
-                // 1 KB of codes / 64 B of scales (the tensor engine moves
-                // these faster than plain bulk copies of the same bytes).
-                // In a last group of fewer than eight tiles the box's rows
-                // past the group belong to the next chunk or lie past the
-                // end (zero-filled): their columns are past N and unused.
+                // the CTA's four tiles of the column group for this k-block:
+                // one 4-row box of codes (a row = one tile's 1 KB of a k64
+                // chunk, rows in memory order) and one 4-row box of scales
+                // per scale group (a row = one tile's 64 B).  In a last group
+                // of fewer than eight tiles the rows past the group belong to
+                // the next chunk or lie past the end (zero-filled): their
+                // columns are past N and never stored.
                 mbar_arrive_expect_tx(&wp_full[sw], 4096u + 256u * gpk);
-                tma_load_2d(wdst, &w_map, 0,
-                            (int)(code_offset(n32, w_kb, p.K, p.N / 32, 1) >> 10), &wp_full[sw],
-                            pol_w);
+                tma_load_2d(wdst, &w_map, 0, (int)(code_offset(n32, w_kb, p.K, p.N / 32, 1) >> 10),
+                            &wp_full[sw], pol_w);
                 for (int gi = 0; gi < gpk; ++gi)
                     tma_load_2d(wdst + 4096 + gi * 256, &s_map, 0,
                                 (int)(scale_offset(n32, w_kb * BK / p.G + gi, p.K, p.G, p.N / 32) >> 6),
@@ -494,15 +485,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             w_issue(0xffffffffu);
     } else if (warp == kMmaWarp) {
         if (rank == 0 && lane == 0) {
-            // One thread issues every MMA of the pair, so its own instruction
-            // latency bounds the rate at 128 tokens (a k-block's four MMAs
-            // take 256 tensor cycles): one barrier wait per k-block (the
-            // leader's dequantisers check the activations before they
-            // release a block), ring slots and phases kept incrementally,
-            // descriptors formed by addition.
             constexpr uint32_t idesc = idesc_pair<BT>();
-            const uint64_t xdesc0 = sw128_desc(smem_u32(smem + L::x_off));
-            uint32_t sx = 0, sa = 0, pa = 0, tcount = 0;
+            uint32_t it = 0, tcount = 0;
             bool ok = true;
             for (int item = pair; item < p.num_items && ok; item += npairs, ++tcount) {
                 int tile, kb0, kb1;
@@ -512,25 +496,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     break;
                 tc_fence_after();
                 const uint32_t d = tmem_base + L::acc_col;
-                for (int kb = kb0; kb < kb1; ++kb) {
-                    ok = role_wait(&a_full[sa], pa, abort_flag, p.hdr, 413);
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                    const int sx = it % L::kSX, sa = it % L::kSA;
+                    ok = role_wait(&x_full[sx], (it / L::kSX) & 1, abort_flag, p.hdr, 412) &&
+                         role_wait(&a_full[sa], (it / L::kSA) & 1, abort_flag, p.hdr, 413);
                     if (!ok)
                         break;
                     tc_fence_after();
-                    const uint64_t bd = xdesc0 + (uint64_t)((sx * L::x_slot) >> 4);
+                    const uint32_t xa = smem_u32(smem + L::x_off + sx * L::x_slot);
                     const uint32_t a = tmem_base + L::a_col + 32 * sa;
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)
-                        tc_mma_ts_pair(d, a + 8 * k, bd + 2 * k, idesc,
+                        tc_mma_ts_pair(d, a + 8 * k, sw128_desc(xa + 32 * k), idesc,
                                        (kb > kb0 || k > 0) ? 1u : 0u);
                     tc_commit_pair(&x_empty[sx]);
                     tc_commit_pair(&a_empty[sa]);
-                    if (++sx == L::kSX)
-                        sx = 0;
-                    if (++sa == L::kSA) {
-                        sa = 0;
-                        pa ^= 1;
-                    }
                 }
                 if (ok)
                     tc_commit_pair(acc_full);
@@ -650,11 +630,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int tile, kb0, kb1;
             item_range(p, item, tile, kb0, kb1);
             const int nb = tile_nb(p, tile);
-            // k-block kb at ring position itk: its E8M0 scales (MXFP8)
-            auto mx_scales = [&](int kb, float (&sca)[2], float (&scb)[2]) {
-                sca[0] = sca[1] = scb[0] = scb[1] = 1.f;
+            for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                const int sw = it % L::kSW, sa = it % L::kSA;
+                float sca[2] = {1.f, 1.f}, scb[2] = {1.f, 1.f};
                 if (F == kMxfp8) {
-                    // rows ra, ra + 8 for the two 32-blocks of this k-block
+                    // E8M0 scales of rows ra, ra + 8 for the two 32-blocks of this k-block
                     const int blocks = p.K / 32;
                     const long long ra =
                         (long long)nb * 2 * BW + (int)rank * BW + q * 32 + h * 16 + g;
@@ -672,69 +652,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         scb[b] = e8m0_to_f32(eb);
                     }
                 }
-            };
-            auto ready = [&](uint32_t itk) -> bool {
-                return role_wait(&wp_full[itk % L::kSW], (itk / L::kSW) & 1, abort_flag, p.hdr,
-                                 431) &&
-                       role_wait(&a_empty[itk % L::kSA], ((itk / L::kSA) & 1) ^ 1, abort_flag,
-                                 p.hdr, 432);
-            };
-            auto decode = [&](uint32_t itk, const float (&sca)[2], const float (&scb)[2],
-                              uint32_t (&vv)[16]) {
-                const uint8_t *wp_slot = smem + L::wp_off + (itk % L::kSW) * L::wp_slot;
-                if (F == kInt4)
-                    dequant_int4(wp_slot, q, h, lane, p.G, gpk, vv);
-                else
-                    dequant_mx(wp_slot, q, h, lane, sca, scb, vv);
-            };
-            auto store = [&](uint32_t itk, const uint32_t (&vv)[16]) {
-                tmem_st_16x256b_x4(tmem_base + ((uint32_t)(q * 32 + h * 16) << 16) + L::a_col +
-                                       32 * (itk % L::kSA),
-                                   vv);
-            };
-            // the store of block itk has completed: hand the slot to the MMA
-            // and the packed weights back to their producer.  In the leader
-            // the block's activations must have landed too (the MMA thread
-            // waits on this barrier alone).
-            auto release = [&](uint32_t itk) {
-                if (rank == 0 && !role_wait(&x_full[itk % L::kSX], (itk / L::kSX) & 1, abort_flag,
-                                            p.hdr, 412))
-                    ok = false;
-                if (lane == 0) {
-                    mbar_arrive(&wp_empty[itk % L::kSW]);
-                    mbar_arrive_cluster(mapa_shared(smem_u32(&a_full[itk % L::kSA]), 0));
-                }
-            };
-            // Two k-blocks per pass: their decodes are independent chains the
-            // scheduler interleaves, so a warp keeps twice the work in flight
-            // (a lone block's decode is bound by its dependency latency, not
-            // by issue).  With one block left the second decode repeats it.
-            for (int kb = kb0; kb < kb1; kb += 2) {
-                const bool two = kb + 1 < kb1;
-                const uint32_t it1 = two ? it + 1 : it;
-                float sa0[2], sb0[2], sa1[2], sb1[2];
-                mx_scales(kb, sa0, sb0);
-                mx_scales(two ? kb + 1 : kb, sa1, sb1);
-                ok = ready(it) && (!two || ready(it + 1));
+                ok = role_wait(&wp_full[sw], (it / L::kSW) & 1, abort_flag, p.hdr, 431) &&
+                     role_wait(&a_empty[sa], ((it / L::kSA) & 1) ^ 1, abort_flag, p.hdr, 432);
                 if (!ok)
                     break;
                 tc_fence_after();
-                uint32_t v0[16], v1[16];
-                decode(it, sa0, sb0, v0);
-                decode(it1, sa1, sb1, v1);
-                store(it, v0);
-                if (two)
-                    store(it1, v1);
+                const uint8_t *wp_slot = smem + L::wp_off + sw * L::wp_slot;
+                uint32_t v[16];
+                if (F == kInt4)
+                    dequant_int4(wp_slot, q, h, lane, p.G, gpk, v);
+                else
+                    dequant_mx(wp_slot, q, h, lane, sca, scb, v);
+                tmem_st_16x256b_x4(
+                    tmem_base + ((uint32_t)(q * 32 + h * 16) << 16) + L::a_col + 32 * sa, v);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                release(it);
-                if (two)
-                    release(it1);
-                it += two ? 2 : 1;
+                if (lane == 0) {
+                    mbar_arrive(&wp_empty[sw]);
+                    mbar_arrive_cluster(mapa_shared(smem_u32(&a_full[sa]), 0));
+                }
             }
-            if (!ok)
-                break;
         }
     }
 
@@ -838,23 +776,20 @@ cudaError_t launch_w4a16_tc(const TcPlan &pl, const void *X, const void *packed,
 {
     alignas(64) CUtensorMap xm, wm, sm;
     const uint8_t *codes = static_cast<const uint8_t *>(packed);
+    const uint8_t *scales = codes + (size_t)N * K / 2;
     if (!x_map(&xm, X, M, K, pl.bm) ||
-        // codes: rows of one tile's 1 KB for one k64 chunk (128 u64), in
-        // memory order; box = 4 rows (the CTA's four tiles of a chunk)
+        // codes and scales of the column-group layout as rows of one tile's
+        // 1 KB (128 u64) and 64 B (8 u64), in memory order; boxes of 4 rows
         !encode_tensor_map_2d(&wm, CU_TENSOR_MAP_DATA_TYPE_UINT64, codes, 128,
                               (uint64_t)(N / 32) * (K / 64), 1024, 128, BW / 32,
                               CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        // scales: rows of one tile's 64 B for one group (8 u64); box = 4 rows
-        !encode_tensor_map_2d(&sm, CU_TENSOR_MAP_DATA_TYPE_UINT64, codes + (size_t)N * K / 2, 8,
+        !encode_tensor_map_2d(&sm, CU_TENSOR_MAP_DATA_TYPE_UINT64, scales, 8,
                               (uint64_t)(N / 32) * (K / G), 64, 8, BW / 32,
                               CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     TcParams p{};
     p.Y = static_cast<uint16_t *>(Y);
     p.Ws = nullptr;
-    // weights are moved with tensor-map boxes over the column-group layout
-    p.codes = codes;
-    p.scales = codes + (size_t)N * K / 2;
     p.hdr = static_cast<WsHeader *>(workspace);
     p.M = M;
     p.N = N;
