@@ -53,10 +53,22 @@ def row_shard(qweight, scales, group_size: int, rank: int, world: int):
 
 def all_reduce_sum(y, group=None):
     """Sum a partial output over the ranks of ``group`` in place (no-op
-    without an initialised process group of more than one rank)."""
+    without an initialised process group of more than one rank).
+
+    16-bit partials are summed in fp32 and rounded once: each rank's partial
+    carries one bf16 rounding from its GEMM's output (at most 2^-9 of its
+    magnitude), and a reduction in bf16 would add one rounding per step of
+    the collective's reduction tree; in fp32 the sum of P <= 8 bf16 values is
+    exact unless their exponents span more than 16 binades."""
+    import torch
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
-        dist.all_reduce(y, op=dist.ReduceOp.SUM, group=group)
+        if y.dtype in (torch.bfloat16, torch.float16):
+            y32 = y.float()
+            dist.all_reduce(y32, op=dist.ReduceOp.SUM, group=group)
+            y.copy_(y32)
+        else:
+            dist.all_reduce(y, op=dist.ReduceOp.SUM, group=group)
     return y
 
 

@@ -58,7 +58,10 @@ def _worker(rank, world, port, out):
                                k1 - k0, G)
         t = torch.from_numpy(yr.copy())
         tp.all_reduce_sum(t)
-        out[rank] = (n0, n1, yc, t.numpy(), k0, k1)
+        # the same partial as the GEMM returns it (bf16), reduced in fp32
+        tb = torch.from_numpy(yr.copy()).to(torch.bfloat16)
+        tp.all_reduce_sum(tb)
+        out[rank] = (n0, n1, yc, t.numpy(), k0, k1, tb.float().numpy(), yr)
     finally:
         dist.destroy_process_group()
 
@@ -84,6 +87,12 @@ def test_column_and_row_parallel_gloo():
     assert [(res[r][4], res[r][5]) for r in range(world)] == [(0, 512), (512, 1024)]
     for r in range(world):
         assert np.allclose(res[r][3], full, rtol=1e-12, atol=1e-12)
+    # bf16 partials: the all-reduce adds them in fp32 and rounds once, so the
+    # result is the bf16 nearest of the exact sum of the rounded partials
+    parts = [torch.from_numpy(res[r][7]).to(torch.bfloat16).double() for r in range(world)]
+    expect = (parts[0] + parts[1]).to(torch.bfloat16).float().numpy()
+    for r in range(world):
+        assert np.array_equal(res[r][6], expect)
 
 
 def test_shard_boundaries_follow_the_shape_rules():
