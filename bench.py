@@ -36,6 +36,9 @@ roofline   every layer of a step runs the same kernel, so the dominant
            at a time (no overlap with a neighbour) are reported beside it.
 L2         every step reads a different copy of the weights from a rotating
            pool of at least 3 x L2 bytes, so weights come from HBM.
+m_sweep    informational: the INT4 5120 -> 17408 layer at M = 1 .. 8192 on
+           the path the library picks, time per layer and the fraction of
+           max(bytes / HBM peak, flops / bf16 burst peak) (--no-sweep skips).
 
 --impl reference runs the fp64 CPU oracle (the baseline arm) on the same
 workload: each step processes a bounded slice of columns of every layer, and
@@ -593,6 +596,38 @@ def summarize(wl, res, steps, world, peaks, peak_kind):
     return out
 
 
+SWEEP_M = (1, 2, 4, 5, 8, 16, 32, 64, 128, 256, 1024, 8192)
+SWEEP_LAYER = (5120, 17408)
+
+
+def m_sweep(args, rank, world, dev, peaks):
+    """Informational: the INT4 5120 -> 17408 layer at every M of SWEEP_M
+    (the path the library picks), each timed like a configuration; time per
+    layer, weight TB/s, TFLOP/s and the fraction of the layer's roofline
+    time max(bytes / HBM peak, flops / burst bf16 peak)."""
+    import torch
+
+    out = []
+    K, N = SWEEP_LAYER
+    for M in SWEEP_M:
+        name = f"sweep_int4_m{M}"
+        WORKLOADS[name] = ("int4", M, [SWEEP_LAYER], 128)
+        wl = Workload(name, rank, dev, args.pool_factor)
+        steps = 10 if M >= 1024 else 50
+        res = measure(wl, steps, 3, world, dev, args, with_e2e=False)
+        us = res["elapsed_ms"] / steps * 1e3
+        t_roof = max(wl.step_bytes / (peaks["hbm_gbs"] * 1e9),
+                     wl.step_flops / (peaks["bf16_tflops"] * 1e12)) * 1e6
+        out.append({"M": M, "us": round(us, 3),
+                    "tbps": round(wl.step_bytes / (us * 1e-6) / 1e12, 4),
+                    "tflops": round(wl.step_flops / (us * 1e-6) / 1e12, 2),
+                    "kernel": wl.kernel, "frac_of_roofline": round(t_roof / us, 4)})
+        del wl, WORKLOADS[name]
+        torch.cuda.empty_cache()
+    return {"layer_KxN": f"{K}x{N}", "format": "int4 g128", "points": out,
+            "roofline": "max(weight bytes / measured HBM, flops / measured bf16 burst)"}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -661,6 +696,8 @@ def run_ours(args, rank, world, local_rank):
         "gpu": props.name,
         "configs": {n: r for n, r in results.items() if n != args.workload},
     }
+    if not args.no_sweep:
+        line["m_sweep"] = m_sweep(args, rank, world, dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.workload, budget_s=args.cpu_budget)
     if world > 1:
@@ -841,6 +878,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-budget", type=float, default=120.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the informational M sweep of the INT4 5120 -> 17408 layer")
     ap.add_argument("--pool-factor", type=float, default=3.0,
                     help="rotating weight pool size in multiples of the L2 size")
     args = ap.parse_args()
