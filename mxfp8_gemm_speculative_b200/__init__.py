@@ -536,6 +536,20 @@ def mxfp8_gemm_packed(x: torch.Tensor, packed: torch.Tensor, N: int, K: int,
     return out
 
 
+def prepare_mxfp8_gemm_packed(x: torch.Tensor, packed: torch.Tensor, N: int, K: int,
+                              out: torch.Tensor | None = None,
+                              workspace_buf: torch.Tensor | None = None, stream=None,
+                              late_weights: bool = False):
+    """(call, out): ``call()`` runs mxfp8_gemm_packed(x, packed) into ``out``."""
+    M, out, ws = _gemm_buffers(x, K, N, out, workspace_buf,
+                               lambda: _mxp_ws_bytes(x.shape[0], N, K), stream)
+    _need_weights(packed, torch.uint8, int(_lib.mxfp8_packed_bytes(N, K)), x.device, "packed")
+    args = (_ptr(x), _ptr(packed), M, N, K, _ptr(out), _ptr(ws), ws.numel(),
+            _options(PATH_AUTO, late_weights), _stream(stream, x.device))
+    return PreparedCall(_lib.mxfp8_gemm_packed_ex, args, "mxfp8_gemm_packed",
+                        (x, packed, out, ws, stream), x.device), out
+
+
 def mxfp8_dequant(wq: torch.Tensor, ws: torch.Tensor, stream=None) -> torch.Tensor:
     """bf16 [N][K] weights of E4M3 wq[N][K] and E8M0 ws[N][K/32]."""
     if wq.dtype not in (torch.uint8, torch.float8_e4m3fn):

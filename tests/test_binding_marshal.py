@@ -24,6 +24,8 @@ class FakeLib:
             # the real query looks at the current device (none here): the
             # streaming path's rule, M <= 32, with a stand-in size
             return lambda M, N, K, G: 4096 if 1 <= M <= 32 else 0
+        if name == "mxfp8_packed_workspace_bytes":
+            return lambda M, N, K: 4096 if 1 <= M <= 16 else 0
         if name.endswith("_bytes") or name == "mxg_status_string":
             return getattr(self._real, name)
 
@@ -170,6 +172,38 @@ def test_mxfp8_calls(fake):
         m.mxfp8_gemm(x, wq, ws[:, :-1])
     with pytest.raises(ValueError):
         m.mxfp8_gemm(x, wq, ws, out=bf16(M + 1, N))
+
+
+def test_mxfp8_packed_calls(fake):
+    m, lib = fake
+    M, K, N = 4, 512, 256
+    x = bf16(M, K)
+    wq = torch.zeros((N, K), dtype=torch.uint8)
+    ws = torch.zeros((N, K // 32), dtype=torch.uint8)
+    packed = m.mxfp8_repack(wq, ws)
+    name, a = lib.calls[-1]
+    assert name == "mxfp8_repack"
+    assert [_val(v) for v in a[:2]] == [wq.data_ptr(), ws.data_ptr()]
+    assert a[2:4] == (N, K) and _val(a[4]) == packed.data_ptr()
+    assert packed.numel() == N * K + N * K // 32
+    y = m.mxfp8_gemm_packed(x, packed, N, K)
+    name, a = lib.calls[-1]
+    assert name == "mxfp8_gemm_packed_ex"
+    assert [_val(v) for v in a[:2]] == [x.data_ptr(), packed.data_ptr()]
+    assert a[2:5] == (M, N, K) and _val(a[5]) == y.data_ptr() and a[7] == 4096 and a[8] is None
+    call, y2 = m.prepare_mxfp8_gemm_packed(x, packed, N, K)
+    call()
+    name, a = lib.calls[-1]
+    assert name == "mxfp8_gemm_packed_ex" and _val(a[5]) == y2.data_ptr()
+    n0 = len(lib.calls)
+    with pytest.raises(ValueError):
+        m.mxfp8_gemm_packed(x, packed[:-16], N, K)         # too few weight bytes
+    with pytest.raises(m.MxgError):
+        m.mxfp8_gemm_packed(bf16(17, K), packed, N, K)    # M <= 16 only
+    with pytest.raises(m.MxgError):
+        m.mxfp8_repack(torch.zeros((96, K), dtype=torch.uint8),
+                       torch.zeros((96, K // 32), dtype=torch.uint8))   # N % 64
+    assert len(lib.calls) == n0
 
 
 def test_bf16_small_calls(fake):
