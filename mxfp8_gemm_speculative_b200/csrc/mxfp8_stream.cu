@@ -133,11 +133,10 @@ __device__ __noinline__ void finish_cut_tile(const Params &p, const float4 *frag
 #pragma unroll
         for (int tt = 0; tt < TT; ++tt)
             __stcg(p.partial + ((size_t)c * TT + tt) * 32 + lane, sum[tt]);
+        __threadfence();   // every lane's stores, before the warp counts itself
         __syncwarp();
-        if (lane == 0) {
-            __threadfence();
+        if (lane == 0)
             atomicAdd(&p.counters[nt], 1);
-        }
         return;
     }
     const int c_last = cta_of_unit(p, tile_begin + p.upt - 1);
@@ -152,6 +151,7 @@ __device__ __noinline__ void finish_cut_tile(const Params &p, const float4 *frag
         }
     }
     __syncwarp();
+    __threadfence();
     for (int cc = c_first + 1; cc <= c_last; ++cc) {
 #pragma unroll
         for (int tt = 0; tt < TT; ++tt) {

@@ -565,13 +565,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 // in order and writes bf16 Y
                 int *cnt = p.counters + tile * 8 + (int)rank * 4 + q;
                 int last = 0;
-                if (lane == 0) {
-                    __threadfence();
+                __threadfence();   // every lane's partial sums, before the warp counts itself
+                __syncwarp();
+                if (lane == 0)
                     last = atomicAdd(cnt, 1) == p.splits - 1;
-                    if (last)
-                        __threadfence();
-                }
                 if (__shfl_sync(0xffffffffu, last, 0)) {
+                    __threadfence();
                     const int c4 = (lane & 7) * 4;        // 4 columns per lane
                     const int nc = nb * 2 * BW + nloc + c4;
                     const float *src0 =

@@ -334,14 +334,19 @@ __device__ __forceinline__ void finish_cut(const Params &p, float4 (&sum)[2 * TT
 #pragma unroll
     for (int j = 0; j < F; ++j)
         __stcg(mine + j * 32 + lane, sum[j]);
+    // every lane's stores are performed at GPU scope before the warp counts
+    // itself (a release by one lane orders only that lane's own accesses)
+    __threadfence();
     __syncwarp();
     int old = 0;
     if (lane == 0)
-        old = atomic_add_acq_rel(&p.counters[tile], 1);   // releases the fragment
+        old = atomic_add_acq_rel(&p.counters[tile], 1);
     old = __shfl_sync(0xFFFFFFFFu, old, 0);
     if (old != c_last - c_first)
         return;
-    // the last contributor (its acquire saw every other release)
+    // the last contributor: its count saw every other contributor's; every
+    // lane fences before reading their fragments
+    __threadfence();
     float4 tot[F];
 #pragma unroll
     for (int j = 0; j < F; ++j)
